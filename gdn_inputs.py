@@ -64,7 +64,11 @@ def quantize(x: np.ndarray, dtype: str) -> np.ndarray:
 
 # --------------------------------------------------------------------------- draws
 def _rngs(seed: int) -> dict:
-    kids = np.random.SeedSequence(seed).spawn(len(_STREAMS))
+    return _rngs_entropy(seed)
+
+
+def _rngs_entropy(entropy) -> dict:
+    kids = np.random.SeedSequence(entropy).spawn(len(_STREAMS))
     return {name: np.random.Generator(np.random.PCG64(s)) for name, s in zip(_STREAMS, kids)}
 
 
@@ -75,6 +79,19 @@ def _normal_f32(rng: np.random.Generator, shape, block: int = 1 << 24) -> np.nda
     for s in range(0, n, block):
         e = min(n, s + block)
         rng.standard_normal(e - s, dtype=np.float32, out=out[s:e])
+    return out.reshape(shape)
+
+
+def _normal_stored(rng: np.random.Generator, shape, dtype: str, block: int = 1 << 24) -> np.ndarray:
+    """N(0,1) drawn in fp32 blocks and quantised block by block into the storage dtype."""
+    n = int(np.prod(shape))
+    out = np.empty(n, dtype=np.uint16 if dtype == BF16 else np.float32)
+    tmp = np.empty(min(block, max(n, 1)), dtype=np.float32)
+    for s in range(0, n, block):
+        e = min(n, s + block)
+        t = tmp[:e - s]
+        rng.standard_normal(e - s, dtype=np.float32, out=t)
+        out[s:e] = quantize(t, dtype)
     return out.reshape(shape)
 
 
@@ -166,9 +183,9 @@ def make_prefill_inputs(shape: GdnShape, lengths, dtype: str, seed: int, c: floa
     cu[1:] = np.cumsum(lengths)
     r = _rngs(seed)
     H, Hv, dk, dv, W = shape.n_qk_heads, shape.n_v_heads, shape.d_k, shape.d_v, shape.conv_width
-    q = quantize(_normal_f32(r["q"], (T, H, dk)), dtype)
-    k = quantize(_normal_f32(r["k"], (T, H, dk)), dtype)
-    v = quantize(_normal_f32(r["v"], (T, Hv, dv)), dtype)
+    q = _normal_stored(r["q"], (T, H, dk), dtype)
+    k = _normal_stored(r["k"], (T, H, dk), dtype)
+    v = _normal_stored(r["v"], (T, Hv, dv), dtype)
     w_q, w_k, w_v = weights if weights is not None else make_conv_weights(shape, seed, weight_std)
     alpha = quantize(draw_alpha(r["x_alpha"], (T, Hv), c), dtype)
     beta = quantize(draw_beta(r["x_beta"], (T, Hv)), dtype)
@@ -177,14 +194,14 @@ def make_prefill_inputs(shape: GdnShape, lengths, dtype: str, seed: int, c: floa
         init = (state_std * _normal_f32(r["state"], (len(lengths), Hv, dk, dv))).astype(np.float32)
     cs = None
     if with_conv_state:
-        cs = quantize(_normal_f32(r["conv_state"], (len(lengths), W - 1, shape.channels)), dtype)
+        cs = _normal_stored(r["conv_state"], (len(lengths), W - 1, shape.channels), dtype)
     return PrefillInputs(shape, dtype, q, k, v, w_q, w_k, w_v, alpha, beta, cu, init, cs,
                          meta={"seed": seed, "c": c, "lengths": lengths.tolist()})
 
 
 @dataclass
 class DecodeInputs:
-    """Fresh per-step inputs for ``steps`` decode steps of a batch (storage dtype)."""
+    """Fresh per-step inputs of a decode batch (storage dtype).  Leading axis: steps."""
     q: np.ndarray       # [steps, B, Hqk, dk]
     k: np.ndarray       # [steps, B, Hqk, dk]
     v: np.ndarray       # [steps, B, Hv, dv]
@@ -192,17 +209,27 @@ class DecodeInputs:
     beta: np.ndarray    # [steps, B, Hv]
 
 
-def make_decode_inputs(shape: GdnShape, batch: int, steps: int, dtype: str, seed: int,
-                       c: float = 0.1) -> DecodeInputs:
-    r = _rngs(seed)
+def make_decode_step(shape: GdnShape, batch: int, step: int, dtype: str, seed: int,
+                     c: float = 0.1) -> DecodeInputs:
+    """Inputs of decode step ``step`` alone (its own seed stream: SeedSequence([seed, step]))."""
+    r = _rngs_entropy([seed, step])
     H, Hv, dk, dv = shape.n_qk_heads, shape.n_v_heads, shape.d_k, shape.d_v
     return DecodeInputs(
-        q=quantize(_normal_f32(r["q"], (steps, batch, H, dk)), dtype),
-        k=quantize(_normal_f32(r["k"], (steps, batch, H, dk)), dtype),
-        v=quantize(_normal_f32(r["v"], (steps, batch, Hv, dv)), dtype),
-        alpha=quantize(draw_alpha(r["x_alpha"], (steps, batch, Hv), c), dtype),
-        beta=quantize(draw_beta(r["x_beta"], (steps, batch, Hv)), dtype),
+        q=_normal_stored(r["q"], (1, batch, H, dk), dtype),
+        k=_normal_stored(r["k"], (1, batch, H, dk), dtype),
+        v=_normal_stored(r["v"], (1, batch, Hv, dv), dtype),
+        alpha=quantize(draw_alpha(r["x_alpha"], (1, batch, Hv), c), dtype),
+        beta=quantize(draw_beta(r["x_beta"], (1, batch, Hv)), dtype),
     )
+
+
+def make_decode_inputs(shape: GdnShape, batch: int, steps: int, dtype: str, seed: int,
+                       c: float = 0.1, first_step: int = 0) -> DecodeInputs:
+    """Steps first_step .. first_step+steps-1 stacked (each drawn by make_decode_step)."""
+    parts = [make_decode_step(shape, batch, s, dtype, seed, c)
+             for s in range(first_step, first_step + steps)]
+    return DecodeInputs(*(np.concatenate([getattr(p, f) for p in parts])
+                          for f in ("q", "k", "v", "alpha", "beta")))
 
 
 # --------------------------------------------------------------------------- workloads
@@ -244,19 +271,27 @@ def workload_weights(index: int):
     return make_conv_weights(WORKLOADS[index]["shape"], workload_seed(index))
 
 
-def warmup_prefill_inputs(index: int, n_seqs: int) -> PrefillInputs:
-    """The seeded prefill whose final states (and last raw rows) seed workloads 3 and 4.
+def warmup_prefill_inputs(index: int, rows) -> PrefillInputs:
+    """The seeded prefills whose final states and last raw rows seed workloads 3 and 4.
 
-    It runs through the same layer (the workload's conv weights), one sequence of
-    ``warm_tokens`` tokens per decode row / packed sequence.
+    One ``warm_tokens``-token sequence per decode row / packed sequence in ``rows``
+    (each row has its own seed stream, so any subset can be drawn alone), run
+    through the same layer (the workload's conv weights); returned packed.
     """
     w = WORKLOADS[index]
-    return make_prefill_inputs(w["shape"], [w["warm_tokens"]] * n_seqs, w["dtype"],
-                               workload_seed(index) + 1000, c=w["c"],
-                               weights=workload_weights(index))
+    rows = [int(r) for r in rows]
+    parts = [make_prefill_inputs(w["shape"], [w["warm_tokens"]], w["dtype"],
+                                 [workload_seed(index), 1000, r], c=w["c"],
+                                 weights=workload_weights(index)) for r in rows]
+    first = parts[0]
+    cat = {f: np.concatenate([getattr(p, f) for p in parts]) for f in ("q", "k", "v", "alpha", "beta")}
+    cu = np.arange(len(rows) + 1, dtype=np.int32) * w["warm_tokens"]
+    return PrefillInputs(w["shape"], w["dtype"], cat["q"], cat["k"], cat["v"], first.w_q, first.w_k,
+                         first.w_v, cat["alpha"], cat["beta"], cu, meta={"rows": rows})
 
 
-def decode_workload_inputs(index: int = 3, steps: int | None = None) -> DecodeInputs:
+def decode_workload_step(step: int, index: int = 3) -> DecodeInputs:
+    """Inputs of one step of the decode workload (all rows)."""
     w = WORKLOADS[index]
-    return make_decode_inputs(w["shape"], w["batch"], steps or w["steps"], w["dtype"],
-                              workload_seed(index) + 2000, c=w["c"])
+    return make_decode_step(w["shape"], w["batch"], step, w["dtype"], workload_seed(index) + 2000,
+                            c=w["c"])

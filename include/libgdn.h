@@ -1,0 +1,174 @@
+/*
+ * libgdn.h -- Gated DeltaNet (GDN) token mixer for NVIDIA B200 (sm_100a).
+ *
+ * The operation (page "ARCHITECTURE PREVIEW / FIELD NOTES", section 03 "Attention",
+ * the GDN figure caption and the "GATED DELTANET" equations; section 01 config
+ * table for the shapes: 48 value heads, 16 QK heads, head dim 128, conv kernel 4):
+ *
+ *   per token t of a sequence, raw rows q_t, k_t [Hqk, dk] and v_t [Hv, dv]:
+ *     ShortConv   x'_t[c] = sum_{j=0..3} w[c][j] * x_{t-3+j}[c]   on every q, k, v channel
+ *                 (causal, depthwise, tap 3 on the current row, no bias, no activation;
+ *                  rows before the sequence start come from the conv state, else zero)
+ *     L2 norm     q^ = q' * q_scale / sqrt(|q'|^2 + l2_eps),  k^ = k' / sqrt(|k'|^2 + l2_eps)
+ *                 per (token, QK head); v^ = v'
+ *   per value head h, reading QK head g = h / (Hv / Hqk), with state S [dk][dv] (fp32):
+ *     S~  = alpha_t S_{t-1}
+ *     e_t = v^_t - S~^T k^_t
+ *     S_t = S~ + beta_t k^_t e_t^T
+ *     y_t = S_t^T q^_t                       (the read uses the updated state)
+ *
+ * Conventions shared by every entry point
+ *  - Ownership: every buffer is a DEVICE pointer owned by the caller.  The library
+ *    allocates nothing and keeps no mutable global state; calls on different streams
+ *    are independent as long as their buffers do not overlap.
+ *  - Asynchrony: every call only enqueues work on `stream` (0 = legacy default stream)
+ *    and returns; nothing synchronises.  Kernel faults surface at the caller's next
+ *    synchronisation.
+ *  - Validation: all argument checks run on the host before any launch; on failure
+ *    nothing is enqueued and nothing is written.  Values stored in device memory
+ *    (cu_seqlens, state_slots) cannot be checked on the host: the kernels clamp them
+ *    so that no access leaves the buffers the host-side sizes describe.
+ *  - Layout: token-major, row-major, innermost dimension last and contiguous.
+ *  - Supported: d_k = d_v = 128, conv_width = 4, n_v_heads a multiple of n_qk_heads,
+ *    compute capability 10.0 (B200).  Anything else returns GDN_ERR_UNSUPPORTED.
+ *  - Errors: a failed launch returns GDN_ERR_CUDA; gdn_last_cuda_error() then gives
+ *    the cudaError_t of the failing call (per host thread).
+ */
+#ifndef LIBGDN_H
+#define LIBGDN_H
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define GDN_API_VERSION 1
+
+#if defined(__GNUC__)
+#define GDN_EXPORT __attribute__((visibility("default")))
+#else
+#define GDN_EXPORT
+#endif
+
+typedef enum {
+    GDN_OK = 0,
+    GDN_ERR_INVALID_ARG = 1,   /* null/misaligned pointer, bad size, inconsistent config */
+    GDN_ERR_UNSUPPORTED = 2,   /* shape or device this build does not implement */
+    GDN_ERR_WORKSPACE = 3,     /* workspace missing, misaligned or too small */
+    GDN_ERR_CUDA = 4,          /* a CUDA runtime call or launch failed */
+    GDN_ERR_TIMEOUT = 5        /* reserved: a bounded device-side wait gave up */
+} gdn_status;
+
+typedef enum {
+    GDN_BF16 = 0,  /* bfloat16 storage */
+    GDN_F32 = 1    /* float32 storage */
+} gdn_dtype;
+/* Every call takes two storage types: `dtype` for q, k, v, alpha, beta and the conv
+ * state (the raw inputs), and `out_dtype` for y.  Whatever they are, all arithmetic is
+ * fp32 (tensor-core products in TF32 with fp32 accumulation) and states are fp32.
+ * Note on precision: rounding y to bfloat16 alone moves its largest entries by up to
+ * 2^-9 of their magnitude, which on typical data is 2-3% of rms(y); use
+ * out_dtype = GDN_F32 where y must stay within 1e-2 of rms(y) of the exact result. */
+
+typedef struct {
+    int n_qk_heads;   /* Hqk: QK heads (16 in the pages' layer)                      */
+    int n_v_heads;    /* Hv: value heads (48); V head h reads QK head h/(Hv/Hqk)     */
+    int d_k;          /* key/query head dim, must be 128                             */
+    int d_v;          /* value head dim, must be 128                                 */
+    int conv_width;   /* ShortConv kernel size, must be 4                            */
+    float q_scale;    /* multiplies q^ after normalisation (1.0: the page has none)  */
+    float l2_eps;     /* epsilon inside the L2 norm's square root (1e-6)             */
+} gdn_config;
+
+/* Human-readable name of a status code (static storage, never NULL). */
+GDN_EXPORT const char *gdn_status_string(gdn_status status);
+
+/* cudaError_t (as int) of the last CUDA failure seen by a libgdn call on this host thread. */
+GDN_EXPORT int gdn_last_cuda_error(void);
+
+/* GDN_API_VERSION of the loaded library. */
+GDN_EXPORT int gdn_api_version(void);
+
+/*
+ * gdn_prefill_workspace_size -- bytes of device workspace that gdn_prefill needs
+ * for `total_tokens` tokens packed into `n_seqs` sequences.  Writes *bytes.
+ * The workspace holds the clamped sequence table, the per-sequence chunk offsets
+ * and the convolved, normalised q^, k^, v^ rows in fp32; it is scratch only (no
+ * state persists between calls) and must not be shared by two calls in flight.
+ */
+GDN_EXPORT gdn_status gdn_prefill_workspace_size(const gdn_config *cfg, gdn_dtype dtype,
+                                      int64_t total_tokens, int n_seqs, size_t *bytes);
+
+/*
+ * gdn_prefill -- the mixer over packed variable-length sequences (chunked prefill).
+ *
+ * Page: "ARCHITECTURE PREVIEW / FIELD NOTES", section 03 (the GATED DELTANET
+ * equations and the ShortConv of the GDN figure); chunked prefill is named in
+ * section 03's performance note.  Internally the recurrence runs in chunks of
+ * 64 tokens (WY/UT form: intra-chunk triangular solve, inter-chunk state scan),
+ * which reaches the same result as the token-by-token recurrence up to rounding.
+ *
+ *   q, k            [T, Hqk, 128]  raw (pre-conv) rows, dtype      16-byte aligned
+ *   v               [T, Hv, 128]   raw rows, dtype                 16-byte aligned
+ *   conv_w_q, conv_w_k [Hqk*128, 4], conv_w_v [Hv*128, 4]  fp32, tap 3 = current row
+ *   alpha, beta     [T, Hv] dtype: decay in (0, 1] and write strength, one per (token, V head)
+ *   cu_seqlens      [n_seqs+1] int32 device: sequence b is rows cu[b] .. cu[b+1]-1;
+ *                   non-decreasing, cu[0] = 0, cu[n_seqs] = total_tokens.  Zero-length
+ *                   sequences are allowed (their final state equals the initial one).
+ *                   Out-of-order values are clamped on the device, never dereferenced.
+ *   total_tokens    T (>= 0, < 2^31)
+ *   initial_state   [n_seqs, Hv, 128(dk), 128(dv)] fp32, dv fastest; NULL = zero state
+ *   final_state     same shape; NULL = not returned; may alias initial_state
+ *   conv_state_in   [n_seqs, 3, 2*Hqk*128 + Hv*128] dtype: the last 3 raw rows
+ *                   (q | k | v channels), oldest first; NULL = zero history
+ *   conv_state_out  same shape; NULL = not returned; may alias conv_state_in
+ *   out             [T, Hv, 128] out_dtype: y
+ *   workspace       >= gdn_prefill_workspace_size() bytes, 256-byte aligned
+ * Returns GDN_OK after enqueueing; n_seqs == 0 or T == 0 with no states is a no-op.
+ */
+GDN_EXPORT gdn_status gdn_prefill(const gdn_config *cfg, gdn_dtype dtype, gdn_dtype out_dtype,
+                       const void *q, const void *k, const void *v,
+                       const float *conv_w_q, const float *conv_w_k, const float *conv_w_v,
+                       const void *alpha, const void *beta,
+                       const int32_t *cu_seqlens, int n_seqs, int64_t total_tokens,
+                       const float *initial_state, float *final_state,
+                       const void *conv_state_in, void *conv_state_out,
+                       void *out, void *workspace, size_t workspace_bytes,
+                       cudaStream_t stream);
+
+/*
+ * gdn_decode_step -- one token for each of `batch` sequences whose states stay
+ * resident in device memory (the one-token case of the same recurrence: the
+ * GATED DELTANET equations of section 03 with the ShortConv history shifted by one
+ * row).  Each state is read once and written once, in place.
+ *
+ *   q, k            [batch, Hqk, 128] raw rows, dtype; v [batch, Hv, 128]
+ *   conv_w_*        as in gdn_prefill
+ *   alpha, beta     [batch, Hv] dtype
+ *   state           [n_state_rows, Hv, 128, 128] fp32, updated in place
+ *   conv_state      [n_state_rows, 3, 2*Hqk*128 + Hv*128] dtype, updated in place
+ *                   (shifted by one row, the current raw row appended); NULL = zero
+ *                   history and nothing written
+ *   state_slots     [batch] int32 device, NULL = identity: row b uses state row
+ *                   state_slots[b] (and the same conv-state row).  Slots of one call
+ *                   must be distinct; a slot outside [0, n_state_rows) skips the row
+ *                   (its out row is written as zeros, no state is touched).
+ *   n_state_rows    rows in state / conv_state (>= batch when state_slots is NULL)
+ *   out             [batch, Hv, 128] out_dtype: y
+ */
+GDN_EXPORT gdn_status gdn_decode_step(const gdn_config *cfg, gdn_dtype dtype, gdn_dtype out_dtype,
+                           const void *q, const void *k, const void *v,
+                           const float *conv_w_q, const float *conv_w_k, const float *conv_w_v,
+                           const void *alpha, const void *beta,
+                           float *state, void *conv_state,
+                           const int32_t *state_slots, int n_state_rows,
+                           void *out, int batch, cudaStream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LIBGDN_H */

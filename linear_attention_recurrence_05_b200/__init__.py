@@ -1,0 +1,151 @@
+"""libgdn: the Gated DeltaNet token mixer on B200 (sm_100a), Python binding.
+
+Thin wrappers over the C ABI of ``include/libgdn.h``: they check tensor
+placement and shapes, allocate outputs and workspace with PyTorch when the caller
+does not pass them, and hand raw device pointers plus the current CUDA stream to
+the library.  Every step of the computation runs in libgdn's CUDA kernels; there
+is no CPU or PyTorch fallback.
+
+    y, S, cs = gdn_prefill(q, k, v, w_q, w_k, w_v, alpha, beta, cu_seqlens, ...)
+    y = gdn_decode_step(q, k, v, w_q, w_k, w_v, alpha, beta, state, conv_state, ...)
+"""
+from __future__ import annotations
+
+import ctypes
+from dataclasses import dataclass
+
+import torch
+
+from . import _native
+from ._native import GDN_BF16, GDN_F32, GdnError  # noqa: F401
+
+__all__ = ["GdnConfig", "gdn_prefill", "gdn_decode_step", "prefill_workspace_size", "GdnError",
+           "library_path"]
+
+
+@dataclass(frozen=True)
+class GdnConfig:
+    n_qk_heads: int = 16
+    n_v_heads: int = 48
+    d_k: int = 128
+    d_v: int = 128
+    conv_width: int = 4
+    q_scale: float = 1.0
+    l2_eps: float = 1e-6
+
+    def c(self) -> _native.GdnConfigC:
+        return _native.GdnConfigC(self.n_qk_heads, self.n_v_heads, self.d_k, self.d_v,
+                                  self.conv_width, self.q_scale, self.l2_eps)
+
+    @property
+    def channels(self) -> int:
+        return 2 * self.n_qk_heads * self.d_k + self.n_v_heads * self.d_v
+
+
+def library_path() -> str:
+    return _native.LIB_PATH
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return GDN_BF16
+    if t.dtype == torch.float32:
+        return GDN_F32
+    raise TypeError(f"unsupported dtype {t.dtype}: bfloat16 or float32")
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("libgdn takes device tensors")
+    if not t.is_contiguous():
+        raise ValueError("libgdn takes contiguous tensors")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def prefill_workspace_size(cfg: GdnConfig, dtype: torch.dtype, total_tokens: int, n_seqs: int) -> int:
+    n = ctypes.c_size_t(0)
+    code = GDN_BF16 if dtype == torch.bfloat16 else GDN_F32
+    c = cfg.c()
+    _native.check("gdn_prefill_workspace_size", _native.lib().gdn_prefill_workspace_size(
+        ctypes.byref(c), code, int(total_tokens), int(n_seqs), ctypes.byref(n)))
+    return int(n.value)
+
+
+def gdn_prefill(q, k, v, conv_w_q, conv_w_k, conv_w_v, alpha, beta, cu_seqlens, *,
+                cfg: GdnConfig | None = None, initial_state=None, final_state=None,
+                return_final_state: bool = True, conv_state_in=None, conv_state_out=None,
+                return_conv_state: bool = False, out=None, out_dtype=torch.float32,
+                workspace=None, stream=None):
+    """Chunked prefill over packed sequences.  Returns (out, final_state, conv_state_out).
+
+    q, k [T, Hqk, 128], v [T, Hv, 128], alpha/beta [T, Hv] (bf16 or fp32, one dtype);
+    conv_w_* fp32 [channels, 4]; cu_seqlens int32 [N+1] on the device;
+    initial_state fp32 [N, Hv, 128, 128] or None; conv_state_in [N, 3, channels] or None.
+    ``out`` (or ``out_dtype``, fp32 by default) fixes y's storage type.
+    """
+    T = q.shape[0]
+    cfg = cfg or GdnConfig(n_qk_heads=q.shape[1], n_v_heads=v.shape[1])
+    n = cu_seqlens.shape[0] - 1
+    code = _dtype_code(q)
+    for t in (k, v, alpha, beta):
+        if t.dtype != q.dtype:
+            raise TypeError("q, k, v, alpha and beta must share one dtype")
+    if cu_seqlens.dtype != torch.int32:
+        raise TypeError("cu_seqlens must be int32")
+    dev = q.device
+    if out is None:
+        out = torch.empty((T, cfg.n_v_heads, cfg.d_v), dtype=out_dtype, device=dev)
+    if final_state is None and return_final_state:
+        final_state = torch.empty((n, cfg.n_v_heads, cfg.d_k, cfg.d_v), dtype=torch.float32,
+                                  device=dev)
+    if conv_state_out is None and return_conv_state:
+        conv_state_out = torch.empty((n, cfg.conv_width - 1, cfg.channels), dtype=q.dtype,
+                                     device=dev)
+    need = prefill_workspace_size(cfg, q.dtype, T, n)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
+    c = cfg.c()
+    st = _native.lib().gdn_prefill(
+        ctypes.byref(c), code, _dtype_code(out), _ptr(q), _ptr(k), _ptr(v), _ptr(conv_w_q), _ptr(conv_w_k),
+        _ptr(conv_w_v), _ptr(alpha), _ptr(beta), _ptr(cu_seqlens), n, T, _ptr(initial_state),
+        _ptr(final_state), _ptr(conv_state_in), _ptr(conv_state_out), _ptr(out), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _stream(stream))
+    _native.check("gdn_prefill", st)
+    return out, final_state, conv_state_out
+
+
+def gdn_decode_step(q, k, v, conv_w_q, conv_w_k, conv_w_v, alpha, beta, state, conv_state=None,
+                    *, state_slots=None, cfg: GdnConfig | None = None, out=None,
+                    out_dtype=torch.float32, stream=None):
+    """One token for each row of the batch; ``state`` (and ``conv_state``) update in place.
+
+    q, k [B, Hqk, 128], v [B, Hv, 128], alpha/beta [B, Hv]; state fp32 [R, Hv, 128, 128];
+    conv_state [R, 3, channels] or None; state_slots int32 [B] (row b uses state row
+    state_slots[b]) or None (identity).  Returns out [B, Hv, 128] (``out_dtype``).
+    """
+    B = q.shape[0]
+    cfg = cfg or GdnConfig(n_qk_heads=q.shape[1], n_v_heads=v.shape[1])
+    code = _dtype_code(q)
+    for t in (k, v, alpha, beta):
+        if t.dtype != q.dtype:
+            raise TypeError("q, k, v, alpha and beta must share one dtype")
+    if state.dtype != torch.float32:
+        raise TypeError("state must be float32")
+    if state_slots is not None and state_slots.dtype != torch.int32:
+        raise TypeError("state_slots must be int32")
+    if out is None:
+        out = torch.empty((B, cfg.n_v_heads, cfg.d_v), dtype=out_dtype, device=q.device)
+    c = cfg.c()
+    st = _native.lib().gdn_decode_step(
+        ctypes.byref(c), code, _dtype_code(out), _ptr(q), _ptr(k), _ptr(v), _ptr(conv_w_q), _ptr(conv_w_k),
+        _ptr(conv_w_v), _ptr(alpha), _ptr(beta), _ptr(state), _ptr(conv_state), _ptr(state_slots),
+        state.shape[0], _ptr(out), B, _stream(stream))
+    _native.check("gdn_decode_step", st)
+    return out

@@ -1,0 +1,171 @@
+// Single-token decode step on resident fp32 states (HBM-bound).
+//
+// The one-token case of the GATED DELTANET equations (page "ARCHITECTURE PREVIEW /
+// FIELD NOTES", section 03) with the kernel-4 ShortConv history shifted by one row.
+// With r = S^T k, p = S^T q (both over the OLD state S):
+//     e = v - alpha r,      y = S_t^T q = alpha p + beta (k.q) e,
+//     S_t = alpha S + beta k e^T.
+// so one read pass over S gives both reductions, and each state is read once and
+// written once.  S rows are streamed with 16-byte loads: warp w owns rows
+// 16w..16w+15 and lane l owns columns 4l..4l+3, so one warp instruction moves one
+// full 512-byte row.
+//
+// One CTA owns one decode row b and one QK head g with its Hv/Hqk value heads: it is
+// the only CTA that touches that row's q/k conv-state channels, so the in-place
+// conv-state shift needs no cross-CTA ordering.
+#include "gdn_common.cuh"
+#include "gdn_internal.h"
+
+namespace gdn {
+
+namespace {
+constexpr int kDecThreads = 256;
+constexpr int kDecWarps = kDecThreads / 32;
+constexpr int kRowsPerWarp = kHeadDim / kDecWarps;  // 16
+}  // namespace
+
+template <class T, class TO>
+__global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(DecodeParams p) {
+    __shared__ __align__(16) float qs[kHeadDim], ks[kHeadDim], vs[kHeadDim], es[kHeadDim];
+    __shared__ __align__(16) float red_r[kDecWarps][kHeadDim], red_p[kDecWarps][kHeadDim];
+    __shared__ float kq_s;
+
+    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    const int b = blockIdx.x / p.n_qk, g = blockIdx.x % p.n_qk;
+    const int G = p.n_v / p.n_qk;
+    const int slot = p.slots ? p.slots[b] : b;
+    const int qkc = p.n_qk * kHeadDim;
+    const int64_t ch = 2 * (int64_t)qkc + (int64_t)p.n_v * kHeadDim;
+    TO *outp = (TO *)p.out;
+
+    if (slot < 0 || slot >= p.n_rows) {  // skipped row: zero output, touch no state
+        for (int e = tid; e < G * kHeadDim; e += kDecThreads)
+            outp[(int64_t)b * p.n_v * kHeadDim + (int64_t)g * G * kHeadDim + e] = from_f32<TO>(0.f);
+        return;
+    }
+    T *cs = p.conv ? (T *)p.conv + (int64_t)slot * 3 * ch : nullptr;
+
+    // ---- q and k: conv (+ shift of their conv-state channels) and L2, warps 0 and 1
+    if (wid < 2) {
+        const bool isq = wid == 0;
+        const T *x = (const T *)(isq ? p.q : p.k) + ((int64_t)b * p.n_qk + g) * kHeadDim;
+        const float *w = isq ? p.wq : p.wk;
+        const int cc = (isq ? 0 : qkc) + g * kHeadDim + 4 * lane;  // conv-state channel
+        const int wc = g * kHeadDim + 4 * lane;                    // weight row
+        float cur[4], hst[3][4], y[4];
+        ld4(x + 4 * lane, cur);
+#pragma unroll
+        for (int j = 0; j < 3; ++j) {
+            if (cs) ld4(cs + (int64_t)j * ch + cc, hst[j]);
+            else hst[j][0] = hst[j][1] = hst[j][2] = hst[j][3] = 0.f;
+        }
+        float ss = 0.f;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            float4 wt = *reinterpret_cast<const float4 *>(w + (int64_t)(wc + c) * kConvW);
+            y[c] = wt.x * hst[0][c] + wt.y * hst[1][c] + wt.z * hst[2][c] + wt.w * cur[c];
+            ss += y[c] * y[c];
+        }
+        ss = warp_sum(ss);
+        const float inv = (isq ? p.q_scale : 1.f) * rsqrtf(ss + p.eps);
+        float *dst = isq ? qs : ks;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) dst[4 * lane + c] = y[c] * inv;
+        if (cs) {  // shift: rows 1,2 move to 0,1; the raw current row becomes row 2
+            st4(cs + 0 * ch + cc, hst[1]);
+            st4(cs + 1 * ch + cc, hst[2]);
+            cp4(cs + 2 * ch + cc, x + 4 * lane);
+        }
+    }
+    __syncthreads();
+    if (wid == 0) {
+        float d = 0.f;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) d += qs[4 * lane + c] * ks[4 * lane + c];
+        d = warp_sum(d);
+        if (lane == 0) kq_s = d;
+    }
+
+    for (int hh = 0; hh < G; ++hh) {
+        const int h = g * G + hh;
+        // ---- v conv for this V head (warp 2), overlapped with the state loads below
+        if (wid == 2) {
+            const T *x = (const T *)p.v + ((int64_t)b * p.n_v + h) * kHeadDim;
+            const int cc = 2 * qkc + h * kHeadDim + 4 * lane;
+            const int wc = h * kHeadDim + 4 * lane;
+            float cur[4], hst[3][4], y[4];
+            ld4(x + 4 * lane, cur);
+#pragma unroll
+            for (int j = 0; j < 3; ++j) {
+                if (cs) ld4(cs + (int64_t)j * ch + cc, hst[j]);
+                else hst[j][0] = hst[j][1] = hst[j][2] = hst[j][3] = 0.f;
+            }
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                float4 wt = *reinterpret_cast<const float4 *>(p.wv + (int64_t)(wc + c) * kConvW);
+                y[c] = wt.x * hst[0][c] + wt.y * hst[1][c] + wt.z * hst[2][c] + wt.w * cur[c];
+                vs[4 * lane + c] = y[c];
+            }
+            if (cs) {
+                st4(cs + 0 * ch + cc, hst[1]);
+                st4(cs + 1 * ch + cc, hst[2]);
+                cp4(cs + 2 * ch + cc, x + 4 * lane);
+            }
+        }
+        float *S = p.state + ((int64_t)slot * p.n_v + h) * kHeadDim * kHeadDim;
+        const int r0 = wid * kRowsPerWarp;
+        float4 s[kRowsPerWarp];
+#pragma unroll
+        for (int i = 0; i < kRowsPerWarp; ++i)
+            s[i] = __ldcs(reinterpret_cast<const float4 *>(S + (int64_t)(r0 + i) * kHeadDim + 4 * lane));
+        const float a = to_f32(((const T *)p.alpha)[(int64_t)b * p.n_v + h]);
+        const float be = to_f32(((const T *)p.beta)[(int64_t)b * p.n_v + h]);
+        float rr[4] = {0.f, 0.f, 0.f, 0.f}, pp[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int i = 0; i < kRowsPerWarp; ++i) {
+            const float kr = ks[r0 + i], qr = qs[r0 + i];
+            rr[0] = fmaf(s[i].x, kr, rr[0]); rr[1] = fmaf(s[i].y, kr, rr[1]);
+            rr[2] = fmaf(s[i].z, kr, rr[2]); rr[3] = fmaf(s[i].w, kr, rr[3]);
+            pp[0] = fmaf(s[i].x, qr, pp[0]); pp[1] = fmaf(s[i].y, qr, pp[1]);
+            pp[2] = fmaf(s[i].z, qr, pp[2]); pp[3] = fmaf(s[i].w, qr, pp[3]);
+        }
+        *reinterpret_cast<float4 *>(&red_r[wid][4 * lane]) = make_float4(rr[0], rr[1], rr[2], rr[3]);
+        *reinterpret_cast<float4 *>(&red_p[wid][4 * lane]) = make_float4(pp[0], pp[1], pp[2], pp[3]);
+        __syncthreads();
+        if (tid < kHeadDim) {
+            float r = 0.f, pq = 0.f;
+#pragma unroll
+            for (int w = 0; w < kDecWarps; ++w) { r += red_r[w][tid]; pq += red_p[w][tid]; }
+            const float e = vs[tid] - a * r;
+            es[tid] = e;
+            outp[((int64_t)b * p.n_v + h) * kHeadDim + tid] = from_f32<TO>(a * pq + be * kq_s * e);
+        }
+        __syncthreads();
+        const float4 e4 = *reinterpret_cast<const float4 *>(&es[4 * lane]);
+#pragma unroll
+        for (int i = 0; i < kRowsPerWarp; ++i) {
+            const float bk = be * ks[r0 + i];
+            float4 o;
+            o.x = fmaf(bk, e4.x, a * s[i].x);
+            o.y = fmaf(bk, e4.y, a * s[i].y);
+            o.z = fmaf(bk, e4.z, a * s[i].z);
+            o.w = fmaf(bk, e4.w, a * s[i].w);
+            __stcs(reinterpret_cast<float4 *>(S + (int64_t)(r0 + i) * kHeadDim + 4 * lane), o);
+        }
+    }
+}
+
+cudaError_t launch_decode(const DecodeParams &p, bool in_bf16, bool out_bf16, cudaStream_t s) {
+    if (p.batch <= 0) return cudaSuccess;
+    const unsigned grid = (unsigned)((int64_t)p.batch * p.n_qk);
+    if (in_bf16) {
+        if (out_bf16) decode_kernel<gdn::bf16, gdn::bf16><<<grid, kDecThreads, 0, s>>>(p);
+        else decode_kernel<gdn::bf16, float><<<grid, kDecThreads, 0, s>>>(p);
+    } else {
+        if (out_bf16) decode_kernel<float, gdn::bf16><<<grid, kDecThreads, 0, s>>>(p);
+        else decode_kernel<float, float><<<grid, kDecThreads, 0, s>>>(p);
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace gdn

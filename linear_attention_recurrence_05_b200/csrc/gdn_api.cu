@@ -1,0 +1,208 @@
+// C ABI of libgdn: argument validation, workspace layout and kernel launches.
+// The declarations and the contract of every entry point are in include/libgdn.h.
+#include <cmath>
+#include <cstring>
+
+#include "gdn_common.cuh"
+#include "gdn_internal.h"
+#include "libgdn.h"
+
+namespace gdn {
+
+static thread_local int t_last_cuda_error = 0;
+
+static size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+PrefillLayout prefill_layout(int n_qk, int n_v, int64_t T, int n_seqs) {
+    PrefillLayout L{};
+    L.max_chunks = (T + kChunk - 1) / kChunk + n_seqs;
+    size_t off = 0;
+    L.off_cu = off;      off = align_up(off + sizeof(int32_t) * (size_t)(n_seqs + 1), 256);
+    L.off_cfirst = off;  off = align_up(off + sizeof(int32_t) * (size_t)(n_seqs + 1), 256);
+    const size_t qk_bytes = (size_t)T * n_qk * 128 * sizeof(float);
+    const size_t v_bytes = (size_t)T * n_v * 128 * sizeof(float);
+    L.off_qh = off;      off = align_up(off + qk_bytes, 256);
+    L.off_kh = off;      off = align_up(off + qk_bytes, 256);
+    L.off_vh = off;      off = align_up(off + v_bytes, 256);
+    L.bytes = off;
+    return L;
+}
+
+}  // namespace gdn
+
+using namespace gdn;
+
+static gdn_status cuda_fail(cudaError_t e) {
+    t_last_cuda_error = (int)e;
+    return GDN_ERR_CUDA;
+}
+
+static bool aligned(const void *p, size_t a) { return ((uintptr_t)p % a) == 0; }
+
+static gdn_status check_config(const gdn_config *cfg, gdn_dtype dtype) {
+    if (!cfg) return GDN_ERR_INVALID_ARG;
+    if (dtype != GDN_BF16 && dtype != GDN_F32) return GDN_ERR_INVALID_ARG;
+    if (cfg->n_qk_heads <= 0 || cfg->n_v_heads <= 0) return GDN_ERR_INVALID_ARG;
+    if (cfg->n_v_heads % cfg->n_qk_heads != 0) return GDN_ERR_INVALID_ARG;
+    if (!std::isfinite(cfg->q_scale) || !std::isfinite(cfg->l2_eps) || cfg->l2_eps < 0.f)
+        return GDN_ERR_INVALID_ARG;
+    if (cfg->d_k != 128 || cfg->d_v != 128 || cfg->conv_width != 4) return GDN_ERR_UNSUPPORTED;
+    // keep channel counts and grid dimensions inside int range
+    // grid dimensions: 2*Hqk + Hv head slots ride in gridDim.y (<= 65535)
+    if (cfg->n_qk_heads > 4096 || cfg->n_v_heads > 16384) return GDN_ERR_UNSUPPORTED;
+    return GDN_OK;
+}
+
+static gdn_status check_device() {
+    int dev = 0, major = 0, minor = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e);
+    e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+    if (e != cudaSuccess) return cuda_fail(e);
+    e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (major != 10 || minor != 0) return GDN_ERR_UNSUPPORTED;  // built for sm_100a only
+    return GDN_OK;
+}
+
+extern "C" {
+
+const char *gdn_status_string(gdn_status s) {
+    switch (s) {
+        case GDN_OK: return "GDN_OK";
+        case GDN_ERR_INVALID_ARG: return "GDN_ERR_INVALID_ARG";
+        case GDN_ERR_UNSUPPORTED: return "GDN_ERR_UNSUPPORTED";
+        case GDN_ERR_WORKSPACE: return "GDN_ERR_WORKSPACE";
+        case GDN_ERR_CUDA: return "GDN_ERR_CUDA";
+        case GDN_ERR_TIMEOUT: return "GDN_ERR_TIMEOUT";
+    }
+    return "GDN_ERR_UNKNOWN";
+}
+
+int gdn_last_cuda_error(void) { return t_last_cuda_error; }
+
+int gdn_api_version(void) { return GDN_API_VERSION; }
+
+gdn_status gdn_prefill_workspace_size(const gdn_config *cfg, gdn_dtype dtype, int64_t total_tokens,
+                                      int n_seqs, size_t *bytes) {
+    gdn_status st = check_config(cfg, dtype);
+    if (st != GDN_OK) return st;
+    if (!bytes || total_tokens < 0 || total_tokens >= ((int64_t)1 << 31) || n_seqs < 0)
+        return GDN_ERR_INVALID_ARG;
+    *bytes = prefill_layout(cfg->n_qk_heads, cfg->n_v_heads, total_tokens, n_seqs).bytes;
+    return GDN_OK;
+}
+
+gdn_status gdn_prefill(const gdn_config *cfg, gdn_dtype dtype, gdn_dtype out_dtype,
+                       const void *q, const void *k,
+                       const void *v, const float *conv_w_q, const float *conv_w_k,
+                       const float *conv_w_v, const void *alpha, const void *beta,
+                       const int32_t *cu_seqlens, int n_seqs, int64_t total_tokens,
+                       const float *initial_state, float *final_state, const void *conv_state_in,
+                       void *conv_state_out, void *out, void *workspace, size_t workspace_bytes,
+                       cudaStream_t stream) {
+    gdn_status st = check_config(cfg, dtype);
+    if (st != GDN_OK) return st;
+    if (out_dtype != GDN_BF16 && out_dtype != GDN_F32) return GDN_ERR_INVALID_ARG;
+    if (n_seqs < 0 || total_tokens < 0 || total_tokens >= ((int64_t)1 << 31))
+        return GDN_ERR_INVALID_ARG;
+    if (n_seqs == 0) return GDN_OK;
+    if ((int64_t)n_seqs * cfg->n_v_heads * 4 >= ((int64_t)1 << 31)) return GDN_ERR_UNSUPPORTED;
+    const size_t eb = dtype == GDN_BF16 ? 2 : 4;
+    if (!cu_seqlens || !aligned(cu_seqlens, 4)) return GDN_ERR_INVALID_ARG;
+    if (total_tokens > 0) {
+        if (!q || !k || !v || !alpha || !beta || !out) return GDN_ERR_INVALID_ARG;
+        if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16))
+            return GDN_ERR_INVALID_ARG;
+        if (!aligned(alpha, eb) || !aligned(beta, eb)) return GDN_ERR_INVALID_ARG;
+    }
+    if (!conv_w_q || !conv_w_k || !conv_w_v) return GDN_ERR_INVALID_ARG;
+    if (!aligned(conv_w_q, 16) || !aligned(conv_w_k, 16) || !aligned(conv_w_v, 16))
+        return GDN_ERR_INVALID_ARG;
+    if ((initial_state && !aligned(initial_state, 16)) || (final_state && !aligned(final_state, 16)))
+        return GDN_ERR_INVALID_ARG;
+    if ((conv_state_in && !aligned(conv_state_in, 16)) ||
+        (conv_state_out && !aligned(conv_state_out, 16)))
+        return GDN_ERR_INVALID_ARG;
+    const PrefillLayout L = prefill_layout(cfg->n_qk_heads, cfg->n_v_heads, total_tokens, n_seqs);
+    if (!workspace || !aligned(workspace, 256) || workspace_bytes < L.bytes) return GDN_ERR_WORKSPACE;
+    st = check_device();
+    if (st != GDN_OK) return st;
+
+    const bool bf = dtype == GDN_BF16;
+    unsigned char *ws = (unsigned char *)workspace;
+    int32_t *cu = (int32_t *)(ws + L.off_cu);
+    int32_t *cfirst = (int32_t *)(ws + L.off_cfirst);
+    cudaError_t e = launch_seq_table(cu_seqlens, n_seqs, total_tokens, cu, cfirst, stream);
+    if (e != cudaSuccess) return cuda_fail(e);
+
+    if (total_tokens > 0) {
+        ConvParams cp{};
+        cp.q = q; cp.k = k; cp.v = v;
+        cp.wq = conv_w_q; cp.wk = conv_w_k; cp.wv = conv_w_v;
+        cp.conv_in = conv_state_in;
+        cp.qh = (float *)(ws + L.off_qh); cp.kh = (float *)(ws + L.off_kh);
+        cp.vh = (float *)(ws + L.off_vh);
+        cp.cu = cu; cp.cfirst = cfirst;
+        cp.n_seqs = n_seqs; cp.n_qk = cfg->n_qk_heads; cp.n_v = cfg->n_v_heads;
+        cp.q_scale = cfg->q_scale; cp.eps = cfg->l2_eps;
+        e = launch_conv_l2(cp, bf, L.max_chunks, stream);
+        if (e != cudaSuccess) return cuda_fail(e);
+    }
+    if (conv_state_out) {
+        e = launch_conv_state_out(q, k, v, conv_state_in, conv_state_out, cu, n_seqs,
+                                  cfg->n_qk_heads, cfg->n_v_heads, bf, stream);
+        if (e != cudaSuccess) return cuda_fail(e);
+    }
+    ScanParams sp{};
+    sp.qh = (const float *)(ws + L.off_qh); sp.kh = (const float *)(ws + L.off_kh);
+    sp.vh = (const float *)(ws + L.off_vh);
+    sp.alpha = alpha; sp.beta = beta; sp.cu = cu;
+    sp.init = initial_state; sp.fin = final_state; sp.out = out;
+    sp.n_seqs = n_seqs; sp.n_qk = cfg->n_qk_heads; sp.n_v = cfg->n_v_heads;
+    e = launch_scan_simt(sp, bf, out_dtype == GDN_BF16, stream);
+    if (e != cudaSuccess) return cuda_fail(e);
+    return GDN_OK;
+}
+
+gdn_status gdn_decode_step(const gdn_config *cfg, gdn_dtype dtype, gdn_dtype out_dtype,
+                           const void *q, const void *k,
+                           const void *v, const float *conv_w_q, const float *conv_w_k,
+                           const float *conv_w_v, const void *alpha, const void *beta, float *state,
+                           void *conv_state, const int32_t *state_slots, int n_state_rows,
+                           void *out, int batch, cudaStream_t stream) {
+    gdn_status st = check_config(cfg, dtype);
+    if (st != GDN_OK) return st;
+    if (out_dtype != GDN_BF16 && out_dtype != GDN_F32) return GDN_ERR_INVALID_ARG;
+    if (batch < 0 || n_state_rows < 0) return GDN_ERR_INVALID_ARG;
+    if (batch == 0) return GDN_OK;
+    if (!state_slots && n_state_rows < batch) return GDN_ERR_INVALID_ARG;
+    if ((int64_t)batch * cfg->n_qk_heads >= ((int64_t)1 << 31)) return GDN_ERR_UNSUPPORTED;
+    const size_t eb = dtype == GDN_BF16 ? 2 : 4;
+    if (!q || !k || !v || !alpha || !beta || !state || !out) return GDN_ERR_INVALID_ARG;
+    if (!conv_w_q || !conv_w_k || !conv_w_v) return GDN_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) ||
+        !aligned(state, 16) || !aligned(conv_w_q, 16) || !aligned(conv_w_k, 16) ||
+        !aligned(conv_w_v, 16))
+        return GDN_ERR_INVALID_ARG;
+    if (!aligned(alpha, eb) || !aligned(beta, eb)) return GDN_ERR_INVALID_ARG;
+    if (conv_state && !aligned(conv_state, 16)) return GDN_ERR_INVALID_ARG;
+    if (state_slots && !aligned(state_slots, 4)) return GDN_ERR_INVALID_ARG;
+    st = check_device();
+    if (st != GDN_OK) return st;
+
+    DecodeParams p{};
+    p.q = q; p.k = k; p.v = v;
+    p.wq = conv_w_q; p.wk = conv_w_k; p.wv = conv_w_v;
+    p.alpha = alpha; p.beta = beta;
+    p.state = state; p.conv = conv_state; p.slots = state_slots;
+    p.n_rows = n_state_rows; p.batch = batch;
+    p.n_qk = cfg->n_qk_heads; p.n_v = cfg->n_v_heads;
+    p.q_scale = cfg->q_scale; p.eps = cfg->l2_eps;
+    p.out = out;
+    cudaError_t e = launch_decode(p, dtype == GDN_BF16, out_dtype == GDN_BF16, stream);
+    if (e != cudaSuccess) return cuda_fail(e);
+    return GDN_OK;
+}
+
+}  // extern "C"

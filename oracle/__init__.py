@@ -144,20 +144,82 @@ def gdn_conv_l2_f64(q, k, v, w_q, w_k, w_v, cu_seqlens, *, n_qk_heads, n_v_heads
 
 
 # ------------------------------------------------------------------ stored-input helpers
+def _group_slices(shape, heads):
+    """QK groups needed by ``heads`` and the V heads of those groups (in order)."""
+    G = shape.n_v_heads // shape.n_qk_heads
+    groups = sorted({int(h) // G for h in heads})
+    vheads = [g * G + j for g in groups for j in range(G)]
+    remap = [groups.index(int(h) // G) * G + int(h) % G for h in heads]
+    return groups, vheads, remap
+
+
 def prefill(inp, heads=None, n_threads=None, q_scale=1.0, l2_eps=1e-6, initial_state=None,
             conv_state=None, mutant=0):
-    """Oracle on a ``gdn_inputs.PrefillInputs`` bundle (stored values widened to fp64)."""
+    """Oracle on a ``gdn_inputs.PrefillInputs`` bundle (stored values widened to fp64).
+
+    With ``heads`` only the QK groups those V heads read are widened and computed; the
+    returned arrays keep the full head axes, NaN outside the selected heads (the conv
+    state is returned for all channels).
+    """
     from gdn_inputs import stored_to_f64
     dt = inp.dtype
+    sh = inp.shape
     init = inp.initial_state if initial_state is None else initial_state
     cs = inp.conv_state if conv_state is None else conv_state
-    return gdn_prefill_f64(
-        stored_to_f64(inp.q, dt), stored_to_f64(inp.k, dt), stored_to_f64(inp.v, dt),
-        inp.w_q, inp.w_k, inp.w_v, stored_to_f64(inp.alpha, dt), stored_to_f64(inp.beta, dt),
-        inp.cu_seqlens, n_qk_heads=inp.shape.n_qk_heads, n_v_heads=inp.shape.n_v_heads,
-        initial_state=None if init is None else np.asarray(init, dtype=np.float64),
-        conv_state=None if cs is None else (cs if cs.dtype == np.float64 else stored_to_f64(cs, dt)),
-        heads=heads, q_scale=q_scale, l2_eps=l2_eps, n_threads=n_threads, mutant=mutant)
+    T, n = inp.total_tokens, inp.n_seqs
+    dk, dv = sh.d_k, sh.d_v
+
+    def f64(a):
+        return a if a.dtype == np.float64 else stored_to_f64(a, dt)
+    if heads is None:
+        groups, vheads, hsel = list(range(sh.n_qk_heads)), list(range(sh.n_v_heads)), None
+    else:
+        groups, vheads, hsel = _group_slices(sh, heads)
+    qkc = sh.n_qk_heads * dk
+    cs_sub = None
+    if cs is not None:
+        qch = [g * dk + i for g in groups for i in range(dk)]
+        vch = [h * dv + i for h in vheads for i in range(dv)]
+        cols = qch + [qkc + c for c in qch] + [2 * qkc + c for c in vch]
+        cs_sub = f64(np.asarray(cs)[:, :, cols])
+    y, fin, _ = gdn_prefill_f64(
+        f64(inp.q[:, groups]), f64(inp.k[:, groups]), f64(inp.v[:, vheads]),
+        inp.w_q.reshape(sh.n_qk_heads, dk, -1)[groups].reshape(len(groups) * dk, -1),
+        inp.w_k.reshape(sh.n_qk_heads, dk, -1)[groups].reshape(len(groups) * dk, -1),
+        inp.w_v.reshape(sh.n_v_heads, dv, -1)[vheads].reshape(len(vheads) * dv, -1),
+        f64(inp.alpha[:, vheads]), f64(inp.beta[:, vheads]), inp.cu_seqlens,
+        n_qk_heads=len(groups), n_v_heads=len(vheads),
+        initial_state=None if init is None else np.asarray(init, dtype=np.float64)[:, vheads],
+        conv_state=cs_sub, heads=hsel, q_scale=q_scale, l2_eps=l2_eps, n_threads=n_threads,
+        mutant=mutant)
+    y_full = np.full((T, sh.n_v_heads, dv), np.nan)
+    fin_full = np.full((n, sh.n_v_heads, dk, dv), np.nan)
+    y_full[:, vheads] = y
+    fin_full[:, vheads] = fin
+    # conv state out: the last W-1 raw rows of every channel (pure data movement)
+    return y_full, fin_full, _conv_state_rows(inp, cs)
+
+
+def _conv_state_rows(inp, cs):
+    from gdn_inputs import stored_to_f64
+    W1 = inp.shape.conv_width - 1
+    n = inp.n_seqs
+    ch = inp.shape.channels
+    out = np.zeros((n, W1, ch))
+    for b in range(n):
+        t0, t1 = int(inp.cu_seqlens[b]), int(inp.cu_seqlens[b + 1])
+        lo = max(t0, t1 - W1)
+        sh = inp.shape
+        qk = sh.n_qk_heads * sh.d_k
+        rows = np.concatenate([inp.q[lo:t1].reshape(t1 - lo, qk), inp.k[lo:t1].reshape(t1 - lo, qk),
+                               inp.v[lo:t1].reshape(t1 - lo, sh.n_v_heads * sh.d_v)], axis=1)
+        rows = rows.astype(np.float64) if rows.dtype != np.uint16 else stored_to_f64(rows, inp.dtype)
+        hist = np.zeros((W1, ch))
+        if cs is not None:
+            c = np.asarray(cs)[b]
+            hist = c.astype(np.float64) if c.dtype != np.uint16 else stored_to_f64(c, inp.dtype)
+        out[b] = np.vstack([hist, rows])[-W1:]
+    return out
 
 
 def decode_steps(shape, dtype, dec, w, state, conv_state, rows=None, heads=None, steps=None,

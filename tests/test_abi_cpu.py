@@ -1,0 +1,151 @@
+"""The C-ABI library loads, exports every entry point the header declares, and rejects
+bad arguments on the host before touching the device (CPU only: no compute call)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import linear_attention_recurrence_05_b200 as gdn
+from linear_attention_recurrence_05_b200 import _native
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "libgdn.h")
+
+
+def header_exports():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"GDN_EXPORT\s+[\w\s\*]*?\b(gdn_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_binding_exports():
+    assert header_exports() == sorted(_native.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol():
+    lib = _native.lib()
+    for name in header_exports():
+        assert hasattr(lib, name), name
+    assert lib.gdn_api_version() == 1
+
+
+def test_status_strings():
+    lib = _native.lib()
+    for code, name in _native.STATUS.items():
+        assert lib.gdn_status_string(code).decode() == name
+    assert lib.gdn_status_string(99).decode() == "GDN_ERR_UNKNOWN"
+
+
+def _cfg(**kw):
+    base = dict(n_qk_heads=16, n_v_heads=48, d_k=128, d_v=128, conv_width=4, q_scale=1.0,
+                l2_eps=1e-6)
+    base.update(kw)
+    return _native.GdnConfigC(*base.values())
+
+
+def _ws(cfg, dtype=0, T=8192, n=1):
+    out = ctypes.c_size_t(0)
+    st = _native.lib().gdn_prefill_workspace_size(ctypes.byref(cfg), dtype, T, n, ctypes.byref(out))
+    return st, out.value
+
+
+def test_workspace_size():
+    st, b = _ws(_cfg(), 0, 8192, 1)
+    assert st == 0
+    # q^, k^ (2 x T x 16 x 128) + v^ (T x 48 x 128) in fp32, plus two small int tables
+    assert b >= 8192 * (2 * 16 + 48) * 128 * 4
+    st4, b4 = _ws(_cfg(), 1, 8192, 1)
+    assert st4 == 0 and b4 == b
+    assert _ws(_cfg(), 0, 0, 3)[0] == 0
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(d_k=64), 2), (dict(d_v=256), 2), (dict(conv_width=3), 2),
+    (dict(n_v_heads=47), 1), (dict(n_qk_heads=0), 1), (dict(l2_eps=-1.0), 1),
+    (dict(q_scale=float("nan")), 1),
+])
+def test_config_rejected(kw, code):
+    assert _ws(_cfg(**kw))[0] == code
+
+
+def test_workspace_size_bad_args():
+    lib = _native.lib()
+    c = _cfg()
+    assert lib.gdn_prefill_workspace_size(ctypes.byref(c), 0, 10, 1, None) == 1
+    assert _ws(c, 0, -1, 1)[0] == 1
+    assert _ws(c, 0, 1 << 31, 1)[0] == 1
+    assert _ws(c, 7, 10, 1)[0] == 1
+    assert lib.gdn_prefill_workspace_size(None, 0, 10, 1, ctypes.byref(ctypes.c_size_t())) == 1
+
+
+def _prefill(**over):
+    """gdn_prefill with fake (never dereferenced) aligned device addresses."""
+    A = 1 << 20
+    args = dict(cfg=_cfg(), dtype=0, odt=1, q=A, k=2 * A, v=3 * A, wq=4 * A, wk=5 * A, wv=6 * A,
+                alpha=7 * A, beta=8 * A, cu=9 * A, n=1, T=100, init=None, fin=None, csi=None,
+                cso=None, out=10 * A, ws=11 * A, wsb=1 << 40, stream=None)
+    args.update(over)
+    c = args["cfg"]
+    return _native.lib().gdn_prefill(
+        ctypes.byref(c) if c is not None else None, args["dtype"], args["odt"], args["q"], args["k"], args["v"],
+        args["wq"], args["wk"], args["wv"], args["alpha"], args["beta"], args["cu"], args["n"],
+        args["T"], args["init"], args["fin"], args["csi"], args["cso"], args["out"], args["ws"],
+        args["wsb"], args["stream"])
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(q=None), 1), (dict(v=None), 1), (dict(out=None), 1), (dict(cu=None), 1),
+    (dict(wq=None), 1), (dict(q=(1 << 20) + 8), 1), (dict(out=(1 << 20) + 4), 1),
+    (dict(alpha=(1 << 20) + 1), 1), (dict(init=(1 << 20) + 8), 1), (dict(cso=(1 << 20) + 2), 1),
+    (dict(T=-5), 1), (dict(n=-1), 1), (dict(T=1 << 31), 1), (dict(dtype=3), 1),
+    (dict(ws=None), 3), (dict(wsb=16), 3), (dict(ws=(11 << 20) + 64), 3),
+    (dict(cfg=None), 1), (dict(cfg=_cfg(d_k=96)), 2), (dict(odt=2), 1),
+])
+def test_prefill_rejects_before_launch(over, code):
+    assert _prefill(**over) == code
+
+
+def test_prefill_zero_sequences_is_noop():
+    assert _prefill(n=0, q=None, k=None, v=None, out=None, ws=None) == 0
+
+
+def _decode(**over):
+    A = 1 << 20
+    args = dict(cfg=_cfg(), dtype=0, odt=1, q=A, k=2 * A, v=3 * A, wq=4 * A, wk=5 * A, wv=6 * A,
+                alpha=7 * A, beta=8 * A, state=9 * A, conv=10 * A, slots=None, rows=4, out=11 * A,
+                batch=4, stream=None)
+    args.update(over)
+    c = args["cfg"]
+    return _native.lib().gdn_decode_step(
+        ctypes.byref(c), args["dtype"], args["odt"], args["q"], args["k"], args["v"], args["wq"],
+        args["wk"], args["wv"], args["alpha"], args["beta"], args["state"], args["conv"], args["slots"],
+        args["rows"], args["out"], args["batch"], args["stream"])
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(state=None), 1), (dict(q=None), 1), (dict(out=None), 1), (dict(state=(9 << 20) + 4), 1),
+    (dict(conv=(10 << 20) + 2), 1), (dict(rows=2), 1), (dict(batch=-1), 1),
+    (dict(slots=(12 << 20) + 2), 1), (dict(cfg=_cfg(conv_width=2)), 2), (dict(odt=-1), 1),
+])
+def test_decode_rejects_before_launch(over, code):
+    assert _decode(**over) == code
+
+
+def test_decode_empty_batch_is_noop():
+    assert _decode(batch=0, q=None) == 0
+
+
+def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
+    monkeypatch.setattr(_native, "LIB_PATH", str(tmp_path / "missing.so"))
+    monkeypatch.setattr(_native, "_lib", None)
+    with pytest.raises(RuntimeError, match="no fallback"):
+        _native.lib()
+
+
+def test_product_does_not_import_oracle():
+    pkg = os.path.join(ROOT, "linear_attention_recurrence_05_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h", ".cpp")):
+                text = open(os.path.join(dirpath, f)).read()
+                assert "oracle" not in text.lower(), f

@@ -1,0 +1,157 @@
+"""gdn_prefill (CUDA, through the C ABI) against the fp64 oracle on the same seeded inputs.
+
+Bound: max|y_gpu - y_oracle| / rms(y_oracle) <= 2e-2 for bf16 storage and <= 1e-4 for
+fp32 storage, and the same bound on final states against rms(S_oracle).
+"""
+import numpy as np
+import pytest
+
+import gdn_inputs as gi
+import oracle
+from gdn_testutil import prefill_dev, rel_err, to_host_f64, tol
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import linear_attention_recurrence_05_b200 as gdn
+    return gdn
+
+
+def _check(inp, lib, heads=None, with_conv=True, label=""):
+    y, fin, cso = prefill_dev(inp, lib, with_conv_out=with_conv)
+    torch.cuda.synchronize()
+    yo, fo, co = oracle.prefill(inp, heads=heads)
+    sel = slice(None) if heads is None else list(heads)
+    ey = rel_err(to_host_f64(y)[:, sel], yo[:, sel])
+    es = rel_err(to_host_f64(fin)[:, sel], fo[:, sel])
+    t = tol(inp.dtype)
+    assert ey <= t, f"{label} output error {ey:.3e} > {t}"
+    assert es <= t, f"{label} final-state error {es:.3e} > {t}"
+    if with_conv:
+        got = to_host_f64(cso)
+        ref = co if inp.conv_state is None or inp.dtype == gi.F32 else co
+        assert np.array_equal(got, ref), f"{label} conv state differs"
+    return ey, es
+
+
+def test_workload0_tiny_fp32(lib):
+    inp = gi.make_workload(0)
+    _check(inp, lib, label="workload0")
+
+
+@pytest.mark.parametrize("dtype", [gi.BF16, gi.F32])
+def test_ragged_varlen_with_states(lib, dtype):
+    """Chunk edges and partial chunks: lengths around 64, an empty sequence, and both
+    initial states and conv states."""
+    shape = gi.GdnShape(n_qk_heads=4, n_v_heads=12)
+    inp = gi.make_prefill_inputs(shape, [1, 63, 64, 65, 0, 130, 200, 2], dtype, seed=77,
+                                 with_initial_state=True, with_conv_state=True)
+    _check(inp, lib, label=f"ragged-{dtype}")
+
+
+@pytest.mark.parametrize("dtype", [gi.BF16, gi.F32])
+def test_pages_heads_short(lib, dtype):
+    shape = gi.PAGES_SHAPE
+    inp = gi.make_prefill_inputs(shape, [300], dtype, seed=78)
+    _check(inp, lib, label=f"h16x48-{dtype}")
+
+
+def test_state_aliasing(lib):
+    """final_state may alias initial_state and conv_state_out may alias conv_state_in."""
+    shape = gi.GdnShape(n_qk_heads=2, n_v_heads=6)
+    inp = gi.make_prefill_inputs(shape, [70, 5, 0], gi.BF16, seed=79, with_initial_state=True,
+                                 with_conv_state=True)
+    from gdn_testutil import to_dev
+    d = inp.dtype
+    st = torch.from_numpy(inp.initial_state).cuda()
+    cs = to_dev(inp.conv_state, d)
+    cfg = lib.GdnConfig(2, 6)
+    y, _, _ = lib.gdn_prefill(
+        to_dev(inp.q, d), to_dev(inp.k, d), to_dev(inp.v, d), to_dev(inp.w_q, d), to_dev(inp.w_k, d),
+        to_dev(inp.w_v, d), to_dev(inp.alpha, d), to_dev(inp.beta, d),
+        torch.from_numpy(inp.cu_seqlens).cuda(), cfg=cfg, initial_state=st, final_state=st,
+        conv_state_in=cs, conv_state_out=cs)
+    torch.cuda.synchronize()
+    yo, fo, co = oracle.prefill(inp)
+    assert rel_err(to_host_f64(y), yo) <= tol(d)
+    assert rel_err(to_host_f64(st), fo) <= tol(d)
+    assert np.array_equal(to_host_f64(cs), co)
+
+
+def test_split_equals_whole_on_gpu(lib):
+    """Prefill of [0:T1] then [T1:T] from the returned states matches the oracle on [0:T]."""
+    shape = gi.GdnShape(n_qk_heads=2, n_v_heads=6)
+    inp = gi.make_prefill_inputs(shape, [300], gi.BF16, seed=80)
+    yo, fo, _ = oracle.prefill(inp)
+    T1 = 137
+    a = gi.make_prefill_inputs(shape, [T1], gi.BF16, seed=80)
+    b = gi.make_prefill_inputs(shape, [300 - T1], gi.BF16, seed=80)
+    for name in ("q", "k", "v", "alpha", "beta"):
+        setattr(a, name, getattr(inp, name)[:T1])
+        setattr(b, name, getattr(inp, name)[T1:])
+    ya, fa, ca = prefill_dev(a, lib, with_conv_out=True)
+    yb, fb, _ = lib.gdn_prefill(*[t for t in prefill_args(b, lib)], cfg=lib.GdnConfig(2, 6),
+                                initial_state=fa, conv_state_in=ca)
+    torch.cuda.synchronize()
+    y = np.concatenate([to_host_f64(ya), to_host_f64(yb)])
+    assert rel_err(y, yo) <= tol(gi.BF16)
+    assert rel_err(to_host_f64(fb), fo) <= tol(gi.BF16)
+
+
+def prefill_args(inp, lib):
+    from gdn_testutil import to_dev
+    d = inp.dtype
+    return (to_dev(inp.q, d), to_dev(inp.k, d), to_dev(inp.v, d), to_dev(inp.w_q, d),
+            to_dev(inp.w_k, d), to_dev(inp.w_v, d), to_dev(inp.alpha, d), to_dev(inp.beta, d),
+            torch.from_numpy(inp.cu_seqlens).cuda())
+
+
+def test_workload1_full_sampled_heads(lib):
+    """T = 8192, 16 QK / 48 V heads, bf16: every token of five sampled V heads."""
+    inp = gi.make_workload(1)
+    _check(inp, lib, heads=[0, 1, 2, 25, 47], with_conv=False, label="workload1")
+
+
+@pytest.mark.slow
+def test_workload2_full_sampled_heads(lib):
+    """T = 262,144 (mean alpha ~ 0.98), bf16: every token of two sampled V heads."""
+    inp = gi.make_workload(2)
+    _check(inp, lib, heads=[4, 46], with_conv=False, label="workload2")
+
+
+@pytest.mark.slow
+def test_workload4_varlen_prefix_states(lib):
+    """32 packed sequences (log-uniform 1K..64K) with nonzero initial states: the states of
+    the sampled (sequence, V head) pairs are the oracle's final states of a seeded 2048-token
+    prefill through the same layer; other pairs start from zero and are not compared."""
+    inp = gi.make_workload(4)
+    n = inp.n_seqs
+    heads = [3, 30]
+    warm = gi.warmup_prefill_inputs(4, range(n))
+    _, wf, wc = oracle.prefill(warm, heads=heads)
+    init = np.zeros((n, 48, 128, 128), np.float32)
+    init[:, heads] = wf[:, heads].astype(np.float32)
+    inp.initial_state = init
+    inp.conv_state = gi.quantize(wc.astype(np.float32), gi.BF16)
+    _check(inp, lib, heads=heads, with_conv=False, label="workload4")
+
+
+def test_bf16_output(lib):
+    """out_dtype = bf16: same bound plus each entry's own bf16 rounding."""
+    from gdn_testutil import rel_err_bf16_out, to_dev
+    shape = gi.GdnShape(n_qk_heads=4, n_v_heads=12)
+    inp = gi.make_prefill_inputs(shape, [200, 65], gi.BF16, seed=81, with_initial_state=True)
+    y, fin, _ = lib.gdn_prefill(*prefill_args(inp, lib), cfg=lib.GdnConfig(4, 12),
+                                initial_state=torch.from_numpy(inp.initial_state).cuda(),
+                                out_dtype=torch.bfloat16)
+    torch.cuda.synchronize()
+    assert y.dtype == torch.bfloat16
+    yo, fo, _ = oracle.prefill(inp)
+    assert rel_err_bf16_out(to_host_f64(y), yo) <= tol(gi.BF16)
+    assert rel_err(to_host_f64(fin), fo) <= tol(gi.BF16)
