@@ -1,0 +1,491 @@
+#!/usr/bin/env python
+"""Throughput of libgdn (the Gated DeltaNet token mixer) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints ONE JSON line (rank 0).  `value` is prefill tokens/s of one GDN layer at the
+pages' shape (T = 8192, 16 QK / 48 V heads, d = 128, bf16 inputs, fp32 state, fp32
+output) with inputs resident in HBM and L2 flushed between steps; the `decode` object
+is the batched decode workload (256 rows x 1024 consecutive steps on resident fp32
+states).  `e2e` repeats the prefill measurement through the public API from pinned
+host buffers, copies included.  `roofline` describes the dominant prefill kernel,
+timed live with the library's launch trace.  `cpu_baseline` is the fp64 oracle on
+the host cores (rank 0, N = 1 only).
+
+With N > 1 (torchrun), every rank runs its own independent problem of the same size
+(the path shards by sequence with no exchange): weak scaling, no data-path collective;
+the time is the max over ranks.  `--impl reference` times the oracle instead (the
+only reference this path has), rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import gdn_inputs as gi  # noqa: E402
+
+METRIC = "GDN prefill tokens/s and decode tokens/s on 1 B200; % of tensor/HBM roofline"
+UNIT = "tokens/s"
+D = 128
+CHUNK = 64
+# algorithmic work of the chunked prefill per (token, V head), full 64-row tiles:
+# W.S, K~^T.u, Q.S (2 d^2 each) + T.(beta gamma K), T.(beta V), P.u (2 C d each)
+# + K.K^T and Q.K^T (2 C d each, shared by the 3 V heads of a QK head)
+PREFILL_FLOP_TV = 6 * D * D + 2 * CHUNK * D * (3 + 2 / 3)
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                  "sm_max_mhz": 1965.0}
+TF32_PER_BF16 = 1.1 / 2.25   # nominal dense tf32 : bf16 tensor throughput on B200
+FP32_LANES_PER_SM = 128
+N_SM = 148
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return json.load(f), "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi clock/throttle samples (200 ms) while the timed region runs."""
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_id: str):
+        self.device_id = device_id
+        self.proc = None
+        self.tmp = None
+
+    def start(self):
+        try:
+            self.tmp = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.device_id, f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=self.tmp, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        return self
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.tmp.flush()
+        self.tmp.seek(0)
+        rows = [r.split(",") for r in self.tmp.read().strip().splitlines() if r.count(",") >= 7]
+        self.tmp.close()
+        os.unlink(self.tmp.name)
+        sm, mx, reasons = [], [], set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for r in rows:
+            try:
+                sm.append(float(r[0]))
+                mx.append(float(r[1]))
+            except ValueError:
+                continue
+            for name, val in zip(names, r[4:8]):
+                if val.strip().lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def device_id_for_smi() -> str:
+    import torch
+    try:
+        u = str(torch.cuda.get_device_properties(torch.cuda.current_device()).uuid)
+        return u if u.startswith("GPU-") else "GPU-" + u
+    except Exception:
+        vis = os.environ.get("CUDA_VISIBLE_DEVICES", "0").split(",")
+        return vis[torch.cuda.current_device()] if vis and vis[0] else "0"
+
+
+# ----------------------------------------------------------------------------- helpers
+def to_dev(a, torch):
+    if a.dtype == np.uint16:
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).cuda()
+    return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+
+class Dist:
+    def __init__(self, torch):
+        self.torch = torch
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        self.pg = None
+
+    def init(self):
+        import datetime
+        torch = self.torch
+        torch.cuda.set_device(self.local)
+        if self.world > 1:
+            import torch.distributed as dist
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                    device_id=torch.device("cuda", self.local))
+            self.pg = dist
+        return self
+
+    def barrier(self):
+        if self.pg:
+            self.pg.barrier()
+        self.torch.cuda.synchronize()
+
+    def max(self, x: float) -> float:
+        if not self.pg:
+            return x
+        t = self.torch.tensor([x], dtype=self.torch.float64, device="cuda")
+        self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.pg:
+            self.pg.destroy_process_group()
+
+
+def gpu_gate_inputs(torch, gen, shape, c, dtype):
+    x = torch.randn(shape, generator=gen, device="cuda")
+    alpha = torch.exp(-c * torch.nn.functional.softplus(x)).to(dtype)
+    beta = torch.sigmoid(torch.randn(shape, generator=gen, device="cuda")).to(dtype)
+    return alpha, beta
+
+
+# ----------------------------------------------------------------------------- prefill
+def bench_prefill(args, dist, torch, gdn, peaks):
+    w = gi.WORKLOADS[1]
+    shape = w["shape"]
+    T = w["lengths"][0]
+    seed = gi.workload_seed(1) + 7919 * dist.rank  # rank 0 runs the workload itself
+    inp = gi.make_prefill_inputs(shape, [T], w["dtype"], seed, c=w["c"],
+                                 weights=gi.workload_weights(1))
+    q, k, v = to_dev(inp.q, torch), to_dev(inp.k, torch), to_dev(inp.v, torch)
+    wq, wk, wv = to_dev(inp.w_q, torch), to_dev(inp.w_k, torch), to_dev(inp.w_v, torch)
+    al, be = to_dev(inp.alpha, torch), to_dev(inp.beta, torch)
+    cu = torch.from_numpy(inp.cu_seqlens).cuda()
+    cfg = gdn.GdnConfig(shape.n_qk_heads, shape.n_v_heads)
+    out = torch.empty((T, shape.n_v_heads, D), dtype=torch.float32, device="cuda")
+    fin = torch.empty((1, shape.n_v_heads, D, D), dtype=torch.float32, device="cuda")
+    ws = torch.empty(gdn.prefill_workspace_size(cfg, torch.bfloat16, T, 1), dtype=torch.uint8,
+                     device="cuda")
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")  # > 126 MB L2
+
+    def call():
+        gdn.gdn_prefill(q, k, v, wq, wk, wv, al, be, cu, cfg=cfg, out=out, final_state=fin,
+                        workspace=ws)
+
+    for _ in range(args.warmup):
+        call()
+    K = args.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(K)]
+    trace = gdn.LaunchTrace(capacity=16 * K)
+    clocks = ClockSampler(device_id_for_smi())
+    dist.barrier()
+    clocks.start()
+    with trace:
+        for i in range(K):
+            flush.zero_()
+            ev[i][0].record()
+            call()
+            ev[i][1].record()
+    dist.barrier()
+    clk = clocks.stop()
+    ms = sum(a.elapsed_time(b) for a, b in ev)
+    ms_max = dist.max(ms)
+    recs = trace.records()
+    per_kernel = {}
+    for name, t in recs:
+        per_kernel.setdefault(name, []).append(t)
+
+    # e2e: public API from pinned host buffers, copies inside the timed region
+    hq, hk, hv = (torch.empty(x.shape, dtype=x.dtype, pin_memory=True) for x in (q, k, v))
+    ha, hb = (torch.empty(x.shape, dtype=x.dtype, pin_memory=True) for x in (al, be))
+    for h, d in ((hq, q), (hk, k), (hv, v), (ha, al), (hb, be)):
+        h.copy_(d)
+    hy = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+    h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv, ha, hb))
+    d2h = hy.numel() * hy.element_size()
+    ev2 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(K)]
+    dist.barrier()
+    for i in range(K):
+        flush.zero_()
+        ev2[i][0].record()
+        for h, d in ((hq, q), (hk, k), (hv, v), (ha, al), (hb, be)):
+            d.copy_(h, non_blocking=True)
+        call()
+        hy.copy_(out, non_blocking=True)
+        ev2[i][1].record()
+    dist.barrier()
+    e2e_ms = dist.max(sum(a.elapsed_time(b) for a, b in ev2))
+
+    tokens_all = T * dist.world * K
+    return {
+        "value": tokens_all / (ms_max / 1e3), "ms_per_step": ms_max / K, "clocks": clk,
+        "per_kernel": {n: {"launches": len(v), "avg_ms": sum(v) / len(v), "total_ms": sum(v)}
+                       for n, v in per_kernel.items()},
+        "launches": trace.count, "tokens_per_launch": T, "n_v_heads": shape.n_v_heads,
+        "e2e": {"value": tokens_all / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / K},
+    }
+
+
+def prefill_roofline(res, peaks, peak_src):
+    pk = res["per_kernel"]
+    dom = max(pk, key=lambda n: pk[n]["total_ms"])
+    avg_s = pk[dom]["avg_ms"] / 1e3
+    T, Hv = res["tokens_per_launch"], res["n_v_heads"]
+    step_ms = sum(v["total_ms"] for v in pk.values())
+    share = {n: round(v["total_ms"] / step_ms, 4) for n, v in pk.items()}
+    if dom == "scan_simt":
+        flops = PREFILL_FLOP_TV * T * Hv
+        peak = N_SM * FP32_LANES_PER_SM * 2 * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12
+        return {"kernel": dom, "bound": "alu", "achieved": flops / avg_s / 1e12, "peak": peak,
+                "unit": "TFLOP/s", "frac": flops / avg_s / 1e12 / peak, "traffic": None,
+                "peak_source": f"148 SMs x 128 fp32 FMA lanes x 2 x {peaks.get('sm_max_mhz')} MHz",
+                "algorithmic_per_launch": flops, "kernel_share": share}
+    if dom.startswith("prefill_tc"):
+        flops = PREFILL_FLOP_TV * T * Hv
+        peak = peaks["bf16_tflops"] * TF32_PER_BF16
+        return {"kernel": dom, "bound": "tensor", "achieved": flops / avg_s / 1e12, "peak": peak,
+                "unit": "TFLOP/s", "frac": flops / avg_s / 1e12 / peak, "traffic": None,
+                "peak_source": f"tf32 = {peak_src} bf16 {peaks['bf16_tflops']} x 1.1/2.25 nominal",
+                "algorithmic_per_launch": flops, "kernel_share": share}
+    # a memory-bound kernel dominates
+    byts = (2 * 16 * D * 2 + 48 * D * 2 + 3 * 16 * 4 * D) * T
+    return {"kernel": dom, "bound": "hbm", "achieved": byts / avg_s / 1e9, "peak": peaks["hbm_gbs"],
+            "unit": "GB/s", "frac": byts / avg_s / 1e9 / peaks["hbm_gbs"], "traffic": None,
+            "peak_source": peak_src, "kernel_share": share}
+
+
+# ----------------------------------------------------------------------------- decode
+def decode_bytes_per_row(shape, in_bytes=2, out_bytes=4):
+    Hqk, Hv = shape.n_qk_heads, shape.n_v_heads
+    ch = shape.channels
+    return (2 * Hv * D * D * 4            # state read + write
+            + 6 * ch * in_bytes           # conv state: 3 rows read, 3 rows written
+            + ch * in_bytes               # this step's raw q, k, v
+            + Hv * D * out_bytes          # y
+            + 2 * Hv * in_bytes)          # alpha, beta
+
+
+def bench_decode(args, dist, torch, gdn, peaks, peak_src):
+    w = gi.WORKLOADS[3]
+    shape = w["shape"]
+    B, steps, warm_T = w["batch"], args.decode_steps, w["warm_tokens"]
+    H, Hv, ch = shape.n_qk_heads, shape.n_v_heads, shape.channels
+    bf = torch.bfloat16
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(gi.workload_seed(3) + 7919 * dist.rank)
+    wq, wk, wv = (to_dev(x, torch) for x in gi.workload_weights(3))
+    cfg = gdn.GdnConfig(H, Hv)
+    # resident states: final states of a seeded warm_T-token prefill per row (libgdn prefill)
+    state = torch.empty((B, Hv, D, D), dtype=torch.float32, device="cuda")
+    conv = torch.empty((B, 3, ch), dtype=bf, device="cuda")
+    per = 32
+    for r0 in range(0, B, per):
+        n = min(per, B - r0)
+        Tw = n * warm_T
+        q = torch.randn((Tw, H, D), generator=gen, device="cuda").to(bf)
+        k = torch.randn((Tw, H, D), generator=gen, device="cuda").to(bf)
+        v = torch.randn((Tw, Hv, D), generator=gen, device="cuda").to(bf)
+        al, be = gpu_gate_inputs(torch, gen, (Tw, Hv), w["c"], bf)
+        cu = torch.arange(n + 1, dtype=torch.int32, device="cuda") * warm_T
+        gdn.gdn_prefill(q, k, v, wq, wk, wv, al, be, cu, cfg=cfg, final_state=state[r0:r0 + n],
+                        conv_state_out=conv[r0:r0 + n], out=torch.empty((Tw, Hv, D), device="cuda"))
+        del q, k, v, al, be
+    torch.cuda.synchronize()
+    # fresh inputs for every step
+    dq = torch.randn((steps, B, H, D), generator=gen, device="cuda").to(bf)
+    dk = torch.randn((steps, B, H, D), generator=gen, device="cuda").to(bf)
+    dv = torch.randn((steps, B, Hv, D), generator=gen, device="cuda").to(bf)
+    da, db = gpu_gate_inputs(torch, gen, (steps, B, Hv), w["c"], bf)
+    out = torch.empty((B, Hv, D), dtype=torch.float32, device="cuda")
+    state0, conv0 = state.clone(), conv.clone()
+
+    def step(i):
+        gdn.gdn_decode_step(dq[i], dk[i], dv[i], wq, wk, wv, da[i], db[i], state, conv, cfg=cfg,
+                            out=out)
+
+    for i in range(args.warmup):
+        step(i % steps)
+    state.copy_(state0)
+    conv.copy_(conv0)
+    trace = gdn.LaunchTrace(capacity=steps + 8)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(device_id_for_smi())
+    dist.barrier()
+    clocks.start()
+    with trace:
+        e0.record()
+        for i in range(steps):
+            step(i)
+        e1.record()
+    dist.barrier()
+    clk = clocks.stop()
+    ms = dist.max(e0.elapsed_time(e1))
+    recs = [t for n, t in trace.records() if n == "decode"]
+    avg_s = sum(recs) / len(recs) / 1e3
+    bpr = decode_bytes_per_row(shape)
+    achieved = bpr * B / avg_s / 1e9
+
+    # e2e: pinned host inputs (a ring of 32 distinct steps), y read back every step
+    ring = 32
+    hq, hk, hv, ha, hb = (torch.empty((ring,) + tuple(x.shape[1:]), dtype=x.dtype, pin_memory=True)
+                          for x in (dq, dk, dv, da, db))
+    for h, d in ((hq, dq), (hk, dk), (hv, dv), (ha, da), (hb, db)):
+        h.copy_(d[:ring])
+    hy = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+    h2d = sum(x[0].numel() * x.element_size() for x in (hq, hk, hv, ha, hb))
+    d2h = hy.numel() * hy.element_size()
+    bq, bk, bv, ba, bb = (torch.empty_like(x[0]) for x in (dq, dk, dv, da, db))
+    state.copy_(state0)
+    conv.copy_(conv0)
+    dist.barrier()
+    e2, e3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e2.record()
+    for i in range(steps):
+        j = i % ring
+        for d, h in ((bq, hq), (bk, hk), (bv, hv), (ba, ha), (bb, hb)):
+            d.copy_(h[j], non_blocking=True)
+        gdn.gdn_decode_step(bq, bk, bv, wq, wk, wv, ba, bb, state, conv, cfg=cfg, out=out)
+        hy.copy_(out, non_blocking=True)
+    e3.record()
+    dist.barrier()
+    e2e_ms = dist.max(e2.elapsed_time(e3))
+    toks = B * steps * dist.world
+    return {
+        "value": toks / (ms / 1e3), "unit": UNIT, "workload": w["name"], "batch": B,
+        "steps": steps, "ms_per_step": ms / steps, "launches": trace.count, "clocks": clk,
+        "roofline": {"kernel": "decode", "bound": "hbm", "achieved": achieved,
+                     "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
+                     "traffic": None, "peak_source": peak_src,
+                     "algorithmic_bytes_per_row": bpr, "rows_per_launch": B},
+        "e2e": {"value": toks / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "note": "host inputs cycle through 32 pinned step sets"},
+    }
+
+
+# ----------------------------------------------------------------------------- oracle
+def oracle_tokens_per_s(target_s: float, seed_offset: int = 0):
+    """Time the fp64 oracle on a prefix of the prefill workload (all 48 V heads),
+    sized to take about target_s seconds.  Returns (tokens/s, threads, sample text, secs)."""
+    import oracle
+    w = gi.WORKLOADS[1]
+    threads = oracle.default_threads()
+
+    def run(T):
+        inp = gi.make_prefill_inputs(w["shape"], [T], w["dtype"], gi.workload_seed(1) + seed_offset,
+                                     c=w["c"], weights=gi.workload_weights(1))
+        t0 = time.perf_counter()
+        oracle.prefill(inp, n_threads=threads)
+        return time.perf_counter() - t0
+    probe_T = 128
+    dt = run(probe_T)
+    T = int(min(8192, max(probe_T, probe_T * target_s / max(dt, 1e-6))))
+    dt = run(T)
+    return T / dt, threads, f"first {T} tokens of the T=8192 layer, all 48 V heads", dt
+
+
+def run_reference(args):
+    """--impl reference: the fp64 oracle timed on the host cores (rank 0 only)."""
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if int(os.environ.get("RANK", "0")) != 0:
+        return
+    import oracle
+    oracle.build()
+    for _ in range(args.warmup):
+        oracle_tokens_per_s(0.2)
+    vals, secs, sample, threads = [], [], "", 1
+    for _ in range(args.steps):
+        v, threads, sample, dt = oracle_tokens_per_s(args.ref_step_s)
+        vals.append(v)
+        secs.append(dt)
+    value = statistics.median(vals)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * statistics.median(secs),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": gi.WORKLOADS[1]["name"], "T": 8192, "n_qk_heads": 16,
+                   "n_v_heads": 48, "d": D, "sample": sample},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------------- main
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--decode-steps", type=int, default=1024)
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-baseline-s", type=float, default=15.0)
+    ap.add_argument("--ref-step-s", type=float, default=5.0)
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    if args.impl == "reference":
+        run_reference(args)
+        return
+
+    import torch
+    import linear_attention_recurrence_05_b200 as gdn
+    dist = Dist(torch).init()
+    peaks, peak_src = load_peaks()
+    pre = bench_prefill(args, dist, torch, gdn, peaks)
+    roof = prefill_roofline(pre, peaks, peak_src)
+    dec = None if args.no_decode else bench_decode(args, dist, torch, gdn, peaks, peak_src)
+    cpu = None
+    if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
+        v, threads, sample, dt = oracle_tokens_per_s(args.cpu_baseline_s)
+        cpu = {"value": v, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": sample,
+               "seconds": dt}
+    if dist.rank == 0:
+        line = {
+            "metric": METRIC, "value": pre["value"], "unit": UNIT, "n_gpus": dist.world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": pre["ms_per_step"],
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic",
+            "config": {"workload": gi.WORKLOADS[1]["name"], "T": 8192, "n_qk_heads": 16,
+                       "n_v_heads": 48, "d": D, "chunk": CHUNK, "inputs": "bf16",
+                       "out": "f32", "state": "f32", "l2": "flushed: 256 MiB write between steps",
+                       "parallelism": f"dp{dist.world} (independent sequences per GPU)"},
+            "clocks": pre["clocks"], "e2e": pre["e2e"], "gpu_launches": pre["launches"],
+            "roofline": roof, "kernels": pre["per_kernel"], "cpu_baseline": cpu, "decode": dec,
+            "peaks": peak_src,
+        }
+        print(json.dumps(line), flush=True)
+    dist.close()
+
+
+if __name__ == "__main__":
+    main()

@@ -167,6 +167,26 @@ GDN_EXPORT gdn_status gdn_decode_step(const gdn_config *cfg, gdn_dtype dtype, gd
                            const int32_t *state_slots, int n_state_rows,
                            void *out, int batch, cudaStream_t stream);
 
+/*
+ * Launch trace (a profiling aid; no counterpart on the pages).  While a trace is
+ * active on a host thread, every kernel that a libgdn call made on that thread
+ * launches is bracketed on its launch stream: entries[i].start is recorded just
+ * before the i-th launch and entries[i].stop just after it, and entries[i].kernel is
+ * set to the kernel's name (static storage).  The caller creates the events (with
+ * timing enabled) and reads elapsed times after synchronising.  Launches beyond
+ * `capacity` are counted but not recorded.  gdn_trace_end() stops the trace and
+ * returns the number of launches seen since gdn_trace_begin().  Tracing never
+ * changes what the kernels compute.
+ */
+typedef struct {
+    cudaEvent_t start;
+    cudaEvent_t stop;
+    const char *kernel;
+} gdn_trace_entry;
+
+GDN_EXPORT void gdn_trace_begin(gdn_trace_entry *entries, int capacity);
+GDN_EXPORT int gdn_trace_end(void);
+
 #ifdef __cplusplus
 }
 #endif

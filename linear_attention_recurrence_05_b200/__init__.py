@@ -149,3 +149,38 @@ def gdn_decode_step(q, k, v, conv_w_q, conv_w_k, conv_w_v, alpha, beta, state, c
         state.shape[0], _ptr(out), B, _stream(stream))
     _native.check("gdn_decode_step", st)
     return out
+
+
+class LaunchTrace:
+    """Context manager around gdn_trace_begin/gdn_trace_end (this host thread only).
+
+    with LaunchTrace(capacity) as tr: ...libgdn calls...
+    torch.cuda.synchronize(); tr.records() -> [(kernel_name, milliseconds), ...]
+    """
+
+    def __init__(self, capacity: int = 1024):
+        self.capacity = int(capacity)
+        self.events = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                       for _ in range(self.capacity)]
+        s = torch.cuda.current_stream()
+        for a, b in self.events:  # materialise the event handles
+            a.record(s)
+            b.record(s)
+        self._arr = (_native.TraceEntryC * max(self.capacity, 1))()
+        for i, (a, b) in enumerate(self.events):
+            self._arr[i].start = a.cuda_event
+            self._arr[i].stop = b.cuda_event
+        self.count = 0
+
+    def __enter__(self):
+        _native.lib().gdn_trace_begin(self._arr, self.capacity)
+        return self
+
+    def __exit__(self, *exc):
+        self.count = _native.lib().gdn_trace_end()
+        return False
+
+    def records(self):
+        n = min(self.count, self.capacity)
+        return [(self._arr[i].kernel.decode(), self.events[i][0].elapsed_time(self.events[i][1]))
+                for i in range(n)]

@@ -19,7 +19,12 @@ STATUS = {0: "GDN_OK", 1: "GDN_ERR_INVALID_ARG", 2: "GDN_ERR_UNSUPPORTED", 3: "G
 
 # every entry point the header declares (checked by the CPU test suite)
 EXPORTS = ("gdn_status_string", "gdn_last_cuda_error", "gdn_api_version",
-           "gdn_prefill_workspace_size", "gdn_prefill", "gdn_decode_step")
+           "gdn_prefill_workspace_size", "gdn_prefill", "gdn_decode_step", "gdn_trace_begin",
+           "gdn_trace_end")
+
+
+class TraceEntryC(ctypes.Structure):
+    _fields_ = [("start", ctypes.c_void_p), ("stop", ctypes.c_void_p), ("kernel", ctypes.c_char_p)]
 
 
 class GdnConfigC(ctypes.Structure):
@@ -73,6 +78,10 @@ def lib():
                                           fp, fp, vp, vp, fp, vp, i32p, ctypes.c_int, vp,
                                           ctypes.c_int, vp]
             L.gdn_decode_step.restype = ctypes.c_int
+            L.gdn_trace_begin.argtypes = [ctypes.POINTER(TraceEntryC), ctypes.c_int]
+            L.gdn_trace_begin.restype = None
+            L.gdn_trace_end.argtypes = []
+            L.gdn_trace_end.restype = ctypes.c_int
             _lib = L
         return _lib
 

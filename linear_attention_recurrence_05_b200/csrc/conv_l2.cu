@@ -76,6 +76,7 @@ __global__ void __launch_bounds__(1024) seq_table_kernel(const int32_t *__restri
 
 cudaError_t launch_seq_table(const int32_t *cu_in, int n_seqs, int64_t T, int32_t *cu,
                              int32_t *cfirst, cudaStream_t s) {
+    TraceLaunch tl(s, "seq_table");
     seq_table_kernel<<<1, 1024, 0, s>>>(cu_in, n_seqs, (int)T, cu, cfirst);
     return cudaGetLastError();
 }
@@ -162,6 +163,7 @@ __global__ void __launch_bounds__(128) conv_l2_kernel(ConvParams p) {
 cudaError_t launch_conv_l2(const ConvParams &p, bool bf16, int64_t max_chunks, cudaStream_t s) {
     if (max_chunks <= 0) return cudaSuccess;
     dim3 grid((unsigned)max_chunks, 2 * p.n_qk + p.n_v);
+    TraceLaunch tl(s, "conv_l2");
     if (bf16) conv_l2_kernel<gdn::bf16><<<grid, 128, 0, s>>>(p);
     else conv_l2_kernel<float><<<grid, 128, 0, s>>>(p);
     return cudaGetLastError();
@@ -204,6 +206,7 @@ cudaError_t launch_conv_state_out(const void *q, const void *k, const void *v,
     if (n_seqs <= 0) return cudaSuccess;
     const int64_t ch4 = (2 * (int64_t)n_qk * kHeadDim + (int64_t)n_v * kHeadDim) / 4;
     dim3 grid((unsigned)n_seqs, (unsigned)((ch4 + 255) / 256));
+    TraceLaunch tl(s, "conv_state_out");
     if (bf16)
         conv_state_out_kernel<gdn::bf16><<<grid, 256, 0, s>>>(
             (const gdn::bf16 *)q, (const gdn::bf16 *)k, (const gdn::bf16 *)v,

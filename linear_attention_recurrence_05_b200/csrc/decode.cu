@@ -158,6 +158,7 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(DecodeParams p) 
 cudaError_t launch_decode(const DecodeParams &p, bool in_bf16, bool out_bf16, cudaStream_t s) {
     if (p.batch <= 0) return cudaSuccess;
     const unsigned grid = (unsigned)((int64_t)p.batch * p.n_qk);
+    TraceLaunch tl(s, "decode");
     if (in_bf16) {
         if (out_bf16) decode_kernel<gdn::bf16, gdn::bf16><<<grid, kDecThreads, 0, s>>>(p);
         else decode_kernel<gdn::bf16, float><<<grid, kDecThreads, 0, s>>>(p);

@@ -11,6 +11,26 @@ namespace gdn {
 
 static thread_local int t_last_cuda_error = 0;
 
+// per-host-thread launch trace (see gdn_trace_begin)
+static thread_local gdn_trace_entry *t_trace = nullptr;
+static thread_local int t_trace_cap = 0;
+static thread_local int t_trace_n = 0;
+static thread_local bool t_trace_on = false;
+
+TraceLaunch::TraceLaunch(cudaStream_t s, const char *kernel) : stream(s), entry(nullptr) {
+    if (!t_trace_on) return;
+    if (t_trace_n < t_trace_cap && t_trace) {
+        entry = &t_trace[t_trace_n];
+        entry->kernel = kernel;
+        cudaEventRecord(entry->start, s);
+    }
+    ++t_trace_n;
+}
+
+TraceLaunch::~TraceLaunch() {
+    if (entry) cudaEventRecord(entry->stop, stream);
+}
+
 static size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 PrefillLayout prefill_layout(int n_qk, int n_v, int64_t T, int n_seqs) {
@@ -82,6 +102,20 @@ const char *gdn_status_string(gdn_status s) {
 int gdn_last_cuda_error(void) { return t_last_cuda_error; }
 
 int gdn_api_version(void) { return GDN_API_VERSION; }
+
+void gdn_trace_begin(gdn_trace_entry *entries, int capacity) {
+    t_trace = entries;
+    t_trace_cap = entries ? (capacity > 0 ? capacity : 0) : 0;
+    t_trace_n = 0;
+    t_trace_on = true;
+}
+
+int gdn_trace_end(void) {
+    t_trace_on = false;
+    t_trace = nullptr;
+    t_trace_cap = 0;
+    return t_trace_n;
+}
 
 gdn_status gdn_prefill_workspace_size(const gdn_config *cfg, gdn_dtype dtype, int64_t total_tokens,
                                       int n_seqs, size_t *bytes) {

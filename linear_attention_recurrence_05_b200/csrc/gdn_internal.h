@@ -5,7 +5,17 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include "libgdn.h"
+
 namespace gdn {
+
+// Brackets one kernel launch with the active launch trace of this host thread (if any).
+struct TraceLaunch {
+    TraceLaunch(cudaStream_t s, const char *kernel);
+    ~TraceLaunch();
+    cudaStream_t stream;
+    gdn_trace_entry *entry;
+};
 
 // Workspace carve-up of one gdn_prefill call (byte offsets from the workspace base).
 struct PrefillLayout {

@@ -206,6 +206,7 @@ static cudaError_t launch_scan_simt_t(const ScanParams &p, cudaStream_t s) {
     cudaError_t e = cudaFuncSetAttribute(scan_simt_kernel<T, TO>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
+    TraceLaunch tl(s, "scan_simt");
     scan_simt_kernel<T, TO><<<grid, kThreads, smem, s>>>(p);
     return cudaGetLastError();
 }
