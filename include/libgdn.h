@@ -168,6 +168,41 @@ GDN_EXPORT gdn_status gdn_decode_step(const gdn_config *cfg, gdn_dtype dtype, gd
                            void *out, int batch, cudaStream_t stream);
 
 /*
+ * gdn_prefill_static_scratch -- gdn_prefill without a caller-supplied workspace.
+ *
+ * No counterpart on the pages: it exists for callers that cannot call cudaMalloc
+ * while they run the mixer (for example a plugin whose host framework forbids device
+ * allocation in its execute step, a runtime that hands out all device memory up front,
+ * or C code with no allocator at hand).  Inputs, outputs, layouts and results are
+ * exactly those of gdn_prefill; only the scratch differs.  It lives in a fixed array
+ * of GDN_STATIC_SCRATCH_BYTES in device memory owned by the library: one copy on each
+ * GPU where the library's module holding it is loaded (with CUDA's default lazy module
+ * loading, the GPUs on which this entry point is used), kept until the process exits.
+ *  - Limit: problems whose gdn_prefill_workspace_size() exceeds GDN_STATIC_SCRATCH_BYTES
+ *    are rejected with GDN_ERR_WORKSPACE before anything is enqueued (at 16 QK / 48 V
+ *    heads that is roughly 1,600 tokens per call).
+ *  - Allocation: none; it calls no cudaMalloc, cudaFree or allocating library routine.
+ *  - Set-up: the first call on each device (with that device current) looks up the
+ *    array's device address with cudaGetSymbolAddress; make that first call before any
+ *    stream capture on that device.
+ *  - Sharing: every call on a device uses the same array, which keeps whatever the last
+ *    call left in it (no byte of it needs to start at zero).  Calls whose work overlaps
+ *    on the GPU (different streams, or different host threads) race on the array: order
+ *    them on one stream or synchronise between them.
+ */
+#define GDN_STATIC_SCRATCH_BYTES (64u << 20)
+
+GDN_EXPORT gdn_status gdn_prefill_static_scratch(
+    const gdn_config *cfg, gdn_dtype dtype, gdn_dtype out_dtype,
+    const void *q, const void *k, const void *v,
+    const float *conv_w_q, const float *conv_w_k, const float *conv_w_v,
+    const void *alpha, const void *beta,
+    const int32_t *cu_seqlens, int n_seqs, int64_t total_tokens,
+    const float *initial_state, float *final_state,
+    const void *conv_state_in, void *conv_state_out,
+    void *out, cudaStream_t stream);
+
+/*
  * Launch trace (a profiling aid; no counterpart on the pages).  While a trace is
  * active on a host thread, every kernel that a libgdn call made on that thread
  * launches is bracketed on its launch stream: entries[i].start is recorded just

@@ -20,7 +20,9 @@ STATUS = {0: "GDN_OK", 1: "GDN_ERR_INVALID_ARG", 2: "GDN_ERR_UNSUPPORTED", 3: "G
 # every entry point the header declares (checked by the CPU test suite)
 EXPORTS = ("gdn_status_string", "gdn_last_cuda_error", "gdn_api_version",
            "gdn_prefill_workspace_size", "gdn_prefill", "gdn_decode_step", "gdn_trace_begin",
-           "gdn_trace_end")
+           "gdn_trace_end", "gdn_prefill_static_scratch")
+
+STATIC_SCRATCH_BYTES = 64 << 20  # GDN_STATIC_SCRATCH_BYTES
 
 
 class TraceEntryC(ctypes.Structure):
@@ -82,6 +84,11 @@ def lib():
             L.gdn_trace_begin.restype = None
             L.gdn_trace_end.argtypes = []
             L.gdn_trace_end.restype = ctypes.c_int
+            L.gdn_prefill_static_scratch.argtypes = [ctypes.POINTER(GdnConfigC), ctypes.c_int,
+                                                     ctypes.c_int, vp, vp, vp, fp, fp, fp, vp, vp,
+                                                     i32p, ctypes.c_int, ctypes.c_int64, fp, fp,
+                                                     vp, vp, vp, vp]
+            L.gdn_prefill_static_scratch.restype = ctypes.c_int
             _lib = L
         return _lib
 

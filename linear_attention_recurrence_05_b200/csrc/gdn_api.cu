@@ -17,6 +17,8 @@ static thread_local int t_trace_cap = 0;
 static thread_local int t_trace_n = 0;
 static thread_local bool t_trace_on = false;
 
+void record_cuda_error(cudaError_t e) { t_last_cuda_error = (int)e; }
+
 TraceLaunch::TraceLaunch(cudaStream_t s, const char *kernel) : stream(s), entry(nullptr) {
     if (!t_trace_on) return;
     if (t_trace_n < t_trace_cap && t_trace) {

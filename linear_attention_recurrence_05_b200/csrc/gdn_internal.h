@@ -62,6 +62,9 @@ struct DecodeParams {
     void *out;
 };
 
+// remembers `e` as this host thread's gdn_last_cuda_error()
+void record_cuda_error(cudaError_t e);
+
 // launchers: return the cudaError_t of the launch
 cudaError_t launch_seq_table(const int32_t *cu_in, int n_seqs, int64_t T, int32_t *cu,
                              int32_t *cfirst, cudaStream_t s);
