@@ -85,7 +85,9 @@ cudaError_t launch_seq_table(const int32_t *cu_in, int n_seqs, int64_t T, int32_
 // grid (max_chunks, 2*Hqk + Hv): CTA = one 64-row chunk of one head slot (q heads,
 // then k heads, then v heads).  Warp w walks rows 16w..16w+15 in order, keeping the
 // 3-row conv history of its lane's 4 channels in registers.
-template <class T>
+// kTf32: round the stored rows to TF32 (for the tensor-core prefill, whose operands
+// are read as TF32; rounding here gives round-to-nearest instead of truncation).
+template <class T, bool kTf32>
 __global__ void __launch_bounds__(128) conv_l2_kernel(ConvParams p) {
     const int n_chunks = p.cfirst[p.n_seqs];
     const int ci = blockIdx.x;
@@ -156,16 +158,30 @@ __global__ void __launch_bounds__(128) conv_l2_kernel(ConvParams p) {
 #pragma unroll
             for (int c = 0; c < 4; ++c) y[c] *= inv;
         }
+        if (kTf32) {
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                uint32_t r;
+                asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(y[c]));
+                y[c] = __uint_as_float(r);
+            }
+        }
         st4(dst + (int64_t)(seq0 + s) * row_stride + c4, y);
     }
 }
 
-cudaError_t launch_conv_l2(const ConvParams &p, bool bf16, int64_t max_chunks, cudaStream_t s) {
+cudaError_t launch_conv_l2(const ConvParams &p, bool bf16, bool tf32, int64_t max_chunks,
+                           cudaStream_t s) {
     if (max_chunks <= 0) return cudaSuccess;
     dim3 grid((unsigned)max_chunks, 2 * p.n_qk + p.n_v);
     TraceLaunch tl(s, "conv_l2");
-    if (bf16) conv_l2_kernel<gdn::bf16><<<grid, 128, 0, s>>>(p);
-    else conv_l2_kernel<float><<<grid, 128, 0, s>>>(p);
+    if (bf16) {
+        if (tf32) conv_l2_kernel<gdn::bf16, true><<<grid, 128, 0, s>>>(p);
+        else conv_l2_kernel<gdn::bf16, false><<<grid, 128, 0, s>>>(p);
+    } else {
+        if (tf32) conv_l2_kernel<float, true><<<grid, 128, 0, s>>>(p);
+        else conv_l2_kernel<float, false><<<grid, 128, 0, s>>>(p);
+    }
     return cudaGetLastError();
 }
 

@@ -182,7 +182,8 @@ gdn_status gdn_prefill(const gdn_config *cfg, gdn_dtype dtype, gdn_dtype out_dty
         cp.cu = cu; cp.cfirst = cfirst;
         cp.n_seqs = n_seqs; cp.n_qk = cfg->n_qk_heads; cp.n_v = cfg->n_v_heads;
         cp.q_scale = cfg->q_scale; cp.eps = cfg->l2_eps;
-        e = launch_conv_l2(cp, bf, L.max_chunks, stream);
+        // bf16 inputs run the tensor-core (TF32) prefill, fp32 inputs the fp32 CUDA-core one
+        e = launch_conv_l2(cp, bf, /*tf32=*/bf, L.max_chunks, stream);
         if (e != cudaSuccess) return cuda_fail(e);
     }
     if (conv_state_out) {
@@ -196,7 +197,8 @@ gdn_status gdn_prefill(const gdn_config *cfg, gdn_dtype dtype, gdn_dtype out_dty
     sp.alpha = alpha; sp.beta = beta; sp.cu = cu;
     sp.init = initial_state; sp.fin = final_state; sp.out = out;
     sp.n_seqs = n_seqs; sp.n_qk = cfg->n_qk_heads; sp.n_v = cfg->n_v_heads;
-    e = launch_scan_simt(sp, bf, out_dtype == GDN_BF16, stream);
+    e = bf ? launch_prefill_tc(sp, bf, out_dtype == GDN_BF16, stream)
+           : launch_scan_simt(sp, bf, out_dtype == GDN_BF16, stream);
     if (e != cudaSuccess) return cuda_fail(e);
     return GDN_OK;
 }

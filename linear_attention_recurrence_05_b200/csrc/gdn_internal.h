@@ -68,11 +68,13 @@ void record_cuda_error(cudaError_t e);
 // launchers: return the cudaError_t of the launch
 cudaError_t launch_seq_table(const int32_t *cu_in, int n_seqs, int64_t T, int32_t *cu,
                              int32_t *cfirst, cudaStream_t s);
-cudaError_t launch_conv_l2(const ConvParams &p, bool bf16, int64_t max_chunks, cudaStream_t s);
+cudaError_t launch_conv_l2(const ConvParams &p, bool bf16, bool tf32, int64_t max_chunks,
+                           cudaStream_t s);
 cudaError_t launch_conv_state_out(const void *q, const void *k, const void *v,
                                   const void *conv_in, void *conv_out, const int32_t *cu,
                                   int n_seqs, int n_qk, int n_v, bool bf16, cudaStream_t s);
 cudaError_t launch_scan_simt(const ScanParams &p, bool in_bf16, bool out_bf16, cudaStream_t s);
+cudaError_t launch_prefill_tc(const ScanParams &p, bool in_bf16, bool out_bf16, cudaStream_t s);
 cudaError_t launch_decode(const DecodeParams &p, bool in_bf16, bool out_bf16, cudaStream_t s);
 
 }  // namespace gdn

@@ -1,0 +1,214 @@
+// Thin wrappers over the sm_100a tensor-core (tcgen05) and mbarrier PTX used by the
+// chunked prefill.  Operands are fp32 values in shared memory read as TF32
+// (kind::tf32, 8 K-elements per instruction), accumulators are fp32 in tensor memory.
+//
+// Shared-memory operand layouts (fp32 elements):
+//  * K-major operands (rows = M or N index, columns = K index) use the no-swizzle
+//    "core matrix" layout: 8-row x 4-column core matrices of 128 contiguous bytes
+//    (row r of a core matrix at +16*r), consecutive along the columns, row groups of 8
+//    rows C*32 bytes apart.  K step s (8 columns) starts at +256*s; LBO = 128 B (next
+//    4 columns), SBO = C*32 B (next 8 rows).
+//  * MN-major operands (rows = K index, columns = M or N index) use the 128-byte
+//    swizzle with 32-byte granules, the only MN-major layout the tensor core takes for
+//    32-bit elements: columns in blocks of 32 (128 B per row, R*128 bytes per block),
+//    and inside each 4-row group the 32-byte granule g of row r sits at g ^ (r % 4).
+//    K step s (8 rows) starts at +1024*s; LBO = R*128 B (next 32 columns), SBO = 512 B
+//    (next 4 rows).
+// A matrix contracted over both of its indices (K of the chunk: over features in
+// K K^T and K S, over tokens in K^T u) is therefore kept in both layouts.
+#pragma once
+
+#include <stdint.h>
+
+namespace gdn {
+namespace tc {
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+    return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+// byte offset of element (r, c) of a [R x C] fp32 tile in the core-matrix (K-major) layout
+__host__ __device__ __forceinline__ uint32_t cm_off(int r, int c, int C) {
+    return (uint32_t)((((r >> 3) * (C >> 2) + (c >> 2)) << 7) + ((r & 7) << 4) + ((c & 3) << 2));
+}
+// byte offset of element (r, c) of a [R x C] fp32 tile in the 32-byte-granule swizzle (MN-major)
+__host__ __device__ __forceinline__ uint32_t mn_off(int r, int c, int R) {
+    return (uint32_t)((c >> 5) * R * 128 + r * 128 + ((((c & 31) >> 3) ^ (r & 3)) << 5) +
+                      ((c & 7) << 2));
+}
+
+// ------------------------------------------------------------------ descriptors
+__device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo,
+                                              uint32_t layout) {
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+    d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+    d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+    d |= (uint64_t)1 << 46;                  // descriptor version for sm_100
+    d |= (uint64_t)(layout & 7u) << 61;      // 0: no swizzle, 1: 128B with 32B granules
+    return d;
+}
+
+// K-major view of a core-matrix tile with C columns (= K extent), K step s
+__device__ __forceinline__ uint64_t desc_kmajor(uint32_t base, int C, int s) {
+    return smem_desc(base + (uint32_t)(s * 256), 128, (uint32_t)(C * 32), 0);
+}
+// MN-major view of a swizzled tile with R rows (= K extent), K step s (8 rows)
+__device__ __forceinline__ uint64_t desc_mnmajor(uint32_t base, int R, int s) {
+    return smem_desc(base + (uint32_t)(s * 1024), (uint32_t)(R * 128), 512, 1);
+}
+
+// instruction descriptor: kind::tf32, fp32 accumulator, M x N, operand majors
+__host__ __device__ constexpr uint32_t idesc_tf32(int M, int N, bool a_mn, bool b_mn) {
+    return (1u << 4)                       // D format: f32
+           | (2u << 7) | (2u << 10)        // A, B format: tf32
+           | ((a_mn ? 1u : 0u) << 15) | ((b_mn ? 1u : 0u) << 16)
+           | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+// ------------------------------------------------------------------ MMA
+__device__ __forceinline__ void mma_tf32(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
+                                         uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+        "l"(a), "l"(b), "r"(idesc), "r"(accumulate));
+}
+
+// D[M x N] (+)= A[M x K] B[K x N], K a multiple of 8, issued by one thread.
+// a_dim / b_dim: the tile's column count C for a K-major operand, its row count R for
+// an MN-major one.
+template <int M, int N, int K, bool A_MN, bool B_MN>
+__device__ __forceinline__ void gemm(uint32_t d_tmem, uint32_t a_base, int a_dim, uint32_t b_base,
+                                     int b_dim, bool accumulate) {
+    constexpr uint32_t id = idesc_tf32(M, N, A_MN, B_MN);
+#pragma unroll
+    for (int s = 0; s < K / 8; ++s) {
+        const uint64_t a = A_MN ? desc_mnmajor(a_base, a_dim, s) : desc_kmajor(a_base, a_dim, s);
+        const uint64_t b = B_MN ? desc_mnmajor(b_base, b_dim, s) : desc_kmajor(b_base, b_dim, s);
+        mma_tf32(d_tmem, a, b, id, (accumulate || s > 0) ? 1u : 0u);
+    }
+}
+
+__device__ __forceinline__ void mma_commit(uint64_t *mbar) {
+    asm volatile(
+        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+            smem_u32(mbar))
+        : "memory");
+}
+
+// ------------------------------------------------------------------ fences
+__device__ __forceinline__ void fence_before_sync() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void fence_after_sync() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+// make this thread's generic-proxy shared-memory writes visible to the tensor core
+__device__ __forceinline__ void fence_smem_to_async() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// ------------------------------------------------------------------ mbarrier
+__device__ __forceinline__ void mbar_init(uint64_t *m, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(m)), "r"(count));
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *m, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(ok)
+        : "r"(smem_u32(m)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+// Bounded wait on phase `parity`: returns false if it has not completed after
+// `max_tries` polls (each poll itself blocks for a hardware-defined short time).
+__device__ __forceinline__ bool mbar_wait(uint64_t *m, uint32_t parity, uint32_t max_tries) {
+    for (uint32_t i = 0; i < max_tries; ++i)
+        if (mbar_try_wait(m, parity)) return true;
+    return false;
+}
+
+// ------------------------------------------------------------------ tensor memory
+__device__ __forceinline__ void tmem_alloc(uint32_t *dst_smem, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(dst_smem)),
+                 "r"(ncols)
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+                 : "memory");
+}
+
+// 32 consecutive columns of this thread's lane (32x32b shape): lane = warp quarter base + laneid
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+    uint32_t r[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+          "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+          "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+          "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+__device__ __forceinline__ void tmem_wait_ld() {
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+        "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
+        "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
+        "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])), "r"(__float_as_uint(v[8])),
+        "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
+        "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
+        "r"(__float_as_uint(v[15])), "r"(__float_as_uint(v[16])), "r"(__float_as_uint(v[17])),
+        "r"(__float_as_uint(v[18])), "r"(__float_as_uint(v[19])), "r"(__float_as_uint(v[20])),
+        "r"(__float_as_uint(v[21])), "r"(__float_as_uint(v[22])), "r"(__float_as_uint(v[23])),
+        "r"(__float_as_uint(v[24])), "r"(__float_as_uint(v[25])), "r"(__float_as_uint(v[26])),
+        "r"(__float_as_uint(v[27])), "r"(__float_as_uint(v[28])), "r"(__float_as_uint(v[29])),
+        "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
+        : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() {
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+// TMEM address of (lane, column)
+__device__ __forceinline__ uint32_t taddr(uint32_t base, int lane, int col) {
+    return base + ((uint32_t)lane << 16) + (uint32_t)col;
+}
+
+// ------------------------------------------------------------------ tf32 rounding
+__device__ __forceinline__ float to_tf32(float x) {
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+    return __uint_as_float(r);
+}
+
+// ------------------------------------------------------------------ cp.async (16 B)
+__device__ __forceinline__ void cp_async16(uint32_t dst_smem, const void *src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst_smem), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+}  // namespace tc
+}  // namespace gdn
