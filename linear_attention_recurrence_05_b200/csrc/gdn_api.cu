@@ -197,7 +197,7 @@ gdn_status gdn_prefill(const gdn_config *cfg, gdn_dtype dtype, gdn_dtype out_dty
     sp.alpha = alpha; sp.beta = beta; sp.cu = cu;
     sp.init = initial_state; sp.fin = final_state; sp.out = out;
     sp.n_seqs = n_seqs; sp.n_qk = cfg->n_qk_heads; sp.n_v = cfg->n_v_heads;
-    e = bf ? launch_prefill_tc(sp, bf, out_dtype == GDN_BF16, stream)
+    e = bf ? launch_prefill_tc(sp, total_tokens, bf, out_dtype == GDN_BF16, stream)
            : launch_scan_simt(sp, bf, out_dtype == GDN_BF16, stream);
     if (e != cudaSuccess) return cuda_fail(e);
     return GDN_OK;

@@ -74,7 +74,8 @@ cudaError_t launch_conv_state_out(const void *q, const void *k, const void *v,
                                   const void *conv_in, void *conv_out, const int32_t *cu,
                                   int n_seqs, int n_qk, int n_v, bool bf16, cudaStream_t s);
 cudaError_t launch_scan_simt(const ScanParams &p, bool in_bf16, bool out_bf16, cudaStream_t s);
-cudaError_t launch_prefill_tc(const ScanParams &p, bool in_bf16, bool out_bf16, cudaStream_t s);
+cudaError_t launch_prefill_tc(const ScanParams &p, int64_t total_tokens, bool in_bf16, bool out_bf16,
+                              cudaStream_t s);
 cudaError_t launch_decode(const DecodeParams &p, bool in_bf16, bool out_bf16, cudaStream_t s);
 
 }  // namespace gdn

@@ -7,19 +7,24 @@
 //     u    = T diag(beta) (V - diag(gamma) K S)                      (the WY/UT solve)
 //     y_t  = gamma_t S^T q_t + sum_{i<=t} exp(g_t - g_i)(q_t.k_i) u_i
 //     S   <- gamma_C S + sum_i exp(g_C - g_i) k_i u_i^T
-// (u = U - W S with U = T diag(beta) V and W = T diag(beta gamma) K, regrouped so
-// that W never has to be formed).
+// (u = U - W S with U = T diag(beta) V and W = T diag(beta gamma) K, regrouped so that
+// W never has to be formed).
 //
-// One CTA owns one (sequence, V head, 64-column half of d_v) and walks the sequence's
-// chunks in order; the column split is exact.  Per chunk, on the tensor core:
-//     MMA_a  [K;Q] K^T        128 x 64 x 128   -> A (strict lower) and P (lower)
-//     MMA_1  K S, Q S          64 x 64 x 128   -> V' = V - gamma*KS ; gamma*QS kept in TMEM
-//     MMA_2  T_beta V'         64 x 64 x 64    -> u, u~ = exp(g_C - g) u
-//     MMA_3  K^T u~           128 x 64 x 64    -> S update (state stays fp32 in registers)
-//     MMA_4  P u (accumulate)  64 x 64 x 64    -> y = gamma*QS + P u
-// and on the CUDA cores the 64 x 64 unit-lower-triangular inverse (16 x 16 blocks).
-// The next chunk's K/Q, V and K (token-major copy) are fetched with cp.async into
-// each buffer as soon as its last reader has finished.
+// One CTA (16 warps) owns one (sequence, V head, 64-column half of d_v) and walks the
+// sequence's chunks in order; the column split is exact.  Per chunk, on the tensor core:
+//     MMA_a  [K;Q] K^T      M=128 N=64 K=128 -> A (strict lower) and P (lower)
+//     MMA_1  [K;Q] S        M=128 N=64 K=128 -> V' = V - gamma*KS ; gamma*QS kept in TMEM
+//     MMA_2  T_beta V'      M=64  N=64 K=64  -> u, u~ = exp(g_C - g) u
+//     MMA_3  K^T u~         M=128 N=64 K=64  -> S update (the state stays fp32 in registers)
+//     MMA_4  [*;P] u        M=128 N=64 K=64  -> accumulated onto gamma*QS: y
+// MMA_4 reads P through a 128-row view whose upper 64 rows are whatever precedes P in
+// shared memory; they land on rows 0-63 of the accumulator, which hold K S and are
+// already consumed.  On the CUDA cores: the 64 x 64 unit-lower-triangular inverse
+// (16 x 16 blocks) and the element-wise epilogues.  Operand tiles arrive by TMA
+// (2-D boxes of 32 fp32 x 64 tokens), each reloaded as soon as its last reader is done.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include "gdn_common.cuh"
 #include "gdn_internal.h"
 #include "tc_sm100.cuh"
@@ -31,50 +36,77 @@ using namespace tc;
 
 constexpr int kN = 64;          // d_v columns per CTA
 constexpr int kNS = kHeadDim / kN;
-constexpr int kThr = 256;
+constexpr int kThr = 512;
 
 // shared-memory map (bytes from a 1024-aligned base)
-constexpr uint32_t OFF_S = 0;          // S        MN-major  [128 d][64 j]            32 KB
-constexpr uint32_t OFF_KQ = 32768;     // [K;Q]    K-major   [128 rows][128 d]        64 KB
-constexpr uint32_t OFF_KMN = 98304;    // K        MN-major  [64 i][128 d]            32 KB
-constexpr uint32_t OFF_V = 131072;     // V plain [64][64] fp32, then V' MN-major      16 KB
-constexpr uint32_t OFF_TB = 147456;    // T plain, then T_beta K-major, then u~ MN-major 16 KB
-constexpr uint32_t OFF_P = 163840;     // P        K-major   [64 t][64 i]             16 KB
-constexpr uint32_t OFF_U = 180224;     // A plain [64][64] fp32, then u MN-major      16 KB
-constexpr uint32_t OFF_MISC = 196608;  // gates, inverse scratch, barriers
+constexpr uint32_t OFF_S = 0;          // S       MN-major R=128 (d) x 64 (j)               32 KB
+constexpr uint32_t OFF_KQ = 32768;     // [K;Q]   K-major, 4 blocks x (K 8 KB | Q 8 KB)      64 KB
+constexpr uint32_t OFF_KMN = 98304;    // K       MN-major R=64 (i) x 128 (d)               32 KB
+constexpr uint32_t OFF_V = 131072;     // V (K-major swizzle, read by threads), then V' MN  16 KB
+constexpr uint32_t OFF_TB = 147456;    // T (fp32 scratch), then T_beta K-major, then u~ MN 16 KB
+constexpr uint32_t OFF_P = 163840;     // P       K-major R=64                               16 KB
+constexpr uint32_t OFF_U = 180224;     // A (fp32 scratch), then u MN-major                16 KB
+constexpr uint32_t OFF_MISC = 196608;
 constexpr uint32_t OFF_G = OFF_MISC;            // g[64]
 constexpr uint32_t OFF_GAM = OFF_MISC + 256;    // gamma[64]
 constexpr uint32_t OFF_BETA = OFF_MISC + 512;   // beta[64]
 constexpr uint32_t OFF_KD = OFF_MISC + 768;     // exp(g_last - g)[64]
 constexpr uint32_t OFF_INV = OFF_MISC + 1024;   // 3 x 256 floats (block products)
-constexpr uint32_t OFF_BAR = OFF_MISC + 4096;   // 5 mbarriers
-constexpr uint32_t OFF_TSLOT = OFF_BAR + 64;  // after 5 x 8 bytes
-constexpr uint32_t kSmem = OFF_MISC + 4096 + 128;
+constexpr uint32_t OFF_BAR = OFF_MISC + 4096;   // mbarriers
+constexpr uint32_t OFF_TSLOT = OFF_BAR + 128;
+constexpr uint32_t kSmem = OFF_TSLOT + 16;
 constexpr uint32_t kSmemAlloc = kSmem + 1024;   // slack to align the base to 1024
 
+enum { B_KQ = 0, B_V, B_KMN, B_A, B_1, B_2, B_3, kNumBars };
+
 // tensor-memory columns
-constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t T_A = 0;      // [K;Q]K^T  M=128
-constexpr uint32_t T_KS = 64;    // K S       M=64
-constexpr uint32_t T_QS = 128;   // Q S, then y  M=64
-constexpr uint32_t T_U = 192;    // u         M=64
-constexpr uint32_t T_DS = 256;   // K^T u~    M=128
+constexpr uint32_t kTmemCols = 256;
+constexpr uint32_t T_A = 0;      // [K;Q]K^T    M=128
+constexpr uint32_t T_1 = 64;     // [K;Q]S, then rows 64.. = y   M=128
+constexpr uint32_t T_U = 128;    // u           M=64
+constexpr uint32_t T_DS = 192;   // K^T u~      M=128
 
 constexpr uint32_t kWaitTries = 1u << 22;
 
-__device__ __forceinline__ void cp_async16_zfill(uint32_t dst, const void *src, bool valid) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
-                 "r"(valid ? 16 : 0)
-                 : "memory");
+// fp32 scratch [64][64] with 16-byte chunks XOR-swizzled by row (conflict-free rows and columns)
+__device__ __forceinline__ int scr(int r, int c) { return r * 64 + ((((c >> 2) ^ (r & 7)) << 2) | (c & 3)); }
+
+__device__ __forceinline__ float4 tf32x4(float a, float b, float c, float d) {
+    return make_float4(to_tf32(a), to_tf32(b), to_tf32(c), to_tf32(d));
 }
 
 template <class TO>
-__device__ __forceinline__ void store_out(TO *p, float v) { *p = from_f32<TO>(v); }
+__device__ __forceinline__ void store_row16(TO *dst, const float (&v)[16]);
+template <>
+__device__ __forceinline__ void store_row16<float>(float *dst, const float (&v)[16]) {
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+        *reinterpret_cast<float4 *>(dst + 4 * k) = make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
+}
+template <>
+__device__ __forceinline__ void store_row16<bf16>(bf16 *dst, const float (&v)[16]) {
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+        uint4 w;
+        __nv_bfloat162 h0 = __floats2bfloat162_rn(v[8 * k], v[8 * k + 1]);
+        __nv_bfloat162 h1 = __floats2bfloat162_rn(v[8 * k + 2], v[8 * k + 3]);
+        __nv_bfloat162 h2 = __floats2bfloat162_rn(v[8 * k + 4], v[8 * k + 5]);
+        __nv_bfloat162 h3 = __floats2bfloat162_rn(v[8 * k + 6], v[8 * k + 7]);
+        w.x = *reinterpret_cast<uint32_t *>(&h0);
+        w.y = *reinterpret_cast<uint32_t *>(&h1);
+        w.z = *reinterpret_cast<uint32_t *>(&h2);
+        w.w = *reinterpret_cast<uint32_t *>(&h3);
+        *reinterpret_cast<uint4 *>(dst + 8 * k) = w;
+    }
+}
 
 }  // namespace
 
 struct TcParams {
-    const float *qh, *kh, *vh;
+    CUtensorMap tm_k;     // k^ rows, K-major 128B swizzle boxes (32 x 64)
+    CUtensorMap tm_q;     // q^ rows, same
+    CUtensorMap tm_kmn;   // k^ rows, MN-major 32B-granule swizzle boxes
+    CUtensorMap tm_v;     // v^ rows, K-major 128B swizzle boxes
     const void *alpha, *beta;
     const int32_t *cu;
     const float *init;
@@ -84,7 +116,7 @@ struct TcParams {
 };
 
 template <class TI, class TO>
-__global__ void __launch_bounds__(kThr, 1) prefill_tc_kernel(TcParams p) {
+__global__ void __launch_bounds__(kThr, 1) prefill_tc_kernel(const __grid_constant__ TcParams p) {
     extern __shared__ unsigned char smem_raw[];
     unsigned char *sm = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
     const uint32_t sb = smem_u32(sm);
@@ -93,19 +125,21 @@ __global__ void __launch_bounds__(kThr, 1) prefill_tc_kernel(TcParams p) {
     float *beta_s = (float *)(sm + OFF_BETA);
     float *kd_s = (float *)(sm + OFF_KD);
     float *inv_s = (float *)(sm + OFF_INV);
-    // one phase per chunk each: 0 MMA_a, 1 K S, 2 Q S, 3 MMA_2, 4 MMA_3 + MMA_4
     uint64_t *bar = (uint64_t *)(sm + OFF_BAR);
     uint32_t *tslot = (uint32_t *)(sm + OFF_TSLOT);
+    float *Ascr = (float *)(sm + OFF_U);   // A scratch (fp32, swizzled rows)
+    float *Tscr = (float *)(sm + OFF_TB);  // T scratch (fp32, swizzled rows)
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int quarter = warp & 3, half = warp >> 2;   // TMEM lane quarter, 32-column half
+    const int quarter = warp & 3, cg = warp >> 2;   // TMEM lane quarter, 16-column group
+    const int col = 16 * cg;                        // first accumulator column of this thread
     const int slice = blockIdx.x % kNS;
     const int h = (blockIdx.x / kNS) % p.n_v;
     const int b = blockIdx.x / (kNS * p.n_v);
     const int gq = h / (p.n_v / p.n_qk);
     const int seq0 = p.cu[b], L = p.cu[b + 1] - p.cu[b];
     const int col0 = slice * kN;
-    const int64_t qk_row = (int64_t)p.n_qk * kHeadDim, v_row = (int64_t)p.n_v * kHeadDim;
+    const int64_t v_row = (int64_t)p.n_v * kHeadDim;
     const TI *al = (const TI *)p.alpha;
     const TI *be = (const TI *)p.beta;
     TO *out = (TO *)p.out;
@@ -113,53 +147,50 @@ __global__ void __launch_bounds__(kThr, 1) prefill_tc_kernel(TcParams p) {
 
     // ---------------------------------------------------------------- set-up
     if (tid == 0) {
-        for (int i = 0; i < 5; ++i) mbar_init(&bar[i], 1);
+        for (int i = 0; i < kNumBars; ++i) mbar_init(&bar[i], 1);
     }
     if (warp == 0) {
         tmem_alloc(tslot, kTmemCols);
         tmem_relinquish();
     }
-    // state: this thread owns S[d][32*half .. 32*half+31] with d = 32*quarter + lane
+    // this thread owns S[d_own][col .. col+15]
     const int d_own = 32 * quarter + lane;
-    float S[32];
-    {
-        const int64_t st_off = (((int64_t)b * p.n_v + h) * kHeadDim + d_own) * kHeadDim + col0 + 32 * half;
+    const int64_t st_off = (((int64_t)b * p.n_v + h) * kHeadDim + d_own) * kHeadDim + col0 + col;
+    float S[16];
 #pragma unroll
-        for (int j = 0; j < 32; ++j) S[j] = p.init ? p.init[st_off + j] : 0.f;
-#pragma unroll
-        for (int j = 0; j < 32; ++j)
-            *(float *)(sm + OFF_S + mn_off(d_own, 32 * half + j, kHeadDim)) = to_tf32(S[j]);
+    for (int k = 0; k < 4; ++k) {
+        float4 v4 = p.init ? *reinterpret_cast<const float4 *>(p.init + st_off + 4 * k)
+                           : make_float4(0.f, 0.f, 0.f, 0.f);
+        S[4 * k] = v4.x; S[4 * k + 1] = v4.y; S[4 * k + 2] = v4.z; S[4 * k + 3] = v4.w;
     }
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+        *reinterpret_cast<float4 *>(sm + OFF_S + mn_off(d_own, col + 4 * k, kHeadDim)) =
+            tf32x4(S[4 * k], S[4 * k + 1], S[4 * k + 2], S[4 * k + 3]);
 
-    // chunk loaders ----------------------------------------------------------
-    auto load_kq = [&](int c) {  // [K;Q] rows, K-major core-matrix layout (group 1)
-        const int n = min(kChunk, L - c * kChunk);
-        const int64_t tok = seq0 + (int64_t)c * kChunk;
-        for (int e = tid; e < 128 * 32; e += kThr) {
-            const int r = e >> 5, q4 = (e & 31) * 4;
-            const int t = r & 63;
-            const float *src = (r < 64 ? p.kh : p.qh) + (tok + (t < n ? t : 0)) * qk_row +
-                               gq * kHeadDim + q4;
-            cp_async16_zfill(sb + OFF_KQ + cm_off(r, q4, 128), src, t < n);
+    // TMA issue (thread 0 only)
+    auto issue_kq = [&](int c) {
+        const int tok = seq0 + c * kChunk;
+        mbar_expect_tx(&bar[B_KQ], 65536);
+#pragma unroll
+        for (int kb = 0; kb < 4; ++kb) {
+            tma_load_2d(sb + OFF_KQ + kb * 16384, &p.tm_k, gq * kHeadDim + 32 * kb, tok, &bar[B_KQ]);
+            tma_load_2d(sb + OFF_KQ + kb * 16384 + 8192, &p.tm_q, gq * kHeadDim + 32 * kb, tok, &bar[B_KQ]);
         }
     };
-    auto load_v = [&](int c) {  // V rows, plain [64][64] (group 2)
-        const int n = min(kChunk, L - c * kChunk);
-        const int64_t tok = seq0 + (int64_t)c * kChunk;
-        for (int e = tid; e < 64 * 16; e += kThr) {
-            const int t = e >> 4, q4 = (e & 15) * 4;
-            const float *src = p.vh + (tok + (t < n ? t : 0)) * v_row + h * kHeadDim + col0 + q4;
-            cp_async16_zfill(sb + OFF_V + (t * 64 + q4) * 4, src, t < n);
-        }
+    auto issue_v = [&](int c) {
+        const int tok = seq0 + c * kChunk;
+        mbar_expect_tx(&bar[B_V], 16384);
+#pragma unroll
+        for (int jb = 0; jb < 2; ++jb)
+            tma_load_2d(sb + OFF_V + jb * 8192, &p.tm_v, h * kHeadDim + col0 + 32 * jb, tok, &bar[B_V]);
     };
-    auto load_kmn = [&](int c) {  // K rows, MN-major swizzled layout (group 3)
-        const int n = min(kChunk, L - c * kChunk);
-        const int64_t tok = seq0 + (int64_t)c * kChunk;
-        for (int e = tid; e < 64 * 32; e += kThr) {
-            const int t = e >> 5, q4 = (e & 31) * 4;
-            const float *src = p.kh + (tok + (t < n ? t : 0)) * qk_row + gq * kHeadDim + q4;
-            cp_async16_zfill(sb + OFF_KMN + mn_off(t, q4, 64), src, t < n);
-        }
+    auto issue_kmn = [&](int c) {
+        const int tok = seq0 + c * kChunk;
+        mbar_expect_tx(&bar[B_KMN], 32768);
+#pragma unroll
+        for (int db = 0; db < 4; ++db)
+            tma_load_2d(sb + OFF_KMN + db * 8192, &p.tm_kmn, gq * kHeadDim + 32 * db, tok, &bar[B_KMN]);
     };
     // gate prefetch: thread t < 64 holds alpha/beta of row t of the next chunk
     float a_next = 1.f, b_next = 0.f;
@@ -172,300 +203,325 @@ __global__ void __launch_bounds__(kThr, 1) prefill_tc_kernel(TcParams p) {
         }
     };
 
-    if (nchunks > 0) {
-        load_kq(0);
-        cp_async_commit();
-        load_v(0);
-        cp_async_commit();
-        load_kmn(0);
-        cp_async_commit();
-        load_gates(0);
-    }
     fence_before_sync();
     __syncthreads();
     fence_after_sync();
     const uint32_t tm = *tslot;
+    if (nchunks > 0) {
+        if (tid == 0) {
+            issue_kq(0);
+            issue_v(0);
+            issue_kmn(0);
+        }
+        load_gates(0);
+    }
     bool failed = false;
-
-    // waits for barrier `i` phase `par` on every thread; all threads agree on failure
+    // every thread waits; all agree on success
     auto wait_bar = [&](int i, uint32_t par) -> bool {
         bool ok = mbar_wait(&bar[i], par, kWaitTries);
         return __syncthreads_or(!ok) == 0;
     };
 
-    for (int c = 0; c < nchunks && !failed; ++c) {
+    for (int c = 0; c < nchunks; ++c) {
         const int n = min(kChunk, L - c * kChunk);
         const int64_t tok = seq0 + (int64_t)c * kChunk;
         const uint32_t par = c & 1;
 
-        // ---- gates of this chunk, K/Q tile
+        // ---- gates, and this chunk's [K;Q]
         if (tid < kChunk) {
             g_s[tid] = safe_log_alpha(a_next);
             beta_s[tid] = b_next;
         }
-        cp_async_wait<2>();  // group 1 of this chunk ([K;Q]) has landed
-        fence_smem_to_async();
-        __syncthreads();
+        fence_smem_to_async();  // S tile written by the previous chunk (or the set-up)
+        if (!wait_bar(B_KQ, par)) { failed = true; break; }
         if (warp == 0) {  // inclusive scan of log alpha, two rows per lane
-            float a0 = g_s[2 * lane], a1 = g_s[2 * lane + 1];
+            const float a0 = g_s[2 * lane], a1 = g_s[2 * lane + 1];
             float s = a0 + a1;
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
-                float y = __shfl_up_sync(0xffffffffu, s, o);
+                const float y = __shfl_up_sync(0xffffffffu, s, o);
                 if (lane >= o) s += y;
             }
-            const float base = s - (a0 + a1);
-            g_s[2 * lane] = base + a0;
+            const float g0 = s - a1;
+            const float glast = __shfl_sync(0xffffffffu, ((n - 1) & 1) ? s : g0, (n - 1) >> 1);
+            g_s[2 * lane] = g0;
             g_s[2 * lane + 1] = s;
-            __syncwarp();
-            const float glast = __shfl_sync(0xffffffffu, (n - 1) & 1 ? s : base + a0, (n - 1) >> 1);
-#pragma unroll
-            for (int k = 0; k < 2; ++k) {
-                const int t = 2 * lane + k;
-                const float gt = k ? s : base + a0;
-                gam_s[t] = expf(gt);
-                kd_s[t] = t < n ? expf(glast - gt) : 0.f;
-            }
+            gam_s[2 * lane] = expf(g0);
+            gam_s[2 * lane + 1] = expf(s);
+            kd_s[2 * lane] = 2 * lane < n ? expf(glast - g0) : 0.f;
+            kd_s[2 * lane + 1] = 2 * lane + 1 < n ? expf(glast - s) : 0.f;
         }
         __syncthreads();
 
-        // ---- MMA_a: [K;Q] K^T ; MMA_1: K S, Q S
+        // ---- MMA_a: [K;Q] K^T ; MMA_1: [K;Q] S
         if (tid == 0) {
             fence_after_sync();
-            gemm<128, 64, 128, false, false>(tm + T_A, sb + OFF_KQ, 128, sb + OFF_KQ, 128, false);
-            mma_commit(&bar[0]);
-            gemm<64, 64, 128, false, true>(tm + T_KS, sb + OFF_KQ, 128, sb + OFF_S, kHeadDim, false);
-            mma_commit(&bar[1]);
-            gemm<64, 64, 128, false, true>(tm + T_QS, sb + OFF_KQ + 64 * 128 * 4, 128, sb + OFF_S,
-                                           kHeadDim, false);
-            mma_commit(&bar[2]);
+            gemm<128, 64, 128, false, false>(tm + T_A, sb + OFF_KQ, 16384, sb + OFF_KQ, 16384, false);
+            mma_commit(&bar[B_A]);
+            gemm<128, 64, 128, false, true>(tm + T_1, sb + OFF_KQ, 16384, sb + OFF_S, kHeadDim, false);
+            mma_commit(&bar[B_1]);
         }
 
-        // ---- epilogue a: A (fp32 scratch in OFF_U) and P (K-major tile)
-        if (!wait_bar(0, par)) { failed = true; break; }
+        // ---- epilogue a: A (fp32 scratch) and P (K-major tile)
+        if (!wait_bar(B_A, par)) { failed = true; break; }
         fence_after_sync();
         {
-            float v[32];
-            tmem_ld32(taddr(tm + T_A, 32 * quarter, 32 * half), v);
+            float v[16];
+            tmem_ld16(taddr(tm + T_A, 32 * quarter, col), v);
             tmem_wait_ld();
-            const int row = 32 * quarter + lane;
-            if (row < 64) {  // K K^T rows -> A
-                const int t = row;
-                float *A = (float *)(sm + OFF_U);
+            if (quarter < 2) {  // K K^T rows -> A = strict lower beta_t exp(g_t - g_i) k_t.k_i
+                const int t = 32 * quarter + lane;
                 const float gt = g_s[t], bt = beta_s[t];
 #pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    const int i = 32 * half + j;
-                    A[t * 64 + i] = (i < t && t < n) ? bt * expf(gt - g_s[i]) * v[j] : 0.f;
+                for (int k = 0; k < 4; ++k) {
+                    float a4[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int i = col + 4 * k + e;
+                        a4[e] = (i < t && t < n) ? bt * expf(gt - g_s[i]) * v[4 * k + e] : 0.f;
+                    }
+                    *reinterpret_cast<float4 *>(&Ascr[scr(t, col + 4 * k)]) = make_float4(a4[0], a4[1], a4[2], a4[3]);
                 }
-            } else {  // Q K^T rows -> P
-                const int t = row - 64;
+            } else {  // Q K^T rows -> P = lower exp(g_t - g_i) q_t.k_i
+                const int t = 32 * quarter + lane - 64;
                 const float gt = g_s[t];
 #pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    const int i = 32 * half + j;
-                    const float pv = (i <= t && t < n) ? expf(gt - g_s[i]) * v[j] : 0.f;
-                    *(float *)(sm + OFF_P + cm_off(t, i, 64)) = to_tf32(pv);
-                }
-            }
-        }
-        // ---- epilogue 1: V' = V - gamma * K S  (M=64 layout: row t at lane 16*quarter + l)
-        cp_async_wait<1>();  // group 2 (V) of this chunk; made visible by the barrier below
-        if (!wait_bar(1, par)) { failed = true; break; }
-        fence_after_sync();
-        {
-            float v[32];
-            tmem_ld32(taddr(tm + T_KS, 32 * quarter, 32 * half), v);
-            tmem_wait_ld();
-            const int t = 16 * quarter + lane;
-            float vp[32];
-            if (lane < 16) {
-                const float gt = gam_s[t];
-                const float *V = (const float *)(sm + OFF_V);
+                for (int k = 0; k < 4; ++k) {
+                    float p4[4];
 #pragma unroll
-                for (int j = 0; j < 32; ++j) vp[j] = V[t * 64 + 32 * half + j] - gt * v[j];
-            }
-            __syncthreads();  // every V value has been read before V' overwrites it
-            if (lane < 16) {
-#pragma unroll
-                for (int j = 0; j < 32; ++j)
-                    *(float *)(sm + OFF_V + mn_off(t, 32 * half + j, 64)) = to_tf32(vp[j]);
-            }
-        }
-        __syncthreads();  // A complete
-
-        // ---- T = (I + A)^-1 by 16 x 16 blocks (plain fp32 in OFF_TB)
-        {
-            const float *A = (const float *)(sm + OFF_U);
-            float *T = (float *)(sm + OFF_TB);
-            if (tid < 64) {  // diagonal blocks: column c of block bb by forward substitution
-                const int bb = tid >> 4, cc = tid & 15;
-                float x[16];
-#pragma unroll
-                for (int r = 0; r < 16; ++r) {
-                    float acc = (r == cc) ? 1.f : 0.f;
-#pragma unroll
-                    for (int m = 0; m < r; ++m)
-                        acc = fmaf(-A[(16 * bb + r) * 64 + 16 * bb + m], x[m], acc);
-                    x[r] = (r < cc) ? 0.f : acc;
-                }
-#pragma unroll
-                for (int r = 0; r < 16; ++r) T[(16 * bb + r) * 64 + 16 * bb + cc] = x[r];
-            } else {  // zero the strictly upper blocks
-                for (int e = tid - 64; e < 64 * 64; e += kThr - 64) {
-                    const int r = e >> 6, cidx = e & 63;
-                    if ((r >> 4) < (cidx >> 4)) T[e] = 0.f;
-                }
-            }
-            __syncthreads();
-            // off-diagonal blocks by distance: T_rc = -T_rr * sum_{k=c}^{r-1} A_rk T_kc
-            for (int dist = 1; dist < 4; ++dist) {
-                const int nb = 4 - dist;  // blocks at this distance: c = 0..nb-1, r = c + dist
-                for (int e = tid; e < nb * 256; e += kThr) {
-                    const int c = e >> 8, rr = (e >> 4) & 15, cc = e & 15;
-                    const int r = c + dist;
-                    float acc = 0.f;
-                    for (int k = c; k < r; ++k) {
-#pragma unroll
-                        for (int m = 0; m < 16; ++m)
-                            acc = fmaf(A[(16 * r + rr) * 64 + 16 * k + m], T[(16 * k + m) * 64 + 16 * c + cc], acc);
+                    for (int e = 0; e < 4; ++e) {
+                        const int i = col + 4 * k + e;
+                        p4[e] = (i <= t && t < n) ? expf(gt - g_s[i]) * v[4 * k + e] : 0.f;
                     }
-                    inv_s[e] = acc;
+                    *reinterpret_cast<float4 *>(sm + OFF_P + kmaj_off(t, col + 4 * k, 64)) =
+                        tf32x4(p4[0], p4[1], p4[2], p4[3]);
                 }
-                __syncthreads();
-                for (int e = tid; e < nb * 256; e += kThr) {
-                    const int c = e >> 8, rr = (e >> 4) & 15, cc = e & 15;
-                    const int r = c + dist;
-                    float acc = 0.f;
-#pragma unroll
-                    for (int m = 0; m < 16; ++m)
-                        acc = fmaf(T[(16 * r + rr) * 64 + 16 * r + m], inv_s[(c << 8) + m * 16 + cc], acc);
-                    T[(16 * r + rr) * 64 + 16 * c + cc] = -acc;
-                }
-                __syncthreads();
             }
-            // T_beta = T diag(beta), rewritten in place as a K-major tile
-            float tv[16];
+        }
+        // ---- epilogue 1: V' = V - gamma * K S (rows 0-63); gamma * Q S in place (rows 64-127)
+        if (!wait_bar(B_1, par)) { failed = true; break; }
+        if (!wait_bar(B_V, par)) { failed = true; break; }
+        fence_after_sync();
+        {
+            float v[16];
+            tmem_ld16(taddr(tm + T_1, 32 * quarter, col), v);
+            tmem_wait_ld();
+            if (quarter < 2) {
+                const int t = 32 * quarter + lane;
+                const float gt = gam_s[t];
 #pragma unroll
-            for (int k = 0; k < 16; ++k) {
-                const int e = tid + kThr * k;
-                tv[k] = T[e] * beta_s[e & 63];
+                for (int k = 0; k < 4; ++k) {
+                    const float4 x = *reinterpret_cast<const float4 *>(sm + OFF_V + kmaj_off(t, col + 4 * k, 64));
+                    v[4 * k] = x.x - gt * v[4 * k];
+                    v[4 * k + 1] = x.y - gt * v[4 * k + 1];
+                    v[4 * k + 2] = x.z - gt * v[4 * k + 2];
+                    v[4 * k + 3] = x.w - gt * v[4 * k + 3];
+                }
+            } else {
+                const float gt = gam_s[32 * quarter + lane - 64];
+#pragma unroll
+                for (int j = 0; j < 16; ++j) v[j] *= gt;
+                tmem_st16(taddr(tm + T_1, 32 * quarter, col), v);
+                tmem_wait_st();
+            }
+            __syncthreads();  // all of V has been read before V' overwrites it
+            if (quarter < 2) {
+                const int t = 32 * quarter + lane;
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    *reinterpret_cast<float4 *>(sm + OFF_V + mn_off(t, col + 4 * k, 64)) =
+                        tf32x4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
+            }
+        }
+
+        // ---- T = (I + A)^-1 by 16 x 16 blocks (fp32 scratch in OFF_TB)
+        if (tid < 64) {  // diagonal blocks: column cc of block bb by forward substitution
+            const int bb = tid >> 4, cc = tid & 15;
+            float x[16];
+#pragma unroll
+            for (int r = 0; r < 16; ++r) {
+                float acc = (r == cc) ? 1.f : 0.f;
+#pragma unroll
+                for (int m = 0; m < r; ++m) acc = fmaf(-Ascr[scr(16 * bb + r, 16 * bb + m)], x[m], acc);
+                x[r] = (r < cc) ? 0.f : acc;
+            }
+#pragma unroll
+            for (int r = 0; r < 16; ++r) Tscr[scr(16 * bb + r, 16 * bb + cc)] = x[r];
+        } else {  // zero the strictly upper blocks
+            for (int e = tid - 64; e < 64 * 64; e += kThr - 64) {
+                const int r = e >> 6, cc = e & 63;
+                if ((r >> 4) < (cc >> 4)) Tscr[scr(r, cc)] = 0.f;
+            }
+        }
+        __syncthreads();
+        // off-diagonal blocks by distance: T_rc = -T_rr * sum_{k=c}^{r-1} A_rk T_kc,
+        // each thread a 4-column strip of one row of one block
+        for (int dist = 1; dist < 4; ++dist) {
+            const int nb = 4 - dist;
+            const int blk = tid >> 6, rr = (tid >> 2) & 15, c4 = (tid & 3) * 4;
+            if (blk < nb) {
+                const int cb = blk, r = blk + dist;
+                float acc[4] = {0.f, 0.f, 0.f, 0.f};
+                for (int k = cb; k < r; ++k) {
+#pragma unroll
+                    for (int m = 0; m < 16; ++m) {
+                        const float a = Ascr[scr(16 * r + rr, 16 * k + m)];
+                        const float4 t4 = *reinterpret_cast<const float4 *>(&Tscr[scr(16 * k + m, 16 * cb + c4)]);
+                        acc[0] = fmaf(a, t4.x, acc[0]);
+                        acc[1] = fmaf(a, t4.y, acc[1]);
+                        acc[2] = fmaf(a, t4.z, acc[2]);
+                        acc[3] = fmaf(a, t4.w, acc[3]);
+                    }
+                }
+                *reinterpret_cast<float4 *>(&inv_s[blk * 256 + rr * 16 + c4]) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+            }
+            __syncthreads();
+            if (blk < nb) {
+                const int cb = blk, r = blk + dist;
+                float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int m = 0; m < 16; ++m) {
+                    const float tr = Tscr[scr(16 * r + rr, 16 * r + m)];
+                    const float4 m4 = *reinterpret_cast<const float4 *>(&inv_s[blk * 256 + m * 16 + c4]);
+                    acc[0] = fmaf(tr, m4.x, acc[0]);
+                    acc[1] = fmaf(tr, m4.y, acc[1]);
+                    acc[2] = fmaf(tr, m4.z, acc[2]);
+                    acc[3] = fmaf(tr, m4.w, acc[3]);
+                }
+                *reinterpret_cast<float4 *>(&Tscr[scr(16 * r + rr, 16 * cb + c4)]) = make_float4(-acc[0], -acc[1], -acc[2], -acc[3]);
+            }
+            __syncthreads();
+        }
+        // T_beta = T diag(beta), rewritten in place as a K-major tile
+        {
+            const int t = tid >> 3, i0 = (tid & 7) * 8;
+            float tv[8];
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {
+                const float4 x = *reinterpret_cast<const float4 *>(&Tscr[scr(t, i0 + 4 * k)]);
+                tv[4 * k] = x.x * beta_s[i0 + 4 * k];
+                tv[4 * k + 1] = x.y * beta_s[i0 + 4 * k + 1];
+                tv[4 * k + 2] = x.z * beta_s[i0 + 4 * k + 2];
+                tv[4 * k + 3] = x.w * beta_s[i0 + 4 * k + 3];
             }
             __syncthreads();
 #pragma unroll
-            for (int k = 0; k < 16; ++k) {
-                const int e = tid + kThr * k;
-                *(float *)(sm + OFF_TB + cm_off(e >> 6, e & 63, 64)) = to_tf32(tv[k]);
-            }
-        }
-        // ---- gamma * Q S, scaled in place in TMEM
-        if (!wait_bar(2, par)) { failed = true; break; }
-        fence_after_sync();
-        {
-            float v[32];
-            tmem_ld32(taddr(tm + T_QS, 32 * quarter, 32 * half), v);
-            tmem_wait_ld();
-            const float gt = gam_s[(16 * quarter + lane) & 63];
-#pragma unroll
-            for (int j = 0; j < 32; ++j) v[j] *= gt;
-            tmem_st32(taddr(tm + T_QS, 32 * quarter, 32 * half), v);
-            tmem_wait_st();
+            for (int k = 0; k < 2; ++k)
+                *reinterpret_cast<float4 *>(sm + OFF_TB + kmaj_off(t, i0 + 4 * k, 64)) =
+                    tf32x4(tv[4 * k], tv[4 * k + 1], tv[4 * k + 2], tv[4 * k + 3]);
         }
         fence_smem_to_async();
         fence_before_sync();
         __syncthreads();
-        // [K;Q] is free: fetch the next chunk's
-        if (c + 1 < nchunks) {
-            load_kq(c + 1);
-            load_gates(c + 1);
-        }
-        cp_async_commit();
 
-        // ---- MMA_2: u = T_beta V'
+        // ---- [K;Q] is free: next chunk's; MMA_2: u = T_beta V'
+        if (c + 1 < nchunks) load_gates(c + 1);
         if (tid == 0) {
+            if (c + 1 < nchunks) issue_kq(c + 1);
             fence_after_sync();
-            gemm<64, 64, 64, false, true>(tm + T_U, sb + OFF_TB, 64, sb + OFF_V, 64, false);
-            mma_commit(&bar[3]);
+            gemm<64, 64, 64, false, true>(tm + T_U, sb + OFF_TB, 8192, sb + OFF_V, 64, false);
+            mma_commit(&bar[B_2]);
         }
-        if (!wait_bar(3, par)) { failed = true; break; }
+        if (!wait_bar(B_2, par)) { failed = true; break; }
         fence_after_sync();
-        // V and T_beta are free: next chunk's V
-        if (c + 1 < nchunks) load_v(c + 1);
-        cp_async_commit();
+        if (tid == 0 && c + 1 < nchunks) issue_v(c + 1);  // V' consumed
         {
-            float v[32];
-            tmem_ld32(taddr(tm + T_U, 32 * quarter, 32 * half), v);
+            float v[16];
+            tmem_ld16(taddr(tm + T_U, 32 * quarter, col), v);
             tmem_wait_ld();
-            if (lane < 16) {
+            if (lane < 16) {  // M=64 layout: row t at lane 16*quarter + l of quarter `quarter`
                 const int t = 16 * quarter + lane;
                 const float kd = kd_s[t];
 #pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    const int jj = 32 * half + j;
-                    *(float *)(sm + OFF_U + mn_off(t, jj, 64)) = to_tf32(v[j]);
-                    *(float *)(sm + OFF_TB + mn_off(t, jj, 64)) = to_tf32(kd * v[j]);
+                for (int k = 0; k < 4; ++k) {
+                    *reinterpret_cast<float4 *>(sm + OFF_U + mn_off(t, col + 4 * k, 64)) =
+                        tf32x4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
+                    *reinterpret_cast<float4 *>(sm + OFF_TB + mn_off(t, col + 4 * k, 64)) =
+                        tf32x4(kd * v[4 * k], kd * v[4 * k + 1], kd * v[4 * k + 2], kd * v[4 * k + 3]);
                 }
             }
         }
-        cp_async_wait<2>();  // group 3 (K, token-major copy) of this chunk
         fence_smem_to_async();
+        if (!wait_bar(B_KMN, par)) { failed = true; break; }
         fence_before_sync();
         __syncthreads();
 
-        // ---- MMA_3: dS = K^T u~ ; MMA_4: y = gamma QS + P u
+        // ---- MMA_3: dS = K^T u~ ; MMA_4: y = gamma QS + P u (128-row view of P)
         if (tid == 0) {
             fence_after_sync();
             gemm<128, 64, 64, true, true>(tm + T_DS, sb + OFF_KMN, 64, sb + OFF_TB, 64, false);
-            gemm<64, 64, 64, false, true>(tm + T_QS, sb + OFF_P, 64, sb + OFF_U, 64, true);
-            mma_commit(&bar[4]);
+            gemm<128, 64, 64, false, true>(tm + T_1, sb + OFF_P - 8192, 8192, sb + OFF_U, 64, true);
+            mma_commit(&bar[B_3]);
         }
-        if (!wait_bar(4, par)) { failed = true; break; }
+        if (!wait_bar(B_3, par)) { failed = true; break; }
         fence_after_sync();
-        if (c + 1 < nchunks) load_kmn(c + 1);
-        cp_async_commit();
+        if (tid == 0 && c + 1 < nchunks) issue_kmn(c + 1);  // K (token-major copy) consumed
         {
-            // state: S <- gamma_C S + dS (fp32 in registers), tf32 copy for the next MMAs
-            float v[32];
-            tmem_ld32(taddr(tm + T_DS, 32 * quarter, 32 * half), v);
+            float v[16];
+            tmem_ld16(taddr(tm + T_DS, 32 * quarter, col), v);
             tmem_wait_ld();
             const float gc = gam_s[n - 1];
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-                S[j] = fmaf(gc, S[j], v[j]);
-                *(float *)(sm + OFF_S + mn_off(d_own, 32 * half + j, kHeadDim)) = to_tf32(S[j]);
-            }
-            // outputs of this chunk
-            float y[32];
-            tmem_ld32(taddr(tm + T_QS, 32 * quarter, 32 * half), y);
-            tmem_wait_ld();
-            const int t = 16 * quarter + lane;
-            if (lane < 16 && t < n) {
-                TO *o = out + (tok + t) * v_row + h * kHeadDim + col0 + 32 * half;
+            for (int j = 0; j < 16; ++j) S[j] = fmaf(gc, S[j], v[j]);
 #pragma unroll
-                for (int j = 0; j < 32; ++j) store_out(o + j, y[j]);
-            }
+            for (int k = 0; k < 4; ++k)
+                *reinterpret_cast<float4 *>(sm + OFF_S + mn_off(d_own, col + 4 * k, kHeadDim)) =
+                    tf32x4(S[4 * k], S[4 * k + 1], S[4 * k + 2], S[4 * k + 3]);
+            float y[16];
+            tmem_ld16(taddr(tm + T_1, 32 * quarter, col), y);
+            tmem_wait_ld();
+            const int t = 32 * quarter + lane - 64;
+            if (quarter >= 2 && t < n) store_row16<TO>(out + (tok + t) * v_row + h * kHeadDim + col0 + col, y);
         }
-        fence_smem_to_async();
         fence_before_sync();
         __syncthreads();
     }
 
     // ---------------------------------------------------------------- tear-down
-    cp_async_wait<0>();
-    const int64_t st_off = (((int64_t)b * p.n_v + h) * kHeadDim + d_own) * kHeadDim + col0 + 32 * half;
     if (p.fin) {
+        if (failed) {
 #pragma unroll
-        for (int j = 0; j < 32; ++j) p.fin[st_off + j] = failed ? __int_as_float(0x7fc00000) : S[j];
+            for (int j = 0; j < 16; ++j) S[j] = __int_as_float(0x7fc00000);
+        }
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+            *reinterpret_cast<float4 *>(p.fin + st_off + 4 * k) = make_float4(S[4 * k], S[4 * k + 1], S[4 * k + 2], S[4 * k + 3]);
     }
-    if (failed) {  // a tensor-core wait gave up: poison this CTA's outputs
+    if (failed) {  // a wait gave up: poison this CTA's outputs
         for (int e = tid; e < L * kN; e += kThr) {
             const int t = e / kN, j = e % kN;
-            store_out(out + (seq0 + t) * v_row + h * kHeadDim + col0 + j, __int_as_float(0x7fc00000));
+            out[(seq0 + t) * v_row + h * kHeadDim + col0 + j] = from_f32<TO>(__int_as_float(0x7fc00000));
         }
     }
     fence_before_sync();
     __syncthreads();
     if (warp == 0) tmem_dealloc(tm, kTmemCols);
+}
+
+// ---------------------------------------------------------------- host side
+static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void *f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = (PFN_cuTensorMapEncodeTiled_v12000)f;
+    }
+    return fn;
+}
+
+// 2-D map over a [rows x width] fp32 matrix, boxes of 32 columns x 64 rows
+static bool encode_rows(CUtensorMap *m, const float *base, int64_t width, int64_t rows,
+                        CUtensorMapSwizzle swz) {
+    auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)width, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)width * 4};
+    cuuint32_t box[2] = {32, 64}, es[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, (void *)base, dims, strides, box, es,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 template <class TI, class TO>
@@ -479,10 +535,19 @@ static cudaError_t launch_tc_t(const TcParams &p, cudaStream_t s) {
     return cudaGetLastError();
 }
 
-cudaError_t launch_prefill_tc(const ScanParams &sp, bool in_bf16, bool out_bf16, cudaStream_t s) {
+cudaError_t launch_prefill_tc(const ScanParams &sp, int64_t total_tokens, bool in_bf16,
+                              bool out_bf16, cudaStream_t s) {
     if (sp.n_seqs <= 0) return cudaSuccess;
-    TcParams p{sp.qh, sp.kh, sp.vh, sp.alpha, sp.beta, sp.cu, sp.init, sp.fin, sp.out,
-               sp.n_seqs, sp.n_qk, sp.n_v};
+    TcParams p{};
+    const int64_t T = total_tokens > 0 ? total_tokens : 1;
+    const int64_t wqk = (int64_t)sp.n_qk * kHeadDim, wv = (int64_t)sp.n_v * kHeadDim;
+    if (!encode_rows(&p.tm_k, sp.kh, wqk, T, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !encode_rows(&p.tm_q, sp.qh, wqk, T, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !encode_rows(&p.tm_kmn, sp.kh, wqk, T, CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B) ||
+        !encode_rows(&p.tm_v, sp.vh, wv, T, CU_TENSOR_MAP_SWIZZLE_128B))
+        return cudaErrorInvalidValue;
+    p.alpha = sp.alpha; p.beta = sp.beta; p.cu = sp.cu; p.init = sp.init; p.fin = sp.fin;
+    p.out = sp.out; p.n_seqs = sp.n_seqs; p.n_qk = sp.n_qk; p.n_v = sp.n_v;
     if (in_bf16) return out_bf16 ? launch_tc_t<gdn::bf16, gdn::bf16>(p, s) : launch_tc_t<gdn::bf16, float>(p, s);
     return out_bf16 ? launch_tc_t<float, gdn::bf16>(p, s) : launch_tc_t<float, float>(p, s);
 }

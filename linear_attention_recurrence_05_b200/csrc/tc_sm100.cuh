@@ -2,20 +2,17 @@
 // chunked prefill.  Operands are fp32 values in shared memory read as TF32
 // (kind::tf32, 8 K-elements per instruction), accumulators are fp32 in tensor memory.
 //
-// Shared-memory operand layouts (fp32 elements):
-//  * K-major operands (rows = M or N index, columns = K index) use the no-swizzle
-//    "core matrix" layout: 8-row x 4-column core matrices of 128 contiguous bytes
-//    (row r of a core matrix at +16*r), consecutive along the columns, row groups of 8
-//    rows C*32 bytes apart.  K step s (8 columns) starts at +256*s; LBO = 128 B (next
-//    4 columns), SBO = C*32 B (next 8 rows).
-//  * MN-major operands (rows = K index, columns = M or N index) use the 128-byte
-//    swizzle with 32-byte granules, the only MN-major layout the tensor core takes for
-//    32-bit elements: columns in blocks of 32 (128 B per row, R*128 bytes per block),
-//    and inside each 4-row group the 32-byte granule g of row r sits at g ^ (r % 4).
-//    K step s (8 rows) starts at +1024*s; LBO = R*128 B (next 32 columns), SBO = 512 B
-//    (next 4 rows).
-// A matrix contracted over both of its indices (K of the chunk: over features in
-// K K^T and K S, over tokens in K^T u) is therefore kept in both layouts.
+// Shared-memory operand layouts (fp32 elements), both made of 128-byte rows grouped
+// in blocks of 32 columns (a [R x C] tile is C/32 blocks of R*128 bytes):
+//  * K-major operands (rows = M or N index, columns = K index): 128-byte swizzle with
+//    16-byte chunks, chunk c of row r at c ^ (r % 8) (what TMA's SWIZZLE_128B writes).
+//    K step s (8 columns) starts at block(s/4) + (s%4)*32 B; SBO = 1024 B (8 rows).
+//  * MN-major operands (rows = K index, columns = M or N index): 128-byte swizzle with
+//    32-byte granules, granule g of row r at g ^ (r % 4) -- the only MN-major layout
+//    the tensor core takes for 32-bit elements (TMA: SWIZZLE_128B_ATOM_32B).
+//    K step s (8 rows) starts at +1024*s; LBO = R*128 B (next 32 columns), SBO = 512 B.
+// A matrix contracted over both of its indices (K of a chunk: over features in K K^T
+// and K S, over tokens in K^T u) is therefore staged in both layouts.
 #pragma once
 
 #include <stdint.h>
@@ -27,11 +24,12 @@ __device__ __forceinline__ uint32_t smem_u32(const void *p) {
     return (uint32_t)__cvta_generic_to_shared(p);
 }
 
-// byte offset of element (r, c) of a [R x C] fp32 tile in the core-matrix (K-major) layout
-__host__ __device__ __forceinline__ uint32_t cm_off(int r, int c, int C) {
-    return (uint32_t)((((r >> 3) * (C >> 2) + (c >> 2)) << 7) + ((r & 7) << 4) + ((c & 3) << 2));
+// byte offset of element (r, c) of a [R x C] fp32 tile, K-major 128B swizzle
+__host__ __device__ __forceinline__ uint32_t kmaj_off(int r, int c, int R) {
+    return (uint32_t)((c >> 5) * R * 128 + r * 128 + ((((c & 31) >> 2) ^ (r & 7)) << 4) +
+                      ((c & 3) << 2));
 }
-// byte offset of element (r, c) of a [R x C] fp32 tile in the 32-byte-granule swizzle (MN-major)
+// byte offset of element (r, c) of a [R x C] fp32 tile, MN-major 32-byte-granule swizzle
 __host__ __device__ __forceinline__ uint32_t mn_off(int r, int c, int R) {
     return (uint32_t)((c >> 5) * R * 128 + r * 128 + ((((c & 31) >> 3) ^ (r & 3)) << 5) +
                       ((c & 7) << 2));
@@ -45,15 +43,15 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo, uint
     d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
     d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
     d |= (uint64_t)1 << 46;                  // descriptor version for sm_100
-    d |= (uint64_t)(layout & 7u) << 61;      // 0: no swizzle, 1: 128B with 32B granules
+    d |= (uint64_t)(layout & 7u) << 61;      // 2: 128B swizzle, 1: 128B with 32B granules
     return d;
 }
 
-// K-major view of a core-matrix tile with C columns (= K extent), K step s
-__device__ __forceinline__ uint64_t desc_kmajor(uint32_t base, int C, int s) {
-    return smem_desc(base + (uint32_t)(s * 256), 128, (uint32_t)(C * 32), 0);
+// K-major view of a tile whose 32-column blocks are `blk` bytes apart, K step s
+__device__ __forceinline__ uint64_t desc_kmajor(uint32_t base, uint32_t blk, int s) {
+    return smem_desc(base + (uint32_t)(s >> 2) * blk + (uint32_t)(s & 3) * 32, 16, 1024, 2);
 }
-// MN-major view of a swizzled tile with R rows (= K extent), K step s (8 rows)
+// MN-major view of a tile with R rows (= K extent), K step s (8 rows)
 __device__ __forceinline__ uint64_t desc_mnmajor(uint32_t base, int R, int s) {
     return smem_desc(base + (uint32_t)(s * 1024), (uint32_t)(R * 128), 512, 1);
 }
@@ -76,16 +74,16 @@ __device__ __forceinline__ void mma_tf32(uint32_t d_tmem, uint64_t a, uint64_t b
 }
 
 // D[M x N] (+)= A[M x K] B[K x N], K a multiple of 8, issued by one thread.
-// a_dim / b_dim: the tile's column count C for a K-major operand, its row count R for
-// an MN-major one.
+// A K-major: a_arg = byte distance between its 32-column blocks; A MN-major: a_arg = its
+// row count R (= K).  Same for B.
 template <int M, int N, int K, bool A_MN, bool B_MN>
-__device__ __forceinline__ void gemm(uint32_t d_tmem, uint32_t a_base, int a_dim, uint32_t b_base,
-                                     int b_dim, bool accumulate) {
+__device__ __forceinline__ void gemm(uint32_t d_tmem, uint32_t a_base, uint32_t a_arg,
+                                     uint32_t b_base, uint32_t b_arg, bool accumulate) {
     constexpr uint32_t id = idesc_tf32(M, N, A_MN, B_MN);
 #pragma unroll
     for (int s = 0; s < K / 8; ++s) {
-        const uint64_t a = A_MN ? desc_mnmajor(a_base, a_dim, s) : desc_kmajor(a_base, a_dim, s);
-        const uint64_t b = B_MN ? desc_mnmajor(b_base, b_dim, s) : desc_kmajor(b_base, b_dim, s);
+        const uint64_t a = A_MN ? desc_mnmajor(a_base, (int)a_arg, s) : desc_kmajor(a_base, a_arg, s);
+        const uint64_t b = B_MN ? desc_mnmajor(b_base, (int)b_arg, s) : desc_kmajor(b_base, b_arg, s);
         mma_tf32(d_tmem, a, b, id, (accumulate || s > 0) ? 1u : 0u);
     }
 }
@@ -163,6 +161,32 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
 #pragma unroll
     for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
+// 16 consecutive columns of this thread's lane
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
+    uint32_t r[16];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+          "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const float (&v)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+        "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
+        "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
+        "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])), "r"(__float_as_uint(v[8])),
+        "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
+        "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
+        "r"(__float_as_uint(v[15]))
+        : "memory");
+}
+
 __device__ __forceinline__ void tmem_wait_ld() {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
@@ -198,6 +222,22 @@ __device__ __forceinline__ float to_tf32(float x) {
     uint32_t r;
     asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
     return __uint_as_float(r);
+}
+
+// ------------------------------------------------------------------ TMA (no multicast)
+__device__ __forceinline__ void mbar_expect_tx(uint64_t *m, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(m)),
+                 "r"(bytes)
+                 : "memory");
+}
+// 2D tile load global -> shared (this CTA), completion counted on mbarrier `m`
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const void *tmap, int x, int y,
+                                            uint64_t *m) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
+        "[%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+        "l"(tmap), "r"(x), "r"(y), "r"(smem_u32(m))
+        : "memory");
 }
 
 // ------------------------------------------------------------------ cp.async (16 B)
