@@ -232,6 +232,7 @@ __global__ void __launch_bounds__(kThr, 1) prefill_tc_kernel(const __grid_consta
             g_s[tid] = safe_log_alpha(a_next);
             beta_s[tid] = b_next;
         }
+        if (c + 1 < nchunks) load_gates(c + 1);  // a whole chunk ahead of their use
         fence_smem_to_async();  // S tile written by the previous chunk (or the set-up)
         if (!wait_bar(B_KQ, par)) { failed = true; break; }
         if (warp == 0) {  // inclusive scan of log alpha, two rows per lane
@@ -300,6 +301,7 @@ __global__ void __launch_bounds__(kThr, 1) prefill_tc_kernel(const __grid_consta
         }
         // ---- epilogue 1: V' = V - gamma * K S (rows 0-63); gamma * Q S in place (rows 64-127)
         if (!wait_bar(B_1, par)) { failed = true; break; }
+        if (tid == 0 && c + 1 < nchunks) issue_kq(c + 1);  // MMA_a and MMA_1 are done with [K;Q]
         if (!wait_bar(B_V, par)) { failed = true; break; }
         fence_after_sync();
         {
@@ -334,71 +336,100 @@ __global__ void __launch_bounds__(kThr, 1) prefill_tc_kernel(const __grid_consta
             }
         }
 
-        // ---- T = (I + A)^-1 by 16 x 16 blocks (fp32 scratch in OFF_TB)
-        if (tid < 64) {  // diagonal blocks: column cc of block bb by forward substitution
+        // ---- T = (I + A)^-1 (fp32 scratch in OFF_TB): 16 x 16 diagonal blocks by forward
+        // substitution, then the two 32 x 32 halves, then the lower-left 32 x 32 block:
+        //   [[X, 0], [Y, Z]]^-1 = [[X^-1, 0], [-Z^-1 Y X^-1, Z^-1]]
+        if (tid < 64) {  // diagonal blocks: column cc of block bb
             const int bb = tid >> 4, cc = tid & 15;
             float x[16];
 #pragma unroll
             for (int r = 0; r < 16; ++r) {
-                float acc = (r == cc) ? 1.f : 0.f;
+                float a0 = (r == cc) ? 1.f : 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
 #pragma unroll
-                for (int m = 0; m < r; ++m) acc = fmaf(-Ascr[scr(16 * bb + r, 16 * bb + m)], x[m], acc);
-                x[r] = (r < cc) ? 0.f : acc;
+                for (int m = 0; m + 3 < r; m += 4) {
+                    const float4 a4 = *reinterpret_cast<const float4 *>(&Ascr[scr(16 * bb + r, 16 * bb + m)]);
+                    a0 = fmaf(-a4.x, x[m], a0);
+                    a1 = fmaf(-a4.y, x[m + 1], a1);
+                    a2 = fmaf(-a4.z, x[m + 2], a2);
+                    a3 = fmaf(-a4.w, x[m + 3], a3);
+                }
+#pragma unroll
+                for (int m = r & ~3; m < r; ++m) a0 = fmaf(-Ascr[scr(16 * bb + r, 16 * bb + m)], x[m], a0);
+                x[r] = (r < cc) ? 0.f : (a0 + a1) + (a2 + a3);
             }
 #pragma unroll
             for (int r = 0; r < 16; ++r) Tscr[scr(16 * bb + r, 16 * bb + cc)] = x[r];
-        } else {  // zero the strictly upper blocks
+        } else {  // zero the strictly upper part outside the diagonal blocks
             for (int e = tid - 64; e < 64 * 64; e += kThr - 64) {
                 const int r = e >> 6, cc = e & 63;
                 if ((r >> 4) < (cc >> 4)) Tscr[scr(r, cc)] = 0.f;
             }
         }
         __syncthreads();
-        // off-diagonal blocks by distance: T_rc = -T_rr * sum_{k=c}^{r-1} A_rk T_kc,
-        // each thread a 4-column strip of one row of one block
-        for (int dist = 1; dist < 4; ++dist) {
-            const int nb = 4 - dist;
-            const int blk = tid >> 6, rr = (tid >> 2) & 15, c4 = (tid & 3) * 4;
-            if (blk < nb) {
-                const int cb = blk, r = blk + dist;
-                float acc[4] = {0.f, 0.f, 0.f, 0.f};
-                for (int k = cb; k < r; ++k) {
+        // 32 x 32 halves hh = 0, 1 (rows/cols 32hh..32hh+31): T_10 = -T_11 A_10 T_00 in
+        // 16-blocks; then the lower-left 32 x 32 block T_bl = -T_br A_bl T_top.  Each
+        // thread computes a 4-column strip of one row (float4 operand loads).
+        if (tid < 128) {
+            const int hh = tid >> 6, rr = (tid >> 2) & 15, c4 = (tid & 3) * 4, o = 32 * hh;
+            float a4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                    for (int m = 0; m < 16; ++m) {
-                        const float a = Ascr[scr(16 * r + rr, 16 * k + m)];
-                        const float4 t4 = *reinterpret_cast<const float4 *>(&Tscr[scr(16 * k + m, 16 * cb + c4)]);
-                        acc[0] = fmaf(a, t4.x, acc[0]);
-                        acc[1] = fmaf(a, t4.y, acc[1]);
-                        acc[2] = fmaf(a, t4.z, acc[2]);
-                        acc[3] = fmaf(a, t4.w, acc[3]);
-                    }
-                }
-                *reinterpret_cast<float4 *>(&inv_s[blk * 256 + rr * 16 + c4]) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+            for (int m = 0; m < 16; ++m) {
+                const float a = Ascr[scr(o + 16 + rr, o + m)];
+                const float4 t4 = *reinterpret_cast<const float4 *>(&Tscr[scr(o + m, o + c4)]);
+                a4[0] = fmaf(a, t4.x, a4[0]); a4[1] = fmaf(a, t4.y, a4[1]);
+                a4[2] = fmaf(a, t4.z, a4[2]); a4[3] = fmaf(a, t4.w, a4[3]);
             }
-            __syncthreads();
-            if (blk < nb) {
-                const int cb = blk, r = blk + dist;
-                float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-                for (int m = 0; m < 16; ++m) {
-                    const float tr = Tscr[scr(16 * r + rr, 16 * r + m)];
-                    const float4 m4 = *reinterpret_cast<const float4 *>(&inv_s[blk * 256 + m * 16 + c4]);
-                    acc[0] = fmaf(tr, m4.x, acc[0]);
-                    acc[1] = fmaf(tr, m4.y, acc[1]);
-                    acc[2] = fmaf(tr, m4.z, acc[2]);
-                    acc[3] = fmaf(tr, m4.w, acc[3]);
-                }
-                *reinterpret_cast<float4 *>(&Tscr[scr(16 * r + rr, 16 * cb + c4)]) = make_float4(-acc[0], -acc[1], -acc[2], -acc[3]);
-            }
-            __syncthreads();
+            *reinterpret_cast<float4 *>(&inv_s[hh * 256 + rr * 16 + c4]) = make_float4(a4[0], a4[1], a4[2], a4[3]);
         }
+        __syncthreads();
+        if (tid < 128) {
+            const int hh = tid >> 6, rr = (tid >> 2) & 15, c4 = (tid & 3) * 4, o = 32 * hh;
+            float a4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int m = 0; m < 16; ++m) {
+                const float t = Tscr[scr(o + 16 + rr, o + 16 + m)];
+                const float4 m4 = *reinterpret_cast<const float4 *>(&inv_s[hh * 256 + m * 16 + c4]);
+                a4[0] = fmaf(t, m4.x, a4[0]); a4[1] = fmaf(t, m4.y, a4[1]);
+                a4[2] = fmaf(t, m4.z, a4[2]); a4[3] = fmaf(t, m4.w, a4[3]);
+            }
+            *reinterpret_cast<float4 *>(&Tscr[scr(o + 16 + rr, o + c4)]) = make_float4(-a4[0], -a4[1], -a4[2], -a4[3]);
+        }
+        __syncthreads();
+        // M = A_bl T_top, kept in the (zero) upper-right block of T
+        if (tid < 256) {
+            const int r = tid >> 3, c4 = (tid & 7) * 4;
+            float a4[4] = {0.f, 0.f, 0.f, 0.f};
+            for (int m = c4; m < 32; ++m) {  // T_top is lower triangular
+                const float a = Ascr[scr(32 + r, m)];
+                const float4 t4 = *reinterpret_cast<const float4 *>(&Tscr[scr(m, c4)]);
+                a4[0] = fmaf(a, t4.x, a4[0]); a4[1] = fmaf(a, t4.y, a4[1]);
+                a4[2] = fmaf(a, t4.z, a4[2]); a4[3] = fmaf(a, t4.w, a4[3]);
+            }
+            *reinterpret_cast<float4 *>(&Tscr[scr(r, 32 + c4)]) = make_float4(a4[0], a4[1], a4[2], a4[3]);
+        }
+        __syncthreads();
+        // T_bl = -T_br M
+        if (tid < 256) {
+            const int r = tid >> 3, c4 = (tid & 7) * 4;
+            float a4[4] = {0.f, 0.f, 0.f, 0.f};
+            for (int m = 0; m <= r; ++m) {  // T_br is lower triangular
+                const float t = Tscr[scr(32 + r, 32 + m)];
+                const float4 m4 = *reinterpret_cast<const float4 *>(&Tscr[scr(m, 32 + c4)]);
+                a4[0] = fmaf(t, m4.x, a4[0]); a4[1] = fmaf(t, m4.y, a4[1]);
+                a4[2] = fmaf(t, m4.z, a4[2]); a4[3] = fmaf(t, m4.w, a4[3]);
+            }
+            *reinterpret_cast<float4 *>(&Tscr[scr(32 + r, c4)]) = make_float4(-a4[0], -a4[1], -a4[2], -a4[3]);
+        }
+        __syncthreads();
         // T_beta = T diag(beta), rewritten in place as a K-major tile
         {
             const int t = tid >> 3, i0 = (tid & 7) * 8;
+            const bool upper_right = t < 32 && i0 >= 32;  // zero in T; held the merge product
             float tv[8];
 #pragma unroll
             for (int k = 0; k < 2; ++k) {
-                const float4 x = *reinterpret_cast<const float4 *>(&Tscr[scr(t, i0 + 4 * k)]);
+                float4 x = *reinterpret_cast<const float4 *>(&Tscr[scr(t, i0 + 4 * k)]);
+                if (upper_right) x = make_float4(0.f, 0.f, 0.f, 0.f);
                 tv[4 * k] = x.x * beta_s[i0 + 4 * k];
                 tv[4 * k + 1] = x.y * beta_s[i0 + 4 * k + 1];
                 tv[4 * k + 2] = x.z * beta_s[i0 + 4 * k + 2];
@@ -414,10 +445,8 @@ __global__ void __launch_bounds__(kThr, 1) prefill_tc_kernel(const __grid_consta
         fence_before_sync();
         __syncthreads();
 
-        // ---- [K;Q] is free: next chunk's; MMA_2: u = T_beta V'
-        if (c + 1 < nchunks) load_gates(c + 1);
+        // ---- MMA_2: u = T_beta V'
         if (tid == 0) {
-            if (c + 1 < nchunks) issue_kq(c + 1);
             fence_after_sync();
             gemm<64, 64, 64, false, true>(tm + T_U, sb + OFF_TB, 8192, sb + OFF_V, 64, false);
             mma_commit(&bar[B_2]);

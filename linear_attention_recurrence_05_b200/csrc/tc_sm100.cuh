@@ -75,16 +75,22 @@ __device__ __forceinline__ void mma_tf32(uint32_t d_tmem, uint64_t a, uint64_t b
 
 // D[M x N] (+)= A[M x K] B[K x N], K a multiple of 8, issued by one thread.
 // A K-major: a_arg = byte distance between its 32-column blocks; A MN-major: a_arg = its
-// row count R (= K).  Same for B.
+// row count R (= K).  Same for B.  Only the 14-bit start-address field changes from one
+// K step to the next, so each step's descriptors are the first step's plus a constant.
 template <int M, int N, int K, bool A_MN, bool B_MN>
 __device__ __forceinline__ void gemm(uint32_t d_tmem, uint32_t a_base, uint32_t a_arg,
                                      uint32_t b_base, uint32_t b_arg, bool accumulate) {
     constexpr uint32_t id = idesc_tf32(M, N, A_MN, B_MN);
+    const uint64_t a0 = A_MN ? desc_mnmajor(a_base, (int)a_arg, 0) : desc_kmajor(a_base, a_arg, 0);
+    const uint64_t b0 = B_MN ? desc_mnmajor(b_base, (int)b_arg, 0) : desc_kmajor(b_base, b_arg, 0);
+    const uint32_t a_blk16 = A_MN ? 0u : (a_arg >> 4), b_blk16 = B_MN ? 0u : (b_arg >> 4);
 #pragma unroll
     for (int s = 0; s < K / 8; ++s) {
-        const uint64_t a = A_MN ? desc_mnmajor(a_base, (int)a_arg, s) : desc_kmajor(a_base, a_arg, s);
-        const uint64_t b = B_MN ? desc_mnmajor(b_base, (int)b_arg, s) : desc_kmajor(b_base, b_arg, s);
-        mma_tf32(d_tmem, a, b, id, (accumulate || s > 0) ? 1u : 0u);
+        // start-address step (16-byte units): MN-major +1024 B per step; K-major +32 B per
+        // step inside a 32-column block, +block per 4 steps
+        const uint32_t da = A_MN ? (uint32_t)(s * 64) : (uint32_t)((s >> 2) * a_blk16 + (s & 3) * 2);
+        const uint32_t db = B_MN ? (uint32_t)(s * 64) : (uint32_t)((s >> 2) * b_blk16 + (s & 3) * 2);
+        mma_tf32(d_tmem, a0 + da, b0 + db, id, (accumulate || s > 0) ? 1u : 0u);
     }
 }
 
