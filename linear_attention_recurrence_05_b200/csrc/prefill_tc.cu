@@ -3,25 +3,28 @@
 // The recurrence of the page "ARCHITECTURE PREVIEW / FIELD NOTES", section 03 (GATED
 // DELTANET equations), in chunks of 64 tokens.  Within a chunk, with
 // g_t = sum_{s<=t} log alpha_s, gamma_t = exp(g_t) and S the state entering the chunk:
-//     A_ti = beta_t exp(g_t - g_i) k_t.k_i  (i < t),   T = (I + A)^-1
-//     u    = T diag(beta) (V - diag(gamma) K S)                      (the WY/UT solve)
+//     A_ti = beta_t exp(g_t - g_i) k_t.k_i  (i < t),   T = (I + A)^-1,  T_beta = T diag(beta)
+//     u    = T_beta (V - diag(gamma) K S)                             (the WY/UT solve)
 //     y_t  = gamma_t S^T q_t + sum_{i<=t} exp(g_t - g_i)(q_t.k_i) u_i
 //     S   <- gamma_C S + sum_i exp(g_C - g_i) k_i u_i^T
 // (u = U - W S with U = T diag(beta) V and W = T diag(beta gamma) K, regrouped so that
 // W never has to be formed).
 //
-// One CTA (16 warps) owns one (sequence, V head, 64-column half of d_v) and walks the
-// sequence's chunks in order; the column split is exact.  Per chunk, on the tensor core:
-//     MMA_a  [K;Q] K^T      M=128 N=64 K=128 -> A (strict lower) and P (lower)
-//     MMA_1  [K;Q] S        M=128 N=64 K=128 -> V' = V - gamma*KS ; gamma*QS kept in TMEM
-//     MMA_2  T_beta V'      M=64  N=64 K=64  -> u, u~ = exp(g_C - g) u
-//     MMA_3  K^T u~         M=128 N=64 K=64  -> S update (the state stays fp32 in registers)
-//     MMA_4  [*;P] u        M=128 N=64 K=64  -> accumulated onto gamma*QS: y
-// MMA_4 reads P through a 128-row view whose upper 64 rows are whatever precedes P in
-// shared memory; they land on rows 0-63 of the accumulator, which hold K S and are
-// already consumed.  On the CUDA cores: the 64 x 64 unit-lower-triangular inverse
-// (16 x 16 blocks) and the element-wise epilogues.  Operand tiles arrive by TMA
-// (2-D boxes of 32 fp32 x 64 tokens), each reloaded as soon as its last reader is done.
+// One CTA owns one (sequence, V head, 64-column slice j of d_v); the column split is
+// exact.  Its 16 warps form two groups that run one chunk apart:
+//  * prep (warps 8-15), state-independent, for chunk c+1:
+//        MMA_a  [K;Q] K^T   (M=128, N=64, K=128)  -> A (strict lower), P (lower)
+//        64 x 64 unit-lower-triangular inverse on CUDA cores -> T_beta
+//  * chain (warps 0-7), the serial state recurrence of chunk c, in transposed form so
+//    that every chain operand lives in tensor memory (A operands read from TMEM):
+//        MMA_1  S^T [K;Q]^T   (M=64, N=128, K=128) -> (K S)^T, (Q S)^T
+//        MMA_2  V'^T T_beta^T (M=64, N=64, K=64)   -> u^T        (V' = V - gamma*K S)
+//        MMA_3  u~^T K        (M=64, N=128, K=64)  -> dS^T       (u~ = exp(g_C - g) u)
+//        MMA_4  u^T P^T       (M=64, N=64, K=64)   accumulated onto (gamma*Q S)^T -> y^T
+// Tensor memory (row j of an M=64 tile at lane 32*(j/16) + j%16 + base, base 0 or 16):
+// the fp32 state lives in the upper half-lanes next to its TF32 operand copy.  Shared
+// memory holds only the K/Q tiles (TMA, no multicast), the V tile and the
+// double-buffered prep outputs.  All waits are bounded.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -37,68 +40,95 @@ using namespace tc;
 constexpr int kN = 64;          // d_v columns per CTA
 constexpr int kNS = kHeadDim / kN;
 constexpr int kThr = 512;
+constexpr int kGroup = 256;     // threads per group
 
 // shared-memory map (bytes from a 1024-aligned base)
-constexpr uint32_t OFF_S = 0;          // S       MN-major R=128 (d) x 64 (j)               32 KB
-constexpr uint32_t OFF_KQ = 32768;     // [K;Q]   K-major, 4 blocks x (K 8 KB | Q 8 KB)      64 KB
-constexpr uint32_t OFF_KMN = 98304;    // K       MN-major R=64 (i) x 128 (d)               32 KB
-constexpr uint32_t OFF_V = 131072;     // V (K-major swizzle, read by threads), then V' MN  16 KB
-constexpr uint32_t OFF_TB = 147456;    // T (fp32 scratch), then T_beta K-major, then u~ MN 16 KB
-constexpr uint32_t OFF_P = 163840;     // P       K-major R=64                               16 KB
-constexpr uint32_t OFF_U = 180224;     // A (fp32 scratch), then u MN-major                16 KB
-constexpr uint32_t OFF_MISC = 196608;
-constexpr uint32_t OFF_G = OFF_MISC;            // g[64]
-constexpr uint32_t OFF_GAM = OFF_MISC + 256;    // gamma[64]
-constexpr uint32_t OFF_BETA = OFF_MISC + 512;   // beta[64]
-constexpr uint32_t OFF_KD = OFF_MISC + 768;     // exp(g_last - g)[64]
-constexpr uint32_t OFF_INV = OFF_MISC + 1024;   // 3 x 256 floats (block products)
-constexpr uint32_t OFF_BAR = OFF_MISC + 4096;   // mbarriers
+constexpr uint32_t OFF_KQ = 0;          // [K;Q]  K-major, 4 blocks x (K 8 KB | Q 8 KB)     64 KB
+constexpr uint32_t OFF_KMN = 65536;     // K      MN-major R=64 (i) x 128 (d)              32 KB
+constexpr uint32_t OFF_V = 98304;       // V      [t][j] K-major swizzle (read by threads)  16 KB
+constexpr uint32_t OFF_TB = 114688;     // T_beta K-major [t][i], 2 buffers                 32 KB
+constexpr uint32_t OFF_P = 147456;      // P      K-major [t][i], 2 buffers                 32 KB
+constexpr uint32_t OFF_AS = 180224;     // A scratch (fp32, swizzled rows)                  16 KB
+constexpr uint32_t OFF_TS = 196608;     // T scratch (fp32, swizzled rows)                  16 KB
+constexpr uint32_t OFF_MISC = 212992;
+constexpr uint32_t OFF_GATE = OFF_MISC;            // 2 buffers x {g, gamma, beta, kd}[64]  2 KB
+constexpr uint32_t OFF_INV = OFF_MISC + 2048;      // 2 x 256 floats (block products)      2 KB
+constexpr uint32_t OFF_BAR = OFF_MISC + 4096;      // mbarriers
 constexpr uint32_t OFF_TSLOT = OFF_BAR + 128;
 constexpr uint32_t kSmem = OFF_TSLOT + 16;
-constexpr uint32_t kSmemAlloc = kSmem + 1024;   // slack to align the base to 1024
+constexpr uint32_t kSmemAlloc = kSmem + 1024;      // slack to align the base to 1024
 
-enum { B_KQ = 0, B_V, B_KMN, B_A, B_1, B_2, B_3, kNumBars };
+enum { B_KQ = 0, B_V, B_KMN, B_A, B_PREP, B_1, B_2, B_3, kNumBars };
 
-// tensor-memory columns
-constexpr uint32_t kTmemCols = 256;
-constexpr uint32_t T_A = 0;      // [K;Q]K^T    M=128
-constexpr uint32_t T_1 = 64;     // [K;Q]S, then rows 64.. = y   M=128
-constexpr uint32_t T_U = 128;    // u           M=64
-constexpr uint32_t T_DS = 192;   // K^T u~      M=128
+// tensor memory: columns (lower half-lanes | upper half-lanes of each M=64 tile)
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t T_A = 0;        // [K;Q]K^T, M=128 (all lanes)                        64 cols
+constexpr uint32_t T_1 = 64;       // lower: [(K S)^T | (Q S)^T -> y^T]  upper: dS^T     128 cols
+constexpr uint32_t T_S = 192;      // lower: S^T (TF32 operand)          upper: S^T fp32 128 cols
+constexpr uint32_t T_V = 320;      // lower: V'^T (operand)              upper: u~^T      64 cols
+constexpr uint32_t T_U = 384;      // lower: u^T (accumulator, then operand)              64 cols
+constexpr uint32_t kUpper = 16u << 16;  // lane offset of the upper half-lanes
 
 constexpr uint32_t kWaitTries = 1u << 22;
 
-// fp32 scratch [64][64] with 16-byte chunks XOR-swizzled by row (conflict-free rows and columns)
+// fp32 scratch [64][64] with 16-byte chunks XOR-swizzled by row
 __device__ __forceinline__ int scr(int r, int c) { return r * 64 + ((((c >> 2) ^ (r & 7)) << 2) | (c & 3)); }
 
 __device__ __forceinline__ float4 tf32x4(float a, float b, float c, float d) {
     return make_float4(to_tf32(a), to_tf32(b), to_tf32(c), to_tf32(d));
 }
 
-template <class TO>
-__device__ __forceinline__ void store_row16(TO *dst, const float (&v)[16]);
-template <>
-__device__ __forceinline__ void store_row16<float>(float *dst, const float (&v)[16]) {
-#pragma unroll
-    for (int k = 0; k < 4; ++k)
-        *reinterpret_cast<float4 *>(dst + 4 * k) = make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
+// named barrier over one 256-thread group; returns true if any thread passed `pred`
+__device__ __forceinline__ bool group_sync_or(int id, bool pred) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\tsetp.ne.b32 p, %1, 0;\n\t"
+        "bar.red.or.pred q, %2, 256, p;\n\tselp.u32 %0, 1, 0, q;\n\t}\n"
+        : "=r"(r)
+        : "r"((uint32_t)pred), "r"(id)
+        : "memory");
+    return r != 0;
 }
-template <>
-__device__ __forceinline__ void store_row16<bf16>(bf16 *dst, const float (&v)[16]) {
+__device__ __forceinline__ void group_sync(int id) {
+    asm volatile("bar.sync %0, 256;" ::"r"(id) : "memory");
+}
+
+// A from tensor memory (K-major), B from a shared-memory descriptor
+__device__ __forceinline__ void mma_ts(uint32_t d, uint32_t a_tmem, uint64_t b, uint32_t id, uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::tf32 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d),
+        "r"(a_tmem), "l"(b), "r"(id), "r"(acc));
+}
+// D[64 x N] (+)= A_tmem[64 x K] B[K x N]; B K-major (b_arg = block stride) or MN-major (b_arg = R)
+template <int N, int K, bool B_MN>
+__device__ __forceinline__ void gemm_ts(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_base, uint32_t b_arg,
+                                        bool accumulate) {
+    constexpr uint32_t id = idesc_tf32(64, N, false, B_MN);
+    const uint64_t b0 = B_MN ? desc_mnmajor(b_base, (int)b_arg, 0) : desc_kmajor(b_base, b_arg, 0);
+    const uint32_t b_blk16 = B_MN ? 0u : (b_arg >> 4);
 #pragma unroll
-    for (int k = 0; k < 2; ++k) {
-        uint4 w;
-        __nv_bfloat162 h0 = __floats2bfloat162_rn(v[8 * k], v[8 * k + 1]);
-        __nv_bfloat162 h1 = __floats2bfloat162_rn(v[8 * k + 2], v[8 * k + 3]);
-        __nv_bfloat162 h2 = __floats2bfloat162_rn(v[8 * k + 4], v[8 * k + 5]);
-        __nv_bfloat162 h3 = __floats2bfloat162_rn(v[8 * k + 6], v[8 * k + 7]);
-        w.x = *reinterpret_cast<uint32_t *>(&h0);
-        w.y = *reinterpret_cast<uint32_t *>(&h1);
-        w.z = *reinterpret_cast<uint32_t *>(&h2);
-        w.w = *reinterpret_cast<uint32_t *>(&h3);
-        *reinterpret_cast<uint4 *>(dst + 8 * k) = w;
+    for (int s = 0; s < K / 8; ++s) {
+        const uint32_t db = B_MN ? (uint32_t)(s * 64) : (uint32_t)((s >> 2) * b_blk16 + (s & 3) * 2);
+        mma_ts(d_tmem, a_tmem + 8 * s, b0 + db, id, (accumulate || s > 0) ? 1u : 0u);
     }
 }
+
+__device__ __forceinline__ uint16_t ld_raw(const bf16 *p) {
+    uint16_t r;
+    asm volatile("ld.global.nc.u16 %0, [%1];" : "=h"(r) : "l"(p));
+    return r;
+}
+__device__ __forceinline__ uint32_t ld_raw(const float *p) {
+    uint32_t r;
+    asm volatile("ld.global.nc.u32 %0, [%1];" : "=r"(r) : "l"(p));
+    return r;
+}
+__device__ __forceinline__ float raw_to_f32(uint16_t r) { return __uint_as_float((uint32_t)r << 16); }
+__device__ __forceinline__ float raw_to_f32(uint32_t r) { return __uint_as_float(r); }
+
+template <class TI> struct RawT { typedef uint32_t type; };
+template <> struct RawT<bf16> { typedef uint16_t type; };
 
 }  // namespace
 
@@ -120,19 +150,11 @@ __global__ void __launch_bounds__(kThr, 1) prefill_tc_kernel(const __grid_consta
     extern __shared__ unsigned char smem_raw[];
     unsigned char *sm = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
     const uint32_t sb = smem_u32(sm);
-    float *g_s = (float *)(sm + OFF_G);
-    float *gam_s = (float *)(sm + OFF_GAM);
-    float *beta_s = (float *)(sm + OFF_BETA);
-    float *kd_s = (float *)(sm + OFF_KD);
-    float *inv_s = (float *)(sm + OFF_INV);
     uint64_t *bar = (uint64_t *)(sm + OFF_BAR);
     uint32_t *tslot = (uint32_t *)(sm + OFF_TSLOT);
-    float *Ascr = (float *)(sm + OFF_U);   // A scratch (fp32, swizzled rows)
-    float *Tscr = (float *)(sm + OFF_TB);  // T scratch (fp32, swizzled rows)
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int quarter = warp & 3, cg = warp >> 2;   // TMEM lane quarter, 16-column group
-    const int col = 16 * cg;                        // first accumulator column of this thread
+    const int quarter = warp & 3;
     const int slice = blockIdx.x % kNS;
     const int h = (blockIdx.x / kNS) % p.n_v;
     const int b = blockIdx.x / (kNS * p.n_v);
@@ -140,12 +162,8 @@ __global__ void __launch_bounds__(kThr, 1) prefill_tc_kernel(const __grid_consta
     const int seq0 = p.cu[b], L = p.cu[b + 1] - p.cu[b];
     const int col0 = slice * kN;
     const int64_t v_row = (int64_t)p.n_v * kHeadDim;
-    const TI *al = (const TI *)p.alpha;
-    const TI *be = (const TI *)p.beta;
-    TO *out = (TO *)p.out;
     const int nchunks = (L + kChunk - 1) / kChunk;
 
-    // ---------------------------------------------------------------- set-up
     if (tid == 0) {
         for (int i = 0; i < kNumBars; ++i) mbar_init(&bar[i], 1);
     }
@@ -153,22 +171,11 @@ __global__ void __launch_bounds__(kThr, 1) prefill_tc_kernel(const __grid_consta
         tmem_alloc(tslot, kTmemCols);
         tmem_relinquish();
     }
-    // this thread owns S[d_own][col .. col+15]
-    const int d_own = 32 * quarter + lane;
-    const int64_t st_off = (((int64_t)b * p.n_v + h) * kHeadDim + d_own) * kHeadDim + col0 + col;
-    float S[16];
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-        float4 v4 = p.init ? *reinterpret_cast<const float4 *>(p.init + st_off + 4 * k)
-                           : make_float4(0.f, 0.f, 0.f, 0.f);
-        S[4 * k] = v4.x; S[4 * k + 1] = v4.y; S[4 * k + 2] = v4.z; S[4 * k + 3] = v4.w;
-    }
-#pragma unroll
-    for (int k = 0; k < 4; ++k)
-        *reinterpret_cast<float4 *>(sm + OFF_S + mn_off(d_own, col + 4 * k, kHeadDim)) =
-            tf32x4(S[4 * k], S[4 * k + 1], S[4 * k + 2], S[4 * k + 3]);
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    const uint32_t tm = *tslot;
 
-    // TMA issue (thread 0 only)
     auto issue_kq = [&](int c) {
         const int tok = seq0 + c * kChunk;
         mbar_expect_tx(&bar[B_KQ], 65536);
@@ -192,336 +199,380 @@ __global__ void __launch_bounds__(kThr, 1) prefill_tc_kernel(const __grid_consta
         for (int db = 0; db < 4; ++db)
             tma_load_2d(sb + OFF_KMN + db * 8192, &p.tm_kmn, gq * kHeadDim + 32 * db, tok, &bar[B_KMN]);
     };
-    // gate prefetch: thread t < 64 holds alpha/beta of row t of the next chunk
-    float a_next = 1.f, b_next = 0.f;
-    auto load_gates = [&](int c) {
-        const int n = min(kChunk, L - c * kChunk);
-        const int64_t tok = seq0 + (int64_t)c * kChunk;
-        if (tid < kChunk) {
-            a_next = tid < n ? to_f32(al[(tok + tid) * p.n_v + h]) : 1.f;
-            b_next = tid < n ? to_f32(be[(tok + tid) * p.n_v + h]) : 0.f;
-        }
-    };
 
-    fence_before_sync();
-    __syncthreads();
-    fence_after_sync();
-    const uint32_t tm = *tslot;
-    if (nchunks > 0) {
-        if (tid == 0) {
+    bool failed = false;
+
+    if (warp < 8) {
+        // ================================================================ chain group
+        const int ch = warp >> 2;                      // which 32 of each 64 columns
+        const bool upper = lane >= 16;
+        const int j = 16 * quarter + (lane & 15);      // row of the M=64 tiles (column of d_v)
+        const int tcol = 32 * ch;                      // this thread's 32 columns of 64
+        const uint32_t lrow = (uint32_t)(32 * quarter) << 16;  // warp's lane quarter
+        auto wait_all = [&](int i, uint32_t par) -> bool {
+            const bool ok = mbar_wait(&bar[i], par, kWaitTries);
+            return !group_sync_or(1, !ok);
+        };
+        // initial state: lower lanes the TF32 copy of S^T, upper lanes S^T in fp32
+        {
+            const float *src = p.init ? p.init + ((int64_t)b * p.n_v + h) * kHeadDim * kHeadDim + col0 + j : nullptr;
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                const int d0 = 64 * ch + 32 * half;
+                float v[32];
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const float s = src ? src[(int64_t)(d0 + i) * kHeadDim] : 0.f;
+                    v[i] = upper ? s : to_tf32(s);
+                }
+                tmem_st32(tm + lrow + T_S + d0, v);
+            }
+            tmem_wait_st();
+        }
+        if (tid == 0 && nchunks > 0) {
             issue_kq(0);
             issue_v(0);
             issue_kmn(0);
         }
-        load_gates(0);
-    }
-    bool failed = false;
-    // every thread waits; all agree on success
-    auto wait_bar = [&](int i, uint32_t par) -> bool {
-        bool ok = mbar_wait(&bar[i], par, kWaitTries);
-        return __syncthreads_or(!ok) == 0;
-    };
+        fence_before_sync();
+        group_sync(1);
 
-    for (int c = 0; c < nchunks; ++c) {
-        const int n = min(kChunk, L - c * kChunk);
-        const int64_t tok = seq0 + (int64_t)c * kChunk;
-        const uint32_t par = c & 1;
+        for (int c = 0; c < nchunks; ++c) {
+            const int n = min(kChunk, L - c * kChunk);
+            const int64_t tok = seq0 + (int64_t)c * kChunk;
+            const uint32_t par = c & 1;
+            const float *gate = (const float *)(sm + OFF_GATE + (c & 1) * 1024);
+            const float *gam_s = gate + 64, *kd_s = gate + 192;
 
-        // ---- gates, and this chunk's [K;Q]
-        if (tid < kChunk) {
-            g_s[tid] = safe_log_alpha(a_next);
-            beta_s[tid] = b_next;
-        }
-        if (c + 1 < nchunks) load_gates(c + 1);  // a whole chunk ahead of their use
-        fence_smem_to_async();  // S tile written by the previous chunk (or the set-up)
-        if (!wait_bar(B_KQ, par)) { failed = true; break; }
-        if (warp == 0) {  // inclusive scan of log alpha, two rows per lane
-            const float a0 = g_s[2 * lane], a1 = g_s[2 * lane + 1];
-            float s = a0 + a1;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const float y = __shfl_up_sync(0xffffffffu, s, o);
-                if (lane >= o) s += y;
+            // ---- MMA_1: S^T [K;Q]^T
+            if (!wait_all(B_KQ, par)) { failed = true; break; }
+            if (tid == 0) {
+                fence_after_sync();
+                gemm_ts<128, 128, false>(tm + T_1, tm + T_S, sb + OFF_KQ, 16384, false);
+                mma_commit(&bar[B_1]);
             }
-            const float g0 = s - a1;
-            const float glast = __shfl_sync(0xffffffffu, ((n - 1) & 1) ? s : g0, (n - 1) >> 1);
-            g_s[2 * lane] = g0;
-            g_s[2 * lane + 1] = s;
-            gam_s[2 * lane] = expf(g0);
-            gam_s[2 * lane + 1] = expf(s);
-            kd_s[2 * lane] = 2 * lane < n ? expf(glast - g0) : 0.f;
-            kd_s[2 * lane + 1] = 2 * lane + 1 < n ? expf(glast - s) : 0.f;
-        }
-        __syncthreads();
-
-        // ---- MMA_a: [K;Q] K^T ; MMA_1: [K;Q] S
-        if (tid == 0) {
+            if (!wait_all(B_1, par)) { failed = true; break; }
+            if (!wait_all(B_PREP, par)) { failed = true; break; }  // gates, T_beta, P of chunk c
+            if (tid == 0 && c + 1 < nchunks) issue_kq(c + 1);      // prep and chain are done with [K;Q]
+            if (!wait_all(B_V, par)) { failed = true; break; }
             fence_after_sync();
-            gemm<128, 64, 128, false, false>(tm + T_A, sb + OFF_KQ, 16384, sb + OFF_KQ, 16384, false);
-            mma_commit(&bar[B_A]);
-            gemm<128, 64, 128, false, true>(tm + T_1, sb + OFF_KQ, 16384, sb + OFF_S, kHeadDim, false);
-            mma_commit(&bar[B_1]);
-        }
 
-        // ---- epilogue a: A (fp32 scratch) and P (K-major tile)
-        if (!wait_bar(B_A, par)) { failed = true; break; }
-        fence_after_sync();
-        {
-            float v[16];
-            tmem_ld16(taddr(tm + T_A, 32 * quarter, col), v);
-            tmem_wait_ld();
-            if (quarter < 2) {  // K K^T rows -> A = strict lower beta_t exp(g_t - g_i) k_t.k_i
-                const int t = 32 * quarter + lane;
-                const float gt = g_s[t], bt = beta_s[t];
+            // ---- epilogue 1: V'^T = V^T - gamma * (K S)^T ; (Q S)^T *= gamma
+            {
+                float v[32];
+                tmem_ld32(tm + lrow + T_1 + tcol, v);
+                tmem_wait_ld();
 #pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    float a4[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int i = col + 4 * k + e;
-                        a4[e] = (i < t && t < n) ? bt * expf(gt - g_s[i]) * v[4 * k + e] : 0.f;
-                    }
-                    *reinterpret_cast<float4 *>(&Ascr[scr(t, col + 4 * k)]) = make_float4(a4[0], a4[1], a4[2], a4[3]);
+                for (int i = 0; i < 32; ++i) {
+                    const int t = tcol + i;
+                    const float x = *(const float *)(sm + OFF_V + kmaj_off(t, j, 64));
+                    v[i] = to_tf32(x - gam_s[t] * v[i]);
                 }
-            } else {  // Q K^T rows -> P = lower exp(g_t - g_i) q_t.k_i
-                const int t = 32 * quarter + lane - 64;
-                const float gt = g_s[t];
+                tmem_st32(tm + lrow + T_V + tcol, v);  // upper half-lanes: u~^T slot, not live yet
+                float w[32];
+                tmem_ld32(tm + lrow + T_1 + 64 + tcol, w);
+                tmem_wait_ld();
 #pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    float p4[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int i = col + 4 * k + e;
-                        p4[e] = (i <= t && t < n) ? expf(gt - g_s[i]) * v[4 * k + e] : 0.f;
-                    }
-                    *reinterpret_cast<float4 *>(sm + OFF_P + kmaj_off(t, col + 4 * k, 64)) =
-                        tf32x4(p4[0], p4[1], p4[2], p4[3]);
-                }
-            }
-        }
-        // ---- epilogue 1: V' = V - gamma * K S (rows 0-63); gamma * Q S in place (rows 64-127)
-        if (!wait_bar(B_1, par)) { failed = true; break; }
-        if (tid == 0 && c + 1 < nchunks) issue_kq(c + 1);  // MMA_a and MMA_1 are done with [K;Q]
-        if (!wait_bar(B_V, par)) { failed = true; break; }
-        fence_after_sync();
-        {
-            float v[16];
-            tmem_ld16(taddr(tm + T_1, 32 * quarter, col), v);
-            tmem_wait_ld();
-            if (quarter < 2) {
-                const int t = 32 * quarter + lane;
-                const float gt = gam_s[t];
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const float4 x = *reinterpret_cast<const float4 *>(sm + OFF_V + kmaj_off(t, col + 4 * k, 64));
-                    v[4 * k] = x.x - gt * v[4 * k];
-                    v[4 * k + 1] = x.y - gt * v[4 * k + 1];
-                    v[4 * k + 2] = x.z - gt * v[4 * k + 2];
-                    v[4 * k + 3] = x.w - gt * v[4 * k + 3];
-                }
-            } else {
-                const float gt = gam_s[32 * quarter + lane - 64];
-#pragma unroll
-                for (int j = 0; j < 16; ++j) v[j] *= gt;
-                tmem_st16(taddr(tm + T_1, 32 * quarter, col), v);
+                for (int i = 0; i < 32; ++i) w[i] *= gam_s[tcol + i];
+                tmem_st32(tm + lrow + T_1 + 64 + tcol, w);  // upper half-lanes: dS^T slot, dead
                 tmem_wait_st();
             }
-            __syncthreads();  // all of V has been read before V' overwrites it
-            if (quarter < 2) {
-                const int t = 32 * quarter + lane;
+            fence_before_sync();
+            group_sync(1);
+            if (tid == 0) {
+                if (c + 1 < nchunks) issue_v(c + 1);  // V of this chunk has been read
+                fence_after_sync();
+                gemm_ts<64, 64, false>(tm + T_U, tm + T_V, sb + OFF_TB + (c & 1) * 16384, 8192, false);
+                mma_commit(&bar[B_2]);
+            }
+            // ---- epilogue 2: u^T rounded in place (operand of MMA_4); u~^T = u^T * kd (upper lanes)
+            if (!wait_all(B_2, par)) { failed = true; break; }
+            fence_after_sync();
+            {
+                float v[32];
+                tmem_ld32(tm + lrow + T_U + tcol, v);
+                tmem_wait_ld();
+                float ut[32];
 #pragma unroll
-                for (int k = 0; k < 4; ++k)
-                    *reinterpret_cast<float4 *>(sm + OFF_V + mn_off(t, col + 4 * k, 64)) =
-                        tf32x4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
+                for (int i = 0; i < 32; ++i) {
+                    const float x = v[i];
+                    v[i] = to_tf32(x);
+                    // the upper thread of each pair takes the scaled copy of the lower thread's row
+                    const float xs = __shfl_xor_sync(0xffffffffu, x, 16);
+                    ut[i] = to_tf32(xs * kd_s[tcol + i]);
+                }
+                tmem_st32(tm + lrow + T_U + tcol, v);   // upper half-lanes unused
+                tmem_st32(tm + lrow + T_V + tcol, ut);  // lower: V'^T (consumed); upper: u~^T
+                tmem_wait_st();
+            }
+            fence_before_sync();
+            if (!wait_all(B_KMN, par)) { failed = true; break; }
+            if (tid == 0) {
+                fence_after_sync();
+                gemm_ts<128, 64, true>(tm + kUpper + T_1, tm + kUpper + T_V, sb + OFF_KMN, 64, false);
+                gemm_ts<64, 64, false>(tm + T_1 + 64, tm + T_U, sb + OFF_P + (c & 1) * 16384, 8192, true);
+                mma_commit(&bar[B_3]);
+            }
+            if (!wait_all(B_3, par)) { failed = true; break; }
+            fence_after_sync();
+            if (tid == 0 && c + 1 < nchunks) issue_kmn(c + 1);
+            // ---- epilogue 3: S^T <- gamma_C S^T + dS^T (upper lanes fp32, lower lanes TF32); y^T out
+            {
+                const float gc = gam_s[n - 1];
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+                    const int d0 = 64 * ch + 32 * half;
+                    float ds[32], s[32];
+                    tmem_ld32(tm + lrow + T_1 + d0, ds);   // upper half-lanes hold dS^T
+                    tmem_ld32(tm + lrow + T_S + d0, s);    // upper half-lanes hold S^T fp32
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        const float sn = fmaf(gc, s[i], ds[i]);           // meaningful on upper lanes
+                        const float from_upper = __shfl_xor_sync(0xffffffffu, sn, 16);
+                        s[i] = upper ? sn : to_tf32(from_upper);
+                    }
+                    tmem_st32(tm + lrow + T_S + d0, s);
+                }
+                float y[32];
+                tmem_ld32(tm + lrow + T_1 + 64 + tcol, y);
+                tmem_wait_ld();
+                tmem_wait_st();
+                if (!upper) {
+                    TO *o = (TO *)p.out + tok * v_row + h * kHeadDim + col0 + j;
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        const int t = tcol + i;
+                        if (t < n) o[(int64_t)t * v_row] = from_f32<TO>(y[i]);
+                    }
+                }
+            }
+            fence_before_sync();
+            group_sync(1);
+        }
+        // ---- final state (upper half-lanes) -> fin;  on failure poison this CTA's outputs
+        if (p.fin) {
+            float *dst = p.fin + ((int64_t)b * p.n_v + h) * kHeadDim * kHeadDim + col0 + j;
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                const int d0 = 64 * ch + 32 * half;
+                float s[32];
+                tmem_ld32(tm + lrow + T_S + d0, s);
+                tmem_wait_ld();
+                if (upper) {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        dst[(int64_t)(d0 + i) * kHeadDim] = failed ? __int_as_float(0x7fc00000) : s[i];
+                }
             }
         }
+        if (failed) {
+            for (int e = tid; e < L * kN; e += kGroup) {
+                const int t = e / kN, jj = e % kN;
+                ((TO *)p.out)[(seq0 + t) * v_row + h * kHeadDim + col0 + jj] =
+                    from_f32<TO>(__int_as_float(0x7fc00000));
+            }
+        }
+    } else {
+        // ================================================================ prep group
+        const int ptid = tid - kGroup;                 // 0..255
+        const int ch = (warp - 8) >> 2;                // which 32 of the 64 columns of [K;Q]K^T
+        const TI *al = (const TI *)p.alpha;
+        const TI *be = (const TI *)p.beta;
+        typedef typename RawT<TI>::type raw_t;
+        raw_t a_raw = 0, b_raw = 0;
+        auto load_gates = [&](int c) {                 // raw bits; converted one chunk later
+            const int n = min(kChunk, L - c * kChunk);
+            const int64_t tok = seq0 + (int64_t)c * kChunk;
+            if (ptid < n) {
+                a_raw = ld_raw(al + (tok + ptid) * p.n_v + h);
+                b_raw = ld_raw(be + (tok + ptid) * p.n_v + h);
+            }
+        };
+        auto wait_all = [&](int i, uint32_t par) -> bool {
+            const bool ok = mbar_wait(&bar[i], par, kWaitTries);
+            return !group_sync_or(2, !ok);
+        };
+        float *Ascr = (float *)(sm + OFF_AS);
+        float *Tscr = (float *)(sm + OFF_TS);
+        float *inv_s = (float *)(sm + OFF_INV);
+        if (nchunks > 0 && ptid < kChunk) load_gates(0);
 
-        // ---- T = (I + A)^-1 (fp32 scratch in OFF_TB): 16 x 16 diagonal blocks by forward
-        // substitution, then the two 32 x 32 halves, then the lower-left 32 x 32 block:
-        //   [[X, 0], [Y, Z]]^-1 = [[X^-1, 0], [-Z^-1 Y X^-1, Z^-1]]
-        if (tid < 64) {  // diagonal blocks: column cc of block bb
-            const int bb = tid >> 4, cc = tid & 15;
-            float x[16];
+        for (int c = 0; c < nchunks; ++c) {
+            const int n = min(kChunk, L - c * kChunk);
+            const uint32_t par = c & 1;
+            float *gate = (float *)(sm + OFF_GATE + (c & 1) * 1024);
+            float *g_s = gate, *gam_s = gate + 64, *beta_s = gate + 128, *kd_s = gate + 192;
+            unsigned char *Pt = sm + OFF_P + (c & 1) * 16384;
+            unsigned char *Tb = sm + OFF_TB + (c & 1) * 16384;
+
+            // ---- gates of chunk c.  [K;Q] of chunk c is issued only after the chain has
+            // finished chunk c-1, so its arrival also frees this gate buffer, P and T_beta.
+            if (!wait_all(B_KQ, par)) { failed = true; break; }
+            if (ptid < kChunk) {
+                g_s[ptid] = ptid < n ? safe_log_alpha(raw_to_f32(a_raw)) : 0.f;
+                beta_s[ptid] = ptid < n ? raw_to_f32(b_raw) : 0.f;
+                if (c + 1 < nchunks) load_gates(c + 1);
+            }
+            group_sync(2);
+            if (ptid < 32) {  // inclusive scan of log alpha, two rows per lane
+                const float a0 = g_s[2 * lane], a1 = g_s[2 * lane + 1];
+                float s = a0 + a1;
 #pragma unroll
-            for (int r = 0; r < 16; ++r) {
-                float a0 = (r == cc) ? 1.f : 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+                for (int o = 1; o < 32; o <<= 1) {
+                    const float y = __shfl_up_sync(0xffffffffu, s, o);
+                    if (lane >= o) s += y;
+                }
+                const float g0 = s - a1;
+                const float glast = __shfl_sync(0xffffffffu, ((n - 1) & 1) ? s : g0, (n - 1) >> 1);
+                g_s[2 * lane] = g0;
+                g_s[2 * lane + 1] = s;
+                gam_s[2 * lane] = expf(g0);
+                gam_s[2 * lane + 1] = expf(s);
+                kd_s[2 * lane] = 2 * lane < n ? expf(glast - g0) : 0.f;
+                kd_s[2 * lane + 1] = 2 * lane + 1 < n ? expf(glast - s) : 0.f;
+            }
+            group_sync(2);
+            if (ptid == 0) {
+                fence_after_sync();
+                gemm<128, 64, 128, false, false>(tm + T_A, sb + OFF_KQ, 16384, sb + OFF_KQ, 16384, false);
+                mma_commit(&bar[B_A]);
+            }
+            // ---- epilogue a: A (fp32 scratch) and P (K-major tile)
+            if (!wait_all(B_A, par)) { failed = true; break; }
+            fence_after_sync();
+            {
+                float v[32];
+                tmem_ld32(taddr(tm + T_A, 32 * quarter, 32 * ch), v);
+                tmem_wait_ld();
+                if (quarter < 2) {  // K K^T rows
+                    const int t = 32 * quarter + lane;
+                    const float gt = g_s[t], bt = beta_s[t];
 #pragma unroll
-                for (int m = 0; m + 3 < r; m += 4) {
-                    const float4 a4 = *reinterpret_cast<const float4 *>(&Ascr[scr(16 * bb + r, 16 * bb + m)]);
-                    a0 = fmaf(-a4.x, x[m], a0);
-                    a1 = fmaf(-a4.y, x[m + 1], a1);
-                    a2 = fmaf(-a4.z, x[m + 2], a2);
-                    a3 = fmaf(-a4.w, x[m + 3], a3);
+                    for (int k = 0; k < 8; ++k) {
+                        float a4[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const int i = 32 * ch + 4 * k + e;
+                            a4[e] = (i < t && t < n) ? bt * expf(gt - g_s[i]) * v[4 * k + e] : 0.f;
+                        }
+                        *reinterpret_cast<float4 *>(&Ascr[scr(t, 32 * ch + 4 * k)]) = make_float4(a4[0], a4[1], a4[2], a4[3]);
+                    }
+                } else {  // Q K^T rows
+                    const int t = 32 * quarter + lane - 64;
+                    const float gt = g_s[t];
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) {
+                        float p4[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const int i = 32 * ch + 4 * k + e;
+                            p4[e] = (i <= t && t < n) ? expf(gt - g_s[i]) * v[4 * k + e] : 0.f;
+                        }
+                        *reinterpret_cast<float4 *>(Pt + kmaj_off(t, 32 * ch + 4 * k, 64)) = tf32x4(p4[0], p4[1], p4[2], p4[3]);
+                    }
+                }
+            }
+            group_sync(2);
+            // ---- T = (I + A)^-1: 16 x 16 diagonal blocks, two 32 x 32 halves, one merge
+            if (ptid < 64) {
+                const int bb = ptid >> 4, cc = ptid & 15;
+                float x[16];
+#pragma unroll
+                for (int r = 0; r < 16; ++r) {
+                    float a0 = (r == cc) ? 1.f : 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+#pragma unroll
+                    for (int m = 0; m + 3 < r; m += 4) {
+                        const float4 a4 = *reinterpret_cast<const float4 *>(&Ascr[scr(16 * bb + r, 16 * bb + m)]);
+                        a0 = fmaf(-a4.x, x[m], a0);
+                        a1 = fmaf(-a4.y, x[m + 1], a1);
+                        a2 = fmaf(-a4.z, x[m + 2], a2);
+                        a3 = fmaf(-a4.w, x[m + 3], a3);
+                    }
+#pragma unroll
+                    for (int m = r & ~3; m < r; ++m) a0 = fmaf(-Ascr[scr(16 * bb + r, 16 * bb + m)], x[m], a0);
+                    x[r] = (r < cc) ? 0.f : (a0 + a1) + (a2 + a3);
                 }
 #pragma unroll
-                for (int m = r & ~3; m < r; ++m) a0 = fmaf(-Ascr[scr(16 * bb + r, 16 * bb + m)], x[m], a0);
-                x[r] = (r < cc) ? 0.f : (a0 + a1) + (a2 + a3);
+                for (int r = 0; r < 16; ++r) Tscr[scr(16 * bb + r, 16 * bb + cc)] = x[r];
+            } else {
+                for (int e = ptid - 64; e < 64 * 64; e += kGroup - 64) {
+                    const int r = e >> 6, cc = e & 63;
+                    if ((r >> 4) < (cc >> 4)) Tscr[scr(r, cc)] = 0.f;
+                }
             }
+            group_sync(2);
+            if (ptid < 128) {  // halves: M = A_10 T_00 (16 x 16 blocks)
+                const int hh = ptid >> 6, rr = (ptid >> 2) & 15, c4 = (ptid & 3) * 4, o = 32 * hh;
+                float a4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int r = 0; r < 16; ++r) Tscr[scr(16 * bb + r, 16 * bb + cc)] = x[r];
-        } else {  // zero the strictly upper part outside the diagonal blocks
-            for (int e = tid - 64; e < 64 * 64; e += kThr - 64) {
-                const int r = e >> 6, cc = e & 63;
-                if ((r >> 4) < (cc >> 4)) Tscr[scr(r, cc)] = 0.f;
+                for (int m = 0; m < 16; ++m) {
+                    const float a = Ascr[scr(o + 16 + rr, o + m)];
+                    const float4 t4 = *reinterpret_cast<const float4 *>(&Tscr[scr(o + m, o + c4)]);
+                    a4[0] = fmaf(a, t4.x, a4[0]); a4[1] = fmaf(a, t4.y, a4[1]);
+                    a4[2] = fmaf(a, t4.z, a4[2]); a4[3] = fmaf(a, t4.w, a4[3]);
+                }
+                *reinterpret_cast<float4 *>(&inv_s[hh * 256 + rr * 16 + c4]) = make_float4(a4[0], a4[1], a4[2], a4[3]);
             }
-        }
-        __syncthreads();
-        // 32 x 32 halves hh = 0, 1 (rows/cols 32hh..32hh+31): T_10 = -T_11 A_10 T_00 in
-        // 16-blocks; then the lower-left 32 x 32 block T_bl = -T_br A_bl T_top.  Each
-        // thread computes a 4-column strip of one row (float4 operand loads).
-        if (tid < 128) {
-            const int hh = tid >> 6, rr = (tid >> 2) & 15, c4 = (tid & 3) * 4, o = 32 * hh;
-            float a4[4] = {0.f, 0.f, 0.f, 0.f};
+            group_sync(2);
+            if (ptid < 128) {  // T_10 = -T_11 M
+                const int hh = ptid >> 6, rr = (ptid >> 2) & 15, c4 = (ptid & 3) * 4, o = 32 * hh;
+                float a4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int m = 0; m < 16; ++m) {
-                const float a = Ascr[scr(o + 16 + rr, o + m)];
-                const float4 t4 = *reinterpret_cast<const float4 *>(&Tscr[scr(o + m, o + c4)]);
-                a4[0] = fmaf(a, t4.x, a4[0]); a4[1] = fmaf(a, t4.y, a4[1]);
-                a4[2] = fmaf(a, t4.z, a4[2]); a4[3] = fmaf(a, t4.w, a4[3]);
+                for (int m = 0; m < 16; ++m) {
+                    const float t = Tscr[scr(o + 16 + rr, o + 16 + m)];
+                    const float4 m4 = *reinterpret_cast<const float4 *>(&inv_s[hh * 256 + m * 16 + c4]);
+                    a4[0] = fmaf(t, m4.x, a4[0]); a4[1] = fmaf(t, m4.y, a4[1]);
+                    a4[2] = fmaf(t, m4.z, a4[2]); a4[3] = fmaf(t, m4.w, a4[3]);
+                }
+                *reinterpret_cast<float4 *>(&Tscr[scr(o + 16 + rr, o + c4)]) = make_float4(-a4[0], -a4[1], -a4[2], -a4[3]);
             }
-            *reinterpret_cast<float4 *>(&inv_s[hh * 256 + rr * 16 + c4]) = make_float4(a4[0], a4[1], a4[2], a4[3]);
-        }
-        __syncthreads();
-        if (tid < 128) {
-            const int hh = tid >> 6, rr = (tid >> 2) & 15, c4 = (tid & 3) * 4, o = 32 * hh;
-            float a4[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-            for (int m = 0; m < 16; ++m) {
-                const float t = Tscr[scr(o + 16 + rr, o + 16 + m)];
-                const float4 m4 = *reinterpret_cast<const float4 *>(&inv_s[hh * 256 + m * 16 + c4]);
-                a4[0] = fmaf(t, m4.x, a4[0]); a4[1] = fmaf(t, m4.y, a4[1]);
-                a4[2] = fmaf(t, m4.z, a4[2]); a4[3] = fmaf(t, m4.w, a4[3]);
+            group_sync(2);
+            {  // merge: M = A_bl T_top into the (zero) upper-right block
+                const int r = ptid >> 3, c4 = (ptid & 7) * 4;
+                float a4[4] = {0.f, 0.f, 0.f, 0.f};
+                for (int m = c4; m < 32; ++m) {
+                    const float a = Ascr[scr(32 + r, m)];
+                    const float4 t4 = *reinterpret_cast<const float4 *>(&Tscr[scr(m, c4)]);
+                    a4[0] = fmaf(a, t4.x, a4[0]); a4[1] = fmaf(a, t4.y, a4[1]);
+                    a4[2] = fmaf(a, t4.z, a4[2]); a4[3] = fmaf(a, t4.w, a4[3]);
+                }
+                *reinterpret_cast<float4 *>(&Tscr[scr(r, 32 + c4)]) = make_float4(a4[0], a4[1], a4[2], a4[3]);
             }
-            *reinterpret_cast<float4 *>(&Tscr[scr(o + 16 + rr, o + c4)]) = make_float4(-a4[0], -a4[1], -a4[2], -a4[3]);
-        }
-        __syncthreads();
-        // M = A_bl T_top, kept in the (zero) upper-right block of T
-        if (tid < 256) {
-            const int r = tid >> 3, c4 = (tid & 7) * 4;
-            float a4[4] = {0.f, 0.f, 0.f, 0.f};
-            for (int m = c4; m < 32; ++m) {  // T_top is lower triangular
-                const float a = Ascr[scr(32 + r, m)];
-                const float4 t4 = *reinterpret_cast<const float4 *>(&Tscr[scr(m, c4)]);
-                a4[0] = fmaf(a, t4.x, a4[0]); a4[1] = fmaf(a, t4.y, a4[1]);
-                a4[2] = fmaf(a, t4.z, a4[2]); a4[3] = fmaf(a, t4.w, a4[3]);
+            group_sync(2);
+            {  // T_bl = -T_br M
+                const int r = ptid >> 3, c4 = (ptid & 7) * 4;
+                float a4[4] = {0.f, 0.f, 0.f, 0.f};
+                for (int m = 0; m <= r; ++m) {
+                    const float t = Tscr[scr(32 + r, 32 + m)];
+                    const float4 m4 = *reinterpret_cast<const float4 *>(&Tscr[scr(m, 32 + c4)]);
+                    a4[0] = fmaf(t, m4.x, a4[0]); a4[1] = fmaf(t, m4.y, a4[1]);
+                    a4[2] = fmaf(t, m4.z, a4[2]); a4[3] = fmaf(t, m4.w, a4[3]);
+                }
+                *reinterpret_cast<float4 *>(&Tscr[scr(32 + r, c4)]) = make_float4(-a4[0], -a4[1], -a4[2], -a4[3]);
             }
-            *reinterpret_cast<float4 *>(&Tscr[scr(r, 32 + c4)]) = make_float4(a4[0], a4[1], a4[2], a4[3]);
-        }
-        __syncthreads();
-        // T_bl = -T_br M
-        if (tid < 256) {
-            const int r = tid >> 3, c4 = (tid & 7) * 4;
-            float a4[4] = {0.f, 0.f, 0.f, 0.f};
-            for (int m = 0; m <= r; ++m) {  // T_br is lower triangular
-                const float t = Tscr[scr(32 + r, 32 + m)];
-                const float4 m4 = *reinterpret_cast<const float4 *>(&Tscr[scr(m, 32 + c4)]);
-                a4[0] = fmaf(t, m4.x, a4[0]); a4[1] = fmaf(t, m4.y, a4[1]);
-                a4[2] = fmaf(t, m4.z, a4[2]); a4[3] = fmaf(t, m4.w, a4[3]);
-            }
-            *reinterpret_cast<float4 *>(&Tscr[scr(32 + r, c4)]) = make_float4(-a4[0], -a4[1], -a4[2], -a4[3]);
-        }
-        __syncthreads();
-        // T_beta = T diag(beta), rewritten in place as a K-major tile
-        {
-            const int t = tid >> 3, i0 = (tid & 7) * 8;
-            const bool upper_right = t < 32 && i0 >= 32;  // zero in T; held the merge product
-            float tv[8];
-#pragma unroll
-            for (int k = 0; k < 2; ++k) {
-                float4 x = *reinterpret_cast<const float4 *>(&Tscr[scr(t, i0 + 4 * k)]);
-                if (upper_right) x = make_float4(0.f, 0.f, 0.f, 0.f);
-                tv[4 * k] = x.x * beta_s[i0 + 4 * k];
-                tv[4 * k + 1] = x.y * beta_s[i0 + 4 * k + 1];
-                tv[4 * k + 2] = x.z * beta_s[i0 + 4 * k + 2];
-                tv[4 * k + 3] = x.w * beta_s[i0 + 4 * k + 3];
-            }
-            __syncthreads();
-#pragma unroll
-            for (int k = 0; k < 2; ++k)
-                *reinterpret_cast<float4 *>(sm + OFF_TB + kmaj_off(t, i0 + 4 * k, 64)) =
-                    tf32x4(tv[4 * k], tv[4 * k + 1], tv[4 * k + 2], tv[4 * k + 3]);
-        }
-        fence_smem_to_async();
-        fence_before_sync();
-        __syncthreads();
-
-        // ---- MMA_2: u = T_beta V'
-        if (tid == 0) {
-            fence_after_sync();
-            gemm<64, 64, 64, false, true>(tm + T_U, sb + OFF_TB, 8192, sb + OFF_V, 64, false);
-            mma_commit(&bar[B_2]);
-        }
-        if (!wait_bar(B_2, par)) { failed = true; break; }
-        fence_after_sync();
-        if (tid == 0 && c + 1 < nchunks) issue_v(c + 1);  // V' consumed
-        {
-            float v[16];
-            tmem_ld16(taddr(tm + T_U, 32 * quarter, col), v);
-            tmem_wait_ld();
-            if (lane < 16) {  // M=64 layout: row t at lane 16*quarter + l of quarter `quarter`
-                const int t = 16 * quarter + lane;
-                const float kd = kd_s[t];
+            group_sync(2);
+            {  // T_beta = T diag(beta) as a K-major tile (the upper-right block is zero)
+                const int t = ptid >> 2, i0 = (ptid & 3) * 16;
+                const bool upper_right = t < 32 && i0 >= 32;
 #pragma unroll
                 for (int k = 0; k < 4; ++k) {
-                    *reinterpret_cast<float4 *>(sm + OFF_U + mn_off(t, col + 4 * k, 64)) =
-                        tf32x4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
-                    *reinterpret_cast<float4 *>(sm + OFF_TB + mn_off(t, col + 4 * k, 64)) =
-                        tf32x4(kd * v[4 * k], kd * v[4 * k + 1], kd * v[4 * k + 2], kd * v[4 * k + 3]);
+                    float4 x = *reinterpret_cast<const float4 *>(&Tscr[scr(t, i0 + 4 * k)]);
+                    if (upper_right) x = make_float4(0.f, 0.f, 0.f, 0.f);
+                    *reinterpret_cast<float4 *>(Tb + kmaj_off(t, i0 + 4 * k, 64)) =
+                        tf32x4(x.x * beta_s[i0 + 4 * k], x.y * beta_s[i0 + 4 * k + 1],
+                               x.z * beta_s[i0 + 4 * k + 2], x.w * beta_s[i0 + 4 * k + 3]);
                 }
             }
+            fence_smem_to_async();  // P and T_beta are read by the chain's MMAs
+            group_sync(2);
+            if (ptid == 0) {
+                asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(&bar[B_PREP])) : "memory");
+            }
         }
-        fence_smem_to_async();
-        if (!wait_bar(B_KMN, par)) { failed = true; break; }
-        fence_before_sync();
-        __syncthreads();
-
-        // ---- MMA_3: dS = K^T u~ ; MMA_4: y = gamma QS + P u (128-row view of P)
-        if (tid == 0) {
-            fence_after_sync();
-            gemm<128, 64, 64, true, true>(tm + T_DS, sb + OFF_KMN, 64, sb + OFF_TB, 64, false);
-            gemm<128, 64, 64, false, true>(tm + T_1, sb + OFF_P - 8192, 8192, sb + OFF_U, 64, true);
-            mma_commit(&bar[B_3]);
-        }
-        if (!wait_bar(B_3, par)) { failed = true; break; }
-        fence_after_sync();
-        if (tid == 0 && c + 1 < nchunks) issue_kmn(c + 1);  // K (token-major copy) consumed
-        {
-            float v[16];
-            tmem_ld16(taddr(tm + T_DS, 32 * quarter, col), v);
-            tmem_wait_ld();
-            const float gc = gam_s[n - 1];
-#pragma unroll
-            for (int j = 0; j < 16; ++j) S[j] = fmaf(gc, S[j], v[j]);
-#pragma unroll
-            for (int k = 0; k < 4; ++k)
-                *reinterpret_cast<float4 *>(sm + OFF_S + mn_off(d_own, col + 4 * k, kHeadDim)) =
-                    tf32x4(S[4 * k], S[4 * k + 1], S[4 * k + 2], S[4 * k + 3]);
-            float y[16];
-            tmem_ld16(taddr(tm + T_1, 32 * quarter, col), y);
-            tmem_wait_ld();
-            const int t = 32 * quarter + lane - 64;
-            if (quarter >= 2 && t < n) store_row16<TO>(out + (tok + t) * v_row + h * kHeadDim + col0 + col, y);
-        }
-        fence_before_sync();
-        __syncthreads();
     }
 
     // ---------------------------------------------------------------- tear-down
-    if (p.fin) {
-        if (failed) {
-#pragma unroll
-            for (int j = 0; j < 16; ++j) S[j] = __int_as_float(0x7fc00000);
-        }
-#pragma unroll
-        for (int k = 0; k < 4; ++k)
-            *reinterpret_cast<float4 *>(p.fin + st_off + 4 * k) = make_float4(S[4 * k], S[4 * k + 1], S[4 * k + 2], S[4 * k + 3]);
-    }
-    if (failed) {  // a wait gave up: poison this CTA's outputs
-        for (int e = tid; e < L * kN; e += kThr) {
-            const int t = e / kN, j = e % kN;
-            out[(seq0 + t) * v_row + h * kHeadDim + col0 + j] = from_f32<TO>(__int_as_float(0x7fc00000));
-        }
-    }
     fence_before_sync();
     __syncthreads();
     if (warp == 0) tmem_dealloc(tm, kTmemCols);
