@@ -128,6 +128,18 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *m, uint32_t parity) {
         : "memory");
     return ok != 0;
 }
+// Same, but the thread may sleep up to `hint_ns` nanoseconds inside the poll instead of
+// returning at once, so that waiting warps leave the issue slots to the working ones.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t *m, uint32_t parity, uint32_t hint_ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(ok)
+        : "r"(smem_u32(m)), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return ok != 0;
+}
 // Bounded wait on phase `parity`: returns false if it has not completed after
 // `max_tries` polls (each poll itself blocks for a hardware-defined short time).
 __device__ __forceinline__ bool mbar_wait(uint64_t *m, uint32_t parity, uint32_t max_tries) {
