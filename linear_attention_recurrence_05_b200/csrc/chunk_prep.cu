@@ -1,0 +1,289 @@
+// State-independent work of the chunked prefill, for every (chunk, V head) at once.
+//
+// For a chunk of n <= 64 tokens of one sequence and one V head h (QK head g = h / (Hv/Hqk)),
+// following the chunked form of the gated delta rule of the page "ARCHITECTURE PREVIEW /
+// FIELD NOTES", section 03 (GATED DELTANET), with g_t = sum_{s<=t} log alpha_s inside the chunk:
+//     A_ti = beta_t exp(g_t - g_i) k_t.k_i        (i < t < n, else 0)
+//     T    = (I + A)^-1,   T_beta = T diag(beta)   (unit lower triangular solve)
+//     P_ti = exp(g_t - g_i) q_t.k_i               (i <= t < n, else 0)
+// T_beta and P are written as 64 x 64 fp32 tiles (row t, column i; values rounded to TF32,
+// the precision the tensor-core chain reads them in) for the chain kernel to stream in.
+// Rows and columns at or past n are zero, so a partial chunk needs no masking downstream.
+//
+// One CTA per (chunk, V head), 256 threads: TMA brings the chunk's K and Q rows, one
+// tcgen05 MMA forms [K;Q] K^T in tensor memory, the warps turn it into A and P, and the
+// inverse runs on CUDA cores in fp32: 16 x 16 diagonal blocks by forward substitution,
+// then two block-merge levels (16 -> 32 -> 64).
+#include "gdn_common.cuh"
+#include "gdn_internal.h"
+#include "tc_sm100.cuh"
+#include "tma_map.cuh"
+
+namespace gdn {
+
+namespace {
+using namespace tc;
+
+constexpr int kPThr = 256;
+
+// shared-memory map (bytes from a 1024-aligned base)
+constexpr uint32_t P_KQ = 0;          // [K;Q] K-major, 4 blocks x (K 8 KB | Q 8 KB)   64 KB
+constexpr uint32_t P_AS = 65536;      // A (fp32, swizzled rows)                       16 KB
+constexpr uint32_t P_TS = 81920;      // T (fp32, swizzled rows)                       16 KB
+constexpr uint32_t P_INV = 98304;     // 2 x 256 floats (block products)                2 KB
+constexpr uint32_t P_GATE = 100352;   // g[64], beta[64]                               512 B
+constexpr uint32_t P_BAR = 100864;    // 2 mbarriers
+constexpr uint32_t P_SLOT = 100880;   // TMEM base
+constexpr uint32_t kPSmem = P_SLOT + 16;
+constexpr uint32_t kPSmemAlloc = kPSmem + 1024;
+constexpr uint32_t kPTmemCols = 64;
+constexpr uint32_t kPWaitTries = 1u << 24;
+
+// fp32 scratch [64][64] with 16-byte chunks XOR-swizzled by row
+__device__ __forceinline__ int scr(int r, int c) { return r * 64 + ((((c >> 2) ^ (r & 7)) << 2) | (c & 3)); }
+
+__device__ __forceinline__ float4 tf32x4(float4 x) {
+    return make_float4(to_tf32(x.x), to_tf32(x.y), to_tf32(x.z), to_tf32(x.w));
+}
+
+struct PrepParams {
+    CUtensorMap tm_k;     // k^ rows, K-major 128B swizzle boxes (32 x 64)
+    CUtensorMap tm_q;     // q^ rows, same
+    const void *alpha, *beta;
+    const int32_t *cu, *cfirst;
+    float *tb, *pm;       // [chunk, Hv, 64, 64]
+    int n_seqs, n_qk, n_v;
+};
+
+}  // namespace
+
+template <class TI>
+__global__ void __launch_bounds__(kPThr) chunk_prep_kernel(const __grid_constant__ PrepParams p) {
+    const int h = blockIdx.x % p.n_v;
+    const int u = blockIdx.x / p.n_v;                  // global chunk index
+    if (u >= p.cfirst[p.n_seqs]) return;               // uniform per CTA
+    const int b = upper_index(p.cfirst, p.n_seqs, u);
+    const int seq0 = p.cu[b];
+    const int r0 = (u - p.cfirst[b]) * kChunk;
+    const int n = min(kChunk, p.cu[b + 1] - seq0 - r0);
+    const int tok = seq0 + r0;
+    const int gq = h / (p.n_v / p.n_qk);
+
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char *sm = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
+    const uint32_t sb = smem_u32(sm);
+    uint64_t *bar = (uint64_t *)(sm + P_BAR);
+    uint32_t *tslot = (uint32_t *)(sm + P_SLOT);
+    float *g_s = (float *)(sm + P_GATE), *beta_s = g_s + 64;
+    float *Ascr = (float *)(sm + P_AS), *Tscr = (float *)(sm + P_TS), *inv_s = (float *)(sm + P_INV);
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    float *tb = p.tb + ((int64_t)u * p.n_v + h) * (kChunk * kChunk);
+    float *pm = p.pm + ((int64_t)u * p.n_v + h) * (kChunk * kChunk);
+
+    if (tid == 0) {
+        mbar_init(&bar[0], 1);
+        mbar_init(&bar[1], 1);
+        mbar_expect_tx(&bar[0], 65536);
+#pragma unroll
+        for (int kb = 0; kb < 4; ++kb) {
+            tma_load_2d(sb + P_KQ + kb * 16384, &p.tm_k, gq * kHeadDim + 32 * kb, tok, &bar[0]);
+            tma_load_2d(sb + P_KQ + kb * 16384 + 8192, &p.tm_q, gq * kHeadDim + 32 * kb, tok, &bar[0]);
+        }
+    }
+    if (warp == 0) {
+        tmem_alloc(tslot, kPTmemCols);
+        tmem_relinquish();
+    }
+    // gates of the chunk: log alpha and beta, zero past n
+    if (tid < kChunk) {
+        const TI *al = (const TI *)p.alpha, *be = (const TI *)p.beta;
+        const int64_t e = (int64_t)(tok + tid) * p.n_v + h;
+        g_s[tid] = tid < n ? safe_log_alpha(to_f32(al[e])) : 0.f;
+        beta_s[tid] = tid < n ? to_f32(be[e]) : 0.f;
+    }
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    const uint32_t tm = *tslot;
+
+    // [K;Q] K^T (M=128: rows 0-63 K K^T, rows 64-127 Q K^T; N=64) into tensor memory
+    bool ok = true;
+    if (tid == 0) {
+        ok = mbar_wait(&bar[0], 0, kPWaitTries);
+        if (ok) {
+            fence_after_sync();
+            gemm<128, 64, 128, false, false>(tm, sb + P_KQ, 16384, sb + P_KQ, 16384, false);
+            mma_commit(&bar[1]);
+        }
+    }
+    if (warp == 1) {  // inclusive scan of log alpha, two rows per lane (meanwhile)
+        const int t0 = 2 * lane, t1 = t0 + 1;
+        const float a0 = g_s[t0], a1 = g_s[t1];
+        float s = a0 + a1;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const float y = __shfl_up_sync(0xffffffffu, s, o);
+            if (lane >= o) s += y;
+        }
+        g_s[t0] = s - a1;
+        g_s[t1] = s;
+    }
+    if (__syncthreads_or(!ok)) {
+        if (tid == 0) mbar_wait(&bar[0], 0, kPWaitTries);  // drain the copies
+        ok = false;
+    } else {
+        ok = mbar_wait(&bar[1], 0, kPWaitTries);
+        ok = !__syncthreads_or(!ok);
+    }
+    fence_after_sync();
+    if (ok) {
+        // A (fp32 scratch) from the K K^T rows, P (TF32, global tile) from the Q K^T rows
+        const int q = warp & 3, ch = warp >> 2;
+        float v[32];
+        tmem_ld32(taddr(tm, 32 * q, 32 * ch), v);
+        tmem_wait_ld();
+        const int t = 32 * (q & 1) + lane;
+        const float gt = g_s[t], bt = beta_s[t];
+        if (q < 2) {
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                float a4[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int i = 32 * ch + 4 * k + e;
+                    a4[e] = (i < t && t < n) ? bt * expf(gt - g_s[i]) * v[4 * k + e] : 0.f;
+                }
+                *reinterpret_cast<float4 *>(&Ascr[scr(t, 32 * ch + 4 * k)]) = make_float4(a4[0], a4[1], a4[2], a4[3]);
+            }
+        } else {
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                float p4[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int i = 32 * ch + 4 * k + e;
+                    p4[e] = (i <= t && t < n) ? expf(gt - g_s[i]) * v[4 * k + e] : 0.f;
+                }
+                *reinterpret_cast<float4 *>(pm + t * 64 + 32 * ch + 4 * k) =
+                    tf32x4(make_float4(p4[0], p4[1], p4[2], p4[3]));
+            }
+        }
+    }
+    fence_before_sync();
+    __syncthreads();
+    if (ok) {
+        // ---- T = (I + A)^-1.  Diagonal 16 x 16 blocks: column cc of block bb by forward
+        // substitution with right-looking updates; the other threads clear the two blocks
+        // above the diagonal that the merge products read.
+        if (tid < 64) {
+            const int bb = tid >> 4, cc = tid & 15, o = 16 * bb;
+            float x[16];
+#pragma unroll
+            for (int r = 0; r < 16; ++r) x[r] = (r == cc) ? 1.f : 0.f;
+#pragma unroll
+            for (int m = 0; m < 15; ++m) {
+                const float xm = x[m];
+#pragma unroll
+                for (int r = m + 1; r < 16; ++r) x[r] = fmaf(-Ascr[scr(o + r, o + m)], xm, x[r]);
+            }
+#pragma unroll
+            for (int r = 0; r < 16; ++r) Tscr[scr(o + r, o + cc)] = x[r];
+        } else {
+            for (int e = tid - 64; e < 512; e += kPThr - 64) {
+                const int blk = e >> 8, r = (e >> 4) & 15, cc = e & 15, o = 32 * blk;
+                Tscr[scr(o + r, o + 16 + cc)] = 0.f;
+            }
+        }
+        __syncthreads();
+        if (tid < 128) {  // 32 x 32 halves: M = A_10 T_00
+            const int hh = tid >> 6, rr = (tid >> 2) & 15, c4 = (tid & 3) * 4, o = 32 * hh;
+            float a4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int m = 0; m < 16; ++m) {
+                const float a = Ascr[scr(o + 16 + rr, o + m)];
+                const float4 t4 = *reinterpret_cast<const float4 *>(&Tscr[scr(o + m, o + c4)]);
+                a4[0] = fmaf(a, t4.x, a4[0]); a4[1] = fmaf(a, t4.y, a4[1]);
+                a4[2] = fmaf(a, t4.z, a4[2]); a4[3] = fmaf(a, t4.w, a4[3]);
+            }
+            *reinterpret_cast<float4 *>(&inv_s[hh * 256 + rr * 16 + c4]) = make_float4(a4[0], a4[1], a4[2], a4[3]);
+        }
+        __syncthreads();
+        if (tid < 128) {  // T_10 = -T_11 M
+            const int hh = tid >> 6, rr = (tid >> 2) & 15, c4 = (tid & 3) * 4, o = 32 * hh;
+            float a4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int m = 0; m < 16; ++m) {
+                const float t = Tscr[scr(o + 16 + rr, o + 16 + m)];
+                const float4 m4 = *reinterpret_cast<const float4 *>(&inv_s[hh * 256 + m * 16 + c4]);
+                a4[0] = fmaf(t, m4.x, a4[0]); a4[1] = fmaf(t, m4.y, a4[1]);
+                a4[2] = fmaf(t, m4.z, a4[2]); a4[3] = fmaf(t, m4.w, a4[3]);
+            }
+            *reinterpret_cast<float4 *>(&Tscr[scr(o + 16 + rr, o + c4)]) = make_float4(-a4[0], -a4[1], -a4[2], -a4[3]);
+        }
+        __syncthreads();
+        {  // merge: M = A_bl T_top, parked in the (otherwise unused) upper-right block
+            const int r = tid >> 3, c4 = (tid & 7) * 4;
+            float a4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int m = 0; m < 32; ++m) {
+                const float a = Ascr[scr(32 + r, m)];
+                const float4 t4 = *reinterpret_cast<const float4 *>(&Tscr[scr(m, c4)]);
+                a4[0] = fmaf(a, t4.x, a4[0]); a4[1] = fmaf(a, t4.y, a4[1]);
+                a4[2] = fmaf(a, t4.z, a4[2]); a4[3] = fmaf(a, t4.w, a4[3]);
+            }
+            *reinterpret_cast<float4 *>(&Tscr[scr(r, 32 + c4)]) = make_float4(a4[0], a4[1], a4[2], a4[3]);
+        }
+        __syncthreads();
+        {  // T_bl = -T_br M
+            const int r = tid >> 3, c4 = (tid & 7) * 4;
+            float a4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int m = 0; m < 32; ++m) {
+                const float t = Tscr[scr(32 + r, 32 + m)];
+                const float4 m4 = *reinterpret_cast<const float4 *>(&Tscr[scr(m, 32 + c4)]);
+                a4[0] = fmaf(t, m4.x, a4[0]); a4[1] = fmaf(t, m4.y, a4[1]);
+                a4[2] = fmaf(t, m4.z, a4[2]); a4[3] = fmaf(t, m4.w, a4[3]);
+            }
+            *reinterpret_cast<float4 *>(&Tscr[scr(32 + r, c4)]) = make_float4(-a4[0], -a4[1], -a4[2], -a4[3]);
+        }
+        __syncthreads();
+    }
+    {  // T_beta = T diag(beta) as TF32 (the upper-right block is zero); NaN if the CTA failed
+        const int t = tid >> 2, i0 = (tid & 3) * 16;
+        const bool upper_right = t < 32 && i0 >= 32;
+        const float nan = __int_as_float(0x7fc00000);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const int i = i0 + 4 * k;
+            float4 x = *reinterpret_cast<const float4 *>(&Tscr[scr(t, i)]);
+            if (upper_right) x = make_float4(0.f, 0.f, 0.f, 0.f);
+            x = make_float4(x.x * beta_s[i], x.y * beta_s[i + 1], x.z * beta_s[i + 2], x.w * beta_s[i + 3]);
+            if (!ok) x = make_float4(nan, nan, nan, nan);
+            *reinterpret_cast<float4 *>(tb + t * 64 + i) = tf32x4(x);
+        }
+    }
+    fence_before_sync();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tm, kPTmemCols);
+}
+
+cudaError_t launch_chunk_prep(const ScanParams &sp, int64_t total_tokens, bool in_bf16, cudaStream_t s) {
+    if (sp.n_seqs <= 0 || total_tokens <= 0) return cudaSuccess;
+    PrepParams p{};
+    const int64_t wqk = (int64_t)sp.n_qk * kHeadDim;
+    if (!encode_rows(&p.tm_k, sp.kh, wqk, total_tokens, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !encode_rows(&p.tm_q, sp.qh, wqk, total_tokens, CU_TENSOR_MAP_SWIZZLE_128B))
+        return cudaErrorInvalidValue;
+    p.alpha = sp.alpha; p.beta = sp.beta; p.cu = sp.cu; p.cfirst = sp.cfirst;
+    p.tb = sp.tb; p.pm = sp.pm; p.n_seqs = sp.n_seqs; p.n_qk = sp.n_qk; p.n_v = sp.n_v;
+    const int64_t grid = sp.max_chunks * sp.n_v;
+    if (grid >= ((int64_t)1 << 31)) return cudaErrorInvalidValue;
+    auto k = in_bf16 ? chunk_prep_kernel<bf16> : chunk_prep_kernel<float>;
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kPSmemAlloc);
+    if (e != cudaSuccess) return e;
+    TraceLaunch tl(s, "chunk_prep");
+    k<<<(unsigned)grid, kPThr, kPSmemAlloc, s>>>(p);
+    return cudaGetLastError();
+}
+
+}  // namespace gdn

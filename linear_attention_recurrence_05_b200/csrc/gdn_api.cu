@@ -35,7 +35,7 @@ TraceLaunch::~TraceLaunch() {
 
 static size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-PrefillLayout prefill_layout(int n_qk, int n_v, int64_t T, int n_seqs) {
+PrefillLayout prefill_layout(int n_qk, int n_v, int64_t T, int n_seqs, bool tc) {
     PrefillLayout L{};
     L.max_chunks = (T + kChunk - 1) / kChunk + n_seqs;
     size_t off = 0;
@@ -46,6 +46,9 @@ PrefillLayout prefill_layout(int n_qk, int n_v, int64_t T, int n_seqs) {
     L.off_qh = off;      off = align_up(off + qk_bytes, 256);
     L.off_kh = off;      off = align_up(off + qk_bytes, 256);
     L.off_vh = off;      off = align_up(off + v_bytes, 256);
+    const size_t tile_bytes = tc && T > 0 ? (size_t)L.max_chunks * n_v * 64 * 64 * sizeof(float) : 0;
+    L.off_tb = off;      off = align_up(off + tile_bytes, 256);
+    L.off_pm = off;      off = align_up(off + tile_bytes, 256);
     L.bytes = off;
     return L;
 }
@@ -125,7 +128,8 @@ gdn_status gdn_prefill_workspace_size(const gdn_config *cfg, gdn_dtype dtype, in
     if (st != GDN_OK) return st;
     if (!bytes || total_tokens < 0 || total_tokens >= ((int64_t)1 << 31) || n_seqs < 0)
         return GDN_ERR_INVALID_ARG;
-    *bytes = prefill_layout(cfg->n_qk_heads, cfg->n_v_heads, total_tokens, n_seqs).bytes;
+    *bytes = prefill_layout(cfg->n_qk_heads, cfg->n_v_heads, total_tokens, n_seqs,
+                            dtype == GDN_BF16).bytes;
     return GDN_OK;
 }
 
@@ -160,7 +164,8 @@ gdn_status gdn_prefill(const gdn_config *cfg, gdn_dtype dtype, gdn_dtype out_dty
     if ((conv_state_in && !aligned(conv_state_in, 16)) ||
         (conv_state_out && !aligned(conv_state_out, 16)))
         return GDN_ERR_INVALID_ARG;
-    const PrefillLayout L = prefill_layout(cfg->n_qk_heads, cfg->n_v_heads, total_tokens, n_seqs);
+    const PrefillLayout L = prefill_layout(cfg->n_qk_heads, cfg->n_v_heads, total_tokens, n_seqs,
+                                           dtype == GDN_BF16);
     if (!workspace || !aligned(workspace, 256) || workspace_bytes < L.bytes) return GDN_ERR_WORKSPACE;
     st = check_device();
     if (st != GDN_OK) return st;
@@ -194,11 +199,20 @@ gdn_status gdn_prefill(const gdn_config *cfg, gdn_dtype dtype, gdn_dtype out_dty
     ScanParams sp{};
     sp.qh = (const float *)(ws + L.off_qh); sp.kh = (const float *)(ws + L.off_kh);
     sp.vh = (const float *)(ws + L.off_vh);
-    sp.alpha = alpha; sp.beta = beta; sp.cu = cu;
+    sp.alpha = alpha; sp.beta = beta; sp.cu = cu; sp.cfirst = cfirst;
+    sp.tb = (float *)(ws + L.off_tb); sp.pm = (float *)(ws + L.off_pm); sp.max_chunks = L.max_chunks;
     sp.init = initial_state; sp.fin = final_state; sp.out = out;
     sp.n_seqs = n_seqs; sp.n_qk = cfg->n_qk_heads; sp.n_v = cfg->n_v_heads;
-    e = bf ? launch_prefill_tc(sp, total_tokens, bf, out_dtype == GDN_BF16, stream)
-           : launch_scan_simt(sp, bf, out_dtype == GDN_BF16, stream);
+    if (bf) {
+        // state-independent chunk work for every (chunk, V head) at once, then the chunk chain
+        if (total_tokens > 0) {
+            e = launch_chunk_prep(sp, total_tokens, bf, stream);
+            if (e != cudaSuccess) return cuda_fail(e);
+        }
+        e = launch_prefill_tc(sp, total_tokens, bf, out_dtype == GDN_BF16, stream);
+    } else {
+        e = launch_scan_simt(sp, bf, out_dtype == GDN_BF16, stream);
+    }
     if (e != cudaSuccess) return cuda_fail(e);
     return GDN_OK;
 }

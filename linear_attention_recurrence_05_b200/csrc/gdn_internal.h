@@ -25,10 +25,12 @@ struct PrefillLayout {
     size_t off_qh;        // [T, Hqk, 128] fp32 conv + L2 output
     size_t off_kh;        // [T, Hqk, 128]
     size_t off_vh;        // [T, Hv, 128]
+    size_t off_tb;        // tensor-core path: [max_chunks, Hv, 64, 64] fp32 T diag(beta) tiles
+    size_t off_pm;        // tensor-core path: [max_chunks, Hv, 64, 64] fp32 P tiles
     size_t bytes;
 };
 
-PrefillLayout prefill_layout(int n_qk, int n_v, int64_t T, int n_seqs);
+PrefillLayout prefill_layout(int n_qk, int n_v, int64_t T, int n_seqs, bool tc);
 
 struct ConvParams {
     const void *q, *k, *v;                 // raw rows
@@ -44,6 +46,9 @@ struct ScanParams {
     const float *qh, *kh, *vh;             // fp32 conv + L2 rows [T, H, 128]
     const void *alpha, *beta;              // [T, Hv]
     const int32_t *cu;                     // clamped bounds [n_seqs+1]
+    const int32_t *cfirst;                 // first chunk index of each sequence [n_seqs+1]
+    float *tb, *pm;                        // chunk-prep tiles (tensor-core path)
+    int64_t max_chunks;
     const float *init;                     // [n_seqs, Hv, 128, 128] or null
     float *fin;                            // or null
     void *out;                             // [T, Hv, 128]
@@ -74,6 +79,7 @@ cudaError_t launch_conv_state_out(const void *q, const void *k, const void *v,
                                   const void *conv_in, void *conv_out, const int32_t *cu,
                                   int n_seqs, int n_qk, int n_v, bool bf16, cudaStream_t s);
 cudaError_t launch_scan_simt(const ScanParams &p, bool in_bf16, bool out_bf16, cudaStream_t s);
+cudaError_t launch_chunk_prep(const ScanParams &p, int64_t total_tokens, bool in_bf16, cudaStream_t s);
 cudaError_t launch_prefill_tc(const ScanParams &p, int64_t total_tokens, bool in_bf16, bool out_bf16,
                               cudaStream_t s);
 cudaError_t launch_decode(const DecodeParams &p, bool in_bf16, bool out_bf16, cudaStream_t s);

@@ -16,28 +16,29 @@
 //     y   = G diag(gamma) (Q S~) + P u,   P_ti = exp(g_t - g_i) q_t.k_i (i <= t)
 //     S~ += K~^T u,                       K~ = diag(exp(g_C - g) / G') K
 //
-// One CTA owns one (sequence, V head); all MMAs are M = 128 with the d_v index on the
-// 128 tensor-memory lanes (transposed form), so every state-dependent A operand is read
-// straight from tensor memory:
+// T_beta and P of every chunk come from the chunk-prep pass (64 x 64 TF32 tiles in the
+// workspace).  One CTA owns one (sequence, V head); all MMAs are M = 128 with the d_v
+// index on the 128 tensor-memory lanes (transposed form), so every state-dependent A
+// operand is read straight from tensor memory:
 //   issuer (warp 0, one thread), per chunk
 //     MMA_1   [X | Y1] = S~^T [K;Q]^T           (N=128, K=128)   X = (K S~)^T, Y1 = (Q S~)^T
 //     MMA_2a  U^T      = V^T T_beta^T           (N=64,  K=64)    V from shared memory
 //     MMA_2b  U^T     -= X W2^T                 (N=64,  K=64)    -> u^T
 //     MMA_3   S~^T    += u^T K~                 (N=128, K=64)
 //     MMA_4   Y       += u^T P^T                (N=64,  K=64)    onto Y = G gamma Y1
-//   prep (warps 5-12), the state-independent work of the same chunk, ahead of the issuer:
-//     gates and their scan, MMA_a = [K;Q] K^T (M=128, N=64, K=128), A and P, the 64 x 64
-//     unit-lower-triangular inverse on CUDA cores, T_beta, W2, K~
+//   scale (warps 5-12), ahead of the issuer: the gates and their scan, G, W2 from T_beta,
+//     K~ from K (in place)
 //   epilogue (warps 1-4): Y = G gamma Y1 into tensor memory for MMA_4, y to global memory,
 //     the occasional rescale of S~, the initial and final state.
-// Shared memory holds the K/Q, K (token-major view) and V tiles (TMA, no multicast) and
-// the prep outputs; all waits are bounded and a timed-out CTA writes NaN to its outputs.
+// Shared memory holds the K/Q, K (token-major view), V, T_beta and P tiles (TMA, no
+// multicast) and W2; all waits are bounded and a timed-out CTA writes NaN to its outputs.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
 #include "gdn_common.cuh"
 #include "gdn_internal.h"
 #include "tc_sm100.cuh"
+#include "tma_map.cuh"
 
 namespace gdn {
 
@@ -46,7 +47,7 @@ using namespace tc;
 
 constexpr int kThr = 416;          // 13 warps
 constexpr int kEpiWarp0 = 1;       // warps 1-4
-constexpr int kPrepWarp0 = 5;      // warps 5-12
+constexpr int kPrepWarp0 = 5;      // warps 5-12 (scale role)
 constexpr int kPrepTid0 = kPrepWarp0 * 32;
 constexpr int kEpiTid0 = kEpiWarp0 * 32;
 constexpr int kBarPrep = 1, kBarEpi = 2;  // named barriers
@@ -55,21 +56,18 @@ constexpr int kBarPrep = 1, kBarEpi = 2;  // named barriers
 constexpr uint32_t OFF_KQ = 0;          // [K;Q]   K-major, 4 blocks x (K 8 KB | Q 8 KB)       64 KB
 constexpr uint32_t OFF_KMN = 65536;     // K~      MN-major (32-byte granules), 64 x 128       32 KB
 constexpr uint32_t OFF_VMN = 98304;     // V       MN-major (32-byte granules), 64 x 128       32 KB
-constexpr uint32_t OFF_TB = 131072;     // T_beta  K-major [t][i]                              16 KB
-constexpr uint32_t OFF_W2 = 147456;     // W2      K-major [t][i]                              16 KB
-constexpr uint32_t OFF_P = 163840;      // P       K-major [t][i]                              16 KB
-constexpr uint32_t OFF_AS = 180224;     // A scratch (fp32, swizzled rows)                     16 KB
-constexpr uint32_t OFF_TS = 196608;     // T scratch (fp32, swizzled rows)                     16 KB
+constexpr uint32_t OFF_TB = 131072;     // T_beta  K-major [t][i], 2 buffers                   32 KB
+constexpr uint32_t OFF_P = 163840;      // P       K-major [t][i], 2 buffers                   32 KB
+constexpr uint32_t OFF_W2 = 196608;     // W2      K-major [t][i]                              16 KB
 constexpr uint32_t OFF_MISC = 212992;
 constexpr uint32_t OFF_GATE = OFF_MISC;            // g, beta, ks, w2s: 4 x 64 floats
 constexpr uint32_t OFF_INFO = OFF_MISC + 1024;     // 2 x ChunkInfo
-constexpr uint32_t OFF_INV = OFF_MISC + 2048;      // 2 x 256 floats (block products)
-constexpr uint32_t OFF_BAR = OFF_MISC + 4096;      // mbarriers
-constexpr uint32_t OFF_FLAGS = OFF_BAR + 128;      // TMEM base, abort flag
+constexpr uint32_t OFF_BAR = OFF_MISC + 2048;      // mbarriers
+constexpr uint32_t OFF_FLAGS = OFF_BAR + 256;      // TMEM base, abort flag, final G
 constexpr uint32_t kSmem = OFF_FLAGS + 16;
 constexpr uint32_t kSmemAlloc = kSmem + 1024;      // slack to align the base to 1024
 
-// per-chunk values the prep hands to the issuer and the epilogue (double-buffered)
+// per-chunk values the scale role hands to the issuer and the epilogue (double-buffered)
 struct ChunkInfo {
     float yscale[64];   // G gamma_t
     float rfac;         // G gamma_C: factor of the rescale of S~, if any
@@ -81,12 +79,15 @@ static_assert(sizeof(ChunkInfo) == 512, "ChunkInfo layout");
 
 enum {
     B_KQ = 0, B_V, B_KMN,        // TMA arrivals
-    B_A, B_1, B_2, B_34,         // MMA completions
-    B_TB, B_PK,                  // prep: T_beta/W2/info ready; K~/P ready
+    B_TBL0, B_TBL1,              // TMA arrivals of T_beta into buffer 0 / 1
+    B_PL0, B_PL1,                // TMA arrivals of P into buffer 0 / 1
+    B_1, B_2, B_34,              // MMA completions
+    B_TB, B_PK,                  // scale role: W2 and chunk info ready; K~ ready
     B_Y1,                        // epilogue: Y1 taken, Y = G gamma Y1 stored, S~ rescaled
-    B_DRAIN0, B_DRAIN1,          // drains on the failure path
+    B_DRAIN0,                    // drain on the failure path
     kNumBars
 };
+static_assert(kNumBars * 8 <= 256, "barrier area");
 
 // tensor memory columns (all 128 lanes)
 constexpr uint32_t kTmemCols = 512;
@@ -94,13 +95,9 @@ constexpr uint32_t T_S = 0;      // S~^T                 128 cols
 constexpr uint32_t T_XY = 128;   // [X | Y1]             128 cols
 constexpr uint32_t T_U = 256;    // u^T                   64 cols
 constexpr uint32_t T_Y = 320;    // G gamma Y1, then y     64 cols
-constexpr uint32_t T_A = 384;    // [K;Q] K^T             64 cols
 
 constexpr float kRescaleBelow = 0x1p-48f;
 constexpr uint32_t kWaitTries = 1u << 22;
-
-// fp32 scratch [64][64] with 16-byte chunks XOR-swizzled by row
-__device__ __forceinline__ int scr(int r, int c) { return r * 64 + ((((c >> 2) ^ (r & 7)) << 2) | (c & 3)); }
 
 __device__ __forceinline__ float4 tf32x4(float a, float b, float c, float d) {
     return make_float4(to_tf32(a), to_tf32(b), to_tf32(c), to_tf32(d));
@@ -180,8 +177,10 @@ struct TcParams {
     CUtensorMap tm_q;     // q^ rows, same
     CUtensorMap tm_kmn;   // k^ rows, 32-byte-granule swizzle boxes (MN-major operand)
     CUtensorMap tm_vmn;   // v^ rows, same
+    CUtensorMap tm_tb;    // T_beta tiles as [chunk*Hv*64, 64] rows, K-major 128B swizzle boxes
+    CUtensorMap tm_pm;    // P tiles, same
     const void *alpha, *beta;
-    const int32_t *cu;
+    const int32_t *cu, *cfirst;
     const float *init;
     float *fin;
     void *out;
@@ -206,6 +205,7 @@ __global__ void __launch_bounds__(kThr, 1) prefill_tc_kernel(const __grid_consta
     const int seq0 = p.cu[b], L = p.cu[b + 1] - p.cu[b];
     const int64_t v_row = (int64_t)p.n_v * kHeadDim;
     const int nchunks = (L + kChunk - 1) / kChunk;
+    const int tile0 = (p.cfirst[b] * p.n_v + h) * kChunk;   // T_beta / P row of chunk 0
 
     if (tid == 0) {
         for (int i = 0; i < kNumBars; ++i) mbar_init(&bar[i], 1);
@@ -245,6 +245,14 @@ __global__ void __launch_bounds__(kThr, 1) prefill_tc_kernel(const __grid_consta
         for (int db = 0; db < 4; ++db)
             tma_load_2d(sb + OFF_KMN + db * 8192, &p.tm_kmn, gq * kHeadDim + 32 * db, tok, &bar[B_KMN]);
     };
+    auto issue_tile = [&](const CUtensorMap *m, uint32_t dst, int bar_i, int c) {  // T_beta or P
+        const int row = tile0 + c * p.n_v * kChunk;
+        mbar_expect_tx(&bar[bar_i], 16384);
+        tma_load_2d(dst, m, 0, row, &bar[bar_i]);
+        tma_load_2d(dst + 8192, m, 32, row, &bar[bar_i]);
+    };
+    auto issue_tb = [&](int c) { issue_tile(&p.tm_tb, sb + OFF_TB + (c & 1) * 16384, B_TBL0 + (c & 1), c); };
+    auto issue_pm = [&](int c) { issue_tile(&p.tm_pm, sb + OFF_P + (c & 1) * 16384, B_PL0 + (c & 1), c); };
 
     // epilogue warps: initial state S~^T (lane j = column j of S) into tensor memory
     if (warp >= kEpiWarp0 && warp < kPrepWarp0) {
@@ -264,6 +272,12 @@ __global__ void __launch_bounds__(kThr, 1) prefill_tc_kernel(const __grid_consta
         issue_kq(0);
         issue_v(0);
         issue_kmn(0);
+        issue_tb(0);
+        issue_pm(0);
+        if (nchunks > 1) {
+            issue_tb(1);
+            issue_pm(1);
+        }
     }
     fence_before_sync();
     __syncthreads();
@@ -274,8 +288,10 @@ __global__ void __launch_bounds__(kThr, 1) prefill_tc_kernel(const __grid_consta
         if (lane == 0) {
             bool ok = true;
             int n_kq = nchunks > 0 ? 1 : 0, n_v = n_kq, n_kmn = n_kq;
+            int n_tb[2] = {nchunks > 0 ? 1 : 0, nchunks > 1 ? 1 : 0}, n_pm[2] = {n_tb[0], n_tb[1]};
             for (int c = 0; c < nchunks; ++c) {
-                const uint32_t par = c & 1;
+                const uint32_t par = c & 1, bpar = (c >> 1) & 1;
+                const int bsel = c & 1;
                 // MMA_1: needs S~ (previous MMA_3, waited below) and [K;Q] of c; Y1 of c-1 was
                 // drained before MMA_4 of c-1
                 if (!(ok = wait_or_abort(&bar[B_KQ], par, abort_flag))) break;
@@ -283,27 +299,31 @@ __global__ void __launch_bounds__(kThr, 1) prefill_tc_kernel(const __grid_consta
                 gemm_ts<128, 128, false, false>(tm + T_XY, tm + T_S, sb + OFF_KQ, 16384, false);
                 mma_commit(&bar[B_1]);
                 // MMA_2a: U^T = V^T T_beta^T (state-independent)
-                if (!(ok = wait_or_abort(&bar[B_TB], par, abort_flag))) break;
+                if (!(ok = wait_or_abort(&bar[B_TB], par, abort_flag))) break;   // W2, info of c
+                if (!(ok = wait_or_abort(&bar[B_TBL0 + bsel], bpar, abort_flag))) break;
                 if (!(ok = wait_or_abort(&bar[B_V], par, abort_flag))) break;
                 fence_after_sync();
-                gemm<128, 64, 64, true, false>(tm + T_U, sb + OFF_VMN, 64, sb + OFF_TB, 8192, false);
+                gemm<128, 64, 64, true, false>(tm + T_U, sb + OFF_VMN, 64, sb + OFF_TB + bsel * 16384, 8192, false);
                 // MMA_2b: U^T -= X W2^T
                 if (!(ok = wait_or_abort(&bar[B_1], par, abort_flag))) break;
-                if (c + 1 < nchunks) { issue_kq(c + 1); ++n_kq; }   // [K;Q] is free (MMA_a(c) done before B_TB)
+                if (c + 1 < nchunks) { issue_kq(c + 1); ++n_kq; }   // [K;Q] of c is consumed
                 fence_after_sync();
                 gemm_ts<64, 64, false, true>(tm + T_U, tm + T_XY, sb + OFF_W2, 8192, true);
                 mma_commit(&bar[B_2]);
                 if (!(ok = wait_or_abort(&bar[B_2], par, abort_flag))) break;
                 if (c + 1 < nchunks) { issue_v(c + 1); ++n_v; }
+                if (c + 2 < nchunks) { issue_tb(c + 2); ++n_tb[bsel]; }  // this T_beta buffer is consumed
                 // MMA_3 / MMA_4: S~ += u^T K~ (after the rescale of S~, if any); Y += u^T P^T
                 if (!(ok = wait_or_abort(&bar[B_Y1], par, abort_flag))) break;
                 if (!(ok = wait_or_abort(&bar[B_PK], par, abort_flag))) break;
+                if (!(ok = wait_or_abort(&bar[B_PL0 + bsel], bpar, abort_flag))) break;
                 fence_after_sync();
                 gemm_ts<128, 64, true, false>(tm + T_S, tm + T_U, sb + OFF_KMN, 64, true);
-                gemm_ts<64, 64, false, false>(tm + T_Y, tm + T_U, sb + OFF_P, 8192, true);
+                gemm_ts<64, 64, false, false>(tm + T_Y, tm + T_U, sb + OFF_P + bsel * 16384, 8192, true);
                 mma_commit(&bar[B_34]);
                 if (!(ok = wait_or_abort(&bar[B_34], par, abort_flag))) break;
                 if (c + 1 < nchunks) { issue_kmn(c + 1); ++n_kmn; }
+                if (c + 2 < nchunks) { issue_pm(c + 2); ++n_pm[bsel]; }
             }
             if (!ok) {
                 // drain this thread's MMAs and the TMA loads it issued, each wait bounded
@@ -312,6 +332,10 @@ __global__ void __launch_bounds__(kThr, 1) prefill_tc_kernel(const __grid_consta
                 if (n_kq) mbar_wait(&bar[B_KQ], (uint32_t)(n_kq - 1) & 1, kWaitTries);
                 if (n_v) mbar_wait(&bar[B_V], (uint32_t)(n_v - 1) & 1, kWaitTries);
                 if (n_kmn) mbar_wait(&bar[B_KMN], (uint32_t)(n_kmn - 1) & 1, kWaitTries);
+                for (int i = 0; i < 2; ++i) {
+                    if (n_tb[i]) mbar_wait(&bar[B_TBL0 + i], (uint32_t)(n_tb[i] - 1) & 1, kWaitTries);
+                    if (n_pm[i]) mbar_wait(&bar[B_PL0 + i], (uint32_t)(n_pm[i] - 1) & 1, kWaitTries);
+                }
             }
         }
     } else if (warp < kPrepWarp0) {
@@ -381,10 +405,8 @@ __global__ void __launch_bounds__(kThr, 1) prefill_tc_kernel(const __grid_consta
         (void)ok;
         if (leader) *s_gfinal = gfinal;   // the final state is written after the tear-down barrier
     } else {
-        // ================================================================ prep
+        // ================================================================ scale role
         const int ptid = tid - kPrepTid0;                // 0..255
-        const int q = warp & 3;                          // tensor-memory lane quarter
-        const int ch = (warp - kPrepWarp0) >> 2;         // which 32 of the 64 columns of [K;Q]K^T
         const TI *al = (const TI *)p.alpha;
         const TI *be = (const TI *)p.beta;
         typedef typename RawT<TI>::type raw_t;
@@ -401,26 +423,18 @@ __global__ void __launch_bounds__(kThr, 1) prefill_tc_kernel(const __grid_consta
             const bool ok = wait_or_abort(&bar[i], par, abort_flag);
             return !bar_or(kBarPrep, 256, !ok);
         };
-        auto pwait_or_sync = [&](bool need, int i, uint32_t par) -> bool {
-            if (need) return pwait(i, par);
-            bar_sync(kBarPrep, 256);
-            return true;
-        };
         float *g_s = (float *)(sm + OFF_GATE);
         float *beta_s = g_s + 64, *ks_s = g_s + 128, *w2s_s = g_s + 192;
-        float *Ascr = (float *)(sm + OFF_AS);
-        float *Tscr = (float *)(sm + OFF_TS);
-        float *inv_s = (float *)(sm + OFF_INV);
         float G = 1.f;                                   // scale of S~ entering the chunk
         if (nchunks > 0 && ptid < kChunk) load_gates(0);
 
         for (int c = 0; c < nchunks; ++c) {
             const int n = min(kChunk, L - c * kChunk);
             const uint32_t par = c & 1, ppar = par ^ 1;
+            const int bsel = c & 1;
             ChunkInfo *ci = &info[par];
-
-            // ---- gates, their scan and the chunk's scales
-            if (!pwait(B_KQ, par)) break;
+            // ---- gates, their scan and the chunk's scales.  info[par] was last read by the
+            // epilogue for chunk c-2, which released B_Y1 before this role's previous B_TB.
             if (ptid < kChunk) {
                 g_s[ptid] = ptid < n ? safe_log_alpha(raw_to_f32(a_raw)) : 0.f;
                 beta_s[ptid] = ptid < n ? raw_to_f32(b_raw) : 0.f;
@@ -442,12 +456,10 @@ __global__ void __launch_bounds__(kThr, 1) prefill_tc_kernel(const __grid_consta
                 const float Gn = G * gC;
                 const bool rflag = Gn < kRescaleBelow;
                 const float kscale = rflag ? 1.f : 1.f / Gn;
-                g_s[t0] = g0;
-                g_s[t1] = g1;
                 ks_s[t0] = t0 < n ? expf(glast - g0) * kscale : 0.f;
                 ks_s[t1] = t1 < n ? expf(glast - g1) * kscale : 0.f;
-                w2s_s[t0] = G * gam0 * beta_s[t0];
-                w2s_s[t1] = G * gam1 * beta_s[t1];
+                w2s_s[t0] = G * gam0;
+                w2s_s[t1] = G * gam1;
                 ci->yscale[t0] = G * gam0;
                 ci->yscale[t1] = G * gam1;
                 if (lane == 0) {
@@ -456,166 +468,47 @@ __global__ void __launch_bounds__(kThr, 1) prefill_tc_kernel(const __grid_consta
                     ci->gnext = rflag ? 1.f : Gn;
                 }
             }
-            bar_sync(kBarPrep, 256);
-            if (ptid == 0) {
-                fence_after_sync();
-                gemm<128, 64, 128, false, false>(tm + T_A, sb + OFF_KQ, 16384, sb + OFF_KQ, 16384, false);
-                mma_commit(&bar[B_A]);
-            }
-            // ---- epilogue a: A (fp32 scratch) and P (K-major tile; free once MMA_4 of c-1 is done)
-            if (c > 0 && !pwait(B_34, ppar)) break;
-            if (!pwait(B_A, par)) break;
-            fence_after_sync();
-            {
-                float v[32];
-                tmem_ld32(taddr(tm + T_A, 32 * q, 32 * ch), v);
-                tmem_wait_ld();
-                if (q < 2) {  // K K^T rows
-                    const int t = 32 * q + lane;
-                    const float gt = g_s[t], bt = beta_s[t];
-#pragma unroll
-                    for (int k = 0; k < 8; ++k) {
-                        float a4[4];
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const int i = 32 * ch + 4 * k + e;
-                            a4[e] = (i < t && t < n) ? bt * expf(gt - g_s[i]) * v[4 * k + e] : 0.f;
-                        }
-                        *reinterpret_cast<float4 *>(&Ascr[scr(t, 32 * ch + 4 * k)]) = make_float4(a4[0], a4[1], a4[2], a4[3]);
-                    }
-                } else {  // Q K^T rows
-                    const int t = 32 * (q - 2) + lane;
-                    const float gt = g_s[t];
-                    unsigned char *Pt = sm + OFF_P;
-#pragma unroll
-                    for (int k = 0; k < 8; ++k) {
-                        float p4[4];
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const int i = 32 * ch + 4 * k + e;
-                            p4[e] = (i <= t && t < n) ? expf(gt - g_s[i]) * v[4 * k + e] : 0.f;
-                        }
-                        *reinterpret_cast<float4 *>(Pt + kmaj_off(t, 32 * ch + 4 * k, 64)) = tf32x4(p4[0], p4[1], p4[2], p4[3]);
-                    }
-                }
-            }
-            fence_before_sync();
-            bar_sync(kBarPrep, 256);
-            // ---- T = (I + A)^-1: 16 x 16 diagonal blocks, two 32 x 32 halves, one merge
-            if (ptid < 64) {  // diagonal blocks: column cc of block bb, right-looking updates
-                const int bb = ptid >> 4, cc = ptid & 15, o = 16 * bb;
-                float x[16];
-#pragma unroll
-                for (int r = 0; r < 16; ++r) x[r] = (r == cc) ? 1.f : 0.f;
-#pragma unroll
-                for (int m = 0; m < 15; ++m) {
-                    const float xm = x[m];
-#pragma unroll
-                    for (int r = m + 1; r < 16; ++r) x[r] = fmaf(-Ascr[scr(o + r, o + m)], xm, x[r]);
-                }
-#pragma unroll
-                for (int r = 0; r < 16; ++r) Tscr[scr(o + r, o + cc)] = x[r];
-            } else {  // zero the 16 x 16 blocks above the diagonal that the products read
-                for (int e = ptid - 64; e < 512; e += 192) {
-                    const int blk = e >> 8, r = (e >> 4) & 15, cc = e & 15;
-                    const int o = 32 * blk;
-                    Tscr[scr(o + r, o + 16 + cc)] = 0.f;
-                }
-            }
-            bar_sync(kBarPrep, 256);
-            if (ptid < 128) {  // halves: M = A_10 T_00 (16 x 16 blocks)
-                const int hh = ptid >> 6, rr = (ptid >> 2) & 15, c4 = (ptid & 3) * 4, o = 32 * hh;
-                float a4[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-                for (int m = 0; m < 16; ++m) {
-                    const float a = Ascr[scr(o + 16 + rr, o + m)];
-                    const float4 t4 = *reinterpret_cast<const float4 *>(&Tscr[scr(o + m, o + c4)]);
-                    a4[0] = fmaf(a, t4.x, a4[0]); a4[1] = fmaf(a, t4.y, a4[1]);
-                    a4[2] = fmaf(a, t4.z, a4[2]); a4[3] = fmaf(a, t4.w, a4[3]);
-                }
-                *reinterpret_cast<float4 *>(&inv_s[hh * 256 + rr * 16 + c4]) = make_float4(a4[0], a4[1], a4[2], a4[3]);
-            }
-            bar_sync(kBarPrep, 256);
-            if (ptid < 128) {  // T_10 = -T_11 M
-                const int hh = ptid >> 6, rr = (ptid >> 2) & 15, c4 = (ptid & 3) * 4, o = 32 * hh;
-                float a4[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-                for (int m = 0; m < 16; ++m) {
-                    const float t = Tscr[scr(o + 16 + rr, o + 16 + m)];
-                    const float4 m4 = *reinterpret_cast<const float4 *>(&inv_s[hh * 256 + m * 16 + c4]);
-                    a4[0] = fmaf(t, m4.x, a4[0]); a4[1] = fmaf(t, m4.y, a4[1]);
-                    a4[2] = fmaf(t, m4.z, a4[2]); a4[3] = fmaf(t, m4.w, a4[3]);
-                }
-                *reinterpret_cast<float4 *>(&Tscr[scr(o + 16 + rr, o + c4)]) = make_float4(-a4[0], -a4[1], -a4[2], -a4[3]);
-            }
-            bar_sync(kBarPrep, 256);
-            {  // merge: M = A_bl T_top, parked in the (unused) upper-right block
-                const int r = ptid >> 3, c4 = (ptid & 7) * 4;
-                float a4[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-                for (int m = 0; m < 32; ++m) {
-                    const float a = Ascr[scr(32 + r, m)];
-                    const float4 t4 = *reinterpret_cast<const float4 *>(&Tscr[scr(m, c4)]);
-                    a4[0] = fmaf(a, t4.x, a4[0]); a4[1] = fmaf(a, t4.y, a4[1]);
-                    a4[2] = fmaf(a, t4.z, a4[2]); a4[3] = fmaf(a, t4.w, a4[3]);
-                }
-                *reinterpret_cast<float4 *>(&Tscr[scr(r, 32 + c4)]) = make_float4(a4[0], a4[1], a4[2], a4[3]);
-            }
-            bar_sync(kBarPrep, 256);
-            {  // T_bl = -T_br M
-                const int r = ptid >> 3, c4 = (ptid & 7) * 4;
-                float a4[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-                for (int m = 0; m < 32; ++m) {
-                    const float t = Tscr[scr(32 + r, 32 + m)];
-                    const float4 m4 = *reinterpret_cast<const float4 *>(&Tscr[scr(m, 32 + c4)]);
-                    a4[0] = fmaf(t, m4.x, a4[0]); a4[1] = fmaf(t, m4.y, a4[1]);
-                    a4[2] = fmaf(t, m4.z, a4[2]); a4[3] = fmaf(t, m4.w, a4[3]);
-                }
-                *reinterpret_cast<float4 *>(&Tscr[scr(32 + r, c4)]) = make_float4(-a4[0], -a4[1], -a4[2], -a4[3]);
-            }
-            // ---- T_beta and W2 (their buffers are free once MMA_2b of c-1 is done)
-            if (!pwait_or_sync(c > 0, B_2, ppar)) break;   // also orders the T products
+            // ---- W2 = G T_beta diag(gamma) (its buffer is free once MMA_2b of c-1 is done)
+            if (!pwait(B_TBL0 + bsel, (c >> 1) & 1)) break;   // also orders the scan
+            if (c > 0 && !pwait(B_2, ppar)) break;
             {
                 const int t = ptid >> 2, i0 = (ptid & 3) * 16;
-                const bool upper_right = t < 32 && i0 >= 32;
-                unsigned char *Tb = sm + OFF_TB, *W2 = sm + OFF_W2;
+                const unsigned char *Tb = sm + OFF_TB + bsel * 16384;
+                unsigned char *W2 = sm + OFF_W2;
 #pragma unroll
                 for (int k = 0; k < 4; ++k) {
                     const int i = i0 + 4 * k;
-                    float4 x = *reinterpret_cast<const float4 *>(&Tscr[scr(t, i)]);
-                    if (upper_right) x = make_float4(0.f, 0.f, 0.f, 0.f);
-                    *reinterpret_cast<float4 *>(Tb + kmaj_off(t, i, 64)) =
-                        tf32x4(x.x * beta_s[i], x.y * beta_s[i + 1], x.z * beta_s[i + 2], x.w * beta_s[i + 3]);
-                    *reinterpret_cast<float4 *>(W2 + kmaj_off(t, i, 64)) =
+                    const uint32_t off = kmaj_off(t, i, 64);
+                    const float4 x = *reinterpret_cast<const float4 *>(Tb + off);
+                    *reinterpret_cast<float4 *>(W2 + off) =
                         tf32x4(x.x * w2s_s[i], x.y * w2s_s[i + 1], x.z * w2s_s[i + 2], x.w * w2s_s[i + 3]);
                 }
             }
             fence_smem_to_async();
             // the epilogue must have taken chunk c-1's info before B_TB moves on
-            if (!pwait_or_sync(c > 0, B_Y1, ppar)) break;
+            if (c > 0) {
+                if (!pwait(B_Y1, ppar)) break;
+            } else {
+                bar_sync(kBarPrep, 256);
+            }
             if (ptid == 0) mbar_arrive(&bar[B_TB]);
             // ---- K~ = diag(exp(g_C - g) / G') K, in place in the MN-major tile
             if (!pwait(B_KMN, par)) break;
             {
                 const int blk = ptid >> 6, t = ptid & 63;
                 unsigned char *row = sm + OFF_KMN + blk * 8192 + t * 128;
-                const float s = ks_s[t];
+                const float sc = ks_s[t];
 #pragma unroll
                 for (int k = 0; k < 8; ++k) {
                     const int kk = (k + t) & 7;   // staggered: rows 128 B apart share banks
                     float4 x = *reinterpret_cast<const float4 *>(row + 16 * kk);
-                    *reinterpret_cast<float4 *>(row + 16 * kk) = tf32x4(x.x * s, x.y * s, x.z * s, x.w * s);
+                    *reinterpret_cast<float4 *>(row + 16 * kk) = tf32x4(x.x * sc, x.y * sc, x.z * sc, x.w * sc);
                 }
             }
             fence_smem_to_async();
             bar_sync(kBarPrep, 256);
             if (ptid == 0) mbar_arrive(&bar[B_PK]);
             G = ci->gnext;
-        }
-        if (*abort_flag && ptid == 0) {  // drain MMA_a
-            mma_commit(&bar[B_DRAIN1]);
-            mbar_wait(&bar[B_DRAIN1], 0, kWaitTries);
         }
     }
 
@@ -653,31 +546,6 @@ __global__ void __launch_bounds__(kThr, 1) prefill_tc_kernel(const __grid_consta
 }
 
 // ---------------------------------------------------------------- host side
-static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    if (!fn) {
-        void *f = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = (PFN_cuTensorMapEncodeTiled_v12000)f;
-    }
-    return fn;
-}
-
-// 2-D map over a [rows x width] fp32 matrix, boxes of 32 columns x 64 rows
-static bool encode_rows(CUtensorMap *m, const float *base, int64_t width, int64_t rows,
-                        CUtensorMapSwizzle swz) {
-    auto enc = tensor_map_encoder();
-    if (!enc) return false;
-    cuuint64_t dims[2] = {(cuuint64_t)width, (cuuint64_t)rows};
-    cuuint64_t strides[1] = {(cuuint64_t)width * 4};
-    cuuint32_t box[2] = {32, 64}, es[2] = {1, 1};
-    return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, (void *)base, dims, strides, box, es,
-               CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 template <class TI, class TO>
 static cudaError_t launch_tc_t(const TcParams &p, cudaStream_t s) {
     auto k = prefill_tc_kernel<TI, TO>;
@@ -695,12 +563,18 @@ cudaError_t launch_prefill_tc(const ScanParams &sp, int64_t total_tokens, bool i
     TcParams p{};
     const int64_t T = total_tokens > 0 ? total_tokens : 1;
     const int64_t wqk = (int64_t)sp.n_qk * kHeadDim, wv = (int64_t)sp.n_v * kHeadDim;
+    // T_beta / P tiles: rows (chunk * Hv + h) * 64 + t of a 64-wide matrix (int32 TMA coordinates)
+    const int64_t tile_rows = (total_tokens > 0 ? sp.max_chunks : 1) * sp.n_v * kChunk;
+    if (tile_rows >= ((int64_t)1 << 31)) return cudaErrorInvalidValue;
     if (!encode_rows(&p.tm_k, sp.kh, wqk, T, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !encode_rows(&p.tm_q, sp.qh, wqk, T, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !encode_rows(&p.tm_kmn, sp.kh, wqk, T, CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B) ||
-        !encode_rows(&p.tm_vmn, sp.vh, wv, T, CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B))
+        !encode_rows(&p.tm_vmn, sp.vh, wv, T, CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B) ||
+        !encode_rows(&p.tm_tb, sp.tb, kChunk, tile_rows, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !encode_rows(&p.tm_pm, sp.pm, kChunk, tile_rows, CU_TENSOR_MAP_SWIZZLE_128B))
         return cudaErrorInvalidValue;
-    p.alpha = sp.alpha; p.beta = sp.beta; p.cu = sp.cu; p.init = sp.init; p.fin = sp.fin;
+    p.alpha = sp.alpha; p.beta = sp.beta; p.cu = sp.cu; p.cfirst = sp.cfirst;
+    p.init = sp.init; p.fin = sp.fin;
     p.out = sp.out; p.n_seqs = sp.n_seqs; p.n_qk = sp.n_qk; p.n_v = sp.n_v;
     if (in_bf16) return out_bf16 ? launch_tc_t<gdn::bf16, gdn::bf16>(p, s) : launch_tc_t<gdn::bf16, float>(p, s);
     return out_bf16 ? launch_tc_t<float, gdn::bf16>(p, s) : launch_tc_t<float, float>(p, s);

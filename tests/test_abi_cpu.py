@@ -53,9 +53,12 @@ def test_workspace_size():
     st, b = _ws(_cfg(), 0, 8192, 1)
     assert st == 0
     # q^, k^ (2 x T x 16 x 128) + v^ (T x 48 x 128) in fp32, plus two small int tables
-    assert b >= 8192 * (2 * 16 + 48) * 128 * 4
+    rows = 8192 * (2 * 16 + 48) * 128 * 4
+    # the tensor-core (bf16) path adds two 64 x 64 fp32 tiles per (chunk, V head)
+    tiles = 2 * (8192 // 64 + 1) * 48 * 64 * 64 * 4
+    assert b >= rows + tiles
     st4, b4 = _ws(_cfg(), 1, 8192, 1)
-    assert st4 == 0 and b4 == b
+    assert st4 == 0 and rows <= b4 < rows + tiles
     assert _ws(_cfg(), 0, 0, 3)[0] == 0
 
 
