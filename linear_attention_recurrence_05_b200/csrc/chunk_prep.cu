@@ -6,18 +6,22 @@
 //     A_ti = beta_t exp(g_t - g_i) k_t.k_i        (i < t < n, else 0)
 //     T    = (I + A)^-1,   T_beta = T diag(beta)   (unit lower triangular solve)
 //     P_ti = exp(g_t - g_i) q_t.k_i               (i <= t < n, else 0)
-// T_beta and P are written as 64 x 64 fp32 tiles (row t, column i; values rounded to TF32,
-// the precision the tensor-core chain reads them in) for the chain kernel to stream in.
-// Rows and columns at or past n are zero, so a partial chunk needs no masking downstream.
+// T_beta, W2 = T diag(beta gamma) and P are written as 64 x 64 fp32 tiles, and
+// K~ = diag(kd) K (kd_t = exp(g_{n-1} - g_t), 0 for t >= n) as a 64 x 128 tile in the
+// MN-major layout of the conv pass's K tile, (row t, column i; values rounded to TF32,
+// the precision the tensor-core chain reads them in), already in the shared-memory layout
+// of an MMA operand (K-major, 128-byte rows with 16-byte chunks XOR-swizzled by row), for
+// the chain kernel to stream in with one bulk copy each.  Rows and columns at or past n are
+// zero, so a partial chunk needs no masking downstream.  A gates record per (chunk, head)
+// carries gamma_t = exp(g_t), kd_t = exp(g_{n-1} - g_t) (0 for t >= n) and gamma_C = exp(g_{n-1}).
 //
-// One CTA per (chunk, V head), 256 threads: TMA brings the chunk's K and Q rows, one
+// One CTA per (chunk, V head), 256 threads: one bulk copy brings the chunk's [K;Q] tile, one
 // tcgen05 MMA forms [K;Q] K^T in tensor memory, the warps turn it into A and P, and the
 // inverse runs on CUDA cores in fp32: 16 x 16 diagonal blocks by forward substitution,
 // then two block-merge levels (16 -> 32 -> 64).
 #include "gdn_common.cuh"
 #include "gdn_internal.h"
 #include "tc_sm100.cuh"
-#include "tma_map.cuh"
 
 namespace gdn {
 
@@ -31,9 +35,9 @@ constexpr uint32_t P_KQ = 0;          // [K;Q] K-major, 4 blocks x (K 8 KB | Q 8
 constexpr uint32_t P_AS = 65536;      // A (fp32, swizzled rows)                       16 KB
 constexpr uint32_t P_TS = 81920;      // T (fp32, swizzled rows)                       16 KB
 constexpr uint32_t P_INV = 98304;     // 2 x 256 floats (block products)                2 KB
-constexpr uint32_t P_GATE = 100352;   // g[64], beta[64]                               512 B
-constexpr uint32_t P_BAR = 100864;    // 2 mbarriers
-constexpr uint32_t P_SLOT = 100880;   // TMEM base
+constexpr uint32_t P_GATE = 100352;   // g[64], beta[64], gamma[64], kd[64]            1 KB
+constexpr uint32_t P_BAR = 101376;    // 2 mbarriers
+constexpr uint32_t P_SLOT = 101392;   // TMEM base
 constexpr uint32_t kPSmem = P_SLOT + 16;
 constexpr uint32_t kPSmemAlloc = kPSmem + 1024;
 constexpr uint32_t kPTmemCols = 64;
@@ -47,11 +51,13 @@ __device__ __forceinline__ float4 tf32x4(float4 x) {
 }
 
 struct PrepParams {
-    CUtensorMap tm_k;     // k^ rows, K-major 128B swizzle boxes (32 x 64)
-    CUtensorMap tm_q;     // q^ rows, same
+    const float *kq;      // [chunk, Hqk] [K;Q] tiles (64 KB each)
+    const float *kmn;     // [chunk, Hqk] K tiles, MN-major (32 KB each)
+    float *kt;            // [chunk, Hv] K~ tiles (32 KB each)
     const void *alpha, *beta;
     const int32_t *cu, *cfirst;
-    float *tb, *pm;       // [chunk, Hv, 64, 64]
+    float *tb, *w2, *pm;  // [chunk, Hv] tiles (16 KB each)
+    float *gr;            // [chunk, Hv] gates records
     int n_seqs, n_qk, n_v;
 };
 
@@ -74,21 +80,19 @@ __global__ void __launch_bounds__(kPThr) chunk_prep_kernel(const __grid_constant
     const uint32_t sb = smem_u32(sm);
     uint64_t *bar = (uint64_t *)(sm + P_BAR);
     uint32_t *tslot = (uint32_t *)(sm + P_SLOT);
-    float *g_s = (float *)(sm + P_GATE), *beta_s = g_s + 64;
+    float *g_s = (float *)(sm + P_GATE), *beta_s = g_s + 64, *gam_s = g_s + 128, *kd_s = g_s + 192;
     float *Ascr = (float *)(sm + P_AS), *Tscr = (float *)(sm + P_TS), *inv_s = (float *)(sm + P_INV);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     float *tb = p.tb + ((int64_t)u * p.n_v + h) * (kChunk * kChunk);
     float *pm = p.pm + ((int64_t)u * p.n_v + h) * (kChunk * kChunk);
+    float *w2 = p.w2 + ((int64_t)u * p.n_v + h) * (kChunk * kChunk);
+    float *gr = p.gr + ((int64_t)u * p.n_v + h) * kGateRec;
 
     if (tid == 0) {
         mbar_init(&bar[0], 1);
         mbar_init(&bar[1], 1);
         mbar_expect_tx(&bar[0], 65536);
-#pragma unroll
-        for (int kb = 0; kb < 4; ++kb) {
-            tma_load_2d(sb + P_KQ + kb * 16384, &p.tm_k, gq * kHeadDim + 32 * kb, tok, &bar[0]);
-            tma_load_2d(sb + P_KQ + kb * 16384 + 8192, &p.tm_q, gq * kHeadDim + 32 * kb, tok, &bar[0]);
-        }
+        bulk_load(sb + P_KQ, p.kq + ((int64_t)u * p.n_qk + gq) * 16384, 65536, &bar[0]);
     }
     if (warp == 0) {
         tmem_alloc(tslot, kPTmemCols);
@@ -125,8 +129,21 @@ __global__ void __launch_bounds__(kPThr) chunk_prep_kernel(const __grid_constant
             const float y = __shfl_up_sync(0xffffffffu, s, o);
             if (lane >= o) s += y;
         }
-        g_s[t0] = s - a1;
-        g_s[t1] = s;
+        const float g0 = s - a1, g1 = s;
+        const float glast = __shfl_sync(0xffffffffu, ((n - 1) & 1) ? g1 : g0, (n - 1) >> 1);
+        g_s[t0] = g0;
+        g_s[t1] = g1;
+        const float gam0 = expf(g0), gam1 = expf(g1);
+        gam_s[t0] = gam0;
+        gam_s[t1] = gam1;
+        gr[kGrGamma + t0] = gam0;
+        gr[kGrGamma + t1] = gam1;
+        const float kd0 = t0 < n ? expf(glast - g0) : 0.f, kd1 = t1 < n ? expf(glast - g1) : 0.f;
+        kd_s[t0] = kd0;
+        kd_s[t1] = kd1;
+        gr[kGrKd + t0] = kd0;
+        gr[kGrKd + t1] = kd1;
+        if (lane == 0) gr[kGrGammaC] = expf(glast);
     }
     if (__syncthreads_or(!ok)) {
         if (tid == 0) mbar_wait(&bar[0], 0, kPWaitTries);  // drain the copies
@@ -164,7 +181,7 @@ __global__ void __launch_bounds__(kPThr) chunk_prep_kernel(const __grid_constant
                     const int i = 32 * ch + 4 * k + e;
                     p4[e] = (i <= t && t < n) ? expf(gt - g_s[i]) * v[4 * k + e] : 0.f;
                 }
-                *reinterpret_cast<float4 *>(pm + t * 64 + 32 * ch + 4 * k) =
+                *reinterpret_cast<float4 *>((unsigned char *)pm + kmaj_off(t, 32 * ch + 4 * k, 64)) =
                     tf32x4(make_float4(p4[0], p4[1], p4[2], p4[3]));
             }
         }
@@ -259,7 +276,20 @@ __global__ void __launch_bounds__(kPThr) chunk_prep_kernel(const __grid_constant
             if (upper_right) x = make_float4(0.f, 0.f, 0.f, 0.f);
             x = make_float4(x.x * beta_s[i], x.y * beta_s[i + 1], x.z * beta_s[i + 2], x.w * beta_s[i + 3]);
             if (!ok) x = make_float4(nan, nan, nan, nan);
-            *reinterpret_cast<float4 *>(tb + t * 64 + i) = tf32x4(x);
+            *reinterpret_cast<float4 *>((unsigned char *)tb + kmaj_off(t, i, 64)) = tf32x4(x);
+            const float4 w = make_float4(x.x * gam_s[i], x.y * gam_s[i + 1], x.z * gam_s[i + 2], x.w * gam_s[i + 3]);
+            *reinterpret_cast<float4 *>((unsigned char *)w2 + kmaj_off(t, i, 64)) = tf32x4(w);
+        }
+    }
+    {  // K~ = diag(kd) K: same tile layout, row t of each 32-feature block scaled by kd_t
+        const float4 *src = reinterpret_cast<const float4 *>(p.kmn + ((int64_t)u * p.n_qk + gq) * 8192);
+        float4 *dst = reinterpret_cast<float4 *>(p.kt + ((int64_t)u * p.n_v + h) * 8192);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            const int i4 = tid + kPThr * k;           // float4 index in the tile
+            const float sc = ok ? kd_s[(i4 >> 3) & 63] : __int_as_float(0x7fc00000);
+            const float4 x = __ldg(src + i4);
+            dst[i4] = tf32x4(make_float4(x.x * sc, x.y * sc, x.z * sc, x.w * sc));
         }
     }
     fence_before_sync();
@@ -270,12 +300,9 @@ __global__ void __launch_bounds__(kPThr) chunk_prep_kernel(const __grid_constant
 cudaError_t launch_chunk_prep(const ScanParams &sp, int64_t total_tokens, bool in_bf16, cudaStream_t s) {
     if (sp.n_seqs <= 0 || total_tokens <= 0) return cudaSuccess;
     PrepParams p{};
-    const int64_t wqk = (int64_t)sp.n_qk * kHeadDim;
-    if (!encode_rows(&p.tm_k, sp.kh, wqk, total_tokens, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !encode_rows(&p.tm_q, sp.qh, wqk, total_tokens, CU_TENSOR_MAP_SWIZZLE_128B))
-        return cudaErrorInvalidValue;
+    p.kq = sp.kq; p.kmn = sp.kmn; p.kt = sp.kt;
     p.alpha = sp.alpha; p.beta = sp.beta; p.cu = sp.cu; p.cfirst = sp.cfirst;
-    p.tb = sp.tb; p.pm = sp.pm; p.n_seqs = sp.n_seqs; p.n_qk = sp.n_qk; p.n_v = sp.n_v;
+    p.tb = sp.tb; p.w2 = sp.w2; p.pm = sp.pm; p.gr = sp.gr; p.n_seqs = sp.n_seqs; p.n_qk = sp.n_qk; p.n_v = sp.n_v;
     const int64_t grid = sp.max_chunks * sp.n_v;
     if (grid >= ((int64_t)1 << 31)) return cudaErrorInvalidValue;
     auto k = in_bf16 ? chunk_prep_kernel<bf16> : chunk_prep_kernel<float>;

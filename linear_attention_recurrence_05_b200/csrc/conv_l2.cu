@@ -85,9 +85,15 @@ cudaError_t launch_seq_table(const int32_t *cu_in, int n_seqs, int64_t T, int32_
 // grid (max_chunks, 2*Hqk + Hv): CTA = one 64-row chunk of one head slot (q heads,
 // then k heads, then v heads).  Warp w walks rows 16w..16w+15 in order, keeping the
 // 3-row conv history of its lane's 4 channels in registers.
-// kTf32: round the stored rows to TF32 (for the tensor-core prefill, whose operands
-// are read as TF32; rounding here gives round-to-nearest instead of truncation).
-template <class T, bool kTf32>
+// kTiles: instead of fp32 rows, write the tensor-core path's chunk tiles, TF32-rounded (the
+// MMAs read them as TF32; rounding here gives round-to-nearest instead of truncation), in
+// the shared-memory layouts the tensor-core kernels copy them into:
+//   [K;Q] of (chunk, QK head): 4 blocks of 32 features x (K 64 rows | Q 64 rows), 128-byte
+//     rows with 16-byte chunks XOR-swizzled by row (K-major operand layout);
+//   K and V of (chunk, head): 4 blocks of 32 features x 64 rows, 128-byte rows with 32-byte
+//     granules XOR-swizzled by row (MN-major operand layout).
+// Rows past the end of the sequence are written as zeros.
+template <class T, bool kTiles>
 __global__ void __launch_bounds__(128) conv_l2_kernel(ConvParams p) {
     const int n_chunks = p.cfirst[p.n_seqs];
     const int ci = blockIdx.x;
@@ -128,7 +134,28 @@ __global__ void __launch_bounds__(128) conv_l2_kernel(ConvParams p) {
     }
     const int rs = r0 + wid * 16;                  // first row of this warp (in sequence)
     const int re = min(rs + 16, r0 + len);
-    if (rs >= re) return;
+    if (!kTiles && rs >= re) return;
+    // tile destinations (float offsets of this lane's 4 features, row 0)
+    float *t_a = nullptr, *t_b = nullptr;          // K-major ([K;Q]) and MN-major (K or V) tile
+    if (kTiles) {
+        if (slot < p.n_qk) {
+            t_a = p.kq + ((int64_t)ci * p.n_qk + slot) * 16384 + 2048;
+        } else if (slot < 2 * p.n_qk) {
+            t_a = p.kq + ((int64_t)ci * p.n_qk + slot - p.n_qk) * 16384;
+            t_b = p.kmn + ((int64_t)ci * p.n_qk + slot - p.n_qk) * 8192;
+        } else {
+            t_b = p.vi + ((int64_t)ci * p.n_v + slot - 2 * p.n_qk) * 8192;
+        }
+    }
+    auto put_tile = [&](int t, const float y[4]) {  // row t of the chunk
+        if (t_a) st4(t_a + (lane >> 3) * 4096 + t * 32 + (((lane & 7) ^ (t & 7)) << 2), y);
+        if (t_b) st4(t_b + (lane >> 3) * 2048 + t * 32 + ((((lane & 7) >> 1) ^ (t & 3)) << 3) + (lane & 1) * 4, y);
+    };
+    if (kTiles) {  // rows of this warp past the end of the sequence
+        const float z[4] = {0.f, 0.f, 0.f, 0.f};
+        for (int s = max(rs, r0 + len); s < r0 + wid * 16 + 16; ++s) put_tile(s - r0, z);
+        if (rs >= re) return;
+    }
     // history rows rs-3, rs-2, rs-1
     float h[3][4];
 #pragma unroll
@@ -158,28 +185,27 @@ __global__ void __launch_bounds__(128) conv_l2_kernel(ConvParams p) {
 #pragma unroll
             for (int c = 0; c < 4; ++c) y[c] *= inv;
         }
-        if (kTf32) {
+        if (kTiles) {
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                uint32_t r;
-                asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(y[c]));
-                y[c] = __uint_as_float(r);
-            }
+            for (int c = 0; c < 4; ++c)  // TF32, nearest with ties away (integer ops)
+                y[c] = __uint_as_float((__float_as_uint(y[c]) + 0x1000u) & 0xFFFFE000u);
+            put_tile(s - r0, y);
+        } else {
+            st4(dst + (int64_t)(seq0 + s) * row_stride + c4, y);
         }
-        st4(dst + (int64_t)(seq0 + s) * row_stride + c4, y);
     }
 }
 
-cudaError_t launch_conv_l2(const ConvParams &p, bool bf16, bool tf32, int64_t max_chunks,
+cudaError_t launch_conv_l2(const ConvParams &p, bool bf16, bool tiles, int64_t max_chunks,
                            cudaStream_t s) {
     if (max_chunks <= 0) return cudaSuccess;
     dim3 grid((unsigned)max_chunks, 2 * p.n_qk + p.n_v);
     TraceLaunch tl(s, "conv_l2");
     if (bf16) {
-        if (tf32) conv_l2_kernel<gdn::bf16, true><<<grid, 128, 0, s>>>(p);
+        if (tiles) conv_l2_kernel<gdn::bf16, true><<<grid, 128, 0, s>>>(p);
         else conv_l2_kernel<gdn::bf16, false><<<grid, 128, 0, s>>>(p);
     } else {
-        if (tf32) conv_l2_kernel<float, true><<<grid, 128, 0, s>>>(p);
+        if (tiles) conv_l2_kernel<float, true><<<grid, 128, 0, s>>>(p);
         else conv_l2_kernel<float, false><<<grid, 128, 0, s>>>(p);
     }
     return cudaGetLastError();

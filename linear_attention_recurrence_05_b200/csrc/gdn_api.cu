@@ -41,14 +41,20 @@ PrefillLayout prefill_layout(int n_qk, int n_v, int64_t T, int n_seqs, bool tc) 
     size_t off = 0;
     L.off_cu = off;      off = align_up(off + sizeof(int32_t) * (size_t)(n_seqs + 1), 256);
     L.off_cfirst = off;  off = align_up(off + sizeof(int32_t) * (size_t)(n_seqs + 1), 256);
-    const size_t qk_bytes = (size_t)T * n_qk * 128 * sizeof(float);
-    const size_t v_bytes = (size_t)T * n_v * 128 * sizeof(float);
+    const size_t qk_bytes = tc ? 0 : (size_t)T * n_qk * 128 * sizeof(float);
+    const size_t v_bytes = tc ? 0 : (size_t)T * n_v * 128 * sizeof(float);
     L.off_qh = off;      off = align_up(off + qk_bytes, 256);
     L.off_kh = off;      off = align_up(off + qk_bytes, 256);
     L.off_vh = off;      off = align_up(off + v_bytes, 256);
-    const size_t tile_bytes = tc && T > 0 ? (size_t)L.max_chunks * n_v * 64 * 64 * sizeof(float) : 0;
-    L.off_tb = off;      off = align_up(off + tile_bytes, 256);
-    L.off_pm = off;      off = align_up(off + tile_bytes, 256);
+    const size_t nc = tc && T > 0 ? (size_t)L.max_chunks : 0;
+    L.off_kq = off;      off = align_up(off + nc * n_qk * 65536, 256);
+    L.off_kmn = off;     off = align_up(off + nc * n_qk * 32768, 256);
+    L.off_vi = off;      off = align_up(off + nc * n_v * 32768, 256);
+    L.off_kt = off;      off = align_up(off + nc * n_v * 32768, 256);
+    L.off_tb = off;      off = align_up(off + nc * n_v * 16384, 256);
+    L.off_w2 = off;      off = align_up(off + nc * n_v * 16384, 256);
+    L.off_pm = off;      off = align_up(off + nc * n_v * 16384, 256);
+    L.off_gr = off;      off = align_up(off + nc * n_v * kGateRec * sizeof(float), 256);
     L.bytes = off;
     return L;
 }
@@ -184,11 +190,13 @@ gdn_status gdn_prefill(const gdn_config *cfg, gdn_dtype dtype, gdn_dtype out_dty
         cp.conv_in = conv_state_in;
         cp.qh = (float *)(ws + L.off_qh); cp.kh = (float *)(ws + L.off_kh);
         cp.vh = (float *)(ws + L.off_vh);
+        cp.kq = (float *)(ws + L.off_kq); cp.kmn = (float *)(ws + L.off_kmn);
+        cp.vi = (float *)(ws + L.off_vi);
         cp.cu = cu; cp.cfirst = cfirst;
         cp.n_seqs = n_seqs; cp.n_qk = cfg->n_qk_heads; cp.n_v = cfg->n_v_heads;
         cp.q_scale = cfg->q_scale; cp.eps = cfg->l2_eps;
         // bf16 inputs run the tensor-core (TF32) prefill, fp32 inputs the fp32 CUDA-core one
-        e = launch_conv_l2(cp, bf, /*tf32=*/bf, L.max_chunks, stream);
+        e = launch_conv_l2(cp, bf, /*tiles=*/bf, L.max_chunks, stream);
         if (e != cudaSuccess) return cuda_fail(e);
     }
     if (conv_state_out) {
@@ -199,8 +207,11 @@ gdn_status gdn_prefill(const gdn_config *cfg, gdn_dtype dtype, gdn_dtype out_dty
     ScanParams sp{};
     sp.qh = (const float *)(ws + L.off_qh); sp.kh = (const float *)(ws + L.off_kh);
     sp.vh = (const float *)(ws + L.off_vh);
+    sp.kq = (const float *)(ws + L.off_kq); sp.kmn = (const float *)(ws + L.off_kmn);
+    sp.vi = (const float *)(ws + L.off_vi);
     sp.alpha = alpha; sp.beta = beta; sp.cu = cu; sp.cfirst = cfirst;
-    sp.tb = (float *)(ws + L.off_tb); sp.pm = (float *)(ws + L.off_pm); sp.max_chunks = L.max_chunks;
+    sp.kt = (float *)(ws + L.off_kt); sp.tb = (float *)(ws + L.off_tb); sp.w2 = (float *)(ws + L.off_w2);
+    sp.pm = (float *)(ws + L.off_pm); sp.gr = (float *)(ws + L.off_gr); sp.max_chunks = L.max_chunks;
     sp.init = initial_state; sp.fin = final_state; sp.out = out;
     sp.n_seqs = n_seqs; sp.n_qk = cfg->n_qk_heads; sp.n_v = cfg->n_v_heads;
     if (bf) {

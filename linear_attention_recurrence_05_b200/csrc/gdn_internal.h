@@ -22,11 +22,20 @@ struct PrefillLayout {
     int64_t max_chunks;   // upper bound of sum_b ceil(L_b / 64)
     size_t off_cu;        // int32 [n_seqs+1]   clamped, non-decreasing sequence bounds
     size_t off_cfirst;    // int32 [n_seqs+1]   first chunk index of each sequence
+    // fp32 path: conv + L2 rows
     size_t off_qh;        // [T, Hqk, 128] fp32 conv + L2 output
     size_t off_kh;        // [T, Hqk, 128]
     size_t off_vh;        // [T, Hv, 128]
-    size_t off_tb;        // tensor-core path: [max_chunks, Hv, 64, 64] fp32 T diag(beta) tiles
-    size_t off_pm;        // tensor-core path: [max_chunks, Hv, 64, 64] fp32 P tiles
+    // tensor-core path: per-chunk tiles already in the shared-memory layout of the kernels
+    // that read them (so each is one contiguous bulk copy); rows past a sequence's end are 0
+    size_t off_kq;        // [max_chunks, Hqk] x 64 KB: [K;Q], K-major 128B-swizzled blocks
+    size_t off_kmn;       // [max_chunks, Hqk] x 32 KB: K, MN-major 32B-granule swizzle
+    size_t off_vi;        // [max_chunks, Hv]  x 32 KB: V, MN-major 32B-granule swizzle
+    size_t off_kt;        // [max_chunks, Hv]  x 32 KB: K~ = diag(kd) K, MN-major like off_kmn
+    size_t off_tb;        // [max_chunks, Hv]  x 16 KB: T diag(beta), K-major 128B-swizzled
+    size_t off_w2;        // [max_chunks, Hv]  x 16 KB: T diag(beta gamma), same
+    size_t off_pm;        // [max_chunks, Hv]  x 16 KB: P, same
+    size_t off_gr;        // [max_chunks, Hv]  x 640 B: gates record (gamma[64], kd[64], gamma_C)
     size_t bytes;
 };
 
@@ -36,18 +45,20 @@ struct ConvParams {
     const void *q, *k, *v;                 // raw rows
     const float *wq, *wk, *wv;             // [ch, 4]
     const void *conv_in;                   // [n_seqs, 3, channels] or null
-    float *qh, *kh, *vh;                   // fp32 outputs
+    float *qh, *kh, *vh;                   // fp32 rows (fp32 path)
+    float *kq, *kmn, *vi;                  // chunk tiles (tensor-core path), or null
     const int32_t *cu, *cfirst;            // workspace tables
     int n_seqs, n_qk, n_v;
     float q_scale, eps;
 };
 
 struct ScanParams {
-    const float *qh, *kh, *vh;             // fp32 conv + L2 rows [T, H, 128]
+    const float *qh, *kh, *vh;             // fp32 conv + L2 rows [T, H, 128] (fp32 path)
+    const float *kq, *kmn, *vi;            // chunk tiles (tensor-core path)
     const void *alpha, *beta;              // [T, Hv]
     const int32_t *cu;                     // clamped bounds [n_seqs+1]
     const int32_t *cfirst;                 // first chunk index of each sequence [n_seqs+1]
-    float *tb, *pm;                        // chunk-prep tiles (tensor-core path)
+    float *kt, *tb, *w2, *pm, *gr;         // chunk-prep tiles and gates records (tensor-core path)
     int64_t max_chunks;
     const float *init;                     // [n_seqs, Hv, 128, 128] or null
     float *fin;                            // or null
@@ -70,10 +81,15 @@ struct DecodeParams {
 // remembers `e` as this host thread's gdn_last_cuda_error()
 void record_cuda_error(cudaError_t e);
 
+// gates record of one (chunk, V head), written by the chunk prep for the chain kernel
+constexpr int kGateRec = 160;            // floats: gamma_t [64], kd_t [64], gamma_C, padding
+constexpr int kGrGamma = 0, kGrKd = 64, kGrGammaC = 128;
+
 // launchers: return the cudaError_t of the launch
 cudaError_t launch_seq_table(const int32_t *cu_in, int n_seqs, int64_t T, int32_t *cu,
                              int32_t *cfirst, cudaStream_t s);
-cudaError_t launch_conv_l2(const ConvParams &p, bool bf16, bool tf32, int64_t max_chunks,
+// tiles: write the tensor-core chunk tiles (TF32-rounded) instead of fp32 rows
+cudaError_t launch_conv_l2(const ConvParams &p, bool bf16, bool tiles, int64_t max_chunks,
                            cudaStream_t s);
 cudaError_t launch_conv_state_out(const void *q, const void *k, const void *v,
                                   const void *conv_in, void *conv_out, const int32_t *cu,

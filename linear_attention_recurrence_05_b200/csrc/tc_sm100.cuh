@@ -236,10 +236,12 @@ __device__ __forceinline__ uint32_t taddr(uint32_t base, int lane, int col) {
 }
 
 // ------------------------------------------------------------------ tf32 rounding
+// Round a finite fp32 value to TF32 (10 explicit mantissa bits), nearest with ties away
+// from zero: add half a unit of the kept last place to the magnitude bits, then drop the 13
+// low bits.  Two integer ops on the ALU pipe (a carry into the exponent is the correct
+// rounding up to the next binade).
 __device__ __forceinline__ float to_tf32(float x) {
-    uint32_t r;
-    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
-    return __uint_as_float(r);
+    return __uint_as_float((__float_as_uint(x) + 0x1000u) & 0xFFFFE000u);
 }
 
 // ------------------------------------------------------------------ TMA (no multicast)
@@ -257,6 +259,32 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const void *tmap, int 
         "l"(tmap), "r"(x), "r"(y), "r"(smem_u32(m))
         : "memory");
 }
+
+// contiguous bulk copy global -> shared (this CTA), completion counted on mbarrier `m`;
+// both addresses 16-byte aligned, `bytes` a multiple of 16
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_t bytes, uint64_t *m) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+        "l"(src), "r"(bytes), "r"(smem_u32(m))
+        : "memory");
+}
+// 2D tile store shared (this CTA) -> global, tracked as a bulk async-group of this thread
+__device__ __forceinline__ void tma_store_2d(const void *tmap, int x, int y, uint32_t src) {
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(tmap),
+                 "r"(x), "r"(y), "r"(src)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// wait until this thread's bulk groups have finished reading shared memory
+__device__ __forceinline__ void bulk_wait_read0() {
+    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+// wait until at most one of this thread's bulk groups is still reading shared memory
+__device__ __forceinline__ void bulk_wait_read1() {
+    asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+}
+// wait until this thread's bulk groups are complete
+__device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 // ------------------------------------------------------------------ cp.async (16 B)
 __device__ __forceinline__ void cp_async16(uint32_t dst_smem, const void *src) {

@@ -34,4 +34,17 @@ inline bool encode_rows(CUtensorMap *m, const float *base, int64_t width, int64_
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// general 2-D map: [rows x width] elements of `dt`, row stride row_bytes, box box_w x box_h
+inline bool encode_2d(CUtensorMap *m, CUtensorMapDataType dt, const void *base, int64_t width,
+                      int64_t rows, int64_t row_bytes, uint32_t box_w, uint32_t box_h,
+                      CUtensorMapSwizzle swz) {
+    auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)width, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)row_bytes};
+    cuuint32_t box[2] = {box_w, box_h}, es[2] = {1, 1};
+    return enc(m, dt, 2, (void *)base, dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace gdn
