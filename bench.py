@@ -44,6 +44,9 @@ CHUNK = 64
 # W.S, K~^T.u, Q.S (2 d^2 each) + T.(beta gamma K), T.(beta V), P.u (2 C d each)
 # + K.K^T and Q.K^T (2 C d each, shared by the 3 V heads of a QK head)
 PREFILL_FLOP_TV = 6 * D * D + 2 * CHUNK * D * (3 + 2 / 3)
+# tensor-core work of the chunk-chain kernel per (token, V head): S^T[K;Q]^T (4 d^2),
+# V^T T_beta^T and X W2^T (2 C d each), u^T K~ (2 d^2), u^T P^T (2 C d)
+CHAIN_FLOP_TV = 6 * D * D + 3 * 2 * CHUNK * D
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
                   "sm_max_mhz": 1965.0}
 TF32_PER_BF16 = 1.1 / 2.25   # nominal dense tf32 : bf16 tensor throughput on B200
@@ -268,7 +271,7 @@ def prefill_roofline(res, peaks, peak_src):
                 "peak_source": f"148 SMs x 128 fp32 FMA lanes x 2 x {peaks.get('sm_max_mhz')} MHz",
                 "algorithmic_per_launch": flops, "kernel_share": share}
     if dom.startswith("prefill_tc"):
-        flops = PREFILL_FLOP_TV * T * Hv
+        flops = CHAIN_FLOP_TV * T * Hv
         peak = peaks["bf16_tflops"] * TF32_PER_BF16
         return {"kernel": dom, "bound": "tensor", "achieved": flops / avg_s / 1e12, "peak": peak,
                 "unit": "TFLOP/s", "frac": flops / avg_s / 1e12 / peak, "traffic": None,

@@ -11,7 +11,7 @@
 // T_beta, W2 and P (64 x 64) and K~ (64 x 128) are written as fp32 tiles rounded to TF32 (the
 // precision the tensor-core chain reads them in), already in the shared-memory layout of
 // an MMA operand (T_beta, W2, P: K-major, 128-byte rows with 16-byte chunks XOR-swizzled by
-// row; K~: MN-major with 32-byte granules), for the chain kernel to stream in with one bulk
+// row; K~: MN-major with 32-byte granules, like the V tile), for the chain kernel to stream in with one bulk
 // copy each.  A gates record per (chunk, head) carries gamma_t, kd_t and gamma_C = exp(g_{n-1}).
 //
 // One CTA per (chunk, V head), 256 threads, about 70 KB of shared memory (three CTAs per

@@ -90,7 +90,7 @@ cudaError_t launch_seq_table(const int32_t *cu_in, int n_seqs, int64_t T, int32_
 // the shared-memory layouts the tensor-core kernels copy them into:
 //   [K;Q] of (chunk, QK head): 4 blocks of 32 features x (K 64 rows | Q 64 rows), 128-byte
 //     rows with 16-byte chunks XOR-swizzled by row (K-major operand layout);
-//   K and V of (chunk, head): 4 blocks of 32 features x 64 rows, 128-byte rows with 32-byte
+//   V of (chunk, V head): 4 blocks of 32 features x 64 rows, 128-byte rows with 32-byte
 //     granules XOR-swizzled by row (MN-major operand layout).
 // Rows past the end of the sequence are written as zeros.
 template <class T, bool kTiles>
@@ -136,13 +136,12 @@ __global__ void __launch_bounds__(128) conv_l2_kernel(ConvParams p) {
     const int re = min(rs + 16, r0 + len);
     if (!kTiles && rs >= re) return;
     // tile destinations (float offsets of this lane's 4 features, row 0)
-    float *t_a = nullptr, *t_b = nullptr;          // K-major ([K;Q]) and MN-major (K or V) tile
+    float *t_a = nullptr, *t_b = nullptr;          // K-major ([K;Q]) and MN-major (V) tile
     if (kTiles) {
         if (slot < p.n_qk) {
             t_a = p.kq + ((int64_t)ci * p.n_qk + slot) * 16384 + 2048;
         } else if (slot < 2 * p.n_qk) {
             t_a = p.kq + ((int64_t)ci * p.n_qk + slot - p.n_qk) * 16384;
-            t_b = p.kmn + ((int64_t)ci * p.n_qk + slot - p.n_qk) * 8192;
         } else {
             t_b = p.vi + ((int64_t)ci * p.n_v + slot - 2 * p.n_qk) * 8192;
         }

@@ -48,7 +48,6 @@ PrefillLayout prefill_layout(int n_qk, int n_v, int64_t T, int n_seqs, bool tc) 
     L.off_vh = off;      off = align_up(off + v_bytes, 256);
     const size_t nc = tc && T > 0 ? (size_t)L.max_chunks : 0;
     L.off_kq = off;      off = align_up(off + nc * n_qk * 65536, 256);
-    L.off_kmn = off;     off = align_up(off + nc * n_qk * 32768, 256);
     L.off_vi = off;      off = align_up(off + nc * n_v * 32768, 256);
     L.off_kt = off;      off = align_up(off + nc * n_v * 32768, 256);
     L.off_tb = off;      off = align_up(off + nc * n_v * 16384, 256);
@@ -190,8 +189,7 @@ gdn_status gdn_prefill(const gdn_config *cfg, gdn_dtype dtype, gdn_dtype out_dty
         cp.conv_in = conv_state_in;
         cp.qh = (float *)(ws + L.off_qh); cp.kh = (float *)(ws + L.off_kh);
         cp.vh = (float *)(ws + L.off_vh);
-        cp.kq = (float *)(ws + L.off_kq); cp.kmn = (float *)(ws + L.off_kmn);
-        cp.vi = (float *)(ws + L.off_vi);
+        cp.kq = (float *)(ws + L.off_kq); cp.vi = (float *)(ws + L.off_vi);
         cp.cu = cu; cp.cfirst = cfirst;
         cp.n_seqs = n_seqs; cp.n_qk = cfg->n_qk_heads; cp.n_v = cfg->n_v_heads;
         cp.q_scale = cfg->q_scale; cp.eps = cfg->l2_eps;
@@ -207,8 +205,7 @@ gdn_status gdn_prefill(const gdn_config *cfg, gdn_dtype dtype, gdn_dtype out_dty
     ScanParams sp{};
     sp.qh = (const float *)(ws + L.off_qh); sp.kh = (const float *)(ws + L.off_kh);
     sp.vh = (const float *)(ws + L.off_vh);
-    sp.kq = (const float *)(ws + L.off_kq); sp.kmn = (const float *)(ws + L.off_kmn);
-    sp.vi = (const float *)(ws + L.off_vi);
+    sp.kq = (const float *)(ws + L.off_kq); sp.vi = (const float *)(ws + L.off_vi);
     sp.alpha = alpha; sp.beta = beta; sp.cu = cu; sp.cfirst = cfirst;
     sp.kt = (float *)(ws + L.off_kt); sp.tb = (float *)(ws + L.off_tb); sp.w2 = (float *)(ws + L.off_w2);
     sp.pm = (float *)(ws + L.off_pm); sp.gr = (float *)(ws + L.off_gr); sp.max_chunks = L.max_chunks;

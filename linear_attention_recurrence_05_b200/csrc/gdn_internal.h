@@ -29,9 +29,8 @@ struct PrefillLayout {
     // tensor-core path: per-chunk tiles already in the shared-memory layout of the kernels
     // that read them (so each is one contiguous bulk copy); rows past a sequence's end are 0
     size_t off_kq;        // [max_chunks, Hqk] x 64 KB: [K;Q], K-major 128B-swizzled blocks
-    size_t off_kmn;       // [max_chunks, Hqk] x 32 KB: K, MN-major 32B-granule swizzle
     size_t off_vi;        // [max_chunks, Hv]  x 32 KB: V, MN-major 32B-granule swizzle
-    size_t off_kt;        // [max_chunks, Hv]  x 32 KB: K~ = diag(kd) K, MN-major like off_kmn
+    size_t off_kt;        // [max_chunks, Hv]  x 32 KB: K~ = diag(kd) K, MN-major like off_vi
     size_t off_tb;        // [max_chunks, Hv]  x 16 KB: T diag(beta), K-major 128B-swizzled
     size_t off_w2;        // [max_chunks, Hv]  x 16 KB: T diag(beta gamma), same
     size_t off_pm;        // [max_chunks, Hv]  x 16 KB: P, same
@@ -46,7 +45,7 @@ struct ConvParams {
     const float *wq, *wk, *wv;             // [ch, 4]
     const void *conv_in;                   // [n_seqs, 3, channels] or null
     float *qh, *kh, *vh;                   // fp32 rows (fp32 path)
-    float *kq, *kmn, *vi;                  // chunk tiles (tensor-core path), or null
+    float *kq, *vi;                        // chunk tiles (tensor-core path), or null
     const int32_t *cu, *cfirst;            // workspace tables
     int n_seqs, n_qk, n_v;
     float q_scale, eps;
@@ -54,7 +53,7 @@ struct ConvParams {
 
 struct ScanParams {
     const float *qh, *kh, *vh;             // fp32 conv + L2 rows [T, H, 128] (fp32 path)
-    const float *kq, *kmn, *vi;            // chunk tiles (tensor-core path)
+    const float *kq, *vi;                  // chunk tiles (tensor-core path)
     const void *alpha, *beta;              // [T, Hv]
     const int32_t *cu;                     // clamped bounds [n_seqs+1]
     const int32_t *cfirst;                 // first chunk index of each sequence [n_seqs+1]
