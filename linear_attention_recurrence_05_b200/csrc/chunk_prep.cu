@@ -190,12 +190,19 @@ __global__ void __launch_bounds__(kPThr) chunk_prep_kernel(const __grid_constant
         const bool factored = -g_s[n - 1] < kMaxChunkDecay;
         const float gt = g_s[t], rowf = gam_s[t] * (q < 2 ? beta_s[t] : 1.f), bt = q < 2 ? beta_s[t] : 1.f;
         float out[32];
+        const int lim = t < n ? (q < 2 ? t : t + 1) : 0;   // columns i < lim are kept
+        if (factored) {   // uniform per CTA
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-            const int i = 32 * ch + e;
-            const bool keep = (q < 2 ? i < t : i <= t) && t < n;
-            const float f = factored ? rowf * ig_s[i] : bt * expf(gt - g_s[i]);
-            out[e] = keep ? f * v[e] : 0.f;
+            for (int e = 0; e < 32; ++e) {
+                const int i = 32 * ch + e;
+                out[e] = i < lim ? rowf * ig_s[i] * v[e] : 0.f;
+            }
+        } else {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+                const int i = 32 * ch + e;
+                out[e] = i < lim ? bt * expf(gt - g_s[i]) * v[e] : 0.f;
+            }
         }
         if (q < 2) {
 #pragma unroll

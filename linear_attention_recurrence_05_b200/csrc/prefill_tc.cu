@@ -62,7 +62,7 @@ constexpr uint32_t kSmemAlloc = kSmem + 1024;              // slack to align the
 enum {
     B_KQ = 0, B_V, B_KMN, B_W2L, B_PL, B_TBL,   // tile arrivals
     B_GR0, B_GR1,                        // arrival of the gates record into buffer 0 / 1
-    B_1, B_2, B_34,                      // MMA completions
+    B_1, B_2, B_3, B_4,                  // MMA completions (MMA_1; 2a+2b; 3; 4)
     B_Y1,                                // epilogue: Y1 taken, Y = gamma Y1 stored, S scaled
     B_DRAIN0,                            // drain on the failure path
     kNumBars
@@ -232,6 +232,8 @@ __global__ void __launch_bounds__(kThr, 1) prefill_tc_kernel(const __grid_consta
                 fence_after_sync();
                 gemm_ts<128, 128, false, false>(tm + T_XY, tm + T_S, sb + OFF_KQ, 16384, false);
                 mma_commit(&bar[B_1]);
+                // MMA_4 of c-1 still reads u^T, which MMA_2a overwrites
+                if (c > 0 && !(ok = wait_or_abort(&bar[B_4], par ^ 1, abort_flag))) break;
                 // MMA_2a: U^T = V^T T_beta^T (state-independent)
                 if (!(ok = wait_or_abort(&bar[B_TBL], par, abort_flag))) break;
                 if (!(ok = wait_or_abort(&bar[B_V], par, abort_flag))) break;
@@ -250,9 +252,11 @@ __global__ void __launch_bounds__(kThr, 1) prefill_tc_kernel(const __grid_consta
                 if (!(ok = wait_or_abort(&bar[B_PL], par, abort_flag))) break;
                 fence_after_sync();
                 gemm_ts<128, 64, true, false>(tm + T_S, tm + T_U, sb + OFF_KMN, 64, true);
+                mma_commit(&bar[B_3]);
                 gemm_ts<64, 64, false, false>(tm + T_Y, tm + T_U, sb + OFF_P, 8192, true);
-                mma_commit(&bar[B_34]);
-                if (!(ok = wait_or_abort(&bar[B_34], par, abort_flag))) break;
+                mma_commit(&bar[B_4]);
+                // the next MMA_1 needs S only; it queues behind MMA_4 in the tensor pipe
+                if (!(ok = wait_or_abort(&bar[B_3], par, abort_flag))) break;
             }
             if (!ok) {  // drain this thread's MMAs (bounded)
                 mma_commit(&bar[B_DRAIN0]);
@@ -277,11 +281,13 @@ __global__ void __launch_bounds__(kThr, 1) prefill_tc_kernel(const __grid_consta
                     issue_tb(c + 1); ++n_tb;
                     issue_w2(c + 1); ++n_w2;
                 }
-                // K~, P, and this gates buffer once MMA_3/4 of c are done (the epilogue took
-                // its gates before MMA_3 could start)
-                if (!(ok = wait_or_abort(&bar[B_34], par, abort_flag))) break;
-                if (c + 1 < nchunks) { issue_kmn(c + 1); ++n_kmn; issue_pm(c + 1); ++n_pm; }
+                // K~ and this gates buffer once MMA_3 of c is done (the epilogue took its gates
+                // before MMA_3 could start); P once MMA_4 of c is done
+                if (!(ok = wait_or_abort(&bar[B_3], par, abort_flag))) break;
+                if (c + 1 < nchunks) { issue_kmn(c + 1); ++n_kmn; }
                 if (c + 2 < nchunks) { issue_gr(c + 2); ++n_gr[c & 1]; }
+                if (!(ok = wait_or_abort(&bar[B_4], par, abort_flag))) break;
+                if (c + 1 < nchunks) { issue_pm(c + 1); ++n_pm; }
             }
             if (!ok) {  // wait (bounded) for the copies this thread started
                 const int counts[6] = {n_kq, n_v, n_kmn, n_w2, n_pm, n_tb};
@@ -335,7 +341,7 @@ __global__ void __launch_bounds__(kThr, 1) prefill_tc_kernel(const __grid_consta
             fence_before_sync();
             bar_sync(kBarEpi, 128);
             if (leader) mbar_arrive(&bar[B_Y1]);
-            if (!ewait(B_34, par)) break;
+            if (!ewait(B_4, par)) break;
             fence_after_sync();
             if (n == kChunk) {
                 // full chunk: rows 32*h2.. staged in buffer h2 (row t, column j) and written
