@@ -50,6 +50,9 @@ CHAIN_FLOP_TV = 6 * D * D + 3 * 2 * CHUNK * D
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
                   "sm_max_mhz": 1965.0}
 TF32_PER_BF16 = 1.1 / 2.25   # nominal dense tf32 : bf16 tensor throughput on B200
+# dram__bytes_read.sum + dram__bytes_write.sum per launch from one ncu capture of the current
+# kernels on this workload (profiles/prefill_tc_T8192_ncu.md, profiles/decode_B256_ncu.md)
+NCU_TRAFFIC_BYTES = {"prefill_tc": 842_870_784 + 186_638_336, "decode": 826_713_088 + 769_751_552}
 FP32_LANES_PER_SM = 128
 N_SM = 148
 
@@ -274,7 +277,8 @@ def prefill_roofline(res, peaks, peak_src):
         flops = CHAIN_FLOP_TV * T * Hv
         peak = peaks["bf16_tflops"] * TF32_PER_BF16
         return {"kernel": dom, "bound": "tensor", "achieved": flops / avg_s / 1e12, "peak": peak,
-                "unit": "TFLOP/s", "frac": flops / avg_s / 1e12 / peak, "traffic": None,
+                "unit": "TFLOP/s", "frac": flops / avg_s / 1e12 / peak,
+                "traffic": NCU_TRAFFIC_BYTES.get("prefill_tc"),
                 "peak_source": f"tf32 = {peak_src} bf16 {peaks['bf16_tflops']} x 1.1/2.25 nominal",
                 "algorithmic_per_launch": flops, "kernel_share": share}
     # a memory-bound kernel dominates
@@ -385,7 +389,7 @@ def bench_decode(args, dist, torch, gdn, peaks, peak_src):
         "steps": steps, "ms_per_step": ms / steps, "launches": trace.count, "clocks": clk,
         "roofline": {"kernel": "decode", "bound": "hbm", "achieved": achieved,
                      "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
-                     "traffic": None, "peak_source": peak_src,
+                     "traffic": NCU_TRAFFIC_BYTES.get("decode"), "peak_source": peak_src,
                      "algorithmic_bytes_per_row": bpr, "rows_per_launch": B},
         "e2e": {"value": toks / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "note": "host inputs cycle through 32 pinned step sets"},
