@@ -69,6 +69,7 @@ struct PrepParams {
     float *tb, *w2, *pm;  // [chunk, Hv] tiles (16 KB each)
     float *gr;            // [chunk, Hv] gates records
     int n_seqs, n_qk, n_v;
+    int64_t chunk_lo;     // first global chunk index of this launch
 };
 
 }  // namespace
@@ -76,7 +77,7 @@ struct PrepParams {
 template <class TI>
 __global__ void __launch_bounds__(kPThr) chunk_prep_kernel(const __grid_constant__ PrepParams p) {
     const int h = blockIdx.x % p.n_v;
-    const int u = blockIdx.x / p.n_v;                  // global chunk index
+    const int u = (int)(p.chunk_lo + blockIdx.x / p.n_v);   // global chunk index
     if (u >= p.cfirst[p.n_seqs]) return;               // uniform per CTA
     const int b = upper_index(p.cfirst, p.n_seqs, u);
     const int seq0 = p.cu[b];
@@ -333,7 +334,9 @@ cudaError_t launch_chunk_prep(const ScanParams &sp, int64_t total_tokens, bool i
     p.kq = sp.kq; p.kt = sp.kt;
     p.alpha = sp.alpha; p.beta = sp.beta; p.cu = sp.cu; p.cfirst = sp.cfirst;
     p.tb = sp.tb; p.w2 = sp.w2; p.pm = sp.pm; p.gr = sp.gr; p.n_seqs = sp.n_seqs; p.n_qk = sp.n_qk; p.n_v = sp.n_v;
-    const int64_t grid = sp.max_chunks * sp.n_v;
+    p.chunk_lo = sp.chunk_lo;
+    const int64_t grid = (sp.chunk_hi - sp.chunk_lo) * sp.n_v;
+    if (grid <= 0) return cudaSuccess;
     if (grid >= ((int64_t)1 << 31)) return cudaErrorInvalidValue;
     auto k = in_bf16 ? chunk_prep_kernel<bf16> : chunk_prep_kernel<float>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kPSmemAlloc);

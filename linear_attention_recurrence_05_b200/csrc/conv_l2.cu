@@ -96,7 +96,7 @@ cudaError_t launch_seq_table(const int32_t *cu_in, int n_seqs, int64_t T, int32_
 template <class T, bool kTiles>
 __global__ void __launch_bounds__(128) conv_l2_kernel(ConvParams p) {
     const int n_chunks = p.cfirst[p.n_seqs];
-    const int ci = blockIdx.x;
+    const int ci = (int)(p.chunk_lo + blockIdx.x);
     if (ci >= n_chunks) return;
     const int b = upper_index(p.cfirst, p.n_seqs, ci);
     const int seq0 = p.cu[b], seq1 = p.cu[b + 1];
@@ -195,10 +195,10 @@ __global__ void __launch_bounds__(128) conv_l2_kernel(ConvParams p) {
     }
 }
 
-cudaError_t launch_conv_l2(const ConvParams &p, bool bf16, bool tiles, int64_t max_chunks,
+cudaError_t launch_conv_l2(const ConvParams &p, bool bf16, bool tiles, int64_t n_chunks,
                            cudaStream_t s) {
-    if (max_chunks <= 0) return cudaSuccess;
-    dim3 grid((unsigned)max_chunks, 2 * p.n_qk + p.n_v);
+    if (n_chunks <= 0) return cudaSuccess;
+    dim3 grid((unsigned)n_chunks, 2 * p.n_qk + p.n_v);
     TraceLaunch tl(s, "conv_l2");
     if (bf16) {
         if (tiles) conv_l2_kernel<gdn::bf16, true><<<grid, 128, 0, s>>>(p);

@@ -1,5 +1,6 @@
 // C ABI of libgdn: argument validation, workspace layout and kernel launches.
 // The declarations and the contract of every entry point are in include/libgdn.h.
+#include <algorithm>
 #include <cmath>
 #include <cstring>
 
@@ -54,8 +55,46 @@ PrefillLayout prefill_layout(int n_qk, int n_v, int64_t T, int n_seqs, bool tc) 
     L.off_w2 = off;      off = align_up(off + nc * n_v * 16384, 256);
     L.off_pm = off;      off = align_up(off + nc * n_v * 16384, 256);
     L.off_gr = off;      off = align_up(off + nc * n_v * kGateRec * sizeof(float), 256);
+    L.n_segments = tc && T > 0 ? plan_segments(n_v, n_seqs, L.max_chunks) : 1;
+    const size_t carry = L.n_segments > 1 ? (size_t)n_seqs * n_v * 128 * 128 * sizeof(float) : 0;
+    L.off_carry = off;   off = align_up(off + carry, 256);
     L.bytes = off;
     return L;
+}
+
+int plan_segments(int n_v, int n_seqs, int64_t max_chunks) {
+    if ((int64_t)n_seqs * n_v > kSegMaxChains || max_chunks < 2 * kSegMinChunks) return 1;
+    return (int)std::min<int64_t>(kSegMax, max_chunks / kSegMinChunks);
+}
+
+// One auxiliary stream and a few events per (host thread, device) for the pipelined path.
+struct AuxStream {
+    cudaStream_t stream = nullptr;
+    cudaEvent_t ev[kSegMax + 2] = {};
+};
+static thread_local AuxStream t_aux[64];
+
+static cudaError_t aux_stream(AuxStream **out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    AuxStream &a = t_aux[dev];
+    if (!a.stream) {
+        AuxStream fresh;
+        e = cudaStreamCreateWithFlags(&fresh.stream, cudaStreamNonBlocking);
+        for (auto &ev : fresh.ev)
+            if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ev, cudaEventDisableTiming);
+        if (e != cudaSuccess) {
+            for (auto &ev : fresh.ev)
+                if (ev) cudaEventDestroy(ev);
+            if (fresh.stream) cudaStreamDestroy(fresh.stream);
+            return e;
+        }
+        a = fresh;
+    }
+    *out = &a;
+    return cudaSuccess;
 }
 
 }  // namespace gdn
@@ -182,8 +221,8 @@ gdn_status gdn_prefill(const gdn_config *cfg, gdn_dtype dtype, gdn_dtype out_dty
     cudaError_t e = launch_seq_table(cu_seqlens, n_seqs, total_tokens, cu, cfirst, stream);
     if (e != cudaSuccess) return cuda_fail(e);
 
+    ConvParams cp{};
     if (total_tokens > 0) {
-        ConvParams cp{};
         cp.q = q; cp.k = k; cp.v = v;
         cp.wq = conv_w_q; cp.wk = conv_w_k; cp.wv = conv_w_v;
         cp.conv_in = conv_state_in;
@@ -193,9 +232,12 @@ gdn_status gdn_prefill(const gdn_config *cfg, gdn_dtype dtype, gdn_dtype out_dty
         cp.cu = cu; cp.cfirst = cfirst;
         cp.n_seqs = n_seqs; cp.n_qk = cfg->n_qk_heads; cp.n_v = cfg->n_v_heads;
         cp.q_scale = cfg->q_scale; cp.eps = cfg->l2_eps;
-        // bf16 inputs run the tensor-core (TF32) prefill, fp32 inputs the fp32 CUDA-core one
-        e = launch_conv_l2(cp, bf, /*tiles=*/bf, L.max_chunks, stream);
-        if (e != cudaSuccess) return cuda_fail(e);
+        // bf16 inputs run the tensor-core (TF32) prefill, fp32 inputs the fp32 CUDA-core one;
+        // the pipelined tensor-core path launches the conv per chunk range below
+        if (L.n_segments == 1) {
+            e = launch_conv_l2(cp, bf, /*tiles=*/bf, L.max_chunks, stream);
+            if (e != cudaSuccess) return cuda_fail(e);
+        }
     }
     if (conv_state_out) {
         e = launch_conv_state_out(q, k, v, conv_state_in, conv_state_out, cu, n_seqs,
@@ -212,12 +254,39 @@ gdn_status gdn_prefill(const gdn_config *cfg, gdn_dtype dtype, gdn_dtype out_dty
     sp.init = initial_state; sp.fin = final_state; sp.out = out;
     sp.n_seqs = n_seqs; sp.n_qk = cfg->n_qk_heads; sp.n_v = cfg->n_v_heads;
     if (bf) {
-        // state-independent chunk work for every (chunk, V head) at once, then the chunk chain
-        if (total_tokens > 0) {
-            e = launch_chunk_prep(sp, total_tokens, bf, stream);
+        sp.carry_in = sp.carry_out = final_state;
+        if (L.n_segments == 1) {
+            // state-independent chunk work for every (chunk, V head) at once, then the chains
+            sp.chunk_lo = 0;
+            sp.chunk_hi = L.max_chunks;
+            if (total_tokens > 0) {
+                e = launch_chunk_prep(sp, total_tokens, bf, stream);
+                if (e != cudaSuccess) return cuda_fail(e);
+            }
+            e = launch_prefill_tc(sp, total_tokens, bf, out_dtype == GDN_BF16, stream);
+        } else {
+            // pipeline over chunk ranges: conv + chunk prep of range s on the auxiliary
+            // stream, the chains of range s on the caller's stream once its prep is done;
+            // the state passes from range to range through the final-state buffer (or a
+            // workspace copy)
+            if (!final_state) sp.carry_in = sp.carry_out = (float *)(ws + L.off_carry);
+            AuxStream *aux = nullptr;
+            e = aux_stream(&aux);
             if (e != cudaSuccess) return cuda_fail(e);
+            const int64_t per = (L.max_chunks + L.n_segments - 1) / L.n_segments;
+            e = cudaEventRecord(aux->ev[0], stream);  // the sequence tables are ready
+            if (e == cudaSuccess) e = cudaStreamWaitEvent(aux->stream, aux->ev[0], 0);
+            for (int sg = 0; sg < L.n_segments && e == cudaSuccess; ++sg) {
+                const int64_t lo = sg * per, hi = std::min<int64_t>(L.max_chunks, lo + per);
+                cp.chunk_lo = sp.chunk_lo = lo;
+                sp.chunk_hi = hi;
+                e = launch_conv_l2(cp, bf, /*tiles=*/true, hi - lo, aux->stream);
+                if (e == cudaSuccess) e = launch_chunk_prep(sp, total_tokens, bf, aux->stream);
+                if (e == cudaSuccess) e = cudaEventRecord(aux->ev[1 + sg], aux->stream);
+                if (e == cudaSuccess) e = cudaStreamWaitEvent(stream, aux->ev[1 + sg], 0);
+                if (e == cudaSuccess) e = launch_prefill_tc(sp, total_tokens, bf, out_dtype == GDN_BF16, stream);
+            }
         }
-        e = launch_prefill_tc(sp, total_tokens, bf, out_dtype == GDN_BF16, stream);
     } else {
         e = launch_scan_simt(sp, bf, out_dtype == GDN_BF16, stream);
     }

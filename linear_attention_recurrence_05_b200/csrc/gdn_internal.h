@@ -35,10 +35,21 @@ struct PrefillLayout {
     size_t off_w2;        // [max_chunks, Hv]  x 16 KB: T diag(beta gamma), same
     size_t off_pm;        // [max_chunks, Hv]  x 16 KB: P, same
     size_t off_gr;        // [max_chunks, Hv]  x 640 B: gates record (gamma[64], kd[64], gamma_C)
+    size_t off_carry;     // [n_seqs, Hv, 128, 128] fp32 state between chunk ranges (segmented
+                          // tensor-core path without a caller final-state buffer), else empty
+    int n_segments;       // tensor-core path: chunk ranges run as a pipeline (1 = one pass)
     size_t bytes;
 };
 
 PrefillLayout prefill_layout(int n_qk, int n_v, int64_t T, int n_seqs, bool tc);
+
+// Few (sequence, V head) chains leave most SMs idle while they run; the chunks are then
+// cut into ranges so that the conv and chunk prep of range s+1 run on the idle SMs while
+// the chains run range s.
+constexpr int64_t kSegMaxChains = 96;     // at most this many chains (148 SMs)
+constexpr int64_t kSegMinChunks = 32;     // chunks per range at least
+constexpr int kSegMax = 8;                // ranges at most
+int plan_segments(int n_v, int n_seqs, int64_t max_chunks);
 
 struct ConvParams {
     const void *q, *k, *v;                 // raw rows
@@ -49,6 +60,7 @@ struct ConvParams {
     const int32_t *cu, *cfirst;            // workspace tables
     int n_seqs, n_qk, n_v;
     float q_scale, eps;
+    int64_t chunk_lo;                      // first global chunk index of this launch
 };
 
 struct ScanParams {
@@ -59,6 +71,10 @@ struct ScanParams {
     const int32_t *cfirst;                 // first chunk index of each sequence [n_seqs+1]
     float *kt, *tb, *w2, *pm, *gr;         // chunk-prep tiles and gates records (tensor-core path)
     int64_t max_chunks;
+    int64_t chunk_lo, chunk_hi;            // global chunk range of one launch (tensor-core path)
+    const float *carry_in;                 // state entering a chunk range that starts inside a
+                                           // sequence (the previous range's output), or null
+    float *carry_out;                      // state at the end of the range (fin or a workspace copy)
     const float *init;                     // [n_seqs, Hv, 128, 128] or null
     float *fin;                            // or null
     void *out;                             // [T, Hv, 128]
@@ -88,7 +104,7 @@ constexpr int kGrGamma = 0, kGrKd = 64, kGrGammaC = 128;
 cudaError_t launch_seq_table(const int32_t *cu_in, int n_seqs, int64_t T, int32_t *cu,
                              int32_t *cfirst, cudaStream_t s);
 // tiles: write the tensor-core chunk tiles (TF32-rounded) instead of fp32 rows
-cudaError_t launch_conv_l2(const ConvParams &p, bool bf16, bool tiles, int64_t max_chunks,
+cudaError_t launch_conv_l2(const ConvParams &p, bool bf16, bool tiles, int64_t n_chunks,
                            cudaStream_t s);
 cudaError_t launch_conv_state_out(const void *q, const void *k, const void *v,
                                   const void *conv_in, void *conv_out, const int32_t *cu,

@@ -138,10 +138,11 @@ struct TcParams {
     // W2, P and the gates record per (chunk, V head)
     const float *kq, *kt, *vi, *tb, *w2, *pm, *gr;
     const int32_t *cu, *cfirst;
-    const float *init;
-    float *fin;
+    const float *init, *carry_in;   // state entering chunk 0 / entering a later first chunk
+    float *carry_out;               // state after the last chunk of the launch
     void *out;
     int n_seqs, n_qk, n_v;
+    int64_t chunk_lo, chunk_hi;     // global chunk range of the launch
 };
 
 template <class TO>
@@ -158,8 +159,15 @@ __global__ void __launch_bounds__(kThr, 1) prefill_tc_kernel(const __grid_consta
     const int b = blockIdx.x / p.n_v;
     const int gq = h / (p.n_v / p.n_qk);
     const int seq0 = p.cu[b], L = p.cu[b + 1] - p.cu[b];
-    const int nchunks = (L + kChunk - 1) / kChunk;
+    const int seq_chunks = (L + kChunk - 1) / kChunk;
     const int64_t cf = p.cfirst[b];                           // global index of chunk 0
+    // this launch's chunks of the sequence: [cb, cb + nchunks) of its seq_chunks; the state
+    // enters from the initial state (cb = 0) or from the previous launch's carry
+    const int cb = (int)max((int64_t)0, p.chunk_lo - cf);
+    const int nchunks = max(0, (int)min((int64_t)seq_chunks, p.chunk_hi - cf) - cb);
+    // nothing in range (a zero-length sequence is handled by the launch that starts at 0)
+    if (seq_chunks > 0 ? nchunks == 0 : p.chunk_lo != 0) return;   // uniform per CTA
+    const float *state_in = cb == 0 ? p.init : p.carry_in;
 
     if (tid == 0) {
         asm volatile("prefetch.tensormap [%0];" ::"l"(&p.tm_out) : "memory");
@@ -180,8 +188,9 @@ __global__ void __launch_bounds__(kThr, 1) prefill_tc_kernel(const __grid_consta
         mbar_expect_tx(&bar[bar_i], bytes);
         bulk_load(sb + dst, src, bytes, &bar[bar_i]);
     };
-    auto qk_tile = [&](const float *base, int c, int64_t floats) { return base + ((cf + c) * p.n_qk + gq) * floats; };
-    auto v_tile = [&](const float *base, int c, int64_t floats) { return base + ((cf + c) * p.n_v + h) * floats; };
+    // (c counts this launch's chunks from 0; the sequence's chunk is cb + c)
+    auto qk_tile = [&](const float *base, int c, int64_t floats) { return base + ((cf + cb + c) * p.n_qk + gq) * floats; };
+    auto v_tile = [&](const float *base, int c, int64_t floats) { return base + ((cf + cb + c) * p.n_v + h) * floats; };
     auto issue_kq = [&](int c) { load(B_KQ, OFF_KQ, qk_tile(p.kq, c, 16384), 65536); };
     auto issue_kmn = [&](int c) { load(B_KMN, OFF_KMN, v_tile(p.kt, c, 8192), 32768); };
     auto issue_v = [&](int c) { load(B_V, OFF_VMN, v_tile(p.vi, c, 8192), 32768); };
@@ -196,7 +205,7 @@ __global__ void __launch_bounds__(kThr, 1) prefill_tc_kernel(const __grid_consta
     if (warp >= kEpiWarp0 && warp < kLoadWarp) {
         const int q = warp & 3, j = 32 * q + lane;
         const uint32_t lrow = (uint32_t)(32 * q) << 16;
-        const float *src = p.init ? p.init + ((int64_t)b * p.n_v + h) * kHeadDim * kHeadDim + j : nullptr;
+        const float *src = state_in ? state_in + ((int64_t)b * p.n_v + h) * kHeadDim * kHeadDim + j : nullptr;
 #pragma unroll
         for (int d0 = 0; d0 < kHeadDim; d0 += 32) {
             float v[32];
@@ -310,8 +319,8 @@ __global__ void __launch_bounds__(kThr, 1) prefill_tc_kernel(const __grid_consta
         for (int c = 0; c < nchunks; ++c) {
             const uint32_t par = c & 1;
             const int bsel = c & 1;
-            const int n = min(kChunk, L - c * kChunk);
-            const int64_t tok = seq0 + (int64_t)c * kChunk;
+            const int n = min(kChunk, L - (cb + c) * kChunk);
+            const int64_t tok = seq0 + (int64_t)(cb + c) * kChunk;
             if (!ewait(B_1, par)) break;
             if (!ewait(B_GR0 + bsel, (c >> 1) & 1)) break;   // the gates record of c
             fence_after_sync();
@@ -406,8 +415,8 @@ __global__ void __launch_bounds__(kThr, 1) prefill_tc_kernel(const __grid_consta
         const int q = warp & 3, j = 32 * q + lane;
         const uint32_t lrow = (uint32_t)(32 * q) << 16;
         const bool failed = *abort_flag != 0;
-        if (p.fin) {
-            float *dst = p.fin + ((int64_t)b * p.n_v + h) * kHeadDim * kHeadDim + j;
+        if (p.carry_out) {
+            float *dst = p.carry_out + ((int64_t)b * p.n_v + h) * kHeadDim * kHeadDim + j;
 #pragma unroll
             for (int d0 = 0; d0 < kHeadDim; d0 += 32) {
                 float s[32];
@@ -420,7 +429,8 @@ __global__ void __launch_bounds__(kThr, 1) prefill_tc_kernel(const __grid_consta
         }
         if (failed) {
             const int64_t v_row = (int64_t)p.n_v * kHeadDim;
-            for (int e = tid - kEpiTid0; e < L * kHeadDim; e += 128) {
+            const int t0 = cb * kChunk, t1 = min(L, (cb + nchunks) * kChunk);
+            for (int e = tid - kEpiTid0 + t0 * kHeadDim; e < t1 * kHeadDim; e += 128) {
                 const int t = e / kHeadDim, jj = e % kHeadDim;
                 ((TO *)p.out)[(seq0 + t) * v_row + h * kHeadDim + jj] = from_f32<TO>(__int_as_float(0x7fc00000));
             }
@@ -454,7 +464,8 @@ cudaError_t launch_prefill_tc(const ScanParams &sp, int64_t total_tokens, bool /
     if (sp.n_seqs <= 0) return cudaSuccess;
     TcParams p{};
     p.kq = sp.kq; p.kt = sp.kt; p.vi = sp.vi; p.tb = sp.tb; p.w2 = sp.w2; p.pm = sp.pm; p.gr = sp.gr;
-    p.cu = sp.cu; p.cfirst = sp.cfirst; p.init = sp.init; p.fin = sp.fin;
+    p.cu = sp.cu; p.cfirst = sp.cfirst; p.init = sp.init; p.carry_in = sp.carry_in; p.carry_out = sp.carry_out;
+    p.chunk_lo = sp.chunk_lo; p.chunk_hi = sp.chunk_hi;
     p.out = sp.out; p.n_seqs = sp.n_seqs; p.n_qk = sp.n_qk; p.n_v = sp.n_v;
     return out_bf16 ? launch_tc_t<gdn::bf16>(p, total_tokens, s) : launch_tc_t<float>(p, total_tokens, s);
 }

@@ -62,6 +62,35 @@ def test_pages_heads_short(lib, dtype):
     _check(inp, lib, label=f"h16x48-{dtype}")
 
 
+def test_pipelined_chunk_ranges(lib):
+    """Few (sequence, head) chains and many chunks run as a pipeline over chunk ranges (the
+    state carried from range to range): sequences that start, end and lie wholly inside a
+    range, an empty one, initial states; with a final-state buffer, without one (the state is
+    carried in the workspace) and with the final state aliasing the initial state."""
+    shape = gi.GdnShape(n_qk_heads=2, n_v_heads=6)
+    inp = gi.make_prefill_inputs(shape, [1500, 0, 700, 1100, 37], gi.BF16, seed=91,
+                                 with_initial_state=True, with_conv_state=True)
+    ey, es = _check(inp, lib, label="pipelined")
+    from gdn_testutil import to_dev
+    d = inp.dtype
+    args = [to_dev(x, d) for x in (inp.q, inp.k, inp.v, inp.w_q, inp.w_k, inp.w_v, inp.alpha, inp.beta)]
+    cu = torch.from_numpy(inp.cu_seqlens).cuda()
+    cfg = lib.GdnConfig(2, 6)
+    st = torch.from_numpy(inp.initial_state).cuda()
+    cs = to_dev(inp.conv_state, d)
+    y_nofin, fin_none, _ = lib.gdn_prefill(*args, cu, cfg=cfg, initial_state=st.clone(),
+                                           return_final_state=False, conv_state_in=cs)
+    alias = st.clone()
+    y_alias, fin_alias, _ = lib.gdn_prefill(*args, cu, cfg=cfg, initial_state=alias, final_state=alias,
+                                            conv_state_in=cs)
+    torch.cuda.synchronize()
+    assert fin_none is None
+    yo, fo, _ = oracle.prefill(inp)
+    assert rel_err(to_host_f64(y_nofin), yo) <= tol(d)
+    assert rel_err(to_host_f64(y_alias), yo) <= tol(d)
+    assert rel_err(to_host_f64(fin_alias), fo) <= tol(d)
+
+
 def test_state_aliasing(lib):
     """final_state may alias initial_state and conv_state_out may alias conv_state_in."""
     shape = gi.GdnShape(n_qk_heads=2, n_v_heads=6)
