@@ -68,7 +68,8 @@ def test_pipelined_chunk_ranges(lib):
     range, an empty one, initial states; with a final-state buffer, without one (the state is
     carried in the workspace) and with the final state aliasing the initial state."""
     shape = gi.GdnShape(n_qk_heads=2, n_v_heads=6)
-    inp = gi.make_prefill_inputs(shape, [1500, 0, 700, 1100, 37], gi.BF16, seed=91,
+    # 6,137 tokens in 5 sequences: 100 chunk slots, 3 ranges of 34 (2 x 6 heads = 12 chains)
+    inp = gi.make_prefill_inputs(shape, [2500, 0, 1400, 2200, 37], gi.BF16, seed=91,
                                  with_initial_state=True, with_conv_state=True)
     ey, es = _check(inp, lib, label="pipelined")
     from gdn_testutil import to_dev
