@@ -5,21 +5,21 @@
 // FIELD NOTES", section 03 (GATED DELTANET), with g_t = sum_{s<=t} log alpha_s inside the
 // chunk, gamma_t = exp(g_t) and kd_t = exp(g_{n-1} - g_t):
 //     A_ti = beta_t exp(g_t - g_i) k_t.k_i        (i < t < n, else 0)
-//     T    = (I + A)^-1,   T_beta = T diag(beta),   W2 = T_beta diag(gamma)
+//     T    = (I + A)^-1,   T_beta = T diag(beta)
 //     P_ti = exp(g_t - g_i) q_t.k_i               (i <= t < n, else 0)
-//     K~   = diag(kd) K                            (rows t >= n zero)
-// T_beta, W2 and P (64 x 64) and K~ (64 x 128) are written as fp32 tiles rounded to TF32 (the
-// precision the tensor-core chain reads them in), already in the shared-memory layout of
-// an MMA operand (T_beta, W2, P: K-major, 128-byte rows with 16-byte chunks XOR-swizzled by
-// row; K~: MN-major with 32-byte granules, like the V tile), for the chain kernel to stream in with one bulk
-// copy each.  A gates record per (chunk, head) carries gamma_t, kd_t and gamma_C = exp(g_{n-1}).
+// T_beta and P (64 x 64) are written as fp32 tiles rounded to TF32 (the precision the
+// tensor-core chain reads them in), already in the shared-memory layout of an MMA operand
+// (K-major, 128-byte rows with 16-byte chunks XOR-swizzled by row), for the chain kernel to
+// stream in with one bulk copy each.  A gates record per (chunk, head) carries gamma_t,
+// kd_t and gamma_C = exp(g_{n-1}), the per-token factors the chain applies in tensor memory.
 //
-// One CTA per (chunk, V head), 256 threads, about 70 KB of shared memory (three CTAs per
-// SM): one bulk copy brings the chunk's [K;Q] tile, one tcgen05 MMA forms [K;Q] K^T in
-// tensor memory while the warps write K~, the warps turn K K^T and Q K^T into A and P, and
-// the inverse runs on CUDA cores in fp32 (16 x 16 diagonal blocks by forward substitution,
-// then two block-merge levels).  The [K;Q] tile's space is reused for the scratch and the
-// output staging; the tiles leave by bulk stores.
+// One CTA per (chunk, group of up to 3 V heads of one QK head): K K^T and Q K^T do not
+// depend on the gates, so one bulk copy of the chunk's [K;Q] tile and one tcgen05 MMA
+// ([K;Q] K^T into tensor memory) serve all the CTA's heads.  Each head then has a group of
+// 4 warps: the warps turn the MMA rows into A (kept in shared memory, transposed) and P
+// (stored straight to global memory), and invert I + A in registers, two threads per
+// column of T (even and odd rows) by forward substitution.  T_beta is staged over the
+// head's scratch and leaves by one bulk store.
 #include "gdn_common.cuh"
 #include "gdn_internal.h"
 #include "tc_sm100.cuh"
@@ -29,27 +29,27 @@ namespace gdn {
 namespace {
 using namespace tc;
 
-constexpr int kPThr = 256;
+constexpr int kGroupThr = 128;   // 4 warps per V head
+constexpr int kMaxGroups = 3;    // V heads per CTA
 
-// shared-memory map (bytes from a 1024-aligned base).  [0, 64 KB) first holds the [K;Q]
-// tile; once the MMA has read it and K~ has been written, it holds the scratch and staging.
-constexpr uint32_t P_KQ = 0;          // [K;Q] K-major, 4 blocks x (K 8 KB | Q 8 KB)   64 KB
-constexpr uint32_t P_AS = 0;          // A (fp32, swizzled rows), then the W2 staging   16 KB
-constexpr uint32_t P_TS = 16384;      // T (fp32, swizzled rows)                       16 KB
-constexpr uint32_t P_PST = 32768;     // P staging (K-major image)                     16 KB
-constexpr uint32_t P_TBST = 49152;    // T_beta staging (K-major image)                16 KB
-constexpr uint32_t P_INV = 65536;     // 2 x 256 floats (block products)                2 KB
-constexpr uint32_t P_GATE = 67584;    // g, beta, gamma, kd, 1/gamma: 5 x 64 floats    1280 B
-constexpr uint32_t P_BAR = 68864;     // 2 mbarriers
-constexpr uint32_t P_SLOT = 68880;    // TMEM base
+// shared-memory map (bytes from a 1024-aligned base).  [0, 64 KB) holds the [K;Q] tile until
+// the MMA has read it, then one scratch per group: -A^T split by row parity, array p holding
+// -A[2s + p][m] at row m, column s (64 x 32 floats), the odd array 64 bytes past a multiple
+// of 8 KB so that the two parities fall in different banks; after the inverse, the T_beta
+// staging (K-major image, 16 KB).
+constexpr uint32_t P_KQ = 0;
+constexpr uint32_t kParStride = 8192 + 64;
+constexpr uint32_t kScrBytes = 2 * kParStride;
+constexpr uint32_t P_GATE = 65536;                 // per group: g, beta, gamma, 1/gamma
+constexpr uint32_t kGateBytes = 4 * 64 * 4;
+constexpr uint32_t P_BAR = P_GATE + kMaxGroups * kGateBytes;   // 2 mbarriers
+constexpr uint32_t P_SLOT = P_BAR + 16;            // TMEM base
 constexpr uint32_t kPSmem = P_SLOT + 16;
 constexpr uint32_t kPSmemAlloc = kPSmem + 1024;
 constexpr uint32_t kPTmemCols = 64;
 constexpr uint32_t kPWaitTries = 1u << 24;
 constexpr float kMaxChunkDecay = 80.f;  // factor exp(g_t - g_i) = gamma_t / gamma_i below this
-
-// fp32 scratch [64][64] with 16-byte chunks XOR-swizzled by row
-__device__ __forceinline__ int scr(int r, int c) { return r * 64 + ((((c >> 2) ^ (r & 7)) << 2) | (c & 3)); }
+static_assert(kMaxGroups * kScrBytes <= 65536, "group scratch inside the tile area");
 
 __device__ __forceinline__ float4 tf32x4(float4 x) {
     return make_float4(to_tf32(x.x), to_tf32(x.y), to_tf32(x.z), to_tf32(x.w));
@@ -61,12 +61,16 @@ __device__ __forceinline__ void bulk_store(void *dst, uint32_t src, uint32_t byt
                  : "memory");
 }
 
+__device__ __forceinline__ void group_sync(int id) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(kGroupThr) : "memory");
+}
+
 struct PrepParams {
     const float *kq;      // [chunk, Hqk] [K;Q] tiles (64 KB each)
-    float *kt;            // [chunk, Hv] K~ tiles (32 KB each)
     const void *alpha, *beta;
     const int32_t *cu, *cfirst;
-    float *tb, *w2, *pm;  // [chunk, Hv] tiles (16 KB each)
+    const int32_t *cseq;  // sequence of each chunk
+    float *tb, *pm;       // [chunk, Hv] tiles (16 KB each)
     float *gr;            // [chunk, Hv] gates records
     int n_seqs, n_qk, n_v;
     int64_t chunk_lo;     // first global chunk index of this launch
@@ -74,28 +78,35 @@ struct PrepParams {
 
 }  // namespace
 
+// blockDim.x = 128 x G, G dividing Hv / Hqk; CTA x covers V heads G*(x mod Hv/G) + [0, G)
+// of chunk chunk_lo + x / (Hv/G)
 template <class TI>
-__global__ void __launch_bounds__(kPThr) chunk_prep_kernel(const __grid_constant__ PrepParams p) {
-    const int h = blockIdx.x % p.n_v;
-    const int u = (int)(p.chunk_lo + blockIdx.x / p.n_v);   // global chunk index
-    if (u >= p.cfirst[p.n_seqs]) return;               // uniform per CTA
-    const int b = upper_index(p.cfirst, p.n_seqs, u);
+__global__ void __launch_bounds__(kGroupThr * kMaxGroups, 2) chunk_prep_kernel(const __grid_constant__ PrepParams p) {
+    const int G = blockDim.x / kGroupThr;
+    const int per_chunk = p.n_v / G;
+    const int u = (int)(p.chunk_lo + blockIdx.x / per_chunk);   // global chunk index
+    if (u >= p.cfirst[p.n_seqs]) return;                       // uniform per CTA
+    const int h0 = (int)(blockIdx.x % per_chunk) * G;
+    const int gq = h0 / (p.n_v / p.n_qk);
+    const int b = p.cseq[u];
     const int seq0 = p.cu[b];
     const int r0 = (u - p.cfirst[b]) * kChunk;
     const int n = min(kChunk, p.cu[b + 1] - seq0 - r0);
     const int tok = seq0 + r0;
-    const int gq = h / (p.n_v / p.n_qk);
 
     extern __shared__ unsigned char smem_raw[];
     unsigned char *sm = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
     const uint32_t sb = smem_u32(sm);
     uint64_t *bar = (uint64_t *)(sm + P_BAR);
     uint32_t *tslot = (uint32_t *)(sm + P_SLOT);
-    float *g_s = (float *)(sm + P_GATE), *beta_s = g_s + 64, *gam_s = g_s + 128, *kd_s = g_s + 192,
-          *ig_s = g_s + 256;
-    float *Ascr = (float *)(sm + P_AS), *Tscr = (float *)(sm + P_TS), *inv_s = (float *)(sm + P_INV);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int grp = tid / kGroupThr, gt = tid % kGroupThr;   // group grp: V head h0 + grp
+    const int h = h0 + grp;
     const int64_t tile = (int64_t)u * p.n_v + h;
+    float *g_s = (float *)(sm + P_GATE + grp * kGateBytes), *beta_s = g_s + 64, *gam_s = g_s + 128,
+          *ig_s = g_s + 192;
+    unsigned char *scr = sm + grp * kScrBytes;
+    const int gbar = 1 + grp;   // named barrier of the group
     float *gr = p.gr + tile * kGateRec;
 
     if (tid == 0) {
@@ -109,11 +120,11 @@ __global__ void __launch_bounds__(kPThr) chunk_prep_kernel(const __grid_constant
         tmem_relinquish();
     }
     // gates of the chunk: log alpha and beta, zero past n
-    if (tid < kChunk) {
+    if (gt < kChunk) {
         const TI *al = (const TI *)p.alpha, *be = (const TI *)p.beta;
-        const int64_t e = (int64_t)(tok + tid) * p.n_v + h;
-        g_s[tid] = tid < n ? safe_log_alpha(to_f32(al[e])) : 0.f;
-        beta_s[tid] = tid < n ? to_f32(be[e]) : 0.f;
+        const int64_t e = (int64_t)(tok + gt) * p.n_v + h;
+        g_s[gt] = gt < n ? safe_log_alpha(to_f32(al[e])) : 0.f;
+        beta_s[gt] = gt < n ? to_f32(be[e]) : 0.f;
     }
     fence_before_sync();
     __syncthreads();
@@ -130,7 +141,7 @@ __global__ void __launch_bounds__(kPThr) chunk_prep_kernel(const __grid_constant
             mma_commit(&bar[1]);
         }
     }
-    if (warp == 1) {  // gates: inclusive scan of log alpha, two rows per lane (meanwhile)
+    if ((gt >> 5) == 1) {  // warp 1 of each group: inclusive scan of log alpha, two rows per lane
         const int t0 = 2 * lane, t1 = t0 + 1;
         const float a0 = g_s[t0], a1 = g_s[t1];
         float s = a0 + a1;
@@ -148,182 +159,113 @@ __global__ void __launch_bounds__(kPThr) chunk_prep_kernel(const __grid_constant
         gam_s[t1] = gam1;
         ig_s[t0] = expf(-g0);      // used only when the chunk's decay stays below kMaxChunkDecay
         ig_s[t1] = expf(-g1);
-        const float kd0 = t0 < n ? expf(glast - g0) : 0.f, kd1 = t1 < n ? expf(glast - g1) : 0.f;
-        kd_s[t0] = kd0;
-        kd_s[t1] = kd1;
         gr[kGrGamma + t0] = gam0;
         gr[kGrGamma + t1] = gam1;
-        gr[kGrKd + t0] = kd0;
-        gr[kGrKd + t1] = kd1;
+        gr[kGrKd + t0] = t0 < n ? expf(glast - g0) : 0.f;
+        gr[kGrKd + t1] = t1 < n ? expf(glast - g1) : 0.f;
         if (lane == 0) gr[kGrGammaC] = expf(glast);
     }
-    if (__syncthreads_or(!ok)) {  // also publishes the gates and the arrived [K;Q] tile
-        if (tid == 0) mbar_wait(&bar[0], 0, kPWaitTries);  // drain the copy
-        ok = false;
+    if (tid == 0) {
+        if (ok) ok = mbar_wait(&bar[1], 0, kPWaitTries);
+        else mbar_wait(&bar[0], 0, kPWaitTries);   // drain the copy
     }
-    // K~ = diag(kd) K from the K-major K tile, written in the MN-major layout (coalesced)
-    {
-        float4 *dst = reinterpret_cast<float4 *>(p.kt + tile * 8192);
-        const float nan = __int_as_float(0x7fc00000);
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-            const int i4 = tid + kPThr * k;                       // float4 of the MN-major tile
-            const int o = 4 * i4, blk = o >> 11, t = (o >> 5) & 63, w = o & 31;
-            const int dl = 8 * ((w >> 3) ^ (t & 3)) + (w & 4);    // its first feature in the block
-            float4 x = *reinterpret_cast<const float4 *>(sm + P_KQ + blk * 16384 + t * 128 +
-                                                         ((((dl >> 2) ^ (t & 7))) << 4));
-            const float sc = ok ? kd_s[t] : nan;
-            dst[i4] = tf32x4(make_float4(x.x * sc, x.y * sc, x.z * sc, x.w * sc));
-        }
-    }
-    if (ok) ok = tid == 0 ? mbar_wait(&bar[1], 0, kPWaitTries) : true;
-    ok = !__syncthreads_or(!ok);  // the MMA is done and K~ has read the K tile
+    ok = !__syncthreads_or(!ok);  // the MMA is done (the tile area is free); gates published
     fence_after_sync();
     if (ok) {
-        // A (fp32 scratch) from the K K^T rows, P (TF32, staged as a K-major image) from the
-        // Q K^T rows.  exp(g_t - g_i) = gamma_t / gamma_i while the chunk's total decay keeps
-        // 1 / gamma finite; otherwise one exponential per element.
-        const int q = warp & 3, ch = warp >> 2;
-        float v[32];
-        tmem_ld32(taddr(tm, 32 * q, 32 * ch), v);
-        tmem_wait_ld();
+        // Row t of K K^T (lane quarters 0-1) becomes row t of -A, written transposed into the
+        // parity arrays; row t of Q K^T (quarters 2-3) becomes row t of P, TF32, stored to
+        // global memory in the K-major image.  exp(g_t - g_i) = gamma_t / gamma_i while the
+        // chunk's total decay keeps 1 / gamma finite; otherwise one exponential per element.
+        const int q = warp & 3;
+        const bool is_a = q < 2;
         const int t = 32 * (q & 1) + lane;
         const bool factored = -g_s[n - 1] < kMaxChunkDecay;
-        const float gt = g_s[t], rowf = gam_s[t] * (q < 2 ? beta_s[t] : 1.f), bt = q < 2 ? beta_s[t] : 1.f;
-        float out[32];
-        const int lim = t < n ? (q < 2 ? t : t + 1) : 0;   // columns i < lim are kept
-        if (factored) {   // uniform per CTA
+        const float bt = is_a ? -beta_s[t] : 1.f, rowf = gam_s[t] * bt, gtv = g_s[t];
+        const int lim = t < n ? (is_a ? t : t + 1) : 0;   // columns i < lim are kept
 #pragma unroll
-            for (int e = 0; e < 32; ++e) {
-                const int i = 32 * ch + e;
-                out[e] = i < lim ? rowf * ig_s[i] * v[e] : 0.f;
+        for (int h2 = 0; h2 < 2; ++h2) {   // columns 32*h2 .. 32*h2 + 31
+            float v[32];
+            tmem_ld32(taddr(tm, 32 * q, 32 * h2), v);
+            tmem_wait_ld();
+            if (factored) {   // uniform per CTA
+#pragma unroll
+                for (int e = 0; e < 32; e += 4) {
+                    const float4 f = *reinterpret_cast<const float4 *>(ig_s + 32 * h2 + e);
+                    const int i = 32 * h2 + e;
+                    v[e] = i < lim ? rowf * f.x * v[e] : 0.f;
+                    v[e + 1] = i + 1 < lim ? rowf * f.y * v[e + 1] : 0.f;
+                    v[e + 2] = i + 2 < lim ? rowf * f.z * v[e + 2] : 0.f;
+                    v[e + 3] = i + 3 < lim ? rowf * f.w * v[e + 3] : 0.f;
+                }
+            } else {
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                    const int i = 32 * h2 + e;
+                    v[e] = i < lim ? bt * expf(gtv - g_s[i]) * v[e] : 0.f;
+                }
             }
-        } else {
+            if (is_a) {
+                float *at = (float *)(scr + (t & 1) * kParStride) + (t >> 1) + 32 * 32 * h2;
 #pragma unroll
-            for (int e = 0; e < 32; ++e) {
-                const int i = 32 * ch + e;
-                out[e] = i < lim ? bt * expf(gt - g_s[i]) * v[e] : 0.f;
+                for (int e = 0; e < 32; ++e) at[e * 32] = v[e];
+            } else {
+                unsigned char *dst = (unsigned char *)(p.pm + tile * 4096);
+#pragma unroll
+                for (int k = 0; k < 8; ++k)
+                    *reinterpret_cast<float4 *>(dst + kmaj_off(t, 32 * h2 + 4 * k, 64)) =
+                        tf32x4(make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]));
             }
         }
-        if (q < 2) {
-#pragma unroll
-            for (int k = 0; k < 8; ++k)
-                *reinterpret_cast<float4 *>(&Ascr[scr(t, 32 * ch + 4 * k)]) =
-                    make_float4(out[4 * k], out[4 * k + 1], out[4 * k + 2], out[4 * k + 3]);
-        } else {
-#pragma unroll
-            for (int k = 0; k < 8; ++k)
-                *reinterpret_cast<float4 *>(sm + P_PST + kmaj_off(t, 32 * ch + 4 * k, 64)) =
-                    tf32x4(make_float4(out[4 * k], out[4 * k + 1], out[4 * k + 2], out[4 * k + 3]));
-        }
-        fence_smem_to_async();
     }
-    fence_before_sync();
-    __syncthreads();
-    if (ok && tid == 0) bulk_store(p.pm + tile * 4096, sb + P_PST, 16384);
+    group_sync(gbar);   // the group's A^T is complete
+
+    // ---- T = (I + A)^-1, column jc by forward substitution with right-looking updates:
+    // once row m of the column is final, every later row r loses A[r][m] T[m][jc].  This
+    // thread holds the rows of parity par (x[s] = T[2s + par][jc], as pairs for the packed
+    // FMA) and takes row m from its partner lane when m has the other parity.  Entries of A
+    // on or above the diagonal are zero in the scratch, so the updates may start at a
+    // multiple of 4; a warp skips the steps before its first column, where its rows are 0.
+    const int jc = gt >> 1, par = gt & 1;
+    const int m_first = 16 * (gt >> 5);   // this warp's columns are m_first .. m_first + 15
+    float2 x[16];
+#pragma unroll
+    for (int s = 0; s < 16; ++s)
+        x[s] = make_float2(2 * (2 * s) + par == jc ? 1.f : 0.f, 2 * (2 * s + 1) + par == jc ? 1.f : 0.f);
     if (ok) {
-        // ---- T = (I + A)^-1.  Diagonal 16 x 16 blocks: column cc of block bb by forward
-        // substitution with right-looking updates; the other threads clear the two blocks
-        // above the diagonal that the merge products read.
-        if (tid < 64) {
-            const int bb = tid >> 4, cc = tid & 15, o = 16 * bb;
-            float x[16];
+        const float *atp = (const float *)(scr + par * kParStride);
 #pragma unroll
-            for (int r = 0; r < 16; ++r) x[r] = (r == cc) ? 1.f : 0.f;
+        for (int m = 0; m < 63; ++m) {
+            if (m < m_first) continue;   // warp-uniform
+            const float2 xs = x[m >> 2];
+            const float mine = (m >> 1) & 1 ? xs.y : xs.x;
+            const float other = __shfl_xor_sync(0xffffffffu, mine, 1);
+            const float xm = (par == (m & 1)) ? mine : other;
+            const float2 xm2 = make_float2(xm, xm);
 #pragma unroll
-            for (int m = 0; m < 15; ++m) {
-                const float xm = x[m];
-#pragma unroll
-                for (int r = m + 1; r < 16; ++r) x[r] = fmaf(-Ascr[scr(o + r, o + m)], xm, x[r]);
-            }
-#pragma unroll
-            for (int r = 0; r < 16; ++r) Tscr[scr(o + r, o + cc)] = x[r];
-        } else {
-            for (int e = tid - 64; e < 512; e += kPThr - 64) {
-                const int blk = e >> 8, r = (e >> 4) & 15, cc = e & 15, o = 32 * blk;
-                Tscr[scr(o + r, o + 16 + cc)] = 0.f;
+            for (int s0 = (m >> 1) & ~3; s0 < 32; s0 += 4) {
+                const float4 a = *reinterpret_cast<const float4 *>(atp + m * 32 + s0);
+                x[s0 >> 1] = __ffma2_rn(make_float2(a.x, a.y), xm2, x[s0 >> 1]);
+                x[(s0 >> 1) + 1] = __ffma2_rn(make_float2(a.z, a.w), xm2, x[(s0 >> 1) + 1]);
             }
         }
-        __syncthreads();
-        if (tid < 128) {  // 32 x 32 halves: M = A_10 T_00
-            const int hh = tid >> 6, rr = (tid >> 2) & 15, c4 = (tid & 3) * 4, o = 32 * hh;
-            float a4[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-            for (int m = 0; m < 16; ++m) {
-                const float a = Ascr[scr(o + 16 + rr, o + m)];
-                const float4 t4 = *reinterpret_cast<const float4 *>(&Tscr[scr(o + m, o + c4)]);
-                a4[0] = fmaf(a, t4.x, a4[0]); a4[1] = fmaf(a, t4.y, a4[1]);
-                a4[2] = fmaf(a, t4.z, a4[2]); a4[3] = fmaf(a, t4.w, a4[3]);
-            }
-            *reinterpret_cast<float4 *>(&inv_s[hh * 256 + rr * 16 + c4]) = make_float4(a4[0], a4[1], a4[2], a4[3]);
-        }
-        __syncthreads();
-        if (tid < 128) {  // T_10 = -T_11 M
-            const int hh = tid >> 6, rr = (tid >> 2) & 15, c4 = (tid & 3) * 4, o = 32 * hh;
-            float a4[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-            for (int m = 0; m < 16; ++m) {
-                const float tv = Tscr[scr(o + 16 + rr, o + 16 + m)];
-                const float4 m4 = *reinterpret_cast<const float4 *>(&inv_s[hh * 256 + m * 16 + c4]);
-                a4[0] = fmaf(tv, m4.x, a4[0]); a4[1] = fmaf(tv, m4.y, a4[1]);
-                a4[2] = fmaf(tv, m4.z, a4[2]); a4[3] = fmaf(tv, m4.w, a4[3]);
-            }
-            *reinterpret_cast<float4 *>(&Tscr[scr(o + 16 + rr, o + c4)]) = make_float4(-a4[0], -a4[1], -a4[2], -a4[3]);
-        }
-        __syncthreads();
-        {  // merge: M = A_bl T_top, parked in the (otherwise unused) upper-right block
-            const int r = tid >> 3, c4 = (tid & 7) * 4;
-            float a4[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-            for (int m = 0; m < 32; ++m) {
-                const float a = Ascr[scr(32 + r, m)];
-                const float4 t4 = *reinterpret_cast<const float4 *>(&Tscr[scr(m, c4)]);
-                a4[0] = fmaf(a, t4.x, a4[0]); a4[1] = fmaf(a, t4.y, a4[1]);
-                a4[2] = fmaf(a, t4.z, a4[2]); a4[3] = fmaf(a, t4.w, a4[3]);
-            }
-            *reinterpret_cast<float4 *>(&Tscr[scr(r, 32 + c4)]) = make_float4(a4[0], a4[1], a4[2], a4[3]);
-        }
-        __syncthreads();
-        {  // T_bl = -T_br M
-            const int r = tid >> 3, c4 = (tid & 7) * 4;
-            float a4[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-            for (int m = 0; m < 32; ++m) {
-                const float tv = Tscr[scr(32 + r, 32 + m)];
-                const float4 m4 = *reinterpret_cast<const float4 *>(&Tscr[scr(m, 32 + c4)]);
-                a4[0] = fmaf(tv, m4.x, a4[0]); a4[1] = fmaf(tv, m4.y, a4[1]);
-                a4[2] = fmaf(tv, m4.z, a4[2]); a4[3] = fmaf(tv, m4.w, a4[3]);
-            }
-            *reinterpret_cast<float4 *>(&Tscr[scr(32 + r, c4)]) = make_float4(-a4[0], -a4[1], -a4[2], -a4[3]);
-        }
-        __syncthreads();
     }
-    {  // T_beta = T diag(beta) and W2 = T_beta diag(gamma), staged (the upper-right block of
-       // T is zero; W2 reuses the A scratch, dead since the merge); NaN if the CTA failed
-        const int t = tid >> 2, i0 = (tid & 3) * 16;
-        const bool upper_right = t < 32 && i0 >= 32;
-        const float nan = __int_as_float(0x7fc00000);
+    group_sync(gbar);   // the group is done reading A^T; its space takes the T_beta staging
+    {   // T_beta = T diag(beta), TF32, as a K-major image; NaN if the CTA failed
+        const float bj = beta_s[jc], nan = __int_as_float(0x7fc00000);
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const int i = i0 + 4 * k;
-            float4 x = *reinterpret_cast<const float4 *>(&Tscr[scr(t, i)]);
-            if (upper_right) x = make_float4(0.f, 0.f, 0.f, 0.f);
-            x = make_float4(x.x * beta_s[i], x.y * beta_s[i + 1], x.z * beta_s[i + 2], x.w * beta_s[i + 3]);
-            if (!ok) x = make_float4(nan, nan, nan, nan);
-            const float4 w = make_float4(x.x * gam_s[i], x.y * gam_s[i + 1], x.z * gam_s[i + 2], x.w * gam_s[i + 3]);
-            *reinterpret_cast<float4 *>(sm + P_TBST + kmaj_off(t, i, 64)) = tf32x4(x);
-            *reinterpret_cast<float4 *>(sm + P_AS + kmaj_off(t, i, 64)) = tf32x4(w);
+        for (int s = 0; s < 32; ++s) {
+            const float xv = (s & 1) ? x[s >> 1].y : x[s >> 1].x;
+            *reinterpret_cast<float *>(scr + kmaj_off(2 * s + par, jc, 64)) = ok ? to_tf32(xv * bj) : nan;
         }
         fence_smem_to_async();
     }
-    fence_before_sync();
-    __syncthreads();
-    if (tid == 0) {
-        bulk_store(p.tb + tile * 4096, sb + P_TBST, 16384);
-        bulk_store(p.w2 + tile * 4096, sb + P_AS, 16384);
+    group_sync(gbar);
+    if (gt == 0) {
+        bulk_store(p.tb + tile * 4096, smem_u32(scr), 16384);
         bulk_commit();
-        bulk_wait0();   // the stores are complete before the CTA's shared memory goes away
+        bulk_wait0();   // the store is complete before the CTA's shared memory goes away
     }
+    fence_before_sync();
     __syncthreads();
     if (warp == 0) tmem_dealloc(tm, kPTmemCols);
 }
@@ -331,18 +273,21 @@ __global__ void __launch_bounds__(kPThr) chunk_prep_kernel(const __grid_constant
 cudaError_t launch_chunk_prep(const ScanParams &sp, int64_t total_tokens, bool in_bf16, cudaStream_t s) {
     if (sp.n_seqs <= 0 || total_tokens <= 0) return cudaSuccess;
     PrepParams p{};
-    p.kq = sp.kq; p.kt = sp.kt;
-    p.alpha = sp.alpha; p.beta = sp.beta; p.cu = sp.cu; p.cfirst = sp.cfirst;
-    p.tb = sp.tb; p.w2 = sp.w2; p.pm = sp.pm; p.gr = sp.gr; p.n_seqs = sp.n_seqs; p.n_qk = sp.n_qk; p.n_v = sp.n_v;
+    p.kq = sp.kq;
+    p.alpha = sp.alpha; p.beta = sp.beta; p.cu = sp.cu; p.cfirst = sp.cfirst; p.cseq = sp.cseq;
+    p.tb = sp.tb; p.pm = sp.pm; p.gr = sp.gr; p.n_seqs = sp.n_seqs; p.n_qk = sp.n_qk; p.n_v = sp.n_v;
     p.chunk_lo = sp.chunk_lo;
-    const int64_t grid = (sp.chunk_hi - sp.chunk_lo) * sp.n_v;
+    // V heads per CTA: 3, 2 or 1, whichever first divides the V heads of a QK head
+    const int ratio = sp.n_v / sp.n_qk;
+    const int G = ratio % 3 == 0 ? 3 : (ratio % 2 == 0 ? 2 : 1);
+    const int64_t grid = (sp.chunk_hi - sp.chunk_lo) * (sp.n_v / G);
     if (grid <= 0) return cudaSuccess;
     if (grid >= ((int64_t)1 << 31)) return cudaErrorInvalidValue;
     auto k = in_bf16 ? chunk_prep_kernel<bf16> : chunk_prep_kernel<float>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kPSmemAlloc);
     if (e != cudaSuccess) return e;
     TraceLaunch tl(s, "chunk_prep");
-    k<<<(unsigned)grid, kPThr, kPSmemAlloc, s>>>(p);
+    k<<<(unsigned)grid, kGroupThr * G, kPSmemAlloc, s>>>(p);
     return cudaGetLastError();
 }
 

@@ -90,8 +90,8 @@ cudaError_t launch_seq_table(const int32_t *cu_in, int n_seqs, int64_t T, int32_
 // the shared-memory layouts the tensor-core kernels copy them into:
 //   [K;Q] of (chunk, QK head): 4 blocks of 32 features x (K 64 rows | Q 64 rows), 128-byte
 //     rows with 16-byte chunks XOR-swizzled by row (K-major operand layout);
-//   V of (chunk, V head): 4 blocks of 32 features x 64 rows, 128-byte rows with 32-byte
-//     granules XOR-swizzled by row (MN-major operand layout).
+//   K of (chunk, QK head) and V of (chunk, V head): 4 blocks of 32 features x 64 rows,
+//     128-byte rows with 32-byte granules XOR-swizzled by row (MN-major operand layout).
 // Rows past the end of the sequence are written as zeros.
 template <class T, bool kTiles>
 __global__ void __launch_bounds__(128) conv_l2_kernel(ConvParams p) {
@@ -102,6 +102,7 @@ __global__ void __launch_bounds__(128) conv_l2_kernel(ConvParams p) {
     const int seq0 = p.cu[b], seq1 = p.cu[b + 1];
     const int r0 = (ci - p.cfirst[b]) * kChunk;  // chunk start within the sequence
     const int len = min(kChunk, seq1 - seq0 - r0);
+    if (kTiles && blockIdx.y == 0 && threadIdx.x == 0) p.cseq[ci] = b;   // for the chunk-prep pass
 
     const int slot = blockIdx.y;
     const T *x;
@@ -136,12 +137,13 @@ __global__ void __launch_bounds__(128) conv_l2_kernel(ConvParams p) {
     const int re = min(rs + 16, r0 + len);
     if (!kTiles && rs >= re) return;
     // tile destinations (float offsets of this lane's 4 features, row 0)
-    float *t_a = nullptr, *t_b = nullptr;          // K-major ([K;Q]) and MN-major (V) tile
+    float *t_a = nullptr, *t_b = nullptr;          // K-major ([K;Q]) and MN-major (K or V) tile
     if (kTiles) {
         if (slot < p.n_qk) {
             t_a = p.kq + ((int64_t)ci * p.n_qk + slot) * 16384 + 2048;
         } else if (slot < 2 * p.n_qk) {
             t_a = p.kq + ((int64_t)ci * p.n_qk + slot - p.n_qk) * 16384;
+            t_b = p.kmn + ((int64_t)ci * p.n_qk + slot - p.n_qk) * 8192;
         } else {
             t_b = p.vi + ((int64_t)ci * p.n_v + slot - 2 * p.n_qk) * 8192;
         }

@@ -49,12 +49,12 @@ PrefillLayout prefill_layout(int n_qk, int n_v, int64_t T, int n_seqs, bool tc) 
     L.off_vh = off;      off = align_up(off + v_bytes, 256);
     const size_t nc = tc && T > 0 ? (size_t)L.max_chunks : 0;
     L.off_kq = off;      off = align_up(off + nc * n_qk * 65536, 256);
+    L.off_kmn = off;     off = align_up(off + nc * n_qk * 32768, 256);
     L.off_vi = off;      off = align_up(off + nc * n_v * 32768, 256);
-    L.off_kt = off;      off = align_up(off + nc * n_v * 32768, 256);
     L.off_tb = off;      off = align_up(off + nc * n_v * 16384, 256);
-    L.off_w2 = off;      off = align_up(off + nc * n_v * 16384, 256);
     L.off_pm = off;      off = align_up(off + nc * n_v * 16384, 256);
     L.off_gr = off;      off = align_up(off + nc * n_v * kGateRec * sizeof(float), 256);
+    L.off_cseq = off;    off = align_up(off + nc * sizeof(int32_t), 256);
     L.n_segments = tc && T > 0 ? plan_segments(n_v, n_seqs, L.max_chunks) : 1;
     const size_t carry = L.n_segments > 1 ? (size_t)n_seqs * n_v * 128 * 128 * sizeof(float) : 0;
     L.off_carry = off;   off = align_up(off + carry, 256);
@@ -228,7 +228,9 @@ gdn_status gdn_prefill(const gdn_config *cfg, gdn_dtype dtype, gdn_dtype out_dty
         cp.conv_in = conv_state_in;
         cp.qh = (float *)(ws + L.off_qh); cp.kh = (float *)(ws + L.off_kh);
         cp.vh = (float *)(ws + L.off_vh);
-        cp.kq = (float *)(ws + L.off_kq); cp.vi = (float *)(ws + L.off_vi);
+        cp.kq = (float *)(ws + L.off_kq); cp.kmn = (float *)(ws + L.off_kmn);
+        cp.cseq = (int32_t *)(ws + L.off_cseq);
+        cp.vi = (float *)(ws + L.off_vi);
         cp.cu = cu; cp.cfirst = cfirst;
         cp.n_seqs = n_seqs; cp.n_qk = cfg->n_qk_heads; cp.n_v = cfg->n_v_heads;
         cp.q_scale = cfg->q_scale; cp.eps = cfg->l2_eps;
@@ -247,10 +249,12 @@ gdn_status gdn_prefill(const gdn_config *cfg, gdn_dtype dtype, gdn_dtype out_dty
     ScanParams sp{};
     sp.qh = (const float *)(ws + L.off_qh); sp.kh = (const float *)(ws + L.off_kh);
     sp.vh = (const float *)(ws + L.off_vh);
-    sp.kq = (const float *)(ws + L.off_kq); sp.vi = (const float *)(ws + L.off_vi);
+    sp.kq = (const float *)(ws + L.off_kq); sp.kmn = (const float *)(ws + L.off_kmn);
+    sp.vi = (const float *)(ws + L.off_vi);
     sp.alpha = alpha; sp.beta = beta; sp.cu = cu; sp.cfirst = cfirst;
-    sp.kt = (float *)(ws + L.off_kt); sp.tb = (float *)(ws + L.off_tb); sp.w2 = (float *)(ws + L.off_w2);
-    sp.pm = (float *)(ws + L.off_pm); sp.gr = (float *)(ws + L.off_gr); sp.max_chunks = L.max_chunks;
+    sp.tb = (float *)(ws + L.off_tb); sp.pm = (float *)(ws + L.off_pm); sp.gr = (float *)(ws + L.off_gr);
+    sp.cseq = (const int32_t *)(ws + L.off_cseq);
+    sp.max_chunks = L.max_chunks;
     sp.init = initial_state; sp.fin = final_state; sp.out = out;
     sp.n_seqs = n_seqs; sp.n_qk = cfg->n_qk_heads; sp.n_v = cfg->n_v_heads;
     if (bf) {

@@ -29,12 +29,12 @@ struct PrefillLayout {
     // tensor-core path: per-chunk tiles already in the shared-memory layout of the kernels
     // that read them (so each is one contiguous bulk copy); rows past a sequence's end are 0
     size_t off_kq;        // [max_chunks, Hqk] x 64 KB: [K;Q], K-major 128B-swizzled blocks
+    size_t off_kmn;       // [max_chunks, Hqk] x 32 KB: K, MN-major 32B-granule swizzle
     size_t off_vi;        // [max_chunks, Hv]  x 32 KB: V, MN-major 32B-granule swizzle
-    size_t off_kt;        // [max_chunks, Hv]  x 32 KB: K~ = diag(kd) K, MN-major like off_vi
     size_t off_tb;        // [max_chunks, Hv]  x 16 KB: T diag(beta), K-major 128B-swizzled
-    size_t off_w2;        // [max_chunks, Hv]  x 16 KB: T diag(beta gamma), same
     size_t off_pm;        // [max_chunks, Hv]  x 16 KB: P, same
     size_t off_gr;        // [max_chunks, Hv]  x 640 B: gates record (gamma[64], kd[64], gamma_C)
+    size_t off_cseq;      // int32 [max_chunks]: sequence of each chunk (written by the conv pass)
     size_t off_carry;     // [n_seqs, Hv, 128, 128] fp32 state between chunk ranges (segmented
                           // tensor-core path without a caller final-state buffer), else empty
     int n_segments;       // tensor-core path: chunk ranges run as a pipeline (1 = one pass)
@@ -56,7 +56,8 @@ struct ConvParams {
     const float *wq, *wk, *wv;             // [ch, 4]
     const void *conv_in;                   // [n_seqs, 3, channels] or null
     float *qh, *kh, *vh;                   // fp32 rows (fp32 path)
-    float *kq, *vi;                        // chunk tiles (tensor-core path), or null
+    float *kq, *kmn, *vi;                  // chunk tiles (tensor-core path), or null
+    int32_t *cseq;                         // chunk -> sequence table, filled with the tiles
     const int32_t *cu, *cfirst;            // workspace tables
     int n_seqs, n_qk, n_v;
     float q_scale, eps;
@@ -65,11 +66,12 @@ struct ConvParams {
 
 struct ScanParams {
     const float *qh, *kh, *vh;             // fp32 conv + L2 rows [T, H, 128] (fp32 path)
-    const float *kq, *vi;                  // chunk tiles (tensor-core path)
+    const float *kq, *kmn, *vi;            // chunk tiles (tensor-core path)
     const void *alpha, *beta;              // [T, Hv]
     const int32_t *cu;                     // clamped bounds [n_seqs+1]
     const int32_t *cfirst;                 // first chunk index of each sequence [n_seqs+1]
-    float *kt, *tb, *w2, *pm, *gr;         // chunk-prep tiles and gates records (tensor-core path)
+    const int32_t *cseq;                   // sequence of each chunk (tensor-core path)
+    float *tb, *pm, *gr;                   // chunk-prep tiles and gates records (tensor-core path)
     int64_t max_chunks;
     int64_t chunk_lo, chunk_hi;            // global chunk range of one launch (tensor-core path)
     const float *carry_in;                 // state entering a chunk range that starts inside a

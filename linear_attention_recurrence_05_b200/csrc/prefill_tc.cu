@@ -5,12 +5,14 @@
 // DELTANET equations), in chunks of 64 tokens.  Within a chunk, with
 // g_t = sum_{s<=t} log alpha_s, gamma_t = exp(g_t), kd_t = exp(g_C - g_t) and S the state
 // entering the chunk:
-//     u   = T_beta V - W2 (K S),          T_beta = (I + A)^-1 diag(beta), W2 = T_beta diag(gamma)
-//     y   = diag(gamma) (Q S) + P u,      P_ti = exp(g_t - g_i) q_t.k_i (i <= t)
-//     S  <- gamma_C S + K~^T u,           K~ = diag(kd) K
-// T_beta, W2, P, K~ and the gates (gamma, kd, gamma_C) of every chunk come from the
-// chunk-prep pass; K, Q and V as tiles from the conv + L2 pass, all already in the
-// shared-memory layout the MMAs read.
+//     u   = T_beta (V - diag(gamma) K S),  T_beta = (I + A)^-1 diag(beta)
+//     y   = diag(gamma) (Q S) + P u,       P_ti = exp(g_t - g_i) q_t.k_i (i <= t)
+//     S  <- gamma_C S + K^T diag(kd) u
+// Every per-token factor applied here (gamma_t, kd_t, gamma_C) is at most 1, so no decay
+// is ever divided out.  T_beta, P and the gates (gamma, kd, gamma_C) of every chunk come
+// from the chunk-prep pass; [K;Q], K and V as tiles from the conv + L2 pass, all already
+// in the shared-memory layout the MMAs read.  The K tiles are those of the QK head, shared
+// by its V heads.
 //
 // One CTA owns one (sequence, V head).  All MMAs are M = 128 with the d_v index on the
 // 128 tensor-memory lanes (transposed form), so every state-dependent A operand is read
@@ -18,12 +20,12 @@
 //   issuer (warp 0, one thread), per chunk
 //     MMA_1   [X | Y1] = S^T [K;Q]^T            (N=128, K=128)   X = (K S)^T, Y1 = (Q S)^T
 //     MMA_2a  U^T      = V^T T_beta^T           (N=64,  K=64)    V from shared memory
-//     MMA_2b  U^T     -= X W2^T                 (N=64,  K=64)    -> u^T
-//     MMA_3   S^T     += u^T K~                 (N=128, K=64)    onto gamma_C S^T
-//     MMA_4   Y       += u^T P^T                (N=64,  K=64)    onto Y = diag(gamma) Y1
-//   epilogue (warps 1-4): between MMA_1 and MMA_3 of a chunk, Y = gamma Y1 and
-//     S^T *= gamma_C in tensor memory; after MMA_4, y to global memory (TMA store); the
-//     initial and final state.
+//     MMA_2b  U^T     -= X' T_beta^T            (N=64,  K=64)    X' = X diag(gamma) -> u^T
+//     MMA_4   Y       += u^T P^T                (N=64,  K=64)    onto Y = Y1 diag(gamma)
+//     MMA_3   S^T     += u~^T K                 (N=128, K=64)    u~ = u diag(kd), onto gamma_C S^T
+//   epilogue (warps 1-4), in tensor memory: after MMA_1, X' (first: MMA_2b waits for it),
+//     then Y and S^T *= gamma_C; after MMA_2b, u~ (MMA_3 waits for it, MMA_4 runs
+//     meanwhile); after MMA_4, y to global memory (TMA store); the initial and final state.
 //   producer (warp 5): the tile loads, each issued as soon as its buffer is consumed.
 // All waits are bounded; a CTA that times out writes NaN to its outputs.
 #include <cuda.h>
@@ -47,23 +49,24 @@ constexpr int kBarEpi = 1;         // named barrier of the epilogue (128 threads
 
 // shared-memory map (bytes from a 1024-aligned base)
 constexpr uint32_t OFF_KQ = 0;          // [K;Q]   K-major, 4 blocks x (K 8 KB | Q 8 KB)       64 KB
-constexpr uint32_t OFF_KMN = 65536;     // K~      MN-major (32-byte granules), 64 x 128       32 KB
+constexpr uint32_t OFF_KMN = 65536;     // K       MN-major (32-byte granules), 64 x 128       32 KB
 constexpr uint32_t OFF_VMN = 98304;     // V       MN-major (32-byte granules), 64 x 128       32 KB
 constexpr uint32_t OFF_TB = 131072;     // T_beta  K-major [t][i]                              16 KB
 constexpr uint32_t OFF_P = 147456;      // P       K-major [t][i]                              16 KB
-constexpr uint32_t OFF_W2 = 163840;     // W2      K-major [t][i]                              16 KB
-constexpr uint32_t OFF_YST = 180224;    // y staging: 2 x (32 rows x 128 columns), TMA stores  32 KB
-constexpr uint32_t OFF_GR = 212992;     // gates records, 2 buffers                          1280 B
+constexpr uint32_t OFF_YST = 163840;    // y staging: 2 x (32 rows x 128 columns), TMA stores  32 KB
+constexpr uint32_t OFF_GR = 196608;     // gates records, 2 buffers                          1280 B
 constexpr uint32_t OFF_BAR = OFF_GR + 2 * kGateRec * 4;   // mbarriers
 constexpr uint32_t OFF_FLAGS = OFF_BAR + 128;             // TMEM base, abort flag
 constexpr uint32_t kSmem = OFF_FLAGS + 16;
 constexpr uint32_t kSmemAlloc = kSmem + 1024;              // slack to align the base to 1024
 
 enum {
-    B_KQ = 0, B_V, B_KMN, B_W2L, B_PL, B_TBL,   // tile arrivals
+    B_KQ = 0, B_V, B_KMN, B_PL,          // tile arrivals (B_V: V and T_beta)
     B_GR0, B_GR1,                        // arrival of the gates record into buffer 0 / 1
     B_1, B_2, B_3, B_4,                  // MMA completions (MMA_1; 2a+2b; 3; 4)
-    B_Y1,                                // epilogue: Y1 taken, Y = gamma Y1 stored, S scaled
+    B_XS,                                // epilogue: X' = X diag(gamma) stored
+    B_Y1,                                // epilogue: Y = Y1 diag(gamma) stored, S scaled
+    B_UT,                                // epilogue: u~ = u diag(kd) stored
     B_DRAIN0,                            // drain on the failure path
     kNumBars
 };
@@ -75,6 +78,7 @@ constexpr uint32_t T_S = 0;      // S^T                  128 cols
 constexpr uint32_t T_XY = 128;   // [X | Y1]             128 cols
 constexpr uint32_t T_U = 256;    // u^T                   64 cols
 constexpr uint32_t T_Y = 320;    // gamma Y1, then y      64 cols
+constexpr uint32_t T_UT = 384;   // u~^T                  64 cols
 
 constexpr uint32_t kWaitTries = 1u << 22;
 
@@ -134,9 +138,9 @@ __device__ __forceinline__ void gemm_ts(uint32_t d_tmem, uint32_t a_tmem, uint32
 
 struct TcParams {
     CUtensorMap tm_out;   // y as [T, Hv*128] rows, boxes of 128 columns x 32 rows (no swizzle)
-    // per-chunk tiles in shared-memory layout: [K;Q] per (chunk, QK head); V, K~, T_beta,
-    // W2, P and the gates record per (chunk, V head)
-    const float *kq, *kt, *vi, *tb, *w2, *pm, *gr;
+    // per-chunk tiles in shared-memory layout: [K;Q] and K per (chunk, QK head); V, T_beta,
+    // P and the gates record per (chunk, V head)
+    const float *kq, *kmn, *vi, *tb, *pm, *gr;
     const int32_t *cu, *cfirst;
     const float *init, *carry_in;   // state entering chunk 0 / entering a later first chunk
     float *carry_out;               // state after the last chunk of the launch
@@ -192,11 +196,13 @@ __global__ void __launch_bounds__(kThr, 1) prefill_tc_kernel(const __grid_consta
     auto qk_tile = [&](const float *base, int c, int64_t floats) { return base + ((cf + cb + c) * p.n_qk + gq) * floats; };
     auto v_tile = [&](const float *base, int c, int64_t floats) { return base + ((cf + cb + c) * p.n_v + h) * floats; };
     auto issue_kq = [&](int c) { load(B_KQ, OFF_KQ, qk_tile(p.kq, c, 16384), 65536); };
-    auto issue_kmn = [&](int c) { load(B_KMN, OFF_KMN, v_tile(p.kt, c, 8192), 32768); };
-    auto issue_v = [&](int c) { load(B_V, OFF_VMN, v_tile(p.vi, c, 8192), 32768); };
-    auto issue_w2 = [&](int c) { load(B_W2L, OFF_W2, v_tile(p.w2, c, 4096), 16384); };
+    auto issue_kmn = [&](int c) { load(B_KMN, OFF_KMN, qk_tile(p.kmn, c, 8192), 32768); };
+    auto issue_v = [&](int c) {  // V and T_beta, one barrier
+        mbar_expect_tx(&bar[B_V], 32768 + 16384);
+        bulk_load(sb + OFF_VMN, v_tile(p.vi, c, 8192), 32768, &bar[B_V]);
+        bulk_load(sb + OFF_TB, v_tile(p.tb, c, 4096), 16384, &bar[B_V]);
+    };
     auto issue_pm = [&](int c) { load(B_PL, OFF_P, v_tile(p.pm, c, 4096), 16384); };
-    auto issue_tb = [&](int c) { load(B_TBL, OFF_TB, v_tile(p.tb, c, 4096), 16384); };
     auto issue_gr = [&](int c) {  // gates record of chunk c into buffer c & 1
         load(B_GR0 + (c & 1), OFF_GR + (c & 1) * kGateRec * 4, v_tile(p.gr, c, kGateRec), kGateRec * 4);
     };
@@ -217,9 +223,7 @@ __global__ void __launch_bounds__(kThr, 1) prefill_tc_kernel(const __grid_consta
     }
     if (tid == 0 && nchunks > 0) {
         issue_kq(0);
-        issue_tb(0);
         issue_v(0);
-        issue_w2(0);
         issue_kmn(0);
         issue_pm(0);
         issue_gr(0);
@@ -233,38 +237,41 @@ __global__ void __launch_bounds__(kThr, 1) prefill_tc_kernel(const __grid_consta
         // ================================================================ issuer
         if (lane == 0) {
             bool ok = true;
-            for (int c = 0; c < nchunks; ++c) {
+            // A wait costs ~100 cycles even when its phase is complete, so the waits for tiles
+            // and for epilogue steps that are normally done sit right after an MMA group,
+            // while the tensor pipe still has queued work.
+            if (nchunks > 0) ok = wait_or_abort(&bar[B_KQ], 0, abort_flag);
+            for (int c = 0; c < nchunks && ok; ++c) {
                 const uint32_t par = c & 1;
-                // MMA_1: needs S (MMA_3 of c-1, waited below) and [K;Q] of c; Y1 of c-1 was
-                // taken before MMA_4 of c-1
-                if (!(ok = wait_or_abort(&bar[B_KQ], par, abort_flag))) break;
+                // MMA_1: needs S (MMA_3 of c-1, waited below) and [K;Q] of c (waited below)
                 fence_after_sync();
                 gemm_ts<128, 128, false, false>(tm + T_XY, tm + T_S, sb + OFF_KQ, 16384, false);
                 mma_commit(&bar[B_1]);
-                // MMA_4 of c-1 still reads u^T, which MMA_2a overwrites
-                if (c > 0 && !(ok = wait_or_abort(&bar[B_4], par ^ 1, abort_flag))) break;
-                // MMA_2a: U^T = V^T T_beta^T (state-independent)
-                if (!(ok = wait_or_abort(&bar[B_TBL], par, abort_flag))) break;
+                // MMA_2a: U^T = V^T T_beta^T (state-independent).  u^T of c-1 is free: MMA_4
+                // of c-1 completed before MMA_3 of c-1, and the epilogue took u~ before that.
                 if (!(ok = wait_or_abort(&bar[B_V], par, abort_flag))) break;
                 fence_after_sync();
                 gemm<128, 64, 64, true, false>(tm + T_U, sb + OFF_VMN, 64, sb + OFF_TB, 8192, false);
-                // MMA_2b: U^T -= X W2^T
-                if (!(ok = wait_or_abort(&bar[B_1], par, abort_flag))) break;
-                if (!(ok = wait_or_abort(&bar[B_W2L], par, abort_flag))) break;
+                // MMA_2b: U^T -= X' T_beta^T once the epilogue has scaled X (after MMA_1)
+                if (!(ok = wait_or_abort(&bar[B_XS], par, abort_flag))) break;
                 fence_after_sync();
-                gemm_ts<64, 64, false, true>(tm + T_U, tm + T_XY, sb + OFF_W2, 8192, true);
+                gemm_ts<64, 64, false, true>(tm + T_U, tm + T_XY, sb + OFF_TB, 8192, true);
                 mma_commit(&bar[B_2]);
-                // MMA_3 / MMA_4: S^T += u^T K~ onto gamma_C S^T; Y += u^T P^T onto gamma Y1
-                if (!(ok = wait_or_abort(&bar[B_2], par, abort_flag))) break;
                 if (!(ok = wait_or_abort(&bar[B_Y1], par, abort_flag))) break;
-                if (!(ok = wait_or_abort(&bar[B_KMN], par, abort_flag))) break;
                 if (!(ok = wait_or_abort(&bar[B_PL], par, abort_flag))) break;
+                if (!(ok = wait_or_abort(&bar[B_KMN], par, abort_flag))) break;
+                // MMA_4: Y += u^T P^T onto Y = Y1 diag(gamma); the epilogue forms u~ meanwhile
+                if (!(ok = wait_or_abort(&bar[B_2], par, abort_flag))) break;
                 fence_after_sync();
-                gemm_ts<128, 64, true, false>(tm + T_S, tm + T_U, sb + OFF_KMN, 64, true);
-                mma_commit(&bar[B_3]);
                 gemm_ts<64, 64, false, false>(tm + T_Y, tm + T_U, sb + OFF_P, 8192, true);
                 mma_commit(&bar[B_4]);
-                // the next MMA_1 needs S only; it queues behind MMA_4 in the tensor pipe
+                // MMA_3: S^T += u~^T K onto gamma_C S^T
+                if (!(ok = wait_or_abort(&bar[B_UT], par, abort_flag))) break;
+                fence_after_sync();
+                gemm_ts<128, 64, true, false>(tm + T_S, tm + T_UT, sb + OFF_KMN, 64, true);
+                mma_commit(&bar[B_3]);
+                // the next MMA_1 reads S and the next [K;Q]
+                if (c + 1 < nchunks && !(ok = wait_or_abort(&bar[B_KQ], par ^ 1, abort_flag))) break;
                 if (!(ok = wait_or_abort(&bar[B_3], par, abort_flag))) break;
             }
             if (!ok) {  // drain this thread's MMAs (bounded)
@@ -276,32 +283,28 @@ __global__ void __launch_bounds__(kThr, 1) prefill_tc_kernel(const __grid_consta
         // ================================================================ tile producer
         if (lane == 0) {
             bool ok = true;
-            int n_kq = nchunks > 0 ? 1 : 0, n_v = n_kq, n_kmn = n_kq, n_w2 = n_kq, n_pm = n_kq, n_tb = n_kq;
+            int n_kq = nchunks > 0 ? 1 : 0, n_v = n_kq, n_kmn = n_kq, n_pm = n_kq;
             int n_gr[2] = {nchunks > 0 ? 1 : 0, nchunks > 1 ? 1 : 0};
             for (int c = 0; c < nchunks && ok; ++c) {
                 const uint32_t par = c & 1;
                 // [K;Q] of c is consumed once MMA_1 of c is done
                 if (!(ok = wait_or_abort(&bar[B_1], par, abort_flag))) break;
                 if (c + 1 < nchunks) { issue_kq(c + 1); ++n_kq; }
-                // V, T_beta and W2 once MMA_2a/2b of c are done
+                // V and T_beta once MMA_2a/2b of c are done
                 if (!(ok = wait_or_abort(&bar[B_2], par, abort_flag))) break;
-                if (c + 1 < nchunks) {
-                    issue_v(c + 1); ++n_v;
-                    issue_tb(c + 1); ++n_tb;
-                    issue_w2(c + 1); ++n_w2;
-                }
-                // K~ and this gates buffer once MMA_3 of c is done (the epilogue took its gates
-                // before MMA_3 could start); P once MMA_4 of c is done
+                if (c + 1 < nchunks) { issue_v(c + 1); ++n_v; }
+                // P once MMA_4 of c is done; K and this gates buffer once MMA_3 of c is done
+                // (the epilogue took the gates of c before MMA_3 could start)
+                if (!(ok = wait_or_abort(&bar[B_4], par, abort_flag))) break;
+                if (c + 1 < nchunks) { issue_pm(c + 1); ++n_pm; }
                 if (!(ok = wait_or_abort(&bar[B_3], par, abort_flag))) break;
                 if (c + 1 < nchunks) { issue_kmn(c + 1); ++n_kmn; }
                 if (c + 2 < nchunks) { issue_gr(c + 2); ++n_gr[c & 1]; }
-                if (!(ok = wait_or_abort(&bar[B_4], par, abort_flag))) break;
-                if (c + 1 < nchunks) { issue_pm(c + 1); ++n_pm; }
             }
             if (!ok) {  // wait (bounded) for the copies this thread started
-                const int counts[6] = {n_kq, n_v, n_kmn, n_w2, n_pm, n_tb};
-                const int bars[6] = {B_KQ, B_V, B_KMN, B_W2L, B_PL, B_TBL};
-                for (int i = 0; i < 6; ++i)
+                const int counts[4] = {n_kq, n_v, n_kmn, n_pm};
+                const int bars[4] = {B_KQ, B_V, B_KMN, B_PL};
+                for (int i = 0; i < 4; ++i)
                     if (counts[i]) mbar_wait(&bar[bars[i]], (uint32_t)(counts[i] - 1) & 1, kWaitTries);
                 for (int i = 0; i < 2; ++i)
                     if (n_gr[i]) mbar_wait(&bar[B_GR0 + i], (uint32_t)(n_gr[i] - 1) & 1, kWaitTries);
@@ -316,24 +319,46 @@ __global__ void __launch_bounds__(kThr, 1) prefill_tc_kernel(const __grid_consta
             const bool ok = leader ? wait_or_abort(&bar[i], par, abort_flag) : true;
             return !bar_or(kBarEpi, 128, !ok);
         };
+        // the group's tensor-memory stores are done: tell the issuer through mbarrier i
+        auto publish = [&](int i) {
+            tmem_wait_st();
+            fence_before_sync();
+            bar_sync(kBarEpi, 128);
+            if (leader) mbar_arrive(&bar[i]);
+        };
+        // columns [src, src + 64) of this warp's lanes, column i times f[i], stored at dst
+        // (f: 16-byte aligned shared memory)
+        auto scale64 = [&](uint32_t src, uint32_t dst, const float *f) {
+            float v0[32], v1[32];
+            tmem_ld32(tm + lrow + src, v0);
+            tmem_ld32(tm + lrow + src + 32, v1);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; i += 4) {
+                const float4 a = *reinterpret_cast<const float4 *>(f + i);
+                const float4 b = *reinterpret_cast<const float4 *>(f + 32 + i);
+                v0[i] *= a.x; v0[i + 1] *= a.y; v0[i + 2] *= a.z; v0[i + 3] *= a.w;
+                v1[i] *= b.x; v1[i + 1] *= b.y; v1[i + 2] *= b.z; v1[i + 3] *= b.w;
+            }
+            tmem_st32(tm + lrow + dst, v0);
+            tmem_st32(tm + lrow + dst + 32, v1);
+        };
         for (int c = 0; c < nchunks; ++c) {
             const uint32_t par = c & 1;
             const int bsel = c & 1;
             const int n = min(kChunk, L - (cb + c) * kChunk);
             const int64_t tok = seq0 + (int64_t)(cb + c) * kChunk;
-            if (!ewait(B_1, par)) break;
-            if (!ewait(B_GR0 + bsel, (c >> 1) & 1)) break;   // the gates record of c
+            {  // MMA_1 done and the gates record of c here (one poll round for both)
+                bool ok = true;
+                if (leader) ok = wait_or_abort(&bar[B_1], par, abort_flag) &&
+                                 wait_or_abort(&bar[B_GR0 + bsel], (c >> 1) & 1, abort_flag);
+                if (bar_or(kBarEpi, 128, !ok)) break;
+            }
             fence_after_sync();
             const float *gr = (const float *)(sm + OFF_GR + bsel * kGateRec * 4);
-#pragma unroll
-            for (int h2 = 0; h2 < 2; ++h2) {  // Y = gamma Y1, the base MMA_4 accumulates onto
-                float v[32];
-                tmem_ld32(tm + lrow + T_XY + 64 + 32 * h2, v);
-                tmem_wait_ld();
-#pragma unroll
-                for (int i = 0; i < 32; ++i) v[i] *= gr[kGrGamma + 32 * h2 + i];
-                tmem_st32(tm + lrow + T_Y + 32 * h2, v);
-            }
+            scale64(T_XY, T_XY, gr + kGrGamma);            // X' = X diag(gamma), for MMA_2b
+            publish(B_XS);
+            scale64(T_XY + 64, T_Y, gr + kGrGamma);        // Y = Y1 diag(gamma), for MMA_4
             {  // S^T *= gamma_C (last read by MMA_1; MMA_3 accumulates onto it)
                 const float gc = gr[kGrGammaC];
 #pragma unroll
@@ -346,10 +371,11 @@ __global__ void __launch_bounds__(kThr, 1) prefill_tc_kernel(const __grid_consta
                     tmem_st32(tm + lrow + T_S + d0, v);
                 }
             }
-            tmem_wait_st();
-            fence_before_sync();
-            bar_sync(kBarEpi, 128);
-            if (leader) mbar_arrive(&bar[B_Y1]);
+            publish(B_Y1);
+            if (!ewait(B_2, par)) break;
+            fence_after_sync();
+            scale64(T_U, T_UT, gr + kGrKd);                // u~ = u diag(kd), for MMA_3
+            publish(B_UT);
             if (!ewait(B_4, par)) break;
             fence_after_sync();
             if (n == kChunk) {
@@ -463,7 +489,7 @@ cudaError_t launch_prefill_tc(const ScanParams &sp, int64_t total_tokens, bool /
                               bool out_bf16, cudaStream_t s) {
     if (sp.n_seqs <= 0) return cudaSuccess;
     TcParams p{};
-    p.kq = sp.kq; p.kt = sp.kt; p.vi = sp.vi; p.tb = sp.tb; p.w2 = sp.w2; p.pm = sp.pm; p.gr = sp.gr;
+    p.kq = sp.kq; p.kmn = sp.kmn; p.vi = sp.vi; p.tb = sp.tb; p.pm = sp.pm; p.gr = sp.gr;
     p.cu = sp.cu; p.cfirst = sp.cfirst; p.init = sp.init; p.carry_in = sp.carry_in; p.carry_out = sp.carry_out;
     p.chunk_lo = sp.chunk_lo; p.chunk_hi = sp.chunk_hi;
     p.out = sp.out; p.n_seqs = sp.n_seqs; p.n_qk = sp.n_qk; p.n_v = sp.n_v;
