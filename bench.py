@@ -45,14 +45,16 @@ CHUNK = 64
 # + K.K^T and Q.K^T (2 C d each, shared by the 3 V heads of a QK head)
 PREFILL_FLOP_TV = 6 * D * D + 2 * CHUNK * D * (3 + 2 / 3)
 # tensor-core work of the chunk-chain kernel per (token, V head): S^T[K;Q]^T (4 d^2),
-# V^T T_beta^T and X W2^T (2 C d each), u^T K~ (2 d^2), u^T P^T (2 C d)
+# V^T T_beta^T and X' T_beta^T (2 C d each), u~^T K (2 d^2), u^T P^T (2 C d)
 CHAIN_FLOP_TV = 6 * D * D + 3 * 2 * CHUNK * D
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
                   "sm_max_mhz": 1965.0}
 TF32_PER_BF16 = 1.1 / 2.25   # nominal dense tf32 : bf16 tensor throughput on B200
 # dram__bytes_read.sum + dram__bytes_write.sum per launch from one ncu capture of the current
-# kernels on this workload (profiles/prefill_tc_T8192_ncu.md, profiles/decode_B256_ncu.md)
-NCU_TRAFFIC_BYTES = {"prefill_tc": 842_870_784 + 186_638_336, "decode": 826_713_088 + 769_751_552}
+# kernels on this workload (profiles/prefill_tc_T8192_ncu.md: one chain launch of the step's
+# four chunk ranges, 2048 tokens; profiles/decode_B256_ncu.md); None while a kernel has
+# changed since its capture
+NCU_TRAFFIC_BYTES = {"prefill_tc": 159_953_408 + 33_269_504, "decode": 826_713_088 + 769_751_552}
 FP32_LANES_PER_SM = 128
 N_SM = 148
 
@@ -207,20 +209,26 @@ def bench_prefill(args, dist, torch, gdn, peaks):
     K = args.steps
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
           for _ in range(K)]
-    trace = gdn.LaunchTrace(capacity=16 * K)
     clocks = ClockSampler(device_id_for_smi())
     dist.barrier()
     clocks.start()
-    with trace:
-        for i in range(K):
-            flush.zero_()
-            ev[i][0].record()
-            call()
-            ev[i][1].record()
+    for i in range(K):
+        flush.zero_()
+        ev[i][0].record()
+        call()
+        ev[i][1].record()
     dist.barrier()
     clk = clocks.stop()
     ms = sum(a.elapsed_time(b) for a, b in ev)
     ms_max = dist.max(ms)
+    # per-kernel durations: the same K steps again under the launch trace (its events add a
+    # little time of their own, so the steps above run without it)
+    trace = gdn.LaunchTrace(capacity=16 * K)
+    with trace:
+        for i in range(K):
+            flush.zero_()
+            call()
+    dist.barrier()
     recs = trace.records()
     per_kernel = {}
     for name, t in recs:
@@ -253,7 +261,7 @@ def bench_prefill(args, dist, torch, gdn, peaks):
         "value": tokens_all / (ms_max / 1e3), "ms_per_step": ms_max / K, "clocks": clk,
         "per_kernel": {n: {"launches": len(v), "avg_ms": sum(v) / len(v), "total_ms": sum(v)}
                        for n, v in per_kernel.items()},
-        "launches": trace.count, "tokens_per_launch": T, "n_v_heads": shape.n_v_heads,
+        "launches": trace.count, "tokens_per_step": T, "steps": K, "n_v_heads": shape.n_v_heads,
         "e2e": {"value": tokens_all / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / K},
     }
@@ -263,7 +271,10 @@ def prefill_roofline(res, peaks, peak_src):
     pk = res["per_kernel"]
     dom = max(pk, key=lambda n: pk[n]["total_ms"])
     avg_s = pk[dom]["avg_ms"] / 1e3
-    T, Hv = res["tokens_per_launch"], res["n_v_heads"]
+    # a step may run a kernel several times over consecutive chunk ranges (pipelined path):
+    # the work of one launch is the step's tokens over its launches per step
+    T = res["tokens_per_step"] * res["steps"] / pk[dom]["launches"]
+    Hv = res["n_v_heads"]
     step_ms = sum(v["total_ms"] for v in pk.values())
     share = {n: round(v["total_ms"] / step_ms, 4) for n, v in pk.items()}
     if dom == "scan_simt":
@@ -272,7 +283,7 @@ def prefill_roofline(res, peaks, peak_src):
         return {"kernel": dom, "bound": "alu", "achieved": flops / avg_s / 1e12, "peak": peak,
                 "unit": "TFLOP/s", "frac": flops / avg_s / 1e12 / peak, "traffic": None,
                 "peak_source": f"148 SMs x 128 fp32 FMA lanes x 2 x {peaks.get('sm_max_mhz')} MHz",
-                "algorithmic_per_launch": flops, "kernel_share": share}
+                "algorithmic_per_launch": flops, "tokens_per_launch": T, "kernel_share": share}
     if dom.startswith("prefill_tc"):
         flops = CHAIN_FLOP_TV * T * Hv
         peak = peaks["bf16_tflops"] * TF32_PER_BF16
@@ -280,7 +291,7 @@ def prefill_roofline(res, peaks, peak_src):
                 "unit": "TFLOP/s", "frac": flops / avg_s / 1e12 / peak,
                 "traffic": NCU_TRAFFIC_BYTES.get("prefill_tc"),
                 "peak_source": f"tf32 = {peak_src} bf16 {peaks['bf16_tflops']} x 1.1/2.25 nominal",
-                "algorithmic_per_launch": flops, "kernel_share": share}
+                "algorithmic_per_launch": flops, "tokens_per_launch": T, "kernel_share": share}
     # a memory-bound kernel dominates
     byts = (2 * 16 * D * 2 + 48 * D * 2 + 3 * 16 * 4 * D) * T
     return {"kernel": dom, "bound": "hbm", "achieved": byts / avg_s / 1e9, "peak": peaks["hbm_gbs"],
@@ -480,7 +491,7 @@ def main():
         line = {
             "metric": METRIC, "value": pre["value"], "unit": UNIT, "n_gpus": dist.world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": pre["ms_per_step"],
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "tf32",
             "data": "synthetic",
             "config": {"workload": gi.WORKLOADS[1]["name"], "T": 8192, "n_qk_heads": 16,
                        "n_v_heads": 48, "d": D, "chunk": CHUNK, "inputs": "bf16",

@@ -180,7 +180,7 @@ GDN_EXPORT gdn_status gdn_decode_step(const gdn_config *cfg, gdn_dtype dtype, gd
  * loading, the GPUs on which this entry point is used), kept until the process exits.
  *  - Limit: problems whose gdn_prefill_workspace_size() exceeds GDN_STATIC_SCRATCH_BYTES
  *    are rejected with GDN_ERR_WORKSPACE before anything is enqueued (at 16 QK / 48 V
- *    heads that is roughly 1,600 tokens per call).
+ *    heads that is roughly 750 tokens per call for bf16 input, 1,600 for fp32 input).
  *  - Allocation: none; it calls no cudaMalloc, cudaFree or allocating library routine.
  *  - Set-up: the first call on each device (with that device current) looks up the
  *    array's device address with cudaGetSymbolAddress; make that first call before any
