@@ -3,11 +3,16 @@
 // Page "ARCHITECTURE PREVIEW / FIELD NOTES", section 03: q, k and v each pass a
 // kernel-4 ShortConv before the gated delta rule.  The conv is causal and depthwise
 // with tap 3 on the current row; q and k are then L2-normalised per (token, head).
-// Memory-bound: each raw row is read once (plus a 3-row halo per 16-row strip, served
-// by L2) and each normalised row written once, in fp32 (rounding these rows to bf16
-// would by itself move y by several percent of its rms).
+// Memory-bound: each raw row is read once (plus a 3-row halo per chunk or 16-row strip,
+// served by L2) and each normalised row written once, in fp32 (rounding these rows to
+// bf16 would by itself move y by several percent of its rms).
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include "gdn_common.cuh"
 #include "gdn_internal.h"
+#include "tc_sm100.cuh"
+#include "tma_map.cuh"
 
 namespace gdn {
 
@@ -82,18 +87,10 @@ cudaError_t launch_seq_table(const int32_t *cu_in, int n_seqs, int64_t T, int32_
 }
 
 // ------------------------------------------------------------------------ conv + L2
-// grid (max_chunks, 2*Hqk + Hv): CTA = one 64-row chunk of one head slot (q heads,
-// then k heads, then v heads).  Warp w walks rows 16w..16w+15 in order, keeping the
-// 3-row conv history of its lane's 4 channels in registers.
-// kTiles: instead of fp32 rows, write the tensor-core path's chunk tiles, TF32-rounded (the
-// MMAs read them as TF32; rounding here gives round-to-nearest instead of truncation), in
-// the shared-memory layouts the tensor-core kernels copy them into:
-//   [K;Q] of (chunk, QK head): 4 blocks of 32 features x (K 64 rows | Q 64 rows), 128-byte
-//     rows with 16-byte chunks XOR-swizzled by row (K-major operand layout);
-//   K of (chunk, QK head) and V of (chunk, V head): 4 blocks of 32 features x 64 rows,
-//     128-byte rows with 32-byte granules XOR-swizzled by row (MN-major operand layout).
-// Rows past the end of the sequence are written as zeros.
-template <class T, bool kTiles>
+// fp32 rows (fp32-input path).  grid (max_chunks, 2*Hqk + Hv): CTA = one 64-row chunk of
+// one head slot (q heads, then k heads, then v heads).  Warp w walks rows 16w..16w+15 in
+// order, keeping the 3-row conv history of its lane's 4 channels in registers.
+template <class T>
 __global__ void __launch_bounds__(128) conv_l2_kernel(ConvParams p) {
     const int n_chunks = p.cfirst[p.n_seqs];
     const int ci = (int)(p.chunk_lo + blockIdx.x);
@@ -102,7 +99,6 @@ __global__ void __launch_bounds__(128) conv_l2_kernel(ConvParams p) {
     const int seq0 = p.cu[b], seq1 = p.cu[b + 1];
     const int r0 = (ci - p.cfirst[b]) * kChunk;  // chunk start within the sequence
     const int len = min(kChunk, seq1 - seq0 - r0);
-    if (kTiles && blockIdx.y == 0 && threadIdx.x == 0) p.cseq[ci] = b;   // for the chunk-prep pass
 
     const int slot = blockIdx.y;
     const T *x;
@@ -135,28 +131,7 @@ __global__ void __launch_bounds__(128) conv_l2_kernel(ConvParams p) {
     }
     const int rs = r0 + wid * 16;                  // first row of this warp (in sequence)
     const int re = min(rs + 16, r0 + len);
-    if (!kTiles && rs >= re) return;
-    // tile destinations (float offsets of this lane's 4 features, row 0)
-    float *t_a = nullptr, *t_b = nullptr;          // K-major ([K;Q]) and MN-major (K or V) tile
-    if (kTiles) {
-        if (slot < p.n_qk) {
-            t_a = p.kq + ((int64_t)ci * p.n_qk + slot) * 16384 + 2048;
-        } else if (slot < 2 * p.n_qk) {
-            t_a = p.kq + ((int64_t)ci * p.n_qk + slot - p.n_qk) * 16384;
-            t_b = p.kmn + ((int64_t)ci * p.n_qk + slot - p.n_qk) * 8192;
-        } else {
-            t_b = p.vi + ((int64_t)ci * p.n_v + slot - 2 * p.n_qk) * 8192;
-        }
-    }
-    auto put_tile = [&](int t, const float y[4]) {  // row t of the chunk
-        if (t_a) st4(t_a + (lane >> 3) * 4096 + t * 32 + (((lane & 7) ^ (t & 7)) << 2), y);
-        if (t_b) st4(t_b + (lane >> 3) * 2048 + t * 32 + ((((lane & 7) >> 1) ^ (t & 3)) << 3) + (lane & 1) * 4, y);
-    };
-    if (kTiles) {  // rows of this warp past the end of the sequence
-        const float z[4] = {0.f, 0.f, 0.f, 0.f};
-        for (int s = max(rs, r0 + len); s < r0 + wid * 16 + 16; ++s) put_tile(s - r0, z);
-        if (rs >= re) return;
-    }
+    if (rs >= re) return;
     // history rows rs-3, rs-2, rs-1
     float h[3][4];
 #pragma unroll
@@ -186,29 +161,202 @@ __global__ void __launch_bounds__(128) conv_l2_kernel(ConvParams p) {
 #pragma unroll
             for (int c = 0; c < 4; ++c) y[c] *= inv;
         }
-        if (kTiles) {
+        st4(dst + (int64_t)(seq0 + s) * row_stride + c4, y);
+    }
+}
+
+// ------------------------------------------------------------------------ conv + L2, tiles
+// The tensor-core path's tiles from bf16 input.  CTA = one 64-row chunk of one head slot:
+// q heads ([K;Q] tile, Q half), k heads ([K;Q] tile, K half), k heads again (the K tile,
+// MN-major), v heads (the V tile, MN-major).  One TMA copy brings the chunk's rows and the
+// 3 rows before them (rows outside the tensor read as zero; at a sequence's start the 3
+// history rows are replaced by the conv state or zeros); each warp then walks 16 rows from
+// shared memory, writes the TF32-rounded rows into an image of the tile in shared memory,
+// and the image leaves by bulk stores, so every global access of the kernel is a bulk
+// transfer.
+namespace {
+using namespace tc;
+
+constexpr int kSlabRows = kChunk + 3;
+constexpr uint32_t kSlabBytes = kSlabRows * kHeadDim * 2;   // bf16 rows, 17,152 B
+constexpr uint32_t C_SLAB = 0;
+constexpr uint32_t C_STAGE = 17408;                          // tile image, 32 KB
+constexpr uint32_t C_BAR = C_STAGE + 32768;
+constexpr uint32_t kConvSmem = C_BAR + 16;
+constexpr uint32_t kConvSmemAlloc = kConvSmem + 1024;
+constexpr uint32_t kConvWaitTries = 1u << 24;
+
+struct ConvTileParams {
+    CUtensorMap tm_q, tm_k, tm_v;   // [T, H*128] bf16 rows, boxes of 128 columns x 67 rows
+    const float *wq, *wk, *wv;      // [ch, 4]
+    const void *conv_in;            // [n_seqs, 3, channels] bf16 or null
+    float *kq, *kmn, *vi;
+    int32_t *cseq;
+    const int32_t *cu, *cfirst;
+    int n_seqs, n_qk, n_v;
+    float q_scale, eps;
+    int64_t chunk_lo;
+};
+
+// largest b in [0, n) with first[b] <= i (first non-decreasing, first[0] <= i < first[n]),
+// found by the whole warp: each step reads 32 points of the remaining range at once
+__device__ __forceinline__ int upper_index_warp(const int32_t *first, int n, int i) {
+    const int lane = threadIdx.x & 31;
+    int lo = 0, hi = n;   // first[lo] <= i, answer in [lo, hi)
+    while (hi - lo > 32) {
+        const int step = (hi - lo + 31) / 32;
+        const int k = lo + lane * step;
+        const unsigned m = __ballot_sync(0xffffffffu, k < hi && __ldg(first + k) <= i);
+        lo += (31 - __clz(m)) * step;
+        hi = min(hi, lo + step);
+    }
+    const int k = lo + lane;
+    const unsigned m = __ballot_sync(0xffffffffu, k < hi && __ldg(first + k) <= i);
+    return lo + (31 - __clz(m));
+}
+
+__device__ __forceinline__ void bf16x4_to_f32(uint2 r, float v[4]) {
+    v[0] = __uint_as_float(r.x << 16);
+    v[1] = __uint_as_float(r.x & 0xffff0000u);
+    v[2] = __uint_as_float(r.y << 16);
+    v[3] = __uint_as_float(r.y & 0xffff0000u);
+}
+
+}  // namespace
+
+__global__ void __launch_bounds__(128) conv_tiles_kernel(const __grid_constant__ ConvTileParams p) {
+    const int n_chunks = p.cfirst[p.n_seqs];
+    const int ci = (int)(p.chunk_lo + blockIdx.x);
+    if (ci >= n_chunks) return;
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    const int b = upper_index_warp(p.cfirst, p.n_seqs, ci);
+    const int seq0 = p.cu[b], seq1 = p.cu[b + 1];
+    const int r0 = (ci - p.cfirst[b]) * kChunk;   // chunk start within the sequence
+    const int len = min(kChunk, seq1 - seq0 - r0);
+    if (blockIdx.y == 0 && threadIdx.x == 0) p.cseq[ci] = b;   // for the chunk-prep pass
+
+    // slot kinds: 0 q ([K;Q] Q half), 1 k ([K;Q] K half), 2 k (K tile), 3 v (V tile)
+    const int slot = blockIdx.y, nq = p.n_qk;
+    const int kind = slot < nq ? 0 : slot < 2 * nq ? 1 : slot < 3 * nq ? 2 : 3;
+    const int head = kind == 3 ? slot - 3 * nq : slot - kind * nq;
+    const CUtensorMap *tm = kind == 0 ? &p.tm_q : kind == 3 ? &p.tm_v : &p.tm_k;
+    const float *w = kind == 0 ? p.wq : kind == 3 ? p.wv : p.wk;
+    const int qkc = nq * kHeadDim;
+    const int cs_chan = (kind == 0 ? 0 : kind == 3 ? 2 * qkc : qkc) + head * kHeadDim;
+    const bool norm = kind != 3;
+    const float scale = kind == 0 ? p.q_scale : 1.f;
+
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char *sm = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
+    uint64_t *bar = (uint64_t *)(sm + C_BAR);
+    if (threadIdx.x == 0) {
+        mbar_init(bar, 1);
+        mbar_expect_tx(bar, kSlabBytes);
+        tma_load_2d(smem_u32(sm + C_SLAB), tm, head * kHeadDim, seq0 + r0 - 3, bar);
+    }
+    float wt[4][4];  // wt[channel][tap], this lane's 4 channels
 #pragma unroll
-            for (int c = 0; c < 4; ++c)  // TF32, nearest with ties away (integer ops)
-                y[c] = __uint_as_float((__float_as_uint(y[c]) + 0x1000u) & 0xFFFFE000u);
-            put_tile(s - r0, y);
-        } else {
-            st4(dst + (int64_t)(seq0 + s) * row_stride + c4, y);
+    for (int c = 0; c < 4; ++c) {
+        const float4 t = *reinterpret_cast<const float4 *>(w + (int64_t)(head * kHeadDim + 4 * lane + c) * kConvW);
+        wt[c][0] = t.x; wt[c][1] = t.y; wt[c][2] = t.z; wt[c][3] = t.w;
+    }
+    __syncthreads();   // the barrier is initialised
+    const bool ok = mbar_wait(bar, 0, kConvWaitTries);
+    if (r0 == 0 && threadIdx.x < 96) {   // history rows of a sequence's first chunk
+        const int j = threadIdx.x >> 5;   // slab row j = row j - 3 of the sequence
+        uint2 h = make_uint2(0u, 0u);
+        if (p.conv_in) {
+            const int64_t cs_row = 2 * (int64_t)qkc + (int64_t)p.n_v * kHeadDim;
+            h = *reinterpret_cast<const uint2 *>((const bf16 *)p.conv_in + ((int64_t)b * 3 + j) * cs_row +
+                                                 cs_chan + 4 * lane);
         }
+        *reinterpret_cast<uint2 *>(sm + C_SLAB + j * 256 + lane * 8) = h;
+    }
+    __syncthreads();
+
+    const unsigned char *slab = sm + C_SLAB + lane * 8;
+    float h[3][4];
+#pragma unroll
+    for (int j = 0; j < 3; ++j) bf16x4_to_f32(*reinterpret_cast<const uint2 *>(slab + (16 * wid + j) * 256), h[j]);
+    const bool mn = kind >= 2;
+    const float nan = __int_as_float(0x7fc00000);
+#pragma unroll 4
+    for (int i = 0; i < 16; ++i) {
+        const int t = 16 * wid + i;
+        float cur[4], y[4];
+        bf16x4_to_f32(*reinterpret_cast<const uint2 *>(slab + (t + 3) * 256), cur);
+        float ss = 0.f;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            y[c] = wt[c][0] * h[0][c] + wt[c][1] * h[1][c] + wt[c][2] * h[2][c] + wt[c][3] * cur[c];
+            ss += y[c] * y[c];
+            h[0][c] = h[1][c]; h[1][c] = h[2][c]; h[2][c] = cur[c];
+        }
+        if (norm) {
+            ss = warp_sum(ss);
+            const float inv = scale * rsqrtf(ss + p.eps);
+#pragma unroll
+            for (int c = 0; c < 4; ++c) y[c] *= inv;
+        }
+        float4 o;   // TF32, nearest with ties away (integer ops); rows past the end are zero
+        o.x = t < len ? __uint_as_float((__float_as_uint(y[0]) + 0x1000u) & 0xFFFFE000u) : 0.f;
+        o.y = t < len ? __uint_as_float((__float_as_uint(y[1]) + 0x1000u) & 0xFFFFE000u) : 0.f;
+        o.z = t < len ? __uint_as_float((__float_as_uint(y[2]) + 0x1000u) & 0xFFFFE000u) : 0.f;
+        o.w = t < len ? __uint_as_float((__float_as_uint(y[3]) + 0x1000u) & 0xFFFFE000u) : 0.f;
+        if (!ok) o = make_float4(nan, nan, nan, nan);
+        const uint32_t off = (lane >> 3) * 8192 + t * 128 +
+                             (mn ? ((((lane & 7) >> 1) ^ (t & 3)) << 5) + (lane & 1) * 16
+                                 : (((lane & 7) ^ (t & 7)) << 4));
+        *reinterpret_cast<float4 *>(sm + C_STAGE + off) = o;
+    }
+    fence_smem_to_async();
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        const uint32_t st = smem_u32(sm + C_STAGE);
+        if (kind <= 1) {   // the 4 feature blocks of the Q or K half of the [K;Q] tile
+            float *dst = p.kq + ((int64_t)ci * nq + head) * 16384 + (kind == 0 ? 2048 : 0);
+#pragma unroll
+            for (int blk = 0; blk < 4; ++blk) bulk_store_s2g(dst + blk * 4096, st + blk * 8192, 8192);
+        } else {
+            float *dst = kind == 2 ? p.kmn + ((int64_t)ci * nq + head) * 8192
+                                   : p.vi + ((int64_t)ci * p.n_v + head) * 8192;
+            bulk_store_s2g(dst, st, 32768);
+        }
+        bulk_commit();
+        bulk_wait_read0();   // the image is read before the CTA's shared memory goes away
     }
 }
 
 cudaError_t launch_conv_l2(const ConvParams &p, bool bf16, bool tiles, int64_t n_chunks,
-                           cudaStream_t s) {
+                           int64_t total_tokens, cudaStream_t s) {
     if (n_chunks <= 0) return cudaSuccess;
+    if (tiles) {   // tensor-core path: bf16 input only
+        if (!bf16) return cudaErrorInvalidValue;
+        ConvTileParams tp{};
+        const int64_t qkc = (int64_t)p.n_qk * kHeadDim, vc = (int64_t)p.n_v * kHeadDim;
+        if (!encode_2d(&tp.tm_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.q, qkc, total_tokens, qkc * 2, kHeadDim,
+                       kSlabRows, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+            !encode_2d(&tp.tm_k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.k, qkc, total_tokens, qkc * 2, kHeadDim,
+                       kSlabRows, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+            !encode_2d(&tp.tm_v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.v, vc, total_tokens, vc * 2, kHeadDim,
+                       kSlabRows, CU_TENSOR_MAP_SWIZZLE_NONE))
+            return cudaErrorInvalidValue;
+        tp.wq = p.wq; tp.wk = p.wk; tp.wv = p.wv; tp.conv_in = p.conv_in;
+        tp.kq = p.kq; tp.kmn = p.kmn; tp.vi = p.vi; tp.cseq = p.cseq; tp.cu = p.cu; tp.cfirst = p.cfirst;
+        tp.n_seqs = p.n_seqs; tp.n_qk = p.n_qk; tp.n_v = p.n_v; tp.q_scale = p.q_scale; tp.eps = p.eps;
+        tp.chunk_lo = p.chunk_lo;
+        cudaError_t e = cudaFuncSetAttribute(conv_tiles_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)kConvSmemAlloc);
+        if (e != cudaSuccess) return e;
+        dim3 grid((unsigned)n_chunks, 3 * p.n_qk + p.n_v);
+        TraceLaunch tl(s, "conv_l2");
+        conv_tiles_kernel<<<grid, 128, kConvSmemAlloc, s>>>(tp);
+        return cudaGetLastError();
+    }
     dim3 grid((unsigned)n_chunks, 2 * p.n_qk + p.n_v);
     TraceLaunch tl(s, "conv_l2");
-    if (bf16) {
-        if (tiles) conv_l2_kernel<gdn::bf16, true><<<grid, 128, 0, s>>>(p);
-        else conv_l2_kernel<gdn::bf16, false><<<grid, 128, 0, s>>>(p);
-    } else {
-        if (tiles) conv_l2_kernel<float, true><<<grid, 128, 0, s>>>(p);
-        else conv_l2_kernel<float, false><<<grid, 128, 0, s>>>(p);
-    }
+    if (bf16) conv_l2_kernel<gdn::bf16><<<grid, 128, 0, s>>>(p);
+    else conv_l2_kernel<float><<<grid, 128, 0, s>>>(p);
     return cudaGetLastError();
 }
 

@@ -237,7 +237,7 @@ gdn_status gdn_prefill(const gdn_config *cfg, gdn_dtype dtype, gdn_dtype out_dty
         // bf16 inputs run the tensor-core (TF32) prefill, fp32 inputs the fp32 CUDA-core one;
         // the pipelined tensor-core path launches the conv per chunk range below
         if (L.n_segments == 1) {
-            e = launch_conv_l2(cp, bf, /*tiles=*/bf, L.max_chunks, stream);
+            e = launch_conv_l2(cp, bf, /*tiles=*/bf, L.max_chunks, total_tokens, stream);
             if (e != cudaSuccess) return cuda_fail(e);
         }
     }
@@ -284,7 +284,7 @@ gdn_status gdn_prefill(const gdn_config *cfg, gdn_dtype dtype, gdn_dtype out_dty
                 const int64_t lo = sg * per, hi = std::min<int64_t>(L.max_chunks, lo + per);
                 cp.chunk_lo = sp.chunk_lo = lo;
                 sp.chunk_hi = hi;
-                e = launch_conv_l2(cp, bf, /*tiles=*/true, hi - lo, aux->stream);
+                e = launch_conv_l2(cp, bf, /*tiles=*/true, hi - lo, total_tokens, aux->stream);
                 if (e == cudaSuccess) e = launch_chunk_prep(sp, total_tokens, bf, aux->stream);
                 if (e == cudaSuccess) e = cudaEventRecord(aux->ev[1 + sg], aux->stream);
                 if (e == cudaSuccess) e = cudaStreamWaitEvent(stream, aux->ev[1 + sg], 0);

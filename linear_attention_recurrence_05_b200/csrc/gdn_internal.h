@@ -107,7 +107,7 @@ cudaError_t launch_seq_table(const int32_t *cu_in, int n_seqs, int64_t T, int32_
                              int32_t *cfirst, cudaStream_t s);
 // tiles: write the tensor-core chunk tiles (TF32-rounded) instead of fp32 rows
 cudaError_t launch_conv_l2(const ConvParams &p, bool bf16, bool tiles, int64_t n_chunks,
-                           cudaStream_t s);
+                           int64_t total_tokens, cudaStream_t s);
 cudaError_t launch_conv_state_out(const void *q, const void *k, const void *v,
                                   const void *conv_in, void *conv_out, const int32_t *cu,
                                   int n_seqs, int n_qk, int n_v, bool bf16, cudaStream_t s);

@@ -274,6 +274,12 @@ __device__ __forceinline__ void tma_store_2d(const void *tmap, int x, int y, uin
                  "r"(x), "r"(y), "r"(src)
                  : "memory");
 }
+// contiguous bulk copy shared (this CTA) -> global, tracked as a bulk async-group; both
+// addresses 16-byte aligned, `bytes` a multiple of 16
+__device__ __forceinline__ void bulk_store_s2g(void *dst, uint32_t src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst), "r"(src), "r"(bytes)
+                 : "memory");
+}
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 // wait until this thread's bulk groups have finished reading shared memory
 __device__ __forceinline__ void bulk_wait_read0() {
