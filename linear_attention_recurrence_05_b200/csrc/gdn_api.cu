@@ -241,11 +241,6 @@ gdn_status gdn_prefill(const gdn_config *cfg, gdn_dtype dtype, gdn_dtype out_dty
             if (e != cudaSuccess) return cuda_fail(e);
         }
     }
-    if (conv_state_out) {
-        e = launch_conv_state_out(q, k, v, conv_state_in, conv_state_out, cu, n_seqs,
-                                  cfg->n_qk_heads, cfg->n_v_heads, bf, stream);
-        if (e != cudaSuccess) return cuda_fail(e);
-    }
     ScanParams sp{};
     sp.qh = (const float *)(ws + L.off_qh); sp.kh = (const float *)(ws + L.off_kh);
     sp.vh = (const float *)(ws + L.off_vh);
@@ -295,6 +290,13 @@ gdn_status gdn_prefill(const gdn_config *cfg, gdn_dtype dtype, gdn_dtype out_dty
         e = launch_scan_simt(sp, bf, out_dtype == GDN_BF16, stream);
     }
     if (e != cudaSuccess) return cuda_fail(e);
+    // last, on the caller's stream: every kernel that reads conv_state_in (the conv passes on
+    // either stream) is ordered before this one, so conv_state_out may alias it
+    if (conv_state_out) {
+        e = launch_conv_state_out(q, k, v, conv_state_in, conv_state_out, cu, n_seqs,
+                                  cfg->n_qk_heads, cfg->n_v_heads, bf, stream);
+        if (e != cudaSuccess) return cuda_fail(e);
+    }
     return GDN_OK;
 }
 

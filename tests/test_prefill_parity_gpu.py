@@ -84,12 +84,19 @@ def test_pipelined_chunk_ranges(lib):
     alias = st.clone()
     y_alias, fin_alias, _ = lib.gdn_prefill(*args, cu, cfg=cfg, initial_state=alias, final_state=alias,
                                             conv_state_in=cs)
+    # the conv state updated in place: every range's conv pass (on the second stream) and
+    # every chain must read the old one
+    cs_alias = cs.clone()
+    y_csal, _, _ = lib.gdn_prefill(*args, cu, cfg=cfg, initial_state=st.clone(), conv_state_in=cs_alias,
+                                   conv_state_out=cs_alias)
     torch.cuda.synchronize()
     assert fin_none is None
-    yo, fo, _ = oracle.prefill(inp)
+    yo, fo, co = oracle.prefill(inp)
     assert rel_err(to_host_f64(y_nofin), yo) <= tol(d)
     assert rel_err(to_host_f64(y_alias), yo) <= tol(d)
     assert rel_err(to_host_f64(fin_alias), fo) <= tol(d)
+    assert rel_err(to_host_f64(y_csal), yo) <= tol(d)
+    assert np.array_equal(to_host_f64(cs_alias), co)
 
 
 def test_state_aliasing(lib):
