@@ -62,6 +62,17 @@ def test_pages_heads_short(lib, dtype):
     _check(inp, lib, label=f"h16x48-{dtype}")
 
 
+@pytest.mark.parametrize("heads", [(2, 2), (2, 4), (1, 4), (2, 10)])
+def test_head_ratios(lib, heads):
+    """V heads per QK head other than 3: the chunk-prep pass then serves 1 or 2 V heads per CTA
+    (ratios 1, 2, 4, 5), and the V -> QK head map changes; ragged lengths, initial and conv
+    states."""
+    shape = gi.GdnShape(n_qk_heads=heads[0], n_v_heads=heads[1])
+    inp = gi.make_prefill_inputs(shape, [130, 1, 64, 200], gi.BF16, seed=83 + heads[1],
+                                 with_initial_state=True, with_conv_state=True)
+    _check(inp, lib, label=f"h{heads[0]}x{heads[1]}")
+
+
 def test_pipelined_chunk_ranges(lib):
     """Few (sequence, head) chains and many chunks run as a pipeline over chunk ranges (the
     state carried from range to range): sequences that start, end and lie wholly inside a
