@@ -395,7 +395,10 @@ def bench_decode(args, dist, torch, gdn, peaks, peak_src):
     dist.barrier()
     e2e_ms = dist.max(e2.elapsed_time(e3))
     toks = B * steps * dist.world
+    multi = bench_decode_multi(args, dist, torch, gdn, peaks, peak_src, shape, cfg, (wq, wk, wv),
+                               (dq, dk, dv, da, db), state, conv, state0, conv0)
     return {
+        "multi": multi,
         "value": toks / (ms / 1e3), "unit": UNIT, "workload": w["name"], "batch": B,
         "steps": steps, "ms_per_step": ms / steps, "launches": trace.count, "clocks": clk,
         "roofline": {"kernel": "decode", "bound": "hbm", "achieved": achieved,
@@ -405,6 +408,60 @@ def bench_decode(args, dist, torch, gdn, peaks, peak_src):
         "e2e": {"value": toks / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "note": "host inputs cycle through 32 pinned step sets"},
     }
+
+
+def bench_decode_multi(args, dist, torch, gdn, peaks, peak_src, shape, cfg, wts, inputs, state, conv,
+                       state0, conv0, n_tok=4):
+    """The same token stream as the single-token run, n_tok tokens per call per row
+    (multi-token verification step): tokens/s, and the HBM roofline of the call."""
+    dq, dk, dv, da, db = inputs
+    steps, B = dq.shape[0], dq.shape[1]
+    calls = steps // n_tok
+    if calls == 0:
+        return None
+    # [steps, B, ...] -> [calls, B, n_tok, ...]
+    mq, mk, mv, ma, mb = (x[:calls * n_tok].view((calls, n_tok) + tuple(x.shape[1:])).transpose(1, 2).contiguous()
+                          for x in (dq, dk, dv, da, db))
+    out = torch.empty((B, n_tok, shape.n_v_heads, D), dtype=torch.float32, device="cuda")
+
+    def call(i, **kw):
+        gdn.gdn_decode_multi(mq[i], mk[i], mv[i], *wts, ma[i], mb[i], state, conv, cfg=cfg, out=out, **kw)
+
+    def timed(**kw):
+        state.copy_(state0)
+        conv.copy_(conv0)
+        for i in range(min(args.warmup, calls)):
+            call(i, **kw)
+        state.copy_(state0)
+        conv.copy_(conv0)
+        trace = gdn.LaunchTrace(capacity=calls + 8)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        dist.barrier()
+        with trace:
+            e0.record()
+            for i in range(calls):
+                call(i, **kw)
+            e1.record()
+        dist.barrier()
+        recs = [t for n, t in trace.records() if n == "decode_multi"]
+        return dist.max(e0.elapsed_time(e1)), sum(recs) / len(recs) / 1e3
+
+    ms, avg_s = timed()
+    ch, Hv = shape.channels, shape.n_v_heads
+    bpr = (2 * Hv * D * D * 4 + 6 * ch * 2 + n_tok * (ch * 2 + Hv * D * 4 + 2 * Hv * 2))
+    achieved = bpr * B / avg_s / 1e9
+    # with the state and conv state after every token written out (rollback checkpoints)
+    ck = torch.empty((B, n_tok, Hv, D, D), dtype=torch.float32, device="cuda")
+    cck = torch.empty((B, n_tok, 3, ch), dtype=conv.dtype, device="cuda")
+    ms_ck, _ = timed(state_ckpt=ck, conv_ckpt=cck)
+    del ck, cck
+    toks = B * calls * n_tok * dist.world
+    return {"value": toks / (ms / 1e3), "unit": UNIT, "n_tok": n_tok, "calls": calls, "batch": B,
+            "ms_per_call": ms / calls, "value_with_checkpoints": toks / (ms_ck / 1e3),
+            "roofline": {"kernel": "decode_multi", "bound": "hbm", "achieved": achieved,
+                         "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
+                         "traffic": None, "peak_source": peak_src, "algorithmic_bytes_per_row": bpr,
+                         "rows_per_launch": B}}
 
 
 # ----------------------------------------------------------------------------- oracle

@@ -168,6 +168,37 @@ GDN_EXPORT gdn_status gdn_decode_step(const gdn_config *cfg, gdn_dtype dtype, gd
                            void *out, int batch, cudaStream_t stream);
 
 /*
+ * gdn_decode_multi -- n_tok consecutive tokens for each of `batch` sequences whose states
+ * stay resident (the verification step of speculative or multi-token decoding): the same
+ * recurrence as gdn_decode_step, run over each row's tokens in order, token 0 first.  Each
+ * state is read once and written once per call whatever n_tok is; optionally the state
+ * and conv state after every token are written out, so that a caller that accepts only the
+ * first m tokens can restore the row from checkpoint m-1 (no counterpart on the pages
+ * beyond their use of multi-token speculative decoding).
+ *
+ *   q, k            [batch, n_tok, Hqk, 128] raw rows, dtype; v [batch, n_tok, Hv, 128]
+ *   conv_w_*        as in gdn_prefill
+ *   alpha, beta     [batch, n_tok, Hv] dtype
+ *   state, conv_state, state_slots, n_state_rows
+ *                   as in gdn_decode_step; both advance by all n_tok tokens
+ *   state_ckpt      [batch, n_tok, Hv, 128, 128] fp32 or NULL: the state of row b after its
+ *                   token j at [b][j] (not written for skipped rows)
+ *   conv_ckpt       [batch, n_tok, 3, 2*Hqk*128 + Hv*128] dtype or NULL: the conv state
+ *                   after token j (its last three raw rows, oldest first)
+ *   out             [batch, n_tok, Hv, 128] out_dtype: y of every token
+ *   n_tok           1 .. 8 (GDN_ERR_UNSUPPORTED above)
+ * Errors as gdn_decode_step; the checkpoints must not overlap state or conv_state.
+ */
+GDN_EXPORT gdn_status gdn_decode_multi(const gdn_config *cfg, gdn_dtype dtype, gdn_dtype out_dtype,
+                            const void *q, const void *k, const void *v,
+                            const float *conv_w_q, const float *conv_w_k, const float *conv_w_v,
+                            const void *alpha, const void *beta,
+                            float *state, void *conv_state,
+                            const int32_t *state_slots, int n_state_rows,
+                            float *state_ckpt, void *conv_ckpt,
+                            void *out, int batch, int n_tok, cudaStream_t stream);
+
+/*
  * gdn_prefill_static_scratch -- gdn_prefill without a caller-supplied workspace.
  *
  * No counterpart on the pages: it exists for callers that cannot call cudaMalloc

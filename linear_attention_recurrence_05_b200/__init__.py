@@ -19,7 +19,7 @@ import torch
 from . import _native
 from ._native import GDN_BF16, GDN_F32, GdnError  # noqa: F401
 
-__all__ = ["GdnConfig", "gdn_prefill", "gdn_decode_step", "prefill_workspace_size", "GdnError",
+__all__ = ["GdnConfig", "gdn_prefill", "gdn_decode_step", "gdn_decode_multi", "prefill_workspace_size", "GdnError",
            "library_path"]
 
 
@@ -148,6 +148,40 @@ def gdn_decode_step(q, k, v, conv_w_q, conv_w_k, conv_w_v, alpha, beta, state, c
         _ptr(conv_w_v), _ptr(alpha), _ptr(beta), _ptr(state), _ptr(conv_state), _ptr(state_slots),
         state.shape[0], _ptr(out), B, _stream(stream))
     _native.check("gdn_decode_step", st)
+    return out
+
+
+def gdn_decode_multi(q, k, v, conv_w_q, conv_w_k, conv_w_v, alpha, beta, state, conv_state=None,
+                     *, state_slots=None, state_ckpt=None, conv_ckpt=None, cfg: GdnConfig | None = None,
+                     out=None, out_dtype=torch.float32, stream=None):
+    """n consecutive tokens for each row of the batch; ``state`` (and ``conv_state``) advance by
+    all of them in place.
+
+    q, k [B, n, Hqk, 128], v [B, n, Hv, 128], alpha/beta [B, n, Hv]; state fp32 [R, Hv, 128, 128];
+    conv_state [R, 3, channels] or None; state_slots int32 [B] or None.  ``state_ckpt``
+    (fp32 [B, n, Hv, 128, 128]) and ``conv_ckpt`` ([B, n, 3, channels], q's dtype), when given,
+    receive the state and the conv state after every token.  Returns out [B, n, Hv, 128].
+    """
+    B, n = q.shape[0], q.shape[1]
+    cfg = cfg or GdnConfig(n_qk_heads=q.shape[2], n_v_heads=v.shape[2])
+    code = _dtype_code(q)
+    for t in (k, v, alpha, beta):
+        if t.dtype != q.dtype:
+            raise TypeError("q, k, v, alpha and beta must share one dtype")
+    if state.dtype != torch.float32 or (state_ckpt is not None and state_ckpt.dtype != torch.float32):
+        raise TypeError("state and state_ckpt must be float32")
+    if conv_ckpt is not None and conv_ckpt.dtype != q.dtype:
+        raise TypeError("conv_ckpt must have q's dtype")
+    if state_slots is not None and state_slots.dtype != torch.int32:
+        raise TypeError("state_slots must be int32")
+    if out is None:
+        out = torch.empty((B, n, cfg.n_v_heads, cfg.d_v), dtype=out_dtype, device=q.device)
+    c = cfg.c()
+    st = _native.lib().gdn_decode_multi(
+        ctypes.byref(c), code, _dtype_code(out), _ptr(q), _ptr(k), _ptr(v), _ptr(conv_w_q), _ptr(conv_w_k),
+        _ptr(conv_w_v), _ptr(alpha), _ptr(beta), _ptr(state), _ptr(conv_state), _ptr(state_slots),
+        state.shape[0], _ptr(state_ckpt), _ptr(conv_ckpt), _ptr(out), B, n, _stream(stream))
+    _native.check("gdn_decode_multi", st)
     return out
 
 

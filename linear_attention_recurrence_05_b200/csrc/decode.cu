@@ -170,3 +170,174 @@ cudaError_t launch_decode(const DecodeParams &p, bool in_bf16, bool out_bf16, cu
 }
 
 }  // namespace gdn
+
+// ---------------------------------------------------------------- multi-token decode
+// n_tok consecutive tokens per row (speculative or multi-token verification): the same
+// recurrence run over the row's tokens in order.  The CTA layout is that of the single-token
+// kernel; each V head's state is loaded into registers once, advanced token by token (the
+// two reductions of token j read the state after token j-1) and stored once, so the state
+// traffic of a call does not grow with n_tok.  Optionally the state and the conv state after
+// every token are written out, for rolling back to an accepted prefix.
+namespace gdn {
+
+template <class T, class TO>
+__global__ void __launch_bounds__(kDecThreads, 2) decode_multi_kernel(DecodeParams p) {
+    __shared__ __align__(16) float qs[kMaxDecTok][kHeadDim], ks[kMaxDecTok][kHeadDim], vs[kMaxDecTok][kHeadDim];
+    __shared__ __align__(16) float es[kHeadDim];
+    __shared__ __align__(16) float red_r[kDecWarps][kHeadDim], red_p[kDecWarps][kHeadDim];
+    __shared__ float kq_s[kMaxDecTok];
+
+    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    const int b = blockIdx.x / p.n_qk, g = blockIdx.x % p.n_qk;
+    const int G = p.n_v / p.n_qk, nt = p.n_tok;
+    const int slot = p.slots ? p.slots[b] : b;
+    const int qkc = p.n_qk * kHeadDim;
+    const int64_t ch = 2 * (int64_t)qkc + (int64_t)p.n_v * kHeadDim;
+    TO *outp = (TO *)p.out;
+
+    if (slot < 0 || slot >= p.n_rows) {  // skipped row: zero output, touch no state
+        for (int j = 0; j < nt; ++j)
+            for (int e = tid; e < G * kHeadDim; e += kDecThreads)
+                outp[((int64_t)b * nt + j) * p.n_v * kHeadDim + (int64_t)g * G * kHeadDim + e] = from_f32<TO>(0.f);
+        return;
+    }
+    T *cs = p.conv ? (T *)p.conv + (int64_t)slot * 3 * ch : nullptr;
+    T *cck = (T *)p.conv_ckpt;
+
+    // conv of one channel group over the row's tokens: history rows 0..2 from the conv state
+    // (oldest first), then the tokens; writes y of token j to dst[j]; shifts the conv state
+    // by nt rows and writes the checkpoints (the last 3 rows after each token)
+    auto conv_tokens = [&](const T *x0, int64_t x_stride, const float *w, int wc, int cc, bool norm, float scale,
+                           float (*dst)[kHeadDim]) {
+        float h[3][4];
+#pragma unroll
+        for (int j = 0; j < 3; ++j) {
+            if (cs) ld4(cs + (int64_t)j * ch + cc, h[j]);
+            else h[j][0] = h[j][1] = h[j][2] = h[j][3] = 0.f;
+        }
+        float wt[4][4];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            const float4 t4 = *reinterpret_cast<const float4 *>(w + (int64_t)(wc + c) * kConvW);
+            wt[c][0] = t4.x; wt[c][1] = t4.y; wt[c][2] = t4.z; wt[c][3] = t4.w;
+        }
+        for (int j = 0; j < nt; ++j) {
+            float cur[4], y[4];
+            ld4(x0 + (int64_t)j * x_stride, cur);
+            float ss = 0.f;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                y[c] = wt[c][0] * h[0][c] + wt[c][1] * h[1][c] + wt[c][2] * h[2][c] + wt[c][3] * cur[c];
+                ss += y[c] * y[c];
+                h[0][c] = h[1][c]; h[1][c] = h[2][c]; h[2][c] = cur[c];
+            }
+            if (norm) {
+                ss = warp_sum(ss);
+                const float inv = scale * rsqrtf(ss + p.eps);
+#pragma unroll
+                for (int c = 0; c < 4; ++c) y[c] *= inv;
+            }
+#pragma unroll
+            for (int c = 0; c < 4; ++c) dst[j][4 * lane + c] = y[c];
+            if (cck) {   // conv state after token j: the last three raw rows
+                T *ck = cck + ((int64_t)b * nt + j) * 3 * ch + cc;
+#pragma unroll
+                for (int r = 0; r < 3; ++r) st4(ck + (int64_t)r * ch, h[r]);
+            }
+        }
+        if (cs) {
+#pragma unroll
+            for (int r = 0; r < 3; ++r) st4(cs + (int64_t)r * ch + cc, h[r]);
+        }
+    };
+
+    // ---- q and k of every token: conv (+ conv-state shift) and L2, warps 0 and 1
+    if (wid < 2) {
+        const bool isq = wid == 0;
+        const T *x = (const T *)(isq ? p.q : p.k) + ((int64_t)b * nt * p.n_qk + g) * kHeadDim + 4 * lane;
+        conv_tokens(x, (int64_t)p.n_qk * kHeadDim, isq ? p.wq : p.wk, g * kHeadDim + 4 * lane,
+                    (isq ? 0 : qkc) + g * kHeadDim + 4 * lane, true, isq ? p.q_scale : 1.f, isq ? qs : ks);
+    }
+    __syncthreads();
+    if (wid < nt) {   // k.q of token wid
+        float d = 0.f;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) d += qs[wid][4 * lane + c] * ks[wid][4 * lane + c];
+        d = warp_sum(d);
+        if (lane == 0) kq_s[wid] = d;
+    }
+
+    for (int hh = 0; hh < G; ++hh) {
+        const int h = g * G + hh;
+        if (wid == 2) {   // v of every token for this V head (no normalisation)
+            const T *x = (const T *)p.v + ((int64_t)b * nt * p.n_v + h) * kHeadDim + 4 * lane;
+            conv_tokens(x, (int64_t)p.n_v * kHeadDim, p.wv, h * kHeadDim + 4 * lane,
+                        2 * qkc + h * kHeadDim + 4 * lane, false, 1.f, vs);
+        }
+        float *S = p.state + ((int64_t)slot * p.n_v + h) * kHeadDim * kHeadDim;
+        const int r0 = wid * kRowsPerWarp;
+        float4 s[kRowsPerWarp];
+#pragma unroll
+        for (int i = 0; i < kRowsPerWarp; ++i)
+            s[i] = __ldcs(reinterpret_cast<const float4 *>(S + (int64_t)(r0 + i) * kHeadDim + 4 * lane));
+        __syncthreads();   // vs of this head (and kq_s) are ready
+        for (int j = 0; j < nt; ++j) {
+            const int64_t tv = ((int64_t)b * nt + j) * p.n_v + h;
+            const float a = to_f32(((const T *)p.alpha)[tv]);
+            const float be = to_f32(((const T *)p.beta)[tv]);
+            float rr[4] = {0.f, 0.f, 0.f, 0.f}, pp[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int i = 0; i < kRowsPerWarp; ++i) {
+                const float kr = ks[j][r0 + i], qr = qs[j][r0 + i];
+                rr[0] = fmaf(s[i].x, kr, rr[0]); rr[1] = fmaf(s[i].y, kr, rr[1]);
+                rr[2] = fmaf(s[i].z, kr, rr[2]); rr[3] = fmaf(s[i].w, kr, rr[3]);
+                pp[0] = fmaf(s[i].x, qr, pp[0]); pp[1] = fmaf(s[i].y, qr, pp[1]);
+                pp[2] = fmaf(s[i].z, qr, pp[2]); pp[3] = fmaf(s[i].w, qr, pp[3]);
+            }
+            *reinterpret_cast<float4 *>(&red_r[wid][4 * lane]) = make_float4(rr[0], rr[1], rr[2], rr[3]);
+            *reinterpret_cast<float4 *>(&red_p[wid][4 * lane]) = make_float4(pp[0], pp[1], pp[2], pp[3]);
+            __syncthreads();
+            if (tid < kHeadDim) {
+                float r = 0.f, pq = 0.f;
+#pragma unroll
+                for (int w = 0; w < kDecWarps; ++w) { r += red_r[w][tid]; pq += red_p[w][tid]; }
+                const float e = vs[j][tid] - a * r;
+                es[tid] = e;
+                outp[tv * kHeadDim + tid] = from_f32<TO>(a * pq + be * kq_s[j] * e);
+            }
+            __syncthreads();
+            const float4 e4 = *reinterpret_cast<const float4 *>(&es[4 * lane]);
+            float *ck = p.state_ckpt ? p.state_ckpt + tv * kHeadDim * kHeadDim : nullptr;
+#pragma unroll
+            for (int i = 0; i < kRowsPerWarp; ++i) {
+                const float bk = be * ks[j][r0 + i];
+                s[i].x = fmaf(bk, e4.x, a * s[i].x);
+                s[i].y = fmaf(bk, e4.y, a * s[i].y);
+                s[i].z = fmaf(bk, e4.z, a * s[i].z);
+                s[i].w = fmaf(bk, e4.w, a * s[i].w);
+                if (ck) __stcs(reinterpret_cast<float4 *>(ck + (int64_t)(r0 + i) * kHeadDim + 4 * lane), s[i]);
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < kRowsPerWarp; ++i)
+            __stcs(reinterpret_cast<float4 *>(S + (int64_t)(r0 + i) * kHeadDim + 4 * lane), s[i]);
+        __syncthreads();   // vs and the reductions are reused by the next V head
+    }
+}
+
+cudaError_t launch_decode_multi(const DecodeParams &p, bool in_bf16, bool out_bf16, cudaStream_t s) {
+    if (p.batch <= 0) return cudaSuccess;
+    if (p.n_tok < 1 || p.n_tok > kMaxDecTok) return cudaErrorInvalidValue;
+    const unsigned grid = (unsigned)((int64_t)p.batch * p.n_qk);
+    TraceLaunch tl(s, "decode_multi");
+    if (in_bf16) {
+        if (out_bf16) decode_multi_kernel<gdn::bf16, gdn::bf16><<<grid, kDecThreads, 0, s>>>(p);
+        else decode_multi_kernel<gdn::bf16, float><<<grid, kDecThreads, 0, s>>>(p);
+    } else {
+        if (out_bf16) decode_multi_kernel<float, gdn::bf16><<<grid, kDecThreads, 0, s>>>(p);
+        else decode_multi_kernel<float, float><<<grid, kDecThreads, 0, s>>>(p);
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace gdn

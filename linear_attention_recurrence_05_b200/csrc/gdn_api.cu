@@ -340,4 +340,48 @@ gdn_status gdn_decode_step(const gdn_config *cfg, gdn_dtype dtype, gdn_dtype out
     return GDN_OK;
 }
 
+gdn_status gdn_decode_multi(const gdn_config *cfg, gdn_dtype dtype, gdn_dtype out_dtype,
+                            const void *q, const void *k, const void *v, const float *conv_w_q,
+                            const float *conv_w_k, const float *conv_w_v, const void *alpha,
+                            const void *beta, float *state, void *conv_state,
+                            const int32_t *state_slots, int n_state_rows, float *state_ckpt,
+                            void *conv_ckpt, void *out, int batch, int n_tok, cudaStream_t stream) {
+    gdn_status st = check_config(cfg, dtype);
+    if (st != GDN_OK) return st;
+    if (out_dtype != GDN_BF16 && out_dtype != GDN_F32) return GDN_ERR_INVALID_ARG;
+    if (batch < 0 || n_state_rows < 0 || n_tok < 1) return GDN_ERR_INVALID_ARG;
+    if (n_tok > gdn::kMaxDecTok) return GDN_ERR_UNSUPPORTED;
+    if (batch == 0) return GDN_OK;
+    if (!state_slots && n_state_rows < batch) return GDN_ERR_INVALID_ARG;
+    if ((int64_t)batch * cfg->n_qk_heads >= ((int64_t)1 << 31)) return GDN_ERR_UNSUPPORTED;
+    const size_t eb = dtype == GDN_BF16 ? 2 : 4;
+    if (!q || !k || !v || !alpha || !beta || !state || !out) return GDN_ERR_INVALID_ARG;
+    if (!conv_w_q || !conv_w_k || !conv_w_v) return GDN_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) ||
+        !aligned(state, 16) || !aligned(conv_w_q, 16) || !aligned(conv_w_k, 16) ||
+        !aligned(conv_w_v, 16))
+        return GDN_ERR_INVALID_ARG;
+    if (!aligned(alpha, eb) || !aligned(beta, eb)) return GDN_ERR_INVALID_ARG;
+    if (conv_state && !aligned(conv_state, 16)) return GDN_ERR_INVALID_ARG;
+    if (state_ckpt && !aligned(state_ckpt, 16)) return GDN_ERR_INVALID_ARG;
+    if (conv_ckpt && !aligned(conv_ckpt, 16)) return GDN_ERR_INVALID_ARG;
+    if (state_slots && !aligned(state_slots, 4)) return GDN_ERR_INVALID_ARG;
+    st = check_device();
+    if (st != GDN_OK) return st;
+
+    DecodeParams p{};
+    p.q = q; p.k = k; p.v = v;
+    p.wq = conv_w_q; p.wk = conv_w_k; p.wv = conv_w_v;
+    p.alpha = alpha; p.beta = beta;
+    p.state = state; p.conv = conv_state; p.slots = state_slots;
+    p.n_rows = n_state_rows; p.batch = batch;
+    p.n_qk = cfg->n_qk_heads; p.n_v = cfg->n_v_heads;
+    p.q_scale = cfg->q_scale; p.eps = cfg->l2_eps;
+    p.out = out;
+    p.n_tok = n_tok; p.state_ckpt = state_ckpt; p.conv_ckpt = conv_ckpt;
+    cudaError_t e = launch_decode_multi(p, dtype == GDN_BF16, out_dtype == GDN_BF16, stream);
+    if (e != cudaSuccess) return cuda_fail(e);
+    return GDN_OK;
+}
+
 }  // extern "C"

@@ -93,7 +93,11 @@ struct DecodeParams {
     int n_rows, batch, n_qk, n_v;
     float q_scale, eps;
     void *out;
+    int n_tok;                             // multi-token decode: tokens per row (1..kMaxDecTok)
+    float *state_ckpt;                     //   or null: state after each token [B, n_tok, Hv, 128, 128]
+    void *conv_ckpt;                       //   or null: conv state after each token [B, n_tok, 3, ch]
 };
+constexpr int kMaxDecTok = 8;
 
 // remembers `e` as this host thread's gdn_last_cuda_error()
 void record_cuda_error(cudaError_t e);
@@ -116,5 +120,6 @@ cudaError_t launch_chunk_prep(const ScanParams &p, int64_t total_tokens, bool in
 cudaError_t launch_prefill_tc(const ScanParams &p, int64_t total_tokens, bool in_bf16, bool out_bf16,
                               cudaStream_t s);
 cudaError_t launch_decode(const DecodeParams &p, bool in_bf16, bool out_bf16, cudaStream_t s);
+cudaError_t launch_decode_multi(const DecodeParams &p, bool in_bf16, bool out_bf16, cudaStream_t s);
 
 }  // namespace gdn

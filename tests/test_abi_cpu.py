@@ -138,6 +138,32 @@ def test_decode_empty_batch_is_noop():
     assert _decode(batch=0, q=None) == 0
 
 
+def _decode_multi(**over):
+    A = 1 << 20
+    args = dict(cfg=_cfg(), dtype=0, odt=1, q=A, k=2 * A, v=3 * A, wq=4 * A, wk=5 * A, wv=6 * A,
+                alpha=7 * A, beta=8 * A, state=9 * A, conv=10 * A, slots=None, rows=4, ck=None, cck=None,
+                out=11 * A, batch=4, n=4, stream=None)
+    args.update(over)
+    c = args["cfg"]
+    return _native.lib().gdn_decode_multi(
+        ctypes.byref(c), args["dtype"], args["odt"], args["q"], args["k"], args["v"], args["wq"],
+        args["wk"], args["wv"], args["alpha"], args["beta"], args["state"], args["conv"], args["slots"],
+        args["rows"], args["ck"], args["cck"], args["out"], args["batch"], args["n"], args["stream"])
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(n=0), 1), (dict(n=-3), 1), (dict(n=9), 2), (dict(state=None), 1), (dict(out=None), 1),
+    (dict(ck=(12 << 20) + 8), 1), (dict(cck=(13 << 20) + 2), 1), (dict(rows=2), 1),
+    (dict(cfg=_cfg(d_k=64)), 2),
+])
+def test_decode_multi_rejects_before_launch(over, code):
+    assert _decode_multi(**over) == code
+
+
+def test_decode_multi_empty_batch_is_noop():
+    assert _decode_multi(batch=0, q=None) == 0
+
+
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(_native, "LIB_PATH", str(tmp_path / "missing.so"))
     monkeypatch.setattr(_native, "_lib", None)

@@ -143,3 +143,66 @@ def test_workload3_full_batch_sampled(lib):
     assert rel_err(yg[:, :, heads], yo[:, :, heads]) <= tol(dtype)
     St = state[rows_t].double().cpu().numpy()
     assert rel_err(St[:, heads], So[:, heads]) <= tol(dtype)
+
+
+def _multi_inputs(dec, dtype):
+    """DecodeInputs are [steps, B, ...]; the multi-token call takes [B, n, ...]."""
+    return [to_dev(np.ascontiguousarray(np.swapaxes(getattr(dec, f), 0, 1)), dtype)
+            for f in ("q", "k", "v", "alpha", "beta")]
+
+
+@pytest.mark.parametrize("dtype,n", [(gi.BF16, 1), (gi.BF16, 3), (gi.BF16, 4), (gi.BF16, 8), (gi.F32, 4)])
+def test_multi_token_with_checkpoints(lib, dtype, n):
+    """gdn_decode_multi over n tokens per row equals n single-token oracle steps: y of every
+    token, the state and conv state after the last one, and the checkpoints after each."""
+    shape = gi.GdnShape(n_qk_heads=4, n_v_heads=12)
+    B = 5
+    w = gi.make_conv_weights(shape, 101)
+    dec = gi.make_decode_inputs(shape, B, n, dtype, seed=102 + n)
+    rng = np.random.default_rng(103)
+    S0 = (0.05 * rng.standard_normal((B, 12, 128, 128))).astype(np.float32)
+    cs0 = gi.quantize(rng.standard_normal((B, 3, shape.channels)).astype(np.float32), dtype)
+    state = torch.from_numpy(S0.copy()).cuda()
+    conv = to_dev(cs0, dtype)
+    ck = torch.full((B, n, 12, 128, 128), float("nan"), dtype=torch.float32, device="cuda")
+    cck = torch.zeros((B, n, 3, shape.channels), dtype=conv.dtype, device="cuda")
+    q, k, v, a, b = _multi_inputs(dec, dtype)
+    y = lib.gdn_decode_multi(q, k, v, *_weights_dev(w, dtype), a, b, state, conv, state_ckpt=ck, conv_ckpt=cck,
+                             cfg=lib.GdnConfig(4, 12))
+    torch.cuda.synchronize()
+    yo, So, co = oracle.decode_steps(shape, dtype, dec, w, S0, cs0)
+    assert rel_err(np.swapaxes(to_host_f64(y), 0, 1), yo) <= tol(dtype)
+    assert rel_err(to_host_f64(state), So) <= tol(dtype)
+    assert np.array_equal(to_host_f64(conv), co)
+    for j in range(n):   # checkpoint j = the oracle after j + 1 tokens
+        _, Sj, cj = oracle.decode_steps(shape, dtype, dec, w, S0, cs0, steps=j + 1)
+        assert rel_err(to_host_f64(ck[:, j]), Sj) <= tol(dtype)
+        assert np.array_equal(to_host_f64(cck[:, j]), cj)
+
+
+def test_multi_token_slots_and_skipped_rows(lib):
+    """state_slots map rows to state rows; a slot of -1 writes zero outputs and touches no
+    state row; no conv state (zero history) and no checkpoints."""
+    dtype = gi.BF16
+    shape = gi.GdnShape(n_qk_heads=2, n_v_heads=6)
+    B, R, n = 4, 6, 3
+    slots = np.array([4, -1, 1, 2], np.int32)
+    w = gi.make_conv_weights(shape, 104)
+    dec = gi.make_decode_inputs(shape, B, n, dtype, seed=105)
+    rng = np.random.default_rng(106)
+    S0 = (0.05 * rng.standard_normal((R, 6, 128, 128))).astype(np.float32)
+    state = torch.from_numpy(S0.copy()).cuda()
+    q, k, v, a, b = _multi_inputs(dec, dtype)
+    y = to_host_f64(lib.gdn_decode_multi(q, k, v, *_weights_dev(w, dtype), a, b, state, None,
+                                         state_slots=torch.from_numpy(slots).cuda(), cfg=lib.GdnConfig(2, 6)))
+    torch.cuda.synchronize()
+    live = [0, 2, 3]
+    sub = gi.DecodeInputs(*(getattr(dec, f)[:, live] for f in ("q", "k", "v", "alpha", "beta")))
+    cs_zero = np.zeros((len(live), 3, shape.channels), np.float32)
+    yo, So, _ = oracle.decode_steps(shape, dtype, sub, w, S0[slots[live]], cs_zero)
+    assert rel_err(np.swapaxes(y[live], 0, 1), yo) <= tol(dtype)
+    assert np.all(y[1] == 0)
+    Sg = to_host_f64(state)
+    assert rel_err(Sg[slots[live]], So) <= tol(dtype)
+    untouched = [r for r in range(R) if r not in slots[live]]
+    assert np.array_equal(Sg[untouched], S0[untouched].astype(np.float64))
