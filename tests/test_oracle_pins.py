@@ -424,3 +424,62 @@ def test_planted_mistakes_are_caught(mutant):
     y, fin, _ = oracle.prefill(p, mutant=mutant)
     yb, fb = _full_pipeline_brute(p)
     assert rel(y, yb) > 1e-3 or rel(fin, fb) > 1e-3, MUTANTS[mutant]
+
+
+# ----------------------------------------------------------------- output tail (gated RMSNorm)
+def test_output_gate_closed_forms():
+    """One-hot y: the RMS over 128 channels is 1/sqrt(128), so o_0 = sqrt(128 / (1 + 128 eps))
+    w_0 SiLU(z_0) and every other channel is 0; SiLU at 0, ln 3 and -ln 3 is 0, (3/4) ln 3 and
+    -(1/4) ln 3 (sigmoid(ln 3) = 3/4)."""
+    from oracle.output_gate import output_gate
+    eps = 1e-6
+    y = np.zeros((3, 2, 128))
+    y[..., 0] = 1.0
+    ln3 = np.log(3.0)
+    z = np.zeros((3, 2, 128))
+    z[0, :, 0], z[1, :, 0], z[2, :, 0] = 0.0, ln3, -ln3
+    w = np.linspace(0.5, 1.5, 128)
+    o = output_gate(y, z, w, eps)
+    amp = np.sqrt(128.0 / (1.0 + 128.0 * eps)) * w[0]
+    np.testing.assert_allclose(o[0, :, 0], 0.0, atol=0)
+    np.testing.assert_allclose(o[1, :, 0], amp * 0.75 * ln3, rtol=1e-14)
+    np.testing.assert_allclose(o[2, :, 0], -amp * 0.25 * ln3, rtol=1e-14)
+    assert np.all(o[..., 1:] == 0)
+
+
+def test_output_gate_invariances():
+    """With eps = 0 the normalisation removes any positive scale of y and is odd in y; the
+    norm is per (token, head): scaling one head leaves the others unchanged."""
+    from oracle.output_gate import output_gate
+    rng = np.random.default_rng(7)
+    y = rng.standard_normal((5, 3, 128))
+    z = rng.standard_normal((5, 3, 128))
+    w = rng.standard_normal(128)
+    o = output_gate(y, z, w, 0.0)
+    np.testing.assert_allclose(output_gate(7.5 * y, z, w, 0.0), o, rtol=1e-13)
+    np.testing.assert_allclose(output_gate(-y, z, w, 0.0), -o, rtol=1e-13)
+    y2 = y.copy()
+    y2[:, 1] *= 100.0
+    o2 = output_gate(y2, z, w, 0.0)
+    np.testing.assert_allclose(o2[:, [0, 2]], o[:, [0, 2]], rtol=1e-13)
+
+
+def test_output_gate_brute_force():
+    """Element by element in plain Python (math module) on a tiny case."""
+    import math
+    from oracle.output_gate import output_gate
+    rng = np.random.default_rng(8)
+    y = rng.standard_normal((2, 2, 128))
+    z = 3.0 * rng.standard_normal((2, 2, 128))
+    w = rng.standard_normal(128)
+    eps = 1e-3
+    o = output_gate(y, z, w, eps)
+    for t in range(2):
+        for h in range(2):
+            s = 0.0
+            for i in range(128):
+                s += y[t, h, i] ** 2
+            inv = 1.0 / math.sqrt(s / 128.0 + eps)
+            for i in range(128):
+                g = z[t, h, i] / (1.0 + math.exp(-z[t, h, i]))
+                assert abs(o[t, h, i] - y[t, h, i] * inv * w[i] * g) <= 1e-12 * (1 + abs(o[t, h, i]))
