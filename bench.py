@@ -267,6 +267,40 @@ def bench_prefill(args, dist, torch, gdn, peaks):
     }
 
 
+def bench_output_gate(args, dist, torch, gdn, peaks, peak_src):
+    """The output tail on a prefill output of the workload's shape: y fp32 [T, Hv, 128] (as
+    gdn_prefill returns it), gate z bf16, out bf16; L2 flushed between steps."""
+    w = gi.WORKLOADS[1]
+    T, Hv = w["lengths"][0], w["shape"].n_v_heads
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(gi.workload_seed(1) + 31 + 7919 * dist.rank)
+    y = torch.randn((T, Hv, D), generator=gen, device="cuda")
+    z = torch.randn((T, Hv, D), generator=gen, device="cuda").to(torch.bfloat16)
+    nw = torch.ones(D, device="cuda")
+    out = torch.empty((T, Hv, D), dtype=torch.bfloat16, device="cuda")
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    cfg = gdn.GdnConfig(w["shape"].n_qk_heads, Hv)
+    for _ in range(args.warmup):
+        gdn.gdn_output_gate(y, z, nw, cfg=cfg, out=out)
+    K = args.steps
+    trace = gdn.LaunchTrace(capacity=K + 4)
+    dist.barrier()
+    with trace:
+        for _ in range(K):
+            flush.zero_()
+            gdn.gdn_output_gate(y, z, nw, cfg=cfg, out=out)
+    dist.barrier()
+    recs = [t for n, t in trace.records() if n == "output_gate"]
+    avg_ms = dist.max(sum(recs) / len(recs))
+    byts = T * Hv * D * (4 + 2 + 2)
+    achieved = byts / (avg_ms / 1e3) / 1e9
+    return {"value": T * dist.world / (avg_ms / 1e3), "unit": UNIT, "workload": f"output-gate-T{T}-h{Hv}",
+            "ms_per_step": avg_ms,
+            "roofline": {"kernel": "output_gate", "bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
+                         "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                         "peak_source": peak_src, "algorithmic_bytes_per_launch": byts}}
+
+
 def prefill_roofline(res, peaks, peak_src):
     pk = res["per_kernel"]
     dom = max(pk, key=lambda n: pk[n]["total_ms"])
@@ -539,6 +573,7 @@ def main():
     pre = bench_prefill(args, dist, torch, gdn, peaks)
     roof = prefill_roofline(pre, peaks, peak_src)
     dec = None if args.no_decode else bench_decode(args, dist, torch, gdn, peaks, peak_src)
+    tail = bench_output_gate(args, dist, torch, gdn, peaks, peak_src)
     cpu = None
     if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
         v, threads, sample, dt = oracle_tokens_per_s(args.cpu_baseline_s)
@@ -555,7 +590,7 @@ def main():
                        "out": "f32", "state": "f32", "l2": "flushed: 256 MiB write between steps",
                        "parallelism": f"dp{dist.world} (independent sequences per GPU)"},
             "clocks": pre["clocks"], "e2e": pre["e2e"], "gpu_launches": pre["launches"],
-            "roofline": roof, "kernels": pre["per_kernel"], "cpu_baseline": cpu, "decode": dec,
+            "roofline": roof, "kernels": pre["per_kernel"], "cpu_baseline": cpu, "decode": dec, "output_gate": tail,
             "peaks": peak_src,
         }
         print(json.dumps(line), flush=True)

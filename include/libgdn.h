@@ -199,6 +199,24 @@ GDN_EXPORT gdn_status gdn_decode_multi(const gdn_config *cfg, gdn_dtype dtype, g
                             void *out, int batch, int n_tok, cudaStream_t stream);
 
 /*
+ * gdn_output_gate -- the mixer's output tail: gated RMS normalisation of y, per (token,
+ * V head) over its 128 values (page "ARCHITECTURE PREVIEW / FIELD NOTES", section 03: the
+ * readout passes a normalisation and an output gate before the output projection; the page
+ * gives no formula, this is its plainest reading):
+ *     out = y / sqrt(mean(y^2) + eps) * norm_w * SiLU(z),   SiLU(z) = z / (1 + exp(-z))
+ *
+ *   y        [n_tokens, Hv, 128] y_dtype (gdn_prefill's or gdn_decode_*'s out)
+ *   z        [n_tokens, Hv, 128] z_dtype: the output-gate input
+ *   norm_w   [128] fp32, shared by the V heads
+ *   eps      >= 0, finite
+ *   out      [n_tokens, Hv, 128] out_dtype; may be y itself when out_dtype == y_dtype
+ * All pointers 16-byte aligned.  Only cfg->n_v_heads and cfg->d_v (128) are used.
+ */
+GDN_EXPORT gdn_status gdn_output_gate(const gdn_config *cfg, gdn_dtype y_dtype, gdn_dtype z_dtype,
+                           gdn_dtype out_dtype, const void *y, const void *z, const float *norm_w,
+                           float eps, void *out, int64_t n_tokens, cudaStream_t stream);
+
+/*
  * gdn_prefill_static_scratch -- gdn_prefill without a caller-supplied workspace.
  *
  * No counterpart on the pages: it exists for callers that cannot call cudaMalloc

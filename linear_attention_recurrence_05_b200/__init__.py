@@ -19,7 +19,7 @@ import torch
 from . import _native
 from ._native import GDN_BF16, GDN_F32, GdnError  # noqa: F401
 
-__all__ = ["GdnConfig", "gdn_prefill", "gdn_decode_step", "gdn_decode_multi", "prefill_workspace_size", "GdnError",
+__all__ = ["GdnConfig", "gdn_prefill", "gdn_decode_step", "gdn_decode_multi", "gdn_output_gate", "prefill_workspace_size", "GdnError",
            "library_path"]
 
 
@@ -182,6 +182,30 @@ def gdn_decode_multi(q, k, v, conv_w_q, conv_w_k, conv_w_v, alpha, beta, state, 
         _ptr(conv_w_v), _ptr(alpha), _ptr(beta), _ptr(state), _ptr(conv_state), _ptr(state_slots),
         state.shape[0], _ptr(state_ckpt), _ptr(conv_ckpt), _ptr(out), B, n, _stream(stream))
     _native.check("gdn_decode_multi", st)
+    return out
+
+
+def gdn_output_gate(y, z, norm_w, *, eps: float = 1e-6, cfg: GdnConfig | None = None, out=None,
+                    out_dtype=None, stream=None):
+    """Gated RMS normalisation of y per (token, V head): y / sqrt(mean(y^2) + eps) * norm_w * SiLU(z).
+
+    y, z [..., Hv, 128] (bf16 or fp32, any mix); norm_w fp32 [128]; ``out`` may be ``y``.
+    Returns out (``out_dtype``, default y's dtype).
+    """
+    if y.shape != z.shape:
+        raise ValueError("y and z must have the same shape")
+    if norm_w.dtype != torch.float32 or norm_w.numel() != y.shape[-1]:
+        raise TypeError("norm_w must be float32 with one weight per channel")
+    Hv = y.shape[-2]
+    cfg = cfg or GdnConfig(n_qk_heads=1, n_v_heads=Hv)
+    if out is None:
+        out = torch.empty(y.shape, dtype=out_dtype or y.dtype, device=y.device)
+    n_tokens = y.numel() // (Hv * y.shape[-1])
+    c = cfg.c()
+    st = _native.lib().gdn_output_gate(ctypes.byref(c), _dtype_code(y), _dtype_code(z), _dtype_code(out),
+                                       _ptr(y), _ptr(z), _ptr(norm_w), float(eps), _ptr(out), n_tokens,
+                                       _stream(stream))
+    _native.check("gdn_output_gate", st)
     return out
 
 

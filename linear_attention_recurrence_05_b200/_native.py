@@ -20,7 +20,7 @@ STATUS = {0: "GDN_OK", 1: "GDN_ERR_INVALID_ARG", 2: "GDN_ERR_UNSUPPORTED", 3: "G
 # every entry point the header declares (checked by the CPU test suite)
 EXPORTS = ("gdn_status_string", "gdn_last_cuda_error", "gdn_api_version",
            "gdn_prefill_workspace_size", "gdn_prefill", "gdn_decode_step", "gdn_decode_multi",
-           "gdn_trace_begin",
+           "gdn_output_gate", "gdn_trace_begin",
            "gdn_trace_end", "gdn_prefill_static_scratch")
 
 STATIC_SCRATCH_BYTES = 64 << 20  # GDN_STATIC_SCRATCH_BYTES
@@ -85,6 +85,9 @@ def lib():
                                            vp, vp, fp, fp, fp, vp, vp, fp, vp, i32p, ctypes.c_int,
                                            fp, vp, vp, ctypes.c_int, ctypes.c_int, vp]
             L.gdn_decode_multi.restype = ctypes.c_int
+            L.gdn_output_gate.argtypes = [ctypes.POINTER(GdnConfigC), ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                          vp, vp, fp, ctypes.c_float, vp, ctypes.c_int64, vp]
+            L.gdn_output_gate.restype = ctypes.c_int
             L.gdn_trace_begin.argtypes = [ctypes.POINTER(TraceEntryC), ctypes.c_int]
             L.gdn_trace_begin.restype = None
             L.gdn_trace_end.argtypes = []

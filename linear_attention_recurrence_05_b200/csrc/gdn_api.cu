@@ -384,4 +384,25 @@ gdn_status gdn_decode_multi(const gdn_config *cfg, gdn_dtype dtype, gdn_dtype ou
     return GDN_OK;
 }
 
+gdn_status gdn_output_gate(const gdn_config *cfg, gdn_dtype y_dtype, gdn_dtype z_dtype,
+                           gdn_dtype out_dtype, const void *y, const void *z, const float *norm_w,
+                           float eps, void *out, int64_t n_tokens, cudaStream_t stream) {
+    if (!cfg) return GDN_ERR_INVALID_ARG;
+    if (cfg->n_v_heads <= 0) return GDN_ERR_INVALID_ARG;
+    if (cfg->d_v != 128) return GDN_ERR_UNSUPPORTED;
+    for (gdn_dtype d : {y_dtype, z_dtype, out_dtype})
+        if (d != GDN_BF16 && d != GDN_F32) return GDN_ERR_INVALID_ARG;
+    if (n_tokens < 0 || !(eps >= 0.f) || !std::isfinite(eps)) return GDN_ERR_INVALID_ARG;
+    if (n_tokens == 0) return GDN_OK;
+    if (!y || !z || !norm_w || !out) return GDN_ERR_INVALID_ARG;
+    if (!aligned(y, 16) || !aligned(z, 16) || !aligned(norm_w, 16) || !aligned(out, 16)) return GDN_ERR_INVALID_ARG;
+    if (n_tokens > ((int64_t)1 << 40) / cfg->n_v_heads) return GDN_ERR_UNSUPPORTED;
+    gdn_status st = check_device();
+    if (st != GDN_OK) return st;
+    cudaError_t e = launch_output_gate(y, y_dtype == GDN_BF16, z, z_dtype == GDN_BF16, norm_w, eps, out,
+                                       out_dtype == GDN_BF16, n_tokens * cfg->n_v_heads, stream);
+    if (e != cudaSuccess) return cuda_fail(e);
+    return GDN_OK;
+}
+
 }  // extern "C"

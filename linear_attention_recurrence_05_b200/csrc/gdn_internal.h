@@ -121,5 +121,7 @@ cudaError_t launch_prefill_tc(const ScanParams &p, int64_t total_tokens, bool in
                               cudaStream_t s);
 cudaError_t launch_decode(const DecodeParams &p, bool in_bf16, bool out_bf16, cudaStream_t s);
 cudaError_t launch_decode_multi(const DecodeParams &p, bool in_bf16, bool out_bf16, cudaStream_t s);
+cudaError_t launch_output_gate(const void *y, bool y_bf16, const void *z, bool z_bf16, const float *w,
+                               float eps, void *out, bool out_bf16, int64_t rows, cudaStream_t s);
 
 }  // namespace gdn

@@ -164,6 +164,28 @@ def test_decode_multi_empty_batch_is_noop():
     assert _decode_multi(batch=0, q=None) == 0
 
 
+def _gate(**over):
+    A = 1 << 20
+    args = dict(cfg=_cfg(), ydt=1, zdt=0, odt=1, y=A, z=2 * A, w=3 * A, eps=1e-6, out=4 * A, n=10, stream=None)
+    args.update(over)
+    c = args["cfg"]
+    return _native.lib().gdn_output_gate(ctypes.byref(c), args["ydt"], args["zdt"], args["odt"], args["y"],
+                                         args["z"], args["w"], args["eps"], args["out"], args["n"], args["stream"])
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(y=None), 1), (dict(z=None), 1), (dict(w=None), 1), (dict(out=None), 1), (dict(n=-1), 1),
+    (dict(eps=-1.0), 1), (dict(eps=float("inf")), 1), (dict(eps=float("nan")), 1), (dict(zdt=7), 1),
+    (dict(z=(2 << 20) + 8), 1), (dict(cfg=_cfg(d_v=64)), 2),
+])
+def test_output_gate_rejects_before_launch(over, code):
+    assert _gate(**over) == code
+
+
+def test_output_gate_no_tokens_is_noop():
+    assert _gate(n=0, y=None, out=None) == 0
+
+
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(_native, "LIB_PATH", str(tmp_path / "missing.so"))
     monkeypatch.setattr(_native, "_lib", None)
