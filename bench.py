@@ -139,8 +139,12 @@ def to_dev(a, torch):
 
 
 class Dist:
-    def __init__(self, torch):
+    """Ranks of a torchrun launch (RANK / LOCAL_RANK / WORLD_SIZE from the environment): NCCL
+    on the local GPU for the timed runs; the same logic over gloo on the CPU in the tests."""
+
+    def __init__(self, torch, backend: str = "nccl", device: str = "cuda"):
         self.torch = torch
+        self.backend, self.device = backend, device
         self.world = int(os.environ.get("WORLD_SIZE", "1"))
         self.rank = int(os.environ.get("RANK", "0"))
         self.local = int(os.environ.get("LOCAL_RANK", "0"))
@@ -149,23 +153,26 @@ class Dist:
     def init(self):
         import datetime
         torch = self.torch
-        torch.cuda.set_device(self.local)
+        if self.device == "cuda":
+            torch.cuda.set_device(self.local)
         if self.world > 1:
             import torch.distributed as dist
-            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                    device_id=torch.device("cuda", self.local))
+            kw = {"device_id": torch.device("cuda", self.local)} if self.device == "cuda" else {}
+            dist.init_process_group(self.backend, timeout=datetime.timedelta(seconds=120), **kw)
             self.pg = dist
         return self
 
     def barrier(self):
         if self.pg:
             self.pg.barrier()
-        self.torch.cuda.synchronize()
+        if self.device == "cuda":
+            self.torch.cuda.synchronize()
 
     def max(self, x: float) -> float:
+        """The largest x over the ranks (a step's time is the slowest rank's)."""
         if not self.pg:
             return x
-        t = self.torch.tensor([x], dtype=self.torch.float64, device="cuda")
+        t = self.torch.tensor([x], dtype=self.torch.float64, device=self.device)
         self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
         return float(t.item())
 

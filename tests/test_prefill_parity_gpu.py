@@ -203,3 +203,26 @@ def test_bf16_output(lib):
     yo, fo, _ = oracle.prefill(inp)
     assert rel_err_bf16_out(to_host_f64(y), yo) <= tol(gi.BF16)
     assert rel_err(to_host_f64(fin), fo) <= tol(gi.BF16)
+
+
+def test_context_parallel_spans(lib):
+    """One sequence in 3 spans through libgdn (span maps M, B from two prefills each, prefix
+    combination, re-run from the true entering state): y and the final state match the oracle
+    over the whole sequence (initial state and conv state given)."""
+    from gdn_testutil import to_dev
+    from linear_attention_recurrence_05_b200.context_parallel import cp_prefill_spans
+    shape = gi.GdnShape(n_qk_heads=2, n_v_heads=6)
+    inp = gi.make_prefill_inputs(shape, [700], gi.BF16, seed=97, with_initial_state=True,
+                                 with_conv_state=True)
+    d = inp.dtype
+    full = [to_dev(x, d) for x in (inp.q, inp.k, inp.v, inp.alpha, inp.beta)]
+    w = [to_dev(x, d) for x in (inp.w_q, inp.w_k, inp.w_v)]
+    bounds = [0, 250, 253, 700]
+    spans = [[x[a:b] for x in full] for a, b in zip(bounds[:-1], bounds[1:])]
+    ys, fin = cp_prefill_spans(spans, w, cfg=lib.GdnConfig(2, 6),
+                               initial_state=torch.from_numpy(inp.initial_state[0]).cuda(),
+                               conv_state=to_dev(inp.conv_state[0], d))
+    torch.cuda.synchronize()
+    yo, fo, _ = oracle.prefill(inp)
+    assert rel_err(to_host_f64(torch.cat(ys)), yo) <= tol(d)
+    assert rel_err(to_host_f64(fin), fo[0]) <= tol(d)
