@@ -167,8 +167,9 @@ __global__ void __launch_bounds__(128) conv_l2_kernel(ConvParams p) {
 
 // ------------------------------------------------------------------------ conv + L2, tiles
 // The tensor-core path's tiles from bf16 input.  CTA = one 64-row chunk of one head slot:
-// q heads ([K;Q] tile, Q half), k heads ([K;Q] tile, K half), k heads again (the K tile,
-// MN-major), v heads (the V tile, MN-major).  One TMA copy brings the chunk's rows and the
+// q heads ([K;Q] tile, Q half), k heads ([K;Q] tile, K half, and the K tile, MN-major, whose
+// rows are stored straight from registers: a warp's 32 lanes cover one row, four whole
+// 128-byte lines), v heads (the V tile, MN-major).  One TMA copy brings the chunk's rows and the
 // 3 rows before them (rows outside the tensor read as zero; at a sequence's start the 3
 // history rows are replaced by the conv state or zeros); each warp then walks 16 rows from
 // shared memory, writes the TF32-rounded rows into an image of the tile in shared memory,
@@ -235,10 +236,10 @@ __global__ void __launch_bounds__(128) conv_tiles_kernel(const __grid_constant__
     const int len = min(kChunk, seq1 - seq0 - r0);
     if (blockIdx.y == 0 && threadIdx.x == 0) p.cseq[ci] = b;   // for the chunk-prep pass
 
-    // slot kinds: 0 q ([K;Q] Q half), 1 k ([K;Q] K half), 2 k (K tile), 3 v (V tile)
+    // slot kinds: 0 q ([K;Q] Q half), 1 k ([K;Q] K half + K tile), 3 v (V tile)
     const int slot = blockIdx.y, nq = p.n_qk;
-    const int kind = slot < nq ? 0 : slot < 2 * nq ? 1 : slot < 3 * nq ? 2 : 3;
-    const int head = kind == 3 ? slot - 3 * nq : slot - kind * nq;
+    const int kind = slot < nq ? 0 : slot < 2 * nq ? 1 : 3;
+    const int head = kind == 3 ? slot - 2 * nq : slot - kind * nq;
     const CUtensorMap *tm = kind == 0 ? &p.tm_q : kind == 3 ? &p.tm_v : &p.tm_k;
     const float *w = kind == 0 ? p.wq : kind == 3 ? p.wv : p.wk;
     const int qkc = nq * kHeadDim;
@@ -278,7 +279,7 @@ __global__ void __launch_bounds__(128) conv_tiles_kernel(const __grid_constant__
     float h[3][4];
 #pragma unroll
     for (int j = 0; j < 3; ++j) bf16x4_to_f32(*reinterpret_cast<const uint2 *>(slab + (16 * wid + j) * 256), h[j]);
-    const bool mn = kind >= 2;
+    const bool mn = kind == 3;
     const float nan = __int_as_float(0x7fc00000);
 #pragma unroll 4
     for (int i = 0; i < 16; ++i) {
@@ -304,10 +305,12 @@ __global__ void __launch_bounds__(128) conv_tiles_kernel(const __grid_constant__
         o.z = t < len ? __uint_as_float((__float_as_uint(y[2]) + 0x1000u) & 0xFFFFE000u) : 0.f;
         o.w = t < len ? __uint_as_float((__float_as_uint(y[3]) + 0x1000u) & 0xFFFFE000u) : 0.f;
         if (!ok) o = make_float4(nan, nan, nan, nan);
-        const uint32_t off = (lane >> 3) * 8192 + t * 128 +
-                             (mn ? ((((lane & 7) >> 1) ^ (t & 3)) << 5) + (lane & 1) * 16
-                                 : (((lane & 7) ^ (t & 7)) << 4));
+        const uint32_t mn_off = (lane >> 3) * 8192 + t * 128 + ((((lane & 7) >> 1) ^ (t & 3)) << 5) + (lane & 1) * 16;
+        const uint32_t off = mn ? mn_off : (lane >> 3) * 8192 + t * 128 + (((lane & 7) ^ (t & 7)) << 4);
         *reinterpret_cast<float4 *>(sm + C_STAGE + off) = o;
+        if (kind == 1)   // the K tile's row t: one warp instruction, four whole 128-byte lines
+            *reinterpret_cast<float4 *>(reinterpret_cast<unsigned char *>(
+                p.kmn + ((int64_t)ci * nq + head) * 8192) + mn_off) = o;
     }
     fence_smem_to_async();
     __syncthreads();
@@ -318,9 +321,7 @@ __global__ void __launch_bounds__(128) conv_tiles_kernel(const __grid_constant__
 #pragma unroll
             for (int blk = 0; blk < 4; ++blk) bulk_store_s2g(dst + blk * 4096, st + blk * 8192, 8192);
         } else {
-            float *dst = kind == 2 ? p.kmn + ((int64_t)ci * nq + head) * 8192
-                                   : p.vi + ((int64_t)ci * p.n_v + head) * 8192;
-            bulk_store_s2g(dst, st, 32768);
+            bulk_store_s2g(p.vi + ((int64_t)ci * p.n_v + head) * 8192, st, 32768);
         }
         bulk_commit();
         bulk_wait_read0();   // the image is read before the CTA's shared memory goes away
@@ -348,7 +349,7 @@ cudaError_t launch_conv_l2(const ConvParams &p, bool bf16, bool tiles, int64_t n
         cudaError_t e = cudaFuncSetAttribute(conv_tiles_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)kConvSmemAlloc);
         if (e != cudaSuccess) return e;
-        dim3 grid((unsigned)n_chunks, 3 * p.n_qk + p.n_v);
+        dim3 grid((unsigned)n_chunks, 2 * p.n_qk + p.n_v);
         TraceLaunch tl(s, "conv_l2");
         conv_tiles_kernel<<<grid, 128, kConvSmemAlloc, s>>>(tp);
         return cudaGetLastError();
