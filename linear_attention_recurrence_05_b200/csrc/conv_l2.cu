@@ -167,22 +167,19 @@ __global__ void __launch_bounds__(128) conv_l2_kernel(ConvParams p) {
 
 // ------------------------------------------------------------------------ conv + L2, tiles
 // The tensor-core path's tiles from bf16 input.  CTA = one 64-row chunk of one head slot:
-// q heads ([K;Q] tile, Q half), k heads ([K;Q] tile, K half, and the K tile, MN-major, whose
-// rows are stored straight from registers: a warp's 32 lanes cover one row, four whole
-// 128-byte lines), v heads (the V tile, MN-major).  One TMA copy brings the chunk's rows and the
-// 3 rows before them (rows outside the tensor read as zero; at a sequence's start the 3
-// history rows are replaced by the conv state or zeros); each warp then walks 16 rows from
-// shared memory, writes the TF32-rounded rows into an image of the tile in shared memory,
-// and the image leaves by bulk stores, so every global access of the kernel is a bulk
-// transfer.
+// q heads ([K;Q] tile, Q half), k heads ([K;Q] tile, K half, and the K tile, MN-major), v
+// heads (the V tile, MN-major).  One TMA copy brings the chunk's rows and the 3 rows before
+// them (rows outside the tensor read as zero; at a sequence's start the 3 history rows are
+// replaced by the conv state or zeros); each warp then walks 16 rows from shared memory and
+// stores each TF32-rounded row straight into the tile: in both layouts the 32 lanes of a
+// warp cover one row of the 4 feature blocks, four whole 128-byte lines.
 namespace {
 using namespace tc;
 
 constexpr int kSlabRows = kChunk + 3;
 constexpr uint32_t kSlabBytes = kSlabRows * kHeadDim * 2;   // bf16 rows, 17,152 B
 constexpr uint32_t C_SLAB = 0;
-constexpr uint32_t C_STAGE = 17408;                          // tile image, 32 KB
-constexpr uint32_t C_BAR = C_STAGE + 32768;
+constexpr uint32_t C_BAR = 17408;
 constexpr uint32_t kConvSmem = C_BAR + 16;
 constexpr uint32_t kConvSmemAlloc = kConvSmem + 1024;
 constexpr uint32_t kConvWaitTries = 1u << 24;
@@ -305,27 +302,21 @@ __global__ void __launch_bounds__(128) conv_tiles_kernel(const __grid_constant__
         o.z = t < len ? __uint_as_float((__float_as_uint(y[2]) + 0x1000u) & 0xFFFFE000u) : 0.f;
         o.w = t < len ? __uint_as_float((__float_as_uint(y[3]) + 0x1000u) & 0xFFFFE000u) : 0.f;
         if (!ok) o = make_float4(nan, nan, nan, nan);
+        // row t of this lane's 4 features (block lane / 8) in the tile's byte layout
         const uint32_t mn_off = (lane >> 3) * 8192 + t * 128 + ((((lane & 7) >> 1) ^ (t & 3)) << 5) + (lane & 1) * 16;
-        const uint32_t off = mn ? mn_off : (lane >> 3) * 8192 + t * 128 + (((lane & 7) ^ (t & 7)) << 4);
-        *reinterpret_cast<float4 *>(sm + C_STAGE + off) = o;
-        if (kind == 1)   // the K tile's row t: one warp instruction, four whole 128-byte lines
-            *reinterpret_cast<float4 *>(reinterpret_cast<unsigned char *>(
-                p.kmn + ((int64_t)ci * nq + head) * 8192) + mn_off) = o;
-    }
-    fence_smem_to_async();
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        const uint32_t st = smem_u32(sm + C_STAGE);
-        if (kind <= 1) {   // the 4 feature blocks of the Q or K half of the [K;Q] tile
-            float *dst = p.kq + ((int64_t)ci * nq + head) * 16384 + (kind == 0 ? 2048 : 0);
-#pragma unroll
-            for (int blk = 0; blk < 4; ++blk) bulk_store_s2g(dst + blk * 4096, st + blk * 8192, 8192);
+        if (mn) {
+            *reinterpret_cast<float4 *>(reinterpret_cast<unsigned char *>(p.vi + ((int64_t)ci * p.n_v + head) * 8192) +
+                                        mn_off) = o;
         } else {
-            bulk_store_s2g(p.vi + ((int64_t)ci * p.n_v + head) * 8192, st, 32768);
+            unsigned char *kq = reinterpret_cast<unsigned char *>(p.kq + ((int64_t)ci * nq + head) * 16384 +
+                                                                 (kind == 0 ? 2048 : 0));
+            *reinterpret_cast<float4 *>(kq + (lane >> 3) * 16384 + t * 128 + (((lane & 7) ^ (t & 7)) << 4)) = o;
+            if (kind == 1)   // the K tile, MN-major
+                *reinterpret_cast<float4 *>(reinterpret_cast<unsigned char *>(
+                    p.kmn + ((int64_t)ci * nq + head) * 8192) + mn_off) = o;
         }
-        bulk_commit();
-        bulk_wait_read0();   // the image is read before the CTA's shared memory goes away
     }
+    if (!ok && threadIdx.x == 0) mbar_wait(bar, 0, kConvWaitTries);   // the copy is done before exit
 }
 
 cudaError_t launch_conv_l2(const ConvParams &p, bool bf16, bool tiles, int64_t n_chunks,
