@@ -8,7 +8,8 @@ pages' shape (T = 8192, 16 QK / 48 V heads, d = 128, bf16 inputs, fp32 state, fp
 output) with inputs resident in HBM and L2 flushed between steps; the `decode` object
 is the batched decode workload (256 rows x 1024 consecutive steps on resident fp32
 states).  `e2e` repeats the prefill measurement through the public API from pinned
-host buffers, copies included.  `roofline` describes the dominant prefill kernel,
+host buffers, every step's copies included (uploads, kernels and downloads of
+consecutive steps overlap on three streams).  `roofline` describes the dominant prefill kernel,
 timed live with the library's launch trace.  `cpu_baseline` is the fp64 oracle on
 the host cores (rank 0, N = 1 only).
 
@@ -241,27 +242,65 @@ def bench_prefill(args, dist, torch, gdn, peaks):
     for name, t in recs:
         per_kernel.setdefault(name, []).append(t)
 
-    # e2e: public API from pinned host buffers, copies inside the timed region
+    # e2e: public API from pinned host buffers, every step's copies inside the timed region.
+    # Steps run as a pipeline on three streams (upload, compute, download) over two sets of
+    # device buffers: step i+1's inputs go up and step i-1's y comes down while step i
+    # computes, so the copies of both directions share the bus with the kernels.
     hq, hk, hv = (torch.empty(x.shape, dtype=x.dtype, pin_memory=True) for x in (q, k, v))
     ha, hb = (torch.empty(x.shape, dtype=x.dtype, pin_memory=True) for x in (al, be))
     for h, d in ((hq, q), (hk, k), (hv, v), (ha, al), (hb, be)):
         h.copy_(d)
-    hy = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
-    h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv, ha, hb))
-    d2h = hy.numel() * hy.element_size()
-    ev2 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in range(K)]
+    host_in = (hq, hk, hv, ha, hb)
+    dev_in = [(q, k, v, al, be)] + [tuple(torch.empty_like(x) for x in (q, k, v, al, be))]
+    dev_out = [out, torch.empty_like(out)]
+    hy = [torch.empty(out.shape, dtype=out.dtype, pin_memory=True) for _ in range(2)]
+    h2d = sum(x.numel() * x.element_size() for x in host_in)
+    d2h = hy[0].numel() * hy[0].element_size()
+    s_up, s_dn = torch.cuda.Stream(), torch.cuda.Stream()
+    comp = torch.cuda.current_stream()
+
+    def ev():
+        return torch.cuda.Event()
+
+    def e2e_steps(n):
+        up_done, comp_done, dn_done = [], [], []
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        start.record(comp)
+        s_up.wait_stream(comp)
+        s_dn.wait_stream(comp)
+        for i in range(n):
+            b = i % 2
+            with torch.cuda.stream(s_up):
+                if i >= 2:
+                    s_up.wait_event(comp_done[i - 2])      # set b no longer read
+                for h, d in zip(host_in, dev_in[b]):
+                    d.copy_(h, non_blocking=True)
+                up_done.append(ev())
+                up_done[i].record(s_up)
+            comp.wait_event(up_done[i])
+            if i >= 2:
+                comp.wait_event(dn_done[i - 2])            # y of set b already read back
+            flush.zero_()
+            xq, xk, xv, xa, xb = dev_in[b]
+            gdn.gdn_prefill(xq, xk, xv, wq, wk, wv, xa, xb, cu, cfg=cfg, out=dev_out[b],
+                            final_state=fin, workspace=ws)
+            comp_done.append(ev())
+            comp_done[i].record(comp)
+            with torch.cuda.stream(s_dn):
+                s_dn.wait_event(comp_done[i])
+                hy[b].copy_(dev_out[b], non_blocking=True)
+                dn_done.append(ev())
+                dn_done[i].record(s_dn)
+        comp.wait_stream(s_up)
+        comp.wait_stream(s_dn)
+        end.record(comp)
+        return start, end
+
+    e2e_steps(max(args.warmup, 3))
     dist.barrier()
-    for i in range(K):
-        flush.zero_()
-        ev2[i][0].record()
-        for h, d in ((hq, q), (hk, k), (hv, v), (ha, al), (hb, be)):
-            d.copy_(h, non_blocking=True)
-        call()
-        hy.copy_(out, non_blocking=True)
-        ev2[i][1].record()
+    e0, e1 = e2e_steps(K)
     dist.barrier()
-    e2e_ms = dist.max(sum(a.elapsed_time(b) for a, b in ev2))
+    e2e_ms = dist.max(e0.elapsed_time(e1))
 
     tokens_all = T * dist.world * K
     return {
@@ -306,6 +345,119 @@ def bench_output_gate(args, dist, torch, gdn, peaks, peak_src):
             "roofline": {"kernel": "output_gate", "bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
                          "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"], "traffic": None,
                          "peak_source": peak_src, "algorithmic_bytes_per_launch": byts}}
+
+
+# ----------------------------------------------------------------------------- QSA indexer
+QSA_FLOP_PER_CAND = 4 * D * 2       # per (query, candidate block): 4 head dot products of 128
+QSA_UNIT = "query tokens/s"
+
+
+def qsa_candidates(B, T, Qn):
+    """Candidate blocks summed over the queries (positions T-Qn .. T-1 of each row)."""
+    i = np.arange(T - Qn, T, dtype=np.int64)
+    return int(B * np.sum((i + 1) // 4))
+
+
+def bench_qsa(args, dist, torch, gdn, peaks, peak_src, wl):
+    """QSA indexer step on resident inputs: the step's new block keys into the cache, then the
+    block scores and top-512 selection of its queries (token sets included); L2 flushed
+    between steps.  prefill: 8192 queries at the end of a 64K-token sequence; decode: 64 rows
+    x 4 query tokens at 128K (the newest block completes within the step)."""
+    cfg = gi.QSA_PREFILL if wl == "prefill" else gi.QSA_DECODE
+    B, T, Qn, eps, theta = cfg["B"], cfg["context"], cfg["queries"], cfg["eps"], cfg["theta"]
+    nb = T // 4
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(gi.BASE_SEED + 4242 + (0 if wl == "prefill" else 1) + 7919 * dist.rank)
+    k = torch.randn((B, T, D), generator=gen, device="cuda").to(torch.bfloat16)
+    q = torch.randn((B, Qn, 4, D), generator=gen, device="cuda").to(torch.bfloat16)
+    w_k = torch.rand(D, generator=gen, device="cuda") + 0.5
+    w_q = torch.rand(D, generator=gen, device="cuda") + 0.5
+    new0 = T - Qn if wl == "prefill" else T - 4        # first token whose key the step adds
+    kbar = torch.zeros((B, nb, D), dtype=torch.bfloat16, device="cuda")
+    i32 = torch.int32
+    gdn.qsa_block_keys(k[:, :new0].contiguous(), w_k, torch.zeros(B, dtype=i32, device="cuda"), kbar,
+                       eps=eps, theta=theta)
+    k_new = k[:, new0:].contiguous()
+    kpos = torch.full((B,), new0, dtype=i32, device="cuda")
+    qpos = torch.full((B,), T - Qn, dtype=i32, device="cuda")
+    nblk = torch.full((B,), nb, dtype=i32, device="cuda")
+    blocks = torch.empty((B, Qn, gdn.QSA_BUDGET), dtype=i32, device="cuda")
+    tokens = torch.empty((B, Qn, gdn.QSA_TOKEN_SLOTS), dtype=i32, device="cuda")
+    ws = torch.empty(gdn.qsa_select_workspace_size(B, Qn, nb), dtype=torch.uint8, device="cuda")
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+
+    def step():
+        gdn.qsa_block_keys(k_new, w_k, kpos, kbar, eps=eps, theta=theta)
+        gdn.qsa_select(q, w_q, qpos, kbar, nblk, eps=eps, theta=theta, blocks=blocks, tokens=tokens,
+                       workspace=ws)
+
+    for _ in range(args.warmup):
+        step()
+    K = args.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    dist.barrier()
+    for i in range(K):
+        flush.zero_()
+        ev[i][0].record()
+        step()
+        ev[i][1].record()
+    dist.barrier()
+    ms = dist.max(sum(a.elapsed_time(b) for a, b in ev)) / K
+    trace = gdn.LaunchTrace(capacity=4 * K + 8)
+    with trace:
+        for _ in range(K):
+            flush.zero_()
+            step()
+    dist.barrier()
+    per = {}
+    for n, t in trace.records():
+        per.setdefault(n, []).append(t)
+    per_kernel = {n: {"launches": len(v), "avg_ms": sum(v) / len(v), "total_ms": sum(v)} for n, v in per.items()}
+    cand = qsa_candidates(B, T, Qn)
+    sc_s = per_kernel["qsa_scores"]["avg_ms"] / 1e3
+    flops = cand * QSA_FLOP_PER_CAND
+    byts = cand * 4 + B * nb * D * 2 + B * Qn * 4 * D * 2       # scores out, keys and queries in
+    t_tensor = flops / (peaks["bf16_tflops"] * 1e12)
+    t_hbm = byts / (peaks["hbm_gbs"] * 1e9)
+    if t_tensor >= t_hbm:
+        roof = {"kernel": "qsa_scores", "bound": "tensor", "achieved": flops / sc_s / 1e12,
+                "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": flops / sc_s / 1e12 / peaks["bf16_tflops"]}
+    else:
+        roof = {"kernel": "qsa_scores", "bound": "hbm", "achieved": byts / sc_s / 1e9, "peak": peaks["hbm_gbs"],
+                "unit": "GB/s", "frac": byts / sc_s / 1e9 / peaks["hbm_gbs"]}
+    roof.update({"traffic": None, "peak_source": peak_src, "algorithmic_flops_per_launch": flops,
+                 "algorithmic_bytes_per_launch": byts, "candidates_per_launch": cand})
+    tk_s = per_kernel["qsa_topk"]["avg_ms"] / 1e3
+    tk_bytes = cand * 4 + B * Qn * (gdn.QSA_BUDGET + gdn.QSA_TOKEN_SLOTS) * 4
+    topk = {"kernel": "qsa_topk", "bound": "hbm", "achieved": tk_bytes / tk_s / 1e9, "peak": peaks["hbm_gbs"],
+            "unit": "GB/s", "frac": tk_bytes / tk_s / 1e9 / peaks["hbm_gbs"], "algorithmic_bytes_per_launch": tk_bytes}
+    return {"value": B * Qn * dist.world / (ms / 1e3), "unit": QSA_UNIT, "ms_per_step": ms,
+            "workload": f"qsa-{wl}-B{B}-ctx{T}-q{Qn}", "kernels": per_kernel, "roofline": roof, "topk": topk,
+            "l2": "flushed: 256 MiB write between steps"}
+
+
+def qsa_oracle_rows_per_s(target_s: float):
+    """The oracle on sampled query rows of the prefill workload (one row = its 4 heads
+    against every candidate block, then the top-512 and token set)."""
+    from oracle import qsa_indexer as qi
+    cfg = gi.QSA_PREFILL
+    T, Qn = cfg["context"], cfg["queries"]
+    inp = gi.make_qsa_inputs(1, T, 8, seed=77)
+    k64 = gi.bf16_bits_to_f32(inp.k[0]).astype(np.float64)
+    q64 = gi.bf16_bits_to_f32(inp.q[0]).astype(np.float64)
+    t0 = time.perf_counter()
+    kb = qi.block_keys(k64, inp.w_k, cfg["eps"], cfg["theta"], operands="bf16")
+    rows = 0
+    while True:
+        j = rows % 8
+        i = T - Qn + j * (Qn // 8)
+        qh = qi.query_heads(q64[j:j + 1], inp.w_q, [i], cfg["eps"], cfg["theta"], operands="bf16")
+        s = qi.block_scores(qh, kb, [i])[0]
+        qi.token_set(qi.top_blocks(s), i)
+        rows += 1
+        dt = time.perf_counter() - t0
+        if dt >= target_s:
+            return rows / dt, rows, dt
 
 
 def prefill_roofline(res, peaks, peak_src):
@@ -564,6 +716,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--decode-steps", type=int, default=1024)
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-qsa", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-baseline-s", type=float, default=15.0)
     ap.add_argument("--ref-step-s", type=float, default=5.0)
@@ -581,6 +734,14 @@ def main():
     roof = prefill_roofline(pre, peaks, peak_src)
     dec = None if args.no_decode else bench_decode(args, dist, torch, gdn, peaks, peak_src)
     tail = bench_output_gate(args, dist, torch, gdn, peaks, peak_src)
+    qsa = None
+    if not args.no_qsa:
+        qsa = {wl: bench_qsa(args, dist, torch, gdn, peaks, peak_src, wl) for wl in ("prefill", "decode")}
+        if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
+            v, n, dt = qsa_oracle_rows_per_s(min(5.0, args.cpu_baseline_s))
+            qsa["cpu_baseline"] = {"value": v, "unit": QSA_UNIT, "cores": 1, "kind": "oracle",
+                                   "sample": f"{n} query rows of qsa-prefill (block keys of the full context once)",
+                                   "seconds": dt}
     cpu = None
     if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
         v, threads, sample, dt = oracle_tokens_per_s(args.cpu_baseline_s)
@@ -598,6 +759,7 @@ def main():
                        "parallelism": f"dp{dist.world} (independent sequences per GPU)"},
             "clocks": pre["clocks"], "e2e": pre["e2e"], "gpu_launches": pre["launches"],
             "roofline": roof, "kernels": pre["per_kernel"], "cpu_baseline": cpu, "decode": dec, "output_gate": tail,
+            "qsa": qsa,
             "peaks": peak_src,
         }
         print(json.dumps(line), flush=True)

@@ -295,3 +295,36 @@ def decode_workload_step(step: int, index: int = 3) -> DecodeInputs:
     w = WORKLOADS[index]
     return make_decode_step(w["shape"], w["batch"], step, w["dtype"], workload_seed(index) + 2000,
                             c=w["c"])
+
+
+# --------------------------------------------------------------------------- QSA indexer
+# The indexer's inputs are projections of the hidden state (outside the path): raw key
+# rows [B, T, 128] and query heads [B, Qn, 4, 128], N(0, 1) stored as bf16, and the two
+# RMSNorm weights ~ U(0.5, 1.5) in fp32.  The workloads are the pages' indexer setting
+# (r = 4, 512-block budget) at long context: a chunk of queries at the end of a sequence
+# whose block-key cache covers all earlier tokens.
+_QSA_STREAMS = ("k", "q", "w_k", "w_q")
+
+
+@dataclass
+class QsaInputs:
+    k: np.ndarray      # uint16 bf16 bits [B, T, 128]
+    q: np.ndarray      # uint16 bf16 bits [B, Qn, 4, 128]
+    w_k: np.ndarray    # float32 [128]
+    w_q: np.ndarray    # float32 [128]
+
+
+def make_qsa_inputs(B: int, T: int, Qn: int, seed: int) -> QsaInputs:
+    kids = np.random.SeedSequence([seed, 0x05A]).spawn(len(_QSA_STREAMS))
+    r = {n: np.random.Generator(np.random.PCG64(s)) for n, s in zip(_QSA_STREAMS, kids)}
+    return QsaInputs(k=_normal_stored(r["k"], (B, T, 128), BF16),
+                     q=_normal_stored(r["q"], (B, Qn, 4, 128), BF16),
+                     w_k=r["w_k"].uniform(0.5, 1.5, 128).astype(np.float32),
+                     w_q=r["w_q"].uniform(0.5, 1.5, 128).astype(np.float32))
+
+
+# chunked prefill at 64K context: 8192 query tokens (positions 57344..65535) of one
+# sequence over its 16384 block keys
+QSA_PREFILL = {"B": 1, "context": 65536, "queries": 8192, "theta": 10000.0, "eps": 1e-6}
+# decode with 3 speculative tokens: 64 rows x 4 query tokens at 128K context
+QSA_DECODE = {"B": 64, "context": 131072, "queries": 4, "theta": 10000.0, "eps": 1e-6}

@@ -251,6 +251,71 @@ GDN_EXPORT gdn_status gdn_prefill_static_scratch(
     const void *conv_state_in, void *conv_state_out,
     void *out, cudaStream_t stream);
 
+/* ========================================================================== QSA indexer
+ *
+ * The block selector in front of the sparse attention layers (page "ARCHITECTURE
+ * PREVIEW / FIELD NOTES", section 03: the QSA indexer figure with its BLOCK SCORE and
+ * CAUSAL SPARSE SET formulas, and the five-step "QSA" list; section 01: 4 query heads
+ * sharing 1 key head, head dim 128, budget 512 blocks = 2048 tokens):
+ *
+ *   block key     kbar_b = RoPE_{4b}( RMSNorm( mean of the indexer keys of tokens 4b..4b+3 ) * w_k )
+ *   query heads   qh_i^h = RoPE_i( RMSNorm( q_i^h ) * w_q ),  h = 0..3
+ *   block score   I[i][b] = sum_h ReLU(<qh_i^h, kbar_b>)  for the blocks complete at token i
+ *                 (4b + 3 <= i); other blocks are not candidates
+ *   block set     B_i = the 512 highest-scoring candidates (all of them when fewer)
+ *   token set     S_i = tokens 4b..4b+3 of every b in B_i, then the tail 4 floor((i+1)/4) .. i
+ *
+ * with RMSNorm(x) = x / sqrt(mean(x^2) + eps) over the 128 dims, and RoPE_p rotating the
+ * pairs (d, d+32), d < 32, by the angle p * theta^(-d/32) (x_d' = x_d cos - x_{d+32} sin,
+ * x_{d+32}' = x_{d+32} cos + x_d sin); dims 64..127 are not rotated.  Equal scores rank the
+ * lower block index first.  Arithmetic: fp32 (angles formed and reduced in fp64); the
+ * rotated query heads and the block keys are rounded to bf16 and the scores are products
+ * of those bf16 values accumulated in fp32 on the tensor cores (kind::f16).
+ *
+ * Layouts (all device memory, row-major, contiguous):
+ *   k       bf16 [B][Tn][128]      indexer keys of tokens kpos[b] .. kpos[b] + Tn - 1
+ *   kbar    bf16 [B][nb_max][128]  block-key cache: entry j of row b is block j (tokens 4j..4j+3)
+ *   q       bf16 [B][Qn][4][128]   indexer query heads of tokens qpos[b] .. qpos[b] + Qn - 1
+ *   w_k, w_q  fp32 [128]           RMSNorm weights (w_q shared by the 4 heads)
+ *   kpos, qpos, n_blocks  int32 [B] (device): first token position of row b's keys /
+ *           queries, and how many cache entries of row b are valid
+ *   scores  fp32 [B][Qn][nb_max]
+ *   blocks  int32 [B][Qn][512]     B_i in ascending block order, then -1
+ *   tokens  int32 [B][Qn][2051]    S_i in ascending order, then -1
+ * Device-side values are clamped, never trusted: a query at position i has
+ * min(floor((i+1)/4), n_blocks[b], nb_max) candidate blocks (none when i < 0); a
+ * key call whose kpos[b] is negative or not a multiple of 4 writes nothing for row b, and
+ * blocks that would land at or past nb_max are not written.
+ * Requirements: compute capability 10.0; pointers 16-byte aligned; B, Tn, Qn >= 0,
+ * Tn % 4 == 0, nb_max >= 1, 4 * nb_max < 2^31; eps >= 0 and theta > 0 finite.
+ * A bounded device-side wait that gives up (never expected) leaves NaN in the affected
+ * scores and -2 in every entry of the affected rows of blocks and tokens.
+ */
+
+/* Writes the block keys of each row's Tn / 4 complete blocks into kbar (other entries untouched). */
+GDN_EXPORT gdn_status gdn_qsa_block_keys(const void *k, const float *w_k, const int32_t *kpos,
+                                         int B, int Tn, float eps, float theta,
+                                         void *kbar, int nb_max, cudaStream_t stream);
+
+/* I[i][b] of every query and every candidate block into `scores` (entries of non-candidate
+ * blocks are unspecified).  Needs no workspace. */
+GDN_EXPORT gdn_status gdn_qsa_block_scores(const void *q, const float *w_q, const int32_t *qpos,
+                                           const void *kbar, const int32_t *n_blocks,
+                                           int B, int Qn, int nb_max, float eps, float theta,
+                                           float *scores, cudaStream_t stream);
+
+/* Bytes of workspace gdn_qsa_select needs (the scores of every query row).  Writes *bytes. */
+GDN_EXPORT gdn_status gdn_qsa_select_workspace_size(int B, int Qn, int nb_max, size_t *bytes);
+
+/* B_i (and S_i when `tokens` is not NULL) of every query.  `workspace` (256-byte aligned,
+ * at least gdn_qsa_select_workspace_size bytes) is scratch; it must not be shared by two
+ * calls in flight. */
+GDN_EXPORT gdn_status gdn_qsa_select(const void *q, const float *w_q, const int32_t *qpos,
+                                     const void *kbar, const int32_t *n_blocks,
+                                     int B, int Qn, int nb_max, float eps, float theta,
+                                     int32_t *blocks, int32_t *tokens,
+                                     void *workspace, size_t workspace_bytes, cudaStream_t stream);
+
 /*
  * Launch trace (a profiling aid; no counterpart on the pages).  While a trace is
  * active on a host thread, every kernel that a libgdn call made on that thread

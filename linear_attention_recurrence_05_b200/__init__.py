@@ -20,7 +20,8 @@ from . import _native
 from ._native import GDN_BF16, GDN_F32, GdnError  # noqa: F401
 
 __all__ = ["GdnConfig", "gdn_prefill", "gdn_decode_step", "gdn_decode_multi", "gdn_output_gate", "prefill_workspace_size", "GdnError",
-           "library_path"]
+           "library_path", "qsa_block_keys", "qsa_block_scores", "qsa_select", "qsa_select_workspace_size",
+           "QSA_BUDGET", "QSA_TOKEN_SLOTS"]
 
 
 @dataclass(frozen=True)
@@ -242,3 +243,81 @@ class LaunchTrace:
         n = min(self.count, self.capacity)
         return [(self._arr[i].kernel.decode(), self.events[i][0].elapsed_time(self.events[i][1]))
                 for i in range(n)]
+
+
+# ----------------------------------------------------------------------------- QSA indexer
+QSA_BUDGET = 512                  # blocks per query
+QSA_TOKEN_SLOTS = 4 * 512 + 3     # token-set entries per query
+
+
+def _qsa_check(name, t, dtype, shape_len):
+    if t.dtype != dtype or t.dim() != shape_len or not t.is_contiguous() or not t.is_cuda:
+        raise TypeError(f"{name}: expected a contiguous CUDA {dtype} tensor of rank {shape_len}")
+
+
+def qsa_block_keys(k, w_k, kpos, kbar, *, eps: float = 1e-6, theta: float = 10000.0, stream=None):
+    """Write the QSA block keys of k [B, Tn, 128] (bf16, tokens kpos[b] .. kpos[b]+Tn-1 of
+    row b, Tn % 4 == 0) into the cache kbar [B, nb_max, 128] (bf16) at blocks kpos[b]/4 ...
+    w_k fp32 [128]; kpos int32 [B] on the device.  Returns kbar."""
+    _qsa_check("k", k, torch.bfloat16, 3)
+    _qsa_check("kbar", kbar, torch.bfloat16, 3)
+    _qsa_check("kpos", kpos, torch.int32, 1)
+    _qsa_check("w_k", w_k, torch.float32, 1)
+    B, Tn, _ = k.shape
+    st = _native.lib().gdn_qsa_block_keys(_ptr(k), _ptr(w_k), _ptr(kpos), B, Tn, float(eps), float(theta),
+                                          _ptr(kbar), kbar.shape[1], _stream(stream))
+    _native.check("gdn_qsa_block_keys", st)
+    return kbar
+
+
+def _qsa_query_args(q, w_q, qpos, kbar, n_blocks):
+    _qsa_check("q", q, torch.bfloat16, 4)
+    _qsa_check("kbar", kbar, torch.bfloat16, 3)
+    _qsa_check("qpos", qpos, torch.int32, 1)
+    _qsa_check("n_blocks", n_blocks, torch.int32, 1)
+    _qsa_check("w_q", w_q, torch.float32, 1)
+    if q.shape[2] != 4 or q.shape[3] != 128 or kbar.shape[2] != 128 or kbar.shape[0] != q.shape[0]:
+        raise ValueError("q must be [B, Qn, 4, 128] and kbar [B, nb_max, 128]")
+    return q.shape[0], q.shape[1], kbar.shape[1]
+
+
+def qsa_block_scores(q, w_q, qpos, kbar, n_blocks, *, eps: float = 1e-6, theta: float = 10000.0,
+                     out=None, stream=None):
+    """Block scores [B, Qn, nb_max] fp32 of the queries q [B, Qn, 4, 128] (bf16, tokens
+    qpos[b] .. of row b) against the block-key cache; entries of blocks that are not
+    candidates of a query are unspecified."""
+    B, Qn, nb = _qsa_query_args(q, w_q, qpos, kbar, n_blocks)
+    if out is None:
+        out = torch.empty((B, Qn, nb), dtype=torch.float32, device=q.device)
+    st = _native.lib().gdn_qsa_block_scores(_ptr(q), _ptr(w_q), _ptr(qpos), _ptr(kbar), _ptr(n_blocks), B, Qn, nb,
+                                            float(eps), float(theta), _ptr(out), _stream(stream))
+    _native.check("gdn_qsa_block_scores", st)
+    return out
+
+
+def qsa_select_workspace_size(B: int, Qn: int, nb_max: int) -> int:
+    n = ctypes.c_size_t(0)
+    st = _native.lib().gdn_qsa_select_workspace_size(B, Qn, nb_max, ctypes.byref(n))
+    _native.check("gdn_qsa_select_workspace_size", st)
+    return int(n.value)
+
+
+def qsa_select(q, w_q, qpos, kbar, n_blocks, *, eps: float = 1e-6, theta: float = 10000.0,
+               blocks=None, tokens=None, with_tokens: bool = False, workspace=None, stream=None):
+    """Top-512 block set (and with ``with_tokens`` or a given ``tokens`` buffer, the token
+    set) of every query.  Returns (blocks int32 [B, Qn, 512], tokens int32 [B, Qn, 2051]
+    or None), ascending and padded with -1."""
+    B, Qn, nb = _qsa_query_args(q, w_q, qpos, kbar, n_blocks)
+    if blocks is None:
+        blocks = torch.empty((B, Qn, QSA_BUDGET), dtype=torch.int32, device=q.device)
+    if tokens is None and with_tokens:
+        tokens = torch.empty((B, Qn, QSA_TOKEN_SLOTS), dtype=torch.int32, device=q.device)
+    need = qsa_select_workspace_size(B, Qn, nb)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
+    st = _native.lib().gdn_qsa_select(_ptr(q), _ptr(w_q), _ptr(qpos), _ptr(kbar), _ptr(n_blocks), B, Qn, nb,
+                                      float(eps), float(theta), _ptr(blocks),
+                                      None if tokens is None else _ptr(tokens), _ptr(workspace),
+                                      workspace.numel() * workspace.element_size(), _stream(stream))
+    _native.check("gdn_qsa_select", st)
+    return blocks, tokens

@@ -21,7 +21,8 @@ STATUS = {0: "GDN_OK", 1: "GDN_ERR_INVALID_ARG", 2: "GDN_ERR_UNSUPPORTED", 3: "G
 EXPORTS = ("gdn_status_string", "gdn_last_cuda_error", "gdn_api_version",
            "gdn_prefill_workspace_size", "gdn_prefill", "gdn_decode_step", "gdn_decode_multi",
            "gdn_output_gate", "gdn_trace_begin",
-           "gdn_trace_end", "gdn_prefill_static_scratch")
+           "gdn_trace_end", "gdn_prefill_static_scratch", "gdn_qsa_block_keys",
+           "gdn_qsa_block_scores", "gdn_qsa_select_workspace_size", "gdn_qsa_select")
 
 STATIC_SCRATCH_BYTES = 64 << 20  # GDN_STATIC_SCRATCH_BYTES
 
@@ -97,6 +98,16 @@ def lib():
                                                      i32p, ctypes.c_int, ctypes.c_int64, fp, fp,
                                                      vp, vp, vp, vp]
             L.gdn_prefill_static_scratch.restype = ctypes.c_int
+            ci, cf = ctypes.c_int, ctypes.c_float
+            L.gdn_qsa_block_keys.argtypes = [vp, fp, i32p, ci, ci, cf, cf, vp, ci, vp]
+            L.gdn_qsa_block_keys.restype = ctypes.c_int
+            L.gdn_qsa_block_scores.argtypes = [vp, fp, i32p, vp, i32p, ci, ci, ci, cf, cf, fp, vp]
+            L.gdn_qsa_block_scores.restype = ctypes.c_int
+            L.gdn_qsa_select_workspace_size.argtypes = [ci, ci, ci, ctypes.POINTER(ctypes.c_size_t)]
+            L.gdn_qsa_select_workspace_size.restype = ctypes.c_int
+            L.gdn_qsa_select.argtypes = [vp, fp, i32p, vp, i32p, ci, ci, ci, cf, cf, i32p, i32p, vp,
+                                         ctypes.c_size_t, vp]
+            L.gdn_qsa_select.restype = ctypes.c_int
             _lib = L
         return _lib
 

@@ -405,4 +405,80 @@ gdn_status gdn_output_gate(const gdn_config *cfg, gdn_dtype y_dtype, gdn_dtype z
     return GDN_OK;
 }
 
+// ------------------------------------------------------------------ QSA indexer
+static bool qsa_scalars_ok(float eps, float theta) {
+    return std::isfinite(eps) && eps >= 0.f && std::isfinite(theta) && theta > 0.f;
+}
+static bool qsa_sizes_ok(int B, int n, int nb_max) {
+    return B >= 0 && n >= 0 && nb_max >= 1 && B <= 65535 && nb_max < (1 << 29) &&
+           (int64_t)B * nb_max < ((int64_t)1 << 31) - 256;
+}
+
+gdn_status gdn_qsa_block_keys(const void *k, const float *w_k, const int32_t *kpos, int B, int Tn,
+                              float eps, float theta, void *kbar, int nb_max, cudaStream_t stream) {
+    if (!qsa_sizes_ok(B, Tn, nb_max) || Tn % 4 != 0 || !qsa_scalars_ok(eps, theta)) return GDN_ERR_INVALID_ARG;
+    if ((int64_t)B * Tn > ((int64_t)1 << 36)) return GDN_ERR_UNSUPPORTED;
+    if (B == 0 || Tn == 0) return GDN_OK;
+    if (!k || !w_k || !kpos || !kbar) return GDN_ERR_INVALID_ARG;
+    if (!aligned(k, 16) || !aligned(w_k, 16) || !aligned(kpos, 16) || !aligned(kbar, 16)) return GDN_ERR_INVALID_ARG;
+    gdn_status st = check_device();
+    if (st != GDN_OK) return st;
+    cudaError_t e = launch_qsa_block_keys(k, w_k, kpos, B, Tn, eps, theta, kbar, nb_max, stream);
+    if (e != cudaSuccess) return cuda_fail(e);
+    return GDN_OK;
+}
+
+static gdn_status qsa_query_args(const void *q, const float *w_q, const int32_t *qpos, const void *kbar,
+                                 const int32_t *n_blocks, int B, int Qn, int nb_max, float eps, float theta) {
+    if (!qsa_sizes_ok(B, Qn, nb_max) || !qsa_scalars_ok(eps, theta)) return GDN_ERR_INVALID_ARG;
+    if ((int64_t)B * Qn >= ((int64_t)1 << 31)) return GDN_ERR_UNSUPPORTED;
+    if (B == 0 || Qn == 0) return GDN_OK;
+    if (!q || !w_q || !qpos || !kbar || !n_blocks) return GDN_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(w_q, 16) || !aligned(qpos, 16) || !aligned(kbar, 16) || !aligned(n_blocks, 16))
+        return GDN_ERR_INVALID_ARG;
+    return GDN_OK;
+}
+
+gdn_status gdn_qsa_block_scores(const void *q, const float *w_q, const int32_t *qpos, const void *kbar,
+                                const int32_t *n_blocks, int B, int Qn, int nb_max, float eps, float theta,
+                                float *scores, cudaStream_t stream) {
+    gdn_status st = qsa_query_args(q, w_q, qpos, kbar, n_blocks, B, Qn, nb_max, eps, theta);
+    if (st != GDN_OK) return st;
+    if (B == 0 || Qn == 0) return GDN_OK;
+    if (!scores || !aligned(scores, 16)) return GDN_ERR_INVALID_ARG;
+    st = check_device();
+    if (st != GDN_OK) return st;
+    cudaError_t e = launch_qsa_scores(q, w_q, qpos, kbar, n_blocks, B, Qn, nb_max, eps, theta, scores, stream);
+    if (e != cudaSuccess) return cuda_fail(e);
+    return GDN_OK;
+}
+
+gdn_status gdn_qsa_select_workspace_size(int B, int Qn, int nb_max, size_t *bytes) {
+    if (!bytes) return GDN_ERR_INVALID_ARG;
+    if (!qsa_sizes_ok(B, Qn, nb_max)) return GDN_ERR_INVALID_ARG;
+    *bytes = (((size_t)B * Qn * nb_max * 4) + 255) & ~(size_t)255;
+    return GDN_OK;
+}
+
+gdn_status gdn_qsa_select(const void *q, const float *w_q, const int32_t *qpos, const void *kbar,
+                          const int32_t *n_blocks, int B, int Qn, int nb_max, float eps, float theta,
+                          int32_t *blocks, int32_t *tokens, void *workspace, size_t workspace_bytes,
+                          cudaStream_t stream) {
+    gdn_status st = qsa_query_args(q, w_q, qpos, kbar, n_blocks, B, Qn, nb_max, eps, theta);
+    if (st != GDN_OK) return st;
+    if (B == 0 || Qn == 0) return GDN_OK;
+    if (!blocks || !aligned(blocks, 16) || (tokens && !aligned(tokens, 16))) return GDN_ERR_INVALID_ARG;
+    size_t need = 0;
+    gdn_qsa_select_workspace_size(B, Qn, nb_max, &need);
+    if (!workspace || !aligned(workspace, 256) || workspace_bytes < need) return GDN_ERR_WORKSPACE;
+    st = check_device();
+    if (st != GDN_OK) return st;
+    float *scores = static_cast<float *>(workspace);
+    cudaError_t e = launch_qsa_scores(q, w_q, qpos, kbar, n_blocks, B, Qn, nb_max, eps, theta, scores, stream);
+    if (e != cudaSuccess) return cuda_fail(e);
+    e = launch_qsa_topk(scores, qpos, n_blocks, B, Qn, nb_max, blocks, tokens, stream);
+    if (e != cudaSuccess) return cuda_fail(e);
+    return GDN_OK;
+}
+
 }  // extern "C"

@@ -106,6 +106,15 @@ void record_cuda_error(cudaError_t e);
 constexpr int kGateRec = 160;            // floats: gamma_t [64], kd_t [64], gamma_C, padding
 constexpr int kGrGamma = 0, kGrKd = 64, kGrGammaC = 128;
 
+// QSA indexer launchers (qsa_indexer.cu)
+cudaError_t launch_qsa_block_keys(const void *k, const float *w, const int32_t *kpos, int B, int Tn,
+                                  float eps, float theta, void *kbar, int nb_max, cudaStream_t s);
+cudaError_t launch_qsa_scores(const void *q, const float *w, const int32_t *qpos, const void *kbar,
+                              const int32_t *n_blocks, int B, int Qn, int nb_max, float eps, float theta,
+                              float *scores, cudaStream_t s);
+cudaError_t launch_qsa_topk(const float *scores, const int32_t *qpos, const int32_t *n_blocks, int B, int Qn,
+                            int nb_max, int32_t *blocks, int32_t *tokens, cudaStream_t s);
+
 // launchers: return the cudaError_t of the launch
 cudaError_t launch_seq_table(const int32_t *cu_in, int n_seqs, int64_t T, int32_t *cu,
                              int32_t *cfirst, cudaStream_t s);

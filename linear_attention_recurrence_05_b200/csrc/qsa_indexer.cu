@@ -1,0 +1,601 @@
+// QSA indexer: block keys, block scores and the top-512 block selection.
+//
+// Page "ARCHITECTURE PREVIEW / FIELD NOTES", section 03, the QSA indexer figure (BLOCK
+// SCORE, CAUSAL SPARSE SET) and the five-step "QSA" list; section 01 for the shapes (4
+// query heads over 1 shared key head, head dim 128, 512 blocks of 4 tokens).
+//
+//   qsa_block_keys_kernel   warp per block: mean of 4 key rows, RMSNorm, rotary encoding at
+//                           the block's first token, bf16 into the block-key cache
+//   qsa_scores_kernel       CTA per (row, 4..64 queries, share of the block range): the
+//                           query heads are normalised and rotated into shared memory once;
+//                           128-block key tiles stream in by TMA; one kind::f16 MMA chain per
+//                           tile gives every (block, query head) dot product in tensor
+//                           memory; the epilogue sums the ReLUs of the 4 heads and stores the
+//                           fp32 scores, query-major
+//   qsa_topk_kernel         CTA per query: 3-digit radix select (11 + 10 + 10 bits of the
+//                           non-negative score's bit pattern) of the 512th largest score,
+//                           then one ordered pass that writes the selected blocks in
+//                           ascending order (equal scores: lower index first) and the tokens
+#include <cuda_bf16.h>
+#include <math.h>
+#include <stdint.h>
+
+#include <algorithm>
+#include <cmath>
+
+#include "gdn_internal.h"
+#include "tc_sm100.cuh"
+#include "tma_map.cuh"
+
+namespace gdn {
+namespace qsa {
+
+using namespace tc;
+
+constexpr int kR = 4;                       // tokens per block
+constexpr int kD = 128;                     // indexer head dim
+constexpr int kHeads = 4;                   // indexer query heads
+constexpr int kKB = 512;                    // block budget
+constexpr int kTok = kR * kKB + kR - 1;     // token-set slots per query
+constexpr uint32_t kWaitTries = 1u << 22;
+
+// ------------------------------------------------------------------ shared pieces
+__device__ __forceinline__ double inv_freq(int d, double log2_theta) {
+    return exp2(-(double)d * (log2_theta / 32.0));
+}
+// cos and sin of pos * f: the angle is formed and reduced to [-pi, pi] in fp64, where the
+// hardware sine/cosine is within about 2^-21 (far below the bf16 rounding that follows)
+__device__ __forceinline__ void rope_cs(int64_t pos, double f, float &c, float &s) {
+    const double two_pi = 6.283185307179586;
+    const double a = (double)pos * f;
+    const double n = rint(a * (1.0 / two_pi));
+    __sincosf((float)fma(-n, two_pi, a), &s, &c);
+}
+__device__ __forceinline__ void unpack4(uint2 u, float (&x)[4]) {
+    x[0] = __uint_as_float(u.x << 16);
+    x[1] = __uint_as_float(u.x & 0xFFFF0000u);
+    x[2] = __uint_as_float(u.y << 16);
+    x[3] = __uint_as_float(u.y & 0xFFFF0000u);
+}
+__device__ __forceinline__ uint2 pack4(const float (&x)[4]) {
+    __nv_bfloat162 a = __floats2bfloat162_rn(x[0], x[1]), b = __floats2bfloat162_rn(x[2], x[3]);
+    return make_uint2(*reinterpret_cast<uint32_t *>(&a), *reinterpret_cast<uint32_t *>(&b));
+}
+// RMSNorm * w, then the rotary encoding, of one 128-dim row held by a warp, 4 dims per lane
+// (lane l: dims 4l..4l+3).  c, s: this lane's 4 cos/sin (lanes 0..15; dims d and d + 32 of
+// a pair sit in lanes l and l + 8).
+__device__ __forceinline__ void norm_rope_row(float (&x)[4], const float4 w, float eps,
+                                              const float (&c)[4], const float (&s)[4], int lane) {
+    float ss = x[0] * x[0] + x[1] * x[1] + x[2] * x[2] + x[3] * x[3];
+#pragma unroll
+    for (int o = 16; o; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    const float r = rsqrtf(ss * (1.f / kD) + eps);
+    x[0] *= r * w.x;
+    x[1] *= r * w.y;
+    x[2] *= r * w.z;
+    x[3] *= r * w.w;
+    float o[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) o[e] = __shfl_xor_sync(0xffffffffu, x[e], 8);
+    if (lane < 8) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) x[e] = x[e] * c[e] - o[e] * s[e];
+    } else if (lane < 16) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) x[e] = x[e] * c[e] + o[e] * s[e];
+    }
+}
+// candidate blocks of a query at position pos: complete blocks, capped by the valid cache
+__device__ __forceinline__ int64_t n_cand(int64_t pos, int64_t cap) {
+    return pos < 0 ? 0 : min((pos + 1) >> 2, cap);
+}
+
+// ------------------------------------------------------------------ block keys
+struct KeyParams {
+    const __nv_bfloat16 *k;
+    const float *w;
+    const int32_t *kpos;
+    __nv_bfloat16 *kbar;
+    int B, Tn, nb_max;
+    float eps, theta;
+};
+
+__global__ void __launch_bounds__(256) qsa_block_keys_kernel(const __grid_constant__ KeyParams p) {
+    const int lane = threadIdx.x & 31;
+    const int nbj = p.Tn / kR;
+    const int64_t gw = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+    if (gw >= (int64_t)p.B * nbj) return;                  // whole warps leave together
+    const int b = (int)(gw / nbj), j = (int)(gw % nbj);
+    const int kp = p.kpos[b];
+    if (kp < 0 || (kp & 3)) return;
+    const int64_t blk = (int64_t)(kp >> 2) + j;
+    if (blk >= p.nb_max) return;
+    const uint2 *src = reinterpret_cast<const uint2 *>(p.k + ((int64_t)b * p.Tn + (int64_t)j * kR) * kD) + lane;
+    float x[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int t = 0; t < kR; ++t) {
+        float r[4];
+        unpack4(__ldg(src + t * (kD / 4)), r);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) x[e] += r[e];
+    }
+#pragma unroll
+    for (int e = 0; e < 4; ++e) x[e] *= 1.f / kR;
+    float c[4] = {1.f, 1.f, 1.f, 1.f}, s[4] = {0.f, 0.f, 0.f, 0.f};
+    if (lane < 16) {
+        const double l2t = log2((double)p.theta);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) rope_cs(kR * blk, inv_freq(4 * (lane & 7) + e, l2t), c[e], s[e]);
+    }
+    const float4 w = __ldg(reinterpret_cast<const float4 *>(p.w) + lane);
+    norm_rope_row(x, w, p.eps, c, s, lane);
+    reinterpret_cast<uint2 *>(p.kbar + ((int64_t)b * p.nb_max + blk) * kD)[lane] = pack4(x);
+}
+
+// ------------------------------------------------------------------ block scores
+constexpr int kStages = 4;
+constexpr uint32_t kTileBytes = 128 * kD * 2;      // 128 blocks x 128 dims, bf16
+constexpr uint32_t kHalf = kTileBytes / 2;         // one 64-dim column block (128-byte rows)
+constexpr uint32_t OFF_Q = 0;                      // query heads: <= 256 rows x 256 B
+constexpr uint32_t OFF_K = 65536;                  // key tiles, kStages deep
+constexpr uint32_t OFF_BAR = OFF_K + kStages * kTileBytes;
+enum { BAR_FULL = 0, BAR_EMPTY = kStages, BAR_TFULL = 2 * kStages, BAR_TEMPTY = 2 * kStages + 2,
+       BAR_Q = 2 * kStages + 4, kNumBars };
+constexpr uint32_t OFF_FLAG = OFF_BAR + 8 * 16;    // TMEM base, abort flag
+constexpr uint32_t kScoreSmem = OFF_FLAG + 16;
+constexpr int kScoreThr = 192;                     // warps 0-3 epilogue, 4 producer, 5 MMA
+constexpr int kMaxQT = 64;                         // queries per CTA (N = 4 x 64 = 256)
+
+struct ScoreParams {
+    CUtensorMap tm_kbar;        // kbar as [B * nb_max, 128] bf16 rows, boxes 64 x 128, 128B swizzle
+    const __nv_bfloat16 *q;
+    const float *w;
+    const int32_t *qpos, *n_blocks;
+    float *scores;
+    int B, Qn, nb_max, qt, n_split;
+    float eps, theta;
+};
+
+__device__ __forceinline__ void arrive(uint64_t *m) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(m)) : "memory");
+}
+// bounded wait that gives up early once another role has raised the abort flag
+__device__ __forceinline__ bool wait_abort(uint64_t *m, uint32_t par, volatile int *abort_flag) {
+    if (mbar_try_wait(m, par)) return true;
+    for (uint32_t i = 0; i < kWaitTries; ++i) {
+        if (mbar_try_wait_sleep(m, par, 40)) return true;
+        if ((i & 63) == 63 && *abort_flag) return false;
+    }
+    *abort_flag = 1;
+    return false;
+}
+
+__global__ void __launch_bounds__(kScoreThr, 1) qsa_scores_kernel(const __grid_constant__ ScoreParams p) {
+    extern __shared__ __align__(1024) unsigned char sm[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int b = blockIdx.y, q0 = blockIdx.x * p.qt;
+    const int nq = min(p.qt, p.Qn - q0);
+    const int N = kHeads * p.qt;                               // MMA N: (query, head) rows
+    const int64_t pos0 = p.qpos[b];
+    const int64_t cap = max(0, min(p.n_blocks[b], p.nb_max));
+    const int64_t ncand = n_cand(pos0 + q0 + nq - 1, cap);     // the tile's last query sees most
+    const int ntiles = (int)((ncand + 127) / 128);
+    const int per = (ntiles + p.n_split - 1) / p.n_split;
+    const int t0 = blockIdx.z * per, t1 = min(ntiles, t0 + per);
+    if (t0 >= t1) return;                                      // uniform per CTA
+    const int nt = t1 - t0;
+
+    uint64_t *bar = reinterpret_cast<uint64_t *>(sm + OFF_BAR);
+    uint32_t *tslot = reinterpret_cast<uint32_t *>(sm + OFF_FLAG);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + OFF_FLAG + 4);
+    uint32_t tcols = 32;
+    while (tcols < 2u * (uint32_t)N) tcols <<= 1;
+
+    if (threadIdx.x == 0) {
+        asm volatile("prefetch.tensormap [%0];" ::"l"(&p.tm_kbar) : "memory");
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&bar[BAR_FULL + s], 1);
+            mbar_init(&bar[BAR_EMPTY + s], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&bar[BAR_TFULL + i], 1);
+            mbar_init(&bar[BAR_TEMPTY + i], 128);
+        }
+        mbar_init(&bar[BAR_Q], 128);
+        *abort_flag = 0;
+    }
+    if (warp == 5) {
+        tmem_alloc(tslot, tcols);
+        tmem_relinquish();
+    }
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    const uint32_t tmem = *tslot;
+
+    if (warp == 4) {
+        // ================================================================ producer
+        if (lane == 0) {
+            int issued = 0;
+            bool ok = true;
+            for (int it = 0; it < nt; ++it) {
+                const int s = it % kStages;
+                if (it >= kStages && !(ok = wait_abort(&bar[BAR_EMPTY + s], (uint32_t)((it / kStages) - 1) & 1, abort_flag)))
+                    break;
+                const uint32_t dst = smem_u32(sm + OFF_K + s * kTileBytes);
+                const int y = b * p.nb_max + (t0 + it) * 128;
+                mbar_expect_tx(&bar[BAR_FULL + s], kTileBytes);
+                tma_load_2d(dst, &p.tm_kbar, 0, y, &bar[BAR_FULL + s]);
+                tma_load_2d(dst + kHalf, &p.tm_kbar, 64, y, &bar[BAR_FULL + s]);
+                ++issued;
+            }
+            if (!ok)  // wait (bounded) for the copies still in flight
+                for (int it = max(0, issued - kStages); it < issued; ++it)
+                    mbar_wait(&bar[BAR_FULL + it % kStages], (uint32_t)(it / kStages) & 1, kWaitTries);
+        }
+        __syncwarp();
+    } else if (warp == 5) {
+        // ================================================================ MMA issuer
+        if (lane == 0) {
+            const uint32_t id = idesc_bf16(128, N);
+            const uint32_t qb = smem_u32(sm + OFF_Q);
+            const uint64_t b0 = desc_kmajor(qb, (uint32_t)N * 128, 0);
+            const uint32_t b_blk16 = ((uint32_t)N * 128) >> 4;
+            int issued = 0;
+            bool ok = wait_abort(&bar[BAR_Q], 0, abort_flag);
+            for (int it = 0; ok && it < nt; ++it) {
+                const int s = it % kStages, buf = it & 1;
+                if (!(ok = wait_abort(&bar[BAR_FULL + s], (uint32_t)(it / kStages) & 1, abort_flag))) break;
+                if (it >= 2 && !(ok = wait_abort(&bar[BAR_TEMPTY + buf], (uint32_t)((it >> 1) - 1) & 1, abort_flag))) break;
+                fence_after_sync();
+                const uint64_t a0 = desc_kmajor(smem_u32(sm + OFF_K + s * kTileBytes), kHalf, 0);
+#pragma unroll
+                for (int st = 0; st < kD / 16; ++st) {
+                    const uint32_t da = (uint32_t)(st >> 2) * (kHalf >> 4) + (uint32_t)(st & 3) * 2;
+                    const uint32_t db = (uint32_t)(st >> 2) * b_blk16 + (uint32_t)(st & 3) * 2;
+                    mma_bf16(tmem + (uint32_t)(buf * N), a0 + da, b0 + db, id, st > 0 ? 1u : 0u);
+                }
+                mma_commit(&bar[BAR_EMPTY + s]);
+                mma_commit(&bar[BAR_TFULL + buf]);
+                ++issued;
+            }
+            // the tensor memory is released only after the last issued MMAs have completed
+            if (issued) mbar_wait(&bar[BAR_TFULL + ((issued - 1) & 1)], (uint32_t)((issued - 1) >> 1) & 1, kWaitTries);
+        }
+        __syncwarp();
+    } else {
+        // ================================================================ epilogue
+        // 1. the CTA's query heads, normalised and rotated, as the MMA's B operand (K-major,
+        //    128-byte swizzle: row n = 4 query + head, two 64-dim column blocks)
+        {
+            double f[4];
+            const double l2t = log2((double)p.theta);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) f[e] = inv_freq(4 * (lane & 7) + e, l2t);
+            const float4 w = __ldg(reinterpret_cast<const float4 *>(p.w) + lane);
+            const int d = 4 * lane;
+            for (int qi = warp; qi < p.qt; qi += 4) {
+                const bool live = qi < nq;
+                float c[4] = {1.f, 1.f, 1.f, 1.f}, s[4] = {0.f, 0.f, 0.f, 0.f};
+                if (live && lane < 16) {
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) rope_cs(pos0 + q0 + qi, f[e], c[e], s[e]);
+                }
+                const uint2 *src = reinterpret_cast<const uint2 *>(p.q + ((int64_t)b * p.Qn + q0 + qi) * kHeads * kD) + lane;
+#pragma unroll
+                for (int h = 0; h < kHeads; ++h) {
+                    const int n = kHeads * qi + h;
+                    float x[4] = {0.f, 0.f, 0.f, 0.f};
+                    if (live) {
+                        unpack4(__ldg(src + h * (kD / 4)), x);
+                        norm_rope_row(x, w, p.eps, c, s, lane);
+                    }
+                    const uint32_t off = (uint32_t)(d >> 6) * (uint32_t)(N * 128) + (uint32_t)n * 128 +
+                                         ((((uint32_t)(d & 63) >> 3) ^ (uint32_t)(n & 7)) << 4) + ((uint32_t)(d & 7) << 1);
+                    *reinterpret_cast<uint2 *>(sm + OFF_Q + off) = pack4(x);
+                }
+            }
+            fence_smem_to_async();
+            arrive(&bar[BAR_Q]);
+        }
+        // 2. per key tile: sum over heads of ReLU(dot), one fp32 score per (query, block)
+        const uint32_t lrow = (uint32_t)(32 * warp) << 16;    // this warp's TMEM lanes
+        bool ok = true;
+        for (int it = 0; it < nt; ++it) {
+            const int buf = it & 1;
+            const int blk = (t0 + it) * 128 + 32 * warp + lane;
+            const bool in = blk < p.nb_max;
+            float *dst = p.scores + ((int64_t)b * p.Qn + q0) * p.nb_max + blk;
+            if (ok) ok = wait_abort(&bar[BAR_TFULL + buf], (uint32_t)(it >> 1) & 1, abort_flag);
+            if (!ok) {   // leave NaN where this tile's scores belong
+                if (in)
+                    for (int qi = 0; qi < nq; ++qi) dst[(int64_t)qi * p.nb_max] = __int_as_float(0x7fc00000);
+                continue;
+            }
+            fence_after_sync();
+            for (int c = 0; c < N / 16; ++c) {
+                float v[16];
+                tmem_ld16(tmem + lrow + (uint32_t)(buf * N + 16 * c), v);
+                tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const int qi = 4 * c + j;
+                    float sc = 0.f;
+#pragma unroll
+                    for (int h = 0; h < kHeads; ++h) {
+                        const float t = v[kHeads * j + h];
+                        sc += t > 0.f ? t : 0.f;
+                    }
+                    if (in && qi < nq) __stcs(dst + (int64_t)qi * p.nb_max, sc);
+                }
+            }
+            fence_before_sync();
+            arrive(&bar[BAR_TEMPTY + buf]);
+        }
+    }
+
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    if (warp == 5) tmem_dealloc(tmem, tcols);
+}
+
+// ------------------------------------------------------------------ top-512 selection
+constexpr int kTopThr = 512;
+constexpr int kTopWarps = kTopThr / 32;
+constexpr int kHist = 2048;
+constexpr int kTopSmemKeys = 40960;                // rows up to this long are staged in shared memory
+
+struct TopkParams {
+    const float *scores;
+    const int32_t *qpos, *n_blocks;
+    int32_t *blocks, *tokens;
+    int B, Qn, nb_max, smem_keys;
+};
+
+// exclusive prefix sum over the CTA's 512 threads (sw: 16 ints of scratch)
+__device__ __forceinline__ int excl_scan512(int x, int *sw) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int v = x;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, v, o);
+        if (lane >= o) v += y;
+    }
+    if (lane == 31) sw[warp] = v;
+    __syncthreads();
+    if (warp == 0) {
+        int t = lane < kTopWarps ? sw[lane] : 0;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, t, o);
+            if (lane >= o) t += y;
+        }
+        if (lane < kTopWarps) sw[lane] = t;
+    }
+    __syncthreads();
+    const int before = (warp ? sw[warp - 1] : 0) + v - x;
+    __syncthreads();
+    return before;
+}
+
+__global__ void __launch_bounds__(kTopThr) qsa_topk_kernel(const __grid_constant__ TopkParams p) {
+    extern __shared__ __align__(16) unsigned char smt[];
+    int *hist = reinterpret_cast<int *>(smt);                          // [kHist]
+    int *sw = hist + kHist;                                            // [16] scan scratch
+    int *sel = sw + 32;                                                // digit, count above
+    int *wcnt = sel + 32;                                              // [16][2] per-warp counts
+    uint32_t *skeys = reinterpret_cast<uint32_t *>(smt + (kHist + 128) * 4);
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int64_t row = blockIdx.x;
+    const int b = (int)(row / p.Qn);
+    const int64_t pos = (int64_t)p.qpos[b] + row % p.Qn;
+    const int64_t cap = max(0, min(p.n_blocks[b], p.nb_max));
+    const int nvis = (int)n_cand(pos, cap);
+    int32_t *ob = p.blocks + row * kKB;
+    int32_t *ot = p.tokens ? p.tokens + row * kTok : nullptr;
+    const int64_t tail0 = pos < 0 ? 0 : ((pos + 1) >> 2) * kR;
+    const int tail_n = pos < 0 ? 0 : (int)(pos - tail0 + 1);
+    const int count = min(nvis, kKB);
+    // tokens after the selected blocks' 4 count: the tail, then -1
+    auto tail_fill = [&]() {
+        if (!ot) return;
+        for (int t = kR * count + tid; t < kTok; t += kTopThr)
+            ot[t] = t - kR * count < tail_n ? (int32_t)(tail0 + (t - kR * count)) : -1;
+    };
+    if (nvis <= kKB) {   // every candidate is selected
+        for (int t = tid; t < kKB; t += kTopThr) ob[t] = t < nvis ? t : -1;
+        if (ot)
+            for (int t = tid; t < kR * count; t += kTopThr) ot[t] = t;
+        tail_fill();
+        return;
+    }
+
+    const uint32_t *grow = reinterpret_cast<const uint32_t *>(p.scores + row * p.nb_max);
+    const uint32_t *keys = grow;
+    if (nvis <= p.smem_keys) {
+        for (int e = tid; e < nvis; e += kTopThr) skeys[e] = __ldcs(grow + e);
+        keys = skeys;
+    }
+    // radix select of the kKB-th largest key (scores are >= +0, so their bit patterns order
+    // like the values; NaN or a set sign bit marks a failed score computation)
+    uint32_t hi = 0;
+    int kk = kKB;
+    bool bad = false;
+#pragma unroll 1
+    for (int pass = 0; pass < 3; ++pass) {
+        const int shift = pass == 0 ? 20 : pass == 1 ? 10 : 0;
+        const int width = pass == 0 ? 11 : 10;
+        const int nbins = 1 << width;
+        for (int i = tid; i < nbins; i += kTopThr) hist[i] = 0;
+        __syncthreads();
+        for (int base = warp * 32; base < nvis; base += kTopThr) {
+            const int e = base + lane;
+            uint32_t dg = 0xFFFFFFFFu;
+            if (e < nvis) {
+                const uint32_t k = keys[e];
+                if (pass == 0 && k > 0x7F800000u) bad = true;
+                if ((k >> (shift + width)) == hi) dg = (k >> shift) & (uint32_t)(nbins - 1);
+            }
+            const uint32_t m = __match_any_sync(0xffffffffu, dg);
+            if (dg != 0xFFFFFFFFu && lane == __ffs(m) - 1) atomicAdd(&hist[dg], __popc(m));
+        }
+        if (pass == 0 && __syncthreads_or(bad)) {
+            for (int t = tid; t < kKB; t += kTopThr) ob[t] = -2;
+            if (ot)
+                for (int t = tid; t < kTok; t += kTopThr) ot[t] = -2;
+            return;
+        }
+        __syncthreads();
+        // bins from the top: thread t holds bins nbins-1-4t .. nbins-4-4t
+        int loc[4], sum = 0;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int bin = nbins - 1 - 4 * tid - j;
+            loc[j] = bin >= 0 ? hist[bin] : 0;
+            sum += loc[j];
+        }
+        const int before = excl_scan512(sum, sw);
+        if (before < kk && kk <= before + sum) {
+            int cum = before;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                if (cum + loc[j] >= kk) {
+                    sel[0] = nbins - 1 - 4 * tid - j;
+                    sel[1] = cum;
+                    break;
+                }
+                cum += loc[j];
+            }
+        }
+        __syncthreads();
+        hi = (hi << width) | (uint32_t)sel[0];
+        kk -= sel[1];
+        __syncthreads();
+    }
+    const uint32_t thr = hi;   // the kKB-th largest key; kk of the keys equal to it are taken
+
+    // ordered pass: warp w covers [w Ew, (w+1) Ew); first its counts, then the writes
+    const int ew = ((nvis + kTopWarps - 1) / kTopWarps + 31) & ~31;
+    const int e0 = warp * ew, e1 = min(nvis, e0 + ew);
+    int gt = 0, eq = 0;
+    for (int base = e0; base < e1; base += 32) {
+        const int e = base + lane;
+        const uint32_t k = e < e1 ? keys[e] : 0u;
+        gt += __popc(__ballot_sync(0xffffffffu, e < e1 && k > thr));
+        eq += __popc(__ballot_sync(0xffffffffu, e < e1 && k == thr));
+    }
+    if (lane == 0) {
+        wcnt[2 * warp] = gt;
+        wcnt[2 * warp + 1] = eq;
+    }
+    __syncthreads();
+    int gt_run = 0, eq_run = 0;
+    for (int w = 0; w < warp; ++w) {
+        gt_run += wcnt[2 * w];
+        eq_run += wcnt[2 * w + 1];
+    }
+    const uint32_t lt = (1u << lane) - 1u;
+    for (int base = e0; base < e1; base += 32) {
+        const int e = base + lane;
+        const uint32_t k = e < e1 ? keys[e] : 0u;
+        const bool g = e < e1 && k > thr, q = e < e1 && k == thr;
+        const uint32_t gb = __ballot_sync(0xffffffffu, g), qb = __ballot_sync(0xffffffffu, q);
+        const bool take = g || (q && eq_run + __popc(qb & lt) < kk);
+        const uint32_t sb = __ballot_sync(0xffffffffu, take);
+        if (take) {
+            const int o = gt_run + min(eq_run, kk) + __popc(sb & lt);
+            ob[o] = e;
+            if (ot) {
+                int4 t4 = make_int4(kR * e, kR * e + 1, kR * e + 2, kR * e + 3);
+                ot[kR * o] = t4.x;
+                ot[kR * o + 1] = t4.y;
+                ot[kR * o + 2] = t4.z;
+                ot[kR * o + 3] = t4.w;
+            }
+        }
+        gt_run += __popc(gb);
+        eq_run += __popc(qb);
+    }
+    tail_fill();
+}
+
+}  // namespace qsa
+
+// ------------------------------------------------------------------ launchers
+cudaError_t launch_qsa_block_keys(const void *k, const float *w, const int32_t *kpos, int B, int Tn,
+                                  float eps, float theta, void *kbar, int nb_max, cudaStream_t s) {
+    qsa::KeyParams p{static_cast<const __nv_bfloat16 *>(k), w, kpos, static_cast<__nv_bfloat16 *>(kbar),
+                     B, Tn, nb_max, eps, theta};
+    const int64_t warps = (int64_t)B * (Tn / qsa::kR);
+    if (warps == 0) return cudaSuccess;
+    TraceLaunch tl(s, "qsa_block_keys");
+    qsa::qsa_block_keys_kernel<<<(unsigned)((warps + 7) / 8), 256, 0, s>>>(p);
+    return cudaGetLastError();
+}
+
+// queries per scores CTA: the smallest multiple of 4 that covers Qn, at most 64
+static int score_qt(int Qn) { return std::min(qsa::kMaxQT, (Qn + 3) & ~3); }
+
+cudaError_t launch_qsa_scores(const void *q, const float *w, const int32_t *qpos, const void *kbar,
+                              const int32_t *n_blocks, int B, int Qn, int nb_max, float eps, float theta,
+                              float *scores, cudaStream_t s) {
+    if (B == 0 || Qn == 0) return cudaSuccess;
+    qsa::ScoreParams p{};
+    if (!encode_2d(&p.tm_kbar, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, kbar, qsa::kD, (int64_t)B * nb_max,
+                   qsa::kD * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B))
+        return cudaErrorInvalidValue;
+    p.q = static_cast<const __nv_bfloat16 *>(q);
+    p.w = w;
+    p.qpos = qpos;
+    p.n_blocks = n_blocks;
+    p.scores = scores;
+    p.B = B;
+    p.Qn = Qn;
+    p.nb_max = nb_max;
+    p.qt = score_qt(Qn);
+    p.eps = eps;
+    p.theta = theta;
+    const int nqt = (Qn + p.qt - 1) / p.qt;
+    // split each query tile's block range so that the CTAs fill whole waves of 148 SMs
+    // (one CTA per SM): pick the split with the fewest tile-times, counting ~4 tile-times
+    // of query-head preparation per CTA
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int64_t tiles = (nb_max + 127) / 128;
+    const int64_t ctas1 = (int64_t)nqt * B;
+    int best = 1;
+    double best_cost = 1e300;
+    for (int ns = 1; ns <= 16 && ns <= tiles; ++ns) {
+        const double waves = std::ceil((double)(ctas1 * ns) / sms);
+        const double cost = waves * (std::ceil((double)tiles / ns) + 4.0);
+        if (cost < best_cost - 1e-9) {
+            best_cost = cost;
+            best = ns;
+        }
+    }
+    p.n_split = best;
+    auto kern = qsa::qsa_scores_kernel;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)qsa::kScoreSmem);
+    if (e != cudaSuccess) return e;
+    TraceLaunch tl(s, "qsa_scores");
+    kern<<<dim3((unsigned)nqt, (unsigned)B, (unsigned)p.n_split), qsa::kScoreThr, qsa::kScoreSmem, s>>>(p);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_qsa_topk(const float *scores, const int32_t *qpos, const int32_t *n_blocks, int B, int Qn,
+                            int nb_max, int32_t *blocks, int32_t *tokens, cudaStream_t s) {
+    if (B == 0 || Qn == 0) return cudaSuccess;
+    qsa::TopkParams p{scores, qpos, n_blocks, blocks, tokens, B, Qn, nb_max,
+                      std::min(nb_max, qsa::kTopSmemKeys)};
+    const size_t smem = (size_t)(qsa::kHist + 128) * 4 + (size_t)p.smem_keys * 4;
+    auto kern = qsa::qsa_topk_kernel;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    TraceLaunch tl(s, "qsa_topk");
+    kern<<<(unsigned)((int64_t)B * Qn), qsa::kTopThr, smem, s>>>(p);
+    return cudaGetLastError();
+}
+
+}  // namespace gdn

@@ -186,6 +186,65 @@ def test_output_gate_no_tokens_is_noop():
     assert _gate(n=0, y=None, out=None) == 0
 
 
+def _qkeys(**over):
+    A = 1 << 20
+    a = dict(k=A, w=2 * A, kpos=3 * A, B=2, Tn=8, eps=1e-6, theta=1e4, kbar=4 * A, nb=16, stream=None)
+    a.update(over)
+    return _native.lib().gdn_qsa_block_keys(a["k"], a["w"], a["kpos"], a["B"], a["Tn"], a["eps"], a["theta"],
+                                            a["kbar"], a["nb"], a["stream"])
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(k=None), 1), (dict(w=None), 1), (dict(kpos=None), 1), (dict(kbar=None), 1), (dict(Tn=6), 1),
+    (dict(B=-1), 1), (dict(nb=0), 1), (dict(eps=-1.0), 1), (dict(theta=0.0), 1), (dict(theta=float("nan")), 1),
+    (dict(k=(1 << 20) + 4), 1), (dict(B=70000), 1), (dict(B=4, nb=1 << 29), 1),
+])
+def test_qsa_block_keys_rejects_before_launch(over, code):
+    assert _qkeys(**over) == code
+
+
+def test_qsa_block_keys_empty_is_noop():
+    assert _qkeys(B=0, k=None, kbar=None) == 0
+    assert _qkeys(Tn=0, k=None, kbar=None) == 0
+
+
+def _qsel(fn="gdn_qsa_select", **over):
+    A = 1 << 20
+    a = dict(q=A, w=2 * A, qpos=3 * A, kbar=4 * A, nblk=5 * A, B=2, Qn=3, nb=100, eps=1e-6, theta=1e4,
+             blocks=6 * A, tokens=None, ws=8 * A, wsb=2560, stream=None)
+    a.update(over)
+    L = _native.lib()
+    head = (a["q"], a["w"], a["qpos"], a["kbar"], a["nblk"], a["B"], a["Qn"], a["nb"], a["eps"], a["theta"])
+    if fn == "gdn_qsa_block_scores":
+        return L.gdn_qsa_block_scores(*head, a["blocks"], a["stream"])
+    return L.gdn_qsa_select(*head, a["blocks"], a["tokens"], a["ws"], a["wsb"], a["stream"])
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(q=None), 1), (dict(w=None), 1), (dict(qpos=None), 1), (dict(kbar=None), 1), (dict(nblk=None), 1),
+    (dict(blocks=None), 1), (dict(Qn=-1), 1), (dict(nb=0), 1), (dict(eps=float("inf")), 1),
+    (dict(theta=-1.0), 1), (dict(tokens=(7 << 20) + 4), 1), (dict(ws=None), 3), (dict(wsb=2559), 3),
+    (dict(ws=(8 << 20) + 16), 3),
+])
+def test_qsa_select_rejects_before_launch(over, code):
+    assert _qsel(**over) == code
+
+
+@pytest.mark.parametrize("over,code", [(dict(q=None), 1), (dict(blocks=None), 1), (dict(B=-2), 1),
+                                       (dict(blocks=(6 << 20) + 4), 1)])
+def test_qsa_block_scores_rejects_before_launch(over, code):
+    assert _qsel("gdn_qsa_block_scores", **over) == code
+
+
+def test_qsa_select_workspace_and_empty():
+    n = ctypes.c_size_t(0)
+    assert _native.lib().gdn_qsa_select_workspace_size(2, 3, 100, ctypes.byref(n)) == 0
+    assert n.value == 2560                      # 2 x 3 x 100 fp32 scores, rounded to 256 bytes
+    assert _native.lib().gdn_qsa_select_workspace_size(2, 3, 0, ctypes.byref(n)) == 1
+    assert _qsel(Qn=0, q=None, blocks=None, ws=None) == 0
+    assert _qsel("gdn_qsa_block_scores", B=0, q=None, blocks=None) == 0
+
+
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(_native, "LIB_PATH", str(tmp_path / "missing.so"))
     monkeypatch.setattr(_native, "_lib", None)
