@@ -717,6 +717,7 @@ def main():
     ap.add_argument("--decode-steps", type=int, default=1024)
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-qsa", action="store_true")
+    ap.add_argument("--qsa-only", action="store_true", help="only the QSA indexer legs (profiling)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-baseline-s", type=float, default=15.0)
     ap.add_argument("--ref-step-s", type=float, default=5.0)
@@ -730,6 +731,12 @@ def main():
     import linear_attention_recurrence_05_b200 as gdn
     dist = Dist(torch).init()
     peaks, peak_src = load_peaks()
+    if args.qsa_only:
+        qsa = {wl: bench_qsa(args, dist, torch, gdn, peaks, peak_src, wl) for wl in ("prefill", "decode")}
+        if dist.rank == 0:
+            print(json.dumps({"metric": "QSA indexer query tokens/s", "qsa": qsa, "peaks": peak_src}), flush=True)
+        dist.close()
+        return
     pre = bench_prefill(args, dist, torch, gdn, peaks)
     roof = prefill_roofline(pre, peaks, peak_src)
     dec = None if args.no_decode else bench_decode(args, dist, torch, gdn, peaks, peak_src)

@@ -409,6 +409,8 @@ gdn_status gdn_output_gate(const gdn_config *cfg, gdn_dtype y_dtype, gdn_dtype z
 static bool qsa_scalars_ok(float eps, float theta) {
     return std::isfinite(eps) && eps >= 0.f && std::isfinite(theta) && theta > 0.f;
 }
+// the select workspace keeps each query's scores on a 128-byte aligned row
+static int64_t qsa_row_stride(int nb_max) { return ((int64_t)nb_max + 31) & ~(int64_t)31; }
 static bool qsa_sizes_ok(int B, int n, int nb_max) {
     return B >= 0 && n >= 0 && nb_max >= 1 && B <= 65535 && nb_max < (1 << 29) &&
            (int64_t)B * nb_max < ((int64_t)1 << 31) - 256;
@@ -448,7 +450,7 @@ gdn_status gdn_qsa_block_scores(const void *q, const float *w_q, const int32_t *
     if (!scores || !aligned(scores, 16)) return GDN_ERR_INVALID_ARG;
     st = check_device();
     if (st != GDN_OK) return st;
-    cudaError_t e = launch_qsa_scores(q, w_q, qpos, kbar, n_blocks, B, Qn, nb_max, eps, theta, scores, stream);
+    cudaError_t e = launch_qsa_scores(q, w_q, qpos, kbar, n_blocks, B, Qn, nb_max, eps, theta, scores, nb_max, stream);
     if (e != cudaSuccess) return cuda_fail(e);
     return GDN_OK;
 }
@@ -456,7 +458,7 @@ gdn_status gdn_qsa_block_scores(const void *q, const float *w_q, const int32_t *
 gdn_status gdn_qsa_select_workspace_size(int B, int Qn, int nb_max, size_t *bytes) {
     if (!bytes) return GDN_ERR_INVALID_ARG;
     if (!qsa_sizes_ok(B, Qn, nb_max)) return GDN_ERR_INVALID_ARG;
-    *bytes = (((size_t)B * Qn * nb_max * 4) + 255) & ~(size_t)255;
+    *bytes = (((size_t)B * Qn * qsa_row_stride(nb_max) * 4) + 255) & ~(size_t)255;
     return GDN_OK;
 }
 
@@ -474,9 +476,10 @@ gdn_status gdn_qsa_select(const void *q, const float *w_q, const int32_t *qpos, 
     st = check_device();
     if (st != GDN_OK) return st;
     float *scores = static_cast<float *>(workspace);
-    cudaError_t e = launch_qsa_scores(q, w_q, qpos, kbar, n_blocks, B, Qn, nb_max, eps, theta, scores, stream);
+    const int64_t ld = qsa_row_stride(nb_max);
+    cudaError_t e = launch_qsa_scores(q, w_q, qpos, kbar, n_blocks, B, Qn, nb_max, eps, theta, scores, ld, stream);
     if (e != cudaSuccess) return cuda_fail(e);
-    e = launch_qsa_topk(scores, qpos, n_blocks, B, Qn, nb_max, blocks, tokens, stream);
+    e = launch_qsa_topk(scores, ld, qpos, n_blocks, B, Qn, nb_max, blocks, tokens, stream);
     if (e != cudaSuccess) return cuda_fail(e);
     return GDN_OK;
 }

@@ -111,9 +111,10 @@ cudaError_t launch_qsa_block_keys(const void *k, const float *w, const int32_t *
                                   float eps, float theta, void *kbar, int nb_max, cudaStream_t s);
 cudaError_t launch_qsa_scores(const void *q, const float *w, const int32_t *qpos, const void *kbar,
                               const int32_t *n_blocks, int B, int Qn, int nb_max, float eps, float theta,
-                              float *scores, cudaStream_t s);
-cudaError_t launch_qsa_topk(const float *scores, const int32_t *qpos, const int32_t *n_blocks, int B, int Qn,
-                            int nb_max, int32_t *blocks, int32_t *tokens, cudaStream_t s);
+                              float *scores, int64_t ld, cudaStream_t s);
+// scores rows of stride ld: a multiple of 4 floats on a 16-byte aligned base
+cudaError_t launch_qsa_topk(const float *scores, int64_t ld, const int32_t *qpos, const int32_t *n_blocks, int B,
+                            int Qn, int nb_max, int32_t *blocks, int32_t *tokens, cudaStream_t s);
 
 // launchers: return the cudaError_t of the launch
 cudaError_t launch_seq_table(const int32_t *cu_in, int n_seqs, int64_t T, int32_t *cu,

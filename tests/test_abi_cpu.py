@@ -211,7 +211,7 @@ def test_qsa_block_keys_empty_is_noop():
 def _qsel(fn="gdn_qsa_select", **over):
     A = 1 << 20
     a = dict(q=A, w=2 * A, qpos=3 * A, kbar=4 * A, nblk=5 * A, B=2, Qn=3, nb=100, eps=1e-6, theta=1e4,
-             blocks=6 * A, tokens=None, ws=8 * A, wsb=2560, stream=None)
+             blocks=6 * A, tokens=None, ws=8 * A, wsb=3072, stream=None)
     a.update(over)
     L = _native.lib()
     head = (a["q"], a["w"], a["qpos"], a["kbar"], a["nblk"], a["B"], a["Qn"], a["nb"], a["eps"], a["theta"])
@@ -223,7 +223,7 @@ def _qsel(fn="gdn_qsa_select", **over):
 @pytest.mark.parametrize("over,code", [
     (dict(q=None), 1), (dict(w=None), 1), (dict(qpos=None), 1), (dict(kbar=None), 1), (dict(nblk=None), 1),
     (dict(blocks=None), 1), (dict(Qn=-1), 1), (dict(nb=0), 1), (dict(eps=float("inf")), 1),
-    (dict(theta=-1.0), 1), (dict(tokens=(7 << 20) + 4), 1), (dict(ws=None), 3), (dict(wsb=2559), 3),
+    (dict(theta=-1.0), 1), (dict(tokens=(7 << 20) + 4), 1), (dict(ws=None), 3), (dict(wsb=3071), 3),
     (dict(ws=(8 << 20) + 16), 3),
 ])
 def test_qsa_select_rejects_before_launch(over, code):
@@ -239,7 +239,7 @@ def test_qsa_block_scores_rejects_before_launch(over, code):
 def test_qsa_select_workspace_and_empty():
     n = ctypes.c_size_t(0)
     assert _native.lib().gdn_qsa_select_workspace_size(2, 3, 100, ctypes.byref(n)) == 0
-    assert n.value == 2560                      # 2 x 3 x 100 fp32 scores, rounded to 256 bytes
+    assert n.value == 3072                      # 2 x 3 rows of 100 fp32 scores, each padded to 128
     assert _native.lib().gdn_qsa_select_workspace_size(2, 3, 0, ctypes.byref(n)) == 1
     assert _qsel(Qn=0, q=None, blocks=None, ws=None) == 0
     assert _qsel("gdn_qsa_block_scores", B=0, q=None, blocks=None) == 0

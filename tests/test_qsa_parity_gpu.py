@@ -195,11 +195,13 @@ def test_select(name):
     assert np.mean(overlaps) >= 0.99 and min(overlaps) >= 0.97, (np.mean(overlaps), min(overlaps))
 
 
-def test_select_ties_take_lower_blocks():
+@pytest.mark.parametrize("T", [4096, 32768])
+def test_select_ties_take_lower_blocks(T):
     """Identical block keys (same raw keys, rotated dims weighted 0) give identical scores:
-    the first 512 candidates are selected."""
+    the first 512 candidates are selected (T = 32768: more equal scores than the candidate
+    set holds, so the row takes the full-row path)."""
     torch, gdn = _mods()
-    B, T, Qn = 1, 4096, 3
+    B, Qn = 1, 3
     inp = gi.make_qsa_inputs(B, T, Qn, seed=55)
     inp.k[:] = inp.k[:, :1, :]                 # every token the same key row
     inp.w_k[:64] = 0.0                          # nothing left for the rotation to move
