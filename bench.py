@@ -55,7 +55,7 @@ TF32_PER_BF16 = 1.1 / 2.25   # nominal dense tf32 : bf16 tensor throughput on B2
 # kernels on this workload (profiles/prefill_tc_T8192_ncu.md: one chain launch of the step's
 # four chunk ranges, 2048 tokens; profiles/decode_B256_ncu.md); None while a kernel has
 # changed since its capture
-NCU_TRAFFIC_BYTES = {"prefill_tc": 159_953_408 + 33_269_504, "decode": 826_713_088 + 769_751_552}
+NCU_TRAFFIC_BYTES = {"prefill_tc": 159_957_760 + 31_570_176, "decode": 826_713_088 + 769_751_552}
 FP32_LANES_PER_SM = 128
 N_SM = 148
 

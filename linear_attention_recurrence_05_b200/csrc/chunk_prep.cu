@@ -187,6 +187,7 @@ __global__ void __launch_bounds__(kGroupThr * kMaxGroups, 2) chunk_prep_kernel(c
             float v[32];
             tmem_ld32(taddr(tm, 32 * q, 32 * h2), v);
             tmem_wait_ld();
+            tmem_regs_after_wait(v);
             if (factored) {   // uniform per CTA
 #pragma unroll
                 for (int e = 0; e < 32; e += 4) {

@@ -333,6 +333,8 @@ __global__ void __launch_bounds__(kThr, 1) prefill_tc_kernel(const __grid_consta
             tmem_ld32(tm + lrow + src, v0);
             tmem_ld32(tm + lrow + src + 32, v1);
             tmem_wait_ld();
+            tmem_regs_after_wait(v0);
+            tmem_regs_after_wait(v1);
 #pragma unroll
             for (int i = 0; i < 32; i += 4) {
                 const float4 a = *reinterpret_cast<const float4 *>(f + i);
@@ -366,6 +368,7 @@ __global__ void __launch_bounds__(kThr, 1) prefill_tc_kernel(const __grid_consta
                     float v[32];
                     tmem_ld32(tm + lrow + T_S + d0, v);
                     tmem_wait_ld();
+                    tmem_regs_after_wait(v);
 #pragma unroll
                     for (int i = 0; i < 32; ++i) v[i] *= gc;
                     tmem_st32(tm + lrow + T_S + d0, v);
@@ -389,6 +392,7 @@ __global__ void __launch_bounds__(kThr, 1) prefill_tc_kernel(const __grid_consta
                     float v[32];
                     tmem_ld32(tm + lrow + T_Y + 32 * h2, v);
                     tmem_wait_ld();
+                    tmem_regs_after_wait(v);
                     if (leader) bulk_wait_read1();
                     bar_sync(kBarEpi, 128);
 #pragma unroll
@@ -412,6 +416,7 @@ __global__ void __launch_bounds__(kThr, 1) prefill_tc_kernel(const __grid_consta
                     float v[32];
                     tmem_ld32(tm + lrow + T_Y + 32 * h2, v);
                     tmem_wait_ld();
+                    tmem_regs_after_wait(v);
 #pragma unroll
                     for (int blk = 0; blk < 8; ++blk) {
                         float a[4] = {v[4 * blk], v[4 * blk + 1], v[4 * blk + 2], v[4 * blk + 3]};
@@ -448,6 +453,7 @@ __global__ void __launch_bounds__(kThr, 1) prefill_tc_kernel(const __grid_consta
                 float s[32];
                 tmem_ld32(tm + lrow + T_S + d0, s);
                 tmem_wait_ld();
+                tmem_regs_after_wait(s);
 #pragma unroll
                 for (int i = 0; i < 32; ++i)
                     dst[(int64_t)(d0 + i) * kHeadDim] = failed ? __int_as_float(0x7fc00000) : s[i];

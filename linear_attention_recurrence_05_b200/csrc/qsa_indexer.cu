@@ -143,9 +143,11 @@ enum { BAR_FULL = 0, BAR_EMPTY = kStages, BAR_TFULL = 2 * kStages, BAR_TEMPTY = 
        BAR_Q = 2 * kStages + 4, kNumBars };
 constexpr uint32_t OFF_FLAG = OFF_BAR + 8 * 16;    // TMEM base, abort flag
 constexpr uint32_t kScoreSmem = OFF_FLAG + 16;
-constexpr int kEpiWarps = 8;                       // two per TMEM lane quadrant
-constexpr int kLoadWarp = kEpiWarps, kMmaWarp = kEpiWarps + 1;
-constexpr int kScoreThr = 32 * (kEpiWarps + 2);    // epilogue warps, producer, MMA issuer
+// Warps: n_epi epilogue warps (4 per group of 16-column chunks, up to 4 groups: one warp
+// per TMEM lane quadrant in each), then the producer, then the MMA issuer; the launch picks
+// n_epi = 4 min(4, N / 16).
+constexpr int kMaxEpiWarps = 16;
+constexpr int kScoreThrMax = 32 * (kMaxEpiWarps + 2);
 constexpr int kMaxQT = 64;                         // queries per CTA (N = 4 x 64 = 256)
 
 struct ScoreParams {
@@ -173,9 +175,10 @@ __device__ __forceinline__ bool wait_abort(uint64_t *m, uint32_t par, volatile i
     return false;
 }
 
-__global__ void __launch_bounds__(kScoreThr, 1) qsa_scores_kernel(const __grid_constant__ ScoreParams p) {
+__global__ void __launch_bounds__(kScoreThrMax, 1) qsa_scores_kernel(const __grid_constant__ ScoreParams p) {
     extern __shared__ __align__(1024) unsigned char sm[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int n_epi = (int)(blockDim.x >> 5) - 2, kLoadWarp = n_epi, kMmaWarp = n_epi + 1;
     const int b = blockIdx.y, q0 = blockIdx.x * p.qt;
     const int nq = min(p.qt, p.Qn - q0);
     const int N = kHeads * p.qt;                               // MMA N: (query, head) rows
@@ -202,9 +205,9 @@ __global__ void __launch_bounds__(kScoreThr, 1) qsa_scores_kernel(const __grid_c
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&bar[BAR_TFULL + i], 1);
-            mbar_init(&bar[BAR_TEMPTY + i], 32 * kEpiWarps);
+            mbar_init(&bar[BAR_TEMPTY + i], 32 * n_epi);
         }
-        mbar_init(&bar[BAR_Q], 32 * kEpiWarps);
+        mbar_init(&bar[BAR_Q], 32 * n_epi);
         *abort_flag = 0;
     }
     if (warp == kMmaWarp) {
@@ -277,7 +280,7 @@ __global__ void __launch_bounds__(kScoreThr, 1) qsa_scores_kernel(const __grid_c
             for (int e = 0; e < 4; ++e) f[e] = inv_freq(4 * (lane & 7) + e, l2t);
             const float4 w = __ldg(reinterpret_cast<const float4 *>(p.w) + lane);
             const int d = 4 * lane;
-            for (int qi = warp; qi < p.qt; qi += kEpiWarps) {
+            for (int qi = warp; qi < p.qt; qi += n_epi) {
                 const bool live = qi < nq;
                 float c[4] = {1.f, 1.f, 1.f, 1.f}, s[4] = {0.f, 0.f, 0.f, 0.f};
                 if (live && lane < 16) {
@@ -302,12 +305,12 @@ __global__ void __launch_bounds__(kScoreThr, 1) qsa_scores_kernel(const __grid_c
             arrive(&bar[BAR_Q]);
         }
         // 2. per key tile: sum over heads of ReLU(dot), one fp32 score per (query, block).
-        //    Warp w reads TMEM lanes 32 (w % 4) .. (its 32 blocks) and one half of the
+        //    Warp w reads TMEM lanes 32 (w % 4) .. (its 32 blocks) and one quarter of the
         //    16-column chunks (4 queries each).
-        const int qd = warp & 3, hf = warp >> 2;
+        const int qd = warp & 3, part = warp >> 2;
         const uint32_t lrow = (uint32_t)(32 * qd) << 16;
-        const int nch = N / 16, half = (nch + 1) / 2;
-        const int c0 = hf * half, c1 = min(nch, c0 + half);
+        const int nch = N / 16, nparts = n_epi / 4, share = (nch + nparts - 1) / nparts;
+        const int c0 = min(nch, part * share), c1 = min(nch, c0 + share);
         bool ok = true;
         for (int it = 0; it < nt; ++it) {
             const int buf = it & 1;
@@ -322,16 +325,18 @@ __global__ void __launch_bounds__(kScoreThr, 1) qsa_scores_kernel(const __grid_c
             }
             fence_after_sync();
             float *dq = dst + (int64_t)(4 * c0) * p.ld;
-            // up to 4 loads of 16 columns (16 queries) in flight per wait
-            for (int c = c0; c < c1; c += 4) {
-                const int g = min(4, c1 - c);                // warp-uniform
-                float v[4][16];
+            // up to 2 loads of 16 columns (8 queries) in flight per wait
+            for (int c = c0; c < c1; c += 2) {
+                const int g = min(2, c1 - c);                // warp-uniform
+                float v[2][16];
 #pragma unroll
-                for (int u = 0; u < 4; ++u)
+                for (int u = 0; u < 2; ++u)
                     if (u < g) tmem_ld16(tmem + lrow + (uint32_t)(buf * N + 16 * (c + u)), v[u]);
                 tmem_wait_ld();
+                tmem_regs_after_wait(v[0]);
+                if (g > 1) tmem_regs_after_wait(v[1]);
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
+                for (int u = 0; u < 2; ++u) {
                     if (u >= g) break;
 #pragma unroll
                     for (int j = 0; j < 4; ++j) {
@@ -410,8 +415,8 @@ __device__ __forceinline__ int excl_scan512(int x, int *sw) {
 
 // The k-th largest of n keys (k <= n) by radix digits of 11, 10 and 10 bits of a
 // non-negative float's bit pattern; also returns how many keys equal to it rank within the
-// k (kk).  With passes = 2 the result is the lower edge of the k-th largest key's 21-bit
-// prefix (a lower bound; kk is then not meaningful).  Called by all threads of the CTA.
+// k (kk).  With passes < 3 the result is the lower edge of the k-th largest key's 11- or
+// 21-bit prefix (a lower bound; kk is then not meaningful).  Called by all threads of the CTA.
 __device__ uint32_t radix_select(const uint32_t *keys, int n, int k, int *hist, int *sw, int *sel, int &kk,
                                  int passes = 3) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -461,7 +466,7 @@ __device__ uint32_t radix_select(const uint32_t *keys, int n, int k, int *hist, 
         kk -= sel[1];
         __syncthreads();
     }
-    return passes == 3 ? hi : hi << 10;
+    return passes == 3 ? hi : passes == 2 ? hi << 10 : hi << 20;
 }
 
 __global__ void __launch_bounds__(kTopThr) qsa_topk_kernel(const __grid_constant__ TopkParams p) {
@@ -697,34 +702,38 @@ cudaError_t launch_qsa_scores(const void *q, const float *w, const int32_t *qpos
     p.B = B;
     p.Qn = Qn;
     p.nb_max = nb_max;
-    p.qt = score_qt(Qn);
     p.eps = eps;
     p.theta = theta;
-    const int nqt = (Qn + p.qt - 1) / p.qt;
-    // split each query tile's block range so that the CTAs fill whole waves of 148 SMs
-    // (one CTA per SM): pick the split with the fewest tile-times, counting ~4 tile-times
-    // of query-head preparation per CTA
+    // queries per CTA (a multiple of 4, at most 64) and the split of each query tile's block
+    // range: the fewest estimated time units over whole waves of one CTA per SM, a 128-block
+    // tile costing ~ qt + 16 units (the epilogue of its 4 qt columns and a fixed share) and a
+    // CTA's query-head preparation ~ 2 qt
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int64_t tiles = (nb_max + 127) / 128;
-    const int64_t ctas1 = (int64_t)nqt * B;
-    int best = 1;
     double best_cost = 1e300;
-    for (int ns = 1; ns <= 16 && ns <= tiles; ++ns) {
-        const double waves = std::ceil((double)(ctas1 * ns) / sms);
-        const double cost = waves * (std::ceil((double)tiles / ns) + 4.0);
-        if (cost < best_cost - 1e-9) {
-            best_cost = cost;
-            best = ns;
+    p.qt = 4;
+    p.n_split = 1;
+    for (int qt = score_qt(Qn); qt >= 4; qt -= 4) {
+        const int64_t ctas1 = (int64_t)((Qn + qt - 1) / qt) * B;
+        for (int ns = 1; ns <= 16 && ns <= tiles; ++ns) {
+            const double waves = std::ceil((double)(ctas1 * ns) / sms);
+            const double cost = waves * (std::ceil((double)tiles / ns) * (qt + 16.0) + 2.0 * qt);
+            if (cost < best_cost - 1e-9) {
+                best_cost = cost;
+                p.qt = qt;
+                p.n_split = ns;
+            }
         }
     }
-    p.n_split = best;
+    const int nqt = (Qn + p.qt - 1) / p.qt;
     auto kern = qsa::qsa_scores_kernel;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)qsa::kScoreSmem);
     if (e != cudaSuccess) return e;
+    const int n_epi = 4 * std::min(4, p.qt / 4);
     TraceLaunch tl(s, "qsa_scores");
-    kern<<<dim3((unsigned)nqt, (unsigned)B, (unsigned)p.n_split), qsa::kScoreThr, qsa::kScoreSmem, s>>>(p);
+    kern<<<dim3((unsigned)nqt, (unsigned)B, (unsigned)p.n_split), 32 * (n_epi + 2), qsa::kScoreSmem, s>>>(p);
     return cudaGetLastError();
 }
 
@@ -732,7 +741,7 @@ cudaError_t launch_qsa_topk(const float *scores, int64_t ld, const int32_t *qpos
                             int Qn, int nb_max, int32_t *blocks, int32_t *tokens, cudaStream_t s) {
     if (B == 0 || Qn == 0) return cudaSuccess;
     qsa::TopkParams p{scores, qpos, n_blocks, blocks, tokens, ld, B, Qn, nb_max};
-    const size_t smem = (size_t)(qsa::kHist + 128) * 4 + (size_t)qsa::kCandCap * 8 +
+    const size_t smem = (size_t)(qsa::kHist + 96) * 4 + (size_t)qsa::kCandCap * 8 +
                         (size_t)2 * ((nb_max + 31) / 32) * 4;
     auto kern = qsa::qsa_topk_kernel;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

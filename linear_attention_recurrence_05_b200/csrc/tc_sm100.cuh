@@ -224,6 +224,15 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const float (&v)[16]) 
 __device__ __forceinline__ void tmem_wait_ld() {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
+// Registers written by tcgen05.ld are valid only after tcgen05.wait::ld, but the wait
+// carries no register dependence, so the compiler may schedule arithmetic on them before
+// it.  Passing each register through an empty volatile asm placed after the wait (volatile
+// asm statements keep their order) makes every use depend on the wait.
+template <int N>
+__device__ __forceinline__ void tmem_regs_after_wait(float (&v)[N]) {
+#pragma unroll
+    for (int i = 0; i < N; ++i) asm volatile("" : "+f"(v[i])::"memory");
+}
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) {
     asm volatile(
         "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
