@@ -387,8 +387,10 @@ struct TopkParams {
     int B, Qn, nb_max;
 };
 
-// exclusive prefix sum over the CTA's 512 threads (sw: 16 ints of scratch)
-__device__ __forceinline__ int excl_scan512(int x, int *sw) {
+constexpr int kBinsPerThr = kHist / kTopThr;
+
+// exclusive prefix sum over the CTA's threads (sw: one int per warp of scratch)
+__device__ __forceinline__ int excl_scan_cta(int x, int *sw) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     int v = x;
 #pragma unroll
@@ -440,21 +442,21 @@ __device__ uint32_t radix_select(const uint32_t *keys, int n, int k, int *hist, 
             if (dg != 0xFFFFFFFFu && lane == __ffs(m) - 1) atomicAdd(&hist[dg], __popc(m));
         }
         __syncthreads();
-        // bins from the top: thread t holds bins nbins-1-4t .. nbins-4-4t
-        int loc[4], sum = 0;
+        // bins from the top: thread t holds bins nbins-1-kB t .. nbins-kB(t+1) (kB = kBinsPerThr)
+        int loc[kBinsPerThr], sum = 0;
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const int bin = nbins - 1 - 4 * tid - j;
+        for (int j = 0; j < kBinsPerThr; ++j) {
+            const int bin = nbins - 1 - kBinsPerThr * tid - j;
             loc[j] = bin >= 0 ? hist[bin] : 0;
             sum += loc[j];
         }
-        const int before = excl_scan512(sum, sw);
+        const int before = excl_scan_cta(sum, sw);
         if (before < kk && kk <= before + sum) {
             int cum = before;
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
+            for (int j = 0; j < kBinsPerThr; ++j) {
                 if (cum + loc[j] >= kk) {
-                    sel[0] = nbins - 1 - 4 * tid - j;
+                    sel[0] = nbins - 1 - kBinsPerThr * tid - j;
                     sel[1] = cum;
                     break;
                 }
@@ -597,7 +599,7 @@ __global__ void __launch_bounds__(kTopThr) qsa_topk_kernel(const __grid_constant
         const int w0 = min(W, tid * wpt), w1 = min(W, w0 + wpt);
         int eqc = 0;
         for (int w = w0; w < w1; ++w) eqc += __popc(bm_eq[w]);
-        int need = kk - excl_scan512(eqc, sw);      // equal keys this thread may still take
+        int need = kk - excl_scan_cta(eqc, sw);      // equal keys this thread may still take
         int selc = 0;
         for (int w = w0; w < w1; ++w) {
             uint32_t e = bm_eq[w], take = 0u;
@@ -618,7 +620,7 @@ __global__ void __launch_bounds__(kTopThr) qsa_topk_kernel(const __grid_constant
             bm_sel[w] = m;
             selc += __popc(m);
         }
-        int o = excl_scan512(selc, sw);
+        int o = excl_scan_cta(selc, sw);
         for (int w = w0; w < w1; ++w) {
             uint32_t m = bm_sel[w];
             while (m) {

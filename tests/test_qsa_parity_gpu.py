@@ -251,3 +251,57 @@ def test_select_full_size_sampled(wl):
             overlaps.append(_check_row(_host(blocks[b, j]), _host(tokens[b, j]), s, A, i,
                                        qi.n_complete(i, nb)))
     assert np.mean(overlaps) >= 0.99, overlaps
+
+
+@pytest.mark.parametrize("ties", [False, True])
+def test_select_long_rows(ties):
+    """Rows of more than 32768 candidate blocks (the CTA-per-query selection): random scores
+    take the sampled candidate path, identical scores the full-row path."""
+    torch, gdn = _mods()
+    B, T, Qn = 2, 160000, 3
+    nb = T // 4
+    inp = gi.make_qsa_inputs(B, T, Qn, seed=31 + int(ties))
+    if ties:
+        inp.k[:] = inp.k[:, :1, :]
+        inp.w_k[:64] = 0.0
+    kbar = _build_cache(torch, gdn, inp, nb)
+    qpos = [T - Qn, T - 50000]
+    blocks, tokens = gdn.qsa_select(to_dev(inp.q, "bf16"), to_dev(inp.w_q, "f32"), _i32(torch, qpos), kbar,
+                                    _i32(torch, [nb] * B), eps=EPS, theta=THETA, with_tokens=True)
+    bl, tk = _host(blocks), _host(tokens)
+    overlaps = []
+    for b in range(B):
+        s, A, pos = _oracle_scores(inp, b, qpos[b], Qn, nb, T)
+        for j in range(Qn):
+            nvis = qi.n_complete(pos[j], nb)
+            overlaps.append(_check_row(bl[b, j], tk[b, j], s[j], A[j], int(pos[j]), nvis))
+            if ties:
+                assert np.array_equal(bl[b, j], np.arange(512))
+    assert np.mean(overlaps) >= 0.99, overlaps
+
+
+@pytest.mark.parametrize("ties", [False, True])
+def test_select_many_queries(ties):
+    """2048 queries (the warp-per-query selection).  Random scores: positions 1900..3947 cross
+    the budget (<= 512 candidates, all candidates, then the sampled threshold) and every row is
+    checked; identical scores take the full-row path and give blocks 0..511."""
+    torch, gdn = _mods()
+    B, Qn = 1, 2048
+    T = 32768 if ties else 12000
+    q0 = T - Qn if ties else 1900
+    nb = T // 4
+    inp = gi.make_qsa_inputs(B, T, Qn, seed=57 + int(ties))
+    if ties:
+        inp.k[:] = inp.k[:, :1, :]
+        inp.w_k[:64] = 0.0
+    kbar = _build_cache(torch, gdn, inp, nb)
+    blocks, tokens = gdn.qsa_select(to_dev(inp.q, "bf16"), to_dev(inp.w_q, "f32"), _i32(torch, [q0]), kbar,
+                                    _i32(torch, [nb]), eps=EPS, theta=THETA, with_tokens=True)
+    bl, tk = _host(blocks), _host(tokens)
+    if ties:
+        assert np.array_equal(bl[0], np.broadcast_to(np.arange(512), (Qn, 512)))
+        return
+    s, A, pos = _oracle_scores(inp, 0, q0, Qn, nb, T)
+    overlaps = [_check_row(bl[0, j], tk[0, j], s[j], A[j], int(pos[j]), qi.n_complete(pos[j], nb))
+                for j in range(Qn)]
+    assert np.mean(overlaps) >= 0.99 and min(overlaps) >= 0.97, (np.mean(overlaps), min(overlaps))
