@@ -304,7 +304,8 @@ GDN_EXPORT gdn_status gdn_qsa_block_scores(const void *q, const float *w_q, cons
                                            int B, int Qn, int nb_max, float eps, float theta,
                                            float *scores, cudaStream_t stream);
 
-/* Bytes of workspace gdn_qsa_select needs (the scores of every query row).  Writes *bytes. */
+/* Bytes of workspace gdn_qsa_select needs: the fp32 scores of every query row, each row
+ * padded to a multiple of 32 floats (a 128-byte aligned start).  Writes *bytes. */
 GDN_EXPORT gdn_status gdn_qsa_select_workspace_size(int B, int Qn, int nb_max, size_t *bytes);
 
 /* B_i (and S_i when `tokens` is not NULL) of every query.  `workspace` (256-byte aligned,

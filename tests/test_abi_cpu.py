@@ -259,3 +259,19 @@ def test_product_does_not_import_oracle():
             if f.endswith((".py", ".cu", ".cuh", ".h", ".cpp")):
                 text = open(os.path.join(dirpath, f)).read()
                 assert "oracle" not in text.lower(), f
+
+
+def test_qsa_binding_rejects_host_tensors_and_dtypes():
+    import torch
+    import linear_attention_recurrence_05_b200 as gdn
+    k = torch.zeros((1, 8, 128), dtype=torch.bfloat16)
+    kbar = torch.zeros((1, 4, 128), dtype=torch.bfloat16)
+    w = torch.ones(128)
+    pos = torch.zeros(1, dtype=torch.int32)
+    with pytest.raises(TypeError):
+        gdn.qsa_block_keys(k, w, pos, kbar)                        # host tensors
+    q = torch.zeros((1, 2, 4, 128), dtype=torch.float32)
+    with pytest.raises(TypeError):
+        gdn.qsa_select(q, w, pos, kbar, pos)                        # fp32 queries
+    with pytest.raises(TypeError):
+        gdn.qsa_block_scores(q.to(torch.bfloat16), w, pos.long(), kbar, pos)   # int64 positions
