@@ -18,3 +18,14 @@ def oracle_lib():
     import oracle
     oracle.build()
     return oracle
+
+
+@pytest.fixture
+def repo_tmp(request):
+    """A fresh scratch directory inside the repository (tests/_build/, ignored by git),
+    removed after the test."""
+    import shutil
+    d = os.path.join(ROOT, "tests", "_build", f"{request.node.name}.{os.getpid()}".replace("/", "_"))
+    os.makedirs(d, exist_ok=True)
+    yield d
+    shutil.rmtree(d, ignore_errors=True)

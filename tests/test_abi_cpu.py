@@ -245,8 +245,8 @@ def test_qsa_select_workspace_and_empty():
     assert _qsel("gdn_qsa_block_scores", B=0, q=None, blocks=None) == 0
 
 
-def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
-    monkeypatch.setattr(_native, "LIB_PATH", str(tmp_path / "missing.so"))
+def test_binding_fails_loudly_without_library(monkeypatch):
+    monkeypatch.setattr(_native, "LIB_PATH", os.path.join(ROOT, "tests", "no-such-dir", "missing.so"))
     monkeypatch.setattr(_native, "_lib", None)
     with pytest.raises(RuntimeError, match="no fallback"):
         _native.lib()

@@ -75,15 +75,15 @@ def _rank_main(rank, world, port, bounds, out_dir):
 
 
 @pytest.mark.parametrize("bounds", [[0, 120, 230], [0, 40, 41 + 60, 230]])
-def test_ranks_equal_whole_sequence(tmp_path, bounds):
+def test_ranks_equal_whole_sequence(repo_tmp, bounds):
     """One span per gloo rank; the last rank's final state is the sequence's."""
     import torch.multiprocessing as mp
     world = len(bounds) - 1
-    mp.start_processes(_rank_main, args=(world, _free_port(), bounds, str(tmp_path)), nprocs=world,
+    mp.start_processes(_rank_main, args=(world, _free_port(), bounds, repo_tmp), nprocs=world,
                        start_method="spawn")
     inp, _, _ = _case(230, 51)
     yo, fo, _ = oracle.prefill(inp)
-    y = np.concatenate([np.load(tmp_path / f"y{r}.npy") for r in range(world)])
+    y = np.concatenate([np.load(os.path.join(repo_tmp, f"y{r}.npy")) for r in range(world)])
     np.testing.assert_allclose(y, yo, rtol=0, atol=1e-9 * np.abs(yo).max())
-    np.testing.assert_allclose(np.load(tmp_path / f"f{world - 1}.npy"), fo[0], rtol=0,
+    np.testing.assert_allclose(np.load(os.path.join(repo_tmp, f"f{world - 1}.npy")), fo[0], rtol=0,
                                atol=1e-9 * np.abs(fo).max())

@@ -29,11 +29,11 @@ def _rank_main(rank, world, port, out_dir):
 
 
 @pytest.mark.parametrize("world", [2, 3])
-def test_dist_max_over_ranks(tmp_path, world):
+def test_dist_max_over_ranks(repo_tmp, world):
     import torch.multiprocessing as mp
-    mp.start_processes(_rank_main, args=(world, _free_port(), str(tmp_path)), nprocs=world,
+    mp.start_processes(_rank_main, args=(world, _free_port(), repo_tmp), nprocs=world,
                        start_method="spawn")
     for r in range(world):
-        rank, w, m = np.load(tmp_path / f"r{r}.npy")
+        rank, w, m = np.load(os.path.join(repo_tmp, f"r{r}.npy"))
         assert (rank, w) == (r, world)
         assert m == 1.5 + (world - 1) * 2.25
