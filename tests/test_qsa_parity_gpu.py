@@ -305,3 +305,28 @@ def test_select_many_queries(ties):
     overlaps = [_check_row(bl[0, j], tk[0, j], s[j], A[j], int(pos[j]), qi.n_complete(pos[j], nb))
                 for j in range(Qn)]
     assert np.mean(overlaps) >= 0.99 and min(overlaps) >= 0.97, (np.mean(overlaps), min(overlaps))
+
+
+def test_select_degenerate_rows():
+    """Clamped device-side values: a row of negative query positions (no candidates, no tail),
+    a row whose cache holds no valid block (tail tokens only), and a normal row."""
+    torch, gdn = _mods()
+    B, T, Qn, nb_max = 3, 6400, 5, 1600
+    inp = gi.make_qsa_inputs(B, T, Qn, seed=77)
+    kbar = _build_cache(torch, gdn, inp, nb_max)
+    qpos, nblk = [-10, 10, 6000], [100, 0, 1600]
+    blocks, tokens = gdn.qsa_select(to_dev(inp.q, "bf16"), to_dev(inp.w_q, "f32"), _i32(torch, qpos), kbar,
+                                    _i32(torch, nblk), eps=EPS, theta=THETA, with_tokens=True)
+    bl, tk = _host(blocks), _host(tokens)
+    assert np.all(bl[0] == -1) and np.all(tk[0] == -1)
+    assert np.all(bl[1] == -1)
+    for j in range(Qn):
+        i = qpos[1] + j
+        want = np.full(qi.TOKEN_SLOTS, -1)
+        tail = np.arange(4 * ((i + 1) // 4), i + 1)
+        want[:len(tail)] = tail
+        assert np.array_equal(tk[1, j], want), j
+    s, A, pos = _oracle_scores(inp, 2, qpos[2], Qn, nblk[2], T)
+    ov = [_check_row(bl[2, j], tk[2, j], s[j], A[j], int(pos[j]), qi.n_complete(pos[j], nblk[2]))
+          for j in range(Qn)]
+    assert min(ov) >= 0.97
