@@ -368,3 +368,41 @@ def test_planted_mistakes(name, monkeypatch):
         except AssertionError:
             caught.append(pin.__name__)
     assert caught, f"no pin catches: {name}"
+
+
+# ----------------------------------------------------------------------------- properties
+from hypothesis import given, settings, strategies as st  # noqa: E402
+
+
+@settings(max_examples=200, deadline=None)
+@given(st.lists(st.sampled_from([0.0, 0.5, 1.0, 2.0, 3.5, float("-inf")]), min_size=0, max_size=12),
+       st.integers(min_value=1, max_value=6))
+def test_top_blocks_property(scores, k):
+    """Any row with ties: the selection holds min(k, finite) blocks, every selected score is
+    >= every unselected finite score, and among equal scores at the cut the lowest indices win."""
+    s = np.array(scores, dtype=np.float64)
+    got = [int(b) for b in qi.top_blocks(s, k) if b >= 0]
+    fin = [b for b in range(len(s)) if np.isfinite(s[b])]
+    assert len(got) == min(k, len(fin)) and got == sorted(got) and set(got) <= set(fin)
+    rest = [b for b in fin if b not in got]
+    if got and rest:
+        cut = min(s[b] for b in got)
+        assert cut >= max(s[b] for b in rest)
+        assert all(b > max(g for g in got if s[g] == cut) for b in rest if s[b] == cut)
+
+
+@settings(max_examples=200, deadline=None)
+@given(st.integers(min_value=0, max_value=400), st.integers(min_value=1, max_value=8))
+def test_token_set_property(i, k):
+    """For any position and budget: the token set is ascending, distinct, within 0..i, holds 4
+    tokens per selected complete block plus the (i + 1) mod 4 tail tokens, and with the
+    whole prefix selected it is exactly 0..i."""
+    nv = qi.n_complete(i)
+    blocks = np.full(k, -1)
+    m = min(k, nv)
+    blocks[:m] = np.arange(nv - m, nv)                 # the most recent blocks
+    t = [int(x) for x in qi.token_set(blocks, i, k) if x >= 0]
+    assert t == sorted(set(t)) and (not t or (t[0] >= 0 and t[-1] <= i))
+    assert len(t) == 4 * m + (i + 1) % 4
+    if m == nv:
+        assert t == list(range(i + 1))
