@@ -11,7 +11,9 @@ states).  `e2e` repeats the prefill measurement through the public API from pinn
 host buffers, every step's copies included (uploads, kernels and downloads of
 consecutive steps overlap on three streams).  `roofline` describes the dominant prefill kernel,
 timed live with the library's launch trace.  `cpu_baseline` is the fp64 oracle on
-the host cores (rank 0, N = 1 only).
+the host cores (rank 0, N = 1 only).  `qsa` holds the QSA indexer's two workloads (chunked
+prefill: 8192 queries at 64K context; decode: 64 rows x 4 tokens at 128K) in query tokens/s
+with the rooflines of its scores and top-512 kernels; `--qsa-only` runs just those.
 
 With N > 1 (torchrun), every rank runs its own independent problem of the same size
 (the path shards by sequence with no exchange): weak scaling, no data-path collective;
