@@ -153,6 +153,16 @@ def _group_slices(shape, heads):
     return groups, vheads, remap
 
 
+def _conv_state_columns(shape, groups, vheads):
+    """Columns of a raw conv-state row (q | k | v channels) that the QK heads ``groups``
+    and the V heads ``vheads`` read, in the order of the sliced problem."""
+    dk, dv = shape.d_k, shape.d_v
+    qkc = shape.n_qk_heads * dk
+    qch = [g * dk + i for g in groups for i in range(dk)]
+    vch = [h * dv + i for h in vheads for i in range(dv)]
+    return qch + [qkc + c for c in qch] + [2 * qkc + c for c in vch]
+
+
 def prefill(inp, heads=None, n_threads=None, q_scale=1.0, l2_eps=1e-6, initial_state=None,
             conv_state=None, mutant=0):
     """Oracle on a ``gdn_inputs.PrefillInputs`` bundle (stored values widened to fp64).
@@ -175,13 +185,9 @@ def prefill(inp, heads=None, n_threads=None, q_scale=1.0, l2_eps=1e-6, initial_s
         groups, vheads, hsel = list(range(sh.n_qk_heads)), list(range(sh.n_v_heads)), None
     else:
         groups, vheads, hsel = _group_slices(sh, heads)
-    qkc = sh.n_qk_heads * dk
     cs_sub = None
     if cs is not None:
-        qch = [g * dk + i for g in groups for i in range(dk)]
-        vch = [h * dv + i for h in vheads for i in range(dv)]
-        cols = qch + [qkc + c for c in qch] + [2 * qkc + c for c in vch]
-        cs_sub = f64(np.asarray(cs)[:, :, cols])
+        cs_sub = f64(np.asarray(cs)[:, :, _conv_state_columns(sh, groups, vheads)])
     y, fin, _ = gdn_prefill_f64(
         f64(inp.q[:, groups]), f64(inp.k[:, groups]), f64(inp.v[:, vheads]),
         inp.w_q.reshape(sh.n_qk_heads, dk, -1)[groups].reshape(len(groups) * dk, -1),
