@@ -28,7 +28,7 @@ _LIBS: dict = {}
 class OracleShape(ctypes.Structure):
     _fields_ = [("n_qk_heads", ctypes.c_int), ("n_v_heads", ctypes.c_int),
                 ("d_k", ctypes.c_int), ("d_v", ctypes.c_int), ("conv_width", ctypes.c_int),
-                ("q_scale", ctypes.c_double), ("l2_eps", ctypes.c_double)]
+                ("q_scale", ctypes.c_double), ("l2_eps", ctypes.c_double), ("conv_silu", ctypes.c_int)]
 
 
 def lib_path(mutant: int = 0) -> str:
@@ -86,7 +86,7 @@ def default_threads() -> int:
 
 def gdn_prefill_f64(q, k, v, w_q, w_k, w_v, alpha, beta, cu_seqlens, *, n_qk_heads, n_v_heads,
                     initial_state=None, conv_state=None, heads=None, q_scale=1.0, l2_eps=1e-6,
-                    n_threads=None, mutant=0):
+                    n_threads=None, mutant=0, conv_silu=False):
     """Run the oracle on fp64 arrays.
 
     Shapes: q,k [T,Hqk,dk]; v [T,Hv,dv]; w_* [channels, W]; alpha,beta [T,Hv];
@@ -106,7 +106,7 @@ def gdn_prefill_f64(q, k, v, w_q, w_k, w_v, alpha, beta, cu_seqlens, *, n_qk_hea
     W = w_q.shape[1]
     n = len(cu) - 1
     assert int(cu[-1]) == T and q.shape == (T, n_qk_heads, dk) and v.shape == (T, n_v_heads, dv)
-    sh = OracleShape(n_qk_heads, n_v_heads, dk, dv, W, float(q_scale), float(l2_eps))
+    sh = OracleShape(n_qk_heads, n_v_heads, dk, dv, W, float(q_scale), float(l2_eps), int(bool(conv_silu)))
     chans = 2 * n_qk_heads * dk + n_v_heads * dv
     out = np.full((T, n_v_heads, dv), np.nan)
     fin = np.full((n, n_v_heads, dk, dv), np.nan)
@@ -125,14 +125,15 @@ def gdn_prefill_f64(q, k, v, w_q, w_k, w_v, alpha, beta, cu_seqlens, *, n_qk_hea
 
 
 def gdn_conv_l2_f64(q, k, v, w_q, w_k, w_v, cu_seqlens, *, n_qk_heads, n_v_heads,
-                    conv_state=None, q_scale=1.0, l2_eps=1e-6, n_threads=None, mutant=0):
+                    conv_state=None, q_scale=1.0, l2_eps=1e-6, n_threads=None, mutant=0,
+                    conv_silu=False):
     """ShortConv + L2 alone: returns (q^, k^, v^) in fp64 with the input shapes."""
     q, k, v = _f64(q), _f64(k), _f64(v)
     w_q, w_k, w_v = _f64(w_q), _f64(w_k), _f64(w_v)
     conv_state = _f64(conv_state)
     cu = np.ascontiguousarray(cu_seqlens, dtype=np.int32)
     dk, dv, W = q.shape[2], v.shape[2], w_q.shape[1]
-    sh = OracleShape(n_qk_heads, n_v_heads, dk, dv, W, float(q_scale), float(l2_eps))
+    sh = OracleShape(n_qk_heads, n_v_heads, dk, dv, W, float(q_scale), float(l2_eps), int(bool(conv_silu)))
     qh, kh, vh = np.zeros_like(q), np.zeros_like(k), np.zeros_like(v)
     rc = _lib(mutant).oracle_gdn_conv_l2(
         ctypes.byref(sh), _dp(q), _dp(k), _dp(v), _dp(w_q), _dp(w_k), _dp(w_v),
@@ -164,7 +165,7 @@ def _conv_state_columns(shape, groups, vheads):
 
 
 def prefill(inp, heads=None, n_threads=None, q_scale=1.0, l2_eps=1e-6, initial_state=None,
-            conv_state=None, mutant=0):
+            conv_state=None, mutant=0, conv_silu=False):
     """Oracle on a ``gdn_inputs.PrefillInputs`` bundle (stored values widened to fp64).
 
     With ``heads`` only the QK groups those V heads read are widened and computed; the
@@ -197,7 +198,7 @@ def prefill(inp, heads=None, n_threads=None, q_scale=1.0, l2_eps=1e-6, initial_s
         n_qk_heads=len(groups), n_v_heads=len(vheads),
         initial_state=None if init is None else np.asarray(init, dtype=np.float64)[:, vheads],
         conv_state=cs_sub, heads=hsel, q_scale=q_scale, l2_eps=l2_eps, n_threads=n_threads,
-        mutant=mutant)
+        mutant=mutant, conv_silu=conv_silu)
     y_full = np.full((T, sh.n_v_heads, dv), np.nan)
     fin_full = np.full((n, sh.n_v_heads, dk, dv), np.nan)
     y_full[:, vheads] = y
@@ -229,7 +230,7 @@ def _conv_state_rows(inp, cs):
 
 
 def decode_steps(shape, dtype, dec, w, state, conv_state, rows=None, heads=None, steps=None,
-                 q_scale=1.0, l2_eps=1e-6, n_threads=None):
+                 q_scale=1.0, l2_eps=1e-6, n_threads=None, conv_silu=False):
     """Run ``steps`` single-token steps for decode rows ``rows`` (default all).
 
     ``dec`` is a ``gdn_inputs.DecodeInputs``; ``state`` [B,Hv,dk,dv] fp64 (or fp32)
@@ -254,7 +255,8 @@ def decode_steps(shape, dtype, dec, w, state, conv_state, rows=None, heads=None,
             stored_to_f64(dec.v[s, rows], dtype), w[0], w[1], w[2],
             stored_to_f64(dec.alpha[s, rows], dtype), stored_to_f64(dec.beta[s, rows], dtype),
             cu, n_qk_heads=shape.n_qk_heads, n_v_heads=shape.n_v_heads, initial_state=st,
-            conv_state=cs, heads=heads, q_scale=q_scale, l2_eps=l2_eps, n_threads=n_threads)
+            conv_state=cs, heads=heads, q_scale=q_scale, l2_eps=l2_eps, n_threads=n_threads,
+            conv_silu=conv_silu)
         ys[s] = y
         if heads is None:
             st = st_new

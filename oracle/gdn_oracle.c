@@ -15,6 +15,8 @@
  *     so tap W-1 multiplies the current row.  Rows before the start of a
  *     sequence come from the conv state (oldest row first) when one is given,
  *     else they are zero.  Packed sequences never see each other's rows.
+ *     Optionally (conv_silu = 1, off by default: the page names no activation) every
+ *     conv output passes SiLU(x) = x / (1 + e^-x) before step 2.
  *  2. Per-head L2 normalisation of q and k after the conv:
  *         q^ = q' * q_scale / sqrt(sum q'^2 + eps),  k^ = k' / sqrt(sum k'^2 + eps).
  *     v is not normalised.
@@ -51,6 +53,7 @@
 typedef struct {
     int n_qk_heads, n_v_heads, d_k, d_v, conv_width;
     double q_scale, l2_eps;
+    int conv_silu;   /* 1: SiLU on every conv output (before the L2 norm of q, k) */
 } oracle_shape;
 
 /* raw value of channel c of conv input row s of sequence b (s < 0: history) */
@@ -86,22 +89,33 @@ static double short_conv(const double *x, int64_t row_stride, int64_t tok0, int 
     return acc;
 }
 
-/* conv then L2 over the head's d channels starting at channel c0 */
+/* SiLU(x) = x * sigmoid(x) = x / (1 + e^-x) */
+static double silu(double x) { return x / (1.0 + exp(-x)); }
+
+/* conv (then SiLU when `act`) then L2 over the head's d channels starting at channel c0 */
 static void conv_l2_head(double *dst, const double *x, int64_t row_stride, int64_t tok0, int s,
                          int c0, int d, const double *w, const double *conv_state,
                          int64_t cs_row_stride, int cs_offset, int b, int W, int normalize,
-                         double scale, double eps)
+                         double scale, double eps, int act)
 {
     double ss = 0.0;
     for (int i = 0; i < d; ++i) {
         dst[i] = short_conv(x, row_stride, tok0, s, c0 + i, w, conv_state, cs_row_stride,
                             cs_offset, b, W);
+#if GDN_ORACLE_MUTANT != 7
+        if (act) dst[i] = silu(dst[i]);
+#endif
         ss += dst[i] * dst[i];
     }
     if (normalize) {
         double inv = scale / sqrt(ss + eps);
         for (int i = 0; i < d; ++i) dst[i] *= inv;
     }
+#if GDN_ORACLE_MUTANT == 7
+    /* planted: the activation after the normalisation */
+    if (act)
+        for (int i = 0; i < d; ++i) dst[i] = silu(dst[i]);
+#endif
 }
 
 /*
@@ -174,11 +188,11 @@ int oracle_gdn_prefill(const oracle_shape *sh,
         for (int t = 0; t < L; ++t) {
             /* 1-2: ShortConv then L2 norm (q, k) */
             conv_l2_head(qh, q, (int64_t)H * dk, tok0, t, g * dk, dk, wq, conv_state, chans, 0,
-                         b, W, 1, sh->q_scale, sh->l2_eps);
+                         b, W, 1, sh->q_scale, sh->l2_eps, sh->conv_silu);
             conv_l2_head(kh, k, (int64_t)H * dk, tok0, t, g * dk, dk, wk, conv_state, chans,
-                         H * dk, b, W, 1, 1.0, sh->l2_eps);
+                         H * dk, b, W, 1, 1.0, sh->l2_eps, sh->conv_silu);
             conv_l2_head(vh, v, (int64_t)Hv * dv, tok0, t, h * dv, dv, wv, conv_state, chans,
-                         2 * H * dk, b, W, 0, 1.0, 0.0);
+                         2 * H * dk, b, W, 0, 1.0, 0.0, sh->conv_silu);
             const double a = alpha[(tok0 + t) * Hv + h];
             const double be = beta[(tok0 + t) * Hv + h];
 
@@ -281,13 +295,14 @@ int oracle_gdn_conv_l2(const oracle_shape *sh,
         for (int t = 0; t < L; ++t) {
             for (int g = 0; g < H; ++g) {
                 conv_l2_head(qh + ((tok0 + t) * H + g) * dk, q, (int64_t)H * dk, tok0, t, g * dk,
-                             dk, wq, conv_state, chans, 0, b, W, 1, sh->q_scale, sh->l2_eps);
+                             dk, wq, conv_state, chans, 0, b, W, 1, sh->q_scale, sh->l2_eps, sh->conv_silu);
                 conv_l2_head(kh + ((tok0 + t) * H + g) * dk, k, (int64_t)H * dk, tok0, t, g * dk,
-                             dk, wk, conv_state, chans, H * dk, b, W, 1, 1.0, sh->l2_eps);
+                             dk, wk, conv_state, chans, H * dk, b, W, 1, 1.0, sh->l2_eps, sh->conv_silu);
             }
             for (int h = 0; h < Hv; ++h)
                 conv_l2_head(vh + ((tok0 + t) * Hv + h) * dv, v, (int64_t)Hv * dv, tok0, t,
-                             h * dv, dv, wv, conv_state, chans, 2 * H * dk, b, W, 0, 1.0, 0.0);
+                             h * dv, dv, wv, conv_state, chans, 2 * H * dk, b, W, 0, 1.0, 0.0,
+                             sh->conv_silu);
         }
     }
     return 0;

@@ -372,9 +372,11 @@ def test_head_mapping_contiguous_groups():
 
 
 # ----------------------------------------------------------------------------- planted mistakes
-def _full_pipeline_brute(p, q_scale=1.0):
-    """Whole mixer rebuilt from library routines: np.convolve, np.linalg.norm and the
-    transition-product brute force (one (seq, V head) at a time)."""
+def _full_pipeline_brute(p, q_scale=1.0, silu=False):
+    """Whole mixer rebuilt from library routines: np.convolve, scipy's logistic function for
+    the optional SiLU, np.linalg.norm and the transition-product brute force (one
+    (seq, V head) at a time)."""
+    from scipy.special import expit
     H, Hv = p.shape.n_qk_heads, p.shape.n_v_heads
     dk, dv = p.shape.d_k, p.shape.d_v
     G = Hv // H
@@ -391,6 +393,8 @@ def _full_pipeline_brute(p, q_scale=1.0):
                           for c in range(xs.shape[1])], axis=1)
             return r.reshape(x[t0:t1].shape)
         qc, kc, vc = conv(p.q, p.w_q), conv(p.k, p.w_k), conv(p.v, p.w_v)
+        if silu:
+            qc, kc, vc = qc * expit(qc), kc * expit(kc), vc * expit(vc)
         qn = q_scale * qc / np.sqrt((qc ** 2).sum(-1, keepdims=True) + 1e-6)
         kn = kc / np.sqrt((kc ** 2).sum(-1, keepdims=True) + 1e-6)
         for h in range(Hv):
@@ -403,17 +407,37 @@ def _full_pipeline_brute(p, q_scale=1.0):
     return out, fins
 
 
-def test_brute_pipeline_matches_oracle():
+@pytest.mark.parametrize("silu", [False, True])
+def test_brute_pipeline_matches_oracle(silu):
     shape = gi.GdnShape(n_qk_heads=2, n_v_heads=6, d_k=6, d_v=5)
     p = gi.make_prefill_inputs(shape, [7, 3], gi.F32, seed=61)
-    y, fin, _ = oracle.prefill(p)
-    yb, fb = _full_pipeline_brute(p)
+    y, fin, _ = oracle.prefill(p, conv_silu=silu)
+    yb, fb = _full_pipeline_brute(p, silu=silu)
     assert rel(y, yb) < 1e-11 and rel(fin, fb) < 1e-11
+    if silu:   # the activation changes the result
+        y0, _, _ = oracle.prefill(p)
+        assert rel(y, y0) > 1e-2
+
+
+def test_conv_silu_closed_forms():
+    """With the identity conv ([0, 0, 0, 1] taps) the conv output of each channel is the raw
+    value x, so q^ is SiLU(x) normalised: SiLU(0) = 0, SiLU(ln 3) = (3/4) ln 3 and
+    SiLU(-ln 3) = -(1/4) ln 3 (the logistic function at ln 3 is 3/4); v is SiLU(x) itself."""
+    shape = gi.GdnShape(n_qk_heads=1, n_v_heads=1, d_k=4, d_v=4)
+    ln3 = np.log(3.0)
+    x = np.array([[[0.0, ln3, -ln3, 2.0]]])
+    w = identity_weights(4)
+    qh, kh, vh = oracle.gdn_conv_l2_f64(x, x, x, w, w, w, np.array([0, 1], np.int32), n_qk_heads=1,
+                                        n_v_heads=1, l2_eps=0.0, conv_silu=True)
+    s = np.array([0.0, 0.75 * ln3, -0.25 * ln3, 2.0 / (1.0 + np.exp(-2.0))])
+    np.testing.assert_allclose(vh[0, 0], s, rtol=1e-15, atol=1e-15)
+    np.testing.assert_allclose(qh[0, 0], s / np.linalg.norm(s), rtol=1e-14)
+    np.testing.assert_allclose(kh[0, 0], s / np.linalg.norm(s), rtol=1e-14)
 
 
 MUTANTS = {1: "error uses the undecayed state", 2: "output reads the state before the write",
            3: "state transposed", 4: "conv taps reversed", 5: "interleaved V->QK head mapping",
-           6: "beta dropped from the write"}
+           6: "beta dropped from the write", 7: "conv SiLU after the L2 normalisation"}
 
 
 @pytest.mark.parametrize("mutant", sorted(MUTANTS))
@@ -421,8 +445,9 @@ def test_planted_mistakes_are_caught(mutant):
     shape = gi.GdnShape(n_qk_heads=2, n_v_heads=6, d_k=6, d_v=6)
     p = gi.make_prefill_inputs(shape, [7, 3], gi.F32, seed=61)
     oracle.build(mutant)
-    y, fin, _ = oracle.prefill(p, mutant=mutant)
-    yb, fb = _full_pipeline_brute(p)
+    silu = mutant == 7   # that mistake lives in the optional activation
+    y, fin, _ = oracle.prefill(p, mutant=mutant, conv_silu=silu)
+    yb, fb = _full_pipeline_brute(p, silu=silu)
     assert rel(y, yb) > 1e-3 or rel(fin, fb) > 1e-3, MUTANTS[mutant]
 
 
