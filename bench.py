@@ -10,8 +10,15 @@ is the batched decode workload (256 rows x 1024 consecutive steps on resident fp
 states).  `e2e` repeats the prefill measurement through the public API from pinned
 host buffers, every step's copies included (uploads, kernels and downloads of
 consecutive steps overlap on three streams).  `roofline` describes the dominant prefill kernel,
-timed live with the library's launch trace.  `cpu_baseline` is the fp64 oracle on
-the host cores (rank 0, N = 1 only).  `qsa` holds the QSA indexer's two workloads (chunked
+timed live with the library's launch trace; its `traffic` is the DRAM bytes of one launch from
+an ncu capture recorded in the profile summaries together with the sha256 of the kernel
+sources it was built from, and is null when the sources have changed since.  `step` gives the
+whole prefill step against the TF32 and bf16 tensor peaks.  `prefill_longctx` (T = 262,144,
+mean alpha 0.98) and `prefill_varlen` (32 packed sequences of log-uniform lengths with initial
+states) are the two other prefill workloads, each with its roofline and oracle baseline.
+`prefill_gated` is the headline prefill with the output tail (gated RMS norm) fused into the
+store of y, beside the same two steps unfused.  `cpu_baseline` is the fp64 oracle on all host
+cores and `cpu_baseline_1core` on one (rank 0, N = 1 only).  `qsa` holds the QSA indexer's two workloads (chunked
 prefill: 8192 queries at 64K context; decode: 64 rows x 4 tokens at 128K) in query tokens/s
 with the rooflines of its scores and top-512 kernels; `--qsa-only` runs just those.
 
@@ -53,11 +60,6 @@ CHAIN_FLOP_TV = 6 * D * D + 3 * 2 * CHUNK * D
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
                   "sm_max_mhz": 1965.0}
 TF32_PER_BF16 = 1.1 / 2.25   # nominal dense tf32 : bf16 tensor throughput on B200
-# dram__bytes_read.sum + dram__bytes_write.sum per launch from one ncu capture of the current
-# kernels on this workload (profiles/prefill_tc_T8192_ncu.md: one chain launch of the step's
-# four chunk ranges, 2048 tokens; profiles/decode_B256_ncu.md); None while a kernel has
-# changed since its capture
-NCU_TRAFFIC_BYTES = {"prefill_tc": 159_957_760 + 31_570_176, "decode": 826_713_088 + 769_751_552}
 FP32_LANES_PER_SM = 128
 N_SM = 148
 
@@ -192,57 +194,117 @@ def gpu_gate_inputs(torch, gen, shape, c, dtype):
 
 
 # ----------------------------------------------------------------------------- prefill
-def bench_prefill(args, dist, torch, gdn, peaks):
-    w = gi.WORKLOADS[1]
+def device_prefill_problem(torch, gdn, idx, rank):
+    """Device-resident inputs of prefill workload ``idx`` (1, 2 or 4), each rank its own draw.
+
+    Workload 1 is drawn on the host by the seeded input module (the same bytes the parity
+    tests give the oracle); workloads 2 and 4 are drawn on the device with a seeded torch
+    generator from the same distributions (their size makes host draws slow).  Workload 4's
+    initial states and conv states are the final states of a seeded 2048-token prefill per
+    sequence, made by libgdn itself (timing inputs only, never compared with anything)."""
+    w = gi.WORKLOADS[idx]
     shape = w["shape"]
-    T = w["lengths"][0]
-    seed = gi.workload_seed(1) + 7919 * dist.rank  # rank 0 runs the workload itself
-    inp = gi.make_prefill_inputs(shape, [T], w["dtype"], seed, c=w["c"],
-                                 weights=gi.workload_weights(1))
-    q, k, v = to_dev(inp.q, torch), to_dev(inp.k, torch), to_dev(inp.v, torch)
-    wq, wk, wv = to_dev(inp.w_q, torch), to_dev(inp.w_k, torch), to_dev(inp.w_v, torch)
-    al, be = to_dev(inp.alpha, torch), to_dev(inp.beta, torch)
-    cu = torch.from_numpy(inp.cu_seqlens).cuda()
-    cfg = gdn.GdnConfig(shape.n_qk_heads, shape.n_v_heads)
-    out = torch.empty((T, shape.n_v_heads, D), dtype=torch.float32, device="cuda")
-    fin = torch.empty((1, shape.n_v_heads, D, D), dtype=torch.float32, device="cuda")
-    ws = torch.empty(gdn.prefill_workspace_size(cfg, torch.bfloat16, T, 1), dtype=torch.uint8,
-                     device="cuda")
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")  # > 126 MB L2
+    H, Hv = shape.n_qk_heads, shape.n_v_heads
+    bf = torch.bfloat16
+    cfg = gdn.GdnConfig(H, Hv)
+    wq, wk, wv = (to_dev(x, torch) for x in gi.workload_weights(idx))
+    p = {"cfg": cfg, "wq": wq, "wk": wk, "wv": wv, "init": None, "conv_in": None, "name": w["name"]}
+    if idx == 1:
+        T = w["lengths"][0]
+        inp = gi.make_prefill_inputs(shape, [T], w["dtype"], gi.workload_seed(1) + 7919 * rank, c=w["c"],
+                                     weights=gi.workload_weights(1))
+        p.update(q=to_dev(inp.q, torch), k=to_dev(inp.k, torch), v=to_dev(inp.v, torch),
+                 al=to_dev(inp.alpha, torch), be=to_dev(inp.beta, torch),
+                 cu=torch.from_numpy(inp.cu_seqlens).cuda(), lengths=[T])
+        return p
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(gi.workload_seed(idx) + 7919 * rank)
+    lengths = list(w["lengths"]) if idx == 2 else [int(x) for x in gi.varlen_lengths(idx)]
+    T, n = sum(lengths), len(lengths)
+    cu = torch.zeros(n + 1, dtype=torch.int32)
+    cu[1:] = torch.cumsum(torch.tensor(lengths, dtype=torch.int64), 0).to(torch.int32)
+    p.update(q=torch.randn((T, H, D), generator=gen, device="cuda").to(bf),
+             k=torch.randn((T, H, D), generator=gen, device="cuda").to(bf),
+             v=torch.randn((T, Hv, D), generator=gen, device="cuda").to(bf),
+             cu=cu.cuda(), lengths=lengths)
+    p["al"], p["be"] = gpu_gate_inputs(torch, gen, (T, Hv), w["c"], bf)
+    if idx == 4:
+        Tw = w["warm_tokens"]
+        init = torch.empty((n, Hv, D, D), dtype=torch.float32, device="cuda")
+        conv = torch.empty((n, 3, cfg.channels), dtype=bf, device="cuda")
+        for r0 in range(0, n, 8):
+            m = min(8, n - r0)
+            q = torch.randn((m * Tw, H, D), generator=gen, device="cuda").to(bf)
+            k = torch.randn((m * Tw, H, D), generator=gen, device="cuda").to(bf)
+            v = torch.randn((m * Tw, Hv, D), generator=gen, device="cuda").to(bf)
+            al, be = gpu_gate_inputs(torch, gen, (m * Tw, Hv), w["c"], bf)
+            wcu = torch.arange(m + 1, dtype=torch.int32, device="cuda") * Tw
+            gdn.gdn_prefill(q, k, v, wq, wk, wv, al, be, wcu, cfg=cfg, final_state=init[r0:r0 + m],
+                            conv_state_out=conv[r0:r0 + m], out=torch.empty((m * Tw, Hv, D), device="cuda"),
+                            max_seqlen=Tw)
+            del q, k, v, al, be
+        torch.cuda.synchronize()
+        p["init"], p["conv_in"] = init, conv
+    return p
 
-    def call():
-        gdn.gdn_prefill(q, k, v, wq, wk, wv, al, be, cu, cfg=cfg, out=out, final_state=fin,
-                        workspace=ws)
 
+def time_prefill(args, dist, torch, gdn, call, flush, steps):
+    """`steps` timed calls (L2 flushed before each, CUDA events around each), after warm-up;
+    then the same number under the launch trace for per-kernel durations."""
     for _ in range(args.warmup):
         call()
-    K = args.steps
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for _ in range(K)]
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
     clocks = ClockSampler(device_id_for_smi())
     dist.barrier()
     clocks.start()
-    for i in range(K):
+    for i in range(steps):
         flush.zero_()
         ev[i][0].record()
         call()
         ev[i][1].record()
     dist.barrier()
     clk = clocks.stop()
-    ms = sum(a.elapsed_time(b) for a, b in ev)
-    ms_max = dist.max(ms)
-    # per-kernel durations: the same K steps again under the launch trace (its events add a
+    ms_max = dist.max(sum(a.elapsed_time(b) for a, b in ev))
+    # per-kernel durations: the same steps again under the launch trace (its events add a
     # little time of their own, so the steps above run without it)
-    trace = gdn.LaunchTrace(capacity=16 * K)
+    trace = gdn.LaunchTrace(capacity=1024 * steps)
     with trace:
-        for i in range(K):
+        for _ in range(steps):
             flush.zero_()
             call()
     dist.barrier()
-    recs = trace.records()
     per_kernel = {}
-    for name, t in recs:
+    for name, t in trace.records():
         per_kernel.setdefault(name, []).append(t)
+    return ms_max, clk, {n: {"launches": len(v), "avg_ms": sum(v) / len(v), "total_ms": sum(v)}
+                         for n, v in per_kernel.items()}, trace.count
+
+
+def bench_prefill(args, dist, torch, gdn, peaks, idx=1, e2e=True):
+    """Prefill of workload ``idx`` on resident inputs; for the headline workload also the same
+    through the public API from pinned host buffers (``e2e``)."""
+    p = device_prefill_problem(torch, gdn, idx, dist.rank)
+    q, k, v, al, be, cu, cfg = p["q"], p["k"], p["v"], p["al"], p["be"], p["cu"], p["cfg"]
+    wq, wk, wv = p["wq"], p["wk"], p["wv"]
+    T, n, Hv = q.shape[0], len(p["lengths"]), cfg.n_v_heads
+    out = torch.empty((T, Hv, D), dtype=torch.float32, device="cuda")
+    fin = torch.empty((n, Hv, D, D), dtype=torch.float32, device="cuda")
+    ms = max(p["lengths"])   # the longest sequence, known on the host
+    ws = torch.empty(gdn.prefill_workspace_size(cfg, torch.bfloat16, T, n, ms), dtype=torch.uint8, device="cuda")
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")  # > 126 MB L2
+
+    def call():
+        gdn.gdn_prefill(q, k, v, wq, wk, wv, al, be, cu, cfg=cfg, initial_state=p["init"],
+                        conv_state_in=p["conv_in"], out=out, final_state=fin, workspace=ws, max_seqlen=ms)
+
+    K = args.steps if idx == 1 else max(1, min(args.steps, args.long_steps))
+    ms_max, clk, per_kernel, launches = time_prefill(args, dist, torch, gdn, call, flush, K)
+    tokens_all = T * dist.world * K
+    res = {"value": tokens_all / (ms_max / 1e3), "ms_per_step": ms_max / K, "clocks": clk,
+           "per_kernel": per_kernel, "launches": launches / K, "tokens_per_step": T, "steps": K,
+           "n_v_heads": Hv, "n_seqs": n, "workload": p["name"], "workspace_bytes": ws.numel()}
+    if not e2e:
+        return res
 
     # e2e: public API from pinned host buffers, every step's copies inside the timed region.
     # Steps run as a pipeline on three streams (upload, compute, download) over two sets of
@@ -264,13 +326,13 @@ def bench_prefill(args, dist, torch, gdn, peaks):
     def ev():
         return torch.cuda.Event()
 
-    def e2e_steps(n):
+    def e2e_steps(n_steps):
         up_done, comp_done, dn_done = [], [], []
         start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         start.record(comp)
         s_up.wait_stream(comp)
         s_dn.wait_stream(comp)
-        for i in range(n):
+        for i in range(n_steps):
             b = i % 2
             with torch.cuda.stream(s_up):
                 if i >= 2:
@@ -285,7 +347,7 @@ def bench_prefill(args, dist, torch, gdn, peaks):
             flush.zero_()
             xq, xk, xv, xa, xb = dev_in[b]
             gdn.gdn_prefill(xq, xk, xv, wq, wk, wv, xa, xb, cu, cfg=cfg, out=dev_out[b],
-                            final_state=fin, workspace=ws)
+                            final_state=fin, workspace=ws, max_seqlen=ms)
             comp_done.append(ev())
             comp_done[i].record(comp)
             with torch.cuda.stream(s_dn):
@@ -303,16 +365,137 @@ def bench_prefill(args, dist, torch, gdn, peaks):
     e0, e1 = e2e_steps(K)
     dist.barrier()
     e2e_ms = dist.max(e0.elapsed_time(e1))
+    res["e2e"] = {"value": tokens_all / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                  "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / K}
+    return res
 
-    tokens_all = T * dist.world * K
-    return {
-        "value": tokens_all / (ms_max / 1e3), "ms_per_step": ms_max / K, "clocks": clk,
-        "per_kernel": {n: {"launches": len(v), "avg_ms": sum(v) / len(v), "total_ms": sum(v)}
-                       for n, v in per_kernel.items()},
-        "launches": trace.count, "tokens_per_step": T, "steps": K, "n_v_heads": shape.n_v_heads,
-        "e2e": {"value": tokens_all / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / K},
-    }
+
+# ----------------------------------------------------------------------------- traffic records
+def kernel_sources_sha256():
+    """sha256 over the library's kernel and ABI sources (file names and bytes, sorted): the
+    identity of the binary whose DRAM traffic a record describes."""
+    import hashlib
+    h = hashlib.sha256()
+    roots = [os.path.join(ROOT, "linear_attention_recurrence_05_b200", "csrc"), os.path.join(ROOT, "include")]
+    for r in roots:
+        for name in sorted(os.listdir(r)):
+            if name.endswith((".cu", ".cuh", ".h")):
+                h.update(name.encode())
+                with open(os.path.join(r, name), "rb") as f:
+                    h.update(f.read())
+    return h.hexdigest()
+
+
+def traffic_records():
+    """`traffic-record:` lines of the ncu summaries: DRAM read + write bytes of one launch of a
+    kernel, the sources it was built from and the work of that launch."""
+    recs = {}
+    pdir = os.path.join(ROOT, "profiles")
+    for name in sorted(os.listdir(pdir)) if os.path.isdir(pdir) else []:
+        if not name.endswith(".md"):
+            continue
+        with open(os.path.join(pdir, name)) as f:
+            for line in f:
+                if line.startswith("traffic-record:"):
+                    try:
+                        r = json.loads(line.split(":", 1)[1])
+                    except ValueError:
+                        continue
+                    recs[(r["kernel"], r["workload"])] = dict(r, file=name)
+    return recs
+
+
+def traffic_for(kernel, workload, units_per_launch, sha):
+    """The recorded per-launch DRAM bytes of `kernel` scaled to `units_per_launch` (tokens or
+    rows; the kernels' traffic grows in proportion to them), or None with the reason when no
+    record matches the sources that were built."""
+    r = traffic_records().get((kernel, workload))
+    if r is None:
+        return None, "no ncu record"
+    if r.get("sources_sha256") != sha:
+        return None, f"stale: {r['file']} was captured on other sources"
+    return r["bytes_per_launch"] * units_per_launch / r["units_per_launch"], r["file"]
+
+
+def prefill_roofline(res, peaks, peak_src, sha):
+    pk = res["per_kernel"]
+    dom = max(pk, key=lambda n: pk[n]["total_ms"])
+    avg_s = pk[dom]["avg_ms"] / 1e3
+    # a step may run a kernel several times over consecutive chunk ranges (pipelined path):
+    # the work of one launch is the step's tokens over its launches per step
+    T = res["tokens_per_step"] * res["steps"] / pk[dom]["launches"]
+    Hv = res["n_v_heads"]
+    step_ms = sum(v["total_ms"] for v in pk.values())
+    share = {n: round(v["total_ms"] / step_ms, 4) for n, v in pk.items()}
+    bf16 = peaks["bf16_tflops"]
+    if dom == "scan_simt":
+        flops = PREFILL_FLOP_TV * T * Hv
+        peak = N_SM * FP32_LANES_PER_SM * 2 * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12
+        return {"kernel": dom, "bound": "alu", "achieved": flops / avg_s / 1e12, "peak": peak,
+                "unit": "TFLOP/s", "frac": flops / avg_s / 1e12 / peak, "traffic": None,
+                "peak_source": f"148 SMs x 128 fp32 FMA lanes x 2 x {peaks.get('sm_max_mhz')} MHz",
+                "algorithmic_per_launch": flops, "tokens_per_launch": T, "kernel_share": share}
+    if dom.startswith("prefill_tc"):
+        flops = CHAIN_FLOP_TV * T * Hv
+        peak = bf16 * TF32_PER_BF16
+        traffic, tsrc = traffic_for(dom, res["workload"], T, sha)
+        ach = flops / avg_s / 1e12
+        return {"kernel": dom, "bound": "tensor", "achieved": ach, "peak": peak,
+                "unit": "TFLOP/s", "frac": ach / peak, "frac_of_bf16_peak": ach / bf16,
+                "traffic": traffic, "traffic_source": tsrc,
+                "peak_source": f"tf32 = {peak_src} bf16 {bf16} x 1.1/2.25 nominal",
+                "algorithmic_per_launch": flops, "tokens_per_launch": T, "kernel_share": share}
+    # a memory-bound kernel dominates
+    byts = (2 * 16 * D * 2 + 48 * D * 2 + 3 * 16 * 4 * D) * T
+    return {"kernel": dom, "bound": "hbm", "achieved": byts / avg_s / 1e9, "peak": peaks["hbm_gbs"],
+            "unit": "GB/s", "frac": byts / avg_s / 1e9 / peaks["hbm_gbs"], "traffic": None,
+            "peak_source": peak_src, "kernel_share": share}
+
+
+def prefill_step_summary(res, peaks):
+    """Whole-step rates of a prefill leg against both tensor peaks and the copy bandwidth."""
+    s = res["ms_per_step"] / 1e3
+    T = res["tokens_per_step"]
+    flops = PREFILL_FLOP_TV * T * res["n_v_heads"]
+    tf32 = peaks["bf16_tflops"] * TF32_PER_BF16
+    return {"tflops": flops / s / 1e12, "frac_of_tf32_peak": flops / s / 1e12 / tf32,
+            "frac_of_bf16_peak": flops / s / 1e12 / peaks["bf16_tflops"],
+            "algorithmic_flops_per_step": flops}
+
+
+def bench_prefill_gated(args, dist, torch, gdn, peaks):
+    """The headline prefill with the output tail fused into the store of y (gdn_prefill_gated:
+    gate input z bf16, gated output bf16), against the same two steps unfused (gdn_prefill with
+    fp32 y, then gdn_output_gate); L2 flushed between steps."""
+    p = device_prefill_problem(torch, gdn, 1, dist.rank)
+    q, k, v, al, be, cu, cfg = p["q"], p["k"], p["v"], p["al"], p["be"], p["cu"], p["cfg"]
+    w3 = (p["wq"], p["wk"], p["wv"])
+    T, Hv = q.shape[0], cfg.n_v_heads
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(gi.workload_seed(1) + 53 + 7919 * dist.rank)
+    z = torch.randn((T, Hv, D), generator=gen, device="cuda").to(torch.bfloat16)
+    nw = torch.ones(D, device="cuda")
+    o = torch.empty((T, Hv, D), dtype=torch.bfloat16, device="cuda")
+    y = torch.empty((T, Hv, D), dtype=torch.float32, device="cuda")
+    fin = torch.empty((1, Hv, D, D), dtype=torch.float32, device="cuda")
+    ws = torch.empty(gdn.prefill_workspace_size(cfg, torch.bfloat16, T, 1, T), dtype=torch.uint8, device="cuda")
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+
+    def fused():
+        gdn.gdn_prefill(q, k, v, *w3, al, be, cu, cfg=cfg, out=o, final_state=fin, workspace=ws, max_seqlen=T,
+                        gate=(z, nw, 1e-6))
+
+    def unfused():
+        gdn.gdn_prefill(q, k, v, *w3, al, be, cu, cfg=cfg, out=y, final_state=fin, workspace=ws, max_seqlen=T)
+        gdn.gdn_output_gate(y, z, nw, cfg=cfg, out=o)
+
+    res = {}
+    for name, fn in (("fused", fused), ("unfused", unfused)):
+        ms, _, per_kernel, _ = time_prefill(args, dist, torch, gdn, fn, flush, args.steps)
+        res[name] = {"value": T * dist.world * args.steps / (ms / 1e3), "ms_per_step": ms / args.steps,
+                     "kernels": {n: round(v["avg_ms"], 4) for n, v in per_kernel.items()}}
+    return {"value": res["fused"]["value"], "unit": UNIT, "workload": f"{p['name']}+gated-rmsnorm-out-bf16",
+            "ms_per_step": res["fused"]["ms_per_step"], "unfused": res["unfused"]}
 
 
 def bench_output_gate(args, dist, torch, gdn, peaks, peak_src):
@@ -462,38 +645,6 @@ def qsa_oracle_rows_per_s(target_s: float):
             return rows / dt, rows, dt
 
 
-def prefill_roofline(res, peaks, peak_src):
-    pk = res["per_kernel"]
-    dom = max(pk, key=lambda n: pk[n]["total_ms"])
-    avg_s = pk[dom]["avg_ms"] / 1e3
-    # a step may run a kernel several times over consecutive chunk ranges (pipelined path):
-    # the work of one launch is the step's tokens over its launches per step
-    T = res["tokens_per_step"] * res["steps"] / pk[dom]["launches"]
-    Hv = res["n_v_heads"]
-    step_ms = sum(v["total_ms"] for v in pk.values())
-    share = {n: round(v["total_ms"] / step_ms, 4) for n, v in pk.items()}
-    if dom == "scan_simt":
-        flops = PREFILL_FLOP_TV * T * Hv
-        peak = N_SM * FP32_LANES_PER_SM * 2 * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12
-        return {"kernel": dom, "bound": "alu", "achieved": flops / avg_s / 1e12, "peak": peak,
-                "unit": "TFLOP/s", "frac": flops / avg_s / 1e12 / peak, "traffic": None,
-                "peak_source": f"148 SMs x 128 fp32 FMA lanes x 2 x {peaks.get('sm_max_mhz')} MHz",
-                "algorithmic_per_launch": flops, "tokens_per_launch": T, "kernel_share": share}
-    if dom.startswith("prefill_tc"):
-        flops = CHAIN_FLOP_TV * T * Hv
-        peak = peaks["bf16_tflops"] * TF32_PER_BF16
-        return {"kernel": dom, "bound": "tensor", "achieved": flops / avg_s / 1e12, "peak": peak,
-                "unit": "TFLOP/s", "frac": flops / avg_s / 1e12 / peak,
-                "traffic": NCU_TRAFFIC_BYTES.get("prefill_tc"),
-                "peak_source": f"tf32 = {peak_src} bf16 {peaks['bf16_tflops']} x 1.1/2.25 nominal",
-                "algorithmic_per_launch": flops, "tokens_per_launch": T, "kernel_share": share}
-    # a memory-bound kernel dominates
-    byts = (2 * 16 * D * 2 + 48 * D * 2 + 3 * 16 * 4 * D) * T
-    return {"kernel": dom, "bound": "hbm", "achieved": byts / avg_s / 1e9, "peak": peaks["hbm_gbs"],
-            "unit": "GB/s", "frac": byts / avg_s / 1e9 / peaks["hbm_gbs"], "traffic": None,
-            "peak_source": peak_src, "kernel_share": share}
-
-
 # ----------------------------------------------------------------------------- decode
 def decode_bytes_per_row(shape, in_bytes=2, out_bytes=4):
     Hqk, Hv = shape.n_qk_heads, shape.n_v_heads
@@ -528,7 +679,8 @@ def bench_decode(args, dist, torch, gdn, peaks, peak_src):
         al, be = gpu_gate_inputs(torch, gen, (Tw, Hv), w["c"], bf)
         cu = torch.arange(n + 1, dtype=torch.int32, device="cuda") * warm_T
         gdn.gdn_prefill(q, k, v, wq, wk, wv, al, be, cu, cfg=cfg, final_state=state[r0:r0 + n],
-                        conv_state_out=conv[r0:r0 + n], out=torch.empty((Tw, Hv, D), device="cuda"))
+                        conv_state_out=conv[r0:r0 + n], out=torch.empty((Tw, Hv, D), device="cuda"),
+                        max_seqlen=warm_T)
         del q, k, v, al, be
     torch.cuda.synchronize()
     # fresh inputs for every step
@@ -590,6 +742,7 @@ def bench_decode(args, dist, torch, gdn, peaks, peak_src):
     dist.barrier()
     e2e_ms = dist.max(e2.elapsed_time(e3))
     toks = B * steps * dist.world
+    dec_traffic, dec_tsrc = traffic_for("decode", w["name"], B, kernel_sources_sha256())
     multi = bench_decode_multi(args, dist, torch, gdn, peaks, peak_src, shape, cfg, (wq, wk, wv),
                                (dq, dk, dv, da, db), state, conv, state0, conv0)
     return {
@@ -598,7 +751,7 @@ def bench_decode(args, dist, torch, gdn, peaks, peak_src):
         "steps": steps, "ms_per_step": ms / steps, "launches": trace.count, "clocks": clk,
         "roofline": {"kernel": "decode", "bound": "hbm", "achieved": achieved,
                      "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
-                     "traffic": NCU_TRAFFIC_BYTES.get("decode"), "peak_source": peak_src,
+                     "traffic": dec_traffic, "traffic_source": dec_tsrc, "peak_source": peak_src,
                      "algorithmic_bytes_per_row": bpr, "rows_per_launch": B},
         "e2e": {"value": toks / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "note": "host inputs cycle through 32 pinned step sets"},
@@ -660,24 +813,44 @@ def bench_decode_multi(args, dist, torch, gdn, peaks, peak_src, shape, cfg, wts,
 
 
 # ----------------------------------------------------------------------------- oracle
-def oracle_tokens_per_s(target_s: float, seed_offset: int = 0):
-    """Time the fp64 oracle on a prefix of the prefill workload (all 48 V heads),
-    sized to take about target_s seconds.  Returns (tokens/s, threads, sample text, secs)."""
+def oracle_tokens_per_s(target_s: float, idx: int = 1, n_threads=None, seed_offset: int = 0):
+    """Time the fp64 oracle on a bounded sample of prefill workload ``idx`` (all 48 V heads),
+    sized to take about target_s seconds: the first T tokens of a seeded draw of the workload's
+    distributions (workload 4: one sequence of the set's first length, with an initial state and
+    a conv state).  The oracle's cost per token does not depend on the values, so tokens/s of
+    the sample is the rate of the whole workload.  Returns (tokens/s, threads, sample, secs)."""
     import oracle
-    w = gi.WORKLOADS[1]
-    threads = oracle.default_threads()
+    w = gi.WORKLOADS[idx]
+    threads = n_threads or oracle.default_threads()
+    cap = w["lengths"][0] if idx != 4 else int(gi.varlen_lengths(idx)[0])
 
     def run(T):
-        inp = gi.make_prefill_inputs(w["shape"], [T], w["dtype"], gi.workload_seed(1) + seed_offset,
-                                     c=w["c"], weights=gi.workload_weights(1))
+        inp = gi.make_prefill_inputs(w["shape"], [T], w["dtype"], gi.workload_seed(idx) + seed_offset,
+                                     c=w["c"], weights=gi.workload_weights(idx),
+                                     with_initial_state=idx == 4, with_conv_state=idx == 4)
         t0 = time.perf_counter()
         oracle.prefill(inp, n_threads=threads)
         return time.perf_counter() - t0
-    probe_T = 128
+    probe_T = 64 if threads == 1 else 128
     dt = run(probe_T)
-    T = int(min(8192, max(probe_T, probe_T * target_s / max(dt, 1e-6))))
+    T = int(min(cap, 8192, max(probe_T, probe_T * target_s / max(dt, 1e-6))))
     dt = run(T)
-    return T / dt, threads, f"first {T} tokens of the T=8192 layer, all 48 V heads", dt
+    what = {1: "the T=8192 layer", 2: "the T=262,144 sequence (mean alpha 0.98)",
+            4: "the first packed sequence, with initial and conv state"}[idx]
+    return T / dt, threads, f"first {T} tokens of {what}, all 48 V heads, {threads} thread(s)", dt
+
+
+def cpu_baseline(idx, target_s, n_threads=None):
+    v, threads, sample, dt = oracle_tokens_per_s(target_s, idx, n_threads)
+    return {"value": v, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": sample, "seconds": dt}
+
+
+def headline_config(world):
+    """`config` of the JSON line: the headline prefill workload (both arms print the same)."""
+    return {"workload": gi.WORKLOADS[1]["name"], "T": 8192, "n_qk_heads": 16, "n_v_heads": 48, "d": D,
+            "chunk": CHUNK, "inputs": "bf16", "out": "f32", "state": "f32",
+            "l2": "flushed: 256 MiB write between steps",
+            "parallelism": f"dp{world} (independent sequences per GPU)"}
 
 
 def run_reference(args):
@@ -700,8 +873,7 @@ def run_reference(args):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * statistics.median(secs),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic",
-        "config": {"workload": gi.WORKLOADS[1]["name"], "T": 8192, "n_qk_heads": 16,
-                   "n_v_heads": 48, "d": D, "sample": sample},
+        "config": headline_config(world),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -718,6 +890,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--decode-steps", type=int, default=1024)
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-long", action="store_true", help="skip the long-context and varlen prefill legs")
+    ap.add_argument("--long-steps", type=int, default=5, help="timed steps of those legs (at most --steps)")
     ap.add_argument("--no-qsa", action="store_true")
     ap.add_argument("--qsa-only", action="store_true", help="only the QSA indexer legs (profiling)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -739,10 +913,23 @@ def main():
             print(json.dumps({"metric": "QSA indexer query tokens/s", "qsa": qsa, "peaks": peak_src}), flush=True)
         dist.close()
         return
+    sha = kernel_sources_sha256()
     pre = bench_prefill(args, dist, torch, gdn, peaks)
-    roof = prefill_roofline(pre, peaks, peak_src)
+    roof = prefill_roofline(pre, peaks, peak_src, sha)
+    more = {}
+    if not args.no_long:
+        for idx, key in ((2, "prefill_longctx"), (4, "prefill_varlen")):
+            r = bench_prefill(args, dist, torch, gdn, peaks, idx=idx, e2e=False)
+            more[key] = {"value": r["value"], "unit": UNIT, "workload": r["workload"],
+                         "ms_per_step": r["ms_per_step"], "steps": r["steps"], "n_seqs": r["n_seqs"],
+                         "tokens_per_step": r["tokens_per_step"], "workspace_bytes": r["workspace_bytes"],
+                         "gpu_launches_per_step": r["launches"], "clocks": r["clocks"],
+                         "roofline": prefill_roofline(r, peaks, peak_src, sha),
+                         "step": prefill_step_summary(r, peaks), "kernels": r["per_kernel"]}
+            torch.cuda.empty_cache()
     dec = None if args.no_decode else bench_decode(args, dist, torch, gdn, peaks, peak_src)
     tail = bench_output_gate(args, dist, torch, gdn, peaks, peak_src)
+    gated = bench_prefill_gated(args, dist, torch, gdn, peaks)
     qsa = None
     if not args.no_qsa:
         qsa = {wl: bench_qsa(args, dist, torch, gdn, peaks, peak_src, wl) for wl in ("prefill", "decode")}
@@ -751,25 +938,24 @@ def main():
             qsa["cpu_baseline"] = {"value": v, "unit": QSA_UNIT, "cores": 1, "kind": "oracle",
                                    "sample": f"{n} query rows of qsa-prefill (block keys of the full context once)",
                                    "seconds": dt}
-    cpu = None
+    cpu = cpu1 = None
     if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
-        v, threads, sample, dt = oracle_tokens_per_s(args.cpu_baseline_s)
-        cpu = {"value": v, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": sample,
-               "seconds": dt}
+        cpu = cpu_baseline(1, args.cpu_baseline_s)
+        cpu1 = cpu_baseline(1, args.cpu_baseline_s / 2, n_threads=1)
+        for idx, key in ((2, "prefill_longctx"), (4, "prefill_varlen")):
+            if key in more:
+                more[key]["cpu_baseline"] = cpu_baseline(idx, args.cpu_baseline_s / 3)
     if dist.rank == 0:
         line = {
             "metric": METRIC, "value": pre["value"], "unit": UNIT, "n_gpus": dist.world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": pre["ms_per_step"],
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "tf32",
             "data": "synthetic",
-            "config": {"workload": gi.WORKLOADS[1]["name"], "T": 8192, "n_qk_heads": 16,
-                       "n_v_heads": 48, "d": D, "chunk": CHUNK, "inputs": "bf16",
-                       "out": "f32", "state": "f32", "l2": "flushed: 256 MiB write between steps",
-                       "parallelism": f"dp{dist.world} (independent sequences per GPU)"},
-            "clocks": pre["clocks"], "e2e": pre["e2e"], "gpu_launches": pre["launches"],
-            "roofline": roof, "kernels": pre["per_kernel"], "cpu_baseline": cpu, "decode": dec, "output_gate": tail,
-            "qsa": qsa,
-            "peaks": peak_src,
+            "config": headline_config(dist.world),
+            "clocks": pre["clocks"], "e2e": pre["e2e"], "gpu_launches": pre["launches"] * args.steps,
+            "roofline": roof, "step": prefill_step_summary(pre, peaks), "kernels": pre["per_kernel"],
+            "cpu_baseline": cpu, "cpu_baseline_1core": cpu1, **more,
+            "decode": dec, "output_gate": tail, "prefill_gated": gated, "qsa": qsa, "peaks": peak_src, "sources_sha256": sha,
         }
         print(json.dumps(line), flush=True)
     dist.close()

@@ -7,8 +7,9 @@
  *
  *   per token t of a sequence, raw rows q_t, k_t [Hqk, dk] and v_t [Hv, dv]:
  *     ShortConv   x'_t[c] = sum_{j=0..3} w[c][j] * x_{t-3+j}[c]   on every q, k, v channel
- *                 (causal, depthwise, tap 3 on the current row, no bias, no activation;
- *                  rows before the sequence start come from the conv state, else zero)
+ *                 (causal, depthwise, tap 3 on the current row, no bias; no activation
+ *                  unless cfg->conv_activation asks for SiLU; rows before the sequence
+ *                  start come from the conv state, else zero)
  *     L2 norm     q^ = q' * q_scale / sqrt(|q'|^2 + l2_eps),  k^ = k' / sqrt(|k'|^2 + l2_eps)
  *                 per (token, QK head); v^ = v'
  *   per value head h, reading QK head g = h / (Hv / Hqk), with state S [dk][dv] (fp32):
@@ -19,8 +20,12 @@
  *
  * Conventions shared by every entry point
  *  - Ownership: every buffer is a DEVICE pointer owned by the caller.  The library
- *    allocates nothing and keeps no mutable global state; calls on different streams
- *    are independent as long as their buffers do not overlap.
+ *    allocates no device memory for its data and calls on different streams are
+ *    independent as long as their buffers do not overlap, with two exceptions, each
+ *    described at its entry point: gdn_prefill keeps one auxiliary stream and five events
+ *    per (host thread, device) for its chunk ranges (see "Auxiliary stream" there), and
+ *    gdn_prefill_static_scratch shares one library-owned scratch array among all its
+ *    calls on a device (see "Sharing" there).
  *  - Asynchrony: every call only enqueues work on `stream` (0 = legacy default stream)
  *    and returns; nothing synchronises.  Kernel faults surface at the caller's next
  *    synchronisation.
@@ -45,7 +50,7 @@
 extern "C" {
 #endif
 
-#define GDN_API_VERSION 1
+#define GDN_API_VERSION 2
 
 #if defined(__GNUC__)
 #define GDN_EXPORT __attribute__((visibility("default")))
@@ -73,6 +78,11 @@ typedef enum {
  * 2^-9 of their magnitude, which on typical data is 2-3% of rms(y); use
  * out_dtype = GDN_F32 where y must stay within 1e-2 of rms(y) of the exact result. */
 
+/* Activation of the ShortConv outputs (gdn_config.conv_activation).  The page names none
+ * (GDN_ACT_NONE, the default reading); GDN_ACT_SILU applies SiLU(x) = x / (1 + e^-x) to every
+ * conv output of q, k and v, before the L2 normalisation of q and k. */
+typedef enum { GDN_ACT_NONE = 0, GDN_ACT_SILU = 1 } gdn_activation;
+
 typedef struct {
     int n_qk_heads;   /* Hqk: QK heads (16 in the pages' layer)                      */
     int n_v_heads;    /* Hv: value heads (48); V head h reads QK head h/(Hv/Hqk)     */
@@ -81,6 +91,7 @@ typedef struct {
     int conv_width;   /* ShortConv kernel size, must be 4                            */
     float q_scale;    /* multiplies q^ after normalisation (1.0: the page has none)  */
     float l2_eps;     /* epsilon inside the L2 norm's square root (1e-6)             */
+    int conv_activation;  /* gdn_activation of the conv outputs (GDN_ACT_NONE)       */
 } gdn_config;
 
 /* Human-readable name of a status code (static storage, never NULL). */
@@ -93,14 +104,22 @@ GDN_EXPORT int gdn_last_cuda_error(void);
 GDN_EXPORT int gdn_api_version(void);
 
 /*
- * gdn_prefill_workspace_size -- bytes of device workspace that gdn_prefill needs
- * for `total_tokens` tokens packed into `n_seqs` sequences.  Writes *bytes.
- * The workspace holds the clamped sequence table, the per-sequence chunk offsets
- * and the convolved, normalised q^, k^, v^ rows in fp32; it is scratch only (no
- * state persists between calls) and must not be shared by two calls in flight.
+ * gdn_prefill_workspace_size -- bytes of device workspace that gdn_prefill prefers for
+ * `total_tokens` tokens packed into `n_seqs` sequences, the longest of which has at most
+ * `max_seqlen` tokens (0 = not known: total_tokens).  Writes *bytes.
+ * The workspace is scratch only (no state persists between calls) and must not be shared
+ * by two calls in flight.  For bf16 input it holds the sequence tables and the per-chunk
+ * tiles of the tensor-core path for one or two chunk RANGES: range r covers chunks
+ * [r*R, (r+1)*R) of every sequence (R chosen from n_seqs and max_seqlen), so its size grows
+ * with n_seqs * R, not with total_tokens (about 4.6 MB per (sequence, chunk slot) at 16 QK /
+ * 48 V heads, plus one fp32 state per (sequence, V head) carried between ranges).  Only when
+ * one range covers the whole problem is it sized by the number of chunks instead.  For fp32
+ * input (the fp32 CUDA-core path) it holds the convolved, normalised rows in fp32 (40 KB per
+ * token at 16 QK / 48 V heads).
  */
 GDN_EXPORT gdn_status gdn_prefill_workspace_size(const gdn_config *cfg, gdn_dtype dtype,
-                                      int64_t total_tokens, int n_seqs, size_t *bytes);
+                                      int64_t total_tokens, int n_seqs, int64_t max_seqlen,
+                                      size_t *bytes);
 
 /*
  * gdn_prefill -- the mixer over packed variable-length sequences (chunked prefill).
@@ -120,24 +139,64 @@ GDN_EXPORT gdn_status gdn_prefill_workspace_size(const gdn_config *cfg, gdn_dtyp
  *                   sequences are allowed (their final state equals the initial one).
  *                   Out-of-order values are clamped on the device, never dereferenced.
  *   total_tokens    T (>= 0, < 2^31)
+ *   max_seqlen      an upper bound of the longest sequence's length, known on the host
+ *                   (0 = not known: T).  It sets how many chunk ranges the call launches;
+ *                   a sequence longer than the bound passed may get NaN for its tokens past
+ *                   the bound and for its final state (never anything else).
  *   initial_state   [n_seqs, Hv, 128(dk), 128(dv)] fp32, dv fastest; NULL = zero state
  *   final_state     same shape; NULL = not returned; may alias initial_state
  *   conv_state_in   [n_seqs, 3, 2*Hqk*128 + Hv*128] dtype: the last 3 raw rows
  *                   (q | k | v channels), oldest first; NULL = zero history
  *   conv_state_out  same shape; NULL = not returned; may alias conv_state_in
  *   out             [T, Hv, 128] out_dtype: y
- *   workspace       >= gdn_prefill_workspace_size() bytes, 256-byte aligned
+ *   workspace       256-byte aligned; gdn_prefill_workspace_size() bytes, or fewer: with
+ *                   bf16 input a smaller workspace makes the chunk ranges shorter (more of
+ *                   them, same results), down to one chunk per sequence per range;
+ *                   GDN_ERR_WORKSPACE when even that does not fit
  * Returns GDN_OK after enqueueing; n_seqs == 0 or T == 0 with no states is a no-op.
+ * Auxiliary stream: a bf16 call with more than one chunk range makes the tiles of range
+ * r+1 on an auxiliary stream while the chains of range r run on `stream` (events order the
+ * two).  The stream and five events are created by the first such call of a host thread on
+ * a device (make it before any stream capture on that device) and kept until the process
+ * exits.  Such calls of one host thread share that stream, so their tile work runs in
+ * call order even when the calls use different streams.
  */
 GDN_EXPORT gdn_status gdn_prefill(const gdn_config *cfg, gdn_dtype dtype, gdn_dtype out_dtype,
                        const void *q, const void *k, const void *v,
                        const float *conv_w_q, const float *conv_w_k, const float *conv_w_v,
                        const void *alpha, const void *beta,
                        const int32_t *cu_seqlens, int n_seqs, int64_t total_tokens,
+                       int64_t max_seqlen,
                        const float *initial_state, float *final_state,
                        const void *conv_state_in, void *conv_state_out,
                        void *out, void *workspace, size_t workspace_bytes,
                        cudaStream_t stream);
+
+/*
+ * gdn_prefill_gated -- gdn_prefill with the mixer's output tail fused into the store of y
+ * (page "ARCHITECTURE PREVIEW / FIELD NOTES", section 03, GDN figure caption: the readout
+ * passes a normalisation and an output gate before the output projection; the page gives no
+ * formula, this is the plainest reading, the same as gdn_output_gate's):
+ *     out_t = y_t / sqrt(mean(y_t^2) + norm_eps) * norm_w * SiLU(z_t)   per (token, V head)
+ * y never reaches memory.  Arguments as gdn_prefill, plus
+ *   z         [T, Hv, 128] z_dtype: the output-gate input, 16-byte aligned
+ *   norm_w    [128] fp32 (shared by the V heads), 16-byte aligned
+ *   norm_eps  >= 0, finite
+ *   out       [T, Hv, 128] out_dtype: the gated output
+ * With fp32 input (the fp32 CUDA-core path) y is first written to `out` and the tail then
+ * runs in place, so out_dtype must be GDN_F32 there (GDN_ERR_UNSUPPORTED otherwise).
+ */
+GDN_EXPORT gdn_status gdn_prefill_gated(const gdn_config *cfg, gdn_dtype dtype, gdn_dtype out_dtype,
+                             const void *q, const void *k, const void *v,
+                             const float *conv_w_q, const float *conv_w_k, const float *conv_w_v,
+                             const void *alpha, const void *beta,
+                             const int32_t *cu_seqlens, int n_seqs, int64_t total_tokens,
+                             int64_t max_seqlen,
+                             const float *initial_state, float *final_state,
+                             const void *conv_state_in, void *conv_state_out,
+                             const void *z, gdn_dtype z_dtype, const float *norm_w, float norm_eps,
+                             void *out, void *workspace, size_t workspace_bytes,
+                             cudaStream_t stream);
 
 /*
  * gdn_decode_step -- one token for each of `batch` sequences whose states stay
@@ -217,6 +276,27 @@ GDN_EXPORT gdn_status gdn_output_gate(const gdn_config *cfg, gdn_dtype y_dtype, 
                            float eps, void *out, int64_t n_tokens, cudaStream_t stream);
 
 /*
+ * gdn_affine_combine -- the states entering consecutive spans of one sequence, from the
+ * spans' affine maps (the prefix combination of a context-parallel prefill).
+ *
+ * Page "ARCHITECTURE PREVIEW / FIELD NOTES", section 03 (GATED DELTANET equations): the
+ * recurrence is affine in the state, so over a span of tokens, per V head,
+ * S_out = M S_in + B, with M [dk x dk] the product of the span's per-token maps
+ * alpha_t (I - beta_t k_t k_t^T) (gdn_prefill's final state for the span's keys and gates,
+ * zero values and zero value history, from the identity state) and B the state the span
+ * leaves from zero (its final state from a zero state).  This call computes
+ *     S_in[0] = S0,   S_in[p+1] = M[p] S_in[p] + B[p],   p = 0 .. n_spans-1
+ *   M, B    [n_spans, Hv, 128, 128] fp32 (row index first, as states are stored)
+ *   S0      [Hv, 128, 128] fp32, or NULL for a zero state
+ *   S_in    [n_spans + 1, Hv, 128, 128] fp32 out: entry p is the state entering span p,
+ *           entry n_spans the state after the last span; must not overlap M, B or S0
+ * fp32 arithmetic.  Only cfg->n_v_heads and the head dims (128) are used.  All pointers
+ * 16-byte aligned.
+ */
+GDN_EXPORT gdn_status gdn_affine_combine(const gdn_config *cfg, const float *M, const float *B, int n_spans,
+                                         const float *S0, float *S_in, cudaStream_t stream);
+
+/*
  * gdn_prefill_static_scratch -- gdn_prefill without a caller-supplied workspace.
  *
  * No counterpart on the pages: it exists for callers that cannot call cudaMalloc
@@ -227,13 +307,18 @@ GDN_EXPORT gdn_status gdn_output_gate(const gdn_config *cfg, gdn_dtype y_dtype, 
  * of GDN_STATIC_SCRATCH_BYTES in device memory owned by the library: one copy on each
  * GPU where the library's module holding it is loaded (with CUDA's default lazy module
  * loading, the GPUs on which this entry point is used), kept until the process exits.
- *  - Limit: problems whose gdn_prefill_workspace_size() exceeds GDN_STATIC_SCRATCH_BYTES
- *    are rejected with GDN_ERR_WORKSPACE before anything is enqueued (at 16 QK / 48 V
- *    heads that is roughly 750 tokens per call for bf16 input, 1,600 for fp32 input).
+ *  - Limit: the call runs gdn_prefill in GDN_STATIC_SCRATCH_BYTES of workspace, with chunk
+ *    ranges as long as fit (longer inputs just take more ranges).  Problems that do not fit
+ *    even with one chunk per sequence per range are rejected with GDN_ERR_WORKSPACE on the
+ *    host, before anything is looked up or enqueued: at 16 QK / 48 V heads, bf16 input,
+ *    a call takes up to 8 sequences of any length; fp32 input needs 40 KB per token
+ *    (about 1,600 tokens per call).
  *  - Allocation: none; it calls no cudaMalloc, cudaFree or allocating library routine.
  *  - Set-up: the first call on each device (with that device current) looks up the
- *    array's device address with cudaGetSymbolAddress; make that first call before any
- *    stream capture on that device.
+ *    array's device address with cudaGetSymbolAddress; a first call that takes more than
+ *    one chunk range also creates gdn_prefill's auxiliary stream and events of the host
+ *    thread (see gdn_prefill).  Make the first call before any stream capture on that
+ *    device.
  *  - Sharing: every call on a device uses the same array, which keeps whatever the last
  *    call left in it (no byte of it needs to start at zero).  Calls whose work overlaps
  *    on the GPU (different streams, or different host threads) race on the array: order

@@ -19,7 +19,7 @@ import torch
 from . import _native
 from ._native import GDN_BF16, GDN_F32, GdnError  # noqa: F401
 
-__all__ = ["GdnConfig", "gdn_prefill", "gdn_decode_step", "gdn_decode_multi", "gdn_output_gate", "prefill_workspace_size", "GdnError",
+__all__ = ["GdnConfig", "affine_combine", "gdn_prefill", "gdn_decode_step", "gdn_decode_multi", "gdn_output_gate", "prefill_workspace_size", "GdnError",
            "library_path", "qsa_block_keys", "qsa_block_scores", "qsa_select", "qsa_select_workspace_size",
            "QSA_BUDGET", "QSA_TOKEN_SLOTS"]
 
@@ -33,10 +33,11 @@ class GdnConfig:
     conv_width: int = 4
     q_scale: float = 1.0
     l2_eps: float = 1e-6
+    conv_activation: int = 0     # 0: none (the page names none), 1: SiLU on the conv outputs
 
     def c(self) -> _native.GdnConfigC:
         return _native.GdnConfigC(self.n_qk_heads, self.n_v_heads, self.d_k, self.d_v,
-                                  self.conv_width, self.q_scale, self.l2_eps)
+                                  self.conv_width, self.q_scale, self.l2_eps, self.conv_activation)
 
     @property
     def channels(self) -> int:
@@ -70,12 +71,14 @@ def _stream(stream) -> ctypes.c_void_p:
     return ctypes.c_void_p(s.cuda_stream)
 
 
-def prefill_workspace_size(cfg: GdnConfig, dtype: torch.dtype, total_tokens: int, n_seqs: int) -> int:
+def prefill_workspace_size(cfg: GdnConfig, dtype: torch.dtype, total_tokens: int, n_seqs: int,
+                           max_seqlen: int | None = None) -> int:
+    """Preferred workspace bytes of gdn_prefill (``max_seqlen``: bound of the longest sequence)."""
     n = ctypes.c_size_t(0)
     code = GDN_BF16 if dtype == torch.bfloat16 else GDN_F32
     c = cfg.c()
     _native.check("gdn_prefill_workspace_size", _native.lib().gdn_prefill_workspace_size(
-        ctypes.byref(c), code, int(total_tokens), int(n_seqs), ctypes.byref(n)))
+        ctypes.byref(c), code, int(total_tokens), int(n_seqs), int(max_seqlen or 0), ctypes.byref(n)))
     return int(n.value)
 
 
@@ -83,8 +86,13 @@ def gdn_prefill(q, k, v, conv_w_q, conv_w_k, conv_w_v, alpha, beta, cu_seqlens, 
                 cfg: GdnConfig | None = None, initial_state=None, final_state=None,
                 return_final_state: bool = True, conv_state_in=None, conv_state_out=None,
                 return_conv_state: bool = False, out=None, out_dtype=torch.float32,
-                workspace=None, stream=None):
+                workspace=None, max_seqlen: int | None = None, gate=None, stream=None):
     """Chunked prefill over packed sequences.  Returns (out, final_state, conv_state_out).
+
+    ``max_seqlen`` is a host-side upper bound of the longest sequence (None: the total); with
+    many sequences it lets the chunk ranges stay short, so the workspace stays small.
+    ``gate`` = (z, norm_w, norm_eps) fuses the output tail into the store of y:
+    out = y / sqrt(mean(y^2) + norm_eps) * norm_w * SiLU(z) per (token, V head).
 
     q, k [T, Hqk, 128], v [T, Hv, 128], alpha/beta [T, Hv] (bf16 or fp32, one dtype);
     conv_w_* fp32 [channels, 4]; cu_seqlens int32 [N+1] on the device;
@@ -109,16 +117,22 @@ def gdn_prefill(q, k, v, conv_w_q, conv_w_k, conv_w_v, alpha, beta, cu_seqlens, 
     if conv_state_out is None and return_conv_state:
         conv_state_out = torch.empty((n, cfg.conv_width - 1, cfg.channels), dtype=q.dtype,
                                      device=dev)
-    need = prefill_workspace_size(cfg, q.dtype, T, n)
+    need = prefill_workspace_size(cfg, q.dtype, T, n, max_seqlen)
     if workspace is None:
         workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
     c = cfg.c()
-    st = _native.lib().gdn_prefill(
-        ctypes.byref(c), code, _dtype_code(out), _ptr(q), _ptr(k), _ptr(v), _ptr(conv_w_q), _ptr(conv_w_k),
-        _ptr(conv_w_v), _ptr(alpha), _ptr(beta), _ptr(cu_seqlens), n, T, _ptr(initial_state),
-        _ptr(final_state), _ptr(conv_state_in), _ptr(conv_state_out), _ptr(out), _ptr(workspace),
-        workspace.numel() * workspace.element_size(), _stream(stream))
-    _native.check("gdn_prefill", st)
+    common = (ctypes.byref(c), code, _dtype_code(out), _ptr(q), _ptr(k), _ptr(v), _ptr(conv_w_q), _ptr(conv_w_k),
+              _ptr(conv_w_v), _ptr(alpha), _ptr(beta), _ptr(cu_seqlens), n, T, int(max_seqlen or 0),
+              _ptr(initial_state), _ptr(final_state), _ptr(conv_state_in), _ptr(conv_state_out))
+    tail = (_ptr(out), _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream))
+    if gate is None:
+        _native.check("gdn_prefill", _native.lib().gdn_prefill(*common, *tail))
+    else:
+        z, norm_w, norm_eps = gate
+        if z.shape != out.shape:
+            raise ValueError("z must have the shape of the output")
+        _native.check("gdn_prefill_gated", _native.lib().gdn_prefill_gated(
+            *common, _ptr(z), _dtype_code(z), _ptr(norm_w), float(norm_eps), *tail))
     return out, final_state, conv_state_out
 
 
@@ -207,6 +221,24 @@ def gdn_output_gate(y, z, norm_w, *, eps: float = 1e-6, cfg: GdnConfig | None = 
                                        _ptr(y), _ptr(z), _ptr(norm_w), float(eps), _ptr(out), n_tokens,
                                        _stream(stream))
     _native.check("gdn_output_gate", st)
+    return out
+
+
+def affine_combine(M, B, S0=None, *, cfg: GdnConfig | None = None, out=None, stream=None):
+    """States entering consecutive spans of one sequence from the spans' affine maps
+    (S_out = M S_in + B per V head): out[0] = S0 (zero if None), out[p+1] = M[p] out[p] + B[p].
+    M, B fp32 [P, Hv, 128, 128]; returns fp32 [P + 1, Hv, 128, 128]."""
+    if M.dtype != torch.float32 or B.dtype != torch.float32 or M.shape != B.shape or M.dim() != 4:
+        raise ValueError("M and B must be fp32 [P, Hv, 128, 128] of one shape")
+    P, Hv = M.shape[0], M.shape[1]
+    cfg = cfg or GdnConfig(n_qk_heads=1, n_v_heads=Hv)
+    if out is None:
+        out = torch.empty((P + 1,) + tuple(M.shape[1:]), dtype=torch.float32, device=M.device)
+    if S0 is not None and (S0.dtype != torch.float32 or tuple(S0.shape) != tuple(M.shape[1:])):
+        raise ValueError("S0 must be fp32 [Hv, 128, 128]")
+    c = cfg.c()
+    _native.check("gdn_affine_combine", _native.lib().gdn_affine_combine(
+        ctypes.byref(c), _ptr(M), _ptr(B), P, _ptr(S0), _ptr(out), _stream(stream)))
     return out
 
 

@@ -19,8 +19,8 @@ STATUS = {0: "GDN_OK", 1: "GDN_ERR_INVALID_ARG", 2: "GDN_ERR_UNSUPPORTED", 3: "G
 
 # every entry point the header declares (checked by the CPU test suite)
 EXPORTS = ("gdn_status_string", "gdn_last_cuda_error", "gdn_api_version",
-           "gdn_prefill_workspace_size", "gdn_prefill", "gdn_decode_step", "gdn_decode_multi",
-           "gdn_output_gate", "gdn_trace_begin",
+           "gdn_prefill_workspace_size", "gdn_prefill", "gdn_prefill_gated", "gdn_decode_step", "gdn_decode_multi",
+           "gdn_output_gate", "gdn_affine_combine", "gdn_trace_begin",
            "gdn_trace_end", "gdn_prefill_static_scratch", "gdn_qsa_block_keys",
            "gdn_qsa_block_scores", "gdn_qsa_select_workspace_size", "gdn_qsa_select")
 
@@ -34,7 +34,7 @@ class TraceEntryC(ctypes.Structure):
 class GdnConfigC(ctypes.Structure):
     _fields_ = [("n_qk_heads", ctypes.c_int), ("n_v_heads", ctypes.c_int), ("d_k", ctypes.c_int),
                 ("d_v", ctypes.c_int), ("conv_width", ctypes.c_int), ("q_scale", ctypes.c_float),
-                ("l2_eps", ctypes.c_float)]
+                ("l2_eps", ctypes.c_float), ("conv_activation", ctypes.c_int)]
 
 
 class GdnError(RuntimeError):
@@ -69,14 +69,19 @@ def lib():
             L.gdn_api_version.argtypes = []
             L.gdn_api_version.restype = ctypes.c_int
             L.gdn_prefill_workspace_size.argtypes = [ctypes.POINTER(GdnConfigC), ctypes.c_int,
-                                                     ctypes.c_int64, ctypes.c_int,
+                                                     ctypes.c_int64, ctypes.c_int, ctypes.c_int64,
                                                      ctypes.POINTER(ctypes.c_size_t)]
             L.gdn_prefill_workspace_size.restype = ctypes.c_int
             L.gdn_prefill.argtypes = [ctypes.POINTER(GdnConfigC), ctypes.c_int, ctypes.c_int, vp, vp,
                                       vp, fp, fp,
-                                      fp, vp, vp, i32p, ctypes.c_int, ctypes.c_int64, fp, fp, vp,
-                                      vp, vp, vp, ctypes.c_size_t, vp]
+                                      fp, vp, vp, i32p, ctypes.c_int, ctypes.c_int64, ctypes.c_int64,
+                                      fp, fp, vp, vp, vp, vp, ctypes.c_size_t, vp]
             L.gdn_prefill.restype = ctypes.c_int
+            L.gdn_prefill_gated.argtypes = [ctypes.POINTER(GdnConfigC), ctypes.c_int, ctypes.c_int, vp, vp, vp,
+                                            fp, fp, fp, vp, vp, i32p, ctypes.c_int, ctypes.c_int64,
+                                            ctypes.c_int64, fp, fp, vp, vp, vp, ctypes.c_int, fp,
+                                            ctypes.c_float, vp, vp, ctypes.c_size_t, vp]
+            L.gdn_prefill_gated.restype = ctypes.c_int
             L.gdn_decode_step.argtypes = [ctypes.POINTER(GdnConfigC), ctypes.c_int, ctypes.c_int, vp,
                                           vp, vp, fp,
                                           fp, fp, vp, vp, fp, vp, i32p, ctypes.c_int, vp,
@@ -89,6 +94,8 @@ def lib():
             L.gdn_output_gate.argtypes = [ctypes.POINTER(GdnConfigC), ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                           vp, vp, fp, ctypes.c_float, vp, ctypes.c_int64, vp]
             L.gdn_output_gate.restype = ctypes.c_int
+            L.gdn_affine_combine.argtypes = [ctypes.POINTER(GdnConfigC), fp, fp, ctypes.c_int, fp, fp, vp]
+            L.gdn_affine_combine.restype = ctypes.c_int
             L.gdn_trace_begin.argtypes = [ctypes.POINTER(TraceEntryC), ctypes.c_int]
             L.gdn_trace_begin.restype = None
             L.gdn_trace_end.argtypes = []

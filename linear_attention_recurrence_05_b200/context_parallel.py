@@ -12,12 +12,14 @@ a prefill of the same keys and gates with zero values from the identity state (t
 S_out = M I + 0).  Combining the maps of the spans before it gives a span's true entering
 state, and one more prefill from that state gives the span's outputs.
 
-Two drivers share that arithmetic: ``cp_prefill`` runs the spans of a process group's ranks
+Two drivers share that plan: ``cp_prefill`` runs the spans of a process group's ranks
 (one span each; one all-gather of 2 x Hv x 128 x 128 fp32 per rank is the only exchange),
 ``cp_prefill_spans`` runs a list of spans one after another in one process.  Both take the
-prefill as a callable with the signature of :func:`gdn_prefill` (the default), the span
-boundaries of one sequence, and return each span's outputs and final state.  The
-sequence's conv history is carried between spans as the 3 raw rows before each span.
+prefill as a callable with the signature of :func:`gdn_prefill` (the default) and the
+combination of the maps as a callable with the signature of :func:`affine_combine` (the
+default; both run in libgdn), and return each span's outputs and final state.  This module
+itself only moves data: the sequence's conv history is carried between spans as the 3 raw
+rows before each span.
 """
 from __future__ import annotations
 
@@ -55,12 +57,17 @@ def span_affine_map(prefill, q, k, v, w, alpha, beta, *, cfg, conv_rows=None):
     return M[0], B[0]
 
 
-def combine_prefix(Ms, Bs, S0):
-    """Entering states of spans 0..P-1: S_0 = S0, S_{p+1} = M_p S_p + B_p (per V head)."""
-    S = [S0.to(Ms[0].dtype)]
-    for M, B in zip(Ms[:-1], Bs[:-1]):
-        S.append(torch.matmul(M, S[-1]) + B)
-    return S
+def combine_prefix(Ms, Bs, S0, combine=None):
+    """Entering states of spans 0..P-1: S_0 = S0, S_{p+1} = M_p S_p + B_p (per V head), by
+    ``combine`` (default: libgdn's gdn_affine_combine)."""
+    if combine is None:
+        from . import affine_combine as combine
+    def stacked(xs):
+        if len(xs) > 1:
+            return torch.stack(xs[:-1]).contiguous()
+        return torch.empty((0,) + tuple(S0.shape), dtype=S0.dtype, device=S0.device)
+    S = combine(stacked(Ms), stacked(Bs), S0.contiguous())
+    return list(S.unbind(0))
 
 
 def _last_rows(x_q, x_k, x_v, prev_rows, n=3):
@@ -74,7 +81,7 @@ def _last_rows(x_q, x_k, x_v, prev_rows, n=3):
     return cur[-n:]
 
 
-def cp_prefill_spans(spans, w, *, cfg, initial_state=None, conv_state=None, prefill=None):
+def cp_prefill_spans(spans, w, *, cfg, initial_state=None, conv_state=None, prefill=None, combine=None):
     """Spans of one sequence in one process.  ``spans``: list of (q, k, v, alpha, beta) of
     consecutive pieces; ``initial_state`` [Hv, 128, 128] or None; ``conv_state`` [3, channels]
     raw rows before the sequence or None.  Returns (list of y per span, final state)."""
@@ -89,7 +96,7 @@ def cp_prefill_spans(spans, w, *, cfg, initial_state=None, conv_state=None, pref
     dev = spans[0][0].device
     S0 = initial_state if initial_state is not None else torch.zeros(
         (cfg.n_v_heads, cfg.d_k, cfg.d_v), dtype=torch.float32, device=dev)
-    S_in = combine_prefix([m for m, _ in maps], [b for _, b in maps], S0)
+    S_in = combine_prefix([m for m, _ in maps], [b for _, b in maps], S0, combine)
     ys, fin = [], None
     for (q, k, v, a, b), rw, S in zip(spans, rows, S_in):
         y, f, _ = prefill(q, k, v, *w, a, b, _one(dev, q.shape[0]), cfg=cfg,
@@ -101,7 +108,7 @@ def cp_prefill_spans(spans, w, *, cfg, initial_state=None, conv_state=None, pref
 
 
 def cp_prefill(q, k, v, w, alpha, beta, *, cfg, group=None, initial_state=None, conv_state=None,
-               prefill=None):
+               prefill=None, combine=None):
     """This rank's span of one sequence (rank order = sequence order).  ``initial_state`` and
     ``conv_state`` are the sequence's (only rank 0's are used).  One all-gather carries every
     span's (M, B) and last raw rows.  Returns (y of this span, final state of the sequence
@@ -134,7 +141,7 @@ def cp_prefill(q, k, v, w, alpha, beta, *, cfg, group=None, initial_state=None, 
         S0 = initial_state.to(torch.float32)
     src = torch.stack([S0]) if rank == 0 else torch.empty((1, Hv, d, d), dtype=torch.float32, device=dev)
     dist.broadcast(src, 0, group=group)   # the sequence's initial state, from rank 0
-    S = combine_prefix([g[0] for g in got[:rank + 1]], [g[1] for g in got[:rank + 1]], src[0])[rank]
+    S = combine_prefix([g[0] for g in got[:rank + 1]], [g[1] for g in got[:rank + 1]], src[0], combine)[rank]
     y, fin, _ = prefill(q, k, v, *w, alpha, beta, _one(dev, q.shape[0]), cfg=cfg,
                         initial_state=S.unsqueeze(0).contiguous(),
                         conv_state_in=None if conv_rows is None else conv_rows.unsqueeze(0))

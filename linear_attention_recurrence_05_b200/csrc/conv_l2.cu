@@ -11,6 +11,7 @@
 
 #include "gdn_common.cuh"
 #include "gdn_internal.h"
+#include "chunk_range.cuh"
 #include "tc_sm100.cuh"
 #include "tma_map.cuh"
 
@@ -93,7 +94,7 @@ cudaError_t launch_seq_table(const int32_t *cu_in, int n_seqs, int64_t T, int32_
 template <class T>
 __global__ void __launch_bounds__(128) conv_l2_kernel(ConvParams p) {
     const int n_chunks = p.cfirst[p.n_seqs];
-    const int ci = (int)(p.chunk_lo + blockIdx.x);
+    const int ci = (int)blockIdx.x;
     if (ci >= n_chunks) return;
     const int b = upper_index(p.cfirst, p.n_seqs, ci);
     const int seq0 = p.cu[b], seq1 = p.cu[b + 1];
@@ -151,7 +152,8 @@ __global__ void __launch_bounds__(128) conv_l2_kernel(ConvParams p) {
         float ss = 0.f;
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
-            y[c] = wt[c][0] * h[0][c] + wt[c][1] * h[1][c] + wt[c][2] * h[2][c] + wt[c][3] * cur[c];
+            y[c] = conv_act(wt[c][0] * h[0][c] + wt[c][1] * h[1][c] + wt[c][2] * h[2][c] + wt[c][3] * cur[c],
+                            p.act);
             ss += y[c] * y[c];
             h[0][c] = h[1][c]; h[1][c] = h[2][c]; h[2][c] = cur[c];
         }
@@ -193,7 +195,8 @@ struct ConvTileParams {
     const int32_t *cu, *cfirst;
     int n_seqs, n_qk, n_v;
     float q_scale, eps;
-    int64_t chunk_lo;
+    int act;
+    ChunkRange rg;
 };
 
 // largest b in [0, n) with first[b] <= i (first non-decreasing, first[0] <= i < first[n]),
@@ -223,15 +226,20 @@ __device__ __forceinline__ void bf16x4_to_f32(uint2 r, float v[4]) {
 }  // namespace
 
 __global__ void __launch_bounds__(128) conv_tiles_kernel(const __grid_constant__ ConvTileParams p) {
-    const int n_chunks = p.cfirst[p.n_seqs];
-    const int ci = (int)(p.chunk_lo + blockIdx.x);
-    if (ci >= n_chunks) return;
+    const int64_t ci = blockIdx.x;   // slot of the range
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-    const int b = upper_index_warp(p.cfirst, p.n_seqs, ci);
+    int b, jc;
+    if (p.rg.compact) {
+        if (ci >= p.cfirst[p.n_seqs]) return;   // uniform per CTA
+        b = upper_index_warp(p.cfirst, p.n_seqs, (int)ci);
+        jc = (int)ci - p.cfirst[b];
+        if (blockIdx.y == 0 && threadIdx.x == 0) p.cseq[ci] = b;   // for the chunk-prep pass
+    } else if (!sliced_slot_chunk(p.rg, ci, p.cfirst, &b, &jc)) {
+        return;   // uniform per CTA
+    }
     const int seq0 = p.cu[b], seq1 = p.cu[b + 1];
-    const int r0 = (ci - p.cfirst[b]) * kChunk;   // chunk start within the sequence
+    const int r0 = jc * kChunk;   // chunk start within the sequence
     const int len = min(kChunk, seq1 - seq0 - r0);
-    if (blockIdx.y == 0 && threadIdx.x == 0) p.cseq[ci] = b;   // for the chunk-prep pass
 
     // slot kinds: 0 q ([K;Q] Q half), 1 k ([K;Q] K half + K tile), 3 v (V tile)
     const int slot = blockIdx.y, nq = p.n_qk;
@@ -286,7 +294,8 @@ __global__ void __launch_bounds__(128) conv_tiles_kernel(const __grid_constant__
         float ss = 0.f;
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
-            y[c] = wt[c][0] * h[0][c] + wt[c][1] * h[1][c] + wt[c][2] * h[2][c] + wt[c][3] * cur[c];
+            y[c] = conv_act(wt[c][0] * h[0][c] + wt[c][1] * h[1][c] + wt[c][2] * h[2][c] + wt[c][3] * cur[c],
+                            p.act);
             ss += y[c] * y[c];
             h[0][c] = h[1][c]; h[1][c] = h[2][c]; h[2][c] = cur[c];
         }
@@ -335,8 +344,8 @@ cudaError_t launch_conv_l2(const ConvParams &p, bool bf16, bool tiles, int64_t n
             return cudaErrorInvalidValue;
         tp.wq = p.wq; tp.wk = p.wk; tp.wv = p.wv; tp.conv_in = p.conv_in;
         tp.kq = p.kq; tp.kmn = p.kmn; tp.vi = p.vi; tp.cseq = p.cseq; tp.cu = p.cu; tp.cfirst = p.cfirst;
-        tp.n_seqs = p.n_seqs; tp.n_qk = p.n_qk; tp.n_v = p.n_v; tp.q_scale = p.q_scale; tp.eps = p.eps;
-        tp.chunk_lo = p.chunk_lo;
+        tp.n_seqs = p.n_seqs; tp.n_qk = p.n_qk; tp.n_v = p.n_v; tp.q_scale = p.q_scale; tp.eps = p.eps; tp.act = p.act;
+        tp.rg = p.rg;
         cudaError_t e = cudaFuncSetAttribute(conv_tiles_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)kConvSmemAlloc);
         if (e != cudaSuccess) return e;

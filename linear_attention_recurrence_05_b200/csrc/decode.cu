@@ -63,7 +63,7 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(DecodeParams p) 
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
             float4 wt = *reinterpret_cast<const float4 *>(w + (int64_t)(wc + c) * kConvW);
-            y[c] = wt.x * hst[0][c] + wt.y * hst[1][c] + wt.z * hst[2][c] + wt.w * cur[c];
+            y[c] = conv_act(wt.x * hst[0][c] + wt.y * hst[1][c] + wt.z * hst[2][c] + wt.w * cur[c], p.act);
             ss += y[c] * y[c];
         }
         ss = warp_sum(ss);
@@ -103,7 +103,7 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(DecodeParams p) 
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
                 float4 wt = *reinterpret_cast<const float4 *>(p.wv + (int64_t)(wc + c) * kConvW);
-                y[c] = wt.x * hst[0][c] + wt.y * hst[1][c] + wt.z * hst[2][c] + wt.w * cur[c];
+                y[c] = conv_act(wt.x * hst[0][c] + wt.y * hst[1][c] + wt.z * hst[2][c] + wt.w * cur[c], p.act);
                 vs[4 * lane + c] = y[c];
             }
             if (cs) {
@@ -261,7 +261,8 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_multi_kernel(DecodePara
             float ss = 0.f;
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
-                y[c] = wt[c][0] * h[0][c] + wt[c][1] * h[1][c] + wt[c][2] * h[2][c] + wt[c][3] * cur[c];
+                y[c] = conv_act(wt[c][0] * h[0][c] + wt[c][1] * h[1][c] + wt[c][2] * h[2][c] + wt[c][3] * cur[c],
+                                p.act);
                 ss += y[c] * y[c];
                 h[0][c] = h[1][c]; h[1][c] = h[2][c]; h[2][c] = cur[c];
             }

@@ -36,7 +36,45 @@ TraceLaunch::~TraceLaunch() {
 
 static size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-PrefillLayout prefill_layout(int n_qk, int n_v, int64_t T, int n_seqs, bool tc) {
+// Carve the tile buffers for `slots` chunk slots, `n_buf` buffers, starting at `off`.
+static size_t carve_tiles(PrefillLayout &L, int n_qk, int n_v, int64_t slots, int n_buf, size_t off) {
+    const size_t ns = (size_t)slots;
+    size_t o = 0;
+    L.b_kq = o;   o = align_up(o + ns * n_qk * 65536, 256);
+    L.b_kmn = o;  o = align_up(o + ns * n_qk * 32768, 256);
+    L.b_vi = o;   o = align_up(o + ns * n_v * 32768, 256);
+    L.b_tb = o;   o = align_up(o + ns * n_v * 16384, 256);
+    L.b_pm = o;   o = align_up(o + ns * n_v * 16384, 256);
+    L.b_gr = o;   o = align_up(o + ns * n_v * kGateRec * sizeof(float), 256);
+    L.b_cseq = o; o = align_up(o + ns * sizeof(int32_t), 256);
+    L.buf_bytes = o;
+    L.off_tiles = off;
+    L.slots = slots;
+    L.n_buf = n_buf;
+    return off + (size_t)n_buf * o;
+}
+
+// The tensor-core layout for a given range plan: compact (one range over every chunk) or
+// sliced with R chunks per sequence per range and n_buf buffers.
+static void tc_layout(PrefillLayout &L, int n_qk, int n_v, int n_seqs, int64_t maxc, bool compact, int R,
+                      int n_buf, size_t off) {
+    if (compact) {
+        L.range0 = ChunkRange{1, 0, 0, 1};
+        L.n_ranges = 1;
+        off = carve_tiles(L, n_qk, n_v, L.max_chunks, 1, off);
+    } else {
+        L.range0 = ChunkRange{0, R, 0, 0};
+        L.n_ranges = (int)((maxc + R - 1) / R);
+        off = carve_tiles(L, n_qk, n_v, (int64_t)n_seqs * R, std::min(n_buf, L.n_ranges), off);
+    }
+    const size_t carry = L.n_ranges > 1 ? (size_t)n_seqs * n_v * 128 * 128 * sizeof(float) : 0;
+    L.off_carry = off;
+    off = align_up(off + carry, 256);
+    L.bytes = off;
+}
+
+bool prefill_layout(int n_qk, int n_v, int64_t T, int n_seqs, int64_t max_seqlen, bool tc, size_t ws_limit,
+                    PrefillLayout *out) {
     PrefillLayout L{};
     L.max_chunks = (T + kChunk - 1) / kChunk + n_seqs;
     size_t off = 0;
@@ -47,30 +85,59 @@ PrefillLayout prefill_layout(int n_qk, int n_v, int64_t T, int n_seqs, bool tc) 
     L.off_qh = off;      off = align_up(off + qk_bytes, 256);
     L.off_kh = off;      off = align_up(off + qk_bytes, 256);
     L.off_vh = off;      off = align_up(off + v_bytes, 256);
-    const size_t nc = tc && T > 0 ? (size_t)L.max_chunks : 0;
-    L.off_kq = off;      off = align_up(off + nc * n_qk * 65536, 256);
-    L.off_kmn = off;     off = align_up(off + nc * n_qk * 32768, 256);
-    L.off_vi = off;      off = align_up(off + nc * n_v * 32768, 256);
-    L.off_tb = off;      off = align_up(off + nc * n_v * 16384, 256);
-    L.off_pm = off;      off = align_up(off + nc * n_v * 16384, 256);
-    L.off_gr = off;      off = align_up(off + nc * n_v * kGateRec * sizeof(float), 256);
-    L.off_cseq = off;    off = align_up(off + nc * sizeof(int32_t), 256);
-    L.n_segments = tc && T > 0 ? plan_segments(n_v, n_seqs, L.max_chunks) : 1;
-    const size_t carry = L.n_segments > 1 ? (size_t)n_seqs * n_v * 128 * 128 * sizeof(float) : 0;
-    L.off_carry = off;   off = align_up(off + carry, 256);
-    L.bytes = off;
-    return L;
+    if (!tc || T == 0 || n_seqs == 0) {   // fp32 rows (one pass), or nothing to tile
+        L.range0 = ChunkRange{1, 0, 0, 1};
+        L.n_ranges = 1;
+        L.n_buf = 1;
+        L.off_tiles = L.off_carry = off;
+        L.bytes = off;
+        *out = L;
+        return L.bytes <= ws_limit;
+    }
+    // preferred plan: few chains -> ranges sized to overlap prep with the chains; many chains
+    // -> ranges that bound the tile memory while every sequence still advances in each range
+    const int64_t ms = (max_seqlen > 0 && max_seqlen < T) ? max_seqlen : T;
+    const int64_t maxc = (ms + kChunk - 1) / kChunk;
+    const bool few = (int64_t)n_seqs * n_v <= kFewChains;
+    int64_t R = few ? std::min<int64_t>(128, std::max<int64_t>(32, (maxc + 3) / 4))
+                    : std::min<int64_t>(64, std::max<int64_t>(8, 512 / n_seqs));
+    R = std::min(R, maxc);
+    const int64_t cap = max_seqlen > 0 ? kMaxRanges : kMaxRangesUnknown;
+    if ((maxc + R - 1) / R > cap) R = (maxc + cap - 1) / cap;
+    const int nr = (int)((maxc + R - 1) / R);
+    // one range, or many chains and no memory to save: global chunk numbering
+    const bool compact = nr == 1 || (!few && (int64_t)std::min(2, nr) * n_seqs * R >= L.max_chunks);
+    tc_layout(L, n_qk, n_v, n_seqs, maxc, compact, (int)std::min<int64_t>(R, INT32_MAX), 2, off);
+    if (L.bytes > ws_limit) {
+        // shrink the ranges to the workspace given: two buffers if one chunk per sequence fits
+        // twice, else one (range r+1 is then prepared after the chains of range r)
+        bool fit = false;
+        for (int nb = 2; nb >= 1 && !fit; --nb) {
+            const size_t per = (size_t)n_seqs * ((size_t)n_qk * 98304 + (size_t)n_v * (65536 + kGateRec * 4)) * nb;
+            const size_t avail = ws_limit > off ? ws_limit - off : 0;
+            int64_t r = std::min<int64_t>(R, (int64_t)(avail / per) + 1);
+            for (; r >= 1; --r) {
+                tc_layout(L, n_qk, n_v, n_seqs, maxc, false, (int)r, nb, off);
+                if (L.bytes <= ws_limit) { fit = true; break; }
+            }
+        }
+        if (!fit) {
+            *out = L;
+            return false;
+        }
+    }
+    *out = L;
+    return true;
 }
 
-int plan_segments(int n_v, int n_seqs, int64_t max_chunks) {
-    if ((int64_t)n_seqs * n_v > kSegMaxChains || max_chunks < 2 * kSegMinChunks) return 1;
-    return (int)std::min<int64_t>(kSegMax, max_chunks / kSegMinChunks);
-}
-
-// One auxiliary stream and a few events per (host thread, device) for the pipelined path.
+// One auxiliary stream and a few events per (host thread, device) for the chunk ranges:
+// created on the first multi-range prefill of the thread on that device, kept for the life
+// of the process.
 struct AuxStream {
     cudaStream_t stream = nullptr;
-    cudaEvent_t ev[kSegMax + 2] = {};
+    cudaEvent_t ev_tab = nullptr;       // sequence tables ready (caller's stream)
+    cudaEvent_t ev_prep[2] = {};        // tiles of the range in buffer i ready (auxiliary stream)
+    cudaEvent_t ev_chain[2] = {};       // chains done with buffer i (caller's stream)
 };
 static thread_local AuxStream t_aux[64];
 
@@ -82,12 +149,14 @@ static cudaError_t aux_stream(AuxStream **out) {
     AuxStream &a = t_aux[dev];
     if (!a.stream) {
         AuxStream fresh;
+        cudaEvent_t *evs[5] = {&fresh.ev_tab, &fresh.ev_prep[0], &fresh.ev_prep[1], &fresh.ev_chain[0],
+                               &fresh.ev_chain[1]};
         e = cudaStreamCreateWithFlags(&fresh.stream, cudaStreamNonBlocking);
-        for (auto &ev : fresh.ev)
-            if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ev, cudaEventDisableTiming);
+        for (auto *ev : evs)
+            if (e == cudaSuccess) e = cudaEventCreateWithFlags(ev, cudaEventDisableTiming);
         if (e != cudaSuccess) {
-            for (auto &ev : fresh.ev)
-                if (ev) cudaEventDestroy(ev);
+            for (auto *ev : evs)
+                if (*ev) cudaEventDestroy(*ev);
             if (fresh.stream) cudaStreamDestroy(fresh.stream);
             return e;
         }
@@ -115,6 +184,7 @@ static gdn_status check_config(const gdn_config *cfg, gdn_dtype dtype) {
     if (cfg->n_v_heads % cfg->n_qk_heads != 0) return GDN_ERR_INVALID_ARG;
     if (!std::isfinite(cfg->q_scale) || !std::isfinite(cfg->l2_eps) || cfg->l2_eps < 0.f)
         return GDN_ERR_INVALID_ARG;
+    if (cfg->conv_activation != GDN_ACT_NONE && cfg->conv_activation != GDN_ACT_SILU) return GDN_ERR_INVALID_ARG;
     if (cfg->d_k != 128 || cfg->d_v != 128 || cfg->conv_width != 4) return GDN_ERR_UNSUPPORTED;
     // keep channel counts and grid dimensions inside int range
     // grid dimensions: 2*Hqk + Hv head slots ride in gridDim.y (<= 65535)
@@ -167,28 +237,40 @@ int gdn_trace_end(void) {
 }
 
 gdn_status gdn_prefill_workspace_size(const gdn_config *cfg, gdn_dtype dtype, int64_t total_tokens,
-                                      int n_seqs, size_t *bytes) {
+                                      int n_seqs, int64_t max_seqlen, size_t *bytes) {
     gdn_status st = check_config(cfg, dtype);
     if (st != GDN_OK) return st;
-    if (!bytes || total_tokens < 0 || total_tokens >= ((int64_t)1 << 31) || n_seqs < 0)
+    if (!bytes || total_tokens < 0 || total_tokens >= ((int64_t)1 << 31) || n_seqs < 0 || max_seqlen < 0)
         return GDN_ERR_INVALID_ARG;
-    *bytes = prefill_layout(cfg->n_qk_heads, cfg->n_v_heads, total_tokens, n_seqs,
-                            dtype == GDN_BF16).bytes;
+    PrefillLayout L;
+    prefill_layout(cfg->n_qk_heads, cfg->n_v_heads, total_tokens, n_seqs, max_seqlen, dtype == GDN_BF16,
+                   SIZE_MAX, &L);
+    *bytes = L.bytes;
     return GDN_OK;
 }
 
-gdn_status gdn_prefill(const gdn_config *cfg, gdn_dtype dtype, gdn_dtype out_dtype,
-                       const void *q, const void *k,
-                       const void *v, const float *conv_w_q, const float *conv_w_k,
-                       const float *conv_w_v, const void *alpha, const void *beta,
-                       const int32_t *cu_seqlens, int n_seqs, int64_t total_tokens,
-                       const float *initial_state, float *final_state, const void *conv_state_in,
-                       void *conv_state_out, void *out, void *workspace, size_t workspace_bytes,
-                       cudaStream_t stream) {
+}  // extern "C"
+
+// gated output of gdn_prefill_gated (z == null: plain y)
+struct GateArgs {
+    const void *z = nullptr;
+    gdn_dtype z_dtype = GDN_BF16;
+    const float *w = nullptr;
+    float eps = 0.f;
+};
+
+static gdn_status prefill_impl(const gdn_config *cfg, gdn_dtype dtype, gdn_dtype out_dtype,
+                               const void *q, const void *k,
+                               const void *v, const float *conv_w_q, const float *conv_w_k,
+                               const float *conv_w_v, const void *alpha, const void *beta,
+                               const int32_t *cu_seqlens, int n_seqs, int64_t total_tokens, int64_t max_seqlen,
+                               const float *initial_state, float *final_state, const void *conv_state_in,
+                               void *conv_state_out, void *out, void *workspace, size_t workspace_bytes,
+                               const GateArgs &gate, cudaStream_t stream) {
     gdn_status st = check_config(cfg, dtype);
     if (st != GDN_OK) return st;
     if (out_dtype != GDN_BF16 && out_dtype != GDN_F32) return GDN_ERR_INVALID_ARG;
-    if (n_seqs < 0 || total_tokens < 0 || total_tokens >= ((int64_t)1 << 31))
+    if (n_seqs < 0 || total_tokens < 0 || total_tokens >= ((int64_t)1 << 31) || max_seqlen < 0)
         return GDN_ERR_INVALID_ARG;
     if (n_seqs == 0) return GDN_OK;
     if ((int64_t)n_seqs * cfg->n_v_heads * 4 >= ((int64_t)1 << 31)) return GDN_ERR_UNSUPPORTED;
@@ -208,13 +290,21 @@ gdn_status gdn_prefill(const gdn_config *cfg, gdn_dtype dtype, gdn_dtype out_dty
     if ((conv_state_in && !aligned(conv_state_in, 16)) ||
         (conv_state_out && !aligned(conv_state_out, 16)))
         return GDN_ERR_INVALID_ARG;
-    const PrefillLayout L = prefill_layout(cfg->n_qk_heads, cfg->n_v_heads, total_tokens, n_seqs,
-                                           dtype == GDN_BF16);
-    if (!workspace || !aligned(workspace, 256) || workspace_bytes < L.bytes) return GDN_ERR_WORKSPACE;
+    if (gate.z) {
+        if (gate.z_dtype != GDN_BF16 && gate.z_dtype != GDN_F32) return GDN_ERR_INVALID_ARG;
+        if (!gate.w || !aligned(gate.w, 16) || !std::isfinite(gate.eps) || gate.eps < 0.f) return GDN_ERR_INVALID_ARG;
+        if (total_tokens > 0 && !aligned(gate.z, 16)) return GDN_ERR_INVALID_ARG;
+        // fp32 input: y in fp32 in `out`, then the tail in place
+        if (dtype == GDN_F32 && out_dtype != GDN_F32) return GDN_ERR_UNSUPPORTED;
+    }
+    if (!workspace || !aligned(workspace, 256)) return GDN_ERR_WORKSPACE;
+    const bool bf = dtype == GDN_BF16;
+    PrefillLayout L;
+    if (!prefill_layout(cfg->n_qk_heads, cfg->n_v_heads, total_tokens, n_seqs, max_seqlen, bf, workspace_bytes, &L))
+        return GDN_ERR_WORKSPACE;
     st = check_device();
     if (st != GDN_OK) return st;
 
-    const bool bf = dtype == GDN_BF16;
     unsigned char *ws = (unsigned char *)workspace;
     int32_t *cu = (int32_t *)(ws + L.off_cu);
     int32_t *cfirst = (int32_t *)(ws + L.off_cfirst);
@@ -222,74 +312,73 @@ gdn_status gdn_prefill(const gdn_config *cfg, gdn_dtype dtype, gdn_dtype out_dty
     if (e != cudaSuccess) return cuda_fail(e);
 
     ConvParams cp{};
-    if (total_tokens > 0) {
-        cp.q = q; cp.k = k; cp.v = v;
-        cp.wq = conv_w_q; cp.wk = conv_w_k; cp.wv = conv_w_v;
-        cp.conv_in = conv_state_in;
-        cp.qh = (float *)(ws + L.off_qh); cp.kh = (float *)(ws + L.off_kh);
-        cp.vh = (float *)(ws + L.off_vh);
-        cp.kq = (float *)(ws + L.off_kq); cp.kmn = (float *)(ws + L.off_kmn);
-        cp.cseq = (int32_t *)(ws + L.off_cseq);
-        cp.vi = (float *)(ws + L.off_vi);
-        cp.cu = cu; cp.cfirst = cfirst;
-        cp.n_seqs = n_seqs; cp.n_qk = cfg->n_qk_heads; cp.n_v = cfg->n_v_heads;
-        cp.q_scale = cfg->q_scale; cp.eps = cfg->l2_eps;
-        // bf16 inputs run the tensor-core (TF32) prefill, fp32 inputs the fp32 CUDA-core one;
-        // the pipelined tensor-core path launches the conv per chunk range below
-        if (L.n_segments == 1) {
-            e = launch_conv_l2(cp, bf, /*tiles=*/bf, L.max_chunks, total_tokens, stream);
-            if (e != cudaSuccess) return cuda_fail(e);
-        }
-    }
+    cp.q = q; cp.k = k; cp.v = v;
+    cp.wq = conv_w_q; cp.wk = conv_w_k; cp.wv = conv_w_v;
+    cp.conv_in = conv_state_in;
+    cp.qh = (float *)(ws + L.off_qh); cp.kh = (float *)(ws + L.off_kh);
+    cp.vh = (float *)(ws + L.off_vh);
+    cp.cu = cu; cp.cfirst = cfirst;
+    cp.n_seqs = n_seqs; cp.n_qk = cfg->n_qk_heads; cp.n_v = cfg->n_v_heads;
+    cp.q_scale = cfg->q_scale; cp.eps = cfg->l2_eps; cp.act = cfg->conv_activation;
     ScanParams sp{};
     sp.qh = (const float *)(ws + L.off_qh); sp.kh = (const float *)(ws + L.off_kh);
     sp.vh = (const float *)(ws + L.off_vh);
-    sp.kq = (const float *)(ws + L.off_kq); sp.kmn = (const float *)(ws + L.off_kmn);
-    sp.vi = (const float *)(ws + L.off_vi);
     sp.alpha = alpha; sp.beta = beta; sp.cu = cu; sp.cfirst = cfirst;
-    sp.tb = (float *)(ws + L.off_tb); sp.pm = (float *)(ws + L.off_pm); sp.gr = (float *)(ws + L.off_gr);
-    sp.cseq = (const int32_t *)(ws + L.off_cseq);
     sp.max_chunks = L.max_chunks;
     sp.init = initial_state; sp.fin = final_state; sp.out = out;
     sp.n_seqs = n_seqs; sp.n_qk = cfg->n_qk_heads; sp.n_v = cfg->n_v_heads;
-    if (bf) {
-        sp.carry_in = sp.carry_out = final_state;
-        if (L.n_segments == 1) {
-            // state-independent chunk work for every (chunk, V head) at once, then the chains
-            sp.chunk_lo = 0;
-            sp.chunk_hi = L.max_chunks;
-            if (total_tokens > 0) {
-                e = launch_chunk_prep(sp, total_tokens, bf, stream);
-                if (e != cudaSuccess) return cuda_fail(e);
-            }
-            e = launch_prefill_tc(sp, total_tokens, bf, out_dtype == GDN_BF16, stream);
-        } else {
-            // pipeline over chunk ranges: conv + chunk prep of range s on the auxiliary
-            // stream, the chains of range s on the caller's stream once its prep is done;
-            // the state passes from range to range through the final-state buffer (or a
-            // workspace copy)
-            if (!final_state) sp.carry_in = sp.carry_out = (float *)(ws + L.off_carry);
-            AuxStream *aux = nullptr;
-            e = aux_stream(&aux);
+    if (!bf) {
+        // fp32 inputs: conv + L2 rows, then the fp32 CUDA-core chunked scan (one pass)
+        if (total_tokens > 0) {
+            e = launch_conv_l2(cp, false, /*tiles=*/false, L.max_chunks, total_tokens, stream);
             if (e != cudaSuccess) return cuda_fail(e);
-            const int64_t per = (L.max_chunks + L.n_segments - 1) / L.n_segments;
-            e = cudaEventRecord(aux->ev[0], stream);  // the sequence tables are ready
-            if (e == cudaSuccess) e = cudaStreamWaitEvent(aux->stream, aux->ev[0], 0);
-            for (int sg = 0; sg < L.n_segments && e == cudaSuccess; ++sg) {
-                const int64_t lo = sg * per, hi = std::min<int64_t>(L.max_chunks, lo + per);
-                cp.chunk_lo = sp.chunk_lo = lo;
-                sp.chunk_hi = hi;
-                e = launch_conv_l2(cp, bf, /*tiles=*/true, hi - lo, total_tokens, aux->stream);
-                if (e == cudaSuccess) e = launch_chunk_prep(sp, total_tokens, bf, aux->stream);
-                if (e == cudaSuccess) e = cudaEventRecord(aux->ev[1 + sg], aux->stream);
-                if (e == cudaSuccess) e = cudaStreamWaitEvent(stream, aux->ev[1 + sg], 0);
-                if (e == cudaSuccess) e = launch_prefill_tc(sp, total_tokens, bf, out_dtype == GDN_BF16, stream);
-            }
         }
+        e = launch_scan_simt(sp, false, out_dtype == GDN_BF16, stream);
+        if (e == cudaSuccess && gate.z && total_tokens > 0)
+            e = launch_output_gate(out, false, gate.z, gate.z_dtype == GDN_BF16, gate.w, gate.eps, out, false,
+                                   total_tokens * cfg->n_v_heads, stream);
+        if (e != cudaSuccess) return cuda_fail(e);
     } else {
-        e = launch_scan_simt(sp, bf, out_dtype == GDN_BF16, stream);
+        // bf16 inputs: per chunk range, conv + L2 tiles and the state-independent chunk work of
+        // every chunk of the range at once, then the chains of the range.  With several ranges
+        // the tiles of range r+1 are made on an auxiliary stream into the other buffer while
+        // the chains run range r on the caller's stream; the state passes from range to range
+        // through the final-state buffer (or a workspace carry).
+        sp.gate_z = gate.z; sp.gate_z_bf16 = gate.z_dtype == GDN_BF16;
+        sp.gate_w = gate.w; sp.gate_eps = gate.eps;
+        sp.carry_in = sp.carry_out = final_state;
+        if (L.n_ranges > 1 && !final_state) sp.carry_in = sp.carry_out = (float *)(ws + L.off_carry);
+        AuxStream *aux = nullptr;
+        if (L.n_ranges > 1) {
+            e = aux_stream(&aux);
+            if (e == cudaSuccess) e = cudaEventRecord(aux->ev_tab, stream);   // the tables are ready
+            if (e == cudaSuccess) e = cudaStreamWaitEvent(aux->stream, aux->ev_tab, 0);
+            if (e != cudaSuccess) return cuda_fail(e);
+        }
+        for (int r = 0; r < L.n_ranges && e == cudaSuccess; ++r) {
+            const int buf = r % L.n_buf;
+            unsigned char *tb = ws + L.off_tiles + (size_t)buf * L.buf_bytes;
+            ChunkRange rg = L.range0;
+            rg.r = r;
+            rg.last = r == L.n_ranges - 1;
+            cp.rg = sp.rg = rg;
+            cp.slots = sp.slots = L.slots;
+            cp.kq = (float *)(tb + L.b_kq); cp.kmn = (float *)(tb + L.b_kmn); cp.vi = (float *)(tb + L.b_vi);
+            cp.cseq = (int32_t *)(tb + L.b_cseq);
+            sp.kq = cp.kq; sp.kmn = cp.kmn; sp.vi = cp.vi; sp.cseq = cp.cseq;
+            sp.tb = (float *)(tb + L.b_tb); sp.pm = (float *)(tb + L.b_pm);
+            sp.gr = (float *)(tb + L.b_gr);
+            cudaStream_t ps = aux ? aux->stream : stream;   // where this range's tiles are made
+            if (aux && r >= L.n_buf) e = cudaStreamWaitEvent(ps, aux->ev_chain[buf], 0);   // buffer free
+            if (e == cudaSuccess && total_tokens > 0) e = launch_conv_l2(cp, true, /*tiles=*/true, L.slots, total_tokens, ps);
+            if (e == cudaSuccess && total_tokens > 0) e = launch_chunk_prep(sp, total_tokens, true, ps);
+            if (e == cudaSuccess && aux) e = cudaEventRecord(aux->ev_prep[buf], ps);
+            if (e == cudaSuccess && aux) e = cudaStreamWaitEvent(stream, aux->ev_prep[buf], 0);
+            if (e == cudaSuccess) e = launch_prefill_tc(sp, total_tokens, true, out_dtype == GDN_BF16, stream);
+            if (e == cudaSuccess && aux) e = cudaEventRecord(aux->ev_chain[buf], stream);
+        }
+        if (e != cudaSuccess) return cuda_fail(e);
     }
-    if (e != cudaSuccess) return cuda_fail(e);
     // last, on the caller's stream: every kernel that reads conv_state_in (the conv passes on
     // either stream) is ordered before this one, so conv_state_out may alias it
     if (conv_state_out) {
@@ -298,6 +387,34 @@ gdn_status gdn_prefill(const gdn_config *cfg, gdn_dtype dtype, gdn_dtype out_dty
         if (e != cudaSuccess) return cuda_fail(e);
     }
     return GDN_OK;
+}
+
+extern "C" {
+
+gdn_status gdn_prefill(const gdn_config *cfg, gdn_dtype dtype, gdn_dtype out_dtype, const void *q, const void *k,
+                       const void *v, const float *conv_w_q, const float *conv_w_k, const float *conv_w_v,
+                       const void *alpha, const void *beta, const int32_t *cu_seqlens, int n_seqs,
+                       int64_t total_tokens, int64_t max_seqlen, const float *initial_state, float *final_state,
+                       const void *conv_state_in, void *conv_state_out, void *out, void *workspace,
+                       size_t workspace_bytes, cudaStream_t stream) {
+    return prefill_impl(cfg, dtype, out_dtype, q, k, v, conv_w_q, conv_w_k, conv_w_v, alpha, beta, cu_seqlens,
+                        n_seqs, total_tokens, max_seqlen, initial_state, final_state, conv_state_in,
+                        conv_state_out, out, workspace, workspace_bytes, GateArgs{}, stream);
+}
+
+gdn_status gdn_prefill_gated(const gdn_config *cfg, gdn_dtype dtype, gdn_dtype out_dtype, const void *q,
+                             const void *k, const void *v, const float *conv_w_q, const float *conv_w_k,
+                             const float *conv_w_v, const void *alpha, const void *beta, const int32_t *cu_seqlens,
+                             int n_seqs, int64_t total_tokens, int64_t max_seqlen, const float *initial_state,
+                             float *final_state, const void *conv_state_in, void *conv_state_out, const void *z,
+                             gdn_dtype z_dtype, const float *norm_w, float norm_eps, void *out, void *workspace,
+                             size_t workspace_bytes, cudaStream_t stream) {
+    if (!z) return GDN_ERR_INVALID_ARG;
+    GateArgs g;
+    g.z = z; g.z_dtype = z_dtype; g.w = norm_w; g.eps = norm_eps;
+    return prefill_impl(cfg, dtype, out_dtype, q, k, v, conv_w_q, conv_w_k, conv_w_v, alpha, beta, cu_seqlens,
+                        n_seqs, total_tokens, max_seqlen, initial_state, final_state, conv_state_in,
+                        conv_state_out, out, workspace, workspace_bytes, g, stream);
 }
 
 gdn_status gdn_decode_step(const gdn_config *cfg, gdn_dtype dtype, gdn_dtype out_dtype,
@@ -333,7 +450,7 @@ gdn_status gdn_decode_step(const gdn_config *cfg, gdn_dtype dtype, gdn_dtype out
     p.state = state; p.conv = conv_state; p.slots = state_slots;
     p.n_rows = n_state_rows; p.batch = batch;
     p.n_qk = cfg->n_qk_heads; p.n_v = cfg->n_v_heads;
-    p.q_scale = cfg->q_scale; p.eps = cfg->l2_eps;
+    p.q_scale = cfg->q_scale; p.eps = cfg->l2_eps; p.act = cfg->conv_activation;
     p.out = out;
     cudaError_t e = launch_decode(p, dtype == GDN_BF16, out_dtype == GDN_BF16, stream);
     if (e != cudaSuccess) return cuda_fail(e);
@@ -376,7 +493,7 @@ gdn_status gdn_decode_multi(const gdn_config *cfg, gdn_dtype dtype, gdn_dtype ou
     p.state = state; p.conv = conv_state; p.slots = state_slots;
     p.n_rows = n_state_rows; p.batch = batch;
     p.n_qk = cfg->n_qk_heads; p.n_v = cfg->n_v_heads;
-    p.q_scale = cfg->q_scale; p.eps = cfg->l2_eps;
+    p.q_scale = cfg->q_scale; p.eps = cfg->l2_eps; p.act = cfg->conv_activation;
     p.out = out;
     p.n_tok = n_tok; p.state_ckpt = state_ckpt; p.conv_ckpt = conv_ckpt;
     cudaError_t e = launch_decode_multi(p, dtype == GDN_BF16, out_dtype == GDN_BF16, stream);
@@ -401,6 +518,21 @@ gdn_status gdn_output_gate(const gdn_config *cfg, gdn_dtype y_dtype, gdn_dtype z
     if (st != GDN_OK) return st;
     cudaError_t e = launch_output_gate(y, y_dtype == GDN_BF16, z, z_dtype == GDN_BF16, norm_w, eps, out,
                                        out_dtype == GDN_BF16, n_tokens * cfg->n_v_heads, stream);
+    if (e != cudaSuccess) return cuda_fail(e);
+    return GDN_OK;
+}
+
+gdn_status gdn_affine_combine(const gdn_config *cfg, const float *M, const float *B, int n_spans, const float *S0,
+                              float *S_in, cudaStream_t stream) {
+    if (!cfg || cfg->n_v_heads <= 0) return GDN_ERR_INVALID_ARG;
+    if (cfg->d_k != 128 || cfg->d_v != 128) return GDN_ERR_UNSUPPORTED;
+    if (cfg->n_v_heads > 65535) return GDN_ERR_UNSUPPORTED;
+    if (n_spans < 0 || !S_in || !aligned(S_in, 16)) return GDN_ERR_INVALID_ARG;
+    if (n_spans > 0 && (!M || !B || !aligned(M, 16) || !aligned(B, 16))) return GDN_ERR_INVALID_ARG;
+    if (S0 && !aligned(S0, 16)) return GDN_ERR_INVALID_ARG;
+    gdn_status st = check_device();
+    if (st != GDN_OK) return st;
+    cudaError_t e = launch_affine_combine(M, B, S0, S_in, n_spans, cfg->n_v_heads, stream);
     if (e != cudaSuccess) return cuda_fail(e);
     return GDN_OK;
 }

@@ -65,6 +65,9 @@ __device__ __forceinline__ float warp_sum(float x) {
     return x;
 }
 
+// the optional activation of the ShortConv outputs: SiLU(y) = y / (1 + e^-y) when act != 0
+__device__ __forceinline__ float conv_act(float y, int act) { return act ? y / (1.f + expf(-y)) : y; }
+
 __device__ __forceinline__ float safe_log_alpha(float a) {
     // alpha in (0, 1]; non-positive or tiny values act as a full reset
     return a > 0.f ? fmaxf(logf(a), kMinLogAlpha) : kMinLogAlpha;

@@ -17,7 +17,20 @@ struct TraceLaunch {
     gdn_trace_entry *entry;
 };
 
-// Workspace carve-up of one gdn_prefill call (byte offsets from the workspace base).
+// Chunk ranges of the tensor-core prefill.  The chunks of a call are processed in ranges:
+// range r holds chunks [r*R, (r+1)*R) of EVERY sequence ("sliced"), so the chains of all
+// sequences advance together and the tiles of one range fit a fixed number of slots; chunk j
+// of sequence b lives in slot b*R + (j - r*R) of the range's buffer.  When slicing would not
+// save memory (one range covers everything) the chunks are numbered globally instead
+// ("compact"): chunk j of sequence b lives in slot cfirst[b] + j.
+struct ChunkRange {
+    int compact;   // 1: one range, global chunk numbering
+    int R;         // chunks per sequence per range (sliced)
+    int r;         // range index (sliced)
+    int last;      // 1 for the last range
+};
+
+// Workspace carve-up and range plan of one gdn_prefill call (byte offsets from the base).
 struct PrefillLayout {
     int64_t max_chunks;   // upper bound of sum_b ceil(L_b / 64)
     size_t off_cu;        // int32 [n_seqs+1]   clamped, non-decreasing sequence bounds
@@ -26,30 +39,38 @@ struct PrefillLayout {
     size_t off_qh;        // [T, Hqk, 128] fp32 conv + L2 output
     size_t off_kh;        // [T, Hqk, 128]
     size_t off_vh;        // [T, Hv, 128]
-    // tensor-core path: per-chunk tiles already in the shared-memory layout of the kernels
-    // that read them (so each is one contiguous bulk copy); rows past a sequence's end are 0
-    size_t off_kq;        // [max_chunks, Hqk] x 64 KB: [K;Q], K-major 128B-swizzled blocks
-    size_t off_kmn;       // [max_chunks, Hqk] x 32 KB: K, MN-major 32B-granule swizzle
-    size_t off_vi;        // [max_chunks, Hv]  x 32 KB: V, MN-major 32B-granule swizzle
-    size_t off_tb;        // [max_chunks, Hv]  x 16 KB: T diag(beta), K-major 128B-swizzled
-    size_t off_pm;        // [max_chunks, Hv]  x 16 KB: P, same
-    size_t off_gr;        // [max_chunks, Hv]  x 640 B: gates record (gamma[64], kd[64], gamma_C)
-    size_t off_cseq;      // int32 [max_chunks]: sequence of each chunk (written by the conv pass)
-    size_t off_carry;     // [n_seqs, Hv, 128, 128] fp32 state between chunk ranges (segmented
-                          // tensor-core path without a caller final-state buffer), else empty
-    int n_segments;       // tensor-core path: chunk ranges run as a pipeline (1 = one pass)
+    // tensor-core path: n_buf buffers of `slots` chunk slots, each holding the tiles already in
+    // the shared-memory layout of the kernels that read them (one contiguous bulk copy each);
+    // rows past a sequence's end are 0.  Offsets inside a buffer:
+    size_t off_tiles;     // first buffer
+    size_t buf_bytes;     // distance between buffers
+    size_t b_kq;          // [slots, Hqk] x 64 KB: [K;Q], K-major 128B-swizzled blocks
+    size_t b_kmn;         // [slots, Hqk] x 32 KB: K, MN-major 32B-granule swizzle
+    size_t b_vi;          // [slots, Hv]  x 32 KB: V, MN-major 32B-granule swizzle
+    size_t b_tb;          // [slots, Hv]  x 16 KB: T diag(beta), K-major 128B-swizzled
+    size_t b_pm;          // [slots, Hv]  x 16 KB: P, same
+    size_t b_gr;          // [slots, Hv]  x 640 B: gates record (gamma[64], kd[64], gamma_C)
+    size_t b_cseq;        // int32 [slots]: sequence of each chunk (compact numbering)
+    size_t off_carry;     // [n_seqs, Hv, 128, 128] fp32 state between ranges (used when the
+                          // caller passes no final-state buffer), else empty
+    int64_t slots;        // chunk slots per buffer
+    int n_buf;            // 1, or 2 (range r+1 is prepared while the chains run range r)
+    int n_ranges;
+    ChunkRange range0;    // compact flag and R (r = 0)
     size_t bytes;
 };
 
-PrefillLayout prefill_layout(int n_qk, int n_v, int64_t T, int n_seqs, bool tc);
+// `ws_limit`: the plan shrinks the ranges to fit this many bytes (SIZE_MAX: preferred plan);
+// returns false when even one chunk per sequence per range does not fit.
+bool prefill_layout(int n_qk, int n_v, int64_t T, int n_seqs, int64_t max_seqlen, bool tc,
+                    size_t ws_limit, PrefillLayout *out);
 
-// Few (sequence, V head) chains leave most SMs idle while they run; the chunks are then
-// cut into ranges so that the conv and chunk prep of range s+1 run on the idle SMs while
-// the chains run range s.
-constexpr int64_t kSegMaxChains = 96;     // at most this many chains (148 SMs)
-constexpr int64_t kSegMinChunks = 32;     // chunks per range at least
-constexpr int kSegMax = 8;                // ranges at most
-int plan_segments(int n_v, int n_seqs, int64_t max_chunks);
+// Few (sequence, V head) chains leave most SMs idle while they run: the ranges then serve to
+// overlap the conv and chunk prep of range r+1 with the chains of range r, and are sized for
+// that; with many chains they bound the tile memory.
+constexpr int64_t kFewChains = 96;        // at most this many chains (148 SMs)
+constexpr int kMaxRanges = 64;            // ranges at most (when the longest sequence is known)
+constexpr int kMaxRangesUnknown = 8;      // ranges at most when it is not
 
 struct ConvParams {
     const void *q, *k, *v;                 // raw rows
@@ -57,11 +78,13 @@ struct ConvParams {
     const void *conv_in;                   // [n_seqs, 3, channels] or null
     float *qh, *kh, *vh;                   // fp32 rows (fp32 path)
     float *kq, *kmn, *vi;                  // chunk tiles (tensor-core path), or null
-    int32_t *cseq;                         // chunk -> sequence table, filled with the tiles
+    int32_t *cseq;                         // slot -> sequence table (compact numbering)
     const int32_t *cu, *cfirst;            // workspace tables
     int n_seqs, n_qk, n_v;
     float q_scale, eps;
-    int64_t chunk_lo;                      // first global chunk index of this launch
+    int act;                               // 1: SiLU on the conv outputs
+    ChunkRange rg;                         // tile path: the range this launch prepares
+    int64_t slots;                         // tile path: slots of the range (grid x)
 };
 
 struct ScanParams {
@@ -70,17 +93,23 @@ struct ScanParams {
     const void *alpha, *beta;              // [T, Hv]
     const int32_t *cu;                     // clamped bounds [n_seqs+1]
     const int32_t *cfirst;                 // first chunk index of each sequence [n_seqs+1]
-    const int32_t *cseq;                   // sequence of each chunk (tensor-core path)
+    const int32_t *cseq;                   // slot -> sequence (tensor-core path, compact numbering)
     float *tb, *pm, *gr;                   // chunk-prep tiles and gates records (tensor-core path)
     int64_t max_chunks;
-    int64_t chunk_lo, chunk_hi;            // global chunk range of one launch (tensor-core path)
-    const float *carry_in;                 // state entering a chunk range that starts inside a
+    ChunkRange rg;                         // tensor-core path: the range of this launch
+    int64_t slots;                         // its slots
+    const float *carry_in;                 // state entering a range that starts inside a
                                            // sequence (the previous range's output), or null
     float *carry_out;                      // state at the end of the range (fin or a workspace copy)
     const float *init;                     // [n_seqs, Hv, 128, 128] or null
     float *fin;                            // or null
     void *out;                             // [T, Hv, 128]
     int n_seqs, n_qk, n_v;
+    // gated output (tensor-core path): out = y / sqrt(mean(y^2) + gate_eps) * gate_w * SiLU(z)
+    const void *gate_z;                    // [T, Hv, 128] or null (plain y)
+    bool gate_z_bf16;
+    const float *gate_w;                   // [128]
+    float gate_eps;
 };
 
 struct DecodeParams {
@@ -92,6 +121,7 @@ struct DecodeParams {
     const int32_t *slots;
     int n_rows, batch, n_qk, n_v;
     float q_scale, eps;
+    int act;                               // 1: SiLU on the conv outputs
     void *out;
     int n_tok;                             // multi-token decode: tokens per row (1..kMaxDecTok)
     float *state_ckpt;                     //   or null: state after each token [B, n_tok, Hv, 128, 128]
@@ -131,6 +161,8 @@ cudaError_t launch_prefill_tc(const ScanParams &p, int64_t total_tokens, bool in
                               cudaStream_t s);
 cudaError_t launch_decode(const DecodeParams &p, bool in_bf16, bool out_bf16, cudaStream_t s);
 cudaError_t launch_decode_multi(const DecodeParams &p, bool in_bf16, bool out_bf16, cudaStream_t s);
+cudaError_t launch_affine_combine(const float *M, const float *B, const float *S0, float *S_in, int n_spans,
+                                  int n_v, cudaStream_t s);
 cudaError_t launch_output_gate(const void *y, bool y_bf16, const void *z, bool z_bf16, const float *w,
                                float eps, void *out, bool out_bf16, int64_t rows, cudaStream_t s);
 

@@ -32,9 +32,13 @@ extern "C" gdn_status gdn_prefill_static_scratch(
     int64_t total_tokens, const float *initial_state, float *final_state,
     const void *conv_state_in, void *conv_state_out, void *out, cudaStream_t stream) {
     size_t need = 0;
-    gdn_status st = gdn_prefill_workspace_size(cfg, dtype, total_tokens, n_seqs, &need);
+    gdn_status st = gdn_prefill_workspace_size(cfg, dtype, total_tokens, n_seqs, 0, &need);
     if (st != GDN_OK) return st;
-    if (need > (size_t)GDN_STATIC_SCRATCH_BYTES) return GDN_ERR_WORKSPACE;  // too large
+    // too large even with the shortest chunk ranges: rejected before anything else
+    gdn::PrefillLayout plan;
+    if (n_seqs > 0 && !gdn::prefill_layout(cfg->n_qk_heads, cfg->n_v_heads, total_tokens, n_seqs, 0,
+                                           dtype == GDN_BF16, (size_t)GDN_STATIC_SCRATCH_BYTES, &plan))
+        return GDN_ERR_WORKSPACE;
 
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -59,8 +63,9 @@ extern "C" gdn_status gdn_prefill_static_scratch(
         scratch = g_scratch_addr[dev];
     }
     // Every byte of the scratch that gdn_prefill reads is written earlier in the same
-    // call (sequence tables, then the conv + L2 rows), so nothing has to be cleared.
+    // call (sequence tables, then the tiles of each chunk range, then the carried states),
+    // so nothing has to be cleared.
     return gdn_prefill(cfg, dtype, out_dtype, q, k, v, conv_w_q, conv_w_k, conv_w_v, alpha, beta,
-                       cu_seqlens, n_seqs, total_tokens, initial_state, final_state, conv_state_in,
+                       cu_seqlens, n_seqs, total_tokens, 0, initial_state, final_state, conv_state_in,
                        conv_state_out, out, scratch, (size_t)GDN_STATIC_SCRATCH_BYTES, stream);
 }

@@ -5,32 +5,39 @@
 // DELTANET equations), in chunks of 64 tokens.  Within a chunk, with
 // g_t = sum_{s<=t} log alpha_s, gamma_t = exp(g_t), kd_t = exp(g_C - g_t) and S the state
 // entering the chunk:
-//     u   = T_beta (V - diag(gamma) K S),  T_beta = (I + A)^-1 diag(beta)
-//     y   = diag(gamma) (Q S) + P u,       P_ti = exp(g_t - g_i) q_t.k_i (i <= t)
+//     u   = T_beta V - T_beta_gamma (K S),  T_beta = (I + A)^-1 diag(beta),
+//                                           T_beta_gamma = T_beta diag(gamma)
+//     y   = diag(gamma) (Q S) + P u,        P_ti = exp(g_t - g_i) q_t.k_i (i <= t)
 //     S  <- gamma_C S + K^T diag(kd) u
 // Every per-token factor applied here (gamma_t, kd_t, gamma_C) is at most 1, so no decay
 // is ever divided out.  T_beta, P and the gates (gamma, kd, gamma_C) of every chunk come
-// from the chunk-prep pass; [K;Q], K and V as tiles from the conv + L2 pass, all already
-// in the shared-memory layout the MMAs read.  The K tiles are those of the QK head, shared
-// by its V heads.
+// from the chunk-prep pass; [K;Q], K and V as tiles from the conv + L2 pass, all already in
+// the shared-memory layout the MMAs read.  The K tiles are those of the QK head, shared by
+// its V heads.  T_beta_gamma is made here, in shared memory, from T_beta and gamma.
 //
-// One CTA owns one (sequence, V head).  All MMAs are M = 128 with the d_v index on the
-// 128 tensor-memory lanes (transposed form), so every state-dependent A operand is read
-// straight from tensor memory:
-//   issuer (warp 0, one thread), per chunk
-//     MMA_1   [X | Y1] = S^T [K;Q]^T            (N=128, K=128)   X = (K S)^T, Y1 = (Q S)^T
-//     MMA_2a  U^T      = V^T T_beta^T           (N=64,  K=64)    V from shared memory
-//     MMA_2b  U^T     -= X' T_beta^T            (N=64,  K=64)    X' = X diag(gamma) -> u^T
-//     MMA_4   Y       += u^T P^T                (N=64,  K=64)    onto Y = Y1 diag(gamma)
-//     MMA_3   S^T     += u~^T K                 (N=128, K=64)    u~ = u diag(kd), onto gamma_C S^T
-//   epilogue (warps 1-4), in tensor memory: after MMA_1, X' (first: MMA_2b waits for it),
-//     then Y and S^T *= gamma_C; after MMA_2b, u~ (MMA_3 waits for it, MMA_4 runs
-//     meanwhile); after MMA_4, y to global memory (TMA store); the initial and final state.
-//   producer (warp 5): the tile loads, each issued as soon as its buffer is consumed.
+// One CTA owns one (sequence, V head) for one range of chunks.  All MMAs are M = 128 with
+// the d_v index on the 128 tensor-memory lanes (transposed form), so every state-dependent
+// A operand is read straight from tensor memory:
+//   issuer (warp 0, one thread), per chunk c
+//     MMA_1   [X | Y1] = S^T [K;Q]^T         (N=128, K=128)   X = (K S)^T, Y1 = (Q S)^T
+//     MMA_2a  U^T      = V^T T_beta^T        (N=64,  K=64)    state-independent
+//     MMA_2b  U^T     -= X T_beta_gamma^T    (N=64,  K=64)    -> u^T
+//     MMA_4   Y       += u^T P^T             (N=64,  K=64)    onto Y = Y1 diag(gamma)
+//     MMA_3   S^T     += u~^T K              (N=128, K=64)    u~ = u diag(kd), onto gamma_C S^T
+//   The only hand-offs on the chain's critical path are the MMA completions and one epilogue
+//   step (u~); the independent MMAs fill the waits: MMA_2a(c) runs while MMA_1(c) completes
+//   (or, when chunk c's tiles arrived early, while MMA_3(c-1) does), MMA_4 while the epilogue
+//   forms u~.  u^T is double-buffered so that MMA_2a(c+1) can start before chunk c ends.
+//   epilogue (warps 1-4), in tensor memory: after MMA_1, Y = Y1 diag(gamma) and
+//     S^T *= gamma_C; after MMA_2b, u~ (over X, which MMA_2b has consumed); after MMA_4, y
+//     to global memory (TMA store); the state entering and leaving the range.
+//   producer (warp 5): the tile loads, each issued as soon as its buffer is consumed (lane 0),
+//     and T_beta_gamma = T_beta diag(gamma) in shared memory (the whole warp).
 // All waits are bounded; a CTA that times out writes NaN to its outputs.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include "chunk_range.cuh"
 #include "gdn_common.cuh"
 #include "gdn_internal.h"
 #include "tc_sm100.cuh"
@@ -51,20 +58,23 @@ constexpr int kBarEpi = 1;         // named barrier of the epilogue (128 threads
 constexpr uint32_t OFF_KQ = 0;          // [K;Q]   K-major, 4 blocks x (K 8 KB | Q 8 KB)       64 KB
 constexpr uint32_t OFF_KMN = 65536;     // K       MN-major (32-byte granules), 64 x 128       32 KB
 constexpr uint32_t OFF_VMN = 98304;     // V       MN-major (32-byte granules), 64 x 128       32 KB
-constexpr uint32_t OFF_TB = 131072;     // T_beta  K-major [t][i]                              16 KB
-constexpr uint32_t OFF_P = 147456;      // P       K-major [t][i]                              16 KB
-constexpr uint32_t OFF_YST = 163840;    // y staging: 2 x (32 rows x 128 columns), TMA stores  32 KB
-constexpr uint32_t OFF_GR = 196608;     // gates records, 2 buffers                          1280 B
+constexpr uint32_t OFF_TB = 131072;     // T_beta        K-major [t][i]                        16 KB
+constexpr uint32_t OFF_TG = 147456;     // T_beta_gamma  K-major [t][i]                        16 KB
+constexpr uint32_t OFF_P = 163840;      // P       K-major [t][i]                              16 KB
+constexpr uint32_t OFF_YST = 180224;    // y staging: 2 x (32 rows x 128 columns), TMA stores  32 KB
+constexpr uint32_t OFF_GR = 212992;     // gates records, 2 buffers                          1280 B
 constexpr uint32_t OFF_BAR = OFF_GR + 2 * kGateRec * 4;   // mbarriers
 constexpr uint32_t OFF_FLAGS = OFF_BAR + 128;             // TMEM base, abort flag
-constexpr uint32_t kSmem = OFF_FLAGS + 16;
+constexpr uint32_t OFF_RED = OFF_FLAGS + 16;              // gated output: 4 x 32 partial row sums,
+                                                          // then 32 row scales
+constexpr uint32_t kSmem = OFF_RED + 5 * 32 * 4;
 constexpr uint32_t kSmemAlloc = kSmem + 1024;              // slack to align the base to 1024
+static_assert(kSmemAlloc <= 232448, "shared memory per CTA");
 
 enum {
-    B_KQ = 0, B_V, B_KMN, B_PL,          // tile arrivals (B_V: V and T_beta)
+    B_KQ = 0, B_V, B_TG, B_KMN, B_PL,    // tile arrivals (B_V: V and T_beta; B_TG: T_beta_gamma made)
     B_GR0, B_GR1,                        // arrival of the gates record into buffer 0 / 1
-    B_1, B_2, B_3, B_4,                  // MMA completions (MMA_1; 2a+2b; 3; 4)
-    B_XS,                                // epilogue: X' = X diag(gamma) stored
+    B_1, B_2A, B_2, B_3, B_4,            // MMA completions (MMA_1; 2a; up to 2b; 3; 4)
     B_Y1,                                // epilogue: Y = Y1 diag(gamma) stored, S scaled
     B_UT,                                // epilogue: u~ = u diag(kd) stored
     B_DRAIN0,                            // drain on the failure path
@@ -74,11 +84,10 @@ static_assert(kNumBars * 8 <= 128, "barrier area");
 
 // tensor memory columns (all 128 lanes)
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t T_S = 0;      // S^T                  128 cols
-constexpr uint32_t T_XY = 128;   // [X | Y1]             128 cols
-constexpr uint32_t T_U = 256;    // u^T                   64 cols
-constexpr uint32_t T_Y = 320;    // gamma Y1, then y      64 cols
-constexpr uint32_t T_UT = 384;   // u~^T                  64 cols
+constexpr uint32_t T_S = 0;      // S^T                               128 cols
+constexpr uint32_t T_XY = 128;   // [X | Y1]; u~^T over X once MMA_2b has read it   128 cols
+constexpr uint32_t T_U = 256;    // u^T, two buffers (chunk parity)    2 x 64 cols
+constexpr uint32_t T_Y = 384;    // gamma Y1, then y                    64 cols
 
 constexpr uint32_t kWaitTries = 1u << 22;
 
@@ -112,6 +121,23 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t *m, uint32_t par, volatil
     return false;
 }
 
+// Reduce-scatter of 32 rows over the 32 lanes of a warp: s[i] holds this lane's value of row i;
+// returns the sum over the warp's lanes of row `lane` (31 shuffles: each step halves the rows a
+// lane keeps and adds its partner's share of them).
+__device__ __forceinline__ float warp_row_sums32(float (&s)[32], int lane) {
+#pragma unroll
+    for (int k = 16; k >= 1; k >>= 1) {
+        const bool up = lane & k;
+#pragma unroll
+        for (int i = 0; i < k; ++i) {
+            const float send = up ? s[i] : s[i + k];
+            const float keep = up ? s[i + k] : s[i];
+            s[i] = keep + __shfl_xor_sync(0xffffffffu, send, k);
+        }
+    }
+    return s[0];
+}
+
 // A from tensor memory (K-major), B from a shared-memory descriptor
 __device__ __forceinline__ void mma_ts(uint32_t d, uint32_t a_tmem, uint64_t b, uint32_t id, uint32_t acc) {
     asm volatile(
@@ -138,18 +164,22 @@ __device__ __forceinline__ void gemm_ts(uint32_t d_tmem, uint32_t a_tmem, uint32
 
 struct TcParams {
     CUtensorMap tm_out;   // y as [T, Hv*128] rows, boxes of 128 columns x 32 rows (no swizzle)
-    // per-chunk tiles in shared-memory layout: [K;Q] and K per (chunk, QK head); V, T_beta,
-    // P and the gates record per (chunk, V head)
+    // per-chunk tiles of the range's buffer, by slot, in shared-memory layout: [K;Q] and K per
+    // (slot, QK head); V, T_beta, P and the gates record per (slot, V head)
     const float *kq, *kmn, *vi, *tb, *pm, *gr;
     const int32_t *cu, *cfirst;
     const float *init, *carry_in;   // state entering chunk 0 / entering a later first chunk
-    float *carry_out;               // state after the last chunk of the launch
+    float *carry_out;               // state after the last chunk of the range
     void *out;
     int n_seqs, n_qk, n_v;
-    int64_t chunk_lo, chunk_hi;     // global chunk range of the launch
+    ChunkRange rg;
+    // gated output (GATED kernels): out = y / sqrt(mean(y^2) + norm_eps) * norm_w * SiLU(z)
+    const void *z;          // [T, Hv, 128] gate input
+    const float *norm_w;    // [128]
+    float norm_eps;
 };
 
-template <class TO>
+template <class TO, class TZ, bool GATED>
 __global__ void __launch_bounds__(kThr, 1) prefill_tc_kernel(const __grid_constant__ TcParams p) {
     extern __shared__ unsigned char smem_raw[];
     unsigned char *sm = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
@@ -164,14 +194,17 @@ __global__ void __launch_bounds__(kThr, 1) prefill_tc_kernel(const __grid_consta
     const int gq = h / (p.n_v / p.n_qk);
     const int seq0 = p.cu[b], L = p.cu[b + 1] - p.cu[b];
     const int seq_chunks = (L + kChunk - 1) / kChunk;
-    const int64_t cf = p.cfirst[b];                           // global index of chunk 0
-    // this launch's chunks of the sequence: [cb, cb + nchunks) of its seq_chunks; the state
-    // enters from the initial state (cb = 0) or from the previous launch's carry
-    const int cb = (int)max((int64_t)0, p.chunk_lo - cf);
-    const int nchunks = max(0, (int)min((int64_t)seq_chunks, p.chunk_hi - cf) - cb);
-    // nothing in range (a zero-length sequence is handled by the launch that starts at 0)
-    if (seq_chunks > 0 ? nchunks == 0 : p.chunk_lo != 0) return;   // uniform per CTA
+    // this range's chunks of the sequence: [cb, cb + nchunks); the state enters from the
+    // initial state (cb = 0) or from the previous range's carry
+    const bool first_range = p.rg.compact || p.rg.r == 0;
+    const int cb = p.rg.compact ? 0 : p.rg.r * p.rg.R;
+    const int nchunks = max(0, (p.rg.compact ? seq_chunks : min(seq_chunks, cb + p.rg.R)) - cb);
+    // nothing in range (a zero-length sequence is handled by the first range)
+    if (seq_chunks > 0 ? nchunks == 0 : !first_range) return;   // uniform per CTA
     const float *state_in = cb == 0 ? p.init : p.carry_in;
+    // a sequence longer than the caller's bound on the longest one still has chunks after
+    // the last range: its later tokens and its final state are set to NaN
+    const bool overflow = !p.rg.compact && p.rg.last && seq_chunks > cb + nchunks;
 
     if (tid == 0) {
         asm volatile("prefetch.tensormap [%0];" ::"l"(&p.tm_out) : "memory");
@@ -192,9 +225,10 @@ __global__ void __launch_bounds__(kThr, 1) prefill_tc_kernel(const __grid_consta
         mbar_expect_tx(&bar[bar_i], bytes);
         bulk_load(sb + dst, src, bytes, &bar[bar_i]);
     };
-    // (c counts this launch's chunks from 0; the sequence's chunk is cb + c)
-    auto qk_tile = [&](const float *base, int c, int64_t floats) { return base + ((cf + cb + c) * p.n_qk + gq) * floats; };
-    auto v_tile = [&](const float *base, int c, int64_t floats) { return base + ((cf + cb + c) * p.n_v + h) * floats; };
+    // (c counts this range's chunks from 0; the sequence's chunk is cb + c)
+    auto slot = [&](int c) { return chunk_slot(p.rg, b, cb + c, p.cfirst); };
+    auto qk_tile = [&](const float *base, int c, int64_t floats) { return base + (slot(c) * p.n_qk + gq) * floats; };
+    auto v_tile = [&](const float *base, int c, int64_t floats) { return base + (slot(c) * p.n_v + h) * floats; };
     auto issue_kq = [&](int c) { load(B_KQ, OFF_KQ, qk_tile(p.kq, c, 16384), 65536); };
     auto issue_kmn = [&](int c) { load(B_KMN, OFF_KMN, qk_tile(p.kmn, c, 8192), 32768); };
     auto issue_v = [&](int c) {  // V and T_beta, one barrier
@@ -222,8 +256,8 @@ __global__ void __launch_bounds__(kThr, 1) prefill_tc_kernel(const __grid_consta
         tmem_wait_st();
     }
     if (tid == 0 && nchunks > 0) {
-        issue_kq(0);
         issue_v(0);
+        issue_kq(0);
         issue_kmn(0);
         issue_pm(0);
         issue_gr(0);
@@ -237,41 +271,67 @@ __global__ void __launch_bounds__(kThr, 1) prefill_tc_kernel(const __grid_consta
         // ================================================================ issuer
         if (lane == 0) {
             bool ok = true;
+            bool a2_issued = false;   // MMA_2a of the current chunk already issued
             // A wait costs ~100 cycles even when its phase is complete, so the waits for tiles
             // and for epilogue steps that are normally done sit right after an MMA group,
             // while the tensor pipe still has queued work.
-            if (nchunks > 0) ok = wait_or_abort(&bar[B_KQ], 0, abort_flag);
+            if (nchunks > 0) {
+                ok = wait_or_abort(&bar[B_V], 0, abort_flag);
+                if (ok) {
+                    fence_after_sync();
+                    gemm<128, 64, 64, true, false>(tm + T_U, sb + OFF_VMN, 64, sb + OFF_TB, 8192, false);
+                    mma_commit(&bar[B_2A]);
+                    a2_issued = true;
+                    ok = wait_or_abort(&bar[B_KQ], 0, abort_flag);
+                }
+            }
             for (int c = 0; c < nchunks && ok; ++c) {
                 const uint32_t par = c & 1;
+                const uint32_t t_u = T_U + 64 * par;
                 // MMA_1: needs S (MMA_3 of c-1, waited below) and [K;Q] of c (waited below)
                 fence_after_sync();
                 gemm_ts<128, 128, false, false>(tm + T_XY, tm + T_S, sb + OFF_KQ, 16384, false);
                 mma_commit(&bar[B_1]);
-                // MMA_2a: U^T = V^T T_beta^T (state-independent).  u^T of c-1 is free: MMA_4
-                // of c-1 completed before MMA_3 of c-1, and the epilogue took u~ before that.
-                if (!(ok = wait_or_abort(&bar[B_V], par, abort_flag))) break;
+                // MMA_2a: U^T = V^T T_beta^T unless issued at the end of chunk c-1; it runs while
+                // MMA_1 completes.  Its u^T buffer held u of c-2, read by MMA_4 of c-2 (complete
+                // before MMA_3 of c-2) and by the epilogue's u~ of c-2 (done before MMA_3 of c-2).
+                if (!a2_issued) {
+                    if (!(ok = wait_or_abort(&bar[B_V], par, abort_flag))) break;
+                    fence_after_sync();
+                    gemm<128, 64, 64, true, false>(tm + t_u, sb + OFF_VMN, 64, sb + OFF_TB, 8192, false);
+                    mma_commit(&bar[B_2A]);
+                }
+                // MMA_2b: U^T -= X T_beta_gamma^T once MMA_1 has written X
+                if (!(ok = wait_or_abort(&bar[B_TG], par, abort_flag))) break;
+                if (!(ok = wait_or_abort(&bar[B_1], par, abort_flag))) break;
                 fence_after_sync();
-                gemm<128, 64, 64, true, false>(tm + T_U, sb + OFF_VMN, 64, sb + OFF_TB, 8192, false);
-                // MMA_2b: U^T -= X' T_beta^T once the epilogue has scaled X (after MMA_1)
-                if (!(ok = wait_or_abort(&bar[B_XS], par, abort_flag))) break;
-                fence_after_sync();
-                gemm_ts<64, 64, false, true>(tm + T_U, tm + T_XY, sb + OFF_TB, 8192, true);
+                gemm_ts<64, 64, false, true>(tm + t_u, tm + T_XY, sb + OFF_TG, 8192, true);
                 mma_commit(&bar[B_2]);
+                // MMA_4: Y += u^T P^T onto Y = Y1 diag(gamma); the epilogue forms u~ meanwhile
                 if (!(ok = wait_or_abort(&bar[B_Y1], par, abort_flag))) break;
                 if (!(ok = wait_or_abort(&bar[B_PL], par, abort_flag))) break;
-                if (!(ok = wait_or_abort(&bar[B_KMN], par, abort_flag))) break;
-                // MMA_4: Y += u^T P^T onto Y = Y1 diag(gamma); the epilogue forms u~ meanwhile
                 if (!(ok = wait_or_abort(&bar[B_2], par, abort_flag))) break;
                 fence_after_sync();
-                gemm_ts<64, 64, false, false>(tm + T_Y, tm + T_U, sb + OFF_P, 8192, true);
+                gemm_ts<64, 64, false, false>(tm + T_Y, tm + t_u, sb + OFF_P, 8192, true);
                 mma_commit(&bar[B_4]);
                 // MMA_3: S^T += u~^T K onto gamma_C S^T
+                if (!(ok = wait_or_abort(&bar[B_KMN], par, abort_flag))) break;
                 if (!(ok = wait_or_abort(&bar[B_UT], par, abort_flag))) break;
                 fence_after_sync();
-                gemm_ts<128, 64, true, false>(tm + T_S, tm + T_UT, sb + OFF_KMN, 64, true);
+                gemm_ts<128, 64, true, false>(tm + T_S, tm + T_XY, sb + OFF_KMN, 64, true);
                 mma_commit(&bar[B_3]);
-                // the next MMA_1 reads S and the next [K;Q]
-                if (c + 1 < nchunks && !(ok = wait_or_abort(&bar[B_KQ], par ^ 1, abort_flag))) break;
+                a2_issued = false;
+                if (c + 1 < nchunks) {
+                    // MMA_2a of c+1 fills the wait for MMA_3 when V and T_beta of c+1 are here
+                    if (mbar_try_wait(&bar[B_V], par ^ 1)) {
+                        fence_after_sync();
+                        gemm<128, 64, 64, true, false>(tm + T_U + 64 * (par ^ 1), sb + OFF_VMN, 64, sb + OFF_TB,
+                                                       8192, false);
+                        mma_commit(&bar[B_2A]);
+                        a2_issued = true;
+                    }
+                    if (!(ok = wait_or_abort(&bar[B_KQ], par ^ 1, abort_flag))) break;
+                }
                 if (!(ok = wait_or_abort(&bar[B_3], par, abort_flag))) break;
             }
             if (!ok) {  // drain this thread's MMAs (bounded)
@@ -281,34 +341,61 @@ __global__ void __launch_bounds__(kThr, 1) prefill_tc_kernel(const __grid_consta
         }
     } else if (warp == kLoadWarp) {
         // ================================================================ tile producer
-        if (lane == 0) {
-            bool ok = true;
-            int n_kq = nchunks > 0 ? 1 : 0, n_v = n_kq, n_kmn = n_kq, n_pm = n_kq;
-            int n_gr[2] = {nchunks > 0 ? 1 : 0, nchunks > 1 ? 1 : 0};
-            for (int c = 0; c < nchunks && ok; ++c) {
-                const uint32_t par = c & 1;
-                // [K;Q] of c is consumed once MMA_1 of c is done
-                if (!(ok = wait_or_abort(&bar[B_1], par, abort_flag))) break;
-                if (c + 1 < nchunks) { issue_kq(c + 1); ++n_kq; }
-                // V and T_beta once MMA_2a/2b of c are done
-                if (!(ok = wait_or_abort(&bar[B_2], par, abort_flag))) break;
-                if (c + 1 < nchunks) { issue_v(c + 1); ++n_v; }
-                // P once MMA_4 of c is done; K and this gates buffer once MMA_3 of c is done
-                // (the epilogue took the gates of c before MMA_3 could start)
-                if (!(ok = wait_or_abort(&bar[B_4], par, abort_flag))) break;
-                if (c + 1 < nchunks) { issue_pm(c + 1); ++n_pm; }
-                if (!(ok = wait_or_abort(&bar[B_3], par, abort_flag))) break;
-                if (c + 1 < nchunks) { issue_kmn(c + 1); ++n_kmn; }
-                if (c + 2 < nchunks) { issue_gr(c + 2); ++n_gr[c & 1]; }
+        // lane 0 issues the tile copies; the whole warp turns T_beta into T_beta_gamma =
+        // T_beta diag(gamma) (column i times gamma_i, TF32) for MMA_2b once T_beta and the
+        // gates of the chunk are in and MMA_2b of the previous chunk has read the buffer
+        // every lane observes the phase itself (so the copied data is visible to it); the warp
+        // agrees on the outcome, so that it stays converged
+        auto wwait = [&](int i, uint32_t par) { return __all_sync(0xffffffffu, wait_or_abort(&bar[i], par, abort_flag)); };
+        auto build_tg = [&](int c) -> bool {
+            if (!wwait(B_V, c & 1)) return false;
+            if (!wwait(B_GR0 + (c & 1), (c >> 1) & 1)) return false;
+            const float *gam = (const float *)(sm + OFF_GR + (c & 1) * kGateRec * 4) + kGrGamma;
+#pragma unroll 4
+            for (int u = lane; u < 1024; u += 32) {   // 16-byte units of the K-major image
+                const uint32_t off = (uint32_t)u * 16;
+                const int t = (off >> 7) & 63;
+                const int i = 32 * (off >> 13) + 4 * (((off >> 4) & 7) ^ (t & 7));   // first column
+                const float4 x = *reinterpret_cast<const float4 *>(sm + OFF_TB + off);
+                const float4 g = *reinterpret_cast<const float4 *>(gam + i);
+                *reinterpret_cast<float4 *>(sm + OFF_TG + off) =
+                    make_float4(to_tf32(x.x * g.x), to_tf32(x.y * g.y), to_tf32(x.z * g.z), to_tf32(x.w * g.w));
             }
-            if (!ok) {  // wait (bounded) for the copies this thread started
-                const int counts[4] = {n_kq, n_v, n_kmn, n_pm};
-                const int bars[4] = {B_KQ, B_V, B_KMN, B_PL};
-                for (int i = 0; i < 4; ++i)
-                    if (counts[i]) mbar_wait(&bar[bars[i]], (uint32_t)(counts[i] - 1) & 1, kWaitTries);
-                for (int i = 0; i < 2; ++i)
-                    if (n_gr[i]) mbar_wait(&bar[B_GR0 + i], (uint32_t)(n_gr[i] - 1) & 1, kWaitTries);
-            }
+            fence_smem_to_async();   // visible to the tensor core
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bar[B_TG]);
+            return true;
+        };
+        bool ok = nchunks == 0 || build_tg(0);
+        int n_kq = nchunks > 0 ? 1 : 0, n_v = n_kq, n_kmn = n_kq, n_pm = n_kq;
+        int n_gr[2] = {nchunks > 0 ? 1 : 0, nchunks > 1 ? 1 : 0};
+        for (int c = 0; c < nchunks && ok; ++c) {
+            const uint32_t par = c & 1;
+            const bool more = c + 1 < nchunks;
+            // [K;Q] of c is consumed once MMA_1 of c is done
+            if (!(ok = wwait(B_1, par))) break;
+            if (more && lane == 0) { issue_kq(c + 1); ++n_kq; }
+            // V and T_beta once MMA_2a of c is done (early enough for MMA_2a of c+1 to be issued
+            // before MMA_1 of c+1)
+            if (!(ok = wwait(B_2A, par))) break;
+            if (more && lane == 0) { issue_v(c + 1); ++n_v; }
+            // P once MMA_4 of c is done; K and this gates buffer once MMA_3 of c is done
+            // (the epilogue took the gates of c before MMA_3 could start)
+            if (!(ok = wwait(B_4, par))) break;
+            if (more && lane == 0) { issue_pm(c + 1); ++n_pm; }
+            if (!(ok = wwait(B_3, par))) break;
+            if (more && lane == 0) { issue_kmn(c + 1); ++n_kmn; }
+            if (c + 2 < nchunks && lane == 0) { issue_gr(c + 2); ++n_gr[c & 1]; }
+            // T_beta_gamma of c+1: MMA_2b of c (before MMA_3 of c) has read the buffer
+            if (more && !(ok = build_tg(c + 1))) break;
+        }
+        if (!ok && lane == 0) {  // wait (bounded) for the copies this thread started
+            const int counts[4] = {n_kq, n_v, n_kmn, n_pm};
+            const int bars[4] = {B_KQ, B_V, B_KMN, B_PL};
+            for (int i = 0; i < 4; ++i)
+                if (counts[i]) mbar_wait(&bar[bars[i]], (uint32_t)(counts[i] - 1) & 1, kWaitTries);
+            for (int i = 0; i < 2; ++i)
+                if (n_gr[i]) mbar_wait(&bar[B_GR0 + i], (uint32_t)(n_gr[i] - 1) & 1, kWaitTries);
         }
     } else {
         // ================================================================ epilogue
@@ -345,6 +432,29 @@ __global__ void __launch_bounds__(kThr, 1) prefill_tc_kernel(const __grid_consta
             tmem_st32(tm + lrow + dst, v0);
             tmem_st32(tm + lrow + dst + 32, v1);
         };
+        // gated output: rows 32*h2 + i (i < 32) of the chunk held in v, this thread's column j,
+        // become y / sqrt(mean_j y^2 + eps) * w_j * SiLU(z); the row sums are reduced over the
+        // warp's lanes in registers, then over the 4 warps in shared memory
+        float *red = (float *)(sm + OFF_RED), *rinv = red + 128;
+        auto gate32 = [&](float(&v)[32], int h2, int n, int64_t tok) {
+            const int j = 32 * q + lane;
+            const int64_t v_row = (int64_t)p.n_v * kHeadDim;
+            const TZ *zp = (const TZ *)p.z + (tok + 32 * h2) * v_row + h * kHeadDim + j;
+            float zv[32], sq[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) zv[i] = 32 * h2 + i < n ? to_f32(zp[(int64_t)i * v_row]) : 0.f;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) sq[i] = v[i] * v[i];
+            red[32 * q + lane] = warp_row_sums32(sq, lane);
+            bar_sync(kBarEpi, 128);
+            if (warp == kEpiWarp0)
+                rinv[lane] = rsqrtf((red[lane] + red[32 + lane] + red[64 + lane] + red[96 + lane]) *
+                                        (1.f / kHeadDim) + p.norm_eps);
+            bar_sync(kBarEpi, 128);
+            const float wj = p.norm_w[j];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = v[i] * rinv[i] * wj * (zv[i] / (1.f + expf(-zv[i])));
+        };
         for (int c = 0; c < nchunks; ++c) {
             const uint32_t par = c & 1;
             const int bsel = c & 1;
@@ -358,8 +468,6 @@ __global__ void __launch_bounds__(kThr, 1) prefill_tc_kernel(const __grid_consta
             }
             fence_after_sync();
             const float *gr = (const float *)(sm + OFF_GR + bsel * kGateRec * 4);
-            scale64(T_XY, T_XY, gr + kGrGamma);            // X' = X diag(gamma), for MMA_2b
-            publish(B_XS);
             scale64(T_XY + 64, T_Y, gr + kGrGamma);        // Y = Y1 diag(gamma), for MMA_4
             {  // S^T *= gamma_C (last read by MMA_1; MMA_3 accumulates onto it)
                 const float gc = gr[kGrGammaC];
@@ -377,7 +485,7 @@ __global__ void __launch_bounds__(kThr, 1) prefill_tc_kernel(const __grid_consta
             publish(B_Y1);
             if (!ewait(B_2, par)) break;
             fence_after_sync();
-            scale64(T_U, T_UT, gr + kGrKd);                // u~ = u diag(kd), for MMA_3
+            scale64(T_U + 64 * par, T_XY, gr + kGrKd);     // u~ = u diag(kd) over X, for MMA_3
             publish(B_UT);
             if (!ewait(B_4, par)) break;
             fence_after_sync();
@@ -393,6 +501,7 @@ __global__ void __launch_bounds__(kThr, 1) prefill_tc_kernel(const __grid_consta
                     tmem_ld32(tm + lrow + T_Y + 32 * h2, v);
                     tmem_wait_ld();
                     tmem_regs_after_wait(v);
+                    if constexpr (GATED) gate32(v, h2, kChunk, tok);
                     if (leader) bulk_wait_read1();
                     bar_sync(kBarEpi, 128);
 #pragma unroll
@@ -417,6 +526,7 @@ __global__ void __launch_bounds__(kThr, 1) prefill_tc_kernel(const __grid_consta
                     tmem_ld32(tm + lrow + T_Y + 32 * h2, v);
                     tmem_wait_ld();
                     tmem_regs_after_wait(v);
+                    if constexpr (GATED) gate32(v, h2, n, tok);
 #pragma unroll
                     for (int blk = 0; blk < 8; ++blk) {
                         float a[4] = {v[4 * blk], v[4 * blk + 1], v[4 * blk + 2], v[4 * blk + 3]};
@@ -447,6 +557,7 @@ __global__ void __launch_bounds__(kThr, 1) prefill_tc_kernel(const __grid_consta
         const uint32_t lrow = (uint32_t)(32 * q) << 16;
         const bool failed = *abort_flag != 0;
         if (p.carry_out) {
+            const bool nan_state = failed || overflow;
             float *dst = p.carry_out + ((int64_t)b * p.n_v + h) * kHeadDim * kHeadDim + j;
 #pragma unroll
             for (int d0 = 0; d0 < kHeadDim; d0 += 32) {
@@ -456,12 +567,13 @@ __global__ void __launch_bounds__(kThr, 1) prefill_tc_kernel(const __grid_consta
                 tmem_regs_after_wait(s);
 #pragma unroll
                 for (int i = 0; i < 32; ++i)
-                    dst[(int64_t)(d0 + i) * kHeadDim] = failed ? __int_as_float(0x7fc00000) : s[i];
+                    dst[(int64_t)(d0 + i) * kHeadDim] = nan_state ? __int_as_float(0x7fc00000) : s[i];
             }
         }
-        if (failed) {
+        if (failed || overflow) {
             const int64_t v_row = (int64_t)p.n_v * kHeadDim;
-            const int t0 = cb * kChunk, t1 = min(L, (cb + nchunks) * kChunk);
+            const int t0 = (failed ? cb : cb + nchunks) * kChunk;
+            const int t1 = overflow ? L : min(L, (cb + nchunks) * kChunk);
             for (int e = tid - kEpiTid0 + t0 * kHeadDim; e < t1 * kHeadDim; e += 128) {
                 const int t = e / kHeadDim, jj = e % kHeadDim;
                 ((TO *)p.out)[(seq0 + t) * v_row + h * kHeadDim + jj] = from_f32<TO>(__int_as_float(0x7fc00000));
@@ -474,7 +586,7 @@ __global__ void __launch_bounds__(kThr, 1) prefill_tc_kernel(const __grid_consta
 }
 
 // ---------------------------------------------------------------- host side
-template <class TO>
+template <class TO, class TZ, bool GATED>
 static cudaError_t launch_tc_t(TcParams p, int64_t total_tokens, cudaStream_t s) {
     const bool obf = sizeof(TO) == 2;
     const int64_t width = (int64_t)p.n_v * kHeadDim;
@@ -482,11 +594,11 @@ static cudaError_t launch_tc_t(TcParams p, int64_t total_tokens, cudaStream_t s)
         !encode_2d(&p.tm_out, obf ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, p.out,
                    width, total_tokens, width * (int64_t)sizeof(TO), kHeadDim, 32, CU_TENSOR_MAP_SWIZZLE_NONE))
         return cudaErrorInvalidValue;
-    auto k = prefill_tc_kernel<TO>;
+    auto k = prefill_tc_kernel<TO, TZ, GATED>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemAlloc);
     if (e != cudaSuccess) return e;
     const unsigned grid = (unsigned)((int64_t)p.n_seqs * p.n_v);
-    TraceLaunch tl(s, "prefill_tc");
+    TraceLaunch tl(s, GATED ? "prefill_tc_gated" : "prefill_tc");
     k<<<grid, kThr, kSmemAlloc, s>>>(p);
     return cudaGetLastError();
 }
@@ -497,9 +609,18 @@ cudaError_t launch_prefill_tc(const ScanParams &sp, int64_t total_tokens, bool /
     TcParams p{};
     p.kq = sp.kq; p.kmn = sp.kmn; p.vi = sp.vi; p.tb = sp.tb; p.pm = sp.pm; p.gr = sp.gr;
     p.cu = sp.cu; p.cfirst = sp.cfirst; p.init = sp.init; p.carry_in = sp.carry_in; p.carry_out = sp.carry_out;
-    p.chunk_lo = sp.chunk_lo; p.chunk_hi = sp.chunk_hi;
+    p.rg = sp.rg;
     p.out = sp.out; p.n_seqs = sp.n_seqs; p.n_qk = sp.n_qk; p.n_v = sp.n_v;
-    return out_bf16 ? launch_tc_t<gdn::bf16>(p, total_tokens, s) : launch_tc_t<float>(p, total_tokens, s);
+    p.z = sp.gate_z; p.norm_w = sp.gate_w; p.norm_eps = sp.gate_eps;
+    using gdn::bf16;
+    if (!sp.gate_z)
+        return out_bf16 ? launch_tc_t<bf16, float, false>(p, total_tokens, s)
+                        : launch_tc_t<float, float, false>(p, total_tokens, s);
+    if (sp.gate_z_bf16)
+        return out_bf16 ? launch_tc_t<bf16, bf16, true>(p, total_tokens, s)
+                        : launch_tc_t<float, bf16, true>(p, total_tokens, s);
+    return out_bf16 ? launch_tc_t<bf16, float, true>(p, total_tokens, s)
+                    : launch_tc_t<float, float, true>(p, total_tokens, s);
 }
 
 }  // namespace gdn

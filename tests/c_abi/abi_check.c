@@ -25,22 +25,46 @@ int main(void) {
         CHECK(t != NULL && strlen(t) > 0);
     }
 
-    gdn_config cfg = {16, 48, 128, 128, 4, 1.0f, 1e-6f};
+    gdn_config cfg = {16, 48, 128, 128, 4, 1.0f, 1e-6f, GDN_ACT_NONE};
     size_t bytes = 0;
-    CHECK(gdn_prefill_workspace_size(&cfg, GDN_BF16, 8192, 1, &bytes) == GDN_OK && bytes > 0);
+    CHECK(gdn_prefill_workspace_size(&cfg, GDN_BF16, 8192, 1, 0, &bytes) == GDN_OK && bytes > 0);
+    /* with the longest sequence known, the size follows the chunk ranges, not the tokens */
+    size_t b1 = 0, b2 = 0;
+    CHECK(gdn_prefill_workspace_size(&cfg, GDN_BF16, 1 << 20, 16, 65536, &b1) == GDN_OK);
+    CHECK(gdn_prefill_workspace_size(&cfg, GDN_BF16, 1 << 21, 16, 65536, &b2) == GDN_OK);
+    CHECK(b1 == b2);
     gdn_config bad = cfg;
+    bad.conv_activation = 7;
+    CHECK(gdn_prefill_workspace_size(&bad, GDN_BF16, 8192, 1, 0, &bytes) == GDN_ERR_INVALID_ARG);
+    bad = cfg;
     bad.d_k = 64;
-    CHECK(gdn_prefill_workspace_size(&bad, GDN_BF16, 8192, 1, &bytes) == GDN_ERR_UNSUPPORTED);
-    CHECK(gdn_prefill_workspace_size(NULL, GDN_BF16, 8192, 1, &bytes) == GDN_ERR_INVALID_ARG);
-    CHECK(gdn_prefill_workspace_size(&cfg, GDN_BF16, -1, 1, &bytes) == GDN_ERR_INVALID_ARG);
+    CHECK(gdn_prefill_workspace_size(&bad, GDN_BF16, 8192, 1, 0, &bytes) == GDN_ERR_UNSUPPORTED);
+    CHECK(gdn_prefill_workspace_size(NULL, GDN_BF16, 8192, 1, 0, &bytes) == GDN_ERR_INVALID_ARG);
+    CHECK(gdn_prefill_workspace_size(&cfg, GDN_BF16, -1, 1, 0, &bytes) == GDN_ERR_INVALID_ARG);
+    CHECK(gdn_prefill_workspace_size(&cfg, GDN_BF16, 100, 1, -1, &bytes) == GDN_ERR_INVALID_ARG);
 
     /* prefill: rejected arguments, then an empty call */
-    CHECK(gdn_prefill(&cfg, GDN_BF16, GDN_F32, NULL, A(2), A(3), A(4), A(5), A(6), A(7), A(8), A(9), 1, 100,
+    CHECK(gdn_prefill(&cfg, GDN_BF16, GDN_F32, NULL, A(2), A(3), A(4), A(5), A(6), A(7), A(8), A(9), 1, 100, 0,
                       NULL, NULL, NULL, NULL, A(10), A(11), (size_t)1 << 40, 0) == GDN_ERR_INVALID_ARG);
-    CHECK(gdn_prefill(&cfg, GDN_BF16, GDN_F32, A(1), A(2), A(3), A(4), A(5), A(6), A(7), A(8), A(9), 1, 100,
+    CHECK(gdn_prefill(&cfg, GDN_BF16, GDN_F32, A(1), A(2), A(3), A(4), A(5), A(6), A(7), A(8), A(9), 1, 100, 0,
                       NULL, NULL, NULL, NULL, A(10), A(11), 16, 0) == GDN_ERR_WORKSPACE);
-    CHECK(gdn_prefill(&cfg, GDN_BF16, GDN_F32, NULL, NULL, NULL, A(4), A(5), A(6), A(7), A(8), A(9), 0, 100,
+    CHECK(gdn_prefill(&cfg, GDN_BF16, GDN_F32, NULL, NULL, NULL, A(4), A(5), A(6), A(7), A(8), A(9), 0, 100, 0,
                       NULL, NULL, NULL, NULL, NULL, NULL, 0, 0) == GDN_OK);
+
+    /* the no-allocation prefill: a problem whose tiles cannot fit GDN_STATIC_SCRATCH_BYTES even
+     * with one chunk per sequence per range (more sequences than one chunk slot each fits) is
+     * rejected on the host, before any device call */
+    {
+        const size_t slot = (size_t)16 * (65536 + 32768) + (size_t)48 * (32768 + 2 * 16384 + 640);
+        const int n = (int)(GDN_STATIC_SCRATCH_BYTES / slot) + 1;
+        CHECK(gdn_prefill_static_scratch(&cfg, GDN_BF16, GDN_F32, A(1), A(2), A(3), A(4), A(5), A(6), A(7), A(8),
+                                         A(9), n, 64 * n, NULL, NULL, NULL, NULL, A(10), 0) == GDN_ERR_WORKSPACE);
+        /* fp32 input keeps 40 KB of rows per token */
+        const int64_t T = (int64_t)GDN_STATIC_SCRATCH_BYTES / (80 * 128 * 4) + 1;
+        CHECK(gdn_prefill_static_scratch(&cfg, GDN_F32, GDN_F32, A(1), A(2), A(3), A(4), A(5), A(6), A(7), A(8),
+                                         A(9), 1, T, NULL, NULL, NULL, NULL, A(10), 0) == GDN_ERR_WORKSPACE);
+        printf("GDN_STATIC_SCRATCH_BYTES %zu\n", (size_t)GDN_STATIC_SCRATCH_BYTES);
+    }
 
     /* decode (single and multi-token) and the output tail */
     CHECK(gdn_decode_step(&cfg, GDN_BF16, GDN_F32, A(1), A(2), A(3), A(4), A(5), A(6), A(7), A(8), NULL, A(10),

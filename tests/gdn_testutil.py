@@ -36,11 +36,11 @@ def rel_err(x: np.ndarray, ref: np.ndarray) -> float:
 
 
 def prefill_dev(inp: gi.PrefillInputs, lib, *, with_conv_out=False, initial_state=None,
-                conv_state=None):
+                conv_state=None, conv_activation=0):
     """Run the CUDA prefill on a stored-input bundle; returns (y, final_state, conv_out) tensors."""
     import torch
     d = inp.dtype
-    cfg = lib.GdnConfig(inp.shape.n_qk_heads, inp.shape.n_v_heads)
+    cfg = lib.GdnConfig(inp.shape.n_qk_heads, inp.shape.n_v_heads, conv_activation=conv_activation)
     init = inp.initial_state if initial_state is None else initial_state
     cs = inp.conv_state if conv_state is None else conv_state
     return lib.gdn_prefill(
@@ -58,3 +58,12 @@ def rel_err_bf16_out(x: np.ndarray, ref: np.ndarray) -> float:
     rms = float(np.sqrt(np.mean(ref[m] ** 2)))
     excess = np.abs(x[m] - ref[m]) - 2.0 ** -9 * np.abs(ref[m]) * 1.001
     return float(max(np.max(excess), 0.0) / max(rms, 1e-30))
+
+
+def prefill_args(inp: gi.PrefillInputs, lib):
+    """Device tensors of a stored-input bundle in gdn_prefill's positional order."""
+    import torch
+    d = inp.dtype
+    return (to_dev(inp.q, d), to_dev(inp.k, d), to_dev(inp.v, d), to_dev(inp.w_q, d),
+            to_dev(inp.w_k, d), to_dev(inp.w_v, d), to_dev(inp.alpha, d), to_dev(inp.beta, d),
+            torch.from_numpy(inp.cu_seqlens).cuda())

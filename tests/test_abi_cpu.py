@@ -26,7 +26,7 @@ def test_library_exports_every_declared_symbol():
     lib = _native.lib()
     for name in header_exports():
         assert hasattr(lib, name), name
-    assert lib.gdn_api_version() == 1
+    assert lib.gdn_api_version() == 2
 
 
 def test_status_strings():
@@ -38,34 +38,50 @@ def test_status_strings():
 
 def _cfg(**kw):
     base = dict(n_qk_heads=16, n_v_heads=48, d_k=128, d_v=128, conv_width=4, q_scale=1.0,
-                l2_eps=1e-6)
+                l2_eps=1e-6, conv_activation=0)
     base.update(kw)
     return _native.GdnConfigC(*base.values())
 
 
-def _ws(cfg, dtype=0, T=8192, n=1):
+def _ws(cfg, dtype=0, T=8192, n=1, max_seqlen=0):
     out = ctypes.c_size_t(0)
-    st = _native.lib().gdn_prefill_workspace_size(ctypes.byref(cfg), dtype, T, n, ctypes.byref(out))
+    st = _native.lib().gdn_prefill_workspace_size(ctypes.byref(cfg), dtype, T, n, max_seqlen,
+                                                  ctypes.byref(out))
     return st, out.value
 
 
-def test_workspace_size():
+# tiles of one (sequence, chunk) slot at 16 QK / 48 V heads: [K;Q] 64 KB and K 32 KB per QK
+# head; V 32 KB, T_beta and P 16 KB each and a 640-byte gates record per V head
+SLOT = 16 * (65536 + 32768) + 48 * (32768 + 2 * 16384 + 640)
+STATE = 128 * 128 * 4
+
+
+def test_workspace_size_bf16_is_two_chunk_ranges():
+    # one 8192-token sequence: ranges of 32 chunks, two buffers, one carried state per head
     st, b = _ws(_cfg(), 0, 8192, 1)
     assert st == 0
+    assert 2 * 32 * SLOT + 48 * STATE <= b < 2 * 32 * SLOT + 48 * STATE + 64 * 1024
+    # the size depends on the range length, not on the number of tokens
+    st2, b2 = _ws(_cfg(), 0, 262144, 1, 262144)
+    st3, b3 = _ws(_cfg(), 0, 2 * 262144, 1, 2 * 262144)
+    assert st2 == st3 == 0 and b2 == b3 < 2 * 128 * SLOT + 48 * STATE + 64 * 1024
+    # 32 packed sequences up to 64K tokens: 16 chunks per sequence per range
+    st4, b4 = _ws(_cfg(), 0, 602887, 32, 65536)
+    assert st4 == 0 and b4 < 2 * 32 * 16 * SLOT + 32 * 48 * STATE + 64 * 1024
+    assert _ws(_cfg(), 0, 0, 3)[0] == 0
+
+
+def test_workspace_size_fp32_rows():
     # q^, k^ (2 x T x 16 x 128) + v^ (T x 48 x 128) in fp32, plus two small int tables
     rows = 8192 * (2 * 16 + 48) * 128 * 4
-    # the tensor-core (bf16) path adds two 64 x 64 fp32 tiles per (chunk, V head)
-    tiles = 2 * (8192 // 64 + 1) * 48 * 64 * 64 * 4
-    assert b >= rows + tiles
-    st4, b4 = _ws(_cfg(), 1, 8192, 1)
-    assert st4 == 0 and rows <= b4 < rows + tiles
-    assert _ws(_cfg(), 0, 0, 3)[0] == 0
+    st, b = _ws(_cfg(), 1, 8192, 1)
+    assert st == 0 and rows <= b < rows + 4096
 
 
 @pytest.mark.parametrize("kw,code", [
     (dict(d_k=64), 2), (dict(d_v=256), 2), (dict(conv_width=3), 2),
     (dict(n_v_heads=47), 1), (dict(n_qk_heads=0), 1), (dict(l2_eps=-1.0), 1),
-    (dict(q_scale=float("nan")), 1),
+    (dict(q_scale=float("nan")), 1), (dict(conv_activation=2), 1), (dict(conv_activation=-1), 1),
 ])
 def test_config_rejected(kw, code):
     assert _ws(_cfg(**kw))[0] == code
@@ -74,25 +90,26 @@ def test_config_rejected(kw, code):
 def test_workspace_size_bad_args():
     lib = _native.lib()
     c = _cfg()
-    assert lib.gdn_prefill_workspace_size(ctypes.byref(c), 0, 10, 1, None) == 1
+    assert lib.gdn_prefill_workspace_size(ctypes.byref(c), 0, 10, 1, 0, None) == 1
     assert _ws(c, 0, -1, 1)[0] == 1
     assert _ws(c, 0, 1 << 31, 1)[0] == 1
     assert _ws(c, 7, 10, 1)[0] == 1
-    assert lib.gdn_prefill_workspace_size(None, 0, 10, 1, ctypes.byref(ctypes.c_size_t())) == 1
+    assert _ws(c, 0, 10, 1, -1)[0] == 1
+    assert lib.gdn_prefill_workspace_size(None, 0, 10, 1, 0, ctypes.byref(ctypes.c_size_t())) == 1
 
 
 def _prefill(**over):
     """gdn_prefill with fake (never dereferenced) aligned device addresses."""
     A = 1 << 20
     args = dict(cfg=_cfg(), dtype=0, odt=1, q=A, k=2 * A, v=3 * A, wq=4 * A, wk=5 * A, wv=6 * A,
-                alpha=7 * A, beta=8 * A, cu=9 * A, n=1, T=100, init=None, fin=None, csi=None,
+                alpha=7 * A, beta=8 * A, cu=9 * A, n=1, T=100, ms=0, init=None, fin=None, csi=None,
                 cso=None, out=10 * A, ws=11 * A, wsb=1 << 40, stream=None)
     args.update(over)
     c = args["cfg"]
     return _native.lib().gdn_prefill(
         ctypes.byref(c) if c is not None else None, args["dtype"], args["odt"], args["q"], args["k"], args["v"],
         args["wq"], args["wk"], args["wv"], args["alpha"], args["beta"], args["cu"], args["n"],
-        args["T"], args["init"], args["fin"], args["csi"], args["cso"], args["out"], args["ws"],
+        args["T"], args["ms"], args["init"], args["fin"], args["csi"], args["cso"], args["out"], args["ws"],
         args["wsb"], args["stream"])
 
 
@@ -102,7 +119,7 @@ def _prefill(**over):
     (dict(alpha=(1 << 20) + 1), 1), (dict(init=(1 << 20) + 8), 1), (dict(cso=(1 << 20) + 2), 1),
     (dict(T=-5), 1), (dict(n=-1), 1), (dict(T=1 << 31), 1), (dict(dtype=3), 1),
     (dict(ws=None), 3), (dict(wsb=16), 3), (dict(ws=(11 << 20) + 64), 3),
-    (dict(cfg=None), 1), (dict(cfg=_cfg(d_k=96)), 2), (dict(odt=2), 1),
+    (dict(cfg=None), 1), (dict(cfg=_cfg(d_k=96)), 2), (dict(odt=2), 1), (dict(ms=-1), 1),
 ])
 def test_prefill_rejects_before_launch(over, code):
     assert _prefill(**over) == code

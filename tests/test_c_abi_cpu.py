@@ -32,3 +32,6 @@ def test_c_client_compiles_links_and_runs():
         os.remove(exe)
     assert r.returncode == 0, r.stdout + r.stderr
     assert "libgdn C ABI ok" in r.stdout
+    # the binding's copy of the no-allocation scratch limit is the header's value
+    line = [ln for ln in r.stdout.splitlines() if ln.startswith("GDN_STATIC_SCRATCH_BYTES")]
+    assert line and int(line[0].split()[1]) == _native.STATIC_SCRATCH_BYTES

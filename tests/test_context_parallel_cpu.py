@@ -27,6 +27,12 @@ def oracle_prefill(q, k, v, w_q, w_k, w_v, alpha, beta, cu, *, cfg, initial_stat
     return torch.from_numpy(y), torch.from_numpy(fin), torch.from_numpy(cso)
 
 
+def oracle_combine(M, B, S0):
+    """The fp64 oracle behind affine_combine's signature."""
+    from oracle.affine import affine_prefix
+    return torch.from_numpy(affine_prefix(M.double().numpy(), B.double().numpy(), S0.double().numpy()))
+
+
 def _case(T, seed):
     inp = gi.make_prefill_inputs(SHAPE, [T], gi.F32, seed=seed, with_initial_state=True,
                                  with_conv_state=True)
@@ -46,7 +52,8 @@ def test_spans_equal_whole_sequence(bounds):
     cfg = GdnConfig(2, 6)
     ys, fin = cp_prefill_spans(_split(full, bounds), w, cfg=cfg,
                                initial_state=torch.from_numpy(inp.initial_state[0]).float(),
-                               conv_state=torch.from_numpy(inp.conv_state[0]).float(), prefill=oracle_prefill)
+                               conv_state=torch.from_numpy(inp.conv_state[0]).float(), prefill=oracle_prefill,
+                               combine=oracle_combine)
     yo, fo, _ = oracle.prefill(inp)
     np.testing.assert_allclose(torch.cat(ys).numpy(), yo, rtol=0, atol=1e-9 * np.abs(yo).max())
     np.testing.assert_allclose(fin.numpy(), fo[0], rtol=0, atol=1e-9 * np.abs(fo).max())
@@ -65,7 +72,7 @@ def _rank_main(rank, world, port, bounds, out_dir):
     try:
         inp, full, w = _case(230, 51)
         q, k, v, a, b = _split(full, bounds)[rank]
-        y, fin = cp_prefill(q, k, v, w, a, b, cfg=GdnConfig(2, 6), prefill=oracle_prefill,
+        y, fin = cp_prefill(q, k, v, w, a, b, cfg=GdnConfig(2, 6), prefill=oracle_prefill, combine=oracle_combine,
                             initial_state=torch.from_numpy(inp.initial_state[0]).float() if rank == 0 else None,
                             conv_state=torch.from_numpy(inp.conv_state[0]).float() if rank == 0 else None)
         np.save(os.path.join(out_dir, f"y{rank}.npy"), y.numpy())
@@ -87,3 +94,25 @@ def test_ranks_equal_whole_sequence(repo_tmp, bounds):
     np.testing.assert_allclose(y, yo, rtol=0, atol=1e-9 * np.abs(yo).max())
     np.testing.assert_allclose(np.load(os.path.join(repo_tmp, f"f{world - 1}.npy")), fo[0], rtol=0,
                                atol=1e-9 * np.abs(fo).max())
+
+
+def test_affine_prefix_closed_forms():
+    """The combination's own pins: identity maps add up the offsets; zero offsets multiply the
+    maps in span order (M[p] ... M[0] S0), which a transposed product would not give."""
+    from oracle.affine import affine_prefix
+    rng = np.random.default_rng(3)
+    P, H, d = 4, 2, 5
+    B = rng.standard_normal((P, H, d, d))
+    S0 = rng.standard_normal((H, d, d))
+    I = np.broadcast_to(np.eye(d), (P, H, d, d))
+    S = affine_prefix(I, B, S0)
+    for p in range(P + 1):
+        np.testing.assert_allclose(S[p], S0 + B[:p].sum(axis=0), atol=1e-12)
+    M = rng.standard_normal((P, H, d, d))
+    S = affine_prefix(M, np.zeros_like(B), S0)
+    for h in range(H):
+        X = S0[h]
+        for p in range(P):
+            X = M[p, h] @ X
+            np.testing.assert_allclose(S[p + 1, h], X, atol=1e-10)
+    assert np.array_equal(affine_prefix(M[:0], B[:0], S0), S0[None])

@@ -23,9 +23,9 @@ def _weights_dev(w, dtype):
     return [to_dev(x, dtype) for x in w]
 
 
-def _run_steps(lib, shape, dtype, dec, w, state, conv, slots=None, n_rows=None):
+def _run_steps(lib, shape, dtype, dec, w, state, conv, slots=None, n_rows=None, act=0):
     """Run every step of ``dec`` on the GPU; returns per-step outputs [steps, B, Hv, dv]."""
-    cfg = lib.GdnConfig(shape.n_qk_heads, shape.n_v_heads)
+    cfg = lib.GdnConfig(shape.n_qk_heads, shape.n_v_heads, conv_activation=act)
     wd = _weights_dev(w, dtype)
     ys = []
     for s in range(dec.q.shape[0]):
@@ -206,3 +206,31 @@ def test_multi_token_slots_and_skipped_rows(lib):
     assert rel_err(Sg[slots[live]], So) <= tol(dtype)
     untouched = [r for r in range(R) if r not in slots[live]]
     assert np.array_equal(Sg[untouched], S0[untouched].astype(np.float64))
+
+
+@pytest.mark.parametrize("dtype", [gi.BF16, gi.F32])
+def test_conv_silu_single_and_multi_token(lib, dtype):
+    """The optional SiLU on the ShortConv outputs in both decode kernels, against oracle steps
+    with the same option."""
+    shape = gi.GdnShape(n_qk_heads=4, n_v_heads=12)
+    B, steps = 3, 4
+    w = gi.make_conv_weights(shape, 111)
+    dec = gi.make_decode_inputs(shape, B, steps, dtype, seed=112)
+    rng = np.random.default_rng(113)
+    S0 = (0.05 * rng.standard_normal((B, 12, 128, 128))).astype(np.float32)
+    cs0 = gi.quantize(rng.standard_normal((B, 3, shape.channels)).astype(np.float32), dtype)
+    yo, So, co = oracle.decode_steps(shape, dtype, dec, w, S0, cs0, conv_silu=True)
+    state = torch.from_numpy(S0.copy()).cuda()
+    conv = to_dev(cs0, dtype)
+    ys = _run_steps(lib, shape, dtype, dec, w, state, conv, act=1)
+    assert rel_err(ys, yo) <= tol(dtype)
+    assert rel_err(to_host_f64(state), So) <= tol(dtype)
+    assert np.array_equal(to_host_f64(conv), co)
+    state = torch.from_numpy(S0.copy()).cuda()
+    conv = to_dev(cs0, dtype)
+    q, k, v, a, b = _multi_inputs(dec, dtype)
+    y = lib.gdn_decode_multi(q, k, v, *_weights_dev(w, dtype), a, b, state, conv,
+                             cfg=lib.GdnConfig(4, 12, conv_activation=1))
+    torch.cuda.synchronize()
+    assert rel_err(np.swapaxes(to_host_f64(y), 0, 1), yo) <= tol(dtype)
+    assert rel_err(to_host_f64(state), So) <= tol(dtype)

@@ -8,7 +8,7 @@ import pytest
 
 import gdn_inputs as gi
 import oracle
-from gdn_testutil import prefill_dev, rel_err, to_host_f64, tol
+from gdn_testutil import prefill_args, prefill_dev, rel_err, to_host_f64, tol
 
 pytestmark = pytest.mark.gpu
 
@@ -23,10 +23,10 @@ def lib():
     return gdn
 
 
-def _check(inp, lib, heads=None, with_conv=True, label=""):
-    y, fin, cso = prefill_dev(inp, lib, with_conv_out=with_conv)
+def _check(inp, lib, heads=None, with_conv=True, label="", silu=False):
+    y, fin, cso = prefill_dev(inp, lib, with_conv_out=with_conv, conv_activation=int(silu))
     torch.cuda.synchronize()
-    yo, fo, co = oracle.prefill(inp, heads=heads)
+    yo, fo, co = oracle.prefill(inp, heads=heads, conv_silu=silu)
     sel = slice(None) if heads is None else list(heads)
     ey = rel_err(to_host_f64(y)[:, sel], yo[:, sel])
     es = rel_err(to_host_f64(fin)[:, sel], fo[:, sel])
@@ -56,6 +56,16 @@ def test_ragged_varlen_with_states(lib, dtype):
 
 
 @pytest.mark.parametrize("dtype", [gi.BF16, gi.F32])
+def test_conv_silu(lib, dtype):
+    """The optional SiLU on the ShortConv outputs (gdn_config.conv_activation = SiLU) against
+    the oracle with the same option: ragged lengths, initial and conv states."""
+    shape = gi.GdnShape(n_qk_heads=4, n_v_heads=12)
+    inp = gi.make_prefill_inputs(shape, [1, 64, 65, 0, 200, 3], dtype, seed=87,
+                                 with_initial_state=True, with_conv_state=True)
+    _check(inp, lib, label=f"silu-{dtype}", silu=True)
+
+
+@pytest.mark.parametrize("dtype", [gi.BF16, gi.F32])
 def test_pages_heads_short(lib, dtype):
     shape = gi.PAGES_SHAPE
     inp = gi.make_prefill_inputs(shape, [300], dtype, seed=78)
@@ -79,7 +89,7 @@ def test_pipelined_chunk_ranges(lib):
     range, an empty one, initial states; with a final-state buffer, without one (the state is
     carried in the workspace) and with the final state aliasing the initial state."""
     shape = gi.GdnShape(n_qk_heads=2, n_v_heads=6)
-    # 6,137 tokens in 5 sequences: 100 chunk slots, 3 ranges of 34 (2 x 6 heads = 12 chains)
+    # 6,137 tokens in 5 sequences (5 x 6 heads = 30 chains): 3 ranges of 32 chunks per sequence
     inp = gi.make_prefill_inputs(shape, [2500, 0, 1400, 2200, 37], gi.BF16, seed=91,
                                  with_initial_state=True, with_conv_state=True)
     ey, es = _check(inp, lib, label="pipelined")
@@ -152,14 +162,6 @@ def test_split_equals_whole_on_gpu(lib):
     assert rel_err(to_host_f64(fb), fo) <= tol(gi.BF16)
 
 
-def prefill_args(inp, lib):
-    from gdn_testutil import to_dev
-    d = inp.dtype
-    return (to_dev(inp.q, d), to_dev(inp.k, d), to_dev(inp.v, d), to_dev(inp.w_q, d),
-            to_dev(inp.w_k, d), to_dev(inp.w_v, d), to_dev(inp.alpha, d), to_dev(inp.beta, d),
-            torch.from_numpy(inp.cu_seqlens).cuda())
-
-
 def test_workload1_full_sampled_heads(lib):
     """T = 8192, 16 QK / 48 V heads, bf16: every token of five sampled V heads."""
     inp = gi.make_workload(1)
@@ -226,3 +228,68 @@ def test_context_parallel_spans(lib):
     yo, fo, _ = oracle.prefill(inp)
     assert rel_err(to_host_f64(torch.cat(ys)), yo) <= tol(d)
     assert rel_err(to_host_f64(fin), fo[0]) <= tol(d)
+
+
+def _trace_count(lib, fn, kernel):
+    tr = lib.LaunchTrace(capacity=4096)
+    with tr:
+        out = fn()
+    torch.cuda.synchronize()
+    return out, sum(1 for n, _ in tr.records() if n == kernel)
+
+
+@pytest.mark.parametrize("with_final", [True, False])
+def test_short_ranges_from_small_workspace(lib, with_final):
+    """A workspace smaller than the preferred one makes the chunk ranges shorter: this ragged
+    problem (an empty sequence, sequences shorter than a chunk, initial and conv states) then
+    runs as 11 ranges of one chunk per sequence, its states carried in the final-state buffer
+    or in the workspace.  Same bound against the oracle, and bit for bit the default run (one
+    range over every chunk)."""
+    from gdn_testutil import to_dev
+    shape = gi.GdnShape(n_qk_heads=4, n_v_heads=12)
+    inp = gi.make_prefill_inputs(shape, [1, 700, 64, 0, 500, 3], gi.BF16, seed=77,
+                                 with_initial_state=True, with_conv_state=True)
+    d = inp.dtype
+    cfg = lib.GdnConfig(4, 12)
+    args = prefill_args(inp, lib)
+    st = torch.from_numpy(inp.initial_state).cuda()
+    cs = to_dev(inp.conv_state, d)
+    T, n = inp.total_tokens, inp.n_seqs
+    pref = lib.prefill_workspace_size(cfg, torch.bfloat16, T, n, 700)
+    slot = 4 * (65536 + 32768) + 12 * (32768 + 2 * 16384 + 640)
+    small = 2 * n * slot + n * 12 * 65536 + (1 << 16)   # two buffers of one chunk per sequence
+    assert small < pref
+    ws = torch.empty(small, dtype=torch.uint8, device="cuda")
+    (y, fin, _), launches = _trace_count(lib, lambda: lib.gdn_prefill(
+        *args, cfg=cfg, initial_state=st, conv_state_in=cs, workspace=ws, max_seqlen=700,
+        return_final_state=with_final), "prefill_tc")
+    assert launches == 11
+    y_ref, fin_ref, _ = lib.gdn_prefill(*args, cfg=cfg, initial_state=st, conv_state_in=cs, max_seqlen=700)
+    torch.cuda.synchronize()
+    yo, fo, _ = oracle.prefill(inp)
+    assert rel_err(to_host_f64(y), yo) <= tol(d)
+    assert np.array_equal(to_host_f64(y), to_host_f64(y_ref))
+    if with_final:
+        assert rel_err(to_host_f64(fin), fo) <= tol(d)
+        assert np.array_equal(to_host_f64(fin), to_host_f64(fin_ref))
+
+
+def test_sequence_longer_than_max_seqlen(lib):
+    """A sequence longer than the max_seqlen bound: with ranges of one chunk per sequence
+    (small workspace) the tokens past the bound's last range and that sequence's final state
+    are NaN; the other sequence, within the bound, is computed as usual."""
+    shape = gi.GdnShape(n_qk_heads=2, n_v_heads=6)
+    inp = gi.make_prefill_inputs(shape, [300, 1000], gi.BF16, seed=85, with_initial_state=True)
+    cfg = lib.GdnConfig(2, 6)
+    slot = 2 * (65536 + 32768) + 6 * (32768 + 2 * 16384 + 640)
+    ws = torch.empty(2 * 2 * slot + 2 * 6 * 65536 + (1 << 14), dtype=torch.uint8, device="cuda")
+    y, fin, _ = lib.gdn_prefill(*prefill_args(inp, lib), cfg=cfg, workspace=ws, max_seqlen=300,
+                                initial_state=torch.from_numpy(inp.initial_state).cuda())
+    torch.cuda.synchronize()
+    yo, fo, _ = oracle.prefill(inp)
+    yh, fh = to_host_f64(y), to_host_f64(fin)
+    assert rel_err(yh[:300], yo[:300]) <= tol(gi.BF16)
+    assert rel_err(fh[0], fo[0]) <= tol(gi.BF16)
+    covered = 300 + 5 * 64          # the bound's 5 chunks of sequence 1
+    assert rel_err(yh[300:covered], yo[300:covered]) <= tol(gi.BF16)
+    assert np.isnan(yh[covered:]).all() and np.isnan(fh[1]).all()

@@ -12,7 +12,7 @@ import numpy as np
 import pytest
 
 import gdn_inputs as gi
-from gdn_testutil import rel_err, to_dev, to_host_f64, tol
+from gdn_testutil import to_dev, to_host_f64
 
 pytestmark = pytest.mark.gpu
 
@@ -52,6 +52,22 @@ def _static_call(lib, native, inp, d):
     return out, fin, cso
 
 
+def _check_against_prefill(gdn, native, inp, d):
+    cfg = gdn.GdnConfig(inp.shape.n_qk_heads, inp.shape.n_v_heads)
+    y_ref, f_ref, c_ref = gdn.gdn_prefill(
+        d["q"], d["k"], d["v"], d["w_q"], d["w_k"], d["w_v"], d["alpha"], d["beta"], d["cu"],
+        cfg=cfg, initial_state=d["init"], conv_state_in=d["cs"], return_conv_state=True)
+    y, f, c = _static_call(gdn, native, inp, d)
+    torch.cuda.synchronize()
+    # the same kernels on the same inputs: the chunk arithmetic is identical and the state
+    # crosses chunk ranges exactly (fp32 in memory), so the results are bit for bit those of
+    # gdn_prefill, whatever range length each call chose
+    assert np.array_equal(to_host_f64(y), to_host_f64(y_ref))
+    assert np.array_equal(to_host_f64(f), to_host_f64(f_ref))
+    assert np.array_equal(to_host_f64(c), to_host_f64(c_ref))
+    assert np.isfinite(to_host_f64(y)).all()
+
+
 def test_static_scratch_matches_prefill_two_calls():
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
@@ -62,16 +78,22 @@ def test_static_scratch_matches_prefill_two_calls():
     cases = [_case(gi.GdnShape(4, 12), [300, 0, 65, 200], gi.BF16, 501),
              _case(gi.GdnShape(2, 6), [129, 7], gi.F32, 502)]
     for inp, d in cases:
-        cfg = gdn.GdnConfig(inp.shape.n_qk_heads, inp.shape.n_v_heads)
-        y_ref, f_ref, c_ref = gdn.gdn_prefill(
-            d["q"], d["k"], d["v"], d["w_q"], d["w_k"], d["w_v"], d["alpha"], d["beta"], d["cu"],
-            cfg=cfg, initial_state=d["init"], conv_state_in=d["cs"], return_conv_state=True)
-        y, f, c = _static_call(gdn, native, inp, d)
-        torch.cuda.synchronize()
-        t = tol(inp.dtype)
-        assert rel_err(to_host_f64(y), to_host_f64(y_ref)) <= t
-        assert rel_err(to_host_f64(f), to_host_f64(f_ref)) <= t
-        assert np.array_equal(to_host_f64(c), to_host_f64(c_ref))
+        _check_against_prefill(gdn, native, inp, d)
+
+
+def test_static_scratch_several_chunk_ranges():
+    """Problems that take more than one chunk range through this entry point: at 2 / 6 heads
+    a 4,200-token sequence runs the same three ranges as gdn_prefill (tiles of range r+1
+    made on the auxiliary stream while the chains run range r); at 16 / 48 heads a
+    4,096-token sequence does not fit the scratch with gdn_prefill's ranges and runs in
+    shorter ones."""
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import linear_attention_recurrence_05_b200 as gdn
+    from linear_attention_recurrence_05_b200 import _native as native
+    for shape, lengths, seed in ((gi.GdnShape(2, 6), [4200], 503), (gi.GdnShape(16, 48), [4096], 504)):
+        inp, d = _case(shape, lengths, gi.BF16, seed)
+        _check_against_prefill(gdn, native, inp, d)
 
 
 def test_static_scratch_rejects_oversized_problem():
@@ -81,11 +103,13 @@ def test_static_scratch_rejects_oversized_problem():
     cfg = native.GdnConfigC(16, 48, 128, 128, 4, 1.0, 1e-6)
     need = ctypes.c_size_t(0)
     T = 4096
-    assert native.lib().gdn_prefill_workspace_size(ctypes.byref(cfg), 0, T, 1,
+    # 16 sequences: even one chunk slot per sequence exceeds the scratch
+    n = 16
+    assert native.lib().gdn_prefill_workspace_size(ctypes.byref(cfg), 0, T, n, 0,
                                                    ctypes.byref(need)) == 0
     assert need.value > native.STATIC_SCRATCH_BYTES
     # rejected on the host, before any pointer is looked at or anything is enqueued
     A = 1 << 20
     st = native.lib().gdn_prefill_static_scratch(
-        ctypes.byref(cfg), 0, 1, A, A, A, A, A, A, A, A, A, 1, T, None, None, None, None, A, None)
+        ctypes.byref(cfg), 0, 1, A, A, A, A, A, A, A, A, A, n, T, None, None, None, None, A, None)
     assert st == 3  # GDN_ERR_WORKSPACE
