@@ -5,9 +5,9 @@
 // FIELD NOTES", section 03 (GATED DELTANET), with g_t = sum_{s<=t} log alpha_s inside the
 // chunk, gamma_t = exp(g_t) and kd_t = exp(g_{n-1} - g_t):
 //     A_ti = beta_t exp(g_t - g_i) k_t.k_i        (i < t < n, else 0)
-//     T    = (I + A)^-1,   T_beta = T diag(beta)
+//     T    = (I + A)^-1,   T_beta = T diag(beta),   T_beta_gamma = T diag(beta gamma)
 //     P_ti = exp(g_t - g_i) q_t.k_i               (i <= t < n, else 0)
-// T_beta and P (64 x 64) are written as fp32 tiles rounded to TF32 (the precision the
+// T_beta, T_beta_gamma and P (64 x 64) are written as fp32 tiles rounded to TF32 (the precision the
 // tensor-core chain reads them in), already in the shared-memory layout of an MMA operand
 // (K-major, 128-byte rows with 16-byte chunks XOR-swizzled by row), for the chain kernel to
 // stream in with one bulk copy each.  A gates record per (chunk, head) carries gamma_t,
@@ -16,11 +16,10 @@
 // One CTA per (chunk, group of up to 3 V heads of one QK head): K K^T and Q K^T do not
 // depend on the gates, so one bulk copy of the chunk's [K;Q] tile and one tcgen05 MMA
 // ([K;Q] K^T into tensor memory) serve all the CTA's heads.  Each head then has a group of
-// 4 warps: the warps turn the MMA rows into -A (kept in shared memory) and P (stored
-// straight to global memory), and invert I + A by 16 x 16 blocks: the four diagonal blocks
-// by forward substitution (a warp each), the six below them by block products, one block
-// diagonal after the other.  T_beta is staged over the head's -A area and leaves by one
-// bulk store.
+// 4 warps: the warps turn the MMA rows into A (kept in shared memory, transposed) and P
+// (stored straight to global memory), and invert I + A in registers, two threads per
+// column of T (even and odd rows) by forward substitution.  T_beta and T_beta_gamma are
+// staged in turn over the head's scratch and each leaves by one bulk store.
 #include "gdn_common.cuh"
 #include "chunk_range.cuh"
 #include "gdn_internal.h"
@@ -35,15 +34,14 @@ constexpr int kGroupThr = 128;   // 4 warps per V head
 constexpr int kMaxGroups = 3;    // V heads per CTA
 
 // shared-memory map (bytes from a 1024-aligned base).  [0, 64 KB) holds the [K;Q] tile until
-// the MMA has read it; then one scratch per group: -A row-major with rows padded to 65 floats
-// (so that a warp walking a column hits 32 banks), T = (I + A)^-1 likewise, and three 16 x 16
-// blocks of products; after the inverse the T_beta / T_beta_gamma staging (K-major image,
-// 16 KB) reuses the -A area.
+// the MMA has read it, then one scratch per group: -A^T split by row parity, array p holding
+// -A[2s + p][m] at row m, column s (64 x 32 floats), the odd array 64 bytes past a multiple
+// of 8 KB so that the two parities fall in different banks; after the inverse, the T_beta
+// staging (K-major image, 16 KB).
 constexpr uint32_t P_KQ = 0;
-constexpr int kLd = 65;                                    // padded row of -A and T (floats)
-constexpr uint32_t kMatBytes = 64 * kLd * 4;               // 16,640
-constexpr uint32_t kScrBytes = 2 * kMatBytes + 3 * 256 * 4;
-constexpr uint32_t P_GATE = (kMaxGroups * kScrBytes + 1023) / 1024 * 1024;   // g, beta, gamma, 1/gamma
+constexpr uint32_t kParStride = 8192 + 64;
+constexpr uint32_t kScrBytes = 2 * kParStride;
+constexpr uint32_t P_GATE = 65536;                 // per group: g, beta, gamma, 1/gamma
 constexpr uint32_t kGateBytes = 4 * 64 * 4;
 constexpr uint32_t P_BAR = P_GATE + kMaxGroups * kGateBytes;   // 2 mbarriers
 constexpr uint32_t P_SLOT = P_BAR + 16;            // TMEM base
@@ -52,8 +50,7 @@ constexpr uint32_t kPSmemAlloc = kPSmem + 1024;
 constexpr uint32_t kPTmemCols = 64;
 constexpr uint32_t kPWaitTries = 1u << 24;
 constexpr float kMaxChunkDecay = 80.f;  // factor exp(g_t - g_i) = gamma_t / gamma_i below this
-static_assert(kScrBytes % 16 == 0 && kMatBytes >= 16384, "staging alignment and size");
-static_assert(2 * (kPSmemAlloc + 1024) <= 233472, "two CTAs per SM");
+static_assert(kMaxGroups * kScrBytes <= 65536, "group scratch inside the tile area");
 
 __device__ __forceinline__ float4 tf32x4(float4 x) {
     return make_float4(to_tf32(x.x), to_tf32(x.y), to_tf32(x.z), to_tf32(x.w));
@@ -74,7 +71,7 @@ struct PrepParams {
     const void *alpha, *beta;
     const int32_t *cu, *cfirst;
     const int32_t *cseq;  // sequence of each slot (compact numbering)
-    float *tb, *pm;       // [slot, Hv] tiles (16 KB each)
+    float *tb, *tg, *pm;  // [slot, Hv] tiles (16 KB each)
     float *gr;            // [slot, Hv] gates records
     int n_seqs, n_qk, n_v;
     ChunkRange rg;        // the range of this launch
@@ -216,9 +213,9 @@ __global__ void __launch_bounds__(kGroupThr * kMaxGroups, 2) chunk_prep_kernel(c
                 }
             }
             if (is_a) {
-                float *am = (float *)scr + t * kLd + 32 * h2;
+                float *at = (float *)(scr + (t & 1) * kParStride) + (t >> 1) + 32 * 32 * h2;
 #pragma unroll
-                for (int e = 0; e < 32; ++e) am[e] = v[e];
+                for (int e = 0; e < 32; ++e) at[e * 32] = v[e];
             } else {
                 unsigned char *dst = (unsigned char *)(p.pm + tile * 4096);
 #pragma unroll
@@ -228,87 +225,59 @@ __global__ void __launch_bounds__(kGroupThr * kMaxGroups, 2) chunk_prep_kernel(c
             }
         }
     }
-    group_sync(gbar);   // the group's -A is complete
+    group_sync(gbar);   // the group's A^T is complete
 
-    // ---- T = (I + A)^-1 by 16 x 16 blocks.  The diagonal blocks D_b = (I + A_bb)^-1 by forward
-    // substitution (warp b of the group: two threads per column, even and odd rows, right-
-    // looking: once row m is final every later row r gains (-A)[r][m] x_m); then, block
-    // diagonal by block diagonal (d = i - j = 1, 2, 3), the blocks below the diagonal:
-    //     T_ij = D_i W_ij,   W_ij = sum_{j <= k < i} (-A)_ik T_kj
-    // (from (I + A) T = I read block row i: A_ii T_ij + T_ij + sum_{k<i} A_ik T_kj = 0).
-    float *Am = (float *)scr, *Tm = Am + 64 * kLd, *Wb = Tm + 64 * kLd;
-    {
-        const int b = gt >> 5, c = (gt >> 1) & 15, par = gt & 1;
-        const float *ab = Am + 16 * b * kLd + 16 * b;   // block (b, b) of -A
-        float x[8];                                     // x[s] = D_b[2s + par][c]
+    // ---- T = (I + A)^-1, column jc by forward substitution with right-looking updates:
+    // once row m of the column is final, every later row r loses A[r][m] T[m][jc].  This
+    // thread holds the rows of parity par (x[s] = T[2s + par][jc], as pairs for the packed
+    // FMA) and takes row m from its partner lane when m has the other parity.  Entries of A
+    // on or above the diagonal are zero in the scratch, so the updates may start at a
+    // multiple of 4; a warp skips the steps before its first column, where its rows are 0.
+    const int jc = gt >> 1, par = gt & 1;
+    const int m_first = 16 * (gt >> 5);   // this warp's columns are m_first .. m_first + 15
+    float2 x[16];
 #pragma unroll
-        for (int s2 = 0; s2 < 8; ++s2) x[s2] = 2 * s2 + par == c ? 1.f : 0.f;
+    for (int s = 0; s < 16; ++s)
+        x[s] = make_float2(2 * (2 * s) + par == jc ? 1.f : 0.f, 2 * (2 * s + 1) + par == jc ? 1.f : 0.f);
+    if (ok) {
+        const float *atp = (const float *)(scr + par * kParStride);
 #pragma unroll
-        for (int m = 0; m < 15; ++m) {
-            const float mine = x[m >> 1];
+        for (int m = 0; m < 63; ++m) {
+            if (m < m_first) continue;   // warp-uniform
+            const float2 xs = x[m >> 2];
+            const float mine = (m >> 1) & 1 ? xs.y : xs.x;
             const float other = __shfl_xor_sync(0xffffffffu, mine, 1);
-            const float xm = par == (m & 1) ? mine : other;
+            const float xm = (par == (m & 1)) ? mine : other;
+            const float2 xm2 = make_float2(xm, xm);
 #pragma unroll
-            for (int s2 = 0; s2 < 8; ++s2)
-                if (2 * s2 + par > m) x[s2] = fmaf(ab[(2 * s2 + par) * kLd + m], xm, x[s2]);
-        }
-        float *tb = Tm + 16 * b * kLd + 16 * b;
-#pragma unroll
-        for (int s2 = 0; s2 < 8; ++s2) tb[(2 * s2 + par) * kLd + c] = x[s2];
-        for (int e = gt; e < 64 * 64; e += kGroupThr) {   // zeros above the block diagonal
-            const int r = e >> 6, col = e & 63;
-            if ((col >> 4) > (r >> 4)) Tm[r * kLd + col] = 0.f;
-        }
-    }
-    group_sync(gbar);
-#pragma unroll 1
-    for (int d = 1; d < 4; ++d) {
-        const int nb = 4 - d;
-        for (int o = gt; o < nb * 256; o += kGroupThr) {
-            const int qb = o >> 8, r = (o >> 4) & 15, cc = o & 15, i = qb + d;
-            const float *arow = Am + (16 * i + r) * kLd;
-            const float *tcol = Tm + 16 * qb + cc;
-            float acc = 0.f;
-            for (int k = 16 * qb; k < 16 * i; ++k) acc = fmaf(arow[k], tcol[k * kLd], acc);
-            Wb[o] = acc;
-        }
-        group_sync(gbar);
-        for (int o = gt; o < nb * 256; o += kGroupThr) {
-            const int qb = o >> 8, r = (o >> 4) & 15, cc = o & 15, i = qb + d;
-            const float *drow = Tm + (16 * i + r) * kLd + 16 * i;   // row r of D_i
-            const float *w = Wb + qb * 256 + cc;
-            float acc = 0.f;
-            for (int m = 0; m <= r; ++m) acc = fmaf(drow[m], w[m * 16], acc);
-            Tm[(16 * i + r) * kLd + 16 * qb + cc] = acc;
-        }
-        group_sync(gbar);
-    }
-    // T_beta = T diag(beta), TF32 as a K-major image staged over the group's -A area and
-    // stored with one bulk copy; NaN if the CTA failed
-    const float nan = __int_as_float(0x7fc00000);
-    const int trow = gt >> 1, ch = 32 * (gt & 1);   // this thread: row trow, columns ch .. ch + 31
-    {
-        group_sync(gbar);   // the -A area is free
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-            const int i0 = ch + 4 * k;
-            float4 o;
-            float *op = &o.x;
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const float f = beta_s[i0 + e];
-                op[e] = ok ? to_tf32(Tm[trow * kLd + i0 + e] * f) : nan;
+            for (int s0 = (m >> 1) & ~3; s0 < 32; s0 += 4) {
+                const float4 a = *reinterpret_cast<const float4 *>(atp + m * 32 + s0);
+                x[s0 >> 1] = __ffma2_rn(make_float2(a.x, a.y), xm2, x[s0 >> 1]);
+                x[(s0 >> 1) + 1] = __ffma2_rn(make_float2(a.z, a.w), xm2, x[(s0 >> 1) + 1]);
             }
-            *reinterpret_cast<float4 *>(scr + kmaj_off(trow, i0, 64)) = o;
+        }
+    }
+    // T_beta = T diag(beta), then T_beta_gamma = T diag(beta gamma), each TF32 as a K-major
+    // image staged over the group's scratch and stored with one bulk copy; NaN if the CTA failed
+    const float nan = __int_as_float(0x7fc00000);
+#pragma unroll 1
+    for (int pass = 0; pass < 2; ++pass) {
+        group_sync(gbar);   // the scratch is free (A^T read, or the previous store has read it)
+        const float fj = pass == 0 ? beta_s[jc] : beta_s[jc] * gam_s[jc];
+#pragma unroll
+        for (int s = 0; s < 32; ++s) {
+            const float xv = (s & 1) ? x[s >> 1].y : x[s >> 1].x;
+            *reinterpret_cast<float *>(scr + kmaj_off(2 * s + par, jc, 64)) = ok ? to_tf32(xv * fj) : nan;
         }
         fence_smem_to_async();
         group_sync(gbar);
         if (gt == 0) {
-            bulk_store(p.tb + tile * 4096, smem_u32(scr), 16384);
+            bulk_store((pass == 0 ? p.tb : p.tg) + tile * 4096, smem_u32(scr), 16384);
             bulk_commit();
-            bulk_wait0();   // the store is complete before the CTA's shared memory goes away
+            bulk_wait_read0();   // the staging may be overwritten once the copy has read it
         }
     }
+    if (gt == 0) bulk_wait0();   // the stores are complete before the CTA's shared memory goes away
     fence_before_sync();
     __syncthreads();
     if (warp == 0) tmem_dealloc(tm, kPTmemCols);
@@ -319,7 +288,7 @@ cudaError_t launch_chunk_prep(const ScanParams &sp, int64_t total_tokens, bool i
     PrepParams p{};
     p.kq = sp.kq;
     p.alpha = sp.alpha; p.beta = sp.beta; p.cu = sp.cu; p.cfirst = sp.cfirst; p.cseq = sp.cseq;
-    p.tb = sp.tb; p.pm = sp.pm; p.gr = sp.gr; p.n_seqs = sp.n_seqs; p.n_qk = sp.n_qk; p.n_v = sp.n_v;
+    p.tb = sp.tb; p.tg = sp.tg; p.pm = sp.pm; p.gr = sp.gr; p.n_seqs = sp.n_seqs; p.n_qk = sp.n_qk; p.n_v = sp.n_v;
     p.rg = sp.rg;
     // V heads per CTA: 3, 2 or 1, whichever first divides the V heads of a QK head
     const int ratio = sp.n_v / sp.n_qk;

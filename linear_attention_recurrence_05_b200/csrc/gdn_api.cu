@@ -44,6 +44,7 @@ static size_t carve_tiles(PrefillLayout &L, int n_qk, int n_v, int64_t slots, in
     L.b_kmn = o;  o = align_up(o + ns * n_qk * 32768, 256);
     L.b_vi = o;   o = align_up(o + ns * n_v * 32768, 256);
     L.b_tb = o;   o = align_up(o + ns * n_v * 16384, 256);
+    L.b_tg = o;   o = align_up(o + ns * n_v * 16384, 256);
     L.b_pm = o;   o = align_up(o + ns * n_v * 16384, 256);
     L.b_gr = o;   o = align_up(o + ns * n_v * kGateRec * sizeof(float), 256);
     L.b_cseq = o; o = align_up(o + ns * sizeof(int32_t), 256);
@@ -113,7 +114,7 @@ bool prefill_layout(int n_qk, int n_v, int64_t T, int n_seqs, int64_t max_seqlen
         // twice, else one (range r+1 is then prepared after the chains of range r)
         bool fit = false;
         for (int nb = 2; nb >= 1 && !fit; --nb) {
-            const size_t per = (size_t)n_seqs * ((size_t)n_qk * 98304 + (size_t)n_v * (65536 + kGateRec * 4)) * nb;
+            const size_t per = (size_t)n_seqs * ((size_t)n_qk * 98304 + (size_t)n_v * (81920 + kGateRec * 4)) * nb;
             const size_t avail = ws_limit > off ? ws_limit - off : 0;
             int64_t r = std::min<int64_t>(R, (int64_t)(avail / per) + 1);
             for (; r >= 1; --r) {
@@ -366,7 +367,7 @@ static gdn_status prefill_impl(const gdn_config *cfg, gdn_dtype dtype, gdn_dtype
             cp.kq = (float *)(tb + L.b_kq); cp.kmn = (float *)(tb + L.b_kmn); cp.vi = (float *)(tb + L.b_vi);
             cp.cseq = (int32_t *)(tb + L.b_cseq);
             sp.kq = cp.kq; sp.kmn = cp.kmn; sp.vi = cp.vi; sp.cseq = cp.cseq;
-            sp.tb = (float *)(tb + L.b_tb); sp.pm = (float *)(tb + L.b_pm);
+            sp.tb = (float *)(tb + L.b_tb); sp.tg = (float *)(tb + L.b_tg); sp.pm = (float *)(tb + L.b_pm);
             sp.gr = (float *)(tb + L.b_gr);
             cudaStream_t ps = aux ? aux->stream : stream;   // where this range's tiles are made
             if (aux && r >= L.n_buf) e = cudaStreamWaitEvent(ps, aux->ev_chain[buf], 0);   // buffer free

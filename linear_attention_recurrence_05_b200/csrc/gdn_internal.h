@@ -48,6 +48,7 @@ struct PrefillLayout {
     size_t b_kmn;         // [slots, Hqk] x 32 KB: K, MN-major 32B-granule swizzle
     size_t b_vi;          // [slots, Hv]  x 32 KB: V, MN-major 32B-granule swizzle
     size_t b_tb;          // [slots, Hv]  x 16 KB: T diag(beta), K-major 128B-swizzled
+    size_t b_tg;          // [slots, Hv]  x 16 KB: T diag(beta gamma), same
     size_t b_pm;          // [slots, Hv]  x 16 KB: P, same
     size_t b_gr;          // [slots, Hv]  x 640 B: gates record (gamma[64], kd[64], gamma_C)
     size_t b_cseq;        // int32 [slots]: sequence of each chunk (compact numbering)
@@ -94,7 +95,7 @@ struct ScanParams {
     const int32_t *cu;                     // clamped bounds [n_seqs+1]
     const int32_t *cfirst;                 // first chunk index of each sequence [n_seqs+1]
     const int32_t *cseq;                   // slot -> sequence (tensor-core path, compact numbering)
-    float *tb, *pm, *gr;                   // chunk-prep tiles and gates records (tensor-core path)
+    float *tb, *tg, *pm, *gr;              // chunk-prep tiles and gates records (tensor-core path)
     int64_t max_chunks;
     ChunkRange rg;                         // tensor-core path: the range of this launch
     int64_t slots;                         // its slots

@@ -10,10 +10,10 @@
 //     y   = diag(gamma) (Q S) + P u,        P_ti = exp(g_t - g_i) q_t.k_i (i <= t)
 //     S  <- gamma_C S + K^T diag(kd) u
 // Every per-token factor applied here (gamma_t, kd_t, gamma_C) is at most 1, so no decay
-// is ever divided out.  T_beta, P and the gates (gamma, kd, gamma_C) of every chunk come
-// from the chunk-prep pass; [K;Q], K and V as tiles from the conv + L2 pass, all already in
-// the shared-memory layout the MMAs read.  The K tiles are those of the QK head, shared by
-// its V heads.  T_beta_gamma is made here, in shared memory, from T_beta and gamma.
+// is ever divided out.  T_beta, T_beta_gamma, P and the gates (gamma, kd, gamma_C) of every
+// chunk come from the chunk-prep pass; [K;Q], K and V as tiles from the conv + L2 pass, all
+// already in the shared-memory layout the MMAs read ([K;Q] and K are the QK head's, shared by
+// its V heads).
 //
 // One CTA owns one (sequence, V head) for one range of chunks.  All MMAs are M = 128 with
 // the d_v index on the 128 tensor-memory lanes (transposed form), so every state-dependent
@@ -24,15 +24,17 @@
 //     MMA_2b  U^T     -= X T_beta_gamma^T    (N=64,  K=64)    -> u^T
 //     MMA_4   Y       += u^T P^T             (N=64,  K=64)    onto Y = Y1 diag(gamma)
 //     MMA_3   S^T     += u~^T K              (N=128, K=64)    u~ = u diag(kd), onto gamma_C S^T
-//   The only hand-offs on the chain's critical path are the MMA completions and one epilogue
-//   step (u~); the independent MMAs fill the waits: MMA_2a(c) runs while MMA_1(c) completes
-//   (or, when chunk c's tiles arrived early, while MMA_3(c-1) does), MMA_4 while the epilogue
-//   forms u~.  u^T is double-buffered so that MMA_2a(c+1) can start before chunk c ends.
-//   epilogue (warps 1-4), in tensor memory: after MMA_1, Y = Y1 diag(gamma) and
-//     S^T *= gamma_C; after MMA_2b, u~ (over X, which MMA_2b has consumed); after MMA_4, y
-//     to global memory (TMA store); the state entering and leaving the range.
-//   producer (warp 5): the tile loads, each issued as soon as its buffer is consumed (lane 0),
-//     and T_beta_gamma = T_beta diag(gamma) in shared memory (the whole warp).
+//   V is double-buffered (a chunk ahead) and T_beta reloaded as soon as MMA_2a has read it, so
+//   MMA_2a(c+1) is normally issued right after MMA_3(c) and runs while the new state is waited
+//   for; MMA_2b reads X straight from MMA_1's output.  The only epilogue step left on the
+//   critical path is u~; MMA_4 runs while it is formed.  u^T is double-buffered in tensor
+//   memory (chunk parity).
+//   epilogue (warps 1-4), in tensor memory: after MMA_1, Y = Y1 diag(gamma) (once the drain
+//     group has read the previous Y) and S^T *= gamma_C; after MMA_2b, u~ (over X, which
+//     MMA_2b has consumed); the state entering and leaving the range.
+//   producer (warp 5): the tile loads, each issued as soon as its buffer is free.
+//   drain group (warps 6-9): after MMA_4, reads Y and frees it at once, then writes y (or the
+//     gated output) through shared memory with TMA stores.
 // All waits are bounded; a CTA that times out writes NaN to its outputs.
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -48,39 +50,42 @@ namespace gdn {
 namespace {
 using namespace tc;
 
-constexpr int kThr = 192;          // 6 warps
-constexpr int kEpiWarp0 = 1;       // warps 1-4
+constexpr int kThr = 320;          // 10 warps
+constexpr int kEpiWarp0 = 1;       // warps 1-4: epilogue
 constexpr int kLoadWarp = 5;       // tile producer
+constexpr int kDrainWarp0 = 6;     // warps 6-9: y out
 constexpr int kEpiTid0 = kEpiWarp0 * 32;
+constexpr int kDrainTid0 = kDrainWarp0 * 32;
 constexpr int kBarEpi = 1;         // named barrier of the epilogue (128 threads)
+constexpr int kBarDrain = 2;       // named barrier of the drain group (128 threads)
 
 // shared-memory map (bytes from a 1024-aligned base)
 constexpr uint32_t OFF_KQ = 0;          // [K;Q]   K-major, 4 blocks x (K 8 KB | Q 8 KB)       64 KB
 constexpr uint32_t OFF_KMN = 65536;     // K       MN-major (32-byte granules), 64 x 128       32 KB
-constexpr uint32_t OFF_VMN = 98304;     // V       MN-major (32-byte granules), 64 x 128       32 KB
-constexpr uint32_t OFF_TB = 131072;     // T_beta        K-major [t][i]                        16 KB
-constexpr uint32_t OFF_TG = 147456;     // T_beta_gamma  K-major [t][i]                        16 KB
-constexpr uint32_t OFF_P = 163840;      // P       K-major [t][i]                              16 KB
-constexpr uint32_t OFF_YST = 180224;    // y staging: 2 x (32 rows x 128 columns), TMA stores  32 KB
-constexpr uint32_t OFF_GR = 212992;     // gates records, 2 buffers                          1280 B
+constexpr uint32_t OFF_V = 98304;       // V       MN-major, 2 buffers (chunk parity)      2 x 32 KB
+constexpr uint32_t OFF_TB = 163840;     // T_beta        K-major [t][i]                        16 KB
+constexpr uint32_t OFF_TG = 180224;     // T_beta_gamma  K-major [t][i]                        16 KB
+constexpr uint32_t OFF_P = 196608;      // P       K-major [t][i]                              16 KB
+constexpr uint32_t OFF_YST = 212992;    // y staging: 32 rows x 128 columns (TMA store box)    16 KB
+constexpr uint32_t OFF_GR = 229376;     // gates records, 2 buffers                          1280 B
 constexpr uint32_t OFF_BAR = OFF_GR + 2 * kGateRec * 4;   // mbarriers
-constexpr uint32_t OFF_FLAGS = OFF_BAR + 128;             // TMEM base, abort flag
-constexpr uint32_t OFF_RED = OFF_FLAGS + 16;              // gated output: 4 x 32 partial row sums,
-                                                          // then 32 row scales
-constexpr uint32_t kSmem = OFF_RED + 5 * 32 * 4;
+constexpr uint32_t OFF_FLAGS = OFF_BAR + 144;             // TMEM base, abort flag
+constexpr uint32_t kSmem = OFF_FLAGS + 16;
 constexpr uint32_t kSmemAlloc = kSmem + 1024;              // slack to align the base to 1024
 static_assert(kSmemAlloc <= 232448, "shared memory per CTA");
 
 enum {
-    B_KQ = 0, B_V, B_TG, B_KMN, B_PL,    // tile arrivals (B_V: V and T_beta; B_TG: T_beta_gamma made)
-    B_GR0, B_GR1,                        // arrival of the gates record into buffer 0 / 1
+    B_KQ = 0, B_V0, B_V1, B_TB, B_TG,    // tile arrivals (B_V: V of buffer 0 / 1)
+    B_KMN, B_PL,
+    B_GR0, B_GR1,                        // gates record into buffer 0 / 1
     B_1, B_2A, B_2, B_3, B_4,            // MMA completions (MMA_1; 2a; up to 2b; 3; 4)
     B_Y1,                                // epilogue: Y = Y1 diag(gamma) stored, S scaled
     B_UT,                                // epilogue: u~ = u diag(kd) stored
+    B_YF,                                // drain group: Y read (tensor memory free for the next chunk)
     B_DRAIN0,                            // drain on the failure path
     kNumBars
 };
-static_assert(kNumBars * 8 <= 128, "barrier area");
+static_assert(kNumBars * 8 <= 144, "barrier area");
 
 // tensor memory columns (all 128 lanes)
 constexpr uint32_t kTmemCols = 512;
@@ -165,8 +170,8 @@ __device__ __forceinline__ void gemm_ts(uint32_t d_tmem, uint32_t a_tmem, uint32
 struct TcParams {
     CUtensorMap tm_out;   // y as [T, Hv*128] rows, boxes of 128 columns x 32 rows (no swizzle)
     // per-chunk tiles of the range's buffer, by slot, in shared-memory layout: [K;Q] and K per
-    // (slot, QK head); V, T_beta, P and the gates record per (slot, V head)
-    const float *kq, *kmn, *vi, *tb, *pm, *gr;
+    // (slot, QK head); V, T_beta, T_beta_gamma, P and the gates record per (slot, V head)
+    const float *kq, *kmn, *vi, *tb, *tg, *pm, *gr;
     const int32_t *cu, *cfirst;
     const float *init, *carry_in;   // state entering chunk 0 / entering a later first chunk
     float *carry_out;               // state after the last chunk of the range
@@ -231,11 +236,9 @@ __global__ void __launch_bounds__(kThr, 1) prefill_tc_kernel(const __grid_consta
     auto v_tile = [&](const float *base, int c, int64_t floats) { return base + (slot(c) * p.n_v + h) * floats; };
     auto issue_kq = [&](int c) { load(B_KQ, OFF_KQ, qk_tile(p.kq, c, 16384), 65536); };
     auto issue_kmn = [&](int c) { load(B_KMN, OFF_KMN, qk_tile(p.kmn, c, 8192), 32768); };
-    auto issue_v = [&](int c) {  // V and T_beta, one barrier
-        mbar_expect_tx(&bar[B_V], 32768 + 16384);
-        bulk_load(sb + OFF_VMN, v_tile(p.vi, c, 8192), 32768, &bar[B_V]);
-        bulk_load(sb + OFF_TB, v_tile(p.tb, c, 4096), 16384, &bar[B_V]);
-    };
+    auto issue_v = [&](int c) { load(B_V0 + (c & 1), OFF_V + (c & 1) * 32768, v_tile(p.vi, c, 8192), 32768); };
+    auto issue_tb = [&](int c) { load(B_TB, OFF_TB, v_tile(p.tb, c, 4096), 16384); };
+    auto issue_tg = [&](int c) { load(B_TG, OFF_TG, v_tile(p.tg, c, 4096), 16384); };
     auto issue_pm = [&](int c) { load(B_PL, OFF_P, v_tile(p.pm, c, 4096), 16384); };
     auto issue_gr = [&](int c) {  // gates record of chunk c into buffer c & 1
         load(B_GR0 + (c & 1), OFF_GR + (c & 1) * kGateRec * 4, v_tile(p.gr, c, kGateRec), kGateRec * 4);
@@ -257,7 +260,10 @@ __global__ void __launch_bounds__(kThr, 1) prefill_tc_kernel(const __grid_consta
     }
     if (tid == 0 && nchunks > 0) {
         issue_v(0);
+        issue_tb(0);
         issue_kq(0);
+        if (nchunks > 1) issue_v(1);
+        issue_tg(0);
         issue_kmn(0);
         issue_pm(0);
         issue_gr(0);
@@ -272,49 +278,54 @@ __global__ void __launch_bounds__(kThr, 1) prefill_tc_kernel(const __grid_consta
         if (lane == 0) {
             bool ok = true;
             bool a2_issued = false;   // MMA_2a of the current chunk already issued
+            // V of chunk c sits in buffer c & 1; that buffer's barrier completes once per two
+            // chunks, so chunk c waits for its phase c >> 1
+            auto vpar = [](int c) { return (uint32_t)((c >> 1) & 1); };
+            auto issue_2a = [&](int c) {   // into u^T buffer c & 1 (D), V of buffer c & 1
+                const int bi = c & 1;
+                fence_after_sync();
+                gemm<128, 64, 64, true, false>(tm + T_U + 64 * bi, sb + OFF_V + bi * 32768, 64, sb + OFF_TB, 8192,
+                                               false);
+                mma_commit(&bar[B_2A]);
+            };
             // A wait costs ~100 cycles even when its phase is complete, so the waits for tiles
             // and for epilogue steps that are normally done sit right after an MMA group,
             // while the tensor pipe still has queued work.
             if (nchunks > 0) {
-                ok = wait_or_abort(&bar[B_V], 0, abort_flag);
+                ok = wait_or_abort(&bar[B_V0], 0, abort_flag) && wait_or_abort(&bar[B_TB], 0, abort_flag);
                 if (ok) {
-                    fence_after_sync();
-                    gemm<128, 64, 64, true, false>(tm + T_U, sb + OFF_VMN, 64, sb + OFF_TB, 8192, false);
-                    mma_commit(&bar[B_2A]);
+                    issue_2a(0);
                     a2_issued = true;
                     ok = wait_or_abort(&bar[B_KQ], 0, abort_flag);
                 }
             }
             for (int c = 0; c < nchunks && ok; ++c) {
                 const uint32_t par = c & 1;
-                const uint32_t t_u = T_U + 64 * par;
+                const int bi = c & 1;
                 // MMA_1: needs S (MMA_3 of c-1, waited below) and [K;Q] of c (waited below)
                 fence_after_sync();
                 gemm_ts<128, 128, false, false>(tm + T_XY, tm + T_S, sb + OFF_KQ, 16384, false);
                 mma_commit(&bar[B_1]);
-                // MMA_2a: U^T = V^T T_beta^T unless issued at the end of chunk c-1; it runs while
-                // MMA_1 completes.  Its u^T buffer held u of c-2, read by MMA_4 of c-2 (complete
-                // before MMA_3 of c-2) and by the epilogue's u~ of c-2 (done before MMA_3 of c-2).
+                // MMA_2a of c unless issued at the end of c-1 (its tiles came late)
                 if (!a2_issued) {
-                    if (!(ok = wait_or_abort(&bar[B_V], par, abort_flag))) break;
-                    fence_after_sync();
-                    gemm<128, 64, 64, true, false>(tm + t_u, sb + OFF_VMN, 64, sb + OFF_TB, 8192, false);
-                    mma_commit(&bar[B_2A]);
+                    if (!(ok = wait_or_abort(&bar[B_V0 + bi], vpar(c), abort_flag))) break;
+                    if (!(ok = wait_or_abort(&bar[B_TB], par, abort_flag))) break;
+                    issue_2a(c);
                 }
                 // MMA_2b: U^T -= X T_beta_gamma^T once MMA_1 has written X
                 if (!(ok = wait_or_abort(&bar[B_TG], par, abort_flag))) break;
                 if (!(ok = wait_or_abort(&bar[B_1], par, abort_flag))) break;
                 fence_after_sync();
-                gemm_ts<64, 64, false, true>(tm + t_u, tm + T_XY, sb + OFF_TG, 8192, true);
+                gemm_ts<64, 64, false, true>(tm + T_U + 64 * bi, tm + T_XY, sb + OFF_TG, 8192, true);
                 mma_commit(&bar[B_2]);
                 // MMA_4: Y += u^T P^T onto Y = Y1 diag(gamma); the epilogue forms u~ meanwhile
                 if (!(ok = wait_or_abort(&bar[B_Y1], par, abort_flag))) break;
                 if (!(ok = wait_or_abort(&bar[B_PL], par, abort_flag))) break;
                 if (!(ok = wait_or_abort(&bar[B_2], par, abort_flag))) break;
                 fence_after_sync();
-                gemm_ts<64, 64, false, false>(tm + T_Y, tm + t_u, sb + OFF_P, 8192, true);
+                gemm_ts<64, 64, false, false>(tm + T_Y, tm + T_U + 64 * bi, sb + OFF_P, 8192, true);
                 mma_commit(&bar[B_4]);
-                // MMA_3: S^T += u~^T K onto gamma_C S^T
+                // MMA_3: S^T += u~^T K onto gamma_C S^T (K in its MN-major tile)
                 if (!(ok = wait_or_abort(&bar[B_KMN], par, abort_flag))) break;
                 if (!(ok = wait_or_abort(&bar[B_UT], par, abort_flag))) break;
                 fence_after_sync();
@@ -322,12 +333,10 @@ __global__ void __launch_bounds__(kThr, 1) prefill_tc_kernel(const __grid_consta
                 mma_commit(&bar[B_3]);
                 a2_issued = false;
                 if (c + 1 < nchunks) {
-                    // MMA_2a of c+1 fills the wait for MMA_3 when V and T_beta of c+1 are here
-                    if (mbar_try_wait(&bar[B_V], par ^ 1)) {
-                        fence_after_sync();
-                        gemm<128, 64, 64, true, false>(tm + T_U + 64 * (par ^ 1), sb + OFF_VMN, 64, sb + OFF_TB,
-                                                       8192, false);
-                        mma_commit(&bar[B_2A]);
+                    // MMA_2a of c+1 fills the wait for MMA_3 (its u^T buffer held u of c-1, read by
+                    // MMA_4 and the epilogue of c-1, both complete before MMA_3 of c-1)
+                    if (mbar_try_wait(&bar[B_V0 + (bi ^ 1)], vpar(c + 1)) && mbar_try_wait(&bar[B_TB], par ^ 1)) {
+                        issue_2a(c + 1);
                         a2_issued = true;
                     }
                     if (!(ok = wait_or_abort(&bar[B_KQ], par ^ 1, abort_flag))) break;
@@ -341,63 +350,44 @@ __global__ void __launch_bounds__(kThr, 1) prefill_tc_kernel(const __grid_consta
         }
     } else if (warp == kLoadWarp) {
         // ================================================================ tile producer
-        // lane 0 issues the tile copies; the whole warp turns T_beta into T_beta_gamma =
-        // T_beta diag(gamma) (column i times gamma_i, TF32) for MMA_2b once T_beta and the
-        // gates of the chunk are in and MMA_2b of the previous chunk has read the buffer
-        // every lane observes the phase itself (so the copied data is visible to it); the warp
-        // agrees on the outcome, so that it stays converged
-        auto wwait = [&](int i, uint32_t par) { return __all_sync(0xffffffffu, wait_or_abort(&bar[i], par, abort_flag)); };
-        auto build_tg = [&](int c) -> bool {
-            if (!wwait(B_V, c & 1)) return false;
-            if (!wwait(B_GR0 + (c & 1), (c >> 1) & 1)) return false;
-            const float *gam = (const float *)(sm + OFF_GR + (c & 1) * kGateRec * 4) + kGrGamma;
-#pragma unroll 4
-            for (int u = lane; u < 1024; u += 32) {   // 16-byte units of the K-major image
-                const uint32_t off = (uint32_t)u * 16;
-                const int t = (off >> 7) & 63;
-                const int i = 32 * (off >> 13) + 4 * (((off >> 4) & 7) ^ (t & 7));   // first column
-                const float4 x = *reinterpret_cast<const float4 *>(sm + OFF_TB + off);
-                const float4 g = *reinterpret_cast<const float4 *>(gam + i);
-                *reinterpret_cast<float4 *>(sm + OFF_TG + off) =
-                    make_float4(to_tf32(x.x * g.x), to_tf32(x.y * g.y), to_tf32(x.z * g.z), to_tf32(x.w * g.w));
+        if (lane == 0) {
+            bool ok = true;
+            int n_kq = nchunks > 0 ? 1 : 0, n_tb = n_kq, n_tg = n_kq, n_kmn = n_kq, n_pm = n_kq;
+            int n_v[2] = {nchunks > 0 ? 1 : 0, nchunks > 1 ? 1 : 0};
+            int n_gr[2] = {nchunks > 0 ? 1 : 0, nchunks > 1 ? 1 : 0};
+            for (int c = 0; c < nchunks && ok; ++c) {
+                const uint32_t par = c & 1;
+                const bool more = c + 1 < nchunks;
+                // MMA_2a of c has read T_beta and its V buffer: T_beta of c+1, V of c+2
+                if (!(ok = wait_or_abort(&bar[B_2A], par, abort_flag))) break;
+                if (more) { issue_tb(c + 1); ++n_tb; }
+                if (c + 2 < nchunks) { issue_v(c + 2); ++n_v[c & 1]; }
+                // [K;Q] of c is consumed once MMA_1 of c is done
+                if (!(ok = wait_or_abort(&bar[B_1], par, abort_flag))) break;
+                if (more) { issue_kq(c + 1); ++n_kq; }
+                // T_beta_gamma once MMA_2b of c is done
+                if (!(ok = wait_or_abort(&bar[B_2], par, abort_flag))) break;
+                if (more) { issue_tg(c + 1); ++n_tg; }
+                // P once MMA_4 of c is done; K and this gates buffer once MMA_3 of c is done
+                // (the epilogue took the gates of c before MMA_3 could start)
+                if (!(ok = wait_or_abort(&bar[B_4], par, abort_flag))) break;
+                if (more) { issue_pm(c + 1); ++n_pm; }
+                if (!(ok = wait_or_abort(&bar[B_3], par, abort_flag))) break;
+                if (more) { issue_kmn(c + 1); ++n_kmn; }
+                if (c + 2 < nchunks) { issue_gr(c + 2); ++n_gr[c & 1]; }
             }
-            fence_smem_to_async();   // visible to the tensor core
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bar[B_TG]);
-            return true;
-        };
-        bool ok = nchunks == 0 || build_tg(0);
-        int n_kq = nchunks > 0 ? 1 : 0, n_v = n_kq, n_kmn = n_kq, n_pm = n_kq;
-        int n_gr[2] = {nchunks > 0 ? 1 : 0, nchunks > 1 ? 1 : 0};
-        for (int c = 0; c < nchunks && ok; ++c) {
-            const uint32_t par = c & 1;
-            const bool more = c + 1 < nchunks;
-            // [K;Q] of c is consumed once MMA_1 of c is done
-            if (!(ok = wwait(B_1, par))) break;
-            if (more && lane == 0) { issue_kq(c + 1); ++n_kq; }
-            // V and T_beta once MMA_2a of c is done (early enough for MMA_2a of c+1 to be issued
-            // before MMA_1 of c+1)
-            if (!(ok = wwait(B_2A, par))) break;
-            if (more && lane == 0) { issue_v(c + 1); ++n_v; }
-            // P once MMA_4 of c is done; K and this gates buffer once MMA_3 of c is done
-            // (the epilogue took the gates of c before MMA_3 could start)
-            if (!(ok = wwait(B_4, par))) break;
-            if (more && lane == 0) { issue_pm(c + 1); ++n_pm; }
-            if (!(ok = wwait(B_3, par))) break;
-            if (more && lane == 0) { issue_kmn(c + 1); ++n_kmn; }
-            if (c + 2 < nchunks && lane == 0) { issue_gr(c + 2); ++n_gr[c & 1]; }
-            // T_beta_gamma of c+1: MMA_2b of c (before MMA_3 of c) has read the buffer
-            if (more && !(ok = build_tg(c + 1))) break;
+            if (!ok) {  // wait (bounded) for the copies this thread started
+                const int counts[5] = {n_kq, n_tb, n_tg, n_kmn, n_pm};
+                const int bars[5] = {B_KQ, B_TB, B_TG, B_KMN, B_PL};
+                for (int i = 0; i < 5; ++i)
+                    if (counts[i]) mbar_wait(&bar[bars[i]], (uint32_t)(counts[i] - 1) & 1, kWaitTries);
+                for (int i = 0; i < 2; ++i) {
+                    if (n_v[i]) mbar_wait(&bar[B_V0 + i], (uint32_t)(n_v[i] - 1) & 1, kWaitTries);
+                    if (n_gr[i]) mbar_wait(&bar[B_GR0 + i], (uint32_t)(n_gr[i] - 1) & 1, kWaitTries);
+                }
+            }
         }
-        if (!ok && lane == 0) {  // wait (bounded) for the copies this thread started
-            const int counts[4] = {n_kq, n_v, n_kmn, n_pm};
-            const int bars[4] = {B_KQ, B_V, B_KMN, B_PL};
-            for (int i = 0; i < 4; ++i)
-                if (counts[i]) mbar_wait(&bar[bars[i]], (uint32_t)(counts[i] - 1) & 1, kWaitTries);
-            for (int i = 0; i < 2; ++i)
-                if (n_gr[i]) mbar_wait(&bar[B_GR0 + i], (uint32_t)(n_gr[i] - 1) & 1, kWaitTries);
-        }
-    } else {
+    } else if (warp < kDrainWarp0) {
         // ================================================================ epilogue
         const int q = warp & 3;
         const uint32_t lrow = (uint32_t)(32 * q) << 16;
@@ -432,38 +422,14 @@ __global__ void __launch_bounds__(kThr, 1) prefill_tc_kernel(const __grid_consta
             tmem_st32(tm + lrow + dst, v0);
             tmem_st32(tm + lrow + dst + 32, v1);
         };
-        // gated output: rows 32*h2 + i (i < 32) of the chunk held in v, this thread's column j,
-        // become y / sqrt(mean_j y^2 + eps) * w_j * SiLU(z); the row sums are reduced over the
-        // warp's lanes in registers, then over the 4 warps in shared memory
-        float *red = (float *)(sm + OFF_RED), *rinv = red + 128;
-        auto gate32 = [&](float(&v)[32], int h2, int n, int64_t tok) {
-            const int j = 32 * q + lane;
-            const int64_t v_row = (int64_t)p.n_v * kHeadDim;
-            const TZ *zp = (const TZ *)p.z + (tok + 32 * h2) * v_row + h * kHeadDim + j;
-            float zv[32], sq[32];
-#pragma unroll
-            for (int i = 0; i < 32; ++i) zv[i] = 32 * h2 + i < n ? to_f32(zp[(int64_t)i * v_row]) : 0.f;
-#pragma unroll
-            for (int i = 0; i < 32; ++i) sq[i] = v[i] * v[i];
-            red[32 * q + lane] = warp_row_sums32(sq, lane);
-            bar_sync(kBarEpi, 128);
-            if (warp == kEpiWarp0)
-                rinv[lane] = rsqrtf((red[lane] + red[32 + lane] + red[64 + lane] + red[96 + lane]) *
-                                        (1.f / kHeadDim) + p.norm_eps);
-            bar_sync(kBarEpi, 128);
-            const float wj = p.norm_w[j];
-#pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] = v[i] * rinv[i] * wj * (zv[i] / (1.f + expf(-zv[i])));
-        };
         for (int c = 0; c < nchunks; ++c) {
             const uint32_t par = c & 1;
             const int bsel = c & 1;
-            const int n = min(kChunk, L - (cb + c) * kChunk);
-            const int64_t tok = seq0 + (int64_t)(cb + c) * kChunk;
-            {  // MMA_1 done and the gates record of c here (one poll round for both)
+            {  // MMA_1 done, the gates record of c here, and Y of c-1 read by the drain group
                 bool ok = true;
                 if (leader) ok = wait_or_abort(&bar[B_1], par, abort_flag) &&
-                                 wait_or_abort(&bar[B_GR0 + bsel], (c >> 1) & 1, abort_flag);
+                                 wait_or_abort(&bar[B_GR0 + bsel], (c >> 1) & 1, abort_flag) &&
+                                 (c == 0 || wait_or_abort(&bar[B_YF], par ^ 1, abort_flag));
                 if (bar_or(kBarEpi, 128, !ok)) break;
             }
             fence_after_sync();
@@ -487,65 +453,82 @@ __global__ void __launch_bounds__(kThr, 1) prefill_tc_kernel(const __grid_consta
             fence_after_sync();
             scale64(T_U + 64 * par, T_XY, gr + kGrKd);     // u~ = u diag(kd) over X, for MMA_3
             publish(B_UT);
-            if (!ewait(B_4, par)) break;
+        }
+    } else {
+        // ================================================================ drain group (warps 6-9)
+        // After MMA_4 of chunk c, read Y (this warp's 32 lanes = columns j of y, 64 tokens) and
+        // free the tensor memory for chunk c+1 at once; then write y (gated when GATED) by 32-row
+        // halves: staged in shared memory and written with one TMA store for a full chunk, or
+        // stored directly (rows of the chunk only) for a sequence's last, partial chunk.
+        const int q = warp & 3, j = 32 * q + lane;
+        const uint32_t lrow = (uint32_t)(32 * q) << 16;
+        const bool dleader = tid == kDrainTid0;
+        const int64_t v_row = (int64_t)p.n_v * kHeadDim;
+        float wj = 0.f;
+        if constexpr (GATED) wj = p.norm_w[j];
+        for (int c = 0; c < nchunks; ++c) {
+            const int n = min(kChunk, L - (cb + c) * kChunk);
+            const int64_t tok = seq0 + (int64_t)(cb + c) * kChunk;
+            {
+                const bool ok = dleader ? wait_or_abort(&bar[B_4], c & 1, abort_flag) : true;
+                if (bar_or(kBarDrain, 128, !ok)) break;
+            }
             fence_after_sync();
-            if (n == kChunk) {
-                // full chunk: rows 32*h2.. staged in buffer h2 (row t, column j) and written
-                // with one TMA store each; a buffer is rewritten once the store issued from it
-                // one chunk earlier has read it (the leader's bulk groups complete in order)
-                const int j = 32 * q + lane;
+            float v[2][32];
+            tmem_ld32(tm + lrow + T_Y, v[0]);
+            tmem_ld32(tm + lrow + T_Y + 32, v[1]);
+            tmem_wait_ld();
+            tmem_regs_after_wait(v[0]);
+            tmem_regs_after_wait(v[1]);
+            fence_before_sync();
+            bar_sync(kBarDrain, 128);
+            if (dleader) mbar_arrive(&bar[B_YF]);              // the epilogue may rewrite Y
 #pragma unroll
-                for (int h2 = 0; h2 < 2; ++h2) {
-                    TO *ys = (TO *)(sm + OFF_YST + h2 * 16384);
-                    float v[32];
-                    tmem_ld32(tm + lrow + T_Y + 32 * h2, v);
-                    tmem_wait_ld();
-                    tmem_regs_after_wait(v);
-                    if constexpr (GATED) gate32(v, h2, kChunk, tok);
-                    if (leader) bulk_wait_read1();
-                    bar_sync(kBarEpi, 128);
+            for (int h2 = 0; h2 < 2; ++h2) {
+                const int row0 = 32 * h2;
+                // the staging (also the scratch of the gated rows) is free once the previous TMA
+                // store has read it
+                if (dleader) bulk_wait_read0();
+                bar_sync(kBarDrain, 128);
+                if constexpr (GATED) {
+                    // out = y / sqrt(mean_j y^2 + eps) * w_j * SiLU(z): row sums over this warp's
+                    // 32 columns in registers, over the 4 warps in a scratch in the staging
+                    float zv[32], sq[32];
+                    const TZ *zp = (const TZ *)p.z + (tok + row0) * v_row + h * kHeadDim + j;
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) ys[i * kHeadDim + j] = from_f32<TO>(v[i]);
+                    for (int i = 0; i < 32; ++i) zv[i] = row0 + i < n ? to_f32(zp[(int64_t)i * v_row]) : 0.f;
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) sq[i] = v[h2][i] * v[h2][i];
+                    float *red = (float *)(sm + OFF_YST), *rinv = red + 128;
+                    red[32 * q + lane] = warp_row_sums32(sq, lane);
+                    bar_sync(kBarDrain, 128);
+                    if (warp == kDrainWarp0)
+                        rinv[lane] = rsqrtf((red[lane] + red[32 + lane] + red[64 + lane] + red[96 + lane]) *
+                                                (1.f / kHeadDim) + p.norm_eps);
+                    bar_sync(kBarDrain, 128);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) v[h2][i] *= rinv[i] * wj * (zv[i] / (1.f + expf(-zv[i])));
+                    bar_sync(kBarDrain, 128);   // the scratch is read before the staging is written
+                }
+                if (n == kChunk) {
+                    TO *ys = (TO *)(sm + OFF_YST);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) ys[i * kHeadDim + j] = from_f32<TO>(v[h2][i]);
                     fence_smem_to_async();
-                    bar_sync(kBarEpi, 128);
-                    if (leader) {
-                        tma_store_2d(&p.tm_out, h * kHeadDim, (int)tok + 32 * h2, sb + OFF_YST + h2 * 16384);
+                    bar_sync(kBarDrain, 128);
+                    if (dleader) {
+                        tma_store_2d(&p.tm_out, h * kHeadDim, (int)tok + row0, sb + OFF_YST);
                         bulk_commit();
                     }
-                }
-            } else {
-                // last, partial chunk: direct stores of rows t < n.  Each lane holds column j
-                // for all t; a 4 x 4 transpose inside each group of 4 lanes gives lane e of the
-                // group 4 consecutive columns of row t0 + e.
-                const int e = lane & 3;
-                const int64_t v_row = (int64_t)p.n_v * kHeadDim;
-                TO *o = (TO *)p.out + tok * v_row + h * kHeadDim + 32 * q + 4 * (lane >> 2);
+                } else {
+                    TO *o = (TO *)p.out + (tok + row0) * v_row + h * kHeadDim + j;
 #pragma unroll
-                for (int h2 = 0; h2 < 2; ++h2) {
-                    float v[32];
-                    tmem_ld32(tm + lrow + T_Y + 32 * h2, v);
-                    tmem_wait_ld();
-                    tmem_regs_after_wait(v);
-                    if constexpr (GATED) gate32(v, h2, n, tok);
-#pragma unroll
-                    for (int blk = 0; blk < 8; ++blk) {
-                        float a[4] = {v[4 * blk], v[4 * blk + 1], v[4 * blk + 2], v[4 * blk + 3]};
-                        float x = (e & 1) ? a[0] : a[1], y2 = (e & 1) ? a[2] : a[3];
-                        x = __shfl_xor_sync(0xffffffffu, x, 1);
-                        y2 = __shfl_xor_sync(0xffffffffu, y2, 1);
-                        if (e & 1) { a[0] = x; a[2] = y2; } else { a[1] = x; a[3] = y2; }
-                        x = (e & 2) ? a[0] : a[2];
-                        y2 = (e & 2) ? a[1] : a[3];
-                        x = __shfl_xor_sync(0xffffffffu, x, 2);
-                        y2 = __shfl_xor_sync(0xffffffffu, y2, 2);
-                        if (e & 2) { a[0] = x; a[1] = y2; } else { a[2] = x; a[3] = y2; }
-                        const int t = 32 * h2 + 4 * blk + e;
-                        if (t < n) st4(o + (int64_t)t * v_row, a);
-                    }
+                    for (int i = 0; i < 32; ++i)
+                        if (row0 + i < n) o[(int64_t)i * v_row] = from_f32<TO>(v[h2][i]);
                 }
             }
         }
-        if (leader) bulk_wait0();   // this thread's y stores are complete
+        if (dleader) bulk_wait0();   // this thread's y stores are complete
     }
 
     // ---------------------------------------------------------------- tear-down
@@ -607,7 +590,7 @@ cudaError_t launch_prefill_tc(const ScanParams &sp, int64_t total_tokens, bool /
                               bool out_bf16, cudaStream_t s) {
     if (sp.n_seqs <= 0) return cudaSuccess;
     TcParams p{};
-    p.kq = sp.kq; p.kmn = sp.kmn; p.vi = sp.vi; p.tb = sp.tb; p.pm = sp.pm; p.gr = sp.gr;
+    p.kq = sp.kq; p.kmn = sp.kmn; p.vi = sp.vi; p.tb = sp.tb; p.tg = sp.tg; p.pm = sp.pm; p.gr = sp.gr;
     p.cu = sp.cu; p.cfirst = sp.cfirst; p.init = sp.init; p.carry_in = sp.carry_in; p.carry_out = sp.carry_out;
     p.rg = sp.rg;
     p.out = sp.out; p.n_seqs = sp.n_seqs; p.n_qk = sp.n_qk; p.n_v = sp.n_v;

@@ -256,7 +256,7 @@ def test_short_ranges_from_small_workspace(lib, with_final):
     cs = to_dev(inp.conv_state, d)
     T, n = inp.total_tokens, inp.n_seqs
     pref = lib.prefill_workspace_size(cfg, torch.bfloat16, T, n, 700)
-    slot = 4 * (65536 + 32768) + 12 * (32768 + 2 * 16384 + 640)
+    slot = 4 * (65536 + 32768) + 12 * (32768 + 3 * 16384 + 640)
     small = 2 * n * slot + n * 12 * 65536 + (1 << 16)   # two buffers of one chunk per sequence
     assert small < pref
     ws = torch.empty(small, dtype=torch.uint8, device="cuda")
@@ -281,7 +281,7 @@ def test_sequence_longer_than_max_seqlen(lib):
     shape = gi.GdnShape(n_qk_heads=2, n_v_heads=6)
     inp = gi.make_prefill_inputs(shape, [300, 1000], gi.BF16, seed=85, with_initial_state=True)
     cfg = lib.GdnConfig(2, 6)
-    slot = 2 * (65536 + 32768) + 6 * (32768 + 2 * 16384 + 640)
+    slot = 2 * (65536 + 32768) + 6 * (32768 + 3 * 16384 + 640)
     ws = torch.empty(2 * 2 * slot + 2 * 6 * 65536 + (1 << 14), dtype=torch.uint8, device="cuda")
     y, fin, _ = lib.gdn_prefill(*prefill_args(inp, lib), cfg=cfg, workspace=ws, max_seqlen=300,
                                 initial_state=torch.from_numpy(inp.initial_state).cuda())
