@@ -55,8 +55,11 @@ CHUNK = 64
 # + K.K^T and Q.K^T (2 C d each, shared by the 3 V heads of a QK head)
 PREFILL_FLOP_TV = 6 * D * D + 2 * CHUNK * D * (3 + 2 / 3)
 # tensor-core work of the chunk-chain kernel per (token, V head): S^T[K;Q]^T (4 d^2),
-# V^T T_beta^T and X' T_beta^T (2 C d each), u~^T K (2 d^2), u^T P^T (2 C d)
-CHAIN_FLOP_TV = 6 * D * D + 3 * 2 * CHUNK * D
+# V^T T_beta^T and X T_beta_gamma^T (2 C d each) on TF32 operands; u~^T K (2 d^2) and
+# u^T P^T (2 C d) on fp16 operands
+CHAIN_FLOP_TV_TF32 = 4 * D * D + 2 * 2 * CHUNK * D
+CHAIN_FLOP_TV_F16 = 2 * D * D + 2 * CHUNK * D
+CHAIN_FLOP_TV = CHAIN_FLOP_TV_TF32 + CHAIN_FLOP_TV_F16
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
                   "sm_max_mhz": 1965.0}
 TF32_PER_BF16 = 1.1 / 2.25   # nominal dense tf32 : bf16 tensor throughput on B200
@@ -437,13 +440,17 @@ def prefill_roofline(res, peaks, peak_src, sha):
                 "algorithmic_per_launch": flops, "tokens_per_launch": T, "kernel_share": share}
     if dom.startswith("prefill_tc"):
         flops = CHAIN_FLOP_TV * T * Hv
-        peak = bf16 * TF32_PER_BF16
+        # the time the chain's MMAs take at peak: the TF32 part at the TF32 rate, the fp16
+        # part at the fp16 (= bf16) rate
+        tf32 = bf16 * TF32_PER_BF16
+        peak = CHAIN_FLOP_TV / (CHAIN_FLOP_TV_TF32 / tf32 + CHAIN_FLOP_TV_F16 / bf16)
         traffic, tsrc = traffic_for(dom, res["workload"], T, sha)
         ach = flops / avg_s / 1e12
         return {"kernel": dom, "bound": "tensor", "achieved": ach, "peak": peak,
                 "unit": "TFLOP/s", "frac": ach / peak, "frac_of_bf16_peak": ach / bf16,
                 "traffic": traffic, "traffic_source": tsrc,
-                "peak_source": f"tf32 = {peak_src} bf16 {bf16} x 1.1/2.25 nominal",
+                "peak_source": (f"{peak_src} bf16 {bf16} for the fp16 third of the MMA flops, "
+                                f"x 1.1/2.25 nominal (tf32) for the other two thirds"),
                 "algorithmic_per_launch": flops, "tokens_per_launch": T, "kernel_share": share}
     # a memory-bound kernel dominates
     byts = (2 * 16 * D * 2 + 48 * D * 2 + 3 * 16 * 4 * D) * T

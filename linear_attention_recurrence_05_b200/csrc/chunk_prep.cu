@@ -7,10 +7,10 @@
 //     A_ti = beta_t exp(g_t - g_i) k_t.k_i        (i < t < n, else 0)
 //     T    = (I + A)^-1,   T_beta = T diag(beta),   T_beta_gamma = T diag(beta gamma)
 //     P_ti = exp(g_t - g_i) q_t.k_i               (i <= t < n, else 0)
-// T_beta, T_beta_gamma and P (64 x 64) are written as fp32 tiles rounded to TF32 (the precision the
-// tensor-core chain reads them in), already in the shared-memory layout of an MMA operand
-// (K-major, 128-byte rows with 16-byte chunks XOR-swizzled by row), for the chain kernel to
-// stream in with one bulk copy each.  A gates record per (chunk, head) carries gamma_t,
+// T_beta and T_beta_gamma (64 x 64) are written as fp32 tiles rounded to TF32, P as an fp16
+// tile (the precisions the tensor-core chain reads them in), already in the shared-memory
+// layout of an MMA operand (K-major, 128-byte rows with 16-byte chunks XOR-swizzled by row),
+// for the chain kernel to stream in with one bulk copy each.  A gates record per (chunk, head) carries gamma_t,
 // kd_t and gamma_C = exp(g_{n-1}), the per-token factors the chain applies in tensor memory.
 //
 // One CTA per (chunk, group of up to 3 V heads of one QK head): K K^T and Q K^T do not
@@ -71,7 +71,7 @@ struct PrepParams {
     const void *alpha, *beta;
     const int32_t *cu, *cfirst;
     const int32_t *cseq;  // sequence of each slot (compact numbering)
-    float *tb, *tg, *pm;  // [slot, Hv] tiles (16 KB each)
+    float *tb, *tg, *pm;  // [slot, Hv] tiles (16 KB each; P 8 KB)
     float *gr;            // [slot, Hv] gates records
     int n_seqs, n_qk, n_v;
     ChunkRange rg;        // the range of this launch
@@ -180,7 +180,7 @@ __global__ void __launch_bounds__(kGroupThr * kMaxGroups, 2) chunk_prep_kernel(c
     fence_after_sync();
     if (ok) {
         // Row t of K K^T (lane quarters 0-1) becomes row t of -A, written transposed into the
-        // parity arrays; row t of Q K^T (quarters 2-3) becomes row t of P, TF32, stored to
+        // parity arrays; row t of Q K^T (quarters 2-3) becomes row t of P, fp16, stored to
         // global memory in the K-major image.  exp(g_t - g_i) = gamma_t / gamma_i while the
         // chunk's total decay keeps 1 / gamma finite; otherwise one exponential per element.
         const int q = warp & 3;
@@ -216,12 +216,12 @@ __global__ void __launch_bounds__(kGroupThr * kMaxGroups, 2) chunk_prep_kernel(c
                 float *at = (float *)(scr + (t & 1) * kParStride) + (t >> 1) + 32 * 32 * h2;
 #pragma unroll
                 for (int e = 0; e < 32; ++e) at[e * 32] = v[e];
-            } else {
-                unsigned char *dst = (unsigned char *)(p.pm + tile * 4096);
+            } else {   // fp16 (nearest even), K-major
+                unsigned char *dst = (unsigned char *)(p.pm + tile * 2048);
 #pragma unroll
                 for (int k = 0; k < 8; ++k)
-                    *reinterpret_cast<float4 *>(dst + kmaj_off(t, 32 * h2 + 4 * k, 64)) =
-                        tf32x4(make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]));
+                    *reinterpret_cast<uint2 *>(dst + kmaj16_off(t, 32 * h2 + 4 * k)) =
+                        make_uint2(pack_f16x2(v[4 * k], v[4 * k + 1]), pack_f16x2(v[4 * k + 2], v[4 * k + 3]));
             }
         }
     }

@@ -169,12 +169,12 @@ __global__ void __launch_bounds__(128) conv_l2_kernel(ConvParams p) {
 
 // ------------------------------------------------------------------------ conv + L2, tiles
 // The tensor-core path's tiles from bf16 input.  CTA = one 64-row chunk of one head slot:
-// q heads ([K;Q] tile, Q half), k heads ([K;Q] tile, K half, and the K tile, MN-major), v
-// heads (the V tile, MN-major).  One TMA copy brings the chunk's rows and the 3 rows before
+// q heads ([K;Q] tile, Q half), k heads ([K;Q] tile, K half, and the fp16 K tile, MN-major),
+// v heads (the V tile, MN-major).  One TMA copy brings the chunk's rows and the 3 rows before
 // them (rows outside the tensor read as zero; at a sequence's start the 3 history rows are
 // replaced by the conv state or zeros); each warp then walks 16 rows from shared memory and
-// stores each TF32-rounded row straight into the tile: in both layouts the 32 lanes of a
-// warp cover one row of the 4 feature blocks, four whole 128-byte lines.
+// stores each row straight into the tiles, TF32-rounded (and fp16 for the K tile): the 32
+// lanes of a warp cover one row, whole 128-byte lines.
 namespace {
 using namespace tc;
 
@@ -320,9 +320,14 @@ __global__ void __launch_bounds__(128) conv_tiles_kernel(const __grid_constant__
             unsigned char *kq = reinterpret_cast<unsigned char *>(p.kq + ((int64_t)ci * nq + head) * 16384 +
                                                                  (kind == 0 ? 2048 : 0));
             *reinterpret_cast<float4 *>(kq + (lane >> 3) * 16384 + t * 128 + (((lane & 7) ^ (t & 7)) << 4)) = o;
-            if (kind == 1)   // the K tile, MN-major
-                *reinterpret_cast<float4 *>(reinterpret_cast<unsigned char *>(
-                    p.kmn + ((int64_t)ci * nq + head) * 8192) + mn_off) = o;
+            if (kind == 1) {   // the K tile, fp16 (nearest even), MN-major
+                const float4 f = ok ? make_float4(t < len ? y[0] : 0.f, t < len ? y[1] : 0.f,
+                                                  t < len ? y[2] : 0.f, t < len ? y[3] : 0.f)
+                                    : o;
+                *reinterpret_cast<uint2 *>(reinterpret_cast<unsigned char *>(
+                    p.kmn + ((int64_t)ci * nq + head) * 4096) + tc::mn16_off(t, 4 * lane, kChunk)) =
+                    make_uint2(tc::pack_f16x2(f.x, f.y), tc::pack_f16x2(f.z, f.w));
+            }
         }
     }
     if (!ok && threadIdx.x == 0) mbar_wait(bar, 0, kConvWaitTries);   // the copy is done before exit

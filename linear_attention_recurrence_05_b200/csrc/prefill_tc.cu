@@ -1,5 +1,5 @@
-// Chunked gated-delta-rule prefill on the sm_100a tensor cores (TF32 MMAs, fp32 state):
-// the serial chain over the chunks of one (sequence, V head).
+// Chunked gated-delta-rule prefill on the sm_100a tensor cores (TF32 and fp16 MMAs, fp32
+// accumulators and state): the serial chain over the chunks of one (sequence, V head).
 //
 // The recurrence of the page "ARCHITECTURE PREVIEW / FIELD NOTES", section 03 (GATED
 // DELTANET equations), in chunks of 64 tokens.  Within a chunk, with
@@ -22,19 +22,25 @@
 //     MMA_1   [X | Y1] = S^T [K;Q]^T         (N=128, K=128)   X = (K S)^T, Y1 = (Q S)^T
 //     MMA_2a  U^T      = V^T T_beta^T        (N=64,  K=64)    state-independent
 //     MMA_2b  U^T     -= X T_beta_gamma^T    (N=64,  K=64)    -> u^T
-//     MMA_4   Y       += u^T P^T             (N=64,  K=64)    onto Y = Y1 diag(gamma)
 //     MMA_3   S^T     += u~^T K              (N=128, K=64)    u~ = u diag(kd), onto gamma_C S^T
+//     MMA_4   Y       += u^T P^T             (N=64,  K=64)    onto Y = Y1 diag(gamma)
+//   MMA_1 and MMA_2a/2b take TF32 operands (fp32 in shared or tensor memory).  MMA_3 and
+//   MMA_4 take fp16 operands (kind::f16): u~ and u as fp16 pairs in tensor memory, written by
+//   the epilogue when it forms u~, and K and P as fp16 tiles.  fp16 carries the 11-bit
+//   significand of TF32; its range (|x| < 65504) holds u, u~ (u times decays <= 1), the unit
+//   keys and P (|P| <= 1) for activations of any sensible size, and a u beyond it turns the
+//   state into inf/NaN rather than into a wrong finite value.
 //   V is double-buffered (a chunk ahead) and T_beta reloaded as soon as MMA_2a has read it, so
 //   MMA_2a(c+1) is normally issued right after MMA_3(c) and runs while the new state is waited
 //   for; MMA_2b reads X straight from MMA_1's output.  The only epilogue step left on the
-//   critical path is u~; MMA_4 runs while it is formed.  u^T is double-buffered in tensor
-//   memory (chunk parity).
+//   critical path is u~.  u^T is double-buffered in tensor memory (chunk parity).
 //   epilogue (warps 1-4), in tensor memory: after MMA_1, Y = Y1 diag(gamma) (once the drain
 //     group has read the previous Y) and S^T *= gamma_C; after MMA_2b, u~ (over X, which
 //     MMA_2b has consumed); the state entering and leaving the range.
 //   producer (warp 5): the tile loads, each issued as soon as its buffer is free.
 //   drain group (warps 6-9): after MMA_4, reads Y and frees it at once, then writes y (or the
-//     gated output) through shared memory with TMA stores.
+//     gated output) through shared memory with TMA stores; a bf16 gate input z arrives by
+//     one TMA load per chunk, issued a chunk ahead.
 // All waits are bounded; a CTA that times out writes NaN to its outputs.
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -61,15 +67,16 @@ constexpr int kBarDrain = 2;       // named barrier of the drain group (128 thre
 
 // shared-memory map (bytes from a 1024-aligned base)
 constexpr uint32_t OFF_KQ = 0;          // [K;Q]   K-major, 4 blocks x (K 8 KB | Q 8 KB)       64 KB
-constexpr uint32_t OFF_KMN = 65536;     // K       MN-major (32-byte granules), 64 x 128       32 KB
+constexpr uint32_t OFF_KMN = 65536;     // K       fp16, MN-major, 64 x 128                    16 KB
+constexpr uint32_t OFF_Z = 81920;       // gate input z of a chunk, bf16, 64 rows x 256 B     16 KB
 constexpr uint32_t OFF_V = 98304;       // V       MN-major, 2 buffers (chunk parity)      2 x 32 KB
 constexpr uint32_t OFF_TB = 163840;     // T_beta        K-major [t][i]                        16 KB
 constexpr uint32_t OFF_TG = 180224;     // T_beta_gamma  K-major [t][i]                        16 KB
-constexpr uint32_t OFF_P = 196608;      // P       K-major [t][i]                              16 KB
+constexpr uint32_t OFF_P = 196608;      // P       fp16, K-major [t][i]                         8 KB
 constexpr uint32_t OFF_YST = 212992;    // y staging: 32 rows x 128 columns (TMA store box)    16 KB
 constexpr uint32_t OFF_GR = 229376;     // gates records, 2 buffers                          1280 B
 constexpr uint32_t OFF_BAR = OFF_GR + 2 * kGateRec * 4;   // mbarriers
-constexpr uint32_t OFF_FLAGS = OFF_BAR + 144;             // TMEM base, abort flag
+constexpr uint32_t OFF_FLAGS = OFF_BAR + 160;             // TMEM base, abort flag
 constexpr uint32_t kSmem = OFF_FLAGS + 16;
 constexpr uint32_t kSmemAlloc = kSmem + 1024;              // slack to align the base to 1024
 static_assert(kSmemAlloc <= 232448, "shared memory per CTA");
@@ -83,15 +90,16 @@ enum {
     B_UT,                                // epilogue: u~ = u diag(kd) stored
     B_YF,                                // drain group: Y read (tensor memory free for the next chunk)
     B_DRAIN0,                            // drain on the failure path
+    B_Z,                                 // gate input of a chunk arrived
     kNumBars
 };
-static_assert(kNumBars * 8 <= 144, "barrier area");
+static_assert(kNumBars * 8 <= 160, "barrier area");
 
 // tensor memory columns (all 128 lanes)
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t T_S = 0;      // S^T                               128 cols
-constexpr uint32_t T_XY = 128;   // [X | Y1]; u~^T over X once MMA_2b has read it   128 cols
-constexpr uint32_t T_U = 256;    // u^T, two buffers (chunk parity)    2 x 64 cols
+constexpr uint32_t T_XY = 128;   // [X | Y1]; fp16 u~^T over X once MMA_2b has read it  128 cols
+constexpr uint32_t T_U = 256;    // u^T, two buffers (chunk parity), then fp16 u^T  2 x 64 cols
 constexpr uint32_t T_Y = 384;    // gamma Y1, then y                    64 cols
 
 constexpr uint32_t kWaitTries = 1u << 22;
@@ -169,8 +177,10 @@ __device__ __forceinline__ void gemm_ts(uint32_t d_tmem, uint32_t a_tmem, uint32
 
 struct TcParams {
     CUtensorMap tm_out;   // y as [T, Hv*128] rows, boxes of 128 columns x 32 rows (no swizzle)
-    // per-chunk tiles of the range's buffer, by slot, in shared-memory layout: [K;Q] and K per
-    // (slot, QK head); V, T_beta, T_beta_gamma, P and the gates record per (slot, V head)
+    CUtensorMap tm_z;     // bf16 z as [T, Hv*128] rows, boxes of 128 columns x 64 rows
+    // per-chunk tiles of the range's buffer, by slot, in shared-memory layout: [K;Q] and K
+    // (fp16) per (slot, QK head); V, T_beta, T_beta_gamma, P (fp16) and the gates record per
+    // (slot, V head)
     const float *kq, *kmn, *vi, *tb, *tg, *pm, *gr;
     const int32_t *cu, *cfirst;
     const float *init, *carry_in;   // state entering chunk 0 / entering a later first chunk
@@ -235,11 +245,11 @@ __global__ void __launch_bounds__(kThr, 1) prefill_tc_kernel(const __grid_consta
     auto qk_tile = [&](const float *base, int c, int64_t floats) { return base + (slot(c) * p.n_qk + gq) * floats; };
     auto v_tile = [&](const float *base, int c, int64_t floats) { return base + (slot(c) * p.n_v + h) * floats; };
     auto issue_kq = [&](int c) { load(B_KQ, OFF_KQ, qk_tile(p.kq, c, 16384), 65536); };
-    auto issue_kmn = [&](int c) { load(B_KMN, OFF_KMN, qk_tile(p.kmn, c, 8192), 32768); };
+    auto issue_kmn = [&](int c) { load(B_KMN, OFF_KMN, qk_tile(p.kmn, c, 4096), 16384); };
     auto issue_v = [&](int c) { load(B_V0 + (c & 1), OFF_V + (c & 1) * 32768, v_tile(p.vi, c, 8192), 32768); };
     auto issue_tb = [&](int c) { load(B_TB, OFF_TB, v_tile(p.tb, c, 4096), 16384); };
     auto issue_tg = [&](int c) { load(B_TG, OFF_TG, v_tile(p.tg, c, 4096), 16384); };
-    auto issue_pm = [&](int c) { load(B_PL, OFF_P, v_tile(p.pm, c, 4096), 16384); };
+    auto issue_pm = [&](int c) { load(B_PL, OFF_P, v_tile(p.pm, c, 2048), 8192); };
     auto issue_gr = [&](int c) {  // gates record of chunk c into buffer c & 1
         load(B_GR0 + (c & 1), OFF_GR + (c & 1) * kGateRec * 4, v_tile(p.gr, c, kGateRec), kGateRec * 4);
     };
@@ -318,19 +328,20 @@ __global__ void __launch_bounds__(kThr, 1) prefill_tc_kernel(const __grid_consta
                 fence_after_sync();
                 gemm_ts<64, 64, false, true>(tm + T_U + 64 * bi, tm + T_XY, sb + OFF_TG, 8192, true);
                 mma_commit(&bar[B_2]);
-                // MMA_4: Y += u^T P^T onto Y = Y1 diag(gamma); the epilogue forms u~ meanwhile
-                if (!(ok = wait_or_abort(&bar[B_Y1], par, abort_flag))) break;
-                if (!(ok = wait_or_abort(&bar[B_PL], par, abort_flag))) break;
-                if (!(ok = wait_or_abort(&bar[B_2], par, abort_flag))) break;
-                fence_after_sync();
-                gemm_ts<64, 64, false, false>(tm + T_Y, tm + T_U + 64 * bi, sb + OFF_P, 8192, true);
-                mma_commit(&bar[B_4]);
-                // MMA_3: S^T += u~^T K onto gamma_C S^T (K in its MN-major tile)
+                // MMA_3: S^T += u~^T K onto gamma_C S^T (fp16: u~ from the epilogue, K tile
+                // MN-major)
                 if (!(ok = wait_or_abort(&bar[B_KMN], par, abort_flag))) break;
                 if (!(ok = wait_or_abort(&bar[B_UT], par, abort_flag))) break;
                 fence_after_sync();
-                gemm_ts<128, 64, true, false>(tm + T_S, tm + T_XY, sb + OFF_KMN, 64, true);
+                gemm_ts_f16<128, 64, true>(tm + T_S, tm + T_XY, sb + OFF_KMN, 64, true);
                 mma_commit(&bar[B_3]);
+                // MMA_4: Y += u^T P^T onto Y = Y1 diag(gamma) (fp16: u from the epilogue's u~
+                // step, P tile); off the state's path, it runs while the new state is waited for
+                if (!(ok = wait_or_abort(&bar[B_Y1], par, abort_flag))) break;
+                if (!(ok = wait_or_abort(&bar[B_PL], par, abort_flag))) break;
+                fence_after_sync();
+                gemm_ts_f16<64, 64, false>(tm + T_Y, tm + T_U + 64 * bi, sb + OFF_P, 0, true);
+                mma_commit(&bar[B_4]);
                 a2_issued = false;
                 if (c + 1 < nchunks) {
                     // MMA_2a of c+1 fills the wait for MMA_3 (its u^T buffer held u of c-1, read by
@@ -368,13 +379,13 @@ __global__ void __launch_bounds__(kThr, 1) prefill_tc_kernel(const __grid_consta
                 // T_beta_gamma once MMA_2b of c is done
                 if (!(ok = wait_or_abort(&bar[B_2], par, abort_flag))) break;
                 if (more) { issue_tg(c + 1); ++n_tg; }
-                // P once MMA_4 of c is done; K and this gates buffer once MMA_3 of c is done
-                // (the epilogue took the gates of c before MMA_3 could start)
-                if (!(ok = wait_or_abort(&bar[B_4], par, abort_flag))) break;
-                if (more) { issue_pm(c + 1); ++n_pm; }
+                // K and this gates buffer once MMA_3 of c is done (the epilogue took the gates
+                // of c before MMA_3 could start); P once MMA_4 of c is done
                 if (!(ok = wait_or_abort(&bar[B_3], par, abort_flag))) break;
                 if (more) { issue_kmn(c + 1); ++n_kmn; }
                 if (c + 2 < nchunks) { issue_gr(c + 2); ++n_gr[c & 1]; }
+                if (!(ok = wait_or_abort(&bar[B_4], par, abort_flag))) break;
+                if (more) { issue_pm(c + 1); ++n_pm; }
             }
             if (!ok) {  // wait (bounded) for the copies this thread started
                 const int counts[5] = {n_kq, n_tb, n_tg, n_kmn, n_pm};
@@ -451,7 +462,32 @@ __global__ void __launch_bounds__(kThr, 1) prefill_tc_kernel(const __grid_consta
             publish(B_Y1);
             if (!ewait(B_2, par)) break;
             fence_after_sync();
-            scale64(T_U + 64 * par, T_XY, gr + kGrKd);     // u~ = u diag(kd) over X, for MMA_3
+            {   // u (fp32, 64 columns) -> fp16 u over its first 32 columns, for MMA_4, and
+                // fp16 u~ = u diag(kd) over X's first 32 columns, for MMA_3
+                const uint32_t src = T_U + 64 * par;
+                const float *kd = gr + kGrKd;
+                float v0[32], v1[32], hu[32], ht[32];
+                tmem_ld32(tm + lrow + src, v0);
+                tmem_ld32(tm + lrow + src + 32, v1);
+                tmem_wait_ld();
+                tmem_regs_after_wait(v0);
+                tmem_regs_after_wait(v1);
+#pragma unroll
+                for (int i = 0; i < 32; i += 4) {
+                    const float4 a = *reinterpret_cast<const float4 *>(kd + i);
+                    const float4 b = *reinterpret_cast<const float4 *>(kd + 32 + i);
+                    hu[i / 2] = __uint_as_float(pack_f16x2(v0[i], v0[i + 1]));
+                    hu[i / 2 + 1] = __uint_as_float(pack_f16x2(v0[i + 2], v0[i + 3]));
+                    hu[16 + i / 2] = __uint_as_float(pack_f16x2(v1[i], v1[i + 1]));
+                    hu[16 + i / 2 + 1] = __uint_as_float(pack_f16x2(v1[i + 2], v1[i + 3]));
+                    ht[i / 2] = __uint_as_float(pack_f16x2(v0[i] * a.x, v0[i + 1] * a.y));
+                    ht[i / 2 + 1] = __uint_as_float(pack_f16x2(v0[i + 2] * a.z, v0[i + 3] * a.w));
+                    ht[16 + i / 2] = __uint_as_float(pack_f16x2(v1[i] * b.x, v1[i + 1] * b.y));
+                    ht[16 + i / 2 + 1] = __uint_as_float(pack_f16x2(v1[i + 2] * b.z, v1[i + 3] * b.w));
+                }
+                tmem_st32(tm + lrow + T_XY, ht);
+                tmem_st32(tm + lrow + src, hu);
+            }
             publish(B_UT);
         }
     } else {
@@ -466,11 +502,40 @@ __global__ void __launch_bounds__(kThr, 1) prefill_tc_kernel(const __grid_consta
         const int64_t v_row = (int64_t)p.n_v * kHeadDim;
         float wj = 0.f;
         if constexpr (GATED) wj = p.norm_w[j];
+        // bf16 z: the chunk's 64 rows by one TMA load into shared memory (rows past the last
+        // token read as zero), issued as soon as the previous chunk's rows have been read
+        constexpr bool kZTile = GATED && sizeof(TZ) == 2;
+        int z_issued = 0, z_done = 0;
+        auto issue_z = [&](int c) {
+            mbar_expect_tx(&bar[B_Z], 64 * kHeadDim * 2);
+            tma_load_2d(sb + OFF_Z, &p.tm_z, h * kHeadDim, (int)(seq0 + (int64_t)(cb + c) * kChunk), &bar[B_Z]);
+            ++z_issued;
+        };
+        if constexpr (kZTile)
+            if (dleader && nchunks > 0) issue_z(0);
+        // fp32 z: read per column into registers, raw (converted where they are used): rows
+        // past a partial chunk's end read its last row, so the 32 loads of a half carry no
+        // condition and are all in flight at once
+        TZ zr[2][32];
+        auto load_z = [&](int c, int h2) {
+            const int n = min(kChunk, L - (cb + c) * kChunk);
+            const TZ *zp = (const TZ *)p.z + (seq0 + (int64_t)(cb + c) * kChunk) * v_row + h * kHeadDim + j;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) zr[h2][i] = __ldg(zp + (int64_t)min(32 * h2 + i, n - 1) * v_row);
+        };
         for (int c = 0; c < nchunks; ++c) {
             const int n = min(kChunk, L - (cb + c) * kChunk);
             const int64_t tok = seq0 + (int64_t)(cb + c) * kChunk;
+            if constexpr (GATED && !kZTile) load_z(c, 0);   // in flight while MMA_4 runs
             {
-                const bool ok = dleader ? wait_or_abort(&bar[B_4], c & 1, abort_flag) : true;
+                bool ok = true;
+                if (dleader) {
+                    ok = wait_or_abort(&bar[B_4], c & 1, abort_flag);
+                    if (kZTile && ok) {
+                        ok = wait_or_abort(&bar[B_Z], c & 1, abort_flag);
+                        z_done += ok;
+                    }
+                }
                 if (bar_or(kBarDrain, 128, !ok)) break;
             }
             fence_after_sync();
@@ -483,6 +548,7 @@ __global__ void __launch_bounds__(kThr, 1) prefill_tc_kernel(const __grid_consta
             fence_before_sync();
             bar_sync(kBarDrain, 128);
             if (dleader) mbar_arrive(&bar[B_YF]);              // the epilogue may rewrite Y
+            if constexpr (GATED && !kZTile) load_z(c, 1);   // in flight while the first half is written
 #pragma unroll
             for (int h2 = 0; h2 < 2; ++h2) {
                 const int row0 = 32 * h2;
@@ -493,10 +559,7 @@ __global__ void __launch_bounds__(kThr, 1) prefill_tc_kernel(const __grid_consta
                 if constexpr (GATED) {
                     // out = y / sqrt(mean_j y^2 + eps) * w_j * SiLU(z): row sums over this warp's
                     // 32 columns in registers, over the 4 warps in a scratch in the staging
-                    float zv[32], sq[32];
-                    const TZ *zp = (const TZ *)p.z + (tok + row0) * v_row + h * kHeadDim + j;
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) zv[i] = row0 + i < n ? to_f32(zp[(int64_t)i * v_row]) : 0.f;
+                    float sq[32];
 #pragma unroll
                     for (int i = 0; i < 32; ++i) sq[i] = v[h2][i] * v[h2][i];
                     float *red = (float *)(sm + OFF_YST), *rinv = red + 128;
@@ -507,8 +570,17 @@ __global__ void __launch_bounds__(kThr, 1) prefill_tc_kernel(const __grid_consta
                                                 (1.f / kHeadDim) + p.norm_eps);
                     bar_sync(kBarDrain, 128);
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) v[h2][i] *= rinv[i] * wj * (zv[i] / (1.f + expf(-zv[i])));
-                    bar_sync(kBarDrain, 128);   // the scratch is read before the staging is written
+                    for (int i = 0; i < 32; ++i) {
+                        float zi;
+                        if constexpr (kZTile)
+                            zi = to_f32(reinterpret_cast<const bf16 *>(sm + OFF_Z)[(row0 + i) * kHeadDim + j]);
+                        else
+                            zi = to_f32(zr[h2][i]);
+                        v[h2][i] *= rinv[i] * wj * (zi / (1.f + expf(-zi)));
+                    }
+                    bar_sync(kBarDrain, 128);   // the scratch (and z) is read before the staging is written
+                    if constexpr (kZTile)
+                        if (h2 == 1 && dleader && c + 1 < nchunks) issue_z(c + 1);
                 }
                 if (n == kChunk) {
                     TO *ys = (TO *)(sm + OFF_YST);
@@ -529,6 +601,8 @@ __global__ void __launch_bounds__(kThr, 1) prefill_tc_kernel(const __grid_consta
             }
         }
         if (dleader) bulk_wait0();   // this thread's y stores are complete
+        if constexpr (kZTile)        // a z load still in flight after a failure
+            if (dleader && z_issued > z_done) mbar_wait(&bar[B_Z], (uint32_t)(z_issued - 1) & 1, kWaitTries);
     }
 
     // ---------------------------------------------------------------- tear-down
@@ -576,6 +650,10 @@ static cudaError_t launch_tc_t(TcParams p, int64_t total_tokens, cudaStream_t s)
     if (total_tokens > 0 &&   // with no tokens there is no output (and `out` may be null)
         !encode_2d(&p.tm_out, obf ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, p.out,
                    width, total_tokens, width * (int64_t)sizeof(TO), kHeadDim, 32, CU_TENSOR_MAP_SWIZZLE_NONE))
+        return cudaErrorInvalidValue;
+    if (GATED && sizeof(TZ) == 2 && total_tokens > 0 &&
+        !encode_2d(&p.tm_z, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.z, width, total_tokens, width * 2, kHeadDim, 64,
+                   CU_TENSOR_MAP_SWIZZLE_NONE))
         return cudaErrorInvalidValue;
     auto k = prefill_tc_kernel<TO, TZ, GATED>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemAlloc);

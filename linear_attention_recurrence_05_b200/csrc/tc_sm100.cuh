@@ -13,9 +13,18 @@
 //    K step s (8 rows) starts at +1024*s; LBO = R*128 B (next 32 columns), SBO = 512 B.
 // A matrix contracted over both of its indices (K of a chunk: over features in K K^T
 // and K S, over tokens in K^T u) is therefore staged in both layouts.
+//
+// fp16 operands (kind::f16, 16 K-elements per instruction): 128-byte rows of 64 elements,
+// 128-byte swizzle with 16-byte chunks (chunk c of row r at c ^ (r % 8)).
+//  * K-major [R x 64]: element (r, c) at r*128 + ((c/8) ^ (r%8))*16 + (c%8)*2; K step s
+//    (16 columns) starts at +32*s; SBO = 1024 B.
+//  * MN-major [R x C] (rows = K index): blocks of 64 columns, R*128 bytes each; K step s
+//    (16 rows) starts at +2048*s; LBO = R*128 B (next 64 columns), SBO = 1024 B (8 rows).
+// A from tensor memory holds two fp16 per 32-bit column, the lower K index in the low half.
 #pragma once
 
 #include <stdint.h>
+#include <cuda_fp16.h>
 
 namespace gdn {
 namespace tc {
@@ -33,6 +42,20 @@ __host__ __device__ __forceinline__ uint32_t kmaj_off(int r, int c, int R) {
 __host__ __device__ __forceinline__ uint32_t mn_off(int r, int c, int R) {
     return (uint32_t)((c >> 5) * R * 128 + r * 128 + ((((c & 31) >> 3) ^ (r & 3)) << 5) +
                       ((c & 7) << 2));
+}
+
+// byte offset of element (r, c) of a [R x 64] fp16 tile, K-major 128B swizzle
+__host__ __device__ __forceinline__ uint32_t kmaj16_off(int r, int c) {
+    return (uint32_t)(r * 128 + ((((c & 63) >> 3) ^ (r & 7)) << 4) + ((c & 7) << 1));
+}
+// byte offset of element (r, c) of a [R x C] fp16 tile, MN-major 128B swizzle
+__host__ __device__ __forceinline__ uint32_t mn16_off(int r, int c, int R) {
+    return (uint32_t)((c >> 6) * R * 128 + r * 128 + ((((c & 63) >> 3) ^ (r & 7)) << 4) + ((c & 7) << 1));
+}
+// two fp16 (nearest even) in one 32-bit word, `lo` in the low half
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+    const __half2 h = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t *>(&h);
 }
 
 // ------------------------------------------------------------------ descriptors
@@ -61,6 +84,13 @@ __host__ __device__ constexpr uint32_t idesc_tf32(int M, int N, bool a_mn, bool 
     return (1u << 4)                       // D format: f32
            | (2u << 7) | (2u << 10)        // A, B format: tf32
            | ((a_mn ? 1u : 0u) << 15) | ((b_mn ? 1u : 0u) << 16)
+           | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+// instruction descriptor: kind::f16 with fp16 A and B, fp32 accumulator, A K-major
+__host__ __device__ constexpr uint32_t idesc_f16(int M, int N, bool b_mn) {
+    return (1u << 4)                       // D format: f32 (A, B format 0: f16)
+           | ((b_mn ? 1u : 0u) << 16)
            | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
@@ -107,6 +137,24 @@ __device__ __forceinline__ void gemm(uint32_t d_tmem, uint32_t a_base, uint32_t 
         const uint32_t da = A_MN ? (uint32_t)(s * 64) : (uint32_t)((s >> 2) * a_blk16 + (s & 3) * 2);
         const uint32_t db = B_MN ? (uint32_t)(s * 64) : (uint32_t)((s >> 2) * b_blk16 + (s & 3) * 2);
         mma_tf32(d_tmem, a0 + da, b0 + db, id, (accumulate || s > 0) ? 1u : 0u);
+    }
+}
+
+// D[128 x N] (+)= A[128 x K] B[K x N] in fp16 (kind::f16), A from tensor memory (K/2
+// columns of packed pairs), B from shared memory: K-major [N x 64] (b_rows unused) or
+// MN-major [K x N] with b_rows = K.
+template <int N, int K, bool B_MN>
+__device__ __forceinline__ void gemm_ts_f16(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_base, int b_rows,
+                                            bool accumulate) {
+    constexpr uint32_t id = idesc_f16(128, N, B_MN);
+    const uint64_t b0 = B_MN ? smem_desc(b_base, (uint32_t)b_rows * 128u, 1024, 2) : smem_desc(b_base, 16, 1024, 2);
+#pragma unroll
+    for (int s = 0; s < K / 16; ++s) {
+        const uint32_t db = B_MN ? (uint32_t)(s * 128) : (uint32_t)(s * 2);   // 16-byte units
+        asm volatile(
+            "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+            "r"(a_tmem + 8u * s), "l"(b0 + db), "r"(id), "r"((accumulate || s > 0) ? 1u : 0u));
     }
 }
 
