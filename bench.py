@@ -391,7 +391,9 @@ def kernel_sources_sha256():
 
 def traffic_records():
     """`traffic-record:` lines of the ncu summaries: DRAM read + write bytes of one launch of a
-    kernel, the sources it was built from and the work of that launch."""
+    kernel, the sources it was built from and the work of that launch.  A record may also name
+    larger workloads of the same kernel (`applies_to`) whose launches move the same bytes per
+    unit of work, so that their figure scales from the captured one."""
     recs = {}
     pdir = os.path.join(ROOT, "profiles")
     for name in sorted(os.listdir(pdir)) if os.path.isdir(pdir) else []:
@@ -404,7 +406,8 @@ def traffic_records():
                         r = json.loads(line.split(":", 1)[1])
                     except ValueError:
                         continue
-                    recs[(r["kernel"], r["workload"])] = dict(r, file=name)
+                    for wl in [r["workload"]] + list(r.get("applies_to", [])):
+                        recs[(r["kernel"], wl)] = dict(r, file=name)
     return recs
 
 

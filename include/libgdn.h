@@ -111,7 +111,7 @@ GDN_EXPORT int gdn_api_version(void);
  * by two calls in flight.  For bf16 input it holds the sequence tables and the per-chunk
  * tiles of the tensor-core path for one or two chunk RANGES: range r covers chunks
  * [r*R, (r+1)*R) of every sequence (R chosen from n_seqs and max_seqlen), so its size grows
- * with n_seqs * R, not with total_tokens (about 4.9 MB per (sequence, chunk slot) at 16 QK /
+ * with n_seqs * R, not with total_tokens (about 3.7 MB per (sequence, chunk slot) at 16 QK /
  * 48 V heads, plus one fp32 state per (sequence, V head) carried between ranges).  Only when
  * one range covers the whole problem is it sized by the number of chunks instead.  For fp32
  * input (the fp32 CUDA-core path) it holds the convolved, normalised rows in fp32 (40 KB per
@@ -311,7 +311,7 @@ GDN_EXPORT gdn_status gdn_affine_combine(const gdn_config *cfg, const float *M, 
  *    ranges as long as fit (longer inputs just take more ranges).  Problems that do not fit
  *    even with one chunk per sequence per range are rejected with GDN_ERR_WORKSPACE on the
  *    host, before anything is looked up or enqueued: at 16 QK / 48 V heads, bf16 input,
- *    a call takes up to 8 sequences of any length; fp32 input needs 40 KB per token
+ *    a call takes up to 9 sequences of any length; fp32 input needs 40 KB per token
  *    (about 1,600 tokens per call).
  *  - Allocation: none; it calls no cudaMalloc, cudaFree or allocating library routine.
  *  - Set-up: the first call on each device (with that device current) looks up the

@@ -7,8 +7,8 @@
 //     A_ti = beta_t exp(g_t - g_i) k_t.k_i        (i < t < n, else 0)
 //     T    = (I + A)^-1,   T_beta = T diag(beta),   T_beta_gamma = T diag(beta gamma)
 //     P_ti = exp(g_t - g_i) q_t.k_i               (i <= t < n, else 0)
-// T_beta and T_beta_gamma (64 x 64) are written as fp32 tiles rounded to TF32, P as an fp16
-// tile (the precisions the tensor-core chain reads them in), already in the shared-memory
+// T_beta and P (64 x 64) are written as fp16 tiles and T_beta_gamma as an fp32 tile rounded to
+// TF32 (the precisions the tensor-core chain reads them in), already in the shared-memory
 // layout of an MMA operand (K-major, 128-byte rows with 16-byte chunks XOR-swizzled by row),
 // for the chain kernel to stream in with one bulk copy each.  A gates record per (chunk, head) carries gamma_t,
 // kd_t and gamma_C = exp(g_{n-1}), the per-token factors the chain applies in tensor memory.
@@ -71,7 +71,7 @@ struct PrepParams {
     const void *alpha, *beta;
     const int32_t *cu, *cfirst;
     const int32_t *cseq;  // sequence of each slot (compact numbering)
-    float *tb, *tg, *pm;  // [slot, Hv] tiles (16 KB each; P 8 KB)
+    float *tb, *tg, *pm;  // [slot, Hv] tiles (T_beta_gamma 16 KB; T_beta and P fp16, 8 KB)
     float *gr;            // [slot, Hv] gates records
     int n_seqs, n_qk, n_v;
     ChunkRange rg;        // the range of this launch
@@ -257,22 +257,40 @@ __global__ void __launch_bounds__(kGroupThr * kMaxGroups, 2) chunk_prep_kernel(c
             }
         }
     }
-    // T_beta = T diag(beta), then T_beta_gamma = T diag(beta gamma), each TF32 as a K-major
-    // image staged over the group's scratch and stored with one bulk copy; NaN if the CTA failed
+    // T_beta = T diag(beta) as fp16 and T_beta_gamma = T diag(beta gamma) as TF32, each a
+    // K-major image staged over the group's scratch and stored with one bulk copy; NaN if the
+    // CTA failed.  fp16 holds T_beta: |T_beta| <= 1 for beta in [0, 1] (and <= 4 for beta up
+    // to 2), and an entry beyond 65504 would become inf, so NaN downstream, never a wrong
+    // finite value.
     const float nan = __int_as_float(0x7fc00000);
+    const float bj = beta_s[jc];
 #pragma unroll 1
     for (int pass = 0; pass < 2; ++pass) {
         group_sync(gbar);   // the scratch is free (A^T read, or the previous store has read it)
-        const float fj = pass == 0 ? beta_s[jc] : beta_s[jc] * gam_s[jc];
+        if (pass == 0) {
 #pragma unroll
-        for (int s = 0; s < 32; ++s) {
-            const float xv = (s & 1) ? x[s >> 1].y : x[s >> 1].x;
-            *reinterpret_cast<float *>(scr + kmaj_off(2 * s + par, jc, 64)) = ok ? to_tf32(xv * fj) : nan;
+            for (int s = 0; s < 32; s += 2) {
+                // rows 2s + par and 2s + 2 + par of column jc: two separate fp16 (columns are
+                // what this thread owns, so no pairs can be packed)
+                const float2 xv = x[s >> 1];
+                *reinterpret_cast<__half *>(scr + kmaj16_off(2 * s + par, jc)) =
+                    __float2half_rn(ok ? xv.x * bj : nan);
+                *reinterpret_cast<__half *>(scr + kmaj16_off(2 * s + 2 + par, jc)) =
+                    __float2half_rn(ok ? xv.y * bj : nan);
+            }
+        } else {
+            const float fj = bj * gam_s[jc];
+#pragma unroll
+            for (int s = 0; s < 32; ++s) {
+                const float xv = (s & 1) ? x[s >> 1].y : x[s >> 1].x;
+                *reinterpret_cast<float *>(scr + kmaj_off(2 * s + par, jc, 64)) = ok ? to_tf32(xv * fj) : nan;
+            }
         }
         fence_smem_to_async();
         group_sync(gbar);
         if (gt == 0) {
-            bulk_store((pass == 0 ? p.tb : p.tg) + tile * 4096, smem_u32(scr), 16384);
+            if (pass == 0) bulk_store(p.tb + tile * 2048, smem_u32(scr), 8192);
+            else bulk_store(p.tg + tile * 4096, smem_u32(scr), 16384);
             bulk_commit();
             bulk_wait_read0();   // the staging may be overwritten once the copy has read it
         }

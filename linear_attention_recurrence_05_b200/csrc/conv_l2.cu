@@ -170,11 +170,11 @@ __global__ void __launch_bounds__(128) conv_l2_kernel(ConvParams p) {
 // ------------------------------------------------------------------------ conv + L2, tiles
 // The tensor-core path's tiles from bf16 input.  CTA = one 64-row chunk of one head slot:
 // q heads ([K;Q] tile, Q half), k heads ([K;Q] tile, K half, and the fp16 K tile, MN-major),
-// v heads (the V tile, MN-major).  One TMA copy brings the chunk's rows and the 3 rows before
+// v heads (the fp16 V tile, MN-major).  One TMA copy brings the chunk's rows and the 3 rows before
 // them (rows outside the tensor read as zero; at a sequence's start the 3 history rows are
 // replaced by the conv state or zeros); each warp then walks 16 rows from shared memory and
-// stores each row straight into the tiles, TF32-rounded (and fp16 for the K tile): the 32
-// lanes of a warp cover one row, whole 128-byte lines.
+// stores each row straight into the tiles, TF32-rounded for [K;Q], fp16 for the K and V tiles:
+// the 32 lanes of a warp cover one row, whole 128-byte lines.
 namespace {
 using namespace tc;
 
@@ -311,11 +311,13 @@ __global__ void __launch_bounds__(128) conv_tiles_kernel(const __grid_constant__
         o.z = t < len ? __uint_as_float((__float_as_uint(y[2]) + 0x1000u) & 0xFFFFE000u) : 0.f;
         o.w = t < len ? __uint_as_float((__float_as_uint(y[3]) + 0x1000u) & 0xFFFFE000u) : 0.f;
         if (!ok) o = make_float4(nan, nan, nan, nan);
-        // row t of this lane's 4 features (block lane / 8) in the tile's byte layout
-        const uint32_t mn_off = (lane >> 3) * 8192 + t * 128 + ((((lane & 7) >> 1) ^ (t & 3)) << 5) + (lane & 1) * 16;
-        if (mn) {
-            *reinterpret_cast<float4 *>(reinterpret_cast<unsigned char *>(p.vi + ((int64_t)ci * p.n_v + head) * 8192) +
-                                        mn_off) = o;
+        if (mn) {   // the V tile, fp16 (nearest even), MN-major
+            const float4 f = ok ? make_float4(t < len ? y[0] : 0.f, t < len ? y[1] : 0.f,
+                                              t < len ? y[2] : 0.f, t < len ? y[3] : 0.f)
+                                : o;
+            *reinterpret_cast<uint2 *>(reinterpret_cast<unsigned char *>(p.vi + ((int64_t)ci * p.n_v + head) * 4096) +
+                                       tc::mn16_off(t, 4 * lane, kChunk)) =
+                make_uint2(tc::pack_f16x2(f.x, f.y), tc::pack_f16x2(f.z, f.w));
         } else {
             unsigned char *kq = reinterpret_cast<unsigned char *>(p.kq + ((int64_t)ci * nq + head) * 16384 +
                                                                  (kind == 0 ? 2048 : 0));

@@ -42,8 +42,8 @@ static size_t carve_tiles(PrefillLayout &L, int n_qk, int n_v, int64_t slots, in
     size_t o = 0;
     L.b_kq = o;   o = align_up(o + ns * n_qk * 65536, 256);
     L.b_kmn = o;  o = align_up(o + ns * n_qk * 16384, 256);   // fp16
-    L.b_vi = o;   o = align_up(o + ns * n_v * 32768, 256);
-    L.b_tb = o;   o = align_up(o + ns * n_v * 16384, 256);
+    L.b_vi = o;   o = align_up(o + ns * n_v * 16384, 256);    // fp16
+    L.b_tb = o;   o = align_up(o + ns * n_v * 8192, 256);     // fp16
     L.b_tg = o;   o = align_up(o + ns * n_v * 16384, 256);
     L.b_pm = o;   o = align_up(o + ns * n_v * 8192, 256);    // fp16
     L.b_gr = o;   o = align_up(o + ns * n_v * kGateRec * sizeof(float), 256);
@@ -114,7 +114,7 @@ bool prefill_layout(int n_qk, int n_v, int64_t T, int n_seqs, int64_t max_seqlen
         // twice, else one (range r+1 is then prepared after the chains of range r)
         bool fit = false;
         for (int nb = 2; nb >= 1 && !fit; --nb) {
-            const size_t per = (size_t)n_seqs * ((size_t)n_qk * 81920 + (size_t)n_v * (73728 + kGateRec * 4)) * nb;
+            const size_t per = (size_t)n_seqs * ((size_t)n_qk * 81920 + (size_t)n_v * (49152 + kGateRec * 4)) * nb;
             const size_t avail = ws_limit > off ? ws_limit - off : 0;
             int64_t r = std::min<int64_t>(R, (int64_t)(avail / per) + 1);
             for (; r >= 1; --r) {

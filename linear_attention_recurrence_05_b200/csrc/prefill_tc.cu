@@ -24,12 +24,14 @@
 //     MMA_2b  U^T     -= X T_beta_gamma^T    (N=64,  K=64)    -> u^T
 //     MMA_3   S^T     += u~^T K              (N=128, K=64)    u~ = u diag(kd), onto gamma_C S^T
 //     MMA_4   Y       += u^T P^T             (N=64,  K=64)    onto Y = Y1 diag(gamma)
-//   MMA_1 and MMA_2a/2b take TF32 operands (fp32 in shared or tensor memory).  MMA_3 and
-//   MMA_4 take fp16 operands (kind::f16): u~ and u as fp16 pairs in tensor memory, written by
-//   the epilogue when it forms u~, and K and P as fp16 tiles.  fp16 carries the 11-bit
-//   significand of TF32; its range (|x| < 65504) holds u, u~ (u times decays <= 1), the unit
-//   keys and P (|P| <= 1) for activations of any sensible size, and a u beyond it turns the
-//   state into inf/NaN rather than into a wrong finite value.
+//   MMA_1 and MMA_2b take TF32 operands (S and X are fp32 accumulators in tensor memory;
+//   [K;Q] and T_beta_gamma fp32 tiles).  MMA_2a, MMA_3 and MMA_4 take fp16 operands
+//   (kind::f16): V, T_beta, K and P as fp16 tiles, u~ and u as fp16 pairs in tensor memory,
+//   written by the epilogue when it forms u~.  fp16 carries the 11-bit significand of TF32; its
+//   range (|x| < 65504) holds the unit keys, P (|P| <= 1), T_beta (|T_beta| <= 1 for beta in
+//   [0, 1], <= 4 for beta up to 2), V, u and u~ (u times decays <= 1) for activations of any
+//   sensible size, and a value beyond it turns the state into inf/NaN rather than into a
+//   wrong finite value.
 //   V is double-buffered (a chunk ahead) and T_beta reloaded as soon as MMA_2a has read it, so
 //   MMA_2a(c+1) is normally issued right after MMA_3(c) and runs while the new state is waited
 //   for; MMA_2b reads X straight from MMA_1's output.  The only epilogue step left on the
@@ -40,7 +42,7 @@
 //   producer (warp 5): the tile loads, each issued as soon as its buffer is free.
 //   drain group (warps 6-9): after MMA_4, reads Y and frees it at once, then writes y (or the
 //     gated output) through shared memory with TMA stores; a bf16 gate input z arrives by
-//     one TMA load per chunk, issued a chunk ahead.
+//     one TMA load per chunk, issued as soon as the previous chunk's rows have been read.
 // All waits are bounded; a CTA that times out writes NaN to its outputs.
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -69,23 +71,24 @@ constexpr int kBarDrain = 2;       // named barrier of the drain group (128 thre
 constexpr uint32_t OFF_KQ = 0;          // [K;Q]   K-major, 4 blocks x (K 8 KB | Q 8 KB)       64 KB
 constexpr uint32_t OFF_KMN = 65536;     // K       fp16, MN-major, 64 x 128                    16 KB
 constexpr uint32_t OFF_Z = 81920;       // gate input z of a chunk, bf16, 64 rows x 256 B     16 KB
-constexpr uint32_t OFF_V = 98304;       // V       MN-major, 2 buffers (chunk parity)      2 x 32 KB
-constexpr uint32_t OFF_TB = 163840;     // T_beta        K-major [t][i]                        16 KB
-constexpr uint32_t OFF_TG = 180224;     // T_beta_gamma  K-major [t][i]                        16 KB
-constexpr uint32_t OFF_P = 196608;      // P       fp16, K-major [t][i]                         8 KB
-constexpr uint32_t OFF_YST = 212992;    // y staging: 32 rows x 128 columns (TMA store box)    16 KB
-constexpr uint32_t OFF_GR = 229376;     // gates records, 2 buffers                          1280 B
+constexpr uint32_t OFF_V = 98304;       // V       fp16, MN-major, 2 buffers (chunk parity)  2 x 16 KB
+constexpr uint32_t OFF_TB = 131072;     // T_beta        fp16, K-major [t][i]                   8 KB
+constexpr uint32_t OFF_TG = 139264;     // T_beta_gamma  K-major [t][i]                        16 KB
+constexpr uint32_t OFF_P = 155648;      // P       fp16, K-major [t][i]                         8 KB
+constexpr uint32_t OFF_YST = 163840;    // y staging: 32 rows x 128 columns (TMA store box)    16 KB
+constexpr uint32_t OFF_GR = 180224;     // gates records, 2 buffers                          1280 B
 constexpr uint32_t OFF_BAR = OFF_GR + 2 * kGateRec * 4;   // mbarriers
-constexpr uint32_t OFF_FLAGS = OFF_BAR + 160;             // TMEM base, abort flag
+constexpr uint32_t OFF_FLAGS = OFF_BAR + 176;             // TMEM base, abort flag
 constexpr uint32_t kSmem = OFF_FLAGS + 16;
 constexpr uint32_t kSmemAlloc = kSmem + 1024;              // slack to align the base to 1024
 static_assert(kSmemAlloc <= 232448, "shared memory per CTA");
 
 enum {
-    B_KQ = 0, B_V0, B_V1, B_TB, B_TG,    // tile arrivals (B_V: V of buffer 0 / 1)
+    B_KQ = 0, B_V0, B_V1, B_TB, B_TG,    // tile arrivals (B_KQ: features 0-63 of [K;Q]; B_V: V of
+    B_KQ1,                               // buffer 0 / 1; B_KQ1: features 64-127 of [K;Q])
     B_KMN, B_PL,
     B_GR0, B_GR1,                        // gates record into buffer 0 / 1
-    B_1, B_2A, B_2, B_3, B_4,            // MMA completions (MMA_1; 2a; up to 2b; 3; 4)
+    B_1A, B_1, B_2A, B_2, B_3, B_4,      // MMA completions (MMA_1 first half; MMA_1; 2a; up to 2b; 3; 4)
     B_Y1,                                // epilogue: Y = Y1 diag(gamma) stored, S scaled
     B_UT,                                // epilogue: u~ = u diag(kd) stored
     B_YF,                                // drain group: Y read (tensor memory free for the next chunk)
@@ -93,7 +96,7 @@ enum {
     B_Z,                                 // gate input of a chunk arrived
     kNumBars
 };
-static_assert(kNumBars * 8 <= 160, "barrier area");
+static_assert(kNumBars * 8 <= 176, "barrier area");
 
 // tensor memory columns (all 128 lanes)
 constexpr uint32_t kTmemCols = 512;
@@ -132,6 +135,17 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t *m, uint32_t par, volatil
     }
     *abort_flag = 1;
     return false;
+}
+
+// SiLU(z) = z / (1 + e^-z) = z/2 (1 + tanh(z/2)) with the hardware tanh (tanh.approx.f32,
+// relative error <= 2^-10.987): one special-function (MUFU) operation per element, whose
+// issue rate in this kernel (~32 cycles per warp instruction on a sub-partition) is what the
+// gated output is bound by.  The error is absolute in effect: |SiLU - exact| <= |z| 2^-12
+// (largest where SiLU(z) -> 0 for z << 0, where 1 + tanh cancels).
+__device__ __forceinline__ float silu_tanh(float z) {
+    float t;
+    asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(0.5f * z));
+    return 0.5f * z * (1.f + t);
 }
 
 // Reduce-scatter of 32 rows over the 32 lanes of a warp: s[i] holds this lane's value of row i;
@@ -179,8 +193,8 @@ struct TcParams {
     CUtensorMap tm_out;   // y as [T, Hv*128] rows, boxes of 128 columns x 32 rows (no swizzle)
     CUtensorMap tm_z;     // bf16 z as [T, Hv*128] rows, boxes of 128 columns x 64 rows
     // per-chunk tiles of the range's buffer, by slot, in shared-memory layout: [K;Q] and K
-    // (fp16) per (slot, QK head); V, T_beta, T_beta_gamma, P (fp16) and the gates record per
-    // (slot, V head)
+    // (fp16) per (slot, QK head); V (fp16), T_beta (fp16), T_beta_gamma, P (fp16) and the gates
+    // record per (slot, V head)
     const float *kq, *kmn, *vi, *tb, *tg, *pm, *gr;
     const int32_t *cu, *cfirst;
     const float *init, *carry_in;   // state entering chunk 0 / entering a later first chunk
@@ -244,10 +258,13 @@ __global__ void __launch_bounds__(kThr, 1) prefill_tc_kernel(const __grid_consta
     auto slot = [&](int c) { return chunk_slot(p.rg, b, cb + c, p.cfirst); };
     auto qk_tile = [&](const float *base, int c, int64_t floats) { return base + (slot(c) * p.n_qk + gq) * floats; };
     auto v_tile = [&](const float *base, int c, int64_t floats) { return base + (slot(c) * p.n_v + h) * floats; };
-    auto issue_kq = [&](int c) { load(B_KQ, OFF_KQ, qk_tile(p.kq, c, 16384), 65536); };
+    // [K;Q] in two halves by feature (blocks 0-1, 2-3): MMA_1 starts on the first half while
+    // the second lands, and each half is reloaded as soon as MMA_1 has read it
+    auto issue_kq0 = [&](int c) { load(B_KQ, OFF_KQ, qk_tile(p.kq, c, 16384), 32768); };
+    auto issue_kq1 = [&](int c) { load(B_KQ1, OFF_KQ + 32768, qk_tile(p.kq, c, 16384) + 8192, 32768); };
     auto issue_kmn = [&](int c) { load(B_KMN, OFF_KMN, qk_tile(p.kmn, c, 4096), 16384); };
-    auto issue_v = [&](int c) { load(B_V0 + (c & 1), OFF_V + (c & 1) * 32768, v_tile(p.vi, c, 8192), 32768); };
-    auto issue_tb = [&](int c) { load(B_TB, OFF_TB, v_tile(p.tb, c, 4096), 16384); };
+    auto issue_v = [&](int c) { load(B_V0 + (c & 1), OFF_V + (c & 1) * 16384, v_tile(p.vi, c, 4096), 16384); };
+    auto issue_tb = [&](int c) { load(B_TB, OFF_TB, v_tile(p.tb, c, 2048), 8192); };
     auto issue_tg = [&](int c) { load(B_TG, OFF_TG, v_tile(p.tg, c, 4096), 16384); };
     auto issue_pm = [&](int c) { load(B_PL, OFF_P, v_tile(p.pm, c, 2048), 8192); };
     auto issue_gr = [&](int c) {  // gates record of chunk c into buffer c & 1
@@ -271,7 +288,8 @@ __global__ void __launch_bounds__(kThr, 1) prefill_tc_kernel(const __grid_consta
     if (tid == 0 && nchunks > 0) {
         issue_v(0);
         issue_tb(0);
-        issue_kq(0);
+        issue_kq0(0);
+        issue_kq1(0);
         if (nchunks > 1) issue_v(1);
         issue_tg(0);
         issue_kmn(0);
@@ -294,8 +312,8 @@ __global__ void __launch_bounds__(kThr, 1) prefill_tc_kernel(const __grid_consta
             auto issue_2a = [&](int c) {   // into u^T buffer c & 1 (D), V of buffer c & 1
                 const int bi = c & 1;
                 fence_after_sync();
-                gemm<128, 64, 64, true, false>(tm + T_U + 64 * bi, sb + OFF_V + bi * 32768, 64, sb + OFF_TB, 8192,
-                                               false);
+                gemm_f16<128, 64, 64, true, false>(tm + T_U + 64 * bi, sb + OFF_V + bi * 16384, 64, sb + OFF_TB, 0,
+                                                   false);
                 mma_commit(&bar[B_2A]);
             };
             // A wait costs ~100 cycles even when its phase is complete, so the waits for tiles
@@ -309,13 +327,25 @@ __global__ void __launch_bounds__(kThr, 1) prefill_tc_kernel(const __grid_consta
                     ok = wait_or_abort(&bar[B_KQ], 0, abort_flag);
                 }
             }
+            // MMA_1 over features 0-63 (A: S^T columns 0-63, B: [K;Q] blocks 0-1), then 64-127
+            auto mma1_lo = [&]() {
+                fence_after_sync();
+                gemm_ts<128, 64, false, false>(tm + T_XY, tm + T_S, sb + OFF_KQ, 16384, false);
+                mma_commit(&bar[B_1A]);
+            };
+            auto mma1_hi = [&]() {
+                gemm_ts<128, 64, false, false>(tm + T_XY, tm + T_S + 64, sb + OFF_KQ + 32768, 16384, true);
+                mma_commit(&bar[B_1]);
+            };
             for (int c = 0; c < nchunks && ok; ++c) {
                 const uint32_t par = c & 1;
                 const int bi = c & 1;
-                // MMA_1: needs S (MMA_3 of c-1, waited below) and [K;Q] of c (waited below)
+                // MMA_1: needs S (MMA_3 of c-1, waited below) and [K;Q] of c (the first half
+                // waited below, the second here)
+                mma1_lo();
+                if (!(ok = wait_or_abort(&bar[B_KQ1], par, abort_flag))) break;
                 fence_after_sync();
-                gemm_ts<128, 128, false, false>(tm + T_XY, tm + T_S, sb + OFF_KQ, 16384, false);
-                mma_commit(&bar[B_1]);
+                mma1_hi();
                 // MMA_2a of c unless issued at the end of c-1 (its tiles came late)
                 if (!a2_issued) {
                     if (!(ok = wait_or_abort(&bar[B_V0 + bi], vpar(c), abort_flag))) break;
@@ -363,7 +393,7 @@ __global__ void __launch_bounds__(kThr, 1) prefill_tc_kernel(const __grid_consta
         // ================================================================ tile producer
         if (lane == 0) {
             bool ok = true;
-            int n_kq = nchunks > 0 ? 1 : 0, n_tb = n_kq, n_tg = n_kq, n_kmn = n_kq, n_pm = n_kq;
+            int n_kq = nchunks > 0 ? 1 : 0, n_kq1 = n_kq, n_tb = n_kq, n_tg = n_kq, n_kmn = n_kq, n_pm = n_kq;
             int n_v[2] = {nchunks > 0 ? 1 : 0, nchunks > 1 ? 1 : 0};
             int n_gr[2] = {nchunks > 0 ? 1 : 0, nchunks > 1 ? 1 : 0};
             for (int c = 0; c < nchunks && ok; ++c) {
@@ -373,9 +403,11 @@ __global__ void __launch_bounds__(kThr, 1) prefill_tc_kernel(const __grid_consta
                 if (!(ok = wait_or_abort(&bar[B_2A], par, abort_flag))) break;
                 if (more) { issue_tb(c + 1); ++n_tb; }
                 if (c + 2 < nchunks) { issue_v(c + 2); ++n_v[c & 1]; }
-                // [K;Q] of c is consumed once MMA_1 of c is done
+                // each half of [K;Q] of c is consumed once its half of MMA_1 of c is done
+                if (!(ok = wait_or_abort(&bar[B_1A], par, abort_flag))) break;
+                if (more) { issue_kq0(c + 1); ++n_kq; }
                 if (!(ok = wait_or_abort(&bar[B_1], par, abort_flag))) break;
-                if (more) { issue_kq(c + 1); ++n_kq; }
+                if (more) { issue_kq1(c + 1); ++n_kq1; }
                 // T_beta_gamma once MMA_2b of c is done
                 if (!(ok = wait_or_abort(&bar[B_2], par, abort_flag))) break;
                 if (more) { issue_tg(c + 1); ++n_tg; }
@@ -388,9 +420,9 @@ __global__ void __launch_bounds__(kThr, 1) prefill_tc_kernel(const __grid_consta
                 if (more) { issue_pm(c + 1); ++n_pm; }
             }
             if (!ok) {  // wait (bounded) for the copies this thread started
-                const int counts[5] = {n_kq, n_tb, n_tg, n_kmn, n_pm};
-                const int bars[5] = {B_KQ, B_TB, B_TG, B_KMN, B_PL};
-                for (int i = 0; i < 5; ++i)
+                const int counts[6] = {n_kq, n_kq1, n_tb, n_tg, n_kmn, n_pm};
+                const int bars[6] = {B_KQ, B_KQ1, B_TB, B_TG, B_KMN, B_PL};
+                for (int i = 0; i < 6; ++i)
                     if (counts[i]) mbar_wait(&bar[bars[i]], (uint32_t)(counts[i] - 1) & 1, kWaitTries);
                 for (int i = 0; i < 2; ++i) {
                     if (n_v[i]) mbar_wait(&bar[B_V0 + i], (uint32_t)(n_v[i] - 1) & 1, kWaitTries);
@@ -569,6 +601,12 @@ __global__ void __launch_bounds__(kThr, 1) prefill_tc_kernel(const __grid_consta
                         rinv[lane] = rsqrtf((red[lane] + red[32 + lane] + red[64 + lane] + red[96 + lane]) *
                                                 (1.f / kHeadDim) + p.norm_eps);
                     bar_sync(kBarDrain, 128);
+                    float rw[32];   // 1 / rms of each row, times this column's weight
+#pragma unroll
+                    for (int i = 0; i < 32; i += 4) {
+                        const float4 r4 = *reinterpret_cast<const float4 *>(rinv + i);
+                        rw[i] = r4.x * wj; rw[i + 1] = r4.y * wj; rw[i + 2] = r4.z * wj; rw[i + 3] = r4.w * wj;
+                    }
 #pragma unroll
                     for (int i = 0; i < 32; ++i) {
                         float zi;
@@ -576,9 +614,9 @@ __global__ void __launch_bounds__(kThr, 1) prefill_tc_kernel(const __grid_consta
                             zi = to_f32(reinterpret_cast<const bf16 *>(sm + OFF_Z)[(row0 + i) * kHeadDim + j]);
                         else
                             zi = to_f32(zr[h2][i]);
-                        v[h2][i] *= rinv[i] * wj * (zi / (1.f + expf(-zi)));
+                        v[h2][i] *= rw[i] * silu_tanh(zi);
                     }
-                    bar_sync(kBarDrain, 128);   // the scratch (and z) is read before the staging is written
+                    bar_sync(kBarDrain, 128);   // the scratch (and z) read before the staging is written
                     if constexpr (kZTile)
                         if (h2 == 1 && dleader && c + 1 < nchunks) issue_z(c + 1);
                 }

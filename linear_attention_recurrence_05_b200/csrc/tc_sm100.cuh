@@ -1,9 +1,10 @@
 // Thin wrappers over the sm_100a tensor-core (tcgen05) and mbarrier PTX used by the
-// chunked prefill.  Operands are fp32 values in shared memory read as TF32
-// (kind::tf32, 8 K-elements per instruction), accumulators are fp32 in tensor memory.
+// chunked prefill.  Operands are fp32 values read as TF32 (kind::tf32, 8 K-elements per
+// instruction) or fp16 values (kind::f16, 16 K-elements per instruction); accumulators are
+// fp32 in tensor memory.
 //
-// Shared-memory operand layouts (fp32 elements), both made of 128-byte rows grouped
-// in blocks of 32 columns (a [R x C] tile is C/32 blocks of R*128 bytes):
+// Shared-memory operand layouts for fp32 elements, made of 128-byte rows grouped in blocks
+// of 32 columns (a [R x C] tile is C/32 blocks of R*128 bytes):
 //  * K-major operands (rows = M or N index, columns = K index): 128-byte swizzle with
 //    16-byte chunks, chunk c of row r at c ^ (r % 8) (what TMA's SWIZZLE_128B writes).
 //    K step s (8 columns) starts at block(s/4) + (s%4)*32 B; SBO = 1024 B (8 rows).
@@ -12,7 +13,8 @@
 //    the tensor core takes for 32-bit elements (TMA: SWIZZLE_128B_ATOM_32B).
 //    K step s (8 rows) starts at +1024*s; LBO = R*128 B (next 32 columns), SBO = 512 B.
 // A matrix contracted over both of its indices (K of a chunk: over features in K K^T
-// and K S, over tokens in K^T u) is therefore staged in both layouts.
+// and K S, over tokens in K^T u) is staged once per layout (here: [K;Q] K-major in fp32 for
+// the feature contractions, K MN-major in fp16 for the token contraction).
 //
 // fp16 operands (kind::f16, 16 K-elements per instruction): 128-byte rows of 64 elements,
 // 128-byte swizzle with 16-byte chunks (chunk c of row r at c ^ (r % 8)).
@@ -37,11 +39,6 @@ __device__ __forceinline__ uint32_t smem_u32(const void *p) {
 __host__ __device__ __forceinline__ uint32_t kmaj_off(int r, int c, int R) {
     return (uint32_t)((c >> 5) * R * 128 + r * 128 + ((((c & 31) >> 2) ^ (r & 7)) << 4) +
                       ((c & 3) << 2));
-}
-// byte offset of element (r, c) of a [R x C] fp32 tile, MN-major 32-byte-granule swizzle
-__host__ __device__ __forceinline__ uint32_t mn_off(int r, int c, int R) {
-    return (uint32_t)((c >> 5) * R * 128 + r * 128 + ((((c & 31) >> 3) ^ (r & 3)) << 5) +
-                      ((c & 7) << 2));
 }
 
 // byte offset of element (r, c) of a [R x 64] fp16 tile, K-major 128B swizzle
@@ -87,10 +84,10 @@ __host__ __device__ constexpr uint32_t idesc_tf32(int M, int N, bool a_mn, bool 
            | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
-// instruction descriptor: kind::f16 with fp16 A and B, fp32 accumulator, A K-major
-__host__ __device__ constexpr uint32_t idesc_f16(int M, int N, bool b_mn) {
+// instruction descriptor: kind::f16 with fp16 A and B, fp32 accumulator, operand majors
+__host__ __device__ constexpr uint32_t idesc_f16(int M, int N, bool a_mn, bool b_mn) {
     return (1u << 4)                       // D format: f32 (A, B format 0: f16)
-           | ((b_mn ? 1u : 0u) << 16)
+           | ((a_mn ? 1u : 0u) << 15) | ((b_mn ? 1u : 0u) << 16)
            | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
@@ -110,7 +107,8 @@ __device__ __forceinline__ void mma_tf32(uint32_t d_tmem, uint64_t a, uint64_t b
         "l"(a), "l"(b), "r"(idesc), "r"(accumulate));
 }
 
-// one kind::f16 MMA (K = 16 bf16 elements = 32 bytes of each operand row)
+// one kind::f16 MMA, both operands from shared memory (K = 16 16-bit elements = 32 bytes of
+// each operand row; fp16 or bf16 as the instruction descriptor says)
 __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
                                          uint32_t accumulate) {
     asm volatile(
@@ -146,7 +144,7 @@ __device__ __forceinline__ void gemm(uint32_t d_tmem, uint32_t a_base, uint32_t 
 template <int N, int K, bool B_MN>
 __device__ __forceinline__ void gemm_ts_f16(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_base, int b_rows,
                                             bool accumulate) {
-    constexpr uint32_t id = idesc_f16(128, N, B_MN);
+    constexpr uint32_t id = idesc_f16(128, N, false, B_MN);
     const uint64_t b0 = B_MN ? smem_desc(b_base, (uint32_t)b_rows * 128u, 1024, 2) : smem_desc(b_base, 16, 1024, 2);
 #pragma unroll
     for (int s = 0; s < K / 16; ++s) {
@@ -155,6 +153,22 @@ __device__ __forceinline__ void gemm_ts_f16(uint32_t d_tmem, uint32_t a_tmem, ui
             "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
             "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
             "r"(a_tmem + 8u * s), "l"(b0 + db), "r"(id), "r"((accumulate || s > 0) ? 1u : 0u));
+    }
+}
+
+// D[M x N] (+)= A[M x K] B[K x N] in fp16 (kind::f16), both operands in shared memory: each
+// K-major [rows x 64] (rows argument unused) or MN-major [K x M|N] with rows = K.
+template <int M, int N, int K, bool A_MN, bool B_MN>
+__device__ __forceinline__ void gemm_f16(uint32_t d_tmem, uint32_t a_base, int a_rows, uint32_t b_base, int b_rows,
+                                         bool accumulate) {
+    constexpr uint32_t id = idesc_f16(M, N, A_MN, B_MN);
+    const uint64_t a0 = A_MN ? smem_desc(a_base, (uint32_t)a_rows * 128u, 1024, 2) : smem_desc(a_base, 16, 1024, 2);
+    const uint64_t b0 = B_MN ? smem_desc(b_base, (uint32_t)b_rows * 128u, 1024, 2) : smem_desc(b_base, 16, 1024, 2);
+#pragma unroll
+    for (int s = 0; s < K / 16; ++s) {
+        const uint32_t da = A_MN ? (uint32_t)(s * 128) : (uint32_t)(s * 2);   // 16-byte units
+        const uint32_t db = B_MN ? (uint32_t)(s * 128) : (uint32_t)(s * 2);
+        mma_bf16(d_tmem, a0 + da, b0 + db, id, (accumulate || s > 0) ? 1u : 0u);
     }
 }
 

@@ -55,7 +55,7 @@ int main(void) {
      * with one chunk per sequence per range (more sequences than one chunk slot each fits) is
      * rejected on the host, before any device call */
     {
-        const size_t slot = (size_t)16 * (65536 + 16384) + (size_t)48 * (32768 + 2 * 16384 + 8192 + 640);
+        const size_t slot = (size_t)16 * (65536 + 16384) + (size_t)48 * (16384 + 8192 + 16384 + 8192 + 640);
         const int n = (int)(GDN_STATIC_SCRATCH_BYTES / slot) + 1;
         CHECK(gdn_prefill_static_scratch(&cfg, GDN_BF16, GDN_F32, A(1), A(2), A(3), A(4), A(5), A(6), A(7), A(8),
                                          A(9), n, 64 * n, NULL, NULL, NULL, NULL, A(10), 0) == GDN_ERR_WORKSPACE);

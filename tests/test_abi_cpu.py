@@ -51,9 +51,9 @@ def _ws(cfg, dtype=0, T=8192, n=1, max_seqlen=0):
 
 
 # tiles of one (sequence, chunk) slot at 16 QK / 48 V heads: [K;Q] 64 KB and K (fp16) 16 KB per
-# QK head; V 32 KB, T_beta and T_beta_gamma 16 KB each, P (fp16) 8 KB and a 640-byte gates
-# record per V head
-SLOT = 16 * (65536 + 16384) + 48 * (32768 + 2 * 16384 + 8192 + 640)
+# QK head; V (fp16) 16 KB, T_beta (fp16) 8 KB, T_beta_gamma 16 KB, P (fp16) 8 KB and a 640-byte
+# gates record per V head
+SLOT = 16 * (65536 + 16384) + 48 * (16384 + 8192 + 16384 + 8192 + 640)
 STATE = 128 * 128 * 4
 
 

@@ -95,18 +95,27 @@ def test_prefill_gated_matches_oracle(lib, dtype, zdt, odt, lengths):
     yo, fo, _ = oracle.prefill(inp)
     ref = output_gate(yo, gi.stored_to_f64(z, zdt), w, 1e-6)
     # y is within tol * rms(y) of the oracle per element; the row normalisation divides that
-    # by the row's own rms, and the gate scales it by |w SiLU(z)| (x 3 for the norm's own change)
+    # by the row's own rms, and the gate scales it by |w SiLU(z)| (x 3 for the norm's own change).
+    # The fused path takes SiLU from the hardware tanh, SiLU(z) = z/2 (1 + tanh(z/2)), whose
+    # relative error bound 2^-10.987 leaves |z| 2^-12 on SiLU: 2^-11 |z| |w| |y / rms(y row)|
+    # more (2x margin), the only term left where SiLU(z) -> 0.
     t = tol(dtype)
+    zf = gi.stored_to_f64(z, zdt)
     row_rms = np.sqrt(np.mean(yo ** 2, axis=-1, keepdims=True))
-    gate = np.abs(w * gi.stored_to_f64(z, zdt) / (1.0 + np.exp(-gi.stored_to_f64(z, zdt))))
-    bound = 3 * t * np.sqrt(np.mean(yo ** 2)) / row_rms * gate + 1e-6 * np.sqrt(np.mean(ref ** 2))
+    gate = np.abs(w * zf / (1.0 + np.exp(-zf)))
+    silu_term = 2.0 ** -11 * np.abs(zf) * np.abs(w) * np.abs(yo) / row_rms
+    bound = (3 * t * np.sqrt(np.mean(yo ** 2)) / row_rms * gate + 1e-6 * np.sqrt(np.mean(ref ** 2))
+             + silu_term * (1 + 3 * t))
     if odt == gi.BF16:
         bound = bound + 2.0 ** -8 * np.abs(ref)
     assert np.all(np.abs(got - ref) <= bound)
     assert rel_err(to_host_f64(fin), fo) <= t
-    # the fused tail against the unfused composition on the same y (fp32 arithmetic only)
+    # the fused tail against the unfused composition on the same y: fp32 arithmetic apart from
+    # the fused path's tanh-based SiLU (bound above, from the GPU's own y)
     o2h = to_host_f64(o2)
+    yh = to_host_f64(y)
+    yn = yh / np.sqrt(np.mean(yh ** 2, axis=-1, keepdims=True) + 1e-6)
+    b2 = 2.0 ** -11 * np.abs(zf) * np.abs(w) * np.abs(yn) + 1e-5 * np.sqrt(np.mean(o2h ** 2))
     if odt == gi.BF16:
-        assert np.all(np.abs(got - o2h) <= 2.0 ** -8 * np.abs(o2h) + 1e-5 * np.sqrt(np.mean(o2h ** 2)))
-    else:
-        assert np.max(np.abs(got - o2h)) / np.sqrt(np.mean(o2h ** 2)) <= 1e-5
+        b2 = b2 + 2.0 ** -8 * np.abs(o2h)
+    assert np.all(np.abs(got - o2h) <= b2)

@@ -72,6 +72,20 @@ def test_pages_heads_short(lib, dtype):
     _check(inp, lib, label=f"h16x48-{dtype}")
 
 
+def test_beta_above_one(lib):
+    """beta in (1, 1.9): each token's map alpha (I - beta k k^T) still contracts, and chunk
+    prep's T_beta = (I + A)^-1 diag(beta), stored as fp16, reaches entries near beta (|T_beta|
+    <= 1 for beta in [0, 1]); several chunks and a partial one (gated delta rule, page
+    "ARCHITECTURE PREVIEW / FIELD NOTES", section 03; the equations admit any beta).  Keys are
+    the usual random ones: with identical keys and beta > 1 the chunked form loses ~6e-2 with
+    TF32 operands throughout (the alternating terms of T_beta V cancel), fp16 or not."""
+    shape = gi.GdnShape(n_qk_heads=1, n_v_heads=3)
+    T = 150
+    inp = gi.make_prefill_inputs(shape, [T], gi.BF16, seed=91)
+    inp.beta = gi.quantize(np.random.default_rng(6).uniform(1.0, 1.9, (T, 3)).astype(np.float32), gi.BF16)
+    _check(inp, lib, label="beta-above-one")
+
+
 @pytest.mark.parametrize("heads", [(2, 2), (2, 4), (1, 4), (2, 10)])
 def test_head_ratios(lib, heads):
     """V heads per QK head other than 3: the chunk-prep pass then serves 1 or 2 V heads per CTA
