@@ -305,7 +305,8 @@ def bench_prefill(args, dist, torch, gdn, peaks, idx=1, e2e=True):
     tokens_all = T * dist.world * K
     res = {"value": tokens_all / (ms_max / 1e3), "ms_per_step": ms_max / K, "clocks": clk,
            "per_kernel": per_kernel, "launches": launches / K, "tokens_per_step": T, "steps": K,
-           "n_v_heads": Hv, "n_seqs": n, "workload": p["name"], "workspace_bytes": ws.numel()}
+           "n_v_heads": Hv, "n_qk_heads": cfg.n_qk_heads, "n_seqs": n, "workload": p["name"],
+           "workspace_bytes": ws.numel()}
     if not e2e:
         return res
 
@@ -455,11 +456,24 @@ def prefill_roofline(res, peaks, peak_src, sha):
                 "peak_source": (f"{peak_src} bf16 {bf16} for the fp16 third of the MMA flops, "
                                 f"x 1.1/2.25 nominal (tf32) for the other two thirds"),
                 "algorithmic_per_launch": flops, "tokens_per_launch": T, "kernel_share": share}
-    # a memory-bound kernel dominates
-    byts = (2 * 16 * D * 2 + 48 * D * 2 + 3 * 16 * 4 * D) * T
+    # a tile-making pass dominates (chunk prep or the conv pass): its algorithmic bytes per
+    # token at the run's head counts, the tiles being what the chain needs and nothing more
+    Hq = res["n_qk_heads"]
+    if dom == "chunk_prep":
+        # reads the [K;Q] tile of every (chunk, QK head); writes T_beta (fp16), T_beta_gamma
+        # (fp32), P (fp16) and the gates record of every (chunk, V head)
+        per_tok = (Hq * 65536 + Hv * (8192 + 16384 + 8192 + 640)) / CHUNK
+    elif dom == "conv_l2":
+        # reads q, k, v (bf16); writes the [K;Q] tile (fp32), the K tile and the V tile (fp16)
+        per_tok = (2 * Hq * D * 2 + Hv * D * 2) + (2 * Hq * D * 4 + Hq * D * 2 + Hv * D * 2)
+    else:
+        per_tok = 2 * Hq * D * 2 + Hv * D * 2 + Hv * D * 4
+    byts = per_tok * T
+    traffic, tsrc = traffic_for(dom, res["workload"], T, sha)
     return {"kernel": dom, "bound": "hbm", "achieved": byts / avg_s / 1e9, "peak": peaks["hbm_gbs"],
-            "unit": "GB/s", "frac": byts / avg_s / 1e9 / peaks["hbm_gbs"], "traffic": None,
-            "peak_source": peak_src, "kernel_share": share}
+            "unit": "GB/s", "frac": byts / avg_s / 1e9 / peaks["hbm_gbs"], "traffic": traffic,
+            "traffic_source": tsrc, "peak_source": peak_src, "algorithmic_per_launch": byts,
+            "tokens_per_launch": T, "kernel_share": share}
 
 
 def prefill_step_summary(res, peaks):
