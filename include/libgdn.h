@@ -72,8 +72,10 @@ typedef enum {
     GDN_F32 = 1    /* float32 storage */
 } gdn_dtype;
 /* Every call takes two storage types: `dtype` for q, k, v, alpha, beta and the conv
- * state (the raw inputs), and `out_dtype` for y.  Whatever they are, all arithmetic is
- * fp32 (tensor-core products in TF32 with fp32 accumulation) and states are fp32.
+ * state (the raw inputs), and `out_dtype` for y.  Whatever they are, accumulation and states
+ * are fp32; the tensor-core products of the bf16 path take operands with an 11-bit
+ * significand (TF32 where an operand is an fp32 accumulator, fp16 for the chunk tiles and
+ * the per-chunk vectors u), and the fp32 path computes in fp32 on the CUDA cores.
  * Note on precision: rounding y to bfloat16 alone moves its largest entries by up to
  * 2^-9 of their magnitude, which on typical data is 2-3% of rms(y); use
  * out_dtype = GDN_F32 where y must stay within 1e-2 of rms(y) of the exact result. */
@@ -185,6 +187,9 @@ GDN_EXPORT gdn_status gdn_prefill(const gdn_config *cfg, gdn_dtype dtype, gdn_dt
  *   out       [T, Hv, 128] out_dtype: the gated output
  * With fp32 input (the fp32 CUDA-core path) y is first written to `out` and the tail then
  * runs in place, so out_dtype must be GDN_F32 there (GDN_ERR_UNSUPPORTED otherwise).
+ * Precision (bf16 input): SiLU is taken from the hardware tanh, z/2 (1 + tanh(z/2)), whose
+ * error is at most |z| 2^-12 in absolute terms (gdn_output_gate uses the exponential); the
+ * rest of the tail is fp32.
  */
 GDN_EXPORT gdn_status gdn_prefill_gated(const gdn_config *cfg, gdn_dtype dtype, gdn_dtype out_dtype,
                              const void *q, const void *k, const void *v,
