@@ -148,29 +148,33 @@ __global__ void __launch_bounds__(kGroupThr * kMaxGroups, 2) chunk_prep_kernel(c
             mma_commit(&bar[1]);
         }
     }
-    if ((gt >> 5) == 1) {  // warp 1 of each group: inclusive scan of log alpha, two rows per lane
+    // warp 1 of each group: inclusive scan of log alpha, two rows per lane, summed in fp64 (with
+    // strong decay g reaches -100 and beyond inside a chunk, and fp32 partial sums would leave
+    // ~1e-4 relative error in the ratios exp(g_t - g_i); each g_t rounded once to fp32 leaves
+    // ~1e-5 at g = -100)
+    if ((gt >> 5) == 1) {
         const int t0 = 2 * lane, t1 = t0 + 1;
-        const float a0 = g_s[t0], a1 = g_s[t1];
-        float s = a0 + a1;
+        const double a0 = g_s[t0], a1 = g_s[t1];
+        double s = a0 + a1;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
-            const float y = __shfl_up_sync(0xffffffffu, s, o);
+            const double y = __shfl_up_sync(0xffffffffu, s, o);
             if (lane >= o) s += y;
         }
-        const float g0 = s - a1, g1 = s;
-        const float glast = __shfl_sync(0xffffffffu, ((n - 1) & 1) ? g1 : g0, (n - 1) >> 1);
-        g_s[t0] = g0;
-        g_s[t1] = g1;
-        const float gam0 = expf(g0), gam1 = expf(g1);
+        const double g0 = s - a1, g1 = s;
+        const double glast = __shfl_sync(0xffffffffu, ((n - 1) & 1) ? g1 : g0, (n - 1) >> 1);
+        g_s[t0] = (float)g0;
+        g_s[t1] = (float)g1;
+        const float gam0 = expf((float)g0), gam1 = expf((float)g1);
         gam_s[t0] = gam0;
         gam_s[t1] = gam1;
-        ig_s[t0] = expf(-g0);      // used only when the chunk's decay stays below kMaxChunkDecay
-        ig_s[t1] = expf(-g1);
+        ig_s[t0] = expf((float)-g0);      // used only when the chunk's decay stays below kMaxChunkDecay
+        ig_s[t1] = expf((float)-g1);
         gr[kGrGamma + t0] = gam0;
         gr[kGrGamma + t1] = gam1;
-        gr[kGrKd + t0] = t0 < n ? expf(glast - g0) : 0.f;
-        gr[kGrKd + t1] = t1 < n ? expf(glast - g1) : 0.f;
-        if (lane == 0) gr[kGrGammaC] = expf(glast);
+        gr[kGrKd + t0] = t0 < n ? expf((float)(glast - g0)) : 0.f;
+        gr[kGrKd + t1] = t1 < n ? expf((float)(glast - g1)) : 0.f;
+        if (lane == 0) gr[kGrGammaC] = expf((float)glast);
     }
     if (tid == 0) {
         if (ok) ok = mbar_wait(&bar[1], 0, kPWaitTries);

@@ -35,7 +35,9 @@ struct SimtSmem {
     float X[kChunk][kXW];
     float S[kHeadDim][kSlice];
     float u[kChunk][kSlice];
-    float g[kChunk];
+    // g_t = sum_{s<=t} log alpha_s in fp64: with strong decay g reaches -100 and beyond inside
+    // a chunk, and fp32 sums would leave ~1e-4 relative error in the ratios exp(g_t - g_i)
+    double g[kChunk];
     float gam[kChunk];
     float beta[kChunk];
     float kd[kChunk];
@@ -96,22 +98,22 @@ __global__ void __launch_bounds__(kThreads, 1) scan_simt_kernel(ScanParams p) {
             sm.beta[tid] = bb;
         }
         __syncthreads();
-        if (tid < 32) {  // inclusive scan of log alpha over 64 rows (two per lane)
-            float a0 = sm.g[2 * tid], a1 = sm.g[2 * tid + 1];
-            float s = a0 + a1;
+        if (tid < 32) {  // inclusive scan of log alpha over 64 rows (two per lane), in fp64
+            const double a0 = sm.g[2 * tid], a1 = sm.g[2 * tid + 1];
+            double s = a0 + a1;
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
-                float y = __shfl_up_sync(0xffffffffu, s, o);
+                const double y = __shfl_up_sync(0xffffffffu, s, o);
                 if (tid >= o) s += y;
             }
-            const float base = s - (a0 + a1);
+            const double base = s - (a0 + a1);
             sm.g[2 * tid] = base + a0;
             sm.g[2 * tid + 1] = s;
         }
         __syncthreads();
         if (tid < kChunk) {
-            sm.gam[tid] = expf(sm.g[tid]);
-            sm.kd[tid] = tid < n ? expf(sm.g[n - 1] - sm.g[tid]) : 0.f;
+            sm.gam[tid] = expf((float)sm.g[tid]);
+            sm.kd[tid] = tid < n ? expf((float)(sm.g[n - 1] - sm.g[tid])) : 0.f;
         }
         // ---- A = strict-lower beta exp(g_t - g_i) K K^T ;  P = lower exp(g_t - g_i) Q K^T
         for (int e = tid; e < kChunk * kChunk; e += kThreads) {
@@ -125,7 +127,7 @@ __global__ void __launch_bounds__(kThreads, 1) scan_simt_kernel(ScanParams p) {
                     dk = fmaf(sm.K[t][r], ki, dk);
                     dq = fmaf(sm.Q[t][r], ki, dq);
                 }
-                const float dec = expf(sm.g[t] - sm.g[i]);
+                const float dec = expf((float)(sm.g[t] - sm.g[i]));
                 pq = dec * dq;
                 if (i < t) a = sm.beta[t] * dec * dk;
             }

@@ -86,6 +86,30 @@ def test_beta_above_one(lib):
     _check(inp, lib, label="beta-above-one")
 
 
+@pytest.mark.parametrize("dtype", [gi.BF16, gi.F32])
+def test_strong_decay_resets_and_degenerate_beta(lib, dtype):
+    """Gates at their edges: strong decay (alpha ~ e^-1.6 per token, so a chunk's total decay
+    passes e^-80 and chunk prep forms exp(g_t - g_i) directly instead of as gamma_t / gamma_i),
+    exact resets (alpha = 0, which the kernels take as e^-80), runs of alpha = 1, and beta = 0
+    (no write) and beta = 1 rows; ragged lengths over several chunks, initial and conv states
+    (gated delta rule, page "ARCHITECTURE PREVIEW / FIELD NOTES", section 03)."""
+    shape = gi.GdnShape(n_qk_heads=2, n_v_heads=6)
+    lengths = [300, 129, 64]
+    inp = gi.make_prefill_inputs(shape, lengths, dtype, seed=97, with_initial_state=True, with_conv_state=True)
+    T = inp.total_tokens
+    rng = np.random.default_rng(98)
+    x = rng.standard_normal((T, 6))
+    alpha = np.exp(-2.0 * np.logaddexp(0.0, x))          # strong decay
+    alpha[rng.random((T, 6)) < 0.03] = 0.0                  # resets
+    alpha[100:140] = 1.0                                    # no decay at all
+    beta = 1.0 / (1.0 + np.exp(-rng.standard_normal((T, 6))))
+    beta[rng.random((T, 6)) < 0.1] = 0.0
+    beta[rng.random((T, 6)) < 0.1] = 1.0
+    inp.alpha = gi.quantize(alpha.astype(np.float32), dtype)
+    inp.beta = gi.quantize(beta.astype(np.float32), dtype)
+    _check(inp, lib, label=f"edge-gates-{dtype}")
+
+
 @pytest.mark.parametrize("heads", [(2, 2), (2, 4), (1, 4), (2, 10)])
 def test_head_ratios(lib, heads):
     """V heads per QK head other than 3: the chunk-prep pass then serves 1 or 2 V heads per CTA
