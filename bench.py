@@ -477,14 +477,20 @@ def prefill_roofline(res, peaks, peak_src, sha):
 
 
 def prefill_step_summary(res, peaks):
-    """Whole-step rates of a prefill leg against both tensor peaks and the copy bandwidth."""
+    """Whole-step rates of a prefill leg against both tensor peaks and the copy bandwidth.
+    The step's minimum bytes per token are the method's own inputs and output: raw q, k, v and
+    alpha, beta in bf16 and y in bf16 (32,960 B at 16/48 heads; this path writes y in fp32)."""
     s = res["ms_per_step"] / 1e3
     T = res["tokens_per_step"]
-    flops = PREFILL_FLOP_TV * T * res["n_v_heads"]
+    Hq, Hv = res["n_qk_heads"], res["n_v_heads"]
+    flops = PREFILL_FLOP_TV * T * Hv
+    byts = (2 * Hq * D * 2 + Hv * D * 2 + Hv * D * 2 + 2 * Hv * 2) * T
     tf32 = peaks["bf16_tflops"] * TF32_PER_BF16
     return {"tflops": flops / s / 1e12, "frac_of_tf32_peak": flops / s / 1e12 / tf32,
             "frac_of_bf16_peak": flops / s / 1e12 / peaks["bf16_tflops"],
-            "algorithmic_flops_per_step": flops}
+            "algorithmic_flops_per_step": flops,
+            "gbs": byts / s / 1e9, "frac_of_hbm": byts / s / 1e9 / peaks["hbm_gbs"],
+            "algorithmic_bytes_per_step": byts}
 
 
 def bench_prefill_gated(args, dist, torch, gdn, peaks):
