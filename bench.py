@@ -32,6 +32,7 @@ from __future__ import annotations
 import argparse
 import json
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -375,9 +376,22 @@ def bench_prefill(args, dist, torch, gdn, peaks, idx=1, e2e=True):
 
 
 # ----------------------------------------------------------------------------- traffic records
+_COMMENT_OR_LITERAL = re.compile(r'//[^\n]*|/\*.*?\*/|("(?:\\.|[^"\\\n])*"|\'(?:\\.|[^\'\\\n])*\')', re.S)
+
+
+def code_only(text):
+    """C/C++/CUDA source with its comments removed (string and character literals kept as
+    written) and its blank lines and trailing blanks dropped: the code the compiler turns
+    into kernels, less comments and layout."""
+    text = _COMMENT_OR_LITERAL.sub(lambda m: m.group(1) or " ", text)
+    return "\n".join(ln for ln in (ln.rstrip() for ln in text.split("\n")) if ln)
+
+
 def kernel_sources_sha256():
-    """sha256 over the library's kernel and ABI sources (file names and bytes, sorted): the
-    identity of the binary whose DRAM traffic a record describes."""
+    """sha256 over the library's kernel and ABI sources (file names and code with comments
+    and blank lines removed, files sorted): the identity of the kernels whose DRAM traffic a
+    record describes.  An edit to a comment leaves it unchanged; any change to the code
+    changes it."""
     import hashlib
     h = hashlib.sha256()
     roots = [os.path.join(ROOT, "linear_attention_recurrence_05_b200", "csrc"), os.path.join(ROOT, "include")]
@@ -385,8 +399,8 @@ def kernel_sources_sha256():
         for name in sorted(os.listdir(r)):
             if name.endswith((".cu", ".cuh", ".h")):
                 h.update(name.encode())
-                with open(os.path.join(r, name), "rb") as f:
-                    h.update(f.read())
+                with open(os.path.join(r, name), encoding="utf-8") as f:
+                    h.update(code_only(f.read()).encode())
     return h.hexdigest()
 
 

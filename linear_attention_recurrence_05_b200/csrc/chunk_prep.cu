@@ -36,8 +36,8 @@ constexpr int kMaxGroups = 3;    // V heads per CTA
 // shared-memory map (bytes from a 1024-aligned base).  [0, 64 KB) holds the [K;Q] tile until
 // the MMA has read it, then one scratch per group: -A^T split by row parity, array p holding
 // -A[2s + p][m] at row m, column s (64 x 32 floats), the odd array 64 bytes past a multiple
-// of 8 KB so that the two parities fall in different banks; after the inverse, the T_beta
-// staging (K-major image, 16 KB).
+// of 8 KB so that the two parities fall in different banks; after the inverse, the staging
+// of T_beta (K-major fp16 image, 8 KB), then of T_beta_gamma (K-major TF32 image, 16 KB).
 constexpr uint32_t P_KQ = 0;
 constexpr uint32_t kParStride = 8192 + 64;
 constexpr uint32_t kScrBytes = 2 * kParStride;

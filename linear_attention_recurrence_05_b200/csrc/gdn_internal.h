@@ -44,12 +44,12 @@ struct PrefillLayout {
     // rows past a sequence's end are 0.  Offsets inside a buffer:
     size_t off_tiles;     // first buffer
     size_t buf_bytes;     // distance between buffers
-    size_t b_kq;          // [slots, Hqk] x 64 KB: [K;Q], K-major 128B-swizzled blocks
-    size_t b_kmn;         // [slots, Hqk] x 32 KB: K, MN-major 32B-granule swizzle
-    size_t b_vi;          // [slots, Hv]  x 32 KB: V, MN-major 32B-granule swizzle
-    size_t b_tb;          // [slots, Hv]  x 16 KB: T diag(beta), K-major 128B-swizzled
-    size_t b_tg;          // [slots, Hv]  x 16 KB: T diag(beta gamma), same
-    size_t b_pm;          // [slots, Hv]  x 16 KB: P, same
+    size_t b_kq;          // [slots, Hqk] x 64 KB: [K;Q] TF32, K-major 128B-swizzled blocks
+    size_t b_kmn;         // [slots, Hqk] x 16 KB: K fp16, MN-major 32B-granule swizzle
+    size_t b_vi;          // [slots, Hv]  x 16 KB: V fp16, MN-major 32B-granule swizzle
+    size_t b_tb;          // [slots, Hv]  x 8 KB: T diag(beta) fp16, K-major 128B-swizzled
+    size_t b_tg;          // [slots, Hv]  x 16 KB: T diag(beta gamma) TF32, K-major 128B-swizzled
+    size_t b_pm;          // [slots, Hv]  x 8 KB: P fp16, K-major 128B-swizzled
     size_t b_gr;          // [slots, Hv]  x 640 B: gates record (gamma[64], kd[64], gamma_C)
     size_t b_cseq;        // int32 [slots]: sequence of each chunk (compact numbering)
     size_t off_carry;     // [n_seqs, Hv, 128, 128] fp32 state between ranges (used when the
@@ -150,7 +150,7 @@ cudaError_t launch_qsa_topk(const float *scores, int64_t ld, const int32_t *qpos
 // launchers: return the cudaError_t of the launch
 cudaError_t launch_seq_table(const int32_t *cu_in, int n_seqs, int64_t T, int32_t *cu,
                              int32_t *cfirst, cudaStream_t s);
-// tiles: write the tensor-core chunk tiles (TF32-rounded) instead of fp32 rows
+// tiles: write the tensor-core chunk tiles ([K;Q] TF32-rounded, K and V fp16) instead of fp32 rows
 cudaError_t launch_conv_l2(const ConvParams &p, bool bf16, bool tiles, int64_t n_chunks,
                            int64_t total_tokens, cudaStream_t s);
 cudaError_t launch_conv_state_out(const void *q, const void *k, const void *v,
