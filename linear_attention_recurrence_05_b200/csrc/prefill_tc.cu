@@ -33,9 +33,9 @@
 //   sensible size, and a value beyond it turns the state into inf/NaN rather than into a
 //   wrong finite value.
 //   V is double-buffered (a chunk ahead) and T_beta reloaded as soon as MMA_2a has read it, so
-//   MMA_2a(c+1) is normally issued right after MMA_3(c) and runs while the new state is waited
-//   for; MMA_2b reads X straight from MMA_1's output.  The only epilogue step left on the
-//   critical path is u~.  u^T is double-buffered in tensor memory (chunk parity).
+//   MMA_2a(c+1) is normally issued right after MMA_3(c) and MMA_4(c), and runs while the new
+//   state is waited for; MMA_2b reads X straight from MMA_1's output.  The only epilogue step
+//   left on the critical path is u~.  u^T is double-buffered in tensor memory (chunk parity).
 //   epilogue (warps 1-4), in tensor memory: after MMA_1, Y = Y1 diag(gamma) (once the drain
 //     group has read the previous Y) and S^T *= gamma_C; after MMA_2b, u~ (over X, which
 //     MMA_2b has consumed); the state entering and leaving the range.
