@@ -236,7 +236,8 @@ __global__ void __launch_bounds__(kThr, 1) prefill_tc_kernel(const __grid_consta
     const bool overflow = !p.rg.compact && p.rg.last && seq_chunks > cb + nchunks;
 
     if (tid == 0) {
-        asm volatile("prefetch.tensormap [%0];" ::"l"(&p.tm_out) : "memory");
+        // the y map is encoded only when the call has tokens (a CTA with chunks implies that)
+        if (nchunks > 0) asm volatile("prefetch.tensormap [%0];" ::"l"(&p.tm_out) : "memory");
         for (int i = 0; i < kNumBars; ++i) mbar_init(&bar[i], 1);
         *abort_flag = 0;
     }

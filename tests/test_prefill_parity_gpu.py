@@ -56,6 +56,22 @@ def test_ragged_varlen_with_states(lib, dtype):
 
 
 @pytest.mark.parametrize("dtype", [gi.BF16, gi.F32])
+@pytest.mark.parametrize("with_init", [True, False])
+def test_no_tokens_at_all(lib, dtype, with_init):
+    """Every sequence empty (total_tokens = 0): y has no rows, each final state is its
+    initial state (zero without one) and the conv states pass through, all bit for bit."""
+    shape = gi.GdnShape(n_qk_heads=2, n_v_heads=6)
+    inp = gi.make_prefill_inputs(shape, [0, 0, 0], dtype, seed=5, with_initial_state=with_init,
+                                 with_conv_state=True)
+    y, fin, cso = prefill_dev(inp, lib, with_conv_out=True)
+    torch.cuda.synchronize()
+    yo, fo, co = oracle.prefill(inp)
+    assert tuple(y.shape) == (0, 6, 128) and yo.shape == (0, 6, 128)
+    assert np.array_equal(to_host_f64(fin), fo)
+    assert np.array_equal(to_host_f64(cso), co)
+
+
+@pytest.mark.parametrize("dtype", [gi.BF16, gi.F32])
 def test_conv_silu(lib, dtype):
     """The optional SiLU on the ShortConv outputs (gdn_config.conv_activation = SiLU) against
     the oracle with the same option: ragged lengths, initial and conv states."""
