@@ -19,8 +19,9 @@ import torch
 from . import _native
 from ._native import GDN_BF16, GDN_F32, GdnError  # noqa: F401
 
-__all__ = ["GdnConfig", "affine_combine", "gdn_prefill", "gdn_decode_step", "gdn_decode_multi", "gdn_output_gate", "prefill_workspace_size", "GdnError",
-           "library_path", "qsa_block_keys", "qsa_block_scores", "qsa_select", "qsa_select_workspace_size",
+__all__ = ["GdnConfig", "affine_combine", "gdn_prefill", "gdn_decode_step", "gdn_decode_multi",
+           "gdn_output_gate", "prefill_workspace_size", "GdnError", "LaunchTrace", "library_path",
+           "qsa_block_keys", "qsa_block_scores", "qsa_select", "qsa_select_workspace_size",
            "QSA_BUDGET", "QSA_TOKEN_SLOTS"]
 
 

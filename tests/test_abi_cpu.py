@@ -29,6 +29,11 @@ def test_library_exports_every_declared_symbol():
     assert lib.gdn_api_version() == 2
 
 
+def test_binding_all_names_exist():
+    missing = [n for n in gdn.__all__ if not hasattr(gdn, n)]
+    assert not missing, missing
+
+
 def test_status_strings():
     lib = _native.lib()
     for code, name in _native.STATUS.items():
