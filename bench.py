@@ -55,11 +55,11 @@ CHUNK = 64
 # W.S, K~^T.u, Q.S (2 d^2 each) + T.(beta gamma K), T.(beta V), P.u (2 C d each)
 # + K.K^T and Q.K^T (2 C d each, shared by the 3 V heads of a QK head)
 PREFILL_FLOP_TV = 6 * D * D + 2 * CHUNK * D * (3 + 2 / 3)
-# tensor-core work of the chunk-chain kernel per (token, V head): S^T[K;Q]^T (4 d^2),
-# V^T T_beta^T and X T_beta_gamma^T (2 C d each) on TF32 operands; u~^T K (2 d^2) and
-# u^T P^T (2 C d) on fp16 operands
-CHAIN_FLOP_TV_TF32 = 4 * D * D + 2 * 2 * CHUNK * D
-CHAIN_FLOP_TV_F16 = 2 * D * D + 2 * CHUNK * D
+# tensor-core work of the chunk-chain kernel per (token, V head): S^T[K;Q]^T (4 d^2) and
+# X T_beta_gamma^T (2 C d) on TF32 operands (5/9 of it); V^T T_beta^T (2 C d), u~^T K (2 d^2)
+# and u^T P^T (2 C d) on fp16 operands (4/9)
+CHAIN_FLOP_TV_TF32 = 4 * D * D + 2 * CHUNK * D
+CHAIN_FLOP_TV_F16 = 2 * D * D + 2 * 2 * CHUNK * D
 CHAIN_FLOP_TV = CHAIN_FLOP_TV_TF32 + CHAIN_FLOP_TV_F16
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
                   "sm_max_mhz": 1965.0}
@@ -467,8 +467,8 @@ def prefill_roofline(res, peaks, peak_src, sha):
         return {"kernel": dom, "bound": "tensor", "achieved": ach, "peak": peak,
                 "unit": "TFLOP/s", "frac": ach / peak, "frac_of_bf16_peak": ach / bf16,
                 "traffic": traffic, "traffic_source": tsrc,
-                "peak_source": (f"{peak_src} bf16 {bf16} for the fp16 third of the MMA flops, "
-                                f"x 1.1/2.25 nominal (tf32) for the other two thirds"),
+                "peak_source": (f"{peak_src} bf16 {bf16} for the fp16 4/9 of the MMA flops, "
+                                f"x 1.1/2.25 nominal (tf32) for the other 5/9"),
                 "algorithmic_per_launch": flops, "tokens_per_launch": T, "kernel_share": share}
     # a tile-making pass dominates (chunk prep or the conv pass): its algorithmic bytes per
     # token at the run's head counts, the tiles being what the chain needs and nothing more

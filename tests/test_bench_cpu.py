@@ -87,3 +87,37 @@ def test_committed_records_are_well_formed(bench):
     for r in recs.values():
         assert r["bytes_per_launch"] > 0 and r["units_per_launch"] > 0
         assert len(r["sources_sha256"]) == 64 and int(r["sources_sha256"], 16) >= 0
+
+
+# The chain kernel's MMAs per chunk of 64 tokens and V head (M = d_v = 128 on the tensor-memory
+# lanes): shape (M, N, K) and operand kind, as the kernel issues them.
+CHAIN_MMAS = {"MMA_1 S^T [K;Q]^T": (128, 128, 128, "tf32"), "MMA_2a V^T T_beta^T": (128, 64, 64, "f16"),
+              "MMA_2b X T_beta_gamma^T": (128, 64, 64, "tf32"), "MMA_3 u~^T K": (128, 128, 64, "f16"),
+              "MMA_4 u^T P^T": (128, 64, 64, "f16")}
+
+
+def test_chain_flops_follow_the_mma_shapes(bench):
+    per_tok = {kind: sum(2 * m * n * k for m, n, k, t in CHAIN_MMAS.values() if t == kind) / 64
+               for kind in ("tf32", "f16")}
+    assert bench.CHAIN_FLOP_TV_TF32 == per_tok["tf32"] == 81920
+    assert bench.CHAIN_FLOP_TV_F16 == per_tok["f16"] == 65536
+    assert bench.CHAIN_FLOP_TV == 147456
+
+
+def test_chain_roofline_blends_the_peaks_by_time(bench):
+    """A launch that ran every MMA at its own peak reports frac = 1."""
+    peaks = {"bf16_tflops": 1654.0, "hbm_gbs": 6553.0}
+    tf32 = 1654.0 * 1.1 / 2.25
+    T, Hv, launches, steps = 2048, 48, 4, 10
+    t_ideal = (bench.CHAIN_FLOP_TV_TF32 / (tf32 * 1e12) + bench.CHAIN_FLOP_TV_F16 / (1654.0 * 1e12)) * T * Hv
+    res = {"per_kernel": {"prefill_tc": {"total_ms": t_ideal * 1e3 * launches * steps, "avg_ms": t_ideal * 1e3,
+                                         "launches": launches * steps},
+                          "chunk_prep": {"total_ms": 1e-3, "avg_ms": 1e-4, "launches": launches * steps}},
+           "tokens_per_step": T * launches, "steps": steps, "n_v_heads": Hv, "n_qk_heads": 16,
+           "workload": "none"}
+    r = bench.prefill_roofline(res, peaks, "measured", "0" * 64)
+    assert r["kernel"] == "prefill_tc" and r["tokens_per_launch"] == T
+    assert abs(r["frac"] - 1.0) < 1e-12
+    assert abs(r["peak"] - 1046.30) < 0.01
+    assert abs(r["frac_of_bf16_peak"] - r["achieved"] / 1654.0) < 1e-12
+    assert r["traffic"] is None
