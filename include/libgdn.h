@@ -74,8 +74,9 @@ typedef enum {
 /* Every call takes two storage types: `dtype` for q, k, v, alpha, beta and the conv
  * state (the raw inputs), and `out_dtype` for y.  Whatever they are, accumulation and states
  * are fp32; the tensor-core products of the bf16 path take operands with an 11-bit
- * significand (TF32 where an operand is an fp32 accumulator, fp16 for the chunk tiles and
- * the per-chunk vectors u), and the fp32 path computes in fp32 on the CUDA cores.
+ * significand (TF32 for the state products and their [K;Q] and T_beta_gamma tiles, fp16 for
+ * the other chunk tiles and the per-chunk vectors u), and the fp32 path computes in fp32 on
+ * the CUDA cores.
  * Note on precision: rounding y to bfloat16 alone moves its largest entries by up to
  * 2^-9 of their magnitude, which on typical data is 2-3% of rms(y); use
  * out_dtype = GDN_F32 where y must stay within 1e-2 of rms(y) of the exact result. */
