@@ -4,8 +4,9 @@
 // kernel-4 ShortConv before the gated delta rule.  The conv is causal and depthwise
 // with tap 3 on the current row; q and k are then L2-normalised per (token, head).
 // Memory-bound: each raw row is read once (plus a 3-row halo per chunk or 16-row strip,
-// served by L2) and each normalised row written once, in fp32 (rounding these rows to
-// bf16 would by itself move y by several percent of its rms).
+// served by L2) and each normalised row written once: as fp32 rows (fp32 input) or into the
+// chain's tiles ([K;Q] rounded to TF32, K and V to fp16, both 11-bit significands; bf16's 8
+// bits would by themselves move y by several percent of its rms).
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
