@@ -55,6 +55,9 @@ CHUNK = 64
 # W.S, K~^T.u, Q.S (2 d^2 each) + T.(beta gamma K), T.(beta V), P.u (2 C d each)
 # + K.K^T and Q.K^T (2 C d each, shared by the 3 V heads of a QK head)
 PREFILL_FLOP_TV = 6 * D * D + 2 * CHUNK * D * (3 + 2 / 3)
+# the same counting only the triangles the chunked form needs: K.K^T and Q.K^T half each
+# (shared by 3 V heads: 1/3 together), T.(beta gamma K), T.(beta V) and P.u half each
+PREFILL_FLOP_TV_TRI = 6 * D * D + 2 * CHUNK * D * 11 / 6
 # tensor-core work of the chunk-chain kernel per (token, V head): S^T[K;Q]^T (4 d^2) and
 # X T_beta_gamma^T (2 C d) on TF32 operands (5/9 of it); V^T T_beta^T (2 C d), u~^T K (2 d^2)
 # and u^T P^T (2 C d) on fp16 operands (4/9)
@@ -498,11 +501,13 @@ def prefill_step_summary(res, peaks):
     T = res["tokens_per_step"]
     Hq, Hv = res["n_qk_heads"], res["n_v_heads"]
     flops = PREFILL_FLOP_TV * T * Hv
+    tri = PREFILL_FLOP_TV_TRI * T * Hv
     byts = (2 * Hq * D * 2 + Hv * D * 2 + Hv * D * 2 + 2 * Hv * 2) * T
     tf32 = peaks["bf16_tflops"] * TF32_PER_BF16
     return {"tflops": flops / s / 1e12, "frac_of_tf32_peak": flops / s / 1e12 / tf32,
             "frac_of_bf16_peak": flops / s / 1e12 / peaks["bf16_tflops"],
             "algorithmic_flops_per_step": flops,
+            "tflops_triangles_only": tri / s / 1e12, "algorithmic_flops_per_step_triangles_only": tri,
             "gbs": byts / s / 1e9, "frac_of_hbm": byts / s / 1e9 / peaks["hbm_gbs"],
             "algorithmic_bytes_per_step": byts}
 
@@ -760,6 +765,7 @@ def bench_decode(args, dist, torch, gdn, peaks, peak_src):
     avg_s = sum(recs) / len(recs) / 1e3
     bpr = decode_bytes_per_row(shape)
     achieved = bpr * B / avg_s / 1e9
+    bpr_min = decode_bytes_per_row(shape, out_bytes=2)   # the minimum: y in bf16
 
     # e2e: pinned host inputs (a ring of 32 distinct steps), y read back every step
     ring = 32
@@ -796,7 +802,9 @@ def bench_decode(args, dist, torch, gdn, peaks, peak_src):
         "roofline": {"kernel": "decode", "bound": "hbm", "achieved": achieved,
                      "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
                      "traffic": dec_traffic, "traffic_source": dec_tsrc, "peak_source": peak_src,
-                     "algorithmic_bytes_per_row": bpr, "rows_per_launch": B},
+                     "algorithmic_bytes_per_row": bpr, "rows_per_launch": B,
+                     "frac_of_min_bytes": bpr_min * B / avg_s / 1e9 / peaks["hbm_gbs"],
+                     "min_bytes_per_row": bpr_min},
         "e2e": {"value": toks / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "note": "host inputs cycle through 32 pinned step sets"},
     }

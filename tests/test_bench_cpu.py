@@ -121,3 +121,24 @@ def test_chain_roofline_blends_the_peaks_by_time(bench):
     assert abs(r["peak"] - 1046.30) < 0.01
     assert abs(r["frac_of_bf16_peak"] - r["achieved"] / 1654.0) < 1e-12
     assert r["traffic"] is None
+
+
+def test_step_work_per_token_matches_the_stated_counts(bench):
+    """Per token at 16 QK / 48 V heads: 7.60 MFLOP with full 64-row tiles, 6.16 MFLOP counting
+    only the needed triangles, and a minimum of 32,960 bytes (raw q, k, v, gates, bf16 y)."""
+    T = 8192
+    res = {"ms_per_step": 1.0, "tokens_per_step": T, "n_qk_heads": 16, "n_v_heads": 48}
+    r = bench.prefill_step_summary(res, {"bf16_tflops": 1654.0, "hbm_gbs": 6553.0})
+    assert round(r["algorithmic_flops_per_step"] / T) == 7602176
+    assert round(r["algorithmic_flops_per_step_triangles_only"] / T) == 6160384
+    assert r["algorithmic_bytes_per_step"] == 32960 * T
+    assert abs(r["gbs"] - 32960 * T / 1e-3 / 1e9) < 1e-6
+    assert abs(r["frac_of_bf16_peak"] - r["tflops"] / 1654.0) < 1e-12
+
+
+def test_decode_bytes_per_row(bench):
+    """State read and written once (6,291,456 B), conv state read and written, this step's raw
+    q, k, v, the gates and y: 6,447,296 B with bf16 y (the minimum), 6,459,584 with fp32 y."""
+    import gdn_inputs as gi
+    assert bench.decode_bytes_per_row(gi.PAGES_SHAPE, out_bytes=2) == 6447296
+    assert bench.decode_bytes_per_row(gi.PAGES_SHAPE) == 6459584
