@@ -142,3 +142,26 @@ def test_decode_bytes_per_row(bench):
     import gdn_inputs as gi
     assert bench.decode_bytes_per_row(gi.PAGES_SHAPE, out_bytes=2) == 6447296
     assert bench.decode_bytes_per_row(gi.PAGES_SHAPE) == 6459584
+
+
+def test_reference_arm_line(repo_tmp):
+    """`bench.py --impl reference` (the fp64 oracle on the host cores) prints one JSON line with
+    the headline config, and ranks other than 0 print nothing."""
+    import subprocess
+    import sys
+    cmd = [sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--steps", "1",
+           "--warmup", "3", "--ref-step-s", "0.5"]
+    env = dict(os.environ, RANK="0", WORLD_SIZE="1")
+    r = subprocess.run(cmd, capture_output=True, text=True, cwd=repo_tmp, env=env, timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [json.loads(ln) for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    ln = lines[0]
+    assert ln["impl"] == "reference" and ln["unit"] == "tokens/s" and ln["value"] > 0
+    assert ln["higher_is_better"] is True and ln["n_gpus"] == 1 and ln["steps"] == 1
+    assert ln["config"]["workload"] == "layer-bf16-T8192-h16x48" and ln["config"]["T"] == 8192
+    assert ln["cpu_baseline"]["kind"] == "oracle" and ln["cpu_baseline"]["cores"] >= 1
+    assert ln["e2e"] == {"value": ln["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+    r1 = subprocess.run(cmd, capture_output=True, text=True, cwd=repo_tmp,
+                        env=dict(os.environ, RANK="1", WORLD_SIZE="2"), timeout=600)
+    assert r1.returncode == 0 and not r1.stdout.strip()
